@@ -1,0 +1,289 @@
+"""fp64 CPU oracle for the HedgeMamba mixer scan.
+
+TEST INFRASTRUCTURE ONLY.  The product (the CUDA library under
+``selective_ssm_sequence_b200`` and its binding) never imports, loads or calls
+anything in this package, and this package never imports the product.  The
+tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg are
+the only callers.
+
+The loops live in ``hm_oracle.c`` (plain C, double precision).  This module
+builds it with gcc, wraps it with ctypes and composes the mixer from those
+steps plus numpy matmuls (a library matmul is a single step of the mixer's
+definition; nothing is blocked or fused).
+
+Page citations (see ``hm_oracle.c`` for the full list):
+  [HM]  HedgeMamba explainer (gsyq.cn 1418924): sec. 2.1 Hedgehog map,
+        sec. 2.3 / 5.2 mixer, sec. 3.1 stage-1 identity init, sec. 5.3 map listing.
+  [LA]  Linear-attention tutorial (cnblogs 22790249): sec. 2 kernel form and
+        associativity, sec. 3 recurrent form, sec. 4.3 RetNet decay.
+  [SSM] SSM article (quant67 56-ssm): sec. 3.2 softplus dt, sec. 4.2 affine
+        composition.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+against closed forms, invariants, a brute-force rational-arithmetic evaluation
+or an independent formulation.  End-to-end numeric values are not printed on
+the pages (no worked example), so absolute values rest on those pins.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hm_oracle.c")
+_LIB = os.path.join(_HERE, "_hm_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile hm_oracle.c into a shared object next to it (gcc, -O2, OpenMP)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        lib.hmo_softplus.restype = ctypes.c_double
+        lib.hmo_softplus.argtypes = [ctypes.c_double]
+        lib.hmo_log_decay.restype = None
+        lib.hmo_log_decay.argtypes = [P, I64, I, P, P]
+        lib.hmo_featmap.restype = None
+        lib.hmo_featmap.argtypes = [P, I64, I, I, I, P, I64, P, I64, P]
+        lib.hmo_scan_recurrent.restype = I64
+        lib.hmo_scan_recurrent.argtypes = [I64, I64, I, I, I, P, P, P, P, P, P, P, P, P]
+        lib.hmo_scan_quadratic.restype = None
+        lib.hmo_scan_quadratic.argtypes = [I64, I64, I, I, I, P, P, P, P, P]
+        lib.hmo_decode_step.restype = I64
+        lib.hmo_decode_step.argtypes = [I64, I, I, I, P, P, P, P, P, P, P]
+        lib.hmo_causal_conv.restype = None
+        lib.hmo_causal_conv.argtypes = [I64, I64, I, I, P, P, P, P]
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> None:
+    """Bound the OpenMP team used by the oracle loops (call before first use)."""
+    os.environ["OMP_NUM_THREADS"] = str(int(n))
+
+
+# --------------------------------------------------------------------------
+# single steps
+# --------------------------------------------------------------------------
+
+def softplus(x: float) -> float:
+    """log(1 + e^x) ([SSM] sec. 3.2: dt goes through softplus)."""
+    return _load().hmo_softplus(float(x))
+
+
+def log_decay(dt, A_log):
+    """l[b,t,h] = -softplus(dt[b,t,h]) * exp(A_log[h]); a = exp(l).
+
+    dt: [..., H]; A_log: [H].  Returns an array shaped like dt."""
+    dt = _f64(dt)
+    A_log = _f64(A_log)
+    H = A_log.shape[0]
+    assert dt.shape[-1] == H
+    out = np.empty_like(dt)
+    _load().hmo_log_decay(_ptr(dt), dt.size // H, H, _ptr(A_log), _ptr(out))
+    return out
+
+
+def featmap(x, W, bias=None, H=1, w_head_stride=0, b_head_stride=0):
+    """Hedgehog map phi = softmax([W x + b, -(W x + b)]) over 2p features
+    ([HM] sec. 2.1, 5.3).  x: [..., d] (row r is head r mod H); W: [p, d]
+    (or [H, p, d] with w_head_stride = p*d).  Returns [..., 2p]."""
+    x = _f64(x)
+    W = _f64(W)
+    d = x.shape[-1]
+    p = W.shape[-2]
+    assert W.shape[-1] == d
+    rows = x.size // d
+    b = None if bias is None else _f64(bias)
+    out = np.empty(x.shape[:-1] + (2 * p,), dtype=np.float64)
+    _load().hmo_featmap(_ptr(x), rows, int(H), d, p, _ptr(W), int(w_head_stride),
+                        _ptr(b), int(b_head_stride), _ptr(out))
+    return out
+
+
+def scan_recurrent(phq, phk, v, log_a=None, S0=None, z0=None, return_state=False):
+    """Decayed normalised recurrence (spec definition):
+    S_t = a_t S_{t-1} + phik_t v_t^T, z_t = a_t z_{t-1} + phik_t,
+    o_t = phiq_t^T S_t / phiq_t^T z_t.  phq, phk: [B, L, H, F]; v: [B, L, H, dv];
+    log_a: [B, L, H] or None (a = 1).  Raises if any denominator is <= 0."""
+    phq, phk, v = _f64(phq), _f64(phk), _f64(v)
+    B, L, H, F = phq.shape
+    dv = v.shape[-1]
+    assert phk.shape == phq.shape and v.shape[:3] == (B, L, H)
+    la = None if log_a is None else _f64(log_a)
+    if la is not None:
+        assert la.shape == (B, L, H)
+    S0a = None if S0 is None else _f64(S0)
+    z0a = None if z0 is None else _f64(z0)
+    o = np.empty((B, L, H, dv), dtype=np.float64)
+    S_out = np.empty((B, H, F, dv), dtype=np.float64)
+    z_out = np.empty((B, H, F), dtype=np.float64)
+    bad = _load().hmo_scan_recurrent(B, L, H, F, dv, _ptr(phq), _ptr(phk), _ptr(v),
+                                     _ptr(la), _ptr(S0a), _ptr(z0a), _ptr(o),
+                                     _ptr(S_out), _ptr(z_out))
+    if bad:
+        raise FloatingPointError("oracle: %d denominators were not > 0" % bad)
+    if return_state:
+        return o, S_out, z_out
+    return o
+
+
+def scan_quadratic(phq, phk, v, log_a=None):
+    """O(L^2) masked form ([LA] sec. 2): o_i = sum_{j<=i} w_ij v_j / sum_j w_ij,
+    w_ij = exp(sum_{j<t<=i} l_t) phiq_i . phik_j.  Zero initial state."""
+    phq, phk, v = _f64(phq), _f64(phk), _f64(v)
+    B, L, H, F = phq.shape
+    dv = v.shape[-1]
+    la = None if log_a is None else _f64(log_a)
+    o = np.empty((B, L, H, dv), dtype=np.float64)
+    _load().hmo_scan_quadratic(B, L, H, F, dv, _ptr(phq), _ptr(phk), _ptr(v), _ptr(la), _ptr(o))
+    return o
+
+
+def decode_step(phq, phk, v, S, z, log_a=None):
+    """One recurrent step per (batch, head); returns (o, S_new, z_new).
+    phq, phk: [B, H, F]; v: [B, H, dv]; S: [B, H, F, dv]; z: [B, H, F];
+    log_a: [B, H] or None."""
+    phq, phk, v = _f64(phq), _f64(phk), _f64(v)
+    B, H, F = phq.shape
+    dv = v.shape[-1]
+    S = _f64(S).copy()
+    z = _f64(z).copy()
+    la = None if log_a is None else _f64(log_a)
+    o = np.empty((B, H, dv), dtype=np.float64)
+    bad = _load().hmo_decode_step(B, H, F, dv, _ptr(phq), _ptr(phk), _ptr(v), _ptr(la),
+                                  _ptr(S), _ptr(z), _ptr(o))
+    if bad:
+        raise FloatingPointError("oracle: %d denominators were not > 0" % bad)
+    return o, S, z
+
+
+def causal_conv(x, w, bias=None):
+    """Depthwise causal conv along the sequence, zero left padding, no
+    activation ([HM] sec. 2.3: short conv kept).  x: [B, L, C]; w: [C, K];
+    bias: [C] or None."""
+    x = _f64(x)
+    w = _f64(w)
+    B, L, C = x.shape
+    K = w.shape[1]
+    b = None if bias is None else _f64(bias)
+    y = np.empty_like(x)
+    _load().hmo_causal_conv(B, L, C, K, _ptr(x), _ptr(w), _ptr(b), _ptr(y))
+    return y
+
+
+def silu(x):
+    """SiLU(x) = x * sigmoid(x) (the gate nonlinearity, [HM] sec. 3.1)."""
+    x = _f64(x)
+    return x / (1.0 + np.exp(-x))
+
+
+# --------------------------------------------------------------------------
+# compositions
+# --------------------------------------------------------------------------
+
+def scan_fwd(q, k, v, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=None,
+             S0=None, z0=None, w_head_stride=0, return_state=False):
+    """Feature map on q and k, then the decayed normalised recurrence.
+
+    q, k: [B, L, H, d]; v: [B, L, H, dv]; W_q, W_k: [p, d] (or per-head); if
+    W_q is None, q and k are taken as feature vectors already (F = d).
+    dt: [B, L, H] or None (a = 1); A_log: [H]."""
+    q, k = _f64(q), _f64(k)
+    B, L, H, d = q.shape
+    if W_q is None:
+        phq, phk = q, k
+    else:
+        phq = featmap(q, W_q, b_q, H=H, w_head_stride=w_head_stride)
+        phk = featmap(k, W_k, b_k, H=H, w_head_stride=w_head_stride)
+    la = None if dt is None else log_decay(dt, A_log)
+    return scan_recurrent(phq, phk, v, la, S0, z0, return_state=return_state)
+
+
+def mixer_fwd(x, W_q, W_k, W_v, W_g, W_dt, conv_w, W_hq, W_hk, A_log, W_o,
+              conv_b=None, b_g=None, b_dt=None, n_heads=8, batches=None):
+    """HedgeMamba mixer forward ([HM] sec. 2.3 and 5.2), plain composition:
+
+      q, k, v, g = x W_{q,k,v,g}^T ;  dt = x W_dt^T (+ b_dt)
+      q, k, v    = causal depthwise conv (width K) of each, + conv bias
+      per head h (d_head = width / H): phi_q = hedgehog(q_h), phi_k = hedgehog(k_h)
+      o          = decayed normalised recurrence(phi_q, phi_k, v, a(dt, A_log))
+      y          = o * SiLU(g (+ b_g))
+      out        = y W_o^T
+
+    x: [B, L, D]; W_q..W_g: [E, D] (E = H * d_head); W_dt: [H, D];
+    conv_w: [3, E, K] (q, k, v); conv_b: [3, E] or None; W_hq, W_hk: [p, d_head];
+    A_log: [H]; W_o: [D, E].  ``batches`` restricts the evaluation to a subset
+    of the batch (each batch row is independent)."""
+    x = _f64(x)
+    if batches is not None:
+        x = x[list(batches)]
+    B, L, D = x.shape
+    H = int(n_heads)
+    E = W_q.shape[0]
+    dh = E // H
+    xf = x.reshape(B * L, D)
+    q = xf @ _f64(W_q).T
+    k = xf @ _f64(W_k).T
+    v = xf @ _f64(W_v).T
+    g = xf @ _f64(W_g).T
+    dt = xf @ _f64(W_dt).T
+    if b_dt is not None:
+        dt = dt + _f64(b_dt)
+    if b_g is not None:
+        g = g + _f64(b_g)
+    cw = _f64(conv_w)
+    cb = [None, None, None] if conv_b is None else [_f64(conv_b)[i] for i in range(3)]
+    q = causal_conv(q.reshape(B, L, E), cw[0], cb[0])
+    k = causal_conv(k.reshape(B, L, E), cw[1], cb[1])
+    v = causal_conv(v.reshape(B, L, E), cw[2], cb[2])
+    o = scan_fwd(q.reshape(B, L, H, dh), k.reshape(B, L, H, dh), v.reshape(B, L, H, dh),
+                 W_q=W_hq, W_k=W_hk, dt=dt.reshape(B, L, H), A_log=A_log)
+    y = o.reshape(B * L, E) * silu(g)
+    out = y @ _f64(W_o).T
+    return out.reshape(B, L, D)
+
+
+def omp_threads_in_use() -> int:
+    """Threads the OpenMP loops will use (OMP_NUM_THREADS or all cores)."""
+    env = os.environ.get("OMP_NUM_THREADS")
+    if env:
+        try:
+            return max(1, int(env))
+        except ValueError:
+            pass
+    return os.cpu_count() or 1
+
+
+if __name__ == "__main__":  # pragma: no cover
+    print(build(force="--force" in sys.argv))

@@ -1,0 +1,268 @@
+"""Seeded synthetic inputs for the HedgeMamba mixer-scan workloads.
+
+This module is shared by the CUDA-path tests/benchmark and by the oracle
+runs, and it holds none of the method's arithmetic: only random numbers,
+shapes and the rounding of generated values to the storage dtype.
+
+Generator (stated so that anyone can regenerate the same bytes):
+  * every tensor has its own 64-bit stream key = FNV-1a-64(name) XOR
+    (seed * 0x9E3779B97F4A7C15 mod 2^64);
+  * splitmix64 over the counter 1, 2, 3, ... under that key gives uint64s;
+  * a uniform in (0, 1) is ((x >> 11) + 0.5) * 2^-53;
+  * normals come from Box-Muller on consecutive uniform pairs (u1, u2):
+    sqrt(-2 ln u1) cos(2 pi u2) and sqrt(-2 ln u1) sin(2 pi u2), in fp64;
+  * values meant for bf16 storage are rounded fp64 -> fp32 (round to nearest
+    even) -> bf16 (round to nearest even), once, here.  Both the GPU run and
+    the oracle consume the rounded values.
+
+The five workloads follow the headline benchmark's configuration list; the
+shapes, dtypes and value distributions are listed in ``CONFIGS``.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional
+
+import numpy as np
+
+_GOLD = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+
+def _fnv1a64(name: str) -> int:
+    h = 0xCBF29CE484222325
+    for ch in name.encode():
+        h ^= ch
+        h = (h * 0x100000001B3) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def _key(seed: int, name: str) -> np.uint64:
+    return np.uint64(_fnv1a64(name) ^ ((int(seed) * 0x9E3779B97F4A7C15) & 0xFFFFFFFFFFFFFFFF))
+
+
+def splitmix64(key: np.uint64, n: int) -> np.ndarray:
+    """n consecutive splitmix64 outputs for counter 1..n under ``key``."""
+    with np.errstate(over="ignore"):
+        ctr = np.arange(1, n + 1, dtype=np.uint64)
+        z = key + ctr * _GOLD
+        z = (z ^ (z >> np.uint64(30))) * _M1
+        z = (z ^ (z >> np.uint64(27))) * _M2
+        z = z ^ (z >> np.uint64(31))
+    return z
+
+
+def uniform(seed: int, name: str, shape, lo: float = 0.0, hi: float = 1.0) -> np.ndarray:
+    n = int(np.prod(shape)) if len(shape) else 1
+    u = ((splitmix64(_key(seed, name), n) >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+    return (lo + (hi - lo) * u).reshape(shape)
+
+
+def normal(seed: int, name: str, shape, std: float = 1.0) -> np.ndarray:
+    n = int(np.prod(shape)) if len(shape) else 1
+    m = (n + 1) // 2
+    u = ((splitmix64(_key(seed, name), 2 * m) >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+    u1, u2 = u[0::2], u[1::2]
+    r = np.sqrt(-2.0 * np.log(u1))
+    z = np.empty(2 * m, dtype=np.float64)
+    z[0::2] = r * np.cos(2.0 * math.pi * u2)
+    z[1::2] = r * np.sin(2.0 * math.pi * u2)
+    return (std * z[:n]).reshape(shape)
+
+
+# --------------------------------------------------------------------------
+# storage rounding (fp64 -> fp32 -> bf16, both round-to-nearest-even)
+# --------------------------------------------------------------------------
+
+def to_bf16_bits(a) -> np.ndarray:
+    """uint16 bf16 bit patterns of ``a`` (fp64 -> fp32 RNE -> bf16 RNE)."""
+    f = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    rounding = np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))
+    r = ((u + rounding) >> np.uint64(16)).astype(np.uint16)
+    nan = np.isnan(f)
+    if nan.any():
+        r[nan] = np.uint16(0x7FC0)
+    return r
+
+
+def bf16_bits_to_f32(bits) -> np.ndarray:
+    b = np.ascontiguousarray(np.asarray(bits, dtype=np.uint16))
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def round_bf16(a) -> np.ndarray:
+    """Values of ``a`` after rounding to bf16, returned as float64."""
+    return bf16_bits_to_f32(to_bf16_bits(a)).astype(np.float64)
+
+
+def round_f32(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float32).astype(np.float64)
+
+
+def store(a, dtype: str) -> np.ndarray:
+    """Round generated fp64 values to the storage dtype ('bf16' or 'f32');
+    returns float64 holding exactly the stored values."""
+    if dtype == "bf16":
+        return round_bf16(a)
+    if dtype == "f32":
+        return round_f32(a)
+    raise ValueError(dtype)
+
+
+# --------------------------------------------------------------------------
+# workloads
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class ScanConfig:
+    name: str
+    B: int
+    L: int
+    H: int
+    d: int
+    p: int
+    dv: int
+    io: str            # 'f32' or 'bf16' storage of q, k, v, W, o
+    decay: bool        # dt/A_log present (False: a_t = 1)
+    seed: int
+    w_std: float       # std of the Hedgehog projection entries
+
+    @property
+    def F(self) -> int:
+        return 2 * self.p
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.L
+
+    @property
+    def token_heads(self) -> int:
+        return self.B * self.L * self.H
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeConfig:
+    name: str
+    B: int
+    H: int
+    d: int
+    p: int
+    dv: int
+    prefill: int
+    steps: int
+    seed: int
+    w_std: float
+
+    @property
+    def F(self) -> int:
+        return 2 * self.p
+
+
+@dataclasses.dataclass(frozen=True)
+class MixerConfig:
+    name: str
+    B: int
+    L: int
+    d_model: int
+    H: int
+    p: int
+    conv: int
+    seed: int
+
+    @property
+    def d_head(self) -> int:
+        return self.d_model // self.H
+
+
+# "N(0, s)" in the configuration list is read as variance s.
+TINY_F32 = ScanConfig("tiny_f32_B1_H2_L256_d32_F64", 1, 256, 2, 32, 32, 32, "f32", False, 0,
+                      math.sqrt(1.0 / 32))
+PREFILL_PYTHIA = ScanConfig("prefill_B4_H8_L2048_d256_F256_bf16", 4, 2048, 8, 256, 128, 256,
+                            "bf16", True, 1, math.sqrt(1.0 / 256))
+PREFILL_LONG = ScanConfig("prefill_B1_H8_L32768_d256_F256_bf16", 1, 32768, 8, 256, 128, 256,
+                          "bf16", True, 2, math.sqrt(1.0 / 256))
+DECODE = DecodeConfig("decode_256x8_F256_dv256_prefill1024_steps512", 256, 8, 256, 128, 256,
+                      1024, 512, 3, math.sqrt(1.0 / 256))
+MIXER = MixerConfig("mixer_B8_L4096_D2048_H8_p128", 8, 4096, 2048, 8, 128, 4, 4)
+
+CONFIGS = {c.name: c for c in (TINY_F32, PREFILL_PYTHIA, PREFILL_LONG, DECODE, MIXER)}
+
+
+def scan_inputs(cfg: ScanConfig, B: Optional[int] = None, L: Optional[int] = None,
+                seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Inputs of a prefill workload as float64 arrays holding the stored values.
+
+    q, k ~ N(0,1) [B,L,H,d]; v ~ N(0,1) [B,L,H,dv]; W_q, W_k ~ N(0, w_std^2)
+    [p, d] (independent); with decay: dt ~ N(0,1) [B,L,H] (fp32) and
+    A_log ~ U(log 1, log 16) [H] (fp32).  B, L or seed may be overridden to
+    make smaller cases of the same distribution."""
+    B = cfg.B if B is None else B
+    L = cfg.L if L is None else L
+    s = cfg.seed if seed is None else seed
+    io = cfg.io
+    out = {
+        "W_q": store(normal(s, "W_q", (cfg.p, cfg.d), cfg.w_std), io),
+        "W_k": store(normal(s, "W_k", (cfg.p, cfg.d), cfg.w_std), io),
+        "q": store(normal(s, "q", (B, L, cfg.H, cfg.d)), io),
+        "k": store(normal(s, "k", (B, L, cfg.H, cfg.d)), io),
+        "v": store(normal(s, "v", (B, L, cfg.H, cfg.dv)), io),
+    }
+    if cfg.decay:
+        out["dt"] = store(normal(s, "dt", (B, L, cfg.H)), "f32")
+        out["A_log"] = store(uniform(s, "A_log", (cfg.H,), 0.0, math.log(16.0)), "f32")
+    return out
+
+
+def decode_inputs(cfg: DecodeConfig, B: Optional[int] = None, steps: Optional[int] = None,
+                  prefill: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Prefill tokens [B, prefill, H, *] and per-step tokens [steps, B, H, *],
+    same distributions as the Pythia-shaped prefill (bf16 q/k/v/W, fp32 dt,
+    A_log ~ U(0, log 16))."""
+    B = cfg.B if B is None else B
+    n = cfg.steps if steps is None else steps
+    P = cfg.prefill if prefill is None else prefill
+    s = cfg.seed
+    return {
+        "W_q": store(normal(s, "W_q", (cfg.p, cfg.d), cfg.w_std), "bf16"),
+        "W_k": store(normal(s, "W_k", (cfg.p, cfg.d), cfg.w_std), "bf16"),
+        "A_log": store(uniform(s, "A_log", (cfg.H,), 0.0, math.log(16.0)), "f32"),
+        "pre_q": store(normal(s, "pre_q", (B, P, cfg.H, cfg.d)), "bf16"),
+        "pre_k": store(normal(s, "pre_k", (B, P, cfg.H, cfg.d)), "bf16"),
+        "pre_v": store(normal(s, "pre_v", (B, P, cfg.H, cfg.dv)), "bf16"),
+        "pre_dt": store(normal(s, "pre_dt", (B, P, cfg.H)), "f32"),
+        "q": store(normal(s, "step_q", (n, B, cfg.H, cfg.d)), "bf16"),
+        "k": store(normal(s, "step_k", (n, B, cfg.H, cfg.d)), "bf16"),
+        "v": store(normal(s, "step_v", (n, B, cfg.H, cfg.dv)), "bf16"),
+        "dt": store(normal(s, "step_dt", (n, B, cfg.H)), "f32"),
+    }
+
+
+def mixer_weights(cfg: MixerConfig) -> Dict[str, np.ndarray]:
+    """Mixer weights: projections N(0, 1/d_model) bf16 ([E, D], [H, D], [D, E]);
+    conv w N(0, 1/K) fp32 [3, E, K]; Hedgehog W N(0, 1/d_head) bf16 [p, d_head];
+    A_log ~ U(log 1, log 16) fp32 [H]."""
+    s = cfg.seed
+    D = cfg.d_model
+    E = cfg.H * cfg.d_head
+    wstd = math.sqrt(1.0 / D)
+    return {
+        "W_q": store(normal(s, "W_q", (E, D), wstd), "bf16"),
+        "W_k": store(normal(s, "W_k", (E, D), wstd), "bf16"),
+        "W_v": store(normal(s, "W_v", (E, D), wstd), "bf16"),
+        "W_g": store(normal(s, "W_g", (E, D), wstd), "bf16"),
+        "W_dt": store(normal(s, "W_dt", (cfg.H, D), wstd), "bf16"),
+        "W_o": store(normal(s, "W_o", (D, E), math.sqrt(1.0 / E)), "bf16"),
+        "conv_w": store(normal(s, "conv_w", (3, E, cfg.conv), math.sqrt(1.0 / cfg.conv)), "f32"),
+        "W_hq": store(normal(s, "W_hq", (cfg.p, cfg.d_head), math.sqrt(1.0 / cfg.d_head)), "bf16"),
+        "W_hk": store(normal(s, "W_hk", (cfg.p, cfg.d_head), math.sqrt(1.0 / cfg.d_head)), "bf16"),
+        "A_log": store(uniform(s, "A_log", (cfg.H,), 0.0, math.log(16.0)), "f32"),
+    }
+
+
+def mixer_x(cfg: MixerConfig, B: Optional[int] = None, L: Optional[int] = None) -> np.ndarray:
+    B = cfg.B if B is None else B
+    L = cfg.L if L is None else L
+    return store(normal(cfg.seed, "x", (B, L, cfg.d_model)), "bf16")
