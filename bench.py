@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of the HedgeMamba mixer scan on B200 (prints one JSON line).
+
+Default workload: the Pythia-1B-shaped single-layer prefill (B=4, H=8,
+L=2048, d = dv = 256, Hedgehog 256->128 so F = 256, bf16 q/k/v, fp32
+state and accumulation, dt ~ N(0,1), A_log ~ U(0, log 16)).  One step is one
+pass of the whole hot path over one batch: the Hedgehog map on q and on k,
+then the decayed normalised chunked scan, each through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|long|decode|mixer|tiny]
+
+Multi-GPU (N > 1, launched by torchrun): every rank runs its own batch (its
+own seed); there is no data-path collective ("weak" scaling).  Times are
+device times (CUDA events) and the reported time is the max over ranks.
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events
+on the launching stream, with a 512 MiB buffer write between steps (outside
+the events) so that no step finds its inputs in the 126 MB L2.
+
+--impl reference times the fp64 CPU oracle (the reference for this method)
+on bounded samples of the same workload on the host cores; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+# ---------------------------------------------------------------- peaks
+
+_FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(_FALLBACK_PEAKS), "fallback"
+
+
+# DRAM bytes per launch of the dominant kernel from an ncu capture of the
+# current kernel version (dram__bytes_read.sum + dram__bytes_write.sum), or
+# None when the kernel changed since the counters were taken.
+NCU_TRAFFIC_BYTES = {}
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in self.samples:
+            try:
+                sm.append(float(s[1]))
+                mx.append(float(s[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, s[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def to_dev(a, dtype, torch):
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+def max_over_ranks(x: float, world: int, torch) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+def oracle_prefill_rate(cfg, budget_s: float = 12.0):
+    """fp64 oracle (feature maps + recurrence) on all B*H heads of the
+    workload for its first T tokens, T grown until ~budget_s of CPU work.
+    Returns (tokens_per_s, threads, sample description, seconds)."""
+    import oracle
+    oracle.build()
+    T = 16
+    while True:
+        inp = wl.scan_inputs(cfg, L=T)
+        t0 = time.perf_counter()
+        oracle.scan_fwd(inp["q"], inp["k"], inp["v"], inp["W_q"], inp["W_k"],
+                        dt=inp.get("dt"), A_log=inp.get("A_log"))
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or T >= cfg.L:
+            break
+        grow = max(2, min(8, int(budget_s / max(dt, 1e-3))))
+        T = min(cfg.L, T * grow)
+    threads = min(oracle.omp_threads_in_use(), cfg.B * cfg.H)
+    sample = ("fp64 oracle (Hedgehog maps + recurrence) on all %d (batch, head) pairs, first %d of "
+              "%d tokens" % (cfg.B * cfg.H, T, cfg.L))
+    return cfg.B * T / dt, threads, sample, dt
+
+
+# ---------------------------------------------------------------- prefill workload
+
+def algorithmic_per_token_head(F: int, d: int, p: int, dv: int):
+    """Algorithmic FLOPs and HBM bytes per (batch, token, head) of the prefill.
+
+    FLOPs: two Hedgehog projections 2*(2*d*p) + the normalised recurrence
+    4*F*(dv + 1) (state update and readout of the numerator, F*dv each as
+    multiply-add, plus the denominator).  Bytes (bf16 io): q, k, v read, o
+    written (2 bytes each element) and dt (4 bytes)."""
+    flops_featmap = 2 * (2 * d * p)
+    flops_scan = 4 * F * (dv + 1)
+    bytes_fused = 2 * (2 * d + dv + dv) + 4
+    return flops_featmap, flops_scan, bytes_fused
+
+
+def bench_prefill(cfg, args, rank, world, torch):
+    import selective_ssm_sequence_b200 as hm
+
+    peaks, peak_kind = load_peaks()
+    seed = cfg.seed + 1000 * rank
+    inp = wl.scan_inputs(cfg, seed=seed)
+    B, L, H, d, p, dv = cfg.B, cfg.L, cfg.H, cfg.d, cfg.p, cfg.dv
+    F = 2 * p
+    q, k, v = (to_dev(inp[n], "bf16", torch) for n in ("q", "k", "v"))
+    Wq, Wk = to_dev(inp["W_q"], "bf16", torch), to_dev(inp["W_k"], "bf16", torch)
+    dtt, A_log = to_dev(inp["dt"], "f32", torch), to_dev(inp["A_log"], "f32", torch)
+    o = torch.empty_like(v)
+    phq = torch.empty(B, L, H, F, device="cuda", dtype=torch.bfloat16)
+    phk = torch.empty_like(phq)
+    fargs = hm.scan_args(phq, phk, v, o, dt=dtt, A_log=A_log)
+    ws = hm.alloc_workspace(hm.hm_scan_workspace_size(fargs))
+    fargs.workspace, fargs.workspace_bytes = ws.data_ptr(), ws.numel()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+
+    def step(ev):
+        ev[0].record(stream)
+        hm.hm_featmap(q, Wq, phq, H=H, stream=stream)
+        ev[1].record(stream)
+        hm.hm_featmap(k, Wk, phk, H=H, stream=stream)
+        ev[2].record(stream)
+        hm.hm_scan_chunked_fwd(fargs, stream)
+        ev[3].record(stream)
+
+    K, W = args.steps, args.warmup
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    for _ in range(W):
+        flush.zero_()
+        step(warm)
+    torch.cuda.synchronize()
+    assert hm.hm_get_device_error() == hm.HM_OK
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = hm.hm_launch_count()
+    for i in range(K):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    launches = hm.hm_launch_count() - launches0
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.stop()
+    assert hm.hm_get_device_error() == hm.HM_OK
+
+    t_fq = [e[0].elapsed_time(e[1]) for e in evs]
+    t_fk = [e[1].elapsed_time(e[2]) for e in evs]
+    t_sc = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    ms_step = max_over_ranks(sum(t_step) / K, world, torch)
+    ms_fmap = max_over_ranks((sum(t_fq) + sum(t_fk)) / (2 * K), world, torch)
+    ms_scan = max_over_ranks(sum(t_sc) / K, world, torch)
+
+    th = B * L * H
+    fl_fm, fl_sc, _ = algorithmic_per_token_head(F, d, p, dv)
+    tokens_total = B * L * world
+    value = tokens_total / (ms_step * 1e-3)
+
+    # dominant call and its roofline
+    bw = peaks["hbm_gbs"]
+    tf = peaks["bf16_tflops"]
+    fm_bytes = th * (2 * d + 2 * F)      # x read, phi written (bf16), per launch
+    fm_flops = th * 2 * d * p
+    sc_bytes = th * (2 * F + 2 * F + 2 * dv + 4 + 2 * dv)  # phiq, phik, v, dt read; o written
+    sc_flops = th * fl_sc
+    if ms_scan >= ms_fmap:
+        name, nbytes, nflops, ms = "scan_chunked (features precomputed)", sc_bytes, sc_flops, ms_scan
+    else:
+        name, nbytes, nflops, ms = "hedgehog_featmap", fm_bytes, fm_flops, ms_fmap
+    intensity = nflops / nbytes
+    ridge = tf * 1e12 / (bw * 1e9)
+    if intensity >= ridge:
+        roof = {"bound": "tensor", "achieved": nflops / (ms * 1e-3) / 1e12, "peak": tf,
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": bw, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = NCU_TRAFFIC_BYTES.get(name)
+    roof["kernel"] = name
+    roof["peak_source"] = peak_kind
+    roof["ms_per_launch"] = ms
+
+    # end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_prefill_e2e(cfg, inp, Wq, Wk, A_log, args, world, torch, hm, flush)
+
+    step_flops = th * (fl_fm + fl_sc)
+    result = {
+        "metric": "tokens/sec of HedgeMamba mixer scan fwd on 1 B200; % of tensor/HBM roofline",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded splitmix64 + Box-Muller, rounded to bf16)",
+        "config": {"workload": cfg.name, "B": B, "L": L, "H": H, "d": d, "F": F, "dv": dv,
+                   "tokens_per_gpu": B * L, "l2": "512 MiB buffer written between timed steps",
+                   "step": "hm_featmap(q), hm_featmap(k), hm_scan_chunked_fwd(features)"},
+        "roofline": roof,
+        "step_roofline": {"bound": "tensor", "flops_per_token_head": fl_fm + fl_sc,
+                          "achieved": step_flops / (ms_step * 1e-3) / 1e12, "peak": tf,
+                          "unit": "TFLOP/s", "frac": step_flops / (ms_step * 1e-3) / 1e12 / tf,
+                          "peak_source": peak_kind},
+        "breakdown_ms": {"featmap_q_and_k": 2 * ms_fmap, "scan": ms_scan},
+        "gpu_launches": int(launches),
+        "e2e": e2e,
+        "clocks": sampler.summary(),
+    }
+    return result
+
+
+def bench_prefill_e2e(cfg, inp, Wq, Wk, A_log, args, world, torch, hm, flush):
+    """Same metric through one hm_scan_chunked_fwd call per step with the
+    step's inputs copied from pinned host memory and the output copied back."""
+    B, L, H, d, p, dv = cfg.B, cfg.L, cfg.H, cfg.d, cfg.p, cfg.dv
+    hq, hk, hv = (torch.from_numpy(inp[n].astype(np.float32)).to(torch.bfloat16).pin_memory()
+                  for n in ("q", "k", "v"))
+    hdt = torch.from_numpy(inp["dt"].astype(np.float32)).pin_memory()
+    ho = torch.empty(B, L, H, dv, dtype=torch.bfloat16).pin_memory()
+    q = torch.empty(hq.shape, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty_like(q)
+    v = torch.empty(hv.shape, dtype=torch.bfloat16, device="cuda")
+    dtt = torch.empty(hdt.shape, dtype=torch.float32, device="cuda")
+    o = torch.empty_like(v)
+    a = hm.scan_args(q, k, v, o, W_q=Wq, W_k=Wk, dt=dtt, A_log=A_log)
+    ws = hm.alloc_workspace(hm.hm_scan_workspace_size(a))
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    stream = torch.cuda.current_stream()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdt))
+    d2h = ho.numel() * ho.element_size()
+
+    def step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        dtt.copy_(hdt, non_blocking=True)
+        hm.hm_scan_chunked_fwd(a, stream)
+        ho.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    K = max(1, min(args.steps, 50))
+    ts = []
+    for _ in range(K):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(sum(x.elapsed_time(y) for x, y in ts) / K, world, torch)
+    return {"value": B * L * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K,
+            "call": "hm_scan_chunked_fwd (feature maps + scan) with pinned-host copies"}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    cfg = wl.PREFILL_PYTHIA
+    # each step: the oracle on every (batch, head) pair for a 64-token slice of
+    # the sequence (a bounded sample of the workload)
+    T = 64
+    inp = wl.scan_inputs(cfg, L=T)
+    for _ in range(args.warmup):
+        oracle.scan_fwd(inp["q"], inp["k"], inp["v"], inp["W_q"], inp["W_k"], dt=inp["dt"],
+                        A_log=inp["A_log"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.scan_fwd(inp["q"], inp["k"], inp["v"], inp["W_q"], inp["W_k"], dt=inp["dt"],
+                        A_log=inp["A_log"])
+    sec = (time.perf_counter() - t0) / max(1, args.steps)
+    value = cfg.B * T / sec
+    cores = min(oracle.omp_threads_in_use(), cfg.B * cfg.H)
+    sample = ("fp64 CPU oracle, all %d (batch, head) pairs x %d tokens per step"
+              % (cfg.B * cfg.H, T))
+    return {
+        "impl": "reference",
+        "metric": "tokens/sec of HedgeMamba mixer scan fwd on 1 B200; % of tensor/HBM roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "L": cfg.L, "H": cfg.H, "d": cfg.d,
+                   "F": cfg.F, "dv": cfg.dv},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill", "long"], default="prefill")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    cfg = {"prefill": wl.PREFILL_PYTHIA, "long": wl.PREFILL_LONG}[args.workload]
+    res = bench_prefill(cfg, args, rank, world, torch)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample, sec = oracle_prefill_rate(cfg)
+        res["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": sample, "seconds": sec}
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,230 @@
+/*
+ * hm.h -- C ABI of the HedgeMamba mixer-scan library (libhm.so), sm_100a.
+ *
+ * The library computes the HedgeMamba mixer's causal, normalised, decayed
+ * linear-attention scan and the pieces around it:
+ *
+ *   Hedgehog feature map   phi(x) = softmax([W x + b, -(W x + b)])   over 2p features
+ *   decay                  a_t = exp(-softplus(dt_t) * exp(A_log_h))  per (token, head)
+ *   recurrence             S_t = a_t S_{t-1} + phi(k_t) v_t^T
+ *                          z_t = a_t z_{t-1} + phi(k_t)
+ *                          o_t = (phi(q_t)^T S_t) / (phi(q_t)^T z_t)
+ *
+ * Sources:
+ *   "HedgeMamba: fusing linear attention and state space models" (gsyq.cn
+ *   news 1418924): sec. 2.1 (Hedgehog map: one Linear layer, concatenation
+ *   with its negation, softmax over the feature axis), sec. 2.3 and sec. 5.2
+ *   (mixer: value projection, two Hedgehog instances for q and k, the doubled
+ *   state giving numerator and denominator, division, gate, out projection;
+ *   short conv kept), sec. 5.3 (feature-map listing walk-through).
+ *   "Linear attention explained" (cnblogs ying-chease 22790249): sec. 2
+ *   (kernel form and associativity), sec. 3 (recurrent form S_i = S_{i-1} +
+ *   phi(k_i) v_i^T), sec. 5 (chunkwise mode for prefill, recurrent mode for
+ *   decode), the Q/K/V/S shape section ([b, h, n, d], S is d x d_v).
+ *   "State space models: Mamba, S4" (quant67 56-ssm): sec. 3.2 (dt through
+ *   softplus), sec. 4.2 (associative affine-map composition, used for the
+ *   state carry between sequence segments), sec. 6 (chunked SSD algorithm:
+ *   matmuls inside a block, recurrence between blocks).
+ *
+ * Conventions shared by every entry point
+ *   Layout    row-major.  Activations are token-major: [B, L, H, X] (X = d,
+ *             F = 2p or dv), i.e. element (b, t, h, x) at ((b*L + t)*H + h)*X + x.
+ *             States: S [B, H, F, dv] (row = feature f, column = value c),
+ *             z [B, H, F].  dt [B, L, H].  A_log [H].  All state is fp32.
+ *             Feature order: f < p is the "+" half (exp(u_f)), f >= p the "-" half.
+ *   Dtypes    hm_dtype per argument; dt, A_log, biases and states are fp32.
+ *   Pointers  device pointers (cudaMalloc'd or equivalent) unless stated.
+ *             Every base pointer must be 16-byte aligned.
+ *   Ownership the caller owns every buffer.  The library never allocates
+ *             or frees device memory and never synchronises the stream
+ *             (except hm_get_device_error, which says so).  All work is
+ *             enqueued on `stream` in order.
+ *   Errors    argument errors are detected on the host before anything is
+ *             enqueued and return HM_ERR_INVALID_ARG (or HM_ERR_UNSUPPORTED
+ *             for a valid shape that has no kernel); nothing is written.
+ *             Launch failures return HM_ERR_CUDA.  A kernel that detects an
+ *             internal fault (a bounded wait that expired) records it in a
+ *             per-device error word and exits early; hm_get_device_error
+ *             reads and clears it.  hm_last_error_detail() gives a
+ *             human-readable reason for the last non-OK status on the
+ *             calling host thread.  There is no CPU fallback: every result is
+ *             produced by this library's own CUDA kernels.
+ */
+#ifndef HM_H_
+#define HM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HM_API __attribute__((visibility("default")))
+#else
+#define HM_API
+#endif
+
+typedef struct CUstream_st *hm_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    HM_OK = 0,
+    HM_ERR_INVALID_ARG = 1,  /* bad pointer, shape, stride or alignment */
+    HM_ERR_UNSUPPORTED = 2,  /* valid arguments, but no kernel for this shape/dtype */
+    HM_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    HM_ERR_TIMEOUT = 4,      /* a kernel's bounded wait expired (device error word) */
+    HM_ERR_DEVICE = 5        /* a kernel reported another internal fault */
+} hm_status;
+
+typedef enum { HM_F32 = 0, HM_BF16 = 1 } hm_dtype;
+
+/* Static description of a status code.  Never NULL. */
+HM_API const char *hm_status_string(hm_status s);
+
+/* Reason for the last non-OK status returned on this host thread ("" if none). */
+HM_API const char *hm_last_error_detail(void);
+
+/* Library version string. */
+HM_API const char *hm_version(void);
+
+/*
+ * hm_featmap -- Hedgehog feature map (HedgeMamba explainer sec. 2.1, 5.3).
+ *
+ *   u = W_h x_r + b_h          (W_h is [p, d], b_h is [p] or absent)
+ *   phi_r = softmax([u, -u])   over the 2p features, "+" half first
+ *
+ * x      [rows, d] of x_dtype; row r belongs to head h = r mod H (so a
+ *        token-major [B, L, H, d] tensor is passed as rows = B*L*H).
+ * W      [p, d] of x_dtype for head 0; head h's matrix starts at
+ *        W + h * w_head_stride elements (w_head_stride = 0: shared by all heads).
+ * bias   fp32 [p] (+ h * p per head when w_head_stride != 0), or NULL.
+ * phi    [rows, 2p] of phi_dtype (written).
+ * Supported: d and p multiples of 16, 16 <= p <= 256, d <= 512.
+ */
+HM_API hm_status hm_featmap(const void *x, hm_dtype x_dtype, int64_t rows, int H, int d, int p,
+                     const void *W, int64_t w_head_stride, const float *bias,
+                     void *phi, hm_dtype phi_dtype, hm_stream_t stream);
+
+/*
+ * hm_scan_chunked_fwd -- prefill: feature maps on q and k, then the decayed
+ * normalised recurrence over the whole sequence (spec definition;
+ * HedgeMamba explainer sec. 2.3 and 5.2; linear-attention tutorial sec. 3 and
+ * sec. 5, chunkwise mode).  Computed chunkwise: inside a chunk by dense
+ * matmuls with the decay applied elementwise to the masked score tile,
+ * between chunks by carrying (S, z); long sequences are split into segments
+ * whose states are combined by the associative affine-map composition
+ * (SSM article sec. 4.2).  These are exact rewrites of the recurrence.
+ */
+typedef struct {
+    int64_t B, L;          /* batch, sequence length (L >= 0; L = 0 writes only the states) */
+    int H;                 /* heads */
+    int d;                 /* q/k head dim (input of the Hedgehog projection) */
+    int p;                 /* Hedgehog projection width; F = 2p.  Ignored when W_q == NULL */
+    int dv;                /* value head dim */
+    hm_dtype io_dtype;     /* dtype of q, k, v, W_q, W_k and o */
+    const void *q;         /* [B, L, H, d] */
+    const void *k;         /* [B, L, H, d] */
+    const void *v;         /* [B, L, H, dv] */
+    const void *W_q;       /* [p, d] (per head: + h*w_head_stride), or NULL: q, k already
+                              are feature vectors (F = d, entries must be > 0) */
+    const void *W_k;       /* [p, d] like W_q; must be NULL iff W_q is NULL */
+    int64_t w_head_stride; /* elements between heads' W (0 = shared) */
+    const float *b_q;      /* [p] bias of the q map (per head like W) or NULL */
+    const float *b_k;      /* [p] bias of the k map or NULL */
+    const float *dt;       /* [B, L, H] fp32, or NULL: a_t = 1 (no decay) */
+    const float *A_log;    /* [H] fp32; required when dt != NULL */
+    const float *S0;       /* [B, H, F, dv] initial state, or NULL (zero) */
+    const float *z0;       /* [B, H, F] initial state, or NULL (zero); NULL iff S0 NULL */
+    void *o;               /* [B, L, H, dv] of io_dtype (written) */
+    float *S_out;          /* [B, H, F, dv] final state, or NULL; may alias S0 */
+    float *z_out;          /* [B, H, F] final state, or NULL; may alias z0 */
+    void *workspace;       /* device scratch of >= hm_scan_workspace_size() bytes, 256-B aligned */
+    size_t workspace_bytes;
+} hm_scan_args;
+
+/* Bytes of workspace hm_scan_chunked_fwd needs for these arguments (0 on
+ * invalid arguments).  Linear in B*L*H (never quadratic in L). */
+HM_API size_t hm_scan_workspace_size(const hm_scan_args *a);
+
+HM_API hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stream);
+
+/*
+ * hm_step_decode -- one recurrent step per (batch, head) (linear-attention
+ * tutorial sec. 3 and sec. 5, recurrent mode): feature maps on the new q and
+ * k, then S <- a S + phi(k) v^T, z <- a z + phi(k), o = phi(q)^T S / phi(q)^T z.
+ * S and z are updated in place.
+ */
+typedef struct {
+    int64_t B;             /* independent sequences */
+    int H, d, p, dv;       /* as in hm_scan_args; F = 2p (or d when W_q == NULL) */
+    hm_dtype io_dtype;     /* dtype of q, k, v, W_q, W_k, o */
+    const void *q;         /* [B, H, d] */
+    const void *k;         /* [B, H, d] */
+    const void *v;         /* [B, H, dv] */
+    const void *W_q, *W_k; /* as in hm_scan_args (NULL: q, k are feature vectors) */
+    int64_t w_head_stride;
+    const float *b_q, *b_k;
+    const float *dt;       /* [B, H] fp32 or NULL (a = 1) */
+    const float *A_log;    /* [H] fp32 */
+    float *S;              /* [B, H, F, dv] fp32, read and written */
+    float *z;              /* [B, H, F] fp32, read and written */
+    void *o;               /* [B, H, dv] of io_dtype (written) */
+    void *workspace;       /* >= hm_decode_workspace_size() bytes, 256-B aligned */
+    size_t workspace_bytes;
+} hm_decode_args;
+
+HM_API size_t hm_decode_workspace_size(const hm_decode_args *a);
+
+HM_API hm_status hm_step_decode(const hm_decode_args *a, hm_stream_t stream);
+
+/*
+ * hm_mixer_fwd -- HedgeMamba mixer forward (HedgeMamba explainer sec. 2.3,
+ * 5.2; conv and gate kept, sec. 2.2/2.3; gate after the normalisation):
+ *
+ *   q, k, v, g = x W_{q,k,v,g}^T ;   dt = x W_dt^T (+ b_dt)
+ *   q, k, v    = depthwise causal conv of width K (zero left padding) + conv_b
+ *   o          = hm_scan_chunked_fwd(q, k, v) per head (d = E/H, Hedgehog W_hq/W_hk)
+ *   out        = (o * SiLU(g + b_g)) W_o^T
+ *
+ * No activation after the conv; no D skip; no RoPE (not part of this path).
+ * All matrices bf16 (fp32 accumulation); intermediates are stored in bf16.
+ */
+typedef struct {
+    int64_t B, L;
+    int d_model;           /* D */
+    int H;                 /* heads; E = H * d_head with d_head = E / H */
+    int E;                 /* width of q/k/v/g (= H * d_head) */
+    int p;                 /* Hedgehog width (F = 2p) */
+    int conv_k;            /* conv width K (1..8) */
+    const void *x;         /* [B, L, D] bf16 */
+    const void *W_q, *W_k, *W_v, *W_g; /* [E, D] bf16 */
+    const void *W_dt;      /* [H, D] bf16 */
+    const float *b_dt;     /* [H] or NULL */
+    const float *b_g;      /* [E] or NULL */
+    const float *conv_w;   /* [3, E, K] fp32 (q, k, v) */
+    const float *conv_b;   /* [3, E] fp32 or NULL */
+    const void *W_hq, *W_hk; /* [p, d_head] bf16, shared across heads */
+    const float *A_log;    /* [H] */
+    const void *W_o;       /* [D, E] bf16 */
+    void *out;             /* [B, L, D] bf16 (written) */
+} hm_mixer_args;
+
+HM_API size_t hm_mixer_workspace_size(const hm_mixer_args *a);
+
+HM_API hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t workspace_bytes,
+                       hm_stream_t stream);
+
+/* Number of kernels this library has enqueued in this process so far (all
+ * devices, all threads).  A diagnostic for launch accounting. */
+HM_API uint64_t hm_launch_count(void);
+
+/* Synchronises `stream`, then returns and clears the calling device's error
+ * word: HM_OK, HM_ERR_TIMEOUT (a bounded wait expired) or HM_ERR_DEVICE. */
+HM_API hm_status hm_get_device_error(hm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HM_H_ */

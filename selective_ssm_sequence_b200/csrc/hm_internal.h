@@ -1,0 +1,140 @@
+// hm_internal.h -- shared declarations of the libhm.so translation units.
+// Not part of the public ABI (that is include/hm.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "hm.h"
+
+namespace hm {
+
+// Per-device error word written by kernels whose bounded waits expire.
+// [0] = status (HM_ERR_TIMEOUT / HM_ERR_DEVICE), [1] = kernel id,
+// [2] = block index, [3] = site / detail.  Kernels receive its address.
+struct DevErr {
+    unsigned int *word;
+};
+
+enum KernelId : unsigned int {
+    KID_FEATMAP_SIMT = 1,
+    KID_FEATMAP_TC = 2,
+    KID_SCAN_SIMT = 3,
+    KID_SCAN_TC_STATE = 4,
+    KID_SCAN_TC_CARRY = 5,
+    KID_SCAN_TC_OUT = 6,
+    KID_DECODE = 7,
+    KID_GEMM_TC = 8,
+    KID_CONV = 9,
+};
+
+unsigned int *device_error_word();  // address of this device's error word (host)
+
+// Host-side count of kernels enqueued by the library (hm_launch_count).
+void count_launches(unsigned int n);
+
+// ---------------------------------------------------------------- device helpers
+
+__device__ __forceinline__ float hm_ld(const float *p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float hm_ld(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ void hm_st(float *p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void hm_st(__nv_bfloat16 *p, int64_t i, float v) { p[i] = __float2bfloat16_rn(v); }
+
+// softplus(x) = log(1 + e^x) without overflow; fp32.
+__device__ __forceinline__ float hm_softplus(float x) {
+    return x > 0.f ? x + log1pf(expf(-x)) : log1pf(expf(x));
+}
+
+// log of the decay a = exp(-softplus(dt) * exp(A_log)).
+__device__ __forceinline__ float hm_log_decay(float dt, float a_log) {
+    float rate = expf(a_log);
+    return rate == 0.f ? 0.f : -hm_softplus(dt) * rate;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ void report_error(DevErr e, unsigned int status, unsigned int kid,
+                                             unsigned int site) {
+    if (atomicCAS(e.word, 0u, status) == 0u) {
+        e.word[1] = kid;
+        e.word[2] = blockIdx.x + 65536u * blockIdx.y;
+        e.word[3] = site;
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+
+// Hedgehog map, SIMT (any dtype, any d/p that the host validated).
+cudaError_t launch_featmap_simt(const void *x, hm_dtype xt, int64_t rows, int H, int d, int p,
+                                const void *W, int64_t w_head_stride, const float *bias,
+                                void *phi, hm_dtype pt, cudaStream_t s);
+
+// Hedgehog map on tcgen05 (bf16 in, bf16 or fp32 out).  Returns
+// cudaErrorNotSupported if the shape has no tensor-core kernel.
+cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, const void *W,
+                              int64_t w_head_stride, const float *bias, void *phi, hm_dtype pt,
+                              DevErr err, cudaStream_t s);
+bool featmap_tc_supported(int64_t rows, int H, int d, int p, int64_t w_head_stride);
+
+// Generic SIMT chunk-free scan over precomputed features (fp32 state).
+struct ScanCore {
+    int64_t B, L;
+    int H, F, dv;
+    hm_dtype feat_dtype;  // dtype of phq/phk
+    hm_dtype io_dtype;    // dtype of v and o
+    const void *phq, *phk, *v;
+    const float *dt, *A_log;
+    const float *S0, *z0;
+    void *o;
+    float *S_out, *z_out;
+};
+cudaError_t launch_scan_simt(const ScanCore &c, cudaStream_t s);
+
+// Tensor-core chunked scan (bf16 features / v / o, F = 256, dv % 128 == 0).
+bool scan_tc_supported(const ScanCore &c);
+size_t scan_tc_workspace(const ScanCore &c);
+cudaError_t launch_scan_tc(const ScanCore &c, void *ws, size_t ws_bytes, DevErr err,
+                           cudaStream_t s);
+
+// Decode step over precomputed features.
+struct DecodeCore {
+    int64_t B;
+    int H, F, dv;
+    hm_dtype feat_dtype, io_dtype;
+    const void *phq, *phk, *v;
+    const float *dt, *A_log;
+    float *S, *z;
+    void *o;
+};
+cudaError_t launch_decode(const DecodeCore &c, cudaStream_t s);
+
+// bf16 GEMM C[M,N] = A[M,K] B[N,K]^T on tcgen05 with a fused epilogue.
+enum GemmEpi : int {
+    EPI_STORE_BF16 = 0,  // C bf16
+    EPI_STORE_F32 = 1,   // C fp32 (+ optional fp32 bias per column)
+};
+bool gemm_tc_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm_tc(const void *A, const void *Bm, int64_t M, int64_t N, int64_t K,
+                           void *C, int64_t ldc, GemmEpi epi, const float *bias, DevErr err,
+                           cudaStream_t s);
+
+// Depthwise causal conv over [B, L, C] bf16 with fp32 weights [C, K]; bf16 out.
+cudaError_t launch_causal_conv(const void *x, int64_t x_ld, int64_t B, int64_t L, int C, int K,
+                               const float *w, const float *bias, void *y, int64_t y_ld,
+                               cudaStream_t s);
+
+// y[r, c] = o[r, c] * SiLU(g[r, c] + b_g[c]) (bf16 in/out).
+cudaError_t launch_gate(const void *o, const void *g, int64_t g_ld, const float *b_g, int64_t rows,
+                        int E, void *y, cudaStream_t s);
+
+}  // namespace hm

@@ -43,33 +43,86 @@ def _key(seed: int, name: str) -> np.uint64:
     return np.uint64(_fnv1a64(name) ^ ((int(seed) * 0x9E3779B97F4A7C15) & 0xFFFFFFFFFFFFFFFF))
 
 
-def splitmix64(key: np.uint64, n: int) -> np.ndarray:
-    """n consecutive splitmix64 outputs for counter 1..n under ``key``."""
+def splitmix64_at(key: np.uint64, ctr: np.ndarray) -> np.ndarray:
+    """splitmix64 outputs for the given counters (uint64 array) under ``key``."""
     with np.errstate(over="ignore"):
-        ctr = np.arange(1, n + 1, dtype=np.uint64)
-        z = key + ctr * _GOLD
+        z = key + ctr.astype(np.uint64) * _GOLD
         z = (z ^ (z >> np.uint64(30))) * _M1
         z = (z ^ (z >> np.uint64(27))) * _M2
         z = z ^ (z >> np.uint64(31))
     return z
 
 
-def uniform(seed: int, name: str, shape, lo: float = 0.0, hi: float = 1.0) -> np.ndarray:
-    n = int(np.prod(shape)) if len(shape) else 1
-    u = ((splitmix64(_key(seed, name), n) >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
-    return (lo + (hi - lo) * u).reshape(shape)
+def splitmix64(key: np.uint64, n: int) -> np.ndarray:
+    """n consecutive splitmix64 outputs for counter 1..n under ``key``."""
+    return splitmix64_at(key, np.arange(1, n + 1, dtype=np.uint64))
 
 
-def normal(seed: int, name: str, shape, std: float = 1.0) -> np.ndarray:
-    n = int(np.prod(shape)) if len(shape) else 1
-    m = (n + 1) // 2
-    u = ((splitmix64(_key(seed, name), 2 * m) >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
-    u1, u2 = u[0::2], u[1::2]
+def _u01(bits: np.ndarray) -> np.ndarray:
+    return ((bits >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+
+
+def _flat_index(shape, index):
+    """Flat (C-order) indices of the sub-block ``index`` (a tuple of slices or
+    ints for the leading dimensions) of an array of ``shape``, built from
+    per-dimension index vectors (the full range is never materialised)."""
+    shape = tuple(int(x) for x in shape)
+    if index is None:
+        return np.arange(int(np.prod(shape)), dtype=np.int64).reshape(shape)
+    index = tuple(index) + (slice(None),) * (len(shape) - len(index))
+    strides = [int(np.prod(shape[i + 1:])) for i in range(len(shape))]
+    out = np.zeros((), dtype=np.int64)
+    for n, ix, st in zip(shape, index, strides):
+        if isinstance(ix, slice):
+            r = np.arange(n, dtype=np.int64)[ix]
+            out = out[..., None] + r * st
+        else:
+            out = out + int(ix) * st
+    return out
+
+
+def uniform(seed: int, name: str, shape, lo: float = 0.0, hi: float = 1.0, index=None) -> np.ndarray:
+    """Uniform(lo, hi) array of ``shape`` (or its sub-block ``index``): element n
+    uses counter n + 1."""
+    idx = _flat_index(shape, index)
+    u = _u01(splitmix64_at(_key(seed, name), (idx + 1).astype(np.uint64)))
+    return lo + (hi - lo) * u
+
+
+def normal(seed: int, name: str, shape, std: float = 1.0, index=None) -> np.ndarray:
+    """N(0, std^2) array of ``shape`` (or its sub-block ``index``).  Element n
+    is the cosine (n even) or sine (n odd) branch of Box-Muller on the uniform
+    pair with counters 2*(n//2) + 1 and 2*(n//2) + 2."""
+    if index is None and int(np.prod(shape)) > (1 << 22):
+        return _normal_chunked(seed, name, shape, std)
+    idx = _flat_index(shape, index)
+    m = (idx // 2).astype(np.uint64)
+    key = _key(seed, name)
+    u1 = _u01(splitmix64_at(key, 2 * m + np.uint64(1)))
+    u2 = _u01(splitmix64_at(key, 2 * m + np.uint64(2)))
     r = np.sqrt(-2.0 * np.log(u1))
-    z = np.empty(2 * m, dtype=np.float64)
-    z[0::2] = r * np.cos(2.0 * math.pi * u2)
-    z[1::2] = r * np.sin(2.0 * math.pi * u2)
-    return (std * z[:n]).reshape(shape)
+    ang = 2.0 * math.pi * u2
+    return std * np.where((idx & 1) == 0, r * np.cos(ang), r * np.sin(ang))
+
+
+def _normal_chunked(seed, name, shape, std):
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float64)
+    key = _key(seed, name)
+    step = 1 << 22
+    for s0 in range(0, n, step):
+        s1 = min(n, s0 + step)
+        m0, m1 = s0 // 2, (s1 + 1) // 2
+        mm = np.arange(m0, m1, dtype=np.uint64)
+        u1 = _u01(splitmix64_at(key, 2 * mm + np.uint64(1)))
+        u2 = _u01(splitmix64_at(key, 2 * mm + np.uint64(2)))
+        r = np.sqrt(-2.0 * np.log(u1))
+        ang = 2.0 * math.pi * u2
+        z = np.empty(2 * (m1 - m0), dtype=np.float64)
+        z[0::2] = r * np.cos(ang)
+        z[1::2] = r * np.sin(ang)
+        out[s0:s1] = z[s0 - 2 * m0:s1 - 2 * m0]
+    return std * out.reshape(shape)
 
 
 # --------------------------------------------------------------------------
@@ -216,27 +269,41 @@ def scan_inputs(cfg: ScanConfig, B: Optional[int] = None, L: Optional[int] = Non
     return out
 
 
-def decode_inputs(cfg: DecodeConfig, B: Optional[int] = None, steps: Optional[int] = None,
-                  prefill: Optional[int] = None) -> Dict[str, np.ndarray]:
-    """Prefill tokens [B, prefill, H, *] and per-step tokens [steps, B, H, *],
-    same distributions as the Pythia-shaped prefill (bf16 q/k/v/W, fp32 dt,
-    A_log ~ U(0, log 16))."""
-    B = cfg.B if B is None else B
-    n = cfg.steps if steps is None else steps
-    P = cfg.prefill if prefill is None else prefill
+def decode_weights(cfg: DecodeConfig) -> Dict[str, np.ndarray]:
+    """Hedgehog W_q, W_k (bf16, N(0, w_std^2)) and A_log ~ U(log 1, log 16)."""
     s = cfg.seed
     return {
         "W_q": store(normal(s, "W_q", (cfg.p, cfg.d), cfg.w_std), "bf16"),
         "W_k": store(normal(s, "W_k", (cfg.p, cfg.d), cfg.w_std), "bf16"),
         "A_log": store(uniform(s, "A_log", (cfg.H,), 0.0, math.log(16.0)), "f32"),
-        "pre_q": store(normal(s, "pre_q", (B, P, cfg.H, cfg.d)), "bf16"),
-        "pre_k": store(normal(s, "pre_k", (B, P, cfg.H, cfg.d)), "bf16"),
-        "pre_v": store(normal(s, "pre_v", (B, P, cfg.H, cfg.dv)), "bf16"),
-        "pre_dt": store(normal(s, "pre_dt", (B, P, cfg.H)), "f32"),
-        "q": store(normal(s, "step_q", (n, B, cfg.H, cfg.d)), "bf16"),
-        "k": store(normal(s, "step_k", (n, B, cfg.H, cfg.d)), "bf16"),
-        "v": store(normal(s, "step_v", (n, B, cfg.H, cfg.dv)), "bf16"),
-        "dt": store(normal(s, "step_dt", (n, B, cfg.H)), "f32"),
+    }
+
+
+def decode_prefill(cfg: DecodeConfig, index=None) -> Dict[str, np.ndarray]:
+    """The seeded prefill tokens [B, prefill, H, *] (bf16 q/k/v ~ N(0,1), fp32
+    dt ~ N(0,1)), or their sub-block ``index`` = (batch slice, token slice,
+    head slice)."""
+    s = cfg.seed
+    B, P, H = cfg.B, cfg.prefill, cfg.H
+    return {
+        "q": store(normal(s, "pre_q", (B, P, H, cfg.d), index=index), "bf16"),
+        "k": store(normal(s, "pre_k", (B, P, H, cfg.d), index=index), "bf16"),
+        "v": store(normal(s, "pre_v", (B, P, H, cfg.dv), index=index), "bf16"),
+        "dt": store(normal(s, "pre_dt", (B, P, H), index=index), "f32"),
+    }
+
+
+def decode_step_tokens(cfg: DecodeConfig, step: int) -> Dict[str, np.ndarray]:
+    """Token of decode step ``step`` for every (batch, head): q, k [B, H, d],
+    v [B, H, dv] (bf16, N(0,1)) and dt [B, H] (fp32, N(0,1))."""
+    s = cfg.seed
+    B, H = cfg.B, cfg.H
+    tag = "step%d_" % step
+    return {
+        "q": store(normal(s, tag + "q", (B, H, cfg.d)), "bf16"),
+        "k": store(normal(s, tag + "k", (B, H, cfg.d)), "bf16"),
+        "v": store(normal(s, tag + "v", (B, H, cfg.dv)), "bf16"),
+        "dt": store(normal(s, tag + "dt", (B, H)), "f32"),
     }
 
 
