@@ -171,6 +171,8 @@ def scan_args(q, k, v, o, W_q=None, W_k=None, dt=None, A_log=None, S0=None, z0=N
     if workspace is not None:
         a.workspace = _ptr(workspace)
         a.workspace_bytes = workspace.numel() * workspace.element_size()
+    # the struct holds raw addresses: keep the tensors alive as long as it lives
+    a._refs = (q, k, v, o, W_q, W_k, dt, A_log, S0, z0, S_out, z_out, b_q, b_k, workspace)
     return a
 
 
@@ -198,6 +200,7 @@ def decode_args(q, k, v, o, S, z, W_q=None, W_k=None, dt=None, A_log=None, b_q=N
     if workspace is not None:
         a.workspace = _ptr(workspace)
         a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a._refs = (q, k, v, o, S, z, W_q, W_k, dt, A_log, b_q, b_k, workspace)
     return a
 
 
@@ -222,6 +225,7 @@ def mixer_args(x, out, W_q, W_k, W_v, W_g, W_dt, conv_w, W_hq, W_hk, A_log, W_o,
     a.b_dt, a.b_g = _ptr(b_dt), _ptr(b_g)
     a.conv_w, a.conv_b = _ptr(conv_w), _ptr(conv_b)
     a.W_hq, a.W_hk, a.A_log = _ptr(W_hq), _ptr(W_hk), _ptr(A_log)
+    a._refs = (x, out, W_q, W_k, W_v, W_g, W_dt, conv_w, W_hq, W_hk, A_log, W_o, conv_b, b_g, b_dt)
     return a
 
 

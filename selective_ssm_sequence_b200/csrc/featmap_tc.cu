@@ -1,0 +1,313 @@
+// featmap_tc.cu -- Hedgehog feature map on the 5th-generation tensor cores.
+//
+//   u = W x (+ b)  ;  phi = softmax([u, -u])  over the 2p features
+//
+// (HedgeMamba explainer sec. 2.1 and 5.3.)  The projection is a dense GEMM
+// (rows x d) . (d x p), so it runs as tcgen05.mma (bf16 operands from shared
+// memory, fp32 accumulator in TMEM).  Per CTA: one head (blockIdx.y) whose
+// W [p, d] is loaded once by TMA and stays in shared memory; 128-row tiles of
+// x stream through a 2-stage TMA ring.  Warp roles:
+//   warp 0      TMA producer (one elected lane)
+//   warp 1      TMEM allocator and MMA issuer (one elected lane)
+//   warps 2..5  epilogue: tcgen05.ld of one accumulator row per thread, the
+//               negate / concatenate / softmax in registers, and the store.
+// Two TMEM accumulators let the MMA of tile i+1 overlap the epilogue of tile i.
+// The kernel is bound by HBM (x in, phi out); MMA and exp work hide under it.
+#include "tc_common.cuh"
+
+namespace hm {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128;     // rows per tile (MMA M)
+constexpr int kStages = 2;   // x tiles in flight
+constexpr int kThreads = 192;
+
+template <int D, int P>
+struct FmLayout {
+    static constexpr int kChunks = D / 64;                  // 128-byte K chunks
+    static constexpr int kWBytes = kChunks * P * 128;       // W tile
+    static constexpr int kXChunkBytes = kBM * 128;          // one K chunk of an x tile
+    static constexpr int kXBytes = kChunks * kXChunkBytes;  // one x tile
+    static constexpr int kOffW = 0;
+    static constexpr int kOffX = kWBytes;
+    static constexpr int kOffBar = kOffX + kStages * kXBytes;
+    static constexpr int kSmem = kOffBar + 256 + 1024;      // + barriers, + alignment slack
+    static constexpr int kTmemCols = 2 * P <= 32 ? 32 : (2 * P <= 64 ? 64 : (2 * P <= 128 ? 128 : (2 * P <= 256 ? 256 : 512)));
+};
+
+struct FmBars {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t wbar;
+    uint64_t accf[2];
+    uint64_t acce[2];
+    uint32_t tmem;
+    int abort;
+};
+
+__device__ __forceinline__ float fexp(float x) { return exp2f(x * 1.4426950408889634f); }
+
+template <int D, int P, typename TP>
+__global__ void __launch_bounds__(kThreads, 1)
+featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
+                  int64_t Tv, int Hv, const float *__restrict__ bias, int bias_per_head,
+                  TP *__restrict__ phi, DevErr err) {
+    using Lay = FmLayout<D, P>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sW = smem + Lay::kOffW;
+    uint8_t *sX = smem + Lay::kOffX;
+    FmBars *bars = (FmBars *)(smem + Lay::kOffBar);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    const int64_t ntiles = (Tv + kBM - 1) / kBM;
+    volatile int *abort_flag = &bars->abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        mbar_init(&bars->wbar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->accf[b], 1);
+            mbar_init(&bars->acce[b], 128);
+        }
+        bars->abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(&bars->tmem, Lay::kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmx);
+            tma_prefetch_desc(&tmw);
+            mbar_arrive_expect_tx(&bars->wbar, Lay::kWBytes);
+            for (int c = 0; c < Lay::kChunks; ++c)
+                tma_load_2d(sW + c * P * 128, &tmw, &bars->wbar, c * 64, h * P);
+            int it = 0;
+            for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!mbar_wait(&bars->empty[s], ph ^ 1, abort_flag, err, KID_FEATMAP_TC, 1)) break;
+                mbar_arrive_expect_tx(&bars->full[s], Lay::kXBytes);
+                uint8_t *dst = sX + s * Lay::kXBytes;
+                for (int c = 0; c < Lay::kChunks; ++c)
+                    tma_load_3d(dst + c * Lay::kXChunkBytes, &tmx, &bars->full[s], c * 64, h,
+                                (int)(tile * kBM));
+            }
+            // make sure no copy is still landing in shared memory before exit
+            const int issued = it;
+            for (int j = issued - kStages; j < issued; ++j) {
+                if (j < 0) continue;
+                const int s = j % kStages;
+                for (uint32_t i = 0; i < kWaitPolls; ++i)
+                    if (mbar_try_wait(&bars->full[s], (j / kStages) & 1)) break;
+            }
+            for (uint32_t i = 0; i < kWaitPolls; ++i)
+                if (mbar_try_wait(&bars->wbar, 0)) break;
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (elect_one()) {
+            constexpr uint32_t idesc = idesc_bf16(kBM, P, false, false);
+            bool ok = mbar_wait(&bars->wbar, 0, abort_flag, err, KID_FEATMAP_TC, 2);
+            int it = 0;
+            for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                const int b = it & 1;
+                const uint32_t bph = (it >> 1) & 1;
+                if (!mbar_wait(&bars->acce[b], bph ^ 1, abort_flag, err, KID_FEATMAP_TC, 3)) break;
+                if (!mbar_wait(&bars->full[s], ph, abort_flag, err, KID_FEATMAP_TC, 4)) break;
+                tc_fence_after();
+                const uint32_t xa = smem_u32(sX + s * Lay::kXBytes);
+                const uint32_t wa = smem_u32(sW);
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const int c = k >> 2, kk = k & 3;
+                    const uint64_t ad = desc_k_sw128(xa + c * Lay::kXChunkBytes + kk * 32);
+                    const uint64_t bd = desc_k_sw128(wa + c * P * 128 + kk * 32);
+                    mma_ss(tmem + b * P, ad, bd, idesc, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars->empty[s]);
+                mma_commit(&bars->accf[b]);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int q = warp & 3;              // TMEM lane quarter of this warp
+        const int row_in_tile = q * 32 + lane;
+        int it = 0;
+        constexpr int F = 2 * P;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int b = it & 1;
+            const uint32_t bph = (it >> 1) & 1;
+            if (!mbar_wait(&bars->accf[b], bph, abort_flag, err, KID_FEATMAP_TC, 5)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem + b * P + ((uint32_t)(q * 32) << 16);
+            const float *bh = bias ? bias + (bias_per_head ? (int64_t)h * P : 0) : nullptr;
+            // pass 1: m = max |u|
+            float m = 0.f;
+#pragma unroll
+            for (int c = 0; c < P; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    float u = __uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f);
+                    m = fmaxf(m, fabsf(u));
+                }
+            }
+            // pass 2: Z = sum exp(u - m) + exp(-u - m)
+            float Z = 0.f;
+#pragma unroll
+            for (int c = 0; c < P; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + c, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    float u = __uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f);
+                    Z += fexp(u - m) + fexp(-u - m);
+                }
+            }
+            const float inv = 1.f / Z;
+            const int64_t t = tile * kBM + row_in_tile;
+            const bool valid = t < Tv;
+            TP *out = phi + (t * Hv + h) * (int64_t)F;
+            // pass 3: normalise and store
+#pragma unroll
+            for (int c = 0; c < P; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + c, r);
+                tmem_wait_ld();
+                if (c + 32 >= P) {
+                    // last chunk read: the accumulator can be reused
+                    tc_fence_before();
+                    mbar_arrive(&bars->acce[b]);
+                }
+                if (valid) {
+#pragma unroll
+                    for (int j0 = 0; j0 < 32; j0 += 8) {
+                        float e1[8], e2[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            float u = __uint_as_float(r[j0 + j]) + (bh ? bh[c + j0 + j] : 0.f);
+                            e1[j] = fexp(u - m) * inv;
+                            e2[j] = fexp(-u - m) * inv;
+                        }
+                        if constexpr (sizeof(TP) == 2) {
+                            uint4 v1, v2;
+                            __nv_bfloat162 *p1 = reinterpret_cast<__nv_bfloat162 *>(&v1);
+                            __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&v2);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                p1[j] = __floats2bfloat162_rn(e1[2 * j], e1[2 * j + 1]);
+                                p2[j] = __floats2bfloat162_rn(e2[2 * j], e2[2 * j + 1]);
+                            }
+                            *reinterpret_cast<uint4 *>(out + c + j0) = v1;
+                            *reinterpret_cast<uint4 *>(out + P + c + j0) = v2;
+                        } else {
+                            float4 *o1 = reinterpret_cast<float4 *>(out + c + j0);
+                            float4 *o2 = reinterpret_cast<float4 *>(out + P + c + j0);
+                            o1[0] = make_float4(e1[0], e1[1], e1[2], e1[3]);
+                            o1[1] = make_float4(e1[4], e1[5], e1[6], e1[7]);
+                            o2[0] = make_float4(e2[0], e2[1], e2[2], e2[3]);
+                            o2[1] = make_float4(e2[4], e2[5], e2[6], e2[7]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, Lay::kTmemCols);
+    }
+}
+
+template <int D, int P, typename TP>
+cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head_stride,
+               const float *bias, void *phi, DevErr err, cudaStream_t s) {
+    using Lay = FmLayout<D, P>;
+    const bool per_head = w_head_stride != 0;
+    const int Hv = per_head ? H : 1;
+    const int64_t Tv = rows / Hv;
+    CUtensorMap tmx, tmw;
+    {
+        uint64_t dims[3] = {(uint64_t)D, (uint64_t)Hv, (uint64_t)Tv};
+        uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)Hv * D * 2};
+        uint32_t box[3] = {64, 1, kBM};
+        if (!tc::make_tmap_bf16(&tmx, x, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        // W rows: head h's [P, D] starts at row h * P when the stride is P * D
+        uint64_t dims[2] = {(uint64_t)D, (uint64_t)Hv * P};
+        uint64_t strides[1] = {(uint64_t)D * 2};
+        uint32_t box[2] = {64, (uint32_t)P};
+        if (!tc::make_tmap_bf16(&tmw, W, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    auto kern = featmap_tc_kernel<D, P, TP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t ntiles = (Tv + kBM - 1) / kBM;
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t per_head_ctas = (sms + Hv - 1) / Hv;
+    if (per_head_ctas > ntiles) per_head_ctas = ntiles;
+    if (per_head_ctas < 1) per_head_ctas = 1;
+    dim3 grid((unsigned)per_head_ctas, (unsigned)Hv);
+    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx, tmw, Tv, Hv, bias, per_head ? 1 : 0, (TP *)phi, err);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool featmap_tc_supported(int64_t rows, int H, int d, int p, int64_t w_head_stride) {
+    if (rows <= 0) return false;
+    if (!(d == 64 || d == 128 || d == 256)) return false;
+    if (!(p == 64 || p == 128)) return false;
+    if (w_head_stride != 0 && (w_head_stride != (int64_t)p * d || rows % H != 0 || H > 65535)) return false;
+    const int Hv = w_head_stride ? H : 1;
+    if (rows / Hv > 0x7fffffffLL - 256) return false;  // TMA coordinates are 32-bit
+    return true;
+}
+
+cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, const void *W,
+                              int64_t w_head_stride, const float *bias, void *phi, hm_dtype pt,
+                              DevErr err, cudaStream_t s) {
+    if (!featmap_tc_supported(rows, H, d, p, w_head_stride)) return cudaErrorNotSupported;
+#define HM_FM_CASE(DD, PP)                                                                  \
+    if (d == DD && p == PP)                                                                 \
+        return pt == HM_BF16                                                                \
+                   ? go<DD, PP, __nv_bfloat16>(x, rows, H, W, w_head_stride, bias, phi, err, s) \
+                   : go<DD, PP, float>(x, rows, H, W, w_head_stride, bias, phi, err, s);
+    HM_FM_CASE(64, 64)
+    HM_FM_CASE(64, 128)
+    HM_FM_CASE(128, 64)
+    HM_FM_CASE(128, 128)
+    HM_FM_CASE(256, 64)
+    HM_FM_CASE(256, 128)
+#undef HM_FM_CASE
+    return cudaErrorNotSupported;
+}
+
+}  // namespace hm

@@ -118,12 +118,15 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
         if (!aligned16(p)) return fail(HM_ERR_INVALID_ARG, "scan: pointers must be 16-byte aligned");
     ScanPlan pl{};
     pl.F = F;
-    pl.feat = a->io_dtype;
-    pl.phi_bytes = a->W_q ? round_up((size_t)rows * F * dsize(pl.feat), 256) : 0;
     ScanCore c{};
     c.B = a->B; c.L = a->L; c.H = a->H; c.F = F; c.dv = a->dv;
-    c.feat_dtype = pl.feat; c.io_dtype = a->io_dtype;
+    c.feat_dtype = a->io_dtype; c.io_dtype = a->io_dtype;
     pl.tc = scan_tc_supported(c);
+    // Features computed here are kept in fp32 for the CUDA-core path: its state
+    // update then adds exact products instead of bf16-rounded ones.
+    pl.feat = pl.tc ? HM_BF16 : HM_F32;
+    c.feat_dtype = pl.feat;
+    pl.phi_bytes = a->W_q ? round_up((size_t)rows * F * dsize(pl.feat), 256) : 0;
     pl.tc_bytes = pl.tc ? round_up(scan_tc_workspace(c), 256) : 0;
     pl.total = 2 * pl.phi_bytes + pl.tc_bytes;
     *plan = pl;

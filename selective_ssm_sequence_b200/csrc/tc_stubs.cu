@@ -1,11 +1,6 @@
 // placeholder until the tensor-core kernels land
 #include "hm_internal.h"
 namespace hm {
-bool featmap_tc_supported(int64_t, int, int, int, int64_t) { return false; }
-cudaError_t launch_featmap_tc(const void *, int64_t, int, int, int, const void *, int64_t,
-                              const float *, void *, hm_dtype, DevErr, cudaStream_t) {
-    return cudaErrorNotSupported;
-}
 bool scan_tc_supported(const ScanCore &) { return false; }
 size_t scan_tc_workspace(const ScanCore &) { return 0; }
 cudaError_t launch_scan_tc(const ScanCore &, void *, size_t, DevErr, cudaStream_t) {

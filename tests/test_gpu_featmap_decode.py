@@ -77,9 +77,10 @@ def _decode_gpu(hm, q, k, v, S, z, Wq, Wk, dt, A_log, io="bf16"):
     tq, tk, tv = dev_tensor(q, io), dev_tensor(k, io), dev_tensor(v, io)
     tS, tz = dev_tensor(S, "f32"), dev_tensor(z, "f32")
     o = torch.empty_like(tv)
-    args = hm.decode_args(tq, tk, tv, o, tS, tz, W_q=dev_tensor(Wq, io), W_k=dev_tensor(Wk, io),
-                          dt=dev_tensor(dt, "f32") if dt is not None else None,
-                          A_log=dev_tensor(A_log, "f32"))
+    tWq, tWk = dev_tensor(Wq, io), dev_tensor(Wk, io)
+    tdt = dev_tensor(dt, "f32") if dt is not None else None
+    tA = dev_tensor(A_log, "f32")
+    args = hm.decode_args(tq, tk, tv, o, tS, tz, W_q=tWq, W_k=tWk, dt=tdt, A_log=tA)
     ws = hm.alloc_workspace(hm.hm_decode_workspace_size(args))
     args.workspace, args.workspace_bytes = ws.data_ptr(), ws.numel()
     hm.hm_step_decode(args)
@@ -176,8 +177,8 @@ def test_decode_fp32_no_decay(hm):
     tq, tk, tv = (dev_tensor(inp[n][:, 39], "f32") for n in ("q", "k", "v"))
     tS, tz = dev_tensor(S32, "f32"), dev_tensor(z32, "f32")
     o = torch.empty_like(tv)
-    args = hm.decode_args(tq, tk, tv, o, tS, tz, W_q=dev_tensor(inp["W_q"], "f32"),
-                          W_k=dev_tensor(inp["W_k"], "f32"))
+    tWq, tWk = dev_tensor(inp["W_q"], "f32"), dev_tensor(inp["W_k"], "f32")
+    args = hm.decode_args(tq, tk, tv, o, tS, tz, W_q=tWq, W_k=tWk)
     ws = hm.alloc_workspace(hm.hm_decode_workspace_size(args))
     args.workspace, args.workspace_bytes = ws.data_ptr(), ws.numel()
     hm.hm_step_decode(args)
