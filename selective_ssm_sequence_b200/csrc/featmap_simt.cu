@@ -20,7 +20,8 @@ template <typename TX, typename TP>
 __global__ void __launch_bounds__(32 * kWarps)
 featmap_simt_kernel(const TX *__restrict__ x, int64_t rows, int H, int d, int p,
                     const TX *__restrict__ W, int64_t w_head_stride,
-                    const float *__restrict__ bias, TP *__restrict__ phi) {
+                    const float *__restrict__ bias, TP *__restrict__ phi,
+                    __nv_bfloat16 *__restrict__ phi_lo) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     for (int64_t r = (int64_t)blockIdx.x * kWarps + warp; r < rows;
@@ -55,8 +56,15 @@ featmap_simt_kernel(const TX *__restrict__ x, int64_t rows, int H, int d, int p,
         for (int t = 0; t < kMaxPerLane; ++t) {
             int j = t * 32 + lane;
             if (j < p) {
-                hm_st(out, j, expf(u[t] - m) * inv);
-                hm_st(out, p + j, expf(-u[t] - m) * inv);
+                const float e1 = expf(u[t] - m) * inv, e2 = expf(-u[t] - m) * inv;
+                hm_st(out, j, e1);
+                hm_st(out, p + j, e2);
+                if (phi_lo) {
+                    // rounding remainder of the bf16 value just stored
+                    __nv_bfloat16 *lo = phi_lo + r * 2 * p;
+                    lo[j] = __float2bfloat16_rn(e1 - __bfloat162float(__float2bfloat16_rn(e1)));
+                    lo[p + j] = __float2bfloat16_rn(e2 - __bfloat162float(__float2bfloat16_rn(e2)));
+                }
             }
         }
     }
@@ -64,12 +72,12 @@ featmap_simt_kernel(const TX *__restrict__ x, int64_t rows, int H, int d, int p,
 
 template <typename TX, typename TP>
 cudaError_t go(const void *x, int64_t rows, int H, int d, int p, const void *W, int64_t ws,
-               const float *bias, void *phi, cudaStream_t s) {
+               const float *bias, void *phi, void *phi_lo, cudaStream_t s) {
     int64_t blocks = (rows + kWarps - 1) / kWarps;
     if (blocks > 148 * 64) blocks = 148 * 64;
     if (blocks < 1) return cudaSuccess;
     featmap_simt_kernel<TX, TP><<<(unsigned)blocks, 32 * kWarps, 0, s>>>(
-        (const TX *)x, rows, H, d, p, (const TX *)W, ws, bias, (TP *)phi);
+        (const TX *)x, rows, H, d, p, (const TX *)W, ws, bias, (TP *)phi, (__nv_bfloat16 *)phi_lo);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -78,15 +86,16 @@ cudaError_t go(const void *x, int64_t rows, int H, int d, int p, const void *W, 
 
 cudaError_t launch_featmap_simt(const void *x, hm_dtype xt, int64_t rows, int H, int d, int p,
                                 const void *W, int64_t w_head_stride, const float *bias,
-                                void *phi, hm_dtype pt, cudaStream_t s) {
+                                void *phi, hm_dtype pt, cudaStream_t s, void *phi_lo) {
     if (rows == 0) return cudaSuccess;
+    if (phi_lo && pt != HM_BF16) return cudaErrorInvalidValue;
     if (xt == HM_F32 && pt == HM_F32)
-        return go<float, float>(x, rows, H, d, p, W, w_head_stride, bias, phi, s);
+        return go<float, float>(x, rows, H, d, p, W, w_head_stride, bias, phi, nullptr, s);
     if (xt == HM_F32 && pt == HM_BF16)
-        return go<float, __nv_bfloat16>(x, rows, H, d, p, W, w_head_stride, bias, phi, s);
+        return go<float, __nv_bfloat16>(x, rows, H, d, p, W, w_head_stride, bias, phi, phi_lo, s);
     if (xt == HM_BF16 && pt == HM_F32)
-        return go<__nv_bfloat16, float>(x, rows, H, d, p, W, w_head_stride, bias, phi, s);
-    return go<__nv_bfloat16, __nv_bfloat16>(x, rows, H, d, p, W, w_head_stride, bias, phi, s);
+        return go<__nv_bfloat16, float>(x, rows, H, d, p, W, w_head_stride, bias, phi, nullptr, s);
+    return go<__nv_bfloat16, __nv_bfloat16>(x, rows, H, d, p, W, w_head_stride, bias, phi, phi_lo, s);
 }
 
 }  // namespace hm

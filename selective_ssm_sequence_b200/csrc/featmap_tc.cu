@@ -54,7 +54,7 @@ template <int D, int P, typename TP>
 __global__ void __launch_bounds__(kThreads, 1)
 featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                   int64_t Tv, int Hv, const float *__restrict__ bias, int bias_per_head,
-                  TP *__restrict__ phi, DevErr err) {
+                  TP *__restrict__ phi, __nv_bfloat16 *__restrict__ phi_lo, DevErr err) {
     using Lay = FmLayout<D, P>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -219,6 +219,22 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                             }
                             *reinterpret_cast<uint4 *>(out + c + j0) = v1;
                             *reinterpret_cast<uint4 *>(out + P + c + j0) = v2;
+                            if (phi_lo) {
+                                // remainder phi - bf16(phi), so that hi + lo carries ~16 bits
+                                uint4 l1, l2;
+                                __nv_bfloat162 *q1 = reinterpret_cast<__nv_bfloat162 *>(&l1);
+                                __nv_bfloat162 *q2 = reinterpret_cast<__nv_bfloat162 *>(&l2);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    float2 h1 = __bfloat1622float2(p1[j]);
+                                    float2 h2 = __bfloat1622float2(p2[j]);
+                                    q1[j] = __floats2bfloat162_rn(e1[2 * j] - h1.x, e1[2 * j + 1] - h1.y);
+                                    q2[j] = __floats2bfloat162_rn(e2[2 * j] - h2.x, e2[2 * j + 1] - h2.y);
+                                }
+                                __nv_bfloat16 *lo = phi_lo + (t * Hv + h) * (int64_t)F;
+                                *reinterpret_cast<uint4 *>(lo + c + j0) = l1;
+                                *reinterpret_cast<uint4 *>(lo + P + c + j0) = l2;
+                            }
                         } else {
                             float4 *o1 = reinterpret_cast<float4 *>(out + c + j0);
                             float4 *o2 = reinterpret_cast<float4 *>(out + P + c + j0);
@@ -244,7 +260,7 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
 
 template <int D, int P, typename TP>
 cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head_stride,
-               const float *bias, void *phi, DevErr err, cudaStream_t s) {
+               const float *bias, void *phi, void *phi_lo, DevErr err, cudaStream_t s) {
     using Lay = FmLayout<D, P>;
     const bool per_head = w_head_stride != 0;
     const int Hv = per_head ? H : 1;
@@ -274,7 +290,8 @@ cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head
     if (per_head_ctas > ntiles) per_head_ctas = ntiles;
     if (per_head_ctas < 1) per_head_ctas = 1;
     dim3 grid((unsigned)per_head_ctas, (unsigned)Hv);
-    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx, tmw, Tv, Hv, bias, per_head ? 1 : 0, (TP *)phi, err);
+    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx, tmw, Tv, Hv, bias, per_head ? 1 : 0, (TP *)phi,
+                                            (__nv_bfloat16 *)phi_lo, err);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -293,13 +310,14 @@ bool featmap_tc_supported(int64_t rows, int H, int d, int p, int64_t w_head_stri
 
 cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, const void *W,
                               int64_t w_head_stride, const float *bias, void *phi, hm_dtype pt,
-                              DevErr err, cudaStream_t s) {
+                              DevErr err, cudaStream_t s, void *phi_lo) {
     if (!featmap_tc_supported(rows, H, d, p, w_head_stride)) return cudaErrorNotSupported;
+    if (phi_lo && pt != HM_BF16) return cudaErrorInvalidValue;
 #define HM_FM_CASE(DD, PP)                                                                  \
     if (d == DD && p == PP)                                                                 \
         return pt == HM_BF16                                                                \
-                   ? go<DD, PP, __nv_bfloat16>(x, rows, H, W, w_head_stride, bias, phi, err, s) \
-                   : go<DD, PP, float>(x, rows, H, W, w_head_stride, bias, phi, err, s);
+                   ? go<DD, PP, __nv_bfloat16>(x, rows, H, W, w_head_stride, bias, phi, phi_lo, err, s) \
+                   : go<DD, PP, float>(x, rows, H, W, w_head_stride, bias, phi, nullptr, err, s);
     HM_FM_CASE(64, 64)
     HM_FM_CASE(64, 128)
     HM_FM_CASE(128, 64)

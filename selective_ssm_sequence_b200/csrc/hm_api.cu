@@ -72,11 +72,11 @@ hm_status check_featmap(const void *x, hm_dtype xt, int64_t rows, int H, int d, 
 
 cudaError_t run_featmap(const void *x, hm_dtype xt, int64_t rows, int H, int d, int p,
                         const void *W, int64_t wstride, const float *bias, void *phi, hm_dtype pt,
-                        cudaStream_t s) {
+                        cudaStream_t s, void *phi_lo = nullptr) {
     if (xt == HM_BF16 && featmap_tc_supported(rows, H, d, p, wstride))
         return launch_featmap_tc(x, rows, H, d, p, W, wstride, bias, phi, pt,
-                                 DevErr{device_error_word()}, s);
-    return launch_featmap_simt(x, xt, rows, H, d, p, W, wstride, bias, phi, pt, s);
+                                 DevErr{device_error_word()}, s, phi_lo);
+    return launch_featmap_simt(x, xt, rows, H, d, p, W, wstride, bias, phi, pt, s, phi_lo);
 }
 
 // ------------------------------------------------------------------ scan
@@ -85,6 +85,7 @@ struct ScanPlan {
     int F;
     hm_dtype feat;
     size_t phi_bytes;  // one of phq / phk (0 when q, k are features already)
+    size_t lo_bytes;   // rounding remainder of phk (tensor-core path with a returned state)
     size_t tc_bytes;   // tensor-core scan scratch
     bool tc;
     size_t total;
@@ -123,12 +124,14 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
     c.feat_dtype = a->io_dtype; c.io_dtype = a->io_dtype;
     pl.tc = scan_tc_supported(c);
     // Features computed here are kept in fp32 for the CUDA-core path: its state
-    // update then adds exact products instead of bf16-rounded ones.
-    pl.feat = pl.tc ? HM_BF16 : HM_F32;
+    // update then adds exact products instead of bf16-rounded ones.  When
+    // W_q == NULL the caller's q / k are the features and keep their dtype.
+    pl.feat = a->W_q ? (pl.tc ? HM_BF16 : HM_F32) : a->io_dtype;
     c.feat_dtype = pl.feat;
     pl.phi_bytes = a->W_q ? round_up((size_t)rows * F * dsize(pl.feat), 256) : 0;
+    pl.lo_bytes = (pl.tc && a->W_q && a->S_out) ? pl.phi_bytes : 0;
     pl.tc_bytes = pl.tc ? round_up(scan_tc_workspace(c), 256) : 0;
-    pl.total = 2 * pl.phi_bytes + pl.tc_bytes;
+    pl.total = 2 * pl.phi_bytes + pl.lo_bytes + pl.tc_bytes;
     *plan = pl;
     return HM_OK;
 }
@@ -312,27 +315,30 @@ hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stream) {
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t rows = a->B * a->L * a->H;
     char *ws = (char *)a->workspace;
-    const void *phq = a->q, *phk = a->k;
+    const void *phq = a->q, *phk = a->k, *phk_lo = nullptr;
     cudaError_t e;
     if (a->W_q && rows > 0) {
         void *wq = ws, *wk = ws + pl.phi_bytes;
+        void *wkl = pl.lo_bytes ? ws + 2 * pl.phi_bytes : nullptr;
         e = run_featmap(a->q, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->w_head_stride, a->b_q,
                         wq, pl.feat, s);
         if (e != cudaSuccess) return cuda_fail(e, "scan: featmap(q)");
         e = run_featmap(a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_k, a->w_head_stride, a->b_k,
-                        wk, pl.feat, s);
+                        wk, pl.feat, s, wkl);
         if (e != cudaSuccess) return cuda_fail(e, "scan: featmap(k)");
         phq = wq;
         phk = wk;
+        phk_lo = wkl;
     }
     ScanCore c{};
     c.B = a->B; c.L = a->L; c.H = a->H; c.F = pl.F; c.dv = a->dv;
     c.feat_dtype = pl.feat; c.io_dtype = a->io_dtype;
-    c.phq = phq; c.phk = phk; c.v = a->v;
+    c.phq = phq; c.phk = phk; c.phk_lo = phk_lo; c.v = a->v;
     c.dt = a->dt; c.A_log = a->A_log; c.S0 = a->S0; c.z0 = a->z0;
     c.o = a->o; c.S_out = a->S_out; c.z_out = a->z_out;
     if (pl.tc)
-        e = launch_scan_tc(c, ws + 2 * pl.phi_bytes, pl.tc_bytes, DevErr{device_error_word()}, s);
+        e = launch_scan_tc(c, ws + 2 * pl.phi_bytes + pl.lo_bytes, pl.tc_bytes,
+                           DevErr{device_error_word()}, s);
     else
         e = launch_scan_simt(c, s);
     return e == cudaSuccess ? HM_OK : cuda_fail(e, "scan launch");

@@ -77,13 +77,14 @@ __device__ __forceinline__ void report_error(DevErr e, unsigned int status, unsi
 // Hedgehog map, SIMT (any dtype, any d/p that the host validated).
 cudaError_t launch_featmap_simt(const void *x, hm_dtype xt, int64_t rows, int H, int d, int p,
                                 const void *W, int64_t w_head_stride, const float *bias,
-                                void *phi, hm_dtype pt, cudaStream_t s);
+                                void *phi, hm_dtype pt, cudaStream_t s, void *phi_lo = nullptr);
 
-// Hedgehog map on tcgen05 (bf16 in, bf16 or fp32 out).  Returns
+// Hedgehog map on tcgen05 (bf16 in, bf16 or fp32 out).  With phi_lo (bf16
+// out only), also writes the rounding remainder phi - bf16(phi).  Returns
 // cudaErrorNotSupported if the shape has no tensor-core kernel.
 cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, const void *W,
                               int64_t w_head_stride, const float *bias, void *phi, hm_dtype pt,
-                              DevErr err, cudaStream_t s);
+                              DevErr err, cudaStream_t s, void *phi_lo = nullptr);
 bool featmap_tc_supported(int64_t rows, int H, int d, int p, int64_t w_head_stride);
 
 // Generic SIMT chunk-free scan over precomputed features (fp32 state).
@@ -93,6 +94,7 @@ struct ScanCore {
     hm_dtype feat_dtype;  // dtype of phq/phk
     hm_dtype io_dtype;    // dtype of v and o
     const void *phq, *phk, *v;
+    const void *phk_lo;   // optional rounding remainder of phk (bf16), tensor-core path
     const float *dt, *A_log;
     const float *S0, *z0;
     void *o;
@@ -100,7 +102,7 @@ struct ScanCore {
 };
 cudaError_t launch_scan_simt(const ScanCore &c, cudaStream_t s);
 
-// Tensor-core chunked scan (bf16 features / v / o, F = 256, dv % 128 == 0).
+// Tensor-core chunked scan (bf16 features / v / o, F = 256, dv = 256).
 bool scan_tc_supported(const ScanCore &c);
 size_t scan_tc_workspace(const ScanCore &c);
 cudaError_t launch_scan_tc(const ScanCore &c, void *ws, size_t ws_bytes, DevErr err,

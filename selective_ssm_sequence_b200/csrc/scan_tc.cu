@@ -1,0 +1,864 @@
+// scan_tc.cu -- chunkwise decayed normalised scan on the 5th-generation tensor cores.
+//
+// Computes, for features phiq, phik (bf16, F = 256), values v (bf16) and the
+// decay a_t = exp(-softplus(dt_t) exp(A_log_h)):
+//   S_t = a_t S_{t-1} + phik_t v_t^T,  z_t = a_t z_{t-1} + phik_t,
+//   o_t = phiq_t^T S_t / phiq_t^T z_t
+// (HedgeMamba explainer sec. 2.3 / 5.2; linear-attention tutorial sec. 3-5).
+//
+// Chunkwise form (chunks of C = 64 tokens; cum_i = sum of log a over the
+// chunk up to token i; gamma = exp(cum_last)):
+//   P        = phiQ phiK^T                                     (tensor cores)
+//   Pt_ij    = P_ij exp(cum_i - cum_j) [j <= i]                (registers; the
+//              decay is applied elementwise, never factorised, so no term
+//              overflows)
+//   O        = Pt V + diag(exp(cum)) phiQ S_prev               (tensor cores)
+//   den      = rowsum(Pt) + exp(cum) (phiQ z_prev)
+//   S        = gamma S_prev + (w phiK)^T V,  w_j = exp(cum_last - cum_j) <= 1
+//   z        = gamma z_prev + sum_j w_j phik_j
+// These are exact rewrites of the recurrence.  The state is kept transposed
+// (S^T, value channel x feature) in TMEM: the state update V^T (w phiK) and the
+// readout S^T (e^cum phiQ)^T then both have the 128 value channels of a CTA as
+// their M dimension, and the readout takes its A operand (a bf16 copy of S^T)
+// straight from TMEM.
+//
+// Long sequences are cut into segments that run in parallel.  Three kernels:
+//   A  scan_state_kernel  local end state of each part (a run of chunks) from a
+//                         zero start, weights relative to the part end; with
+//                         hi / lo bf16 splits of w * phik the state update is
+//                         accurate to ~16 bits (used for the returned state).
+//   B  scan_carry_kernel  composes the parts' affine maps (S -> g S + S_part,
+//                         SSM article sec. 4.2) in fp32 to get each segment's
+//                         start state and the final state.
+//   C  scan_out_kernel    the chunk loop above over one segment, from its start
+//                         state, writing o.
+// One CTA owns (batch, head, half of the value channels, segment).
+#include <algorithm>
+
+#include "tc_common.cuh"
+
+namespace hm {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kC = 64;        // tokens per chunk
+constexpr int kF = 256;       // feature dimension
+constexpr int kN = 128;       // value channels per CTA
+constexpr int kBlk = kC * 128;  // one [64 rows x 128 B] block = 8 KB
+constexpr int kTileF = 4 * kBlk;   // [64 x 256] bf16 tile = 32 KB
+constexpr int kTileV = 2 * kBlk;   // [64 x 128] bf16 tile = 16 KB
+
+__device__ __forceinline__ float fexp(float x) { return exp2f(x * 1.4426950408889634f); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+struct Geo {
+    int64_t B, L;
+    int H, dv;
+    int nchunks;     // ceil(L / C)
+    int seg_chunks;  // chunks per output segment (multiple of part_chunks)
+    int G;           // output segments
+    int part_chunks; // chunks per state part
+    int NP;          // parts in the whole sequence
+    int NPc;         // parts whose state phase A computes (a prefix)
+};
+
+// ------------------------------------------------------------------ phase A
+
+struct AAux {
+    float w[2][kC];
+    float red[4];
+    float suf;         // sum of log a over the chunks already processed (later ones)
+    uint64_t full[2], empty[2], built, done;
+    uint32_t tmem;
+    int abort;
+};
+
+constexpr int kAOffAux = 2 * (2 * kTileF + kTileV);
+constexpr int kASmem = kAOffAux + (int)sizeof(AAux) + 1024;
+
+// One CTA: (batch, head, value half, part).  Chunks of the part run from the
+// last to the first so that the suffix sums of log a (the weights relative to
+// the part end) are accumulated from small to large magnitudes.
+__global__ void __launch_bounds__(192, 1)
+scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constant__ CUtensorMap tmkl,
+                  const __grid_constant__ CUtensorMap tmv, Geo g, const float *__restrict__ dt,
+                  const float *__restrict__ A_log, int split, int add_lo, float *__restrict__ S_part,
+                  float *__restrict__ z_part, float *__restrict__ lsum_part, DevErr err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    AAux *X = (AAux *)(smem + kAOffAux);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = blockIdx.x & 1;
+    const int part = (blockIdx.x >> 1) % g.NPc;
+    const int64_t bh = (blockIdx.x >> 1) / g.NPc;
+    const int64_t b = bh / g.H;
+    const int h = (int)(bh % g.H);
+    const int dv0 = half * kN;
+    const int c_first = part * g.part_chunks;
+    const int c_last = min(g.nchunks, c_first + g.part_chunks) - 1;
+    const int n = c_last - c_first + 1;
+    volatile int *abort_flag = &X->abort;
+    auto stage = [&](int s) { return smem + s * (2 * kTileF + kTileV); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&X->full[s], 1);
+            mbar_init(&X->empty[s], 1);
+        }
+        mbar_init(&X->built, 1);
+        mbar_init(&X->done, 1);
+        X->abort = 0;
+        X->suf = 0.f;
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(&X->tmem, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = X->tmem;
+
+    if (warp == 0) {
+        if (elect_one()) {
+            tma_prefetch_desc(&tmkh);
+            tma_prefetch_desc(&tmkl);
+            tma_prefetch_desc(&tmv);
+            int it = 0;
+            for (; it < n; ++it) {
+                const int s = it & 1;
+                if (!mbar_wait(&X->empty[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_STATE, 1)) break;
+                const int t0 = (c_last - it) * kC;
+                uint8_t *st = stage(s);
+                mbar_arrive_expect_tx(&X->full[s], add_lo ? 2 * kTileF + kTileV : kTileF + kTileV);
+                for (int bb = 0; bb < 4; ++bb)
+                    tma_load_4d(st + bb * kBlk, &tmkh, &X->full[s], bb * 64, h, t0, (int)b);
+                if (add_lo)
+                    for (int bb = 0; bb < 4; ++bb)
+                        tma_load_4d(st + kTileF + bb * kBlk, &tmkl, &X->full[s], bb * 64, h, t0, (int)b);
+                for (int bb = 0; bb < 2; ++bb)
+                    tma_load_4d(st + 2 * kTileF + bb * kBlk, &tmv, &X->full[s], dv0 + bb * 64, h, t0, (int)b);
+            }
+            for (int j = it - 2; j < it; ++j) {
+                if (j < 0) continue;
+                for (uint32_t i = 0; i < kWaitPolls; ++i)
+                    if (mbar_try_wait(&X->full[j & 1], (j >> 1) & 1)) break;
+            }
+        }
+    } else if (warp == 1) {
+        if (elect_one()) {
+            constexpr uint32_t idesc = idesc_bf16(128, 256, true, true);
+            for (int it = 0; it < n; ++it) {
+                const int s = it & 1;
+                if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_STATE, 2)) break;
+                if (!mbar_wait(&X->built, it & 1, abort_flag, err, KID_SCAN_TC_STATE, 3)) break;
+                tc_fence_after();
+                const uint32_t kh = smem_u32(stage(s));
+                const uint32_t kl = kh + kTileF;
+                const uint32_t vv = kh + 2 * kTileF;
+                for (int k = 0; k < kC / 16; ++k) {
+                    const uint64_t ad = desc_mn_sw128(vv + k * 2048, kBlk, 1024);
+                    mma_ss(tmem, ad, desc_mn_sw128(kh + k * 2048, kBlk, 1024), idesc,
+                           (it > 0 || k > 0) ? 1u : 0u);
+                    if (split) mma_ss(tmem, ad, desc_mn_sw128(kl + k * 2048, kBlk, 1024), idesc, 1u);
+                }
+                mma_commit(&X->empty[s]);
+            }
+            mma_commit(&X->done);
+        }
+    } else {
+        // builders: warps 2..5 (128 threads)
+        const int tb = threadIdx.x - 64;
+        const int f0 = 2 * tb;
+        const int bb = f0 >> 6, cc = (f0 & 63) >> 3, wi = f0 & 7;
+        const float alog = dt ? A_log[h] : 0.f;
+        float zacc0 = 0.f, zacc1 = 0.f;
+        bool ok = true;
+        for (int it = 0; it < n; ++it) {
+            const int s = it & 1;
+            const int t0 = (c_last - it) * kC;
+            // log a of the chunk's tokens and their exclusive suffix sums
+            float l = 0.f;
+            if (tb < kC && dt && t0 + tb < g.L) l = hm_log_decay(dt[(b * g.L + t0 + tb) * g.H + h], alog);
+            float x = l;  // inclusive suffix sum within the warp
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                float y = __shfl_down_sync(0xffffffffu, x, o);
+                if (lane + o < 32) x += y;
+            }
+            if (tb == 32) X->red[0] = x;       // sum over tokens 32..63
+            if (tb == 0) X->red[1] = 0.f;
+            named_sync(1, 128);
+            if (tb < 32) x += X->red[0];
+            // exclusive suffix: the inclusive value of the next token
+            float ex = __shfl_down_sync(0xffffffffu, x, 1);
+            if (lane == 31) ex = (tb == 31) ? X->red[0] : 0.f;
+            if (tb == 0) X->red[2] = x;        // chunk total
+            const float suf = X->suf;
+            if (tb < kC) X->w[s][tb] = fexp(suf + ex);
+            named_sync(1, 128);
+            if (tb == 0) X->suf = suf + X->red[2];
+            if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_STATE, 4)) {
+                ok = false;
+                break;
+            }
+            // weighted features, split into bf16 hi + lo, written back in place
+            const uint32_t kh = smem_u32(stage(s)) + bb * kBlk;
+            const uint32_t kl = kh + kTileF;
+#pragma unroll 4
+            for (int j = 0; j < kC; ++j) {
+                const uint32_t off = sw128_off(j, cc) + wi * 2;
+                float2 k = unpack_bf16x2(lds32(kh + off));
+                if (add_lo) {
+                    float2 k2 = unpack_bf16x2(lds32(kl + off));
+                    k.x += k2.x;
+                    k.y += k2.y;
+                }
+                const float wj = X->w[s][j];
+                const float kt0 = wj * k.x, kt1 = wj * k.y;
+                const uint32_t hi = pack_bf16x2(kt0, kt1);
+                const float2 hf = unpack_bf16x2(hi);
+                sts32(kh + off, hi);
+                if (split) {
+                    sts32(kl + off, pack_bf16x2(kt0 - hf.x, kt1 - hf.y));
+                    zacc0 += kt0;
+                    zacc1 += kt1;
+                } else {
+                    zacc0 += hf.x;
+                    zacc1 += hf.y;
+                }
+            }
+            fence_proxy_async_smem();
+            named_sync(1, 128);
+            if (tb == 0) mbar_arrive(&X->built);
+        }
+        if (ok && mbar_wait(&X->done, 0, abort_flag, err, KID_SCAN_TC_STATE, 5)) {
+            tc_fence_after();
+            const int q = warp & 3;
+            const int ch = 32 * q + lane;
+            const int64_t pidx = bh * g.NPc + part;
+            float *Sp = S_part + pidx * (int64_t)kF * g.dv + dv0 + ch;
+            for (int c0 = 0; c0 < kF; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + c0 + ((uint32_t)(32 * q) << 16), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) Sp[(int64_t)(c0 + j) * g.dv] = __uint_as_float(r[j]);
+            }
+            if (half == 0) {
+                z_part[pidx * kF + f0] = zacc0;
+                z_part[pidx * kF + f0 + 1] = zacc1;
+                if (tb == 0) lsum_part[pidx] = X->suf;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ------------------------------------------------------------------ phase B
+
+// Per (batch, head) and state element: walks the parts in order,
+//   acc <- exp(lsum_p) acc + part_p,
+// storing the state at each segment start and, when every part was
+// computed, the final state.  Elements [0, F*dv) are S, [F*dv, F*dv + F) are z.
+__global__ void scan_carry_kernel(Geo g, const float *__restrict__ S_part, const float *__restrict__ z_part,
+                                  const float *__restrict__ lsum_part, const float *__restrict__ S0,
+                                  const float *__restrict__ z0, float *__restrict__ S_start,
+                                  float *__restrict__ z_start, float *__restrict__ S_out,
+                                  float *__restrict__ z_out) {
+    const int64_t bh = blockIdx.y;
+    const int64_t nS = (int64_t)kF * g.dv;
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= nS + kF) return;
+    const bool isz = e >= nS;
+    const int64_t idx = isz ? e - nS : e;
+    float acc = 0.f;
+    if (isz) {
+        if (z0) acc = z0[bh * kF + idx];
+    } else if (S0) {
+        acc = S0[bh * nS + idx];
+    }
+    const int pps = g.seg_chunks / g.part_chunks;
+    for (int p = 0; p <= g.NPc; ++p) {
+        if (p > 0 && p % pps == 0 && p / pps < g.G) {
+            const int seg = p / pps;
+            if (isz) z_start[(bh * g.G + seg) * kF + idx] = acc;
+            else S_start[(bh * g.G + seg) * nS + idx] = acc;
+        }
+        if (p == g.NPc) break;
+        const float gam = expf(lsum_part[bh * g.NPc + p]);
+        const float add = isz ? z_part[(bh * g.NPc + p) * kF + idx] : S_part[(bh * g.NPc + p) * nS + idx];
+        acc = fmaf(gam, acc, add);
+    }
+    if (g.NPc == g.NP) {
+        if (isz) {
+            if (z_out) z_out[bh * kF + idx] = acc;
+        } else if (S_out) {
+            S_out[bh * nS + idx] = acc;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ phase C
+
+// TMEM columns
+constexpr uint32_t kColS = 0;    // S^T fp32        [128 value lanes x 256 features]
+constexpr uint32_t kColSB = 256; // S^T bf16 pairs  [128 x 128]
+constexpr uint32_t kColO = 384;  // O^T fp32        [128 x 64 tokens]
+constexpr uint32_t kColP = 448;  // P fp32, M = 64  [64 x 64]
+
+struct CAux {
+    float cum[2][kC];
+    float qs[2][kC];
+    float w[2][kC];
+    float rden[2][kC];   // 1 / den
+    float den_intra[kC];
+    float z[kF];
+    float gam[2];
+    float redb[4];
+    float redd[4];
+    uint64_t full[2], empty[2];
+    uint64_t p_full, p_empty, epib_done, o_full, o_empty, s_full, sbf_ready;
+    uint64_t den_ready[2];
+    uint32_t tmem;
+    int abort;
+};
+
+constexpr int kCStage = 2 * kTileF + kTileV;           // Q, K, V of one chunk
+constexpr int kCOffP = 2 * kCStage;
+constexpr int kCOffAux = kCOffP + kC * 128;
+constexpr int kCSmem = kCOffAux + (int)sizeof(CAux) + 1024;
+
+struct OutArgs {
+    Geo g;
+    const float *dt, *A_log;
+    __nv_bfloat16 *o;
+    const float *S0, *z0;            // segment 0 start state (caller layout) or null
+    const float *S_start, *z_start;  // segments >= 1: [BH][G][F*dv], [BH][G][F]
+};
+
+// sum of log a over the 64 tokens of the chunk starting at t0, reduced over
+// the first two warps of a 128-thread group (named barrier `bar_id`)
+__device__ __forceinline__ float chunk_log_total(const OutArgs &a, int64_t b, int h, float alog,
+                                                 int64_t t0, int tg, float *red, int bar_id) {
+    float l = 0.f;
+    if (tg < kC && a.dt && t0 + tg < a.g.L) l = hm_log_decay(a.dt[(b * a.g.L + t0 + tg) * a.g.H + h], alog);
+    l = warp_sum(l);
+    if ((tg & 31) == 0 && tg < kC) red[tg >> 5] = l;
+    named_sync(bar_id, 128);
+    const float tot = red[0] + red[1];
+    named_sync(bar_id, 128);
+    return tot;
+}
+
+__global__ void __launch_bounds__(448, 1)
+scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                const __grid_constant__ CUtensorMap tmv, OutArgs a, DevErr err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    CAux *X = (CAux *)(smem + kCOffAux);
+    const Geo &g = a.g;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = blockIdx.x & 1;
+    const int seg = (blockIdx.x >> 1) % g.G;
+    const int64_t bh = (blockIdx.x >> 1) / g.G;
+    const int64_t b = bh / g.H;
+    const int h = (int)(bh % g.H);
+    const int dv0 = half * kN;
+    const int c_begin = seg * g.seg_chunks;
+    const int c_end = min(g.nchunks, c_begin + g.seg_chunks);
+    const int nch = c_end - c_begin;
+    const float alog = a.dt ? a.A_log[h] : 0.f;
+    volatile int *abort_flag = &X->abort;
+    const uint32_t sbase = smem_u32(smem);
+    auto sQ = [&](int s) { return sbase + s * kCStage; };
+    auto sK = [&](int s) { return sbase + s * kCStage + kTileF; };
+    auto sV = [&](int s) { return sbase + s * kCStage + 2 * kTileF; };
+    const uint32_t sP = sbase + kCOffP;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&X->full[s], 1);
+            mbar_init(&X->empty[s], 1);
+            mbar_init(&X->den_ready[s], 1);
+        }
+        mbar_init(&X->p_full, 1);
+        mbar_init(&X->p_empty, 128);
+        mbar_init(&X->epib_done, 1);
+        mbar_init(&X->o_full, 1);
+        mbar_init(&X->o_empty, 128);
+        mbar_init(&X->s_full, 1);
+        mbar_init(&X->sbf_ready, 128);
+        X->abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(&X->tmem, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = X->tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+            int it = 0;
+            for (; it < nch; ++it) {
+                const int s = it & 1;
+                if (!mbar_wait(&X->empty[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 1)) break;
+                const int t0 = (c_begin + it) * kC;
+                mbar_arrive_expect_tx(&X->full[s], kCStage);
+                uint8_t *q = smem + s * kCStage;
+                for (int bb = 0; bb < 4; ++bb)
+                    tma_load_4d(q + bb * kBlk, &tmq, &X->full[s], bb * 64, h, t0, (int)b);
+                for (int bb = 0; bb < 4; ++bb)
+                    tma_load_4d(q + kTileF + bb * kBlk, &tmk, &X->full[s], bb * 64, h, t0, (int)b);
+                for (int bb = 0; bb < 2; ++bb)
+                    tma_load_4d(q + 2 * kTileF + bb * kBlk, &tmv, &X->full[s], dv0 + bb * 64, h, t0, (int)b);
+            }
+            for (int j = it - 2; j < it; ++j) {
+                if (j < 0) continue;
+                for (uint32_t i = 0; i < kWaitPolls; ++i)
+                    if (mbar_try_wait(&X->full[j & 1], (j >> 1) & 1)) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            constexpr uint32_t idP = idesc_bf16(64, 64, false, false);     // P = phiQ phiK^T
+            constexpr uint32_t idOi = idesc_bf16(128, 64, false, false);   // O^T = S^T phiQ~^T
+            constexpr uint32_t idOa = idesc_bf16(128, 64, true, false);    // O^T += V^T Pt^T
+            constexpr uint32_t idS = idesc_bf16(128, 256, true, true);     // S^T += V^T K~
+            for (int it = 0; it < nch; ++it) {
+                const int s = it & 1;
+                const uint32_t par = it & 1;
+                if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 2)) break;
+                if (!mbar_wait(&X->p_empty, par ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 3)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < kF / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBlk + (k & 3) * 32;
+                    mma_ss(tmem + kColP, desc_k_sw128(sQ(s) + off), desc_k_sw128(sK(s) + off), idP,
+                           k > 0 ? 1u : 0u);
+                }
+                mma_commit(&X->p_full);
+                if (!mbar_wait(&X->epib_done, par, abort_flag, err, KID_SCAN_TC_OUT, 4)) break;
+                if (!mbar_wait(&X->sbf_ready, par, abort_flag, err, KID_SCAN_TC_OUT, 5)) break;
+                if (!mbar_wait(&X->o_empty, par ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 6)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < kF / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kBlk + (k & 3) * 32;
+                    mma_ts(tmem + kColO, tmem + kColSB + k * 8, desc_k_sw128(sQ(s) + off), idOi,
+                           k > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int k = 0; k < kC / 16; ++k)
+                    mma_ss(tmem + kColO, desc_mn_sw128(sV(s) + k * 2048, kBlk, 1024),
+                           desc_k_sw128(sP + k * 32), idOa, 1u);
+                mma_commit(&X->o_full);
+#pragma unroll
+                for (int k = 0; k < kC / 16; ++k)
+                    mma_ss(tmem + kColS, desc_mn_sw128(sV(s) + k * 2048, kBlk, 1024),
+                           desc_mn_sw128(sK(s) + k * 2048, kBlk, 1024), idS, 1u);
+                mma_commit(&X->s_full);
+                mma_commit(&X->empty[s]);
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ WG-B: scores, features
+        const int tb = threadIdx.x - 64;
+        const int q = warp & 3;
+        {
+            const float *zi = nullptr;
+            if (seg == 0) zi = a.z0 ? a.z0 + bh * kF : nullptr;
+            else zi = a.z_start + (bh * g.G + seg) * kF;
+            for (int f = tb; f < kF; f += 128) X->z[f] = zi ? zi[f] : 0.f;
+        }
+        named_sync(1, 128);
+        for (int it = 0; it < nch; ++it) {
+            const int s = it & 1;
+            const int64_t t0 = (int64_t)(c_begin + it) * kC;
+            // (1) decay of the chunk: cum, exp(cum), weights, gamma
+            {
+                float l = 0.f;
+                if (tb < kC && a.dt && t0 + tb < g.L) l = hm_log_decay(a.dt[(b * g.L + t0 + tb) * g.H + h], alog);
+                float x = l;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    float y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                if (tb == 31) X->redb[0] = x;
+                named_sync(1, 128);
+                if (tb >= 32 && tb < kC) x += X->redb[0];
+                if (tb == kC - 1) X->redb[1] = x;
+                named_sync(1, 128);
+                const float total = X->redb[1];
+                if (tb < kC) {
+                    X->cum[s][tb] = x;
+                    X->qs[s][tb] = fexp(x);
+                    X->w[s][tb] = fexp(total - x);
+                }
+                if (tb == 0) X->gam[s] = fexp(total);
+                named_sync(1, 128);
+            }
+            // (2) scores: Pt = P * exp(cum_i - cum_j) on j <= i, row sums; Pt -> smem (bf16)
+            if (!mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7)) break;
+            if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8)) break;
+            tc_fence_after();
+            {
+                uint32_t pr[64];
+                const uint32_t ta = tmem + kColP + ((uint32_t)(32 * q) << 16);
+                tmem_ld32(ta, pr);
+                tmem_ld32(ta + 32, pr + 32);
+                tmem_wait_ld();
+                if (lane < 16) {
+                    const int i = 16 * q + lane;
+                    const float ci = X->cum[s][i];
+                    float rs = 0.f;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = cc * 8 + 2 * e;
+                            const float e0 = (j <= i) ? __uint_as_float(pr[j]) * fexp(ci - X->cum[s][j]) : 0.f;
+                            const float e1 = (j + 1 <= i) ? __uint_as_float(pr[j + 1]) * fexp(ci - X->cum[s][j + 1]) : 0.f;
+                            pk[e] = pack_bf16x2(e0, e1);
+                            const float2 r = unpack_bf16x2(pk[e]);
+                            rs += r.x + r.y;
+                        }
+                        sts128(sP + sw128_off(i, cc), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                    }
+                    X->den_intra[i] = rs;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&X->p_empty);
+            named_sync(1, 128);
+            // (3) phiQ rows scaled by exp(cum_i) in place; den = rowsum + e^cum phiq . z
+            {
+                const int i = tb >> 1, hf = tb & 1;
+                const float qsi = X->qs[s][i];
+                float dot = 0.f;
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+                    const int bb = 2 * hf + blk;
+                    const uint32_t base = sQ(s) + bb * kBlk;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const uint32_t ad = base + sw128_off(i, cc);
+                        uint4 v = lds128(ad);
+                        uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
+                        const int f = bb * 64 + cc * 8;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = unpack_bf16x2(pv[e]);
+                            pv[e] = pack_bf16x2(x.x * qsi, x.y * qsi);
+                            const float2 r = unpack_bf16x2(pv[e]);
+                            dot += r.x * X->z[f + 2 * e] + r.y * X->z[f + 2 * e + 1];
+                        }
+                        sts128(ad, v);
+                    }
+                }
+                dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+                if (hf == 0) X->rden[s][i] = 1.f / (X->den_intra[i] + dot);
+            }
+            // (4) weighted features w_j phik_j in place (bf16) and the z update
+            {
+                const int f0 = 2 * tb;
+                const int bb = f0 >> 6, cc = (f0 & 63) >> 3, wi = f0 & 7;
+                const uint32_t base = sK(s) + bb * kBlk;
+                float z0a = 0.f, z1a = 0.f;
+#pragma unroll 8
+                for (int j = 0; j < kC; ++j) {
+                    const uint32_t ad = base + sw128_off(j, cc) + wi * 2;
+                    const float2 k = unpack_bf16x2(lds32(ad));
+                    const float wj = X->w[s][j];
+                    const uint32_t pk = pack_bf16x2(wj * k.x, wj * k.y);
+                    const float2 r = unpack_bf16x2(pk);
+                    z0a += r.x;
+                    z1a += r.y;
+                    sts32(ad, pk);
+                }
+                named_sync(1, 128);  // every reader of z in step (3) is done
+                const float gm = X->gam[s];
+                X->z[f0] = fmaf(gm, X->z[f0], z0a);
+                X->z[f0 + 1] = fmaf(gm, X->z[f0 + 1], z1a);
+            }
+            fence_proxy_async_smem();
+            named_sync(1, 128);
+            if (tb == 0) {
+                mbar_arrive(&X->epib_done);
+                mbar_arrive(&X->den_ready[s]);
+            }
+        }
+    } else if (warp < 10) {
+        // ------------------------------------------------------------ WG-C: outputs
+        const int q = warp & 3;
+        const int ch = 32 * q + lane;
+        for (int it = 0; it < nch; ++it) {
+            const int s = it & 1;
+            if (!mbar_wait(&X->o_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 9)) break;
+            if (!mbar_wait(&X->den_ready[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 10)) break;
+            tc_fence_after();
+            uint32_t r[64];
+            const uint32_t ta = tmem + kColO + ((uint32_t)(32 * q) << 16);
+            tmem_ld32(ta, r);
+            tmem_ld32(ta + 32, r + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&X->o_empty);
+            const int64_t t0 = (int64_t)(c_begin + it) * kC;
+            __nv_bfloat16 *op = a.o + ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
+            const int64_t tstride = (int64_t)g.H * g.dv;
+#pragma unroll
+            for (int i = 0; i < kC; ++i)
+                if (t0 + i < g.L) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]) * X->rden[s][i]);
+        }
+    } else {
+        // ------------------------------------------------------------ WG-D: state pass
+        const int td = threadIdx.x - 320;
+        const int q = warp & 3;
+        const int ch = 32 * q + lane;
+        const uint32_t lanebase = (uint32_t)(32 * q) << 16;
+        bool ok = true;
+        // prologue: start state -> bf16 copy (for the first readout) and fp32 x gamma_0
+        {
+            const float gam0 = fexp(chunk_log_total(a, b, h, alog, (int64_t)c_begin * kC, td, X->redd, 2));
+            const float *src = nullptr;
+            if (seg == 0) src = a.S0 ? a.S0 + bh * (int64_t)kF * g.dv : nullptr;
+            else src = a.S_start + (bh * g.G + seg) * (int64_t)kF * g.dv;
+            for (int c0 = 0; c0 < kF; c0 += 32) {
+                uint32_t v[32], pk[16];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    v[j] = __float_as_uint(src ? src[(int64_t)(c0 + j) * g.dv + dv0 + ch] : 0.f);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
+                tmem_st16(tmem + kColS + c0 + lanebase, v);
+                tmem_st16(tmem + kColS + c0 + 16 + lanebase, v + 16);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&X->sbf_ready);
+        }
+        for (int it = 0; ok && it + 1 < nch; ++it) {
+            const float gn = fexp(chunk_log_total(a, b, h, alog, (int64_t)(c_begin + it + 1) * kC, td, X->redd, 2));
+            if (!mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            for (int c0 = 0; c0 < kF; c0 += 32) {
+                uint32_t v[32], pk[16];
+                tmem_ld32(tmem + kColS + c0 + lanebase, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gn);
+                tmem_st16(tmem + kColS + c0 + lanebase, v);
+                tmem_st16(tmem + kColS + c0 + 16 + lanebase, v + 16);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&X->sbf_ready);
+        }
+        // the MMAs of the last chunk must be complete before TMEM is released
+        if (ok && nch > 0) mbar_wait(&X->s_full, (nch - 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 12);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+struct Plan {
+    Geo g;
+    size_t off_Spart, off_zpart, off_lsum, off_Sstart, off_zstart, total;
+};
+
+int num_sms() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0, v = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            sms = v;
+        else
+            sms = 148;
+    }
+    return sms;
+}
+
+size_t rup(size_t x) { return (x + 255) / 256 * 256; }
+
+Plan make_plan(const ScanCore &c, bool want_state) {
+    Plan p{};
+    Geo &g = p.g;
+    g.B = c.B;
+    g.L = c.L;
+    g.H = c.H;
+    g.dv = c.dv;
+    g.nchunks = (int)((c.L + kC - 1) / kC);
+    const int64_t heads2 = c.B * c.H * (c.dv / kN);  // CTAs per segment (value halves)
+    const int sms = num_sms();
+    int G = (int)std::max<int64_t>(1, sms / std::max<int64_t>(1, heads2));
+    if (G > g.nchunks) G = std::max(1, g.nchunks);
+    int seg_chunks = g.nchunks > 0 ? (g.nchunks + G - 1) / G : 1;
+    // parts: divide each segment so that the state phase fills the GPU
+    const int seg_state = want_state ? G : G - 1;
+    int pps = 1;
+    if (seg_state > 0) {
+        for (int d = seg_chunks; d >= 1; --d) {
+            if (seg_chunks % d) continue;
+            if (heads2 * seg_state * d <= sms) {
+                pps = d;
+                break;
+            }
+        }
+    }
+    g.part_chunks = seg_chunks / pps;
+    g.seg_chunks = seg_chunks;
+    g.G = g.nchunks > 0 ? (g.nchunks + seg_chunks - 1) / seg_chunks : 1;
+    g.NP = g.nchunks > 0 ? (g.nchunks + g.part_chunks - 1) / g.part_chunks : 0;
+    g.NPc = want_state ? g.NP : std::min(g.NP, (g.G - 1) * pps);
+    const int64_t BH = c.B * c.H;
+    const size_t nS = (size_t)kF * c.dv;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = rup(off + bytes); return o; };
+    p.off_Spart = take(sizeof(float) * BH * g.NPc * nS);
+    p.off_zpart = take(sizeof(float) * BH * g.NPc * kF);
+    p.off_lsum = take(sizeof(float) * BH * g.NPc);
+    p.off_Sstart = take(sizeof(float) * BH * g.G * nS);
+    p.off_zstart = take(sizeof(float) * BH * g.G * kF);
+    p.total = off;
+    return p;
+}
+
+bool tmap_tokens(CUtensorMap *m, const void *base, int64_t B, int64_t L, int H, int X, int box_x) {
+    // [B, L, H, X] bf16 viewed as (X, H, L, B); box (box_x, 1, C, 1)
+    uint64_t dims[4] = {(uint64_t)X, (uint64_t)H, (uint64_t)L, (uint64_t)B};
+    uint64_t strides[3] = {(uint64_t)X * 2, (uint64_t)H * X * 2, (uint64_t)L * H * X * 2};
+    uint32_t box[4] = {(uint32_t)box_x, 1, kC, 1};
+    return make_tmap_bf16(m, base, 4, dims, strides, box);
+}
+
+}  // namespace
+
+bool scan_tc_supported(const ScanCore &c) {
+    return c.io_dtype == HM_BF16 && c.feat_dtype == HM_BF16 && c.F == kF && c.dv % kN == 0 &&
+           c.dv == 2 * kN && c.L < (int64_t)1 << 30 && c.B < 65536 && c.H < 65536;
+}
+
+size_t scan_tc_workspace(const ScanCore &c) { return make_plan(c, true).total; }
+
+cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws, size_t ws_bytes,
+                                DevErr err, cudaStream_t s) {
+    const bool want_state = c.S_out != nullptr;
+    Plan p = make_plan(c, want_state);
+    if (p.total > ws_bytes) return cudaErrorInvalidValue;
+    Geo &g = p.g;
+    const int64_t BH = c.B * c.H;
+    const size_t nS = (size_t)kF * c.dv;
+    char *w = (char *)ws;
+    float *S_part = (float *)(w + p.off_Spart), *z_part = (float *)(w + p.off_zpart);
+    float *lsum = (float *)(w + p.off_lsum);
+    float *S_start = (float *)(w + p.off_Sstart), *z_start = (float *)(w + p.off_zstart);
+    cudaError_t e;
+    if (g.nchunks == 0) {
+        // empty sequence: the final state is the initial state
+        if (want_state) {
+            e = c.S0 ? cudaMemcpyAsync(c.S_out, c.S0, sizeof(float) * BH * nS, cudaMemcpyDeviceToDevice, s)
+                     : cudaMemsetAsync(c.S_out, 0, sizeof(float) * BH * nS, s);
+            if (e != cudaSuccess) return e;
+            e = c.z0 ? cudaMemcpyAsync(c.z_out, c.z0, sizeof(float) * BH * kF, cudaMemcpyDeviceToDevice, s)
+                     : cudaMemsetAsync(c.z_out, 0, sizeof(float) * BH * kF, s);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
+    CUtensorMap tq, tk, tkl, tv;
+    if (!tmap_tokens(&tq, c.phq, c.B, c.L, c.H, kF, 64) || !tmap_tokens(&tk, c.phk, c.B, c.L, c.H, kF, 64) ||
+        !tmap_tokens(&tv, c.v, c.B, c.L, c.H, c.dv, 64))
+        return cudaErrorInvalidValue;
+    // with a returned state, the weighted features of the state phase are split
+    // into bf16 hi + lo (and phik's own rounding remainder is added when given)
+    const bool split = want_state;
+    const bool add_lo = want_state && phk_lo != nullptr;
+    if (!tmap_tokens(&tkl, add_lo ? phk_lo : c.phk, c.B, c.L, c.H, kF, 64)) return cudaErrorInvalidValue;
+
+    if (g.NPc > 0) {
+        e = cudaFuncSetAttribute(scan_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kASmem);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = (unsigned)(2 * g.NPc * BH);
+        scan_state_kernel<<<grid, 192, kASmem, s>>>(tk, tkl, tv, g, c.dt, c.A_log, split ? 1 : 0,
+                                                    add_lo ? 1 : 0, S_part, z_part, lsum, err);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        dim3 gb((unsigned)((nS + kF + 255) / 256), (unsigned)BH);
+        scan_carry_kernel<<<gb, 256, 0, s>>>(g, S_part, z_part, lsum, c.S0, c.z0, S_start, z_start,
+                                             c.S_out, c.z_out);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    OutArgs oa{};
+    oa.g = g;
+    oa.dt = c.dt;
+    oa.A_log = c.A_log;
+    oa.o = (__nv_bfloat16 *)c.o;
+    oa.S0 = c.S0;
+    oa.z0 = c.z0;
+    oa.S_start = S_start;
+    oa.z_start = z_start;
+    e = cudaFuncSetAttribute(scan_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCSmem);
+    if (e != cudaSuccess) return e;
+    scan_out_kernel<<<(unsigned)(2 * g.G * BH), 448, kCSmem, s>>>(tq, tk, tv, oa, err);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_tc(const ScanCore &c, void *ws, size_t ws_bytes, DevErr err, cudaStream_t s) {
+    return launch_scan_tc_impl(c, c.phk_lo, ws, ws_bytes, err, s);
+}
+
+}  // namespace hm

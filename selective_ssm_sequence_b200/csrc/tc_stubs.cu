@@ -1,11 +1,6 @@
 // placeholder until the tensor-core kernels land
 #include "hm_internal.h"
 namespace hm {
-bool scan_tc_supported(const ScanCore &) { return false; }
-size_t scan_tc_workspace(const ScanCore &) { return 0; }
-cudaError_t launch_scan_tc(const ScanCore &, void *, size_t, DevErr, cudaStream_t) {
-    return cudaErrorNotSupported;
-}
 bool gemm_tc_supported(int64_t, int64_t, int64_t) { return false; }
 cudaError_t launch_gemm_tc(const void *, const void *, int64_t, int64_t, int64_t, void *, int64_t,
                            GemmEpi, const float *, DevErr, cudaStream_t) {
