@@ -8,7 +8,7 @@ pass of the whole hot path over one batch: the Hedgehog map on q and on k,
 then the decayed normalised chunked scan, each through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill|long|decode|mixer|tiny]
+                    [--workload prefill|long|decode|mixer]
 
 Multi-GPU (N > 1, launched by torchrun): every rank runs its own batch (its
 own seed); there is no data-path collective ("weak" scaling).  Times are
@@ -211,13 +211,35 @@ def bench_prefill(cfg, args, rank, world, torch):
     stream = torch.cuda.current_stream()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
 
+    calls = [lambda: hm.hm_featmap(q, Wq, phq, H=H),
+             lambda: hm.hm_featmap(k, Wk, phk, H=H),
+             lambda: hm.hm_scan_chunked_fwd(fargs)]
+    # Each C-ABI call is captured once into its own CUDA graph and replayed:
+    # the timed region then holds device work only (no Python / ctypes / host
+    # enqueue latency), and the per-call events still give the breakdown.
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    graphs = []
+    n0 = hm.hm_launch_count()
+    for c in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            c()
+        graphs.append(g)
+    launches_per_step = hm.hm_launch_count() - n0
+    torch.cuda.synchronize()
+
     def step(ev):
         ev[0].record(stream)
-        hm.hm_featmap(q, Wq, phq, H=H, stream=stream)
+        graphs[0].replay()
         ev[1].record(stream)
-        hm.hm_featmap(k, Wk, phk, H=H, stream=stream)
+        graphs[1].replay()
         ev[2].record(stream)
-        hm.hm_scan_chunked_fwd(fargs, stream)
+        graphs[2].replay()
         ev[3].record(stream)
 
     K, W = args.steps, args.warmup
@@ -232,12 +254,11 @@ def bench_prefill(cfg, args, rank, world, torch):
     assert hm.hm_get_device_error() == hm.HM_OK
     barrier(world)
     torch.cuda.synchronize()
-    launches0 = hm.hm_launch_count()
     for i in range(K):
         flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
-    launches = hm.hm_launch_count() - launches0
+    launches = launches_per_step * K
     barrier(world)
     torch.cuda.synchronize()
     sampler.stop()
@@ -301,7 +322,8 @@ def bench_prefill(cfg, args, rank, world, torch):
         "data": "synthetic (seeded splitmix64 + Box-Muller, rounded to bf16)",
         "config": {"workload": cfg.name, "B": B, "L": L, "H": H, "d": d, "F": F, "dv": dv,
                    "tokens_per_gpu": B * L, "l2": "512 MiB buffer written between timed steps",
-                   "step": "hm_featmap(q), hm_featmap(k), hm_scan_chunked_fwd(features)"},
+                   "step": "hm_featmap(q), hm_featmap(k), hm_scan_chunked_fwd(features)",
+                   "launch": "each call replayed from a CUDA graph captured once"},
         "roofline": roof,
         "step_roofline": {"bound": "tensor", "flops_per_token_head": fl_fm + fl_sc,
                           "achieved": step_flops / (ms_step * 1e-3) / 1e12, "peak": tf,
@@ -365,6 +387,150 @@ def bench_prefill_e2e(cfg, inp, Wq, Wk, A_log, args, world, torch, hm, flush):
             "call": "hm_scan_chunked_fwd (feature maps + scan) with pinned-host copies"}
 
 
+# ---------------------------------------------------------------- decode workload
+
+def bench_decode(cfg, args, rank, world, torch):
+    """512 consecutive hm_step_decode calls over 256 sequences x 8 heads with
+    an fp32 state (256 x 256 per head); the state starts from the GPU's own
+    1024-token prefill (hm_scan_chunked_fwd) of the seeded prompt.  The
+    per-step tokens cycle through 16 seeded steps.  Each step is replayed from a
+    CUDA graph (one featmap launch per q / k and one decode launch)."""
+    import selective_ssm_sequence_b200 as hm
+    peaks, peak_kind = load_peaks()
+    w = wl.decode_weights(cfg)
+    B, H, F, dv = cfg.B, cfg.H, cfg.F, cfg.dv
+    tWq, tWk = to_dev(w["W_q"], "bf16", torch), to_dev(w["W_k"], "bf16", torch)
+    tA = to_dev(w["A_log"], "f32", torch)
+    S = torch.empty(B, H, F, dv, device="cuda")
+    z = torch.empty(B, H, F, device="cuda")
+    # prefill in batch slices (keeps host-side generation small)
+    for b0 in range(0, B, 32):
+        pre = wl.decode_prefill(cfg, index=(slice(b0, b0 + 32),))
+        q, k, v = (to_dev(pre[n], "bf16", torch) for n in ("q", "k", "v"))
+        dtt = to_dev(pre["dt"], "f32", torch)
+        o = torch.empty_like(v)
+        a = hm.scan_args(q, k, v, o, W_q=tWq, W_k=tWk, dt=dtt, A_log=tA, S_out=S[b0:b0 + 32],
+                         z_out=z[b0:b0 + 32])
+        ws = hm.alloc_workspace(hm.hm_scan_workspace_size(a))
+        a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+        hm.hm_scan_chunked_fwd(a)
+    torch.cuda.synchronize()
+    nstep_tokens = 16
+    toks = [wl.decode_step_tokens(cfg, t) for t in range(nstep_tokens)]
+    tq = [to_dev(t["q"], "bf16", torch) for t in toks]
+    tk = [to_dev(t["k"], "bf16", torch) for t in toks]
+    tv = [to_dev(t["v"], "bf16", torch) for t in toks]
+    tdt = [to_dev(t["dt"], "f32", torch) for t in toks]
+    o = torch.empty(B, H, dv, dtype=torch.bfloat16, device="cuda")
+    dargs = [hm.decode_args(tq[i], tk[i], tv[i], o, S, z, W_q=tWq, W_k=tWk, dt=tdt[i], A_log=tA)
+             for i in range(nstep_tokens)]
+    ws = hm.alloc_workspace(hm.hm_decode_workspace_size(dargs[0]))
+    for a in dargs:
+        a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    stream = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    graphs = []
+    n0 = hm.hm_launch_count()
+    for a in dargs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            hm.hm_step_decode(a)
+        graphs.append(g)
+    per_step = (hm.hm_launch_count() - n0) // nstep_tokens
+    torch.cuda.synchronize()
+    steps = args.steps if args.steps else cfg.steps
+    for i in range(max(3, args.warmup)):
+        graphs[i % nstep_tokens].replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        graphs[i % nstep_tokens].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    assert hm.hm_get_device_error() == hm.HM_OK
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, torch)
+    state_bytes = B * H * (2 * F * dv * 4 + 2 * F * 4)
+    io_bytes = B * H * (2 * cfg.d * 2 + dv * 2 + 4 + dv * 2)
+    gbs = (state_bytes + io_bytes) / (ms * 1e-3) / 1e9
+    return {
+        "metric": "decode tokens/sec (one token per sequence per step)",
+        "value": B * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 io, fp32 state", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": B, "H": H, "F": F, "dv": dv,
+                   "l2": "state 1.08 GB per step, larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
+                     "bytes_per_step": state_bytes + io_bytes, "peak_source": peak_kind,
+                     "kernel": "whole step (2 featmap + 1 decode launch)"},
+        "gpu_launches": per_step * steps,
+        "clocks": sampler.summary(),
+    }
+
+
+# ---------------------------------------------------------------- mixer workload
+
+def bench_mixer(cfg, args, rank, world, torch):
+    """Full mixer forward (B8 L4096 D2048 H8), one hm_mixer_fwd per step,
+    replayed from a CUDA graph."""
+    import selective_ssm_sequence_b200 as hm
+    peaks, peak_kind = load_peaks()
+    w = wl.mixer_weights(cfg)
+    t = {k: to_dev(v, "f32" if k in ("conv_w", "A_log") else "bf16", torch) for k, v in w.items()}
+    x = to_dev(wl.mixer_x(cfg), "bf16", torch)
+    out = torch.empty_like(x)
+    a = hm.mixer_args(x, out, t["W_q"], t["W_k"], t["W_v"], t["W_g"], t["W_dt"], t["conv_w"],
+                      t["W_hq"], t["W_hk"], t["A_log"], t["W_o"], n_heads=cfg.H)
+    ws = hm.alloc_workspace(hm.hm_mixer_workspace_size(a))
+    stream = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        hm.hm_mixer_fwd(a, ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    n0 = hm.hm_launch_count()
+    with torch.cuda.graph(g, stream=cap):
+        hm.hm_mixer_fwd(a, ws)
+    per_step = hm.hm_launch_count() - n0
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    evs = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    sampler.stop()
+    assert hm.hm_get_device_error() == hm.HM_OK
+    ms = max_over_ranks(sum(x.elapsed_time(y) for x, y in evs) / args.steps, world, torch)
+    D, E, L, B = cfg.d_model, cfg.d_model, cfg.L, cfg.B
+    flops_tok = 2 * D * 4 * E + 2 * D * cfg.H + 2 * E * D + 2 * 2 * cfg.d_head * cfg.p * cfg.H \
+        + 4 * 2 * cfg.p * (cfg.d_head + 1) * cfg.H + 3 * 2 * cfg.conv * E
+    tf = flops_tok * B * L / (ms * 1e-3) / 1e12
+    return {
+        "metric": "mixer forward tokens/sec", "value": B * L * world / (ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": cfg.name, "B": B, "L": L, "d_model": D, "H": cfg.H},
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16_tflops"], "flops_per_token": flops_tok,
+                     "peak_source": peak_kind, "kernel": "whole mixer forward"},
+        "gpu_launches": per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -412,7 +578,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "long"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "long", "decode", "mixer"], default="prefill")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -431,9 +597,14 @@ def main():
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    cfg = {"prefill": wl.PREFILL_PYTHIA, "long": wl.PREFILL_LONG}[args.workload]
-    res = bench_prefill(cfg, args, rank, world, torch)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.workload == "decode":
+        res = bench_decode(wl.DECODE, args, rank, world, torch)
+    elif args.workload == "mixer":
+        res = bench_mixer(wl.MIXER, args, rank, world, torch)
+    else:
+        cfg = {"prefill": wl.PREFILL_PYTHIA, "long": wl.PREFILL_LONG}[args.workload]
+        res = bench_prefill(cfg, args, rank, world, torch)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in ("prefill", "long"):
         rate, cores, sample, sec = oracle_prefill_rate(cfg)
         res["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                "sample": sample, "seconds": sec}

@@ -9,9 +9,11 @@
 // x stream through a 2-stage TMA ring.  Warp roles:
 //   warp 0      TMA producer (one elected lane)
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2..5  epilogue: tcgen05.ld of one accumulator row per thread, the
+//   warps 2..9  two epilogue warpgroups taking alternate tiles: one
+//               accumulator row per thread, read from TMEM in two passes (a
+//               running max / normaliser, then the normalised features), the
 //               negate / concatenate / softmax in registers, and the store.
-// Two TMEM accumulators let the MMA of tile i+1 overlap the epilogue of tile i.
+// Four TMEM accumulators let the MMAs run ahead of both epilogue warpgroups.
 // The kernel is bound by HBM (x in, phi out); MMA and exp work hide under it.
 #include "tc_common.cuh"
 
@@ -23,7 +25,8 @@ using namespace tc;
 
 constexpr int kBM = 128;     // rows per tile (MMA M)
 constexpr int kStages = 2;   // x tiles in flight
-constexpr int kThreads = 192;
+constexpr int kEpiWG = 2;    // epilogue warpgroups (alternate tiles)
+constexpr int kThreads = 64 + 128 * kEpiWG;
 
 template <int D, int P>
 struct FmLayout {
@@ -35,15 +38,16 @@ struct FmLayout {
     static constexpr int kOffX = kWBytes;
     static constexpr int kOffBar = kOffX + kStages * kXBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;      // + barriers, + alignment slack
-    static constexpr int kTmemCols = 2 * P <= 32 ? 32 : (2 * P <= 64 ? 64 : (2 * P <= 128 ? 128 : (2 * P <= 256 ? 256 : 512)));
+    static constexpr int kAcc = 512 / P >= 4 ? 4 : 2;       // TMEM accumulators
+    static constexpr int kTmemCols = kAcc * P <= 256 ? 256 : 512;
 };
 
 struct FmBars {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t wbar;
-    uint64_t accf[2];
-    uint64_t acce[2];
+    uint64_t accf[4];
+    uint64_t acce[4];
     uint32_t tmem;
     int abort;
 };
@@ -56,6 +60,7 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                   int64_t Tv, int Hv, const float *__restrict__ bias, int bias_per_head,
                   TP *__restrict__ phi, __nv_bfloat16 *__restrict__ phi_lo, DevErr err) {
     using Lay = FmLayout<D, P>;
+    constexpr int NA = Lay::kAcc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *sW = smem + Lay::kOffW;
@@ -74,7 +79,7 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
             mbar_init(&bars->empty[s], 1);
         }
         mbar_init(&bars->wbar, 1);
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NA; ++b) {
             mbar_init(&bars->accf[b], 1);
             mbar_init(&bars->acce[b], 128);
         }
@@ -126,8 +131,8 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
             for (int64_t tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1;
-                const int b = it & 1;
-                const uint32_t bph = (it >> 1) & 1;
+                const int b = it % NA;
+                const uint32_t bph = (it / NA) & 1;
                 if (!mbar_wait(&bars->acce[b], bph ^ 1, abort_flag, err, KID_FEATMAP_TC, 3)) break;
                 if (!mbar_wait(&bars->full[s], ph, abort_flag, err, KID_FEATMAP_TC, 4)) break;
                 tc_fence_after();
@@ -146,103 +151,97 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
         }
     } else {
         // ---------------------------------------------------------------- epilogue
+        // warpgroup e takes tiles e, e + kEpiWG, ...; each thread one row.
+        const int e = (warp - 2) >> 2;
         const int q = warp & 3;              // TMEM lane quarter of this warp
         const int row_in_tile = q * 32 + lane;
-        int it = 0;
         constexpr int F = 2 * P;
-        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-            const int b = it & 1;
-            const uint32_t bph = (it >> 1) & 1;
+        const float *bh = bias ? bias + (bias_per_head ? (int64_t)h * P : 0) : nullptr;
+        int it = e;
+        for (int64_t tile = blockIdx.x + (int64_t)e * gridDim.x; tile < ntiles;
+             tile += (int64_t)kEpiWG * gridDim.x, it += kEpiWG) {
+            const int b = it % NA;
+            const uint32_t bph = (it / NA) & 1;
             if (!mbar_wait(&bars->accf[b], bph, abort_flag, err, KID_FEATMAP_TC, 5)) break;
             tc_fence_after();
             const uint32_t tbase = tmem + b * P + ((uint32_t)(q * 32) << 16);
-            const float *bh = bias ? bias + (bias_per_head ? (int64_t)h * P : 0) : nullptr;
-            // pass 1: m = max |u|
-            float m = 0.f;
-#pragma unroll
+            // pass 1: running max m of |u| and normaliser Z = sum exp(u - m) + exp(-u - m),
+            // rescaled whenever m grows (one extra exp per 32 columns)
+            float m = 0.f, Z = 0.f;
+#pragma unroll 1
             for (int c = 0; c < P; c += 32) {
                 uint32_t r[32];
                 tmem_ld32(tbase + c, r);
                 tmem_wait_ld();
+                float mc = m;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mc = fmaxf(mc, fabsf(__uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f)));
+                float zc = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    float u = __uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f);
-                    m = fmaxf(m, fabsf(u));
+                    const float u = __uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f);
+                    zc += fexp(u - mc) + fexp(-u - mc);
                 }
-            }
-            // pass 2: Z = sum exp(u - m) + exp(-u - m)
-            float Z = 0.f;
-#pragma unroll
-            for (int c = 0; c < P; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tbase + c, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    float u = __uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f);
-                    Z += fexp(u - m) + fexp(-u - m);
-                }
+                Z = Z * fexp(m - mc) + zc;
+                m = mc;
             }
             const float inv = 1.f / Z;
             const int64_t t = tile * kBM + row_in_tile;
             const bool valid = t < Tv;
             TP *out = phi + (t * Hv + h) * (int64_t)F;
-            // pass 3: normalise and store
-#pragma unroll
+            __nv_bfloat16 *lo = phi_lo ? phi_lo + (t * Hv + h) * (int64_t)F : nullptr;
+            // pass 2: normalised features, stored
+#pragma unroll 1
             for (int c = 0; c < P; c += 32) {
                 uint32_t r[32];
                 tmem_ld32(tbase + c, r);
                 tmem_wait_ld();
                 if (c + 32 >= P) {
-                    // last chunk read: the accumulator can be reused
                     tc_fence_before();
-                    mbar_arrive(&bars->acce[b]);
+                    mbar_arrive(&bars->acce[b]);   // last read of this accumulator
                 }
-                if (valid) {
+                if (!valid) continue;
 #pragma unroll
-                    for (int j0 = 0; j0 < 32; j0 += 8) {
-                        float e1[8], e2[8];
+                for (int j0 = 0; j0 < 32; j0 += 8) {
+                    float e1[8], e2[8];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            float u = __uint_as_float(r[j0 + j]) + (bh ? bh[c + j0 + j] : 0.f);
-                            e1[j] = fexp(u - m) * inv;
-                            e2[j] = fexp(-u - m) * inv;
+                    for (int j = 0; j < 8; ++j) {
+                        const float u = __uint_as_float(r[j0 + j]) + (bh ? bh[c + j0 + j] : 0.f);
+                        e1[j] = fexp(u - m) * inv;
+                        e2[j] = fexp(-u - m) * inv;
+                    }
+                    if constexpr (sizeof(TP) == 2) {
+                        uint4 v1, v2;
+                        uint32_t *p1 = reinterpret_cast<uint32_t *>(&v1);
+                        uint32_t *p2 = reinterpret_cast<uint32_t *>(&v2);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            p1[j] = pack_bf16x2(e1[2 * j], e1[2 * j + 1]);
+                            p2[j] = pack_bf16x2(e2[2 * j], e2[2 * j + 1]);
                         }
-                        if constexpr (sizeof(TP) == 2) {
-                            uint4 v1, v2;
-                            __nv_bfloat162 *p1 = reinterpret_cast<__nv_bfloat162 *>(&v1);
-                            __nv_bfloat162 *p2 = reinterpret_cast<__nv_bfloat162 *>(&v2);
+                        *reinterpret_cast<uint4 *>(out + c + j0) = v1;
+                        *reinterpret_cast<uint4 *>(out + P + c + j0) = v2;
+                        if (lo) {
+                            // remainder phi - bf16(phi), so that hi + lo carries ~16 bits
+                            uint4 l1, l2;
+                            uint32_t *q1 = reinterpret_cast<uint32_t *>(&l1);
+                            uint32_t *q2 = reinterpret_cast<uint32_t *>(&l2);
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
-                                p1[j] = __floats2bfloat162_rn(e1[2 * j], e1[2 * j + 1]);
-                                p2[j] = __floats2bfloat162_rn(e2[2 * j], e2[2 * j + 1]);
+                                const float2 h1 = unpack_bf16x2(p1[j]), h2 = unpack_bf16x2(p2[j]);
+                                q1[j] = pack_bf16x2(e1[2 * j] - h1.x, e1[2 * j + 1] - h1.y);
+                                q2[j] = pack_bf16x2(e2[2 * j] - h2.x, e2[2 * j + 1] - h2.y);
                             }
-                            *reinterpret_cast<uint4 *>(out + c + j0) = v1;
-                            *reinterpret_cast<uint4 *>(out + P + c + j0) = v2;
-                            if (phi_lo) {
-                                // remainder phi - bf16(phi), so that hi + lo carries ~16 bits
-                                uint4 l1, l2;
-                                __nv_bfloat162 *q1 = reinterpret_cast<__nv_bfloat162 *>(&l1);
-                                __nv_bfloat162 *q2 = reinterpret_cast<__nv_bfloat162 *>(&l2);
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    float2 h1 = __bfloat1622float2(p1[j]);
-                                    float2 h2 = __bfloat1622float2(p2[j]);
-                                    q1[j] = __floats2bfloat162_rn(e1[2 * j] - h1.x, e1[2 * j + 1] - h1.y);
-                                    q2[j] = __floats2bfloat162_rn(e2[2 * j] - h2.x, e2[2 * j + 1] - h2.y);
-                                }
-                                __nv_bfloat16 *lo = phi_lo + (t * Hv + h) * (int64_t)F;
-                                *reinterpret_cast<uint4 *>(lo + c + j0) = l1;
-                                *reinterpret_cast<uint4 *>(lo + P + c + j0) = l2;
-                            }
-                        } else {
-                            float4 *o1 = reinterpret_cast<float4 *>(out + c + j0);
-                            float4 *o2 = reinterpret_cast<float4 *>(out + P + c + j0);
-                            o1[0] = make_float4(e1[0], e1[1], e1[2], e1[3]);
-                            o1[1] = make_float4(e1[4], e1[5], e1[6], e1[7]);
-                            o2[0] = make_float4(e2[0], e2[1], e2[2], e2[3]);
-                            o2[1] = make_float4(e2[4], e2[5], e2[6], e2[7]);
+                            *reinterpret_cast<uint4 *>(lo + c + j0) = l1;
+                            *reinterpret_cast<uint4 *>(lo + P + c + j0) = l2;
                         }
+                    } else {
+                        float4 *o1 = reinterpret_cast<float4 *>(out + c + j0);
+                        float4 *o2 = reinterpret_cast<float4 *>(out + P + c + j0);
+                        o1[0] = make_float4(e1[0], e1[1], e1[2], e1[3]);
+                        o1[1] = make_float4(e1[4], e1[5], e1[6], e1[7]);
+                        o2[0] = make_float4(e2[0], e2[1], e2[2], e2[3]);
+                        o2[1] = make_float4(e2[4], e2[5], e2[6], e2[7]);
                     }
                 }
             }
@@ -280,7 +279,7 @@ cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head
         if (!tc::make_tmap_bf16(&tmw, W, 2, dims, strides, box)) return cudaErrorInvalidValue;
     }
     auto kern = featmap_tc_kernel<D, P, TP>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmem);
+    cudaError_t e = ensure_smem_limit(kern, Lay::kSmem);
     if (e != cudaSuccess) return e;
     const int64_t ntiles = (Tv + kBM - 1) / kBM;
     int sms = 148;

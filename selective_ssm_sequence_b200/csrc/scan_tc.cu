@@ -87,6 +87,7 @@ struct Geo {
 
 struct AAux {
     float w[2][kC];
+    float zred[4][kF];
     float red[4];
     float suf;         // sum of log a over the chunks already processed (later ones)
     uint64_t full[2], empty[2], built, done;
@@ -186,19 +187,26 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
             mma_commit(&X->done);
         }
     } else {
-        // builders: warps 2..5 (128 threads)
+        // builders: warps 2..5 (128 threads).  Thread: one 16-byte chunk (8
+        // features) of the 256-feature row (lane -> block, chunk) for the 16
+        // tokens of its warp's group.
         const int tb = threadIdx.x - 64;
-        const int f0 = 2 * tb;
-        const int bb = f0 >> 6, cc = (f0 & 63) >> 3, wi = f0 & 7;
+        const int bb = lane >> 3, cc = lane & 7;
+        const int tg = tb >> 5;
         const float alog = dt ? A_log[h] : 0.f;
-        float zacc0 = 0.f, zacc1 = 0.f;
+        float za[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) za[e] = 0.f;
+        auto token_l = [&](int t0) {
+            return (tb < kC && dt && t0 + tb < g.L) ? hm_log_decay(dt[(b * g.L + t0 + tb) * g.H + h], alog) : 0.f;
+        };
+        float l_next = token_l(c_last * kC);
         bool ok = true;
         for (int it = 0; it < n; ++it) {
             const int s = it & 1;
-            const int t0 = (c_last - it) * kC;
-            // log a of the chunk's tokens and their exclusive suffix sums
-            float l = 0.f;
-            if (tb < kC && dt && t0 + tb < g.L) l = hm_log_decay(dt[(b * g.L + t0 + tb) * g.H + h], alog);
+            const float l = l_next;
+            if (it + 1 < n) l_next = token_l((c_last - it - 1) * kC);
+            // exclusive suffix sums of log a within the chunk
             float x = l;  // inclusive suffix sum within the warp
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -206,7 +214,6 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
                 if (lane + o < 32) x += y;
             }
             if (tb == 32) X->red[0] = x;       // sum over tokens 32..63
-            if (tb == 0) X->red[1] = 0.f;
             named_sync(1, 128);
             if (tb < 32) x += X->red[0];
             // exclusive suffix: the inclusive value of the next token
@@ -225,32 +232,47 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
             const uint32_t kh = smem_u32(stage(s)) + bb * kBlk;
             const uint32_t kl = kh + kTileF;
 #pragma unroll 4
-            for (int j = 0; j < kC; ++j) {
-                const uint32_t off = sw128_off(j, cc) + wi * 2;
-                float2 k = unpack_bf16x2(lds32(kh + off));
-                if (add_lo) {
-                    float2 k2 = unpack_bf16x2(lds32(kl + off));
-                    k.x += k2.x;
-                    k.y += k2.y;
-                }
+            for (int jj = 0; jj < 16; ++jj) {
+                const int j = tg * 16 + jj;
+                const uint32_t off = sw128_off(j, cc);
+                uint4 vh = lds128(kh + off);
+                uint4 vl = make_uint4(0, 0, 0, 0);
+                if (add_lo) vl = lds128(kl + off);
+                uint32_t *ph = reinterpret_cast<uint32_t *>(&vh);
+                uint32_t *pl = reinterpret_cast<uint32_t *>(&vl);
                 const float wj = X->w[s][j];
-                const float kt0 = wj * k.x, kt1 = wj * k.y;
-                const uint32_t hi = pack_bf16x2(kt0, kt1);
-                const float2 hf = unpack_bf16x2(hi);
-                sts32(kh + off, hi);
-                if (split) {
-                    sts32(kl + off, pack_bf16x2(kt0 - hf.x, kt1 - hf.y));
-                    zacc0 += kt0;
-                    zacc1 += kt1;
-                } else {
-                    zacc0 += hf.x;
-                    zacc1 += hf.y;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 k = unpack_bf16x2(ph[e]);
+                    if (add_lo) {
+                        const float2 k2 = unpack_bf16x2(pl[e]);
+                        k.x += k2.x;
+                        k.y += k2.y;
+                    }
+                    const float kt0 = wj * k.x, kt1 = wj * k.y;
+                    ph[e] = pack_bf16x2(kt0, kt1);
+                    const float2 hf = unpack_bf16x2(ph[e]);
+                    if (split) {
+                        pl[e] = pack_bf16x2(kt0 - hf.x, kt1 - hf.y);
+                        za[2 * e] += kt0;
+                        za[2 * e + 1] += kt1;
+                    } else {
+                        za[2 * e] += hf.x;
+                        za[2 * e + 1] += hf.y;
+                    }
                 }
+                sts128(kh + off, vh);
+                if (split) sts128(kl + off, vl);
             }
             fence_proxy_async_smem();
             named_sync(1, 128);
             if (tb == 0) mbar_arrive(&X->built);
         }
+        // z of the part: reduce the four token groups' partial sums
+        const int f0 = bb * 64 + cc * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) X->zred[tg][f0 + e] = za[e];
+        named_sync(1, 128);
         if (ok && mbar_wait(&X->done, 0, abort_flag, err, KID_SCAN_TC_STATE, 5)) {
             tc_fence_after();
             const int q = warp & 3;
@@ -265,8 +287,11 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
                 for (int j = 0; j < 32; ++j) Sp[(int64_t)(c0 + j) * g.dv] = __uint_as_float(r[j]);
             }
             if (half == 0) {
-                z_part[pidx * kF + f0] = zacc0;
-                z_part[pidx * kF + f0 + 1] = zacc1;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int f = 2 * tb + e;
+                    z_part[pidx * kF + f] = X->zred[0][f] + X->zred[1][f] + X->zred[2][f] + X->zred[3][f];
+                }
                 if (tb == 0) lsum_part[pidx] = X->suf;
             }
         }
@@ -330,7 +355,7 @@ __global__ void scan_carry_kernel(Geo g, const float *__restrict__ S_part, const
 constexpr uint32_t kColS = 0;    // S^T fp32        [128 value lanes x 256 features]
 constexpr uint32_t kColSB = 256; // S^T bf16 pairs  [128 x 128]
 constexpr uint32_t kColO = 384;  // O^T fp32        [128 x 64 tokens]
-constexpr uint32_t kColP = 448;  // P fp32, M = 64  [64 x 64]
+constexpr uint32_t kColP = 448;  // [phiQ; phiK] phiK^T fp32 [128 x 64]; lanes 0..63 = P
 
 struct CAux {
     float cum[2][kC];
@@ -339,6 +364,7 @@ struct CAux {
     float rden[2][kC];   // 1 / den
     float den_intra[kC];
     float z[kF];
+    float zred[4][kF];   // per token-group partial sums of the weighted features
     float gam[2];
     float redb[4];
     float redd[4];
@@ -349,7 +375,13 @@ struct CAux {
     int abort;
 };
 
-constexpr int kCStage = 2 * kTileF + kTileV;           // Q, K, V of one chunk
+// Phase C stage: for each 64-feature block bb, the 64 phiQ rows and the 64
+// phiK rows are stored back to back ([Q | K], 16 KB), so that one M = 128
+// operand [phiQ; phiK] gives the score tile P = phiQ phiK^T in TMEM lanes
+// 0..63 with the plain 128-lane accumulator layout (lanes 64..127 hold
+// phiK phiK^T, which is not used).
+constexpr int kQKBlk = 2 * kBlk;                       // [Q | K] of one feature block
+constexpr int kCStage = 4 * kQKBlk + kTileV;           // Q, K, V of one chunk
 constexpr int kCOffP = 2 * kCStage;
 constexpr int kCOffAux = kCOffP + kC * 128;
 constexpr int kCSmem = kCOffAux + (int)sizeof(CAux) + 1024;
@@ -362,12 +394,16 @@ struct OutArgs {
     const float *S_start, *z_start;  // segments >= 1: [BH][G][F*dv], [BH][G][F]
 };
 
-// sum of log a over the 64 tokens of the chunk starting at t0, reduced over
-// the first two warps of a 128-thread group (named barrier `bar_id`)
-__device__ __forceinline__ float chunk_log_total(const OutArgs &a, int64_t b, int h, float alog,
-                                                 int64_t t0, int tg, float *red, int bar_id) {
-    float l = 0.f;
-    if (tg < kC && a.dt && t0 + tg < a.g.L) l = hm_log_decay(a.dt[(b * a.g.L + t0 + tg) * a.g.H + h], alog);
+// log a of token t0 + tg for the first 64 threads of a group (0 otherwise)
+__device__ __forceinline__ float token_log_decay(const OutArgs &a, int64_t b, int h, float alog,
+                                                 int64_t t0, int tg) {
+    if (tg < kC && a.dt && t0 + tg < a.g.L) return hm_log_decay(a.dt[(b * a.g.L + t0 + tg) * a.g.H + h], alog);
+    return 0.f;
+}
+
+// sum of the 64 per-token values l over the first two warps of a 128-thread
+// group (named barrier `bar_id`)
+__device__ __forceinline__ float chunk_total(float l, int tg, float *red, int bar_id) {
     l = warp_sum(l);
     if ((tg & 31) == 0 && tg < kC) red[tg >> 5] = l;
     named_sync(bar_id, 128);
@@ -396,9 +432,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     const float alog = a.dt ? a.A_log[h] : 0.f;
     volatile int *abort_flag = &X->abort;
     const uint32_t sbase = smem_u32(smem);
+    // block bb of phiQ at sQ(s) + bb * kQKBlk, of phiK at sK(s) + bb * kQKBlk
     auto sQ = [&](int s) { return sbase + s * kCStage; };
-    auto sK = [&](int s) { return sbase + s * kCStage + kTileF; };
-    auto sV = [&](int s) { return sbase + s * kCStage + 2 * kTileF; };
+    auto sK = [&](int s) { return sbase + s * kCStage + kBlk; };
+    auto sV = [&](int s) { return sbase + s * kCStage + 4 * kQKBlk; };
     const uint32_t sP = sbase + kCOffP;
 
     if (threadIdx.x == 0) {
@@ -436,12 +473,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 const int t0 = (c_begin + it) * kC;
                 mbar_arrive_expect_tx(&X->full[s], kCStage);
                 uint8_t *q = smem + s * kCStage;
-                for (int bb = 0; bb < 4; ++bb)
-                    tma_load_4d(q + bb * kBlk, &tmq, &X->full[s], bb * 64, h, t0, (int)b);
-                for (int bb = 0; bb < 4; ++bb)
-                    tma_load_4d(q + kTileF + bb * kBlk, &tmk, &X->full[s], bb * 64, h, t0, (int)b);
+                for (int bb = 0; bb < 4; ++bb) {
+                    tma_load_4d(q + bb * kQKBlk, &tmq, &X->full[s], bb * 64, h, t0, (int)b);
+                    tma_load_4d(q + bb * kQKBlk + kBlk, &tmk, &X->full[s], bb * 64, h, t0, (int)b);
+                }
                 for (int bb = 0; bb < 2; ++bb)
-                    tma_load_4d(q + 2 * kTileF + bb * kBlk, &tmv, &X->full[s], dv0 + bb * 64, h, t0, (int)b);
+                    tma_load_4d(q + 4 * kQKBlk + bb * kBlk, &tmv, &X->full[s], dv0 + bb * 64, h, t0, (int)b);
             }
             for (int j = it - 2; j < it; ++j) {
                 if (j < 0) continue;
@@ -452,7 +489,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (elect_one()) {
-            constexpr uint32_t idP = idesc_bf16(64, 64, false, false);     // P = phiQ phiK^T
+            constexpr uint32_t idP = idesc_bf16(128, 64, false, false);    // [phiQ; phiK] phiK^T
             constexpr uint32_t idOi = idesc_bf16(128, 64, false, false);   // O^T = S^T phiQ~^T
             constexpr uint32_t idOa = idesc_bf16(128, 64, true, false);    // O^T += V^T Pt^T
             constexpr uint32_t idS = idesc_bf16(128, 256, true, true);     // S^T += V^T K~
@@ -464,7 +501,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kF / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBlk + (k & 3) * 32;
+                    const uint32_t off = (k >> 2) * kQKBlk + (k & 3) * 32;
                     mma_ss(tmem + kColP, desc_k_sw128(sQ(s) + off), desc_k_sw128(sK(s) + off), idP,
                            k > 0 ? 1u : 0u);
                 }
@@ -475,7 +512,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kF / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kBlk + (k & 3) * 32;
+                    const uint32_t off = (k >> 2) * kQKBlk + (k & 3) * 32;
                     mma_ts(tmem + kColO, tmem + kColSB + k * 8, desc_k_sw128(sQ(s) + off), idOi,
                            k > 0 ? 1u : 0u);
                 }
@@ -487,7 +524,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
                 for (int k = 0; k < kC / 16; ++k)
                     mma_ss(tmem + kColS, desc_mn_sw128(sV(s) + k * 2048, kBlk, 1024),
-                           desc_mn_sw128(sK(s) + k * 2048, kBlk, 1024), idS, 1u);
+                           desc_mn_sw128(sK(s) + k * 2048, kQKBlk, 1024), idS, 1u);
                 mma_commit(&X->s_full);
                 mma_commit(&X->empty[s]);
             }
@@ -503,13 +540,14 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int f = tb; f < kF; f += 128) X->z[f] = zi ? zi[f] : 0.f;
         }
         named_sync(1, 128);
+        // log a of the next chunk's tokens is fetched one chunk ahead
+        float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, tb);
         for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
-            const int64_t t0 = (int64_t)(c_begin + it) * kC;
             // (1) decay of the chunk: cum, exp(cum), weights, gamma
             {
-                float l = 0.f;
-                if (tb < kC && a.dt && t0 + tb < g.L) l = hm_log_decay(a.dt[(b * g.L + t0 + tb) * g.H + h], alog);
+                const float l = l_next;
+                if (it + 1 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 1) * kC, tb);
                 float x = l;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -540,8 +578,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 tmem_ld32(ta, pr);
                 tmem_ld32(ta + 32, pr + 32);
                 tmem_wait_ld();
-                if (lane < 16) {
-                    const int i = 16 * q + lane;
+                if (q < 2) {  // lanes 0..63 hold the 64 rows of P
+                    const int i = 32 * q + lane;
                     const float ci = X->cum[s][i];
                     float rs = 0.f;
 #pragma unroll
@@ -572,7 +610,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
                 for (int blk = 0; blk < 2; ++blk) {
                     const int bb = 2 * hf + blk;
-                    const uint32_t base = sQ(s) + bb * kBlk;
+                    const uint32_t base = sQ(s) + bb * kQKBlk;
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc) {
                         const uint32_t ad = base + sw128_off(i, cc);
@@ -592,27 +630,44 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 dot += __shfl_xor_sync(0xffffffffu, dot, 1);
                 if (hf == 0) X->rden[s][i] = 1.f / (X->den_intra[i] + dot);
             }
-            // (4) weighted features w_j phik_j in place (bf16) and the z update
+            // (4) weighted features w_j phik_j in place (bf16) and the z update.
+            // Thread: one 16-byte chunk (8 features) of the 256-feature row
+            // (lane -> block, chunk) for the 16 tokens of its warp's group.
             {
-                const int f0 = 2 * tb;
-                const int bb = f0 >> 6, cc = (f0 & 63) >> 3, wi = f0 & 7;
-                const uint32_t base = sK(s) + bb * kBlk;
-                float z0a = 0.f, z1a = 0.f;
-#pragma unroll 8
-                for (int j = 0; j < kC; ++j) {
-                    const uint32_t ad = base + sw128_off(j, cc) + wi * 2;
-                    const float2 k = unpack_bf16x2(lds32(ad));
+                const int bb = lane >> 3, cc = lane & 7;
+                const int tg = tb >> 5;
+                const uint32_t base = sK(s) + bb * kQKBlk;
+                float za[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) za[e] = 0.f;
+#pragma unroll 4
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = tg * 16 + jj;
+                    const uint32_t ad = base + sw128_off(j, cc);
+                    uint4 v = lds128(ad);
+                    uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
                     const float wj = X->w[s][j];
-                    const uint32_t pk = pack_bf16x2(wj * k.x, wj * k.y);
-                    const float2 r = unpack_bf16x2(pk);
-                    z0a += r.x;
-                    z1a += r.y;
-                    sts32(ad, pk);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 k = unpack_bf16x2(pv[e]);
+                        pv[e] = pack_bf16x2(wj * k.x, wj * k.y);
+                        const float2 r = unpack_bf16x2(pv[e]);
+                        za[2 * e] += r.x;
+                        za[2 * e + 1] += r.y;
+                    }
+                    sts128(ad, v);
                 }
-                named_sync(1, 128);  // every reader of z in step (3) is done
+                const int f0 = bb * 64 + cc * 8;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) X->zred[tg][f0 + e] = za[e];
+                named_sync(1, 128);  // partial sums written; every reader of z in step (3) is done
                 const float gm = X->gam[s];
-                X->z[f0] = fmaf(gm, X->z[f0], z0a);
-                X->z[f0 + 1] = fmaf(gm, X->z[f0 + 1], z1a);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int f = 2 * tb + e;
+                    const float add = X->zred[0][f] + X->zred[1][f] + X->zred[2][f] + X->zred[3][f];
+                    X->z[f] = fmaf(gm, X->z[f], add);
+                }
             }
             fence_proxy_async_smem();
             named_sync(1, 128);
@@ -652,8 +707,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
         bool ok = true;
         // prologue: start state -> bf16 copy (for the first readout) and fp32 x gamma_0
+        float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, td);
         {
-            const float gam0 = fexp(chunk_log_total(a, b, h, alog, (int64_t)c_begin * kC, td, X->redd, 2));
+            const float gam0 = fexp(chunk_total(l_next, td, X->redd, 2));
+            if (nch > 1) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + 1) * kC, td);
             const float *src = nullptr;
             if (seg == 0) src = a.S0 ? a.S0 + bh * (int64_t)kF * g.dv : nullptr;
             else src = a.S_start + (bh * g.G + seg) * (int64_t)kF * g.dv;
@@ -675,12 +732,14 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_arrive(&X->sbf_ready);
         }
         for (int it = 0; ok && it + 1 < nch; ++it) {
-            const float gn = fexp(chunk_log_total(a, b, h, alog, (int64_t)(c_begin + it + 1) * kC, td, X->redd, 2));
+            const float gn = fexp(chunk_total(l_next, td, X->redd, 2));
+            if (it + 2 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 2) * kC, td);
             if (!mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+#pragma unroll 2
             for (int c0 = 0; c0 < kF; c0 += 32) {
                 uint32_t v[32], pk[16];
                 tmem_ld32(tmem + kColS + c0 + lanebase, v);
@@ -828,7 +887,7 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
     if (!tmap_tokens(&tkl, add_lo ? phk_lo : c.phk, c.B, c.L, c.H, kF, 64)) return cudaErrorInvalidValue;
 
     if (g.NPc > 0) {
-        e = cudaFuncSetAttribute(scan_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kASmem);
+        e = ensure_smem_limit(scan_state_kernel, kASmem);
         if (e != cudaSuccess) return e;
         const unsigned grid = (unsigned)(2 * g.NPc * BH);
         scan_state_kernel<<<grid, 192, kASmem, s>>>(tk, tkl, tv, g, c.dt, c.A_log, split ? 1 : 0,
@@ -850,7 +909,7 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
     oa.z0 = c.z0;
     oa.S_start = S_start;
     oa.z_start = z_start;
-    e = cudaFuncSetAttribute(scan_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCSmem);
+    e = ensure_smem_limit(scan_out_kernel, kCSmem);
     if (e != cudaSuccess) return e;
     scan_out_kernel<<<(unsigned)(2 * g.G * BH), 448, kCSmem, s>>>(tq, tk, tv, oa, err);
     count_launches(1);

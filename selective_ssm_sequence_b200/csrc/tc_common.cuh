@@ -275,6 +275,22 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
            | ((uint32_t)(M >> 4) << 24);
 }
 
+// ------------------------------------------------------------------ host: launch setup
+
+// Raise a kernel's dynamic shared-memory limit once per device (the setting
+// persists; repeating it on every call only adds host latency).
+template <typename Kern>
+cudaError_t ensure_smem_limit(Kern kern, int bytes) {
+    static int done_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && done_bytes[dev] >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done_bytes[dev] = bytes;
+    return e;
+}
+
 // ------------------------------------------------------------------ host: tensor maps
 
 // Encode a tiled bf16 tensor map (dims innermost first; strides in bytes for
