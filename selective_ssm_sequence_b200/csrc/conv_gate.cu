@@ -5,9 +5,9 @@
 //   y[b, t, c] = bias[c] + sum_{j<K} w[c, j] * x[b, t-(K-1)+j, c],  x = 0 before t = 0,
 // no activation.  Gate (sec. 2.3 / 5.2: applied after num/den):
 //   y = o * SiLU(g + b_g).
-// Each thread handles 8 adjacent channels (one 16-byte bf16 vector) of a run
-// of consecutive tokens, keeping the last K-1 inputs in registers so every
-// input element is read once.
+// Each thread handles 8 adjacent channels of a run of consecutive tokens,
+// keeping the last K-1 inputs in registers so every input element is read
+// once.  Inputs may be fp32 (projection outputs kept unrounded) or bf16.
 #include "hm_internal.h"
 
 namespace hm {
@@ -35,8 +35,18 @@ __device__ __forceinline__ bf8 pack(const float *f) {
     return v;
 }
 
-template <int K>
-__global__ void causal_conv_kernel(const __nv_bfloat16 *__restrict__ x, int64_t x_ld, int64_t L,
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *f) {
+    unpack(*reinterpret_cast<const bf8 *>(p), f);
+}
+__device__ __forceinline__ void load8(const float *p, float *f) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <int K, typename TX>
+__global__ void causal_conv_kernel(const TX *__restrict__ x, int64_t x_ld, int64_t L,
                                    int C, const float *__restrict__ w, const float *__restrict__ bias,
                                    __nv_bfloat16 *__restrict__ y, int64_t y_ld, int64_t runs) {
     const int cvec = C / 8;
@@ -61,8 +71,7 @@ __global__ void causal_conv_kernel(const __nv_bfloat16 *__restrict__ x, int64_t 
     for (int j = 0; j < K - 1; ++j) {
         int64_t s = t0 - (K - 1) + j;
         if (s >= 0) {
-            bf8 v = *reinterpret_cast<const bf8 *>(x + (b * L + s) * x_ld + c0);
-            unpack(v, hist[j]);
+            load8(x + (b * L + s) * x_ld + c0, hist[j]);
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) hist[j][i] = 0.f;
@@ -71,8 +80,7 @@ __global__ void causal_conv_kernel(const __nv_bfloat16 *__restrict__ x, int64_t 
     const int64_t t1 = (t0 + kTokRun < L) ? t0 + kTokRun : L;
     for (int64_t t = t0; t < t1; ++t) {
         float cur[8];
-        bf8 v = *reinterpret_cast<const bf8 *>(x + (b * L + t) * x_ld + c0);
-        unpack(v, cur);
+        load8(x + (b * L + t) * x_ld + c0, cur);
         float out[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -93,7 +101,8 @@ __global__ void causal_conv_kernel(const __nv_bfloat16 *__restrict__ x, int64_t 
     }
 }
 
-__global__ void gate_kernel(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ g,
+template <typename TO, typename TG>
+__global__ void gate_kernel(const TO *__restrict__ o, const TG *__restrict__ g,
                             int64_t g_ld, const float *__restrict__ b_g, int64_t rows, int E,
                             __nv_bfloat16 *__restrict__ y) {
     const int evec = E / 8;
@@ -102,8 +111,8 @@ __global__ void gate_kernel(const __nv_bfloat16 *__restrict__ o, const __nv_bflo
     const int64_t r = gid / evec;
     const int c0 = (int)(gid % evec) * 8;
     float fo[8], fg[8], out[8];
-    unpack(*reinterpret_cast<const bf8 *>(o + r * E + c0), fo);
-    unpack(*reinterpret_cast<const bf8 *>(g + r * g_ld + c0), fg);
+    load8(o + r * E + c0, fo);
+    load8(g + r * g_ld + c0, fg);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         float gg = fg[i] + (b_g ? b_g[c0 + i] : 0.f);
@@ -114,19 +123,23 @@ __global__ void gate_kernel(const __nv_bfloat16 *__restrict__ o, const __nv_bflo
 
 }  // namespace
 
-cudaError_t launch_causal_conv(const void *x, int64_t x_ld, int64_t B, int64_t L, int C, int K,
-                               const float *w, const float *bias, void *y, int64_t y_ld,
+cudaError_t launch_causal_conv(const void *x, bool x_f32, int64_t x_ld, int64_t B, int64_t L, int C,
+                               int K, const float *w, const float *bias, void *y, int64_t y_ld,
                                cudaStream_t s) {
     if (B * L == 0) return cudaSuccess;
     const int64_t runs = B * ((L + kTokRun - 1) / kTokRun);
     const int64_t threads = runs * (C / 8);
     const unsigned blocks = (unsigned)((threads + 255) / 256);
-    auto xb = (const __nv_bfloat16 *)x;
     auto yb = (__nv_bfloat16 *)y;
     switch (K) {
-#define HM_CONV_CASE(KK)                                                                        \
-    case KK:                                                                                    \
-        causal_conv_kernel<KK><<<blocks, 256, 0, s>>>(xb, x_ld, L, C, w, bias, yb, y_ld, runs); \
+#define HM_CONV_CASE(KK)                                                                           \
+    case KK:                                                                                       \
+        if (x_f32)                                                                                 \
+            causal_conv_kernel<KK, float><<<blocks, 256, 0, s>>>((const float *)x, x_ld, L, C, w,  \
+                                                                 bias, yb, y_ld, runs);            \
+        else                                                                                       \
+            causal_conv_kernel<KK, __nv_bfloat16><<<blocks, 256, 0, s>>>(                          \
+                (const __nv_bfloat16 *)x, x_ld, L, C, w, bias, yb, y_ld, runs);                    \
         break;
         HM_CONV_CASE(1)
         HM_CONV_CASE(2)
@@ -144,12 +157,23 @@ cudaError_t launch_causal_conv(const void *x, int64_t x_ld, int64_t B, int64_t L
     return cudaGetLastError();
 }
 
-cudaError_t launch_gate(const void *o, const void *g, int64_t g_ld, const float *b_g, int64_t rows,
-                        int E, void *y, cudaStream_t s) {
+cudaError_t launch_gate(const void *o, bool o_f32, const void *g, bool g_f32, int64_t g_ld,
+                        const float *b_g, int64_t rows, int E, void *y, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     const int64_t threads = rows * (E / 8);
-    gate_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
-        (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)g, g_ld, b_g, rows, E, (__nv_bfloat16 *)y);
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    auto yb = (__nv_bfloat16 *)y;
+    if (o_f32 && g_f32)
+        gate_kernel<float, float><<<blocks, 256, 0, s>>>((const float *)o, (const float *)g, g_ld, b_g, rows, E, yb);
+    else if (o_f32)
+        gate_kernel<float, __nv_bfloat16><<<blocks, 256, 0, s>>>((const float *)o, (const __nv_bfloat16 *)g, g_ld,
+                                                                  b_g, rows, E, yb);
+    else if (g_f32)
+        gate_kernel<__nv_bfloat16, float><<<blocks, 256, 0, s>>>((const __nv_bfloat16 *)o, (const float *)g, g_ld,
+                                                                  b_g, rows, E, yb);
+    else
+        gate_kernel<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, s>>>(
+            (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)g, g_ld, b_g, rows, E, yb);
     count_launches(1);
     return cudaGetLastError();
 }

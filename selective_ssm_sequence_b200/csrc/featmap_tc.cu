@@ -81,7 +81,7 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
         mbar_init(&bars->wbar, 1);
         for (int b = 0; b < NA; ++b) {
             mbar_init(&bars->accf[b], 1);
-            mbar_init(&bars->acce[b], 128);
+            mbar_init(&bars->acce[b], 4);   // one arrival per epilogue warp
         }
         bars->abort = 0;
         mbar_fence_init();
@@ -198,7 +198,8 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                 tmem_wait_ld();
                 if (c + 32 >= P) {
                     tc_fence_before();
-                    mbar_arrive(&bars->acce[b]);   // last read of this accumulator
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->acce[b]);   // last read of this accumulator
                 }
                 if (!valid) continue;
 #pragma unroll

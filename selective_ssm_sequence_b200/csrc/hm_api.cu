@@ -175,7 +175,7 @@ hm_status check_decode(const hm_decode_args *a, DecodePlan *plan) {
 // ------------------------------------------------------------------ mixer
 
 struct MixerPlan {
-    size_t off_g, off_qkv_raw, off_dt, off_q, off_k, off_v, off_o, off_scan;
+    size_t off_g, off_qkv_raw, off_dt, off_q, off_k, off_v, off_o, off_scan;   // byte offsets
     size_t scan_bytes;
     size_t total;
     hm_scan_args scan;
@@ -203,13 +203,15 @@ hm_status check_mixer(const hm_mixer_args *a, MixerPlan *plan) {
     const size_t E = (size_t)a->E;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 256); return o; };
-    pl.off_g = take((size_t)M * E * 2);
-    pl.off_qkv_raw = take((size_t)M * E * 2);
+    // fp32: projection output (q, k, v in turn), gate pre-activation, scan output
+    pl.off_qkv_raw = take((size_t)M * E * 4);
+    pl.off_g = take((size_t)M * E * 4);
+    pl.off_o = take((size_t)M * E * 4);
     pl.off_dt = take((size_t)M * a->H * 4);
+    // bf16: conv outputs (the scan's q, k, v); q's buffer is reused for the gated y
     pl.off_q = take((size_t)M * E * 2);
     pl.off_k = take((size_t)M * E * 2);
     pl.off_v = take((size_t)M * E * 2);
-    pl.off_o = take((size_t)M * E * 2);
     hm_scan_args s{};
     s.B = a->B; s.L = a->L; s.H = a->H; s.d = a->E / a->H; s.p = a->p; s.dv = a->E / a->H;
     s.io_dtype = HM_BF16;
@@ -302,8 +304,13 @@ size_t hm_scan_workspace_size(const hm_scan_args *a) {
     return pl.total;
 }
 
-hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stream) {
-    g_detail[0] = 0;
+}  // extern "C"
+
+namespace hm {
+namespace {
+
+// The prefill; with o_f32 (tensor-core path only) o is written as fp32.
+hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
     ScanPlan pl;
     hm_status st = check_scan(a, &pl);
     if (st != HM_OK) return st;
@@ -336,6 +343,7 @@ hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stream) {
     c.phq = phq; c.phk = phk; c.phk_lo = phk_lo; c.v = a->v;
     c.dt = a->dt; c.A_log = a->A_log; c.S0 = a->S0; c.z0 = a->z0;
     c.o = a->o; c.S_out = a->S_out; c.z_out = a->z_out;
+    c.o_f32 = o_f32 && pl.tc;
     if (pl.tc)
         e = launch_scan_tc(c, ws + 2 * pl.phi_bytes + pl.lo_bytes, pl.tc_bytes,
                            DevErr{device_error_word()}, s);
@@ -343,6 +351,23 @@ hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stream) {
         e = launch_scan_simt(c, s);
     return e == cudaSuccess ? HM_OK : cuda_fail(e, "scan launch");
 }
+
+bool scan_uses_tc(const hm_scan_args *a) {
+    ScanPlan pl;
+    return check_scan(a, &pl) == HM_OK && pl.tc;
+}
+
+}  // namespace
+}  // namespace hm
+
+using namespace hm;
+
+extern "C" hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stream) {
+    g_detail[0] = 0;
+    return scan_impl(a, false, stream);
+}
+
+extern "C" {
 
 size_t hm_decode_workspace_size(const hm_decode_args *a) {
     DecodePlan pl;
@@ -407,21 +432,25 @@ hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t ws_bytes,
     char *ws = (char *)workspace;
     const int E = a->E, D = a->d_model, H = a->H;
     DevErr err{device_error_word()};
-    void *g = ws + pl.off_g, *raw = ws + pl.off_qkv_raw, *qc = ws + pl.off_q, *kc = ws + pl.off_k,
-         *vc = ws + pl.off_v, *o = ws + pl.off_o;
+    // Intermediates stay in fp32 where the next step can take fp32 (projection
+    // outputs into the conv, the gate pre-activation, the scan output into the
+    // gate): each bf16 rounding of an intermediate adds ~2^-9 relative error.
+    float *raw = (float *)(ws + pl.off_qkv_raw), *g = (float *)(ws + pl.off_g);
+    void *o = ws + pl.off_o;
+    void *qc = ws + pl.off_q, *kc = ws + pl.off_k, *vc = ws + pl.off_v;
     float *dt = (float *)(ws + pl.off_dt);
     cudaError_t e;
-    // q, k, v: projection into `raw`, then conv into their own buffers
+    // q, k, v: projection (fp32) into `raw`, then the causal conv into bf16 buffers
     const void *Wp[3] = {a->W_q, a->W_k, a->W_v};
     void *dst[3] = {qc, kc, vc};
     for (int i = 0; i < 3; ++i) {
-        e = launch_gemm_tc(a->x, Wp[i], M, E, D, raw, E, EPI_STORE_BF16, nullptr, err, s);
+        e = launch_gemm_tc(a->x, Wp[i], M, E, D, raw, E, EPI_STORE_F32, nullptr, err, s);
         if (e != cudaSuccess) return cuda_fail(e, "mixer: projection GEMM");
-        e = launch_causal_conv(raw, E, a->B, a->L, E, a->conv_k, a->conv_w + (size_t)i * E * a->conv_k,
+        e = launch_causal_conv(raw, true, E, a->B, a->L, E, a->conv_k, a->conv_w + (size_t)i * E * a->conv_k,
                                a->conv_b ? a->conv_b + (size_t)i * E : nullptr, dst[i], E, s);
         if (e != cudaSuccess) return cuda_fail(e, "mixer: causal conv");
     }
-    e = launch_gemm_tc(a->x, a->W_g, M, E, D, g, E, EPI_STORE_BF16, nullptr, err, s);
+    e = launch_gemm_tc(a->x, a->W_g, M, E, D, g, E, EPI_STORE_F32, a->b_g, err, s);
     if (e != cudaSuccess) return cuda_fail(e, "mixer: gate GEMM");
     {
         const unsigned blocks = (unsigned)((M * 32 + 255) / 256);
@@ -440,12 +469,14 @@ hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t ws_bytes,
     sa.o = o;
     sa.workspace = ws + pl.off_scan;
     sa.workspace_bytes = pl.scan_bytes;
-    st = hm_scan_chunked_fwd(&sa, stream);
+    const bool o_f32 = scan_uses_tc(&sa);
+    st = scan_impl(&sa, o_f32, stream);
     if (st != HM_OK) return st;
-    // y = o * SiLU(g + b_g) (into the raw buffer), out = y W_o^T
-    e = launch_gate(o, g, E, a->b_g, M, E, raw, s);
+    // y = o * SiLU(g) (gate bias already added by the GEMM epilogue), bf16 into
+    // q's buffer; out = y W_o^T
+    e = launch_gate(o, o_f32, g, true, E, nullptr, M, E, qc, s);
     if (e != cudaSuccess) return cuda_fail(e, "mixer: gate");
-    e = launch_gemm_tc(raw, a->W_o, M, D, E, a->out, D, EPI_STORE_BF16, nullptr, err, s);
+    e = launch_gemm_tc(qc, a->W_o, M, D, E, a->out, D, EPI_STORE_BF16, nullptr, err, s);
     if (e != cudaSuccess) return cuda_fail(e, "mixer: out projection");
     return HM_OK;
 }

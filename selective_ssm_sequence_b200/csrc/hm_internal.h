@@ -98,6 +98,7 @@ struct ScanCore {
     const float *dt, *A_log;
     const float *S0, *z0;
     void *o;
+    bool o_f32;           // tensor-core path: write o as fp32 instead of io_dtype
     float *S_out, *z_out;
 };
 cudaError_t launch_scan_simt(const ScanCore &c, cudaStream_t s);
@@ -130,13 +131,13 @@ cudaError_t launch_gemm_tc(const void *A, const void *Bm, int64_t M, int64_t N, 
                            void *C, int64_t ldc, GemmEpi epi, const float *bias, DevErr err,
                            cudaStream_t s);
 
-// Depthwise causal conv over [B, L, C] bf16 with fp32 weights [C, K]; bf16 out.
-cudaError_t launch_causal_conv(const void *x, int64_t x_ld, int64_t B, int64_t L, int C, int K,
-                               const float *w, const float *bias, void *y, int64_t y_ld,
+// Depthwise causal conv over [B, L, C] (fp32 or bf16 in) with fp32 weights [C, K]; bf16 out.
+cudaError_t launch_causal_conv(const void *x, bool x_f32, int64_t x_ld, int64_t B, int64_t L, int C,
+                               int K, const float *w, const float *bias, void *y, int64_t y_ld,
                                cudaStream_t s);
 
-// y[r, c] = o[r, c] * SiLU(g[r, c] + b_g[c]) (bf16 in/out).
-cudaError_t launch_gate(const void *o, const void *g, int64_t g_ld, const float *b_g, int64_t rows,
-                        int E, void *y, cudaStream_t s);
+// y[r, c] = o[r, c] * SiLU(g[r, c] + b_g[c]) (o, g fp32 or bf16; y bf16).
+cudaError_t launch_gate(const void *o, bool o_f32, const void *g, bool g_f32, int64_t g_ld,
+                        const float *b_g, int64_t rows, int E, void *y, cudaStream_t s);
 
 }  // namespace hm

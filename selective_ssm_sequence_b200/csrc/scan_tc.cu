@@ -382,14 +382,15 @@ struct CAux {
 // phiK phiK^T, which is not used).
 constexpr int kQKBlk = 2 * kBlk;                       // [Q | K] of one feature block
 constexpr int kCStage = 4 * kQKBlk + kTileV;           // Q, K, V of one chunk
-constexpr int kCOffP = 2 * kCStage;
-constexpr int kCOffAux = kCOffP + kC * 128;
+constexpr int kCOffP = 2 * kCStage;               // Pt as bf16 hi (8 KB) then lo (8 KB)
+constexpr int kCOffAux = kCOffP + 2 * kC * 128;
 constexpr int kCSmem = kCOffAux + (int)sizeof(CAux) + 1024;
 
 struct OutArgs {
     Geo g;
     const float *dt, *A_log;
-    __nv_bfloat16 *o;
+    void *o;
+    int o_f32;                       // o stored as fp32 (else bf16)
     const float *S0, *z0;            // segment 0 start state (caller layout) or null
     const float *S_start, *z_start;  // segments >= 1: [BH][G][F*dv], [BH][G][F]
 };
@@ -445,12 +446,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_init(&X->den_ready[s], 1);
         }
         mbar_init(&X->p_full, 1);
-        mbar_init(&X->p_empty, 128);
+        mbar_init(&X->p_empty, 4);      // one arrival per warp of the group
         mbar_init(&X->epib_done, 1);
         mbar_init(&X->o_full, 1);
-        mbar_init(&X->o_empty, 128);
+        mbar_init(&X->o_empty, 4);
         mbar_init(&X->s_full, 1);
-        mbar_init(&X->sbf_ready, 128);
+        mbar_init(&X->sbf_ready, 4);
         X->abort = 0;
         mbar_fence_init();
     }
@@ -517,9 +518,11 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                            k > 0 ? 1u : 0u);
                 }
 #pragma unroll
-                for (int k = 0; k < kC / 16; ++k)
-                    mma_ss(tmem + kColO, desc_mn_sw128(sV(s) + k * 2048, kBlk, 1024),
-                           desc_k_sw128(sP + k * 32), idOa, 1u);
+                for (int k = 0; k < kC / 16; ++k) {
+                    const uint64_t va = desc_mn_sw128(sV(s) + k * 2048, kBlk, 1024);
+                    mma_ss(tmem + kColO, va, desc_k_sw128(sP + k * 32), idOa, 1u);
+                    mma_ss(tmem + kColO, va, desc_k_sw128(sP + kC * 128 + k * 32), idOa, 1u);
+                }
                 mma_commit(&X->o_full);
 #pragma unroll
                 for (int k = 0; k < kC / 16; ++k)
@@ -568,40 +571,79 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (tb == 0) X->gam[s] = fexp(total);
                 named_sync(1, 128);
             }
-            // (2) scores: Pt = P * exp(cum_i - cum_j) on j <= i, row sums; Pt -> smem (bf16)
+            // (2) once P is in TMEM (MMA1 done, so phiK is free): warps 4, 5 (the
+            // owners of TMEM lanes 0..63) form the decayed scores Pt while warps
+            // 2, 3 rebuild the weighted features w_j phik_j in place.
             if (!mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7)) break;
             if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8)) break;
             tc_fence_after();
-            {
-                uint32_t pr[64];
+            if (q < 2) {
+                // Pt = P * exp(cum_i - cum_j) on j <= i, row sums; Pt -> smem as bf16
+                // hi + lo (the PV product runs twice: a few-token weighted average
+                // would otherwise carry the 2^-9 rounding of each weight)
                 const uint32_t ta = tmem + kColP + ((uint32_t)(32 * q) << 16);
-                tmem_ld32(ta, pr);
-                tmem_ld32(ta + 32, pr + 32);
-                tmem_wait_ld();
-                if (q < 2) {  // lanes 0..63 hold the 64 rows of P
-                    const int i = 32 * q + lane;
-                    const float ci = X->cum[s][i];
-                    float rs = 0.f;
+                const int i = 32 * q + lane;
+                const float ci = X->cum[s][i];
+                float rs = 0.f;
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        uint32_t pk[4];
+                for (int hcol = 0; hcol < 2; ++hcol) {
+                    uint32_t pr[32];
+                    tmem_ld32(ta + 32 * hcol, pr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int cc = 4 * hcol + c4;
+                        uint32_t pk[4], pl[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int j = cc * 8 + 2 * e;
-                            const float e0 = (j <= i) ? __uint_as_float(pr[j]) * fexp(ci - X->cum[s][j]) : 0.f;
-                            const float e1 = (j + 1 <= i) ? __uint_as_float(pr[j + 1]) * fexp(ci - X->cum[s][j + 1]) : 0.f;
+                            const int jl = c4 * 8 + 2 * e;      // column within this half
+                            const int j = 32 * hcol + jl;
+                            const float e0 = (j <= i) ? __uint_as_float(pr[jl]) * fexp(ci - X->cum[s][j]) : 0.f;
+                            const float e1 = (j + 1 <= i) ? __uint_as_float(pr[jl + 1]) * fexp(ci - X->cum[s][j + 1]) : 0.f;
                             pk[e] = pack_bf16x2(e0, e1);
                             const float2 r = unpack_bf16x2(pk[e]);
-                            rs += r.x + r.y;
+                            pl[e] = pack_bf16x2(e0 - r.x, e1 - r.y);
+                            rs += e0 + e1;
                         }
                         sts128(sP + sw128_off(i, cc), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                        sts128(sP + kC * 128 + sw128_off(i, cc), make_uint4(pl[0], pl[1], pl[2], pl[3]));
                     }
-                    X->den_intra[i] = rs;
                 }
+                X->den_intra[i] = rs;
+                tc_fence_before();
+            } else {
+                // weighted features in place (bf16): thread = one 16-byte chunk
+                // (8 features) of the row for the 32 tokens of its warp
+                const int bb = lane >> 3, cc = lane & 7;
+                const int tg = q - 2;
+                const uint32_t base = sK(s) + bb * kQKBlk;
+                float za[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) za[e] = 0.f;
+#pragma unroll 4
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = tg * 32 + jj;
+                    const uint32_t ad = base + sw128_off(j, cc);
+                    uint4 v = lds128(ad);
+                    uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
+                    const float wj = X->w[s][j];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 k = unpack_bf16x2(pv[e]);
+                        pv[e] = pack_bf16x2(wj * k.x, wj * k.y);
+                        const float2 r = unpack_bf16x2(pv[e]);
+                        za[2 * e] += r.x;
+                        za[2 * e + 1] += r.y;
+                    }
+                    sts128(ad, v);
+                }
+                const int f0 = bb * 64 + cc * 8;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) X->zred[tg][f0 + e] = za[e];
             }
-            tc_fence_before();
-            mbar_arrive(&X->p_empty);
-            named_sync(1, 128);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->p_empty);
+            named_sync(1, 128);   // den_intra and the z partial sums are complete
             // (3) phiQ rows scaled by exp(cum_i) in place; den = rowsum + e^cum phiq . z
             {
                 const int i = tb >> 1, hf = tb & 1;
@@ -630,43 +672,14 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 dot += __shfl_xor_sync(0xffffffffu, dot, 1);
                 if (hf == 0) X->rden[s][i] = 1.f / (X->den_intra[i] + dot);
             }
-            // (4) weighted features w_j phik_j in place (bf16) and the z update.
-            // Thread: one 16-byte chunk (8 features) of the 256-feature row
-            // (lane -> block, chunk) for the 16 tokens of its warp's group.
+            named_sync(1, 128);   // every reader of z in step (3) is done
+            // (4) z <- gamma z + sum_j w_j phik_j
             {
-                const int bb = lane >> 3, cc = lane & 7;
-                const int tg = tb >> 5;
-                const uint32_t base = sK(s) + bb * kQKBlk;
-                float za[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) za[e] = 0.f;
-#pragma unroll 4
-                for (int jj = 0; jj < 16; ++jj) {
-                    const int j = tg * 16 + jj;
-                    const uint32_t ad = base + sw128_off(j, cc);
-                    uint4 v = lds128(ad);
-                    uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
-                    const float wj = X->w[s][j];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 k = unpack_bf16x2(pv[e]);
-                        pv[e] = pack_bf16x2(wj * k.x, wj * k.y);
-                        const float2 r = unpack_bf16x2(pv[e]);
-                        za[2 * e] += r.x;
-                        za[2 * e + 1] += r.y;
-                    }
-                    sts128(ad, v);
-                }
-                const int f0 = bb * 64 + cc * 8;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) X->zred[tg][f0 + e] = za[e];
-                named_sync(1, 128);  // partial sums written; every reader of z in step (3) is done
                 const float gm = X->gam[s];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int f = 2 * tb + e;
-                    const float add = X->zred[0][f] + X->zred[1][f] + X->zred[2][f] + X->zred[3][f];
-                    X->z[f] = fmaf(gm, X->z[f], add);
+                    X->z[f] = fmaf(gm, X->z[f], X->zred[0][f] + X->zred[1][f]);
                 }
             }
             fence_proxy_async_smem();
@@ -691,13 +704,22 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             tmem_ld32(ta + 32, r + 32);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&X->o_empty);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->o_empty);
             const int64_t t0 = (int64_t)(c_begin + it) * kC;
-            __nv_bfloat16 *op = a.o + ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
+            const int64_t obase = ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
             const int64_t tstride = (int64_t)g.H * g.dv;
+            if (a.o_f32) {
+                float *op = (float *)a.o + obase;
 #pragma unroll
-            for (int i = 0; i < kC; ++i)
-                if (t0 + i < g.L) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]) * X->rden[s][i]);
+                for (int i = 0; i < kC; ++i)
+                    if (t0 + i < g.L) op[i * tstride] = __uint_as_float(r[i]) * X->rden[s][i];
+            } else {
+                __nv_bfloat16 *op = (__nv_bfloat16 *)a.o + obase;
+#pragma unroll
+                for (int i = 0; i < kC; ++i)
+                    if (t0 + i < g.L) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]) * X->rden[s][i]);
+            }
         }
     } else {
         // ------------------------------------------------------------ WG-D: state pass
@@ -729,7 +751,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&X->sbf_ready);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
         for (int it = 0; ok && it + 1 < nch; ++it) {
             const float gn = fexp(chunk_total(l_next, td, X->redd, 2));
@@ -754,7 +777,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&X->sbf_ready);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
         // the MMAs of the last chunk must be complete before TMEM is released
         if (ok && nch > 0) mbar_wait(&X->s_full, (nch - 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 12);
@@ -904,7 +928,8 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
     oa.g = g;
     oa.dt = c.dt;
     oa.A_log = c.A_log;
-    oa.o = (__nv_bfloat16 *)c.o;
+    oa.o = c.o;
+    oa.o_f32 = c.o_f32 ? 1 : 0;
     oa.S0 = c.S0;
     oa.z0 = c.z0;
     oa.S_start = S_start;
