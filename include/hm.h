@@ -215,6 +215,24 @@ HM_API size_t hm_mixer_workspace_size(const hm_mixer_args *a);
 HM_API hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t workspace_bytes,
                        hm_stream_t stream);
 
+/*
+ * hm_step_decode_noalloc -- hm_step_decode for callers that cannot allocate
+ * device memory (for example a plugin whose host application owns all device
+ * memory and offers no allocator, or a serving loop that must not allocate
+ * after start-up).  There is no counterpart in the paper; it is a deployment
+ * convenience.  Same arguments and results as hm_step_decode, except that
+ * workspace / workspace_bytes are ignored: the feature vectors live in a fixed
+ * device array inside the library (two planes of 524,288 fp32 values, 4 MiB,
+ * held by every GPU that loads the library until the process exits).
+ * Limit: when W_q != NULL, B * H * F must not exceed 524,288; larger calls
+ * return HM_ERR_INVALID_ARG before anything is enqueued (use hm_step_decode).
+ * All calls share that array, so calls whose kernels may overlap on a GPU
+ * (several streams or host threads on one device) race and must be serialised
+ * by the caller.  The first call on each device looks up the array's device
+ * address; make that first call before any stream capture.
+ */
+HM_API hm_status hm_step_decode_noalloc(const hm_decode_args *a, hm_stream_t stream);
+
 /* Number of kernels this library has enqueued in this process so far (all
  * devices, all threads).  A diagnostic for launch accounting. */
 HM_API uint64_t hm_launch_count(void);

@@ -70,6 +70,8 @@ lib.hm_decode_workspace_size.restype = _SZ
 lib.hm_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]
 lib.hm_step_decode.restype = _I
 lib.hm_step_decode.argtypes = [ctypes.POINTER(DecodeArgs), _P]
+lib.hm_step_decode_noalloc.restype = _I
+lib.hm_step_decode_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _P]
 lib.hm_mixer_workspace_size.restype = _SZ
 lib.hm_mixer_workspace_size.argtypes = [ctypes.POINTER(MixerArgs)]
 lib.hm_mixer_fwd.restype = _I
@@ -82,7 +84,7 @@ lib.hm_get_device_error.argtypes = [_P]
 EXPORTED = ("hm_status_string", "hm_last_error_detail", "hm_version", "hm_featmap",
             "hm_scan_workspace_size", "hm_scan_chunked_fwd", "hm_decode_workspace_size",
             "hm_step_decode", "hm_mixer_workspace_size", "hm_mixer_fwd", "hm_get_device_error",
-            "hm_launch_count")
+            "hm_launch_count", "hm_step_decode_noalloc")
 
 
 class HMError(RuntimeError):
@@ -210,6 +212,14 @@ def hm_decode_workspace_size(args: DecodeArgs) -> int:
 
 def hm_step_decode(args: DecodeArgs, stream=None) -> None:
     _check(lib.hm_step_decode(ctypes.byref(args), _stream(stream)), "hm_step_decode")
+
+
+def hm_step_decode_noalloc(args: DecodeArgs, stream=None) -> None:
+    """hm_step_decode without a caller-provided workspace: for callers that
+    cannot allocate device memory.  The feature vectors use a fixed 4 MiB
+    device array inside the library (B * H * F <= 524288 when W_q is given);
+    calls that overlap on the GPU share that array and must be serialised."""
+    _check(lib.hm_step_decode_noalloc(ctypes.byref(args), _stream(stream)), "hm_step_decode_noalloc")
 
 
 def mixer_args(x, out, W_q, W_k, W_v, W_g, W_dt, conv_w, W_hq, W_hk, A_log, W_o, n_heads: int,

@@ -44,6 +44,12 @@ hm_status fail(hm_status s, const char *fmt, ...) {
     return s;
 }
 
+}  // namespace
+
+void set_error_detail(const char *msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg ? msg : ""); }
+
+namespace {
+
 hm_status cuda_fail(cudaError_t e, const char *what) {
     return fail(HM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }

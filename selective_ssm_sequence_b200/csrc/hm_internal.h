@@ -34,6 +34,9 @@ unsigned int *device_error_word();  // address of this device's error word (host
 // Host-side count of kernels enqueued by the library (hm_launch_count).
 void count_launches(unsigned int n);
 
+// Sets the text hm_last_error_detail() returns on this host thread.
+void set_error_detail(const char *msg);
+
 // ---------------------------------------------------------------- device helpers
 
 __device__ __forceinline__ float hm_ld(const float *p, int64_t i) { return p[i]; }
