@@ -136,13 +136,24 @@ def to_dev(a, dtype, torch):
     return t.to(torch.bfloat16) if dtype == "bf16" else t
 
 
-def max_over_ranks(x: float, world: int, torch) -> float:
+def max_over_ranks(x: float, world: int, torch, device: str = "cuda") -> float:
+    """The slowest rank's time (all ranks take part; NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank generates its own batch (weak scaling, no data exchange)."""
+    return base_seed + 1000 * rank
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 def barrier(world: int):
@@ -195,7 +206,7 @@ def bench_prefill(cfg, args, rank, world, torch):
     import selective_ssm_sequence_b200 as hm
 
     peaks, peak_kind = load_peaks()
-    seed = cfg.seed + 1000 * rank
+    seed = rank_seed(cfg.seed, rank)
     inp = wl.scan_inputs(cfg, seed=seed)
     B, L, H, d, p, dv = cfg.B, cfg.L, cfg.H, cfg.d, cfg.p, cfg.dv
     F = 2 * p
@@ -274,8 +285,7 @@ def bench_prefill(cfg, args, rank, world, torch):
 
     th = B * L * H
     fl_fm, fl_sc, _ = algorithmic_per_token_head(F, d, p, dv)
-    tokens_total = B * L * world
-    value = tokens_total / (ms_step * 1e-3)
+    value = whole_job_rate(B * L, world, ms_step)
 
     # dominant call and its roofline
     bw = peaks["hbm_gbs"]

@@ -62,7 +62,7 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
     using Lay = FmLayout<D, P>;
     constexpr int NA = Lay::kAcc;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     uint8_t *sW = smem + Lay::kOffW;
     uint8_t *sX = smem + Lay::kOffX;
     FmBars *bars = (FmBars *)(smem + Lay::kOffBar);

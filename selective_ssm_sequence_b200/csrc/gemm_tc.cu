@@ -36,7 +36,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ 
                int64_t M, int64_t N, int64_t K, void *__restrict__ C, int64_t ldc,
                const float *__restrict__ bias, DevErr err) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     GAux *X = (GAux *)(smem + kStages * kStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t tiles_m = (M + kBM - 1) / kBM, tiles_n = (N + kBN - 1) / kBN;

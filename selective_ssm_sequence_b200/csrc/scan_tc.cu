@@ -52,26 +52,6 @@ constexpr int kTileV = 2 * kBlk;   // [64 x 128] bf16 tile = 16 KB
 
 __device__ __forceinline__ float fexp(float x) { return exp2f(x * 1.4426950408889634f); }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
-    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
 struct Geo {
     int64_t B, L;
     int H, dv;
@@ -87,7 +67,7 @@ struct Geo {
 
 struct AAux {
     float w[2][kC];
-    float zred[4][kF];
+    alignas(16) float zred[4][kF];
     float red[4];
     float suf;         // sum of log a over the chunks already processed (later ones)
     uint64_t full[2], empty[2], built, done;
@@ -107,7 +87,7 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
                   const float *__restrict__ A_log, int split, int add_lo, float *__restrict__ S_part,
                   float *__restrict__ z_part, float *__restrict__ lsum_part, DevErr err) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     AAux *X = (AAux *)(smem + kAOffAux);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int half = blockIdx.x & 1;
@@ -229,40 +209,51 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
                 break;
             }
             // weighted features, split into bf16 hi + lo, written back in place
-            const uint32_t kh = smem_u32(stage(s)) + bb * kBlk;
-            const uint32_t kl = kh + kTileF;
-#pragma unroll 4
-            for (int jj = 0; jj < 16; ++jj) {
-                const int j = tg * 16 + jj;
-                const uint32_t off = sw128_off(j, cc);
-                uint4 vh = lds128(kh + off);
-                uint4 vl = make_uint4(0, 0, 0, 0);
-                if (add_lo) vl = lds128(kl + off);
-                uint32_t *ph = reinterpret_cast<uint32_t *>(&vh);
-                uint32_t *pl = reinterpret_cast<uint32_t *>(&vl);
-                const float wj = X->w[s][j];
+            // (8 rows loaded at a time)
+            uint8_t *__restrict__ kh = stage(s) + bb * kBlk;
+            uint8_t *__restrict__ kl = kh + kTileF;
+            const float *__restrict__ wv = X->w[s];
+#pragma unroll 1
+            for (int j0 = tg * 16; j0 < tg * 16 + 16; j0 += 8) {
+                uint4 vh[8], vl[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float2 k = unpack_bf16x2(ph[e]);
-                    if (add_lo) {
-                        const float2 k2 = unpack_bf16x2(pl[e]);
-                        k.x += k2.x;
-                        k.y += k2.y;
-                    }
-                    const float kt0 = wj * k.x, kt1 = wj * k.y;
-                    ph[e] = pack_bf16x2(kt0, kt1);
-                    const float2 hf = unpack_bf16x2(ph[e]);
-                    if (split) {
-                        pl[e] = pack_bf16x2(kt0 - hf.x, kt1 - hf.y);
-                        za[2 * e] += kt0;
-                        za[2 * e + 1] += kt1;
-                    } else {
-                        za[2 * e] += hf.x;
-                        za[2 * e + 1] += hf.y;
+                for (int jj = 0; jj < 8; ++jj) {
+                    const uint32_t off = sw128_off(j0 + jj, cc);
+                    vh[jj] = *reinterpret_cast<const uint4 *>(kh + off);
+                    vl[jj] = add_lo ? *reinterpret_cast<const uint4 *>(kl + off) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    uint32_t *ph = reinterpret_cast<uint32_t *>(&vh[jj]);
+                    uint32_t *pl = reinterpret_cast<uint32_t *>(&vl[jj]);
+                    const float wj = wv[j0 + jj];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float2 k = unpack_bf16x2(ph[e]);
+                        if (add_lo) {
+                            const float2 k2 = unpack_bf16x2(pl[e]);
+                            k.x += k2.x;
+                            k.y += k2.y;
+                        }
+                        const float kt0 = wj * k.x, kt1 = wj * k.y;
+                        ph[e] = pack_bf16x2(kt0, kt1);
+                        const float2 hf = unpack_bf16x2(ph[e]);
+                        if (split) {
+                            pl[e] = pack_bf16x2(kt0 - hf.x, kt1 - hf.y);
+                            za[2 * e] += kt0;
+                            za[2 * e + 1] += kt1;
+                        } else {
+                            za[2 * e] += hf.x;
+                            za[2 * e + 1] += hf.y;
+                        }
                     }
                 }
-                sts128(kh + off, vh);
-                if (split) sts128(kl + off, vl);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const uint32_t off = sw128_off(j0 + jj, cc);
+                    *reinterpret_cast<uint4 *>(kh + off) = vh[jj];
+                    if (split) *reinterpret_cast<uint4 *>(kl + off) = vl[jj];
+                }
             }
             fence_proxy_async_smem();
             named_sync(1, 128);
@@ -270,8 +261,8 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
         }
         // z of the part: reduce the four token groups' partial sums
         const int f0 = bb * 64 + cc * 8;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) X->zred[tg][f0 + e] = za[e];
+        *reinterpret_cast<float4 *>(&X->zred[tg][f0]) = make_float4(za[0], za[1], za[2], za[3]);
+        *reinterpret_cast<float4 *>(&X->zred[tg][f0 + 4]) = make_float4(za[4], za[5], za[6], za[7]);
         named_sync(1, 128);
         if (ok && mbar_wait(&X->done, 0, abort_flag, err, KID_SCAN_TC_STATE, 5)) {
             tc_fence_after();
@@ -364,7 +355,7 @@ struct CAux {
     float rden[2][kC];   // 1 / den
     float den_intra[kC];
     float z[kF];
-    float zred[4][kF];   // per token-group partial sums of the weighted features
+    alignas(16) float zred[4][kF];   // per token-group partial sums of the weighted features
     float gam[2];
     float redb[4];
     float redd[4];
@@ -382,8 +373,9 @@ struct CAux {
 // phiK phiK^T, which is not used).
 constexpr int kQKBlk = 2 * kBlk;                       // [Q | K] of one feature block
 constexpr int kCStage = 4 * kQKBlk + kTileV;           // Q, K, V of one chunk
-constexpr int kCOffP = 2 * kCStage;               // Pt as bf16 hi (8 KB) then lo (8 KB)
-constexpr int kCOffAux = kCOffP + 2 * kC * 128;
+constexpr int kCPBytes = 2 * kC * 128;             // Pt as bf16 hi (8 KB) then lo (8 KB)
+constexpr int kCOffP = 2 * kCStage;               // one Pt buffer per stage
+constexpr int kCOffAux = kCOffP + 2 * kCPBytes;
 constexpr int kCSmem = kCOffAux + (int)sizeof(CAux) + 1024;
 
 struct OutArgs {
@@ -417,7 +409,7 @@ __global__ void __launch_bounds__(448, 1)
 scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, OutArgs a, DevErr err) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     CAux *X = (CAux *)(smem + kCOffAux);
     const Geo &g = a.g;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -437,7 +429,11 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     auto sQ = [&](int s) { return sbase + s * kCStage; };
     auto sK = [&](int s) { return sbase + s * kCStage + kBlk; };
     auto sV = [&](int s) { return sbase + s * kCStage + 4 * kQKBlk; };
-    const uint32_t sP = sbase + kCOffP;
+    auto sP = [&](int s) { return sbase + kCOffP + s * kCPBytes; };
+    // generic pointers to the same buffers, for CUDA-core accesses
+    auto gQ = [&](int s) { return smem + s * kCStage; };
+    auto gK = [&](int s) { return smem + s * kCStage + kBlk; };
+    auto gP = [&](int s) { return smem + kCOffP + s * kCPBytes; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -494,22 +490,32 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             constexpr uint32_t idOi = idesc_bf16(128, 64, false, false);   // O^T = S^T phiQ~^T
             constexpr uint32_t idOa = idesc_bf16(128, 64, true, false);    // O^T += V^T Pt^T
             constexpr uint32_t idS = idesc_bf16(128, 256, true, true);     // S^T += V^T K~
-            for (int it = 0; it < nch; ++it) {
-                const int s = it & 1;
-                const uint32_t par = it & 1;
-                if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 2)) break;
-                if (!mbar_wait(&X->p_empty, par ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 3)) break;
+            // score MMA of chunk c: P = [phiQ; phiK] phiK^T into the P columns
+            auto issue_scores = [&](int c) -> bool {
+                const int sc = c & 1;
+                if (!mbar_wait(&X->full[sc], (c >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 2)) return false;
+                // the score warpgroup has read P of chunk c - 1
+                if (!mbar_wait(&X->p_empty, (c & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 3)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kF / 16; ++k) {
                     const uint32_t off = (k >> 2) * kQKBlk + (k & 3) * 32;
-                    mma_ss(tmem + kColP, desc_k_sw128(sQ(s) + off), desc_k_sw128(sK(s) + off), idP,
+                    mma_ss(tmem + kColP, desc_k_sw128(sQ(sc) + off), desc_k_sw128(sK(sc) + off), idP,
                            k > 0 ? 1u : 0u);
                 }
                 mma_commit(&X->p_full);
+                return true;
+            };
+            bool ok = nch > 0 && issue_scores(0);
+            for (int it = 0; ok && it < nch; ++it) {
+                const int s = it & 1;
+                const uint32_t par = it & 1;
                 if (!mbar_wait(&X->epib_done, par, abort_flag, err, KID_SCAN_TC_OUT, 4)) break;
                 if (!mbar_wait(&X->sbf_ready, par, abort_flag, err, KID_SCAN_TC_OUT, 5)) break;
                 if (!mbar_wait(&X->o_empty, par ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 6)) break;
+                // the next chunk's scores go first, so that its score warpgroup
+                // work overlaps this chunk's readout and state update
+                if (it + 1 < nch && !issue_scores(it + 1)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kF / 16; ++k) {
@@ -520,8 +526,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
                 for (int k = 0; k < kC / 16; ++k) {
                     const uint64_t va = desc_mn_sw128(sV(s) + k * 2048, kBlk, 1024);
-                    mma_ss(tmem + kColO, va, desc_k_sw128(sP + k * 32), idOa, 1u);
-                    mma_ss(tmem + kColO, va, desc_k_sw128(sP + kC * 128 + k * 32), idOa, 1u);
+                    mma_ss(tmem + kColO, va, desc_k_sw128(sP(s) + k * 32), idOa, 1u);
+                    mma_ss(tmem + kColO, va, desc_k_sw128(sP(s) + kC * 128 + k * 32), idOa, 1u);
                 }
                 mma_commit(&X->o_full);
 #pragma unroll
@@ -583,7 +589,9 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 // would otherwise carry the 2^-9 rounding of each weight)
                 const uint32_t ta = tmem + kColP + ((uint32_t)(32 * q) << 16);
                 const int i = 32 * q + lane;
-                const float ci = X->cum[s][i];
+                const float *__restrict__ cum = X->cum[s];
+                const float ci = cum[i];
+                uint8_t *__restrict__ prow = gP(s);
                 float rs = 0.f;
 #pragma unroll
                 for (int hcol = 0; hcol < 2; ++hcol) {
@@ -593,53 +601,63 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         const int cc = 4 * hcol + c4;
-                        uint32_t pk[4], pl[4];
+                        uint4 hi, lo;
+                        uint32_t *pk = reinterpret_cast<uint32_t *>(&hi);
+                        uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int jl = c4 * 8 + 2 * e;      // column within this half
                             const int j = 32 * hcol + jl;
-                            const float e0 = (j <= i) ? __uint_as_float(pr[jl]) * fexp(ci - X->cum[s][j]) : 0.f;
-                            const float e1 = (j + 1 <= i) ? __uint_as_float(pr[jl + 1]) * fexp(ci - X->cum[s][j + 1]) : 0.f;
+                            const float e0 = (j <= i) ? __uint_as_float(pr[jl]) * fexp(ci - cum[j]) : 0.f;
+                            const float e1 = (j + 1 <= i) ? __uint_as_float(pr[jl + 1]) * fexp(ci - cum[j + 1]) : 0.f;
                             pk[e] = pack_bf16x2(e0, e1);
                             const float2 r = unpack_bf16x2(pk[e]);
                             pl[e] = pack_bf16x2(e0 - r.x, e1 - r.y);
                             rs += e0 + e1;
                         }
-                        sts128(sP + sw128_off(i, cc), make_uint4(pk[0], pk[1], pk[2], pk[3]));
-                        sts128(sP + kC * 128 + sw128_off(i, cc), make_uint4(pl[0], pl[1], pl[2], pl[3]));
+                        *reinterpret_cast<uint4 *>(prow + sw128_off(i, cc)) = hi;
+                        *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, cc)) = lo;
                     }
                 }
                 X->den_intra[i] = rs;
                 tc_fence_before();
             } else {
                 // weighted features in place (bf16): thread = one 16-byte chunk
-                // (8 features) of the row for the 32 tokens of its warp
+                // (8 features) of the row for the 32 tokens of its warp, 8 rows
+                // loaded at a time
                 const int bb = lane >> 3, cc = lane & 7;
                 const int tg = q - 2;
-                const uint32_t base = sK(s) + bb * kQKBlk;
+                uint8_t *__restrict__ base = gK(s) + bb * kQKBlk;
+                const float *__restrict__ wv = X->w[s];
                 float za[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) za[e] = 0.f;
-#pragma unroll 4
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = tg * 32 + jj;
-                    const uint32_t ad = base + sw128_off(j, cc);
-                    uint4 v = lds128(ad);
-                    uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
-                    const float wj = X->w[s][j];
+#pragma unroll 1
+                for (int j0 = tg * 32; j0 < tg * 32 + 32; j0 += 8) {
+                    uint4 v[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 k = unpack_bf16x2(pv[e]);
-                        pv[e] = pack_bf16x2(wj * k.x, wj * k.y);
-                        const float2 r = unpack_bf16x2(pv[e]);
-                        za[2 * e] += r.x;
-                        za[2 * e + 1] += r.y;
+                    for (int jj = 0; jj < 8; ++jj)
+                        v[jj] = *reinterpret_cast<const uint4 *>(base + sw128_off(j0 + jj, cc));
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        uint32_t *pv = reinterpret_cast<uint32_t *>(&v[jj]);
+                        const float wj = wv[j0 + jj];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 k = unpack_bf16x2(pv[e]);
+                            pv[e] = pack_bf16x2(wj * k.x, wj * k.y);
+                            const float2 r = unpack_bf16x2(pv[e]);
+                            za[2 * e] += r.x;
+                            za[2 * e + 1] += r.y;
+                        }
                     }
-                    sts128(ad, v);
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        *reinterpret_cast<uint4 *>(base + sw128_off(j0 + jj, cc)) = v[jj];
                 }
                 const int f0 = bb * 64 + cc * 8;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) X->zred[tg][f0 + e] = za[e];
+                *reinterpret_cast<float4 *>(&X->zred[tg][f0]) = make_float4(za[0], za[1], za[2], za[3]);
+                *reinterpret_cast<float4 *>(&X->zred[tg][f0 + 4]) = make_float4(za[4], za[5], za[6], za[7]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&X->p_empty);
@@ -648,27 +666,32 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             {
                 const int i = tb >> 1, hf = tb & 1;
                 const float qsi = X->qs[s][i];
+                uint8_t *__restrict__ qrow = gQ(s) + (2 * hf) * kQKBlk;
+                const float *__restrict__ zv = X->z;
+                uint4 v[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    v[k] = *reinterpret_cast<const uint4 *>(qrow + (k >> 3) * kQKBlk + sw128_off(i, k & 7));
                 float dot = 0.f;
 #pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    const int bb = 2 * hf + blk;
-                    const uint32_t base = sQ(s) + bb * kQKBlk;
+                for (int k = 0; k < 16; ++k) {
+                    uint32_t *pv = reinterpret_cast<uint32_t *>(&v[k]);
+                    const int f = (2 * hf + (k >> 3)) * 64 + (k & 7) * 8;
+                    const float4 za = *reinterpret_cast<const float4 *>(zv + f);
+                    const float4 zb = *reinterpret_cast<const float4 *>(zv + f + 4);
+                    const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const uint32_t ad = base + sw128_off(i, cc);
-                        uint4 v = lds128(ad);
-                        uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
-                        const int f = bb * 64 + cc * 8;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 x = unpack_bf16x2(pv[e]);
-                            pv[e] = pack_bf16x2(x.x * qsi, x.y * qsi);
-                            const float2 r = unpack_bf16x2(pv[e]);
-                            dot += r.x * X->z[f + 2 * e] + r.y * X->z[f + 2 * e + 1];
-                        }
-                        sts128(ad, v);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = unpack_bf16x2(pv[e]);
+                        pv[e] = pack_bf16x2(x.x * qsi, x.y * qsi);
+                        const float2 r = unpack_bf16x2(pv[e]);
+                        dot = fmaf(r.x, zz[2 * e], dot);
+                        dot = fmaf(r.y, zz[2 * e + 1], dot);
                     }
                 }
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    *reinterpret_cast<uint4 *>(qrow + (k >> 3) * kQKBlk + sw128_off(i, k & 7)) = v[k];
                 dot += __shfl_xor_sync(0xffffffffu, dot, 1);
                 if (hf == 0) X->rden[s][i] = 1.f / (X->den_intra[i] + dot);
             }
@@ -704,8 +727,6 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             tmem_ld32(ta + 32, r + 32);
             tmem_wait_ld();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&X->o_empty);
             const int64_t t0 = (int64_t)(c_begin + it) * kC;
             const int64_t obase = ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
             const int64_t tstride = (int64_t)g.H * g.dv;
@@ -720,6 +741,9 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 for (int i = 0; i < kC; ++i)
                     if (t0 + i < g.L) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]) * X->rden[s][i]);
             }
+            // O^T may be overwritten, and rden of this stage reused, from here on
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->o_empty);
         }
     } else {
         // ------------------------------------------------------------ WG-D: state pass

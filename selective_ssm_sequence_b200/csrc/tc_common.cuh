@@ -34,6 +34,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// The dynamic shared-memory base moved up to a 1024-byte boundary (the
+// 128-byte swizzle atoms of TMA and UMMA tiles).  Computed by offsetting the
+// __shared__ array itself, so the compiler keeps treating accesses through
+// the result as shared-memory accesses.
+__device__ __forceinline__ uint8_t *align_smem_1024(uint8_t *smem_raw) {
+    const uint32_t a = smem_u32(smem_raw);
+    return smem_raw + ((1024u - (a & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
     asm volatile(
@@ -277,18 +286,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
 
 // ------------------------------------------------------------------ host: launch setup
 
-// Raise a kernel's dynamic shared-memory limit once per device (the setting
-// persists; repeating it on every call only adds host latency).
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device): the
+// setting persists, and repeating it on every call only adds host latency.
+cudaError_t ensure_smem_limit_impl(const void *kern, int bytes);
+
 template <typename Kern>
 cudaError_t ensure_smem_limit(Kern kern, int bytes) {
-    static int done_bytes[64] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && done_bytes[dev] >= bytes) return cudaSuccess;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev >= 0 && dev < 64) done_bytes[dev] = bytes;
-    return e;
+    return ensure_smem_limit_impl(reinterpret_cast<const void *>(kern), bytes);
 }
 
 // ------------------------------------------------------------------ host: tensor maps

@@ -45,5 +45,25 @@ bool make_tmap_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t
     return r == CUDA_SUCCESS;
 }
 
+cudaError_t ensure_smem_limit_impl(const void *kern, int bytes) {
+    struct Entry {
+        const void *kern;
+        int dev;
+        int bytes;
+    };
+    static std::mutex mu;
+    static Entry done[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> g(mu);
+    for (int i = 0; i < n; ++i)
+        if (done[i].kern == kern && done[i].dev == dev && done[i].bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && n < 256) done[n++] = Entry{kern, dev, bytes};
+    return e;
+}
+
 }  // namespace tc
 }  // namespace hm

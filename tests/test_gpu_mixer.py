@@ -62,14 +62,18 @@ def test_mixer_with_biases(hm):
     assert rel_err(out, ref) <= TOL_BF16
 
 
-def test_mixer_stage1_identity(hm):
-    """Stage-1 identity initialisation (HedgeMamba explainer sec. 3.1): a = 1,
-    conv kernel [0, 0, 0, 1], gate weights 0 with bias SiLU^-1(1): the mixer
-    reduces to out_proj(linear attention(q, k, v))."""
+def test_mixer_stage1_conv_and_gate_identity(hm):
+    """Stage-1 identity initialisation of the conv and the gate (HedgeMamba
+    explainer sec. 3.1): conv kernel [0, 0, 0, 1] and gate weights 0 with bias
+    SiLU^-1(1) make both identities, so the mixer reduces to
+    out_proj(decayed linear attention(q, k, v)).  The decay stays on: with
+    a = 1 as well, late outputs are long averages and the tensor's rms (the
+    metric's floor) shrinks below the bf16 storage error of v and y on the
+    first tokens (a known limit, recorded in the design notes); the a = 1 scan
+    itself is covered by the scan tests."""
     cfg, w = _small_weights(53, 512, 2, 128)
     x = wl.mixer_x(cfg, B=2, L=257)
     E = cfg.H * cfg.d_head
-    w["A_log"] = np.full(cfg.H, -np.inf)
     w["conv_w"] = np.zeros((3, E, 4))
     w["conv_w"][:, :, -1] = 1.0
     w["W_g"] = np.zeros_like(w["W_g"])
@@ -81,7 +85,8 @@ def test_mixer_stage1_identity(hm):
     q = (xf @ w["W_q"].T).reshape(B, L, cfg.H, cfg.d_head)
     k = (xf @ w["W_k"].T).reshape(B, L, cfg.H, cfg.d_head)
     v = (xf @ w["W_v"].T).reshape(B, L, cfg.H, cfg.d_head)
-    o = oracle.scan_fwd(q, k, v, W_q=w["W_hq"], W_k=w["W_hk"])
+    dt = (xf @ w["W_dt"].T).reshape(B, L, cfg.H)
+    o = oracle.scan_fwd(q, k, v, W_q=w["W_hq"], W_k=w["W_hk"], dt=dt, A_log=w["A_log"])
     gate = oracle.silu(b_g)
     ref = (o.reshape(B * L, E) * gate) @ w["W_o"].T
     assert rel_err(out, ref.reshape(B, L, D)) <= TOL_BF16
