@@ -63,37 +63,103 @@ NCU_TRAFFIC_BYTES = {}
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled in the background."""
+    """SM clock and clock-event (throttle) reasons of one GPU, read in the
+    background while the timed region runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Reads only: NVML queries every 5 ms (pynvml), else `nvidia-smi -lms 50`.
+    summary() keeps the samples taken between mark_start() and mark_stop(),
+    the host-side bounds of the timed region."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.samples = []
-        self.proc = None
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.device = device
+        self.samples = []        # (host time, sm MHz, max sm MHz, set of reason names)
+        self.t0 = self.t1 = None
+        self.source = None
+        self._stop = threading.Event()
         self.thread = None
+        self.proc = None
+        self.nv = self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = self._nvml_handle(device)
+        except Exception:
+            self.nv = self.handle = None
+
+    def _nvml_handle(self, device):
+        nv = self.nv
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(device)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", str(self.gpu)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        if self.handle is not None:
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+        else:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "--query-gpu=" + self.SMI_FIELDS, "--format=csv,noheader,nounits",
+                     "-lms", "50", "-i", str(self.device)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                return
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
+    def _poll_nvml(self):
+        nv, hd = self.nv, self.handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        masks = [(n, getattr(nv, attr, 0)) for n, attr in self.REASONS]
+        try:
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(hd, nv.NVML_CLOCK_SM))
+        except Exception:
+            mx = None
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                sm = float(nv.nvmlDeviceGetClockInfo(hd, nv.NVML_CLOCK_SM))
+                bits = int(get_reasons(hd))
+                self.samples.append((t, sm, mx, {n for n, m in masks if m and bits & m}))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append(parts)
+            if len(parts) < 9:
+                continue
+            try:
+                sm, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            rs = {n for n, val in zip(names, parts[5:9]) if val.lower().startswith("active")}
+            self.samples.append((time.perf_counter(), sm, mx, rs))
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_stop(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -104,22 +170,19 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for s in self.samples:
-            try:
-                sm.append(float(s[1]))
-                mx.append(float(s[2]))
-            except ValueError:
-                continue
-            for n, val in zip(names, s[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        lo = self.t0 if self.t0 is not None else -float("inf")
+        hi = self.t1 if self.t1 is not None else float("inf")
+        inside = [x for x in self.samples if lo <= x[0] <= hi]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0,
+                    "source": self.source}
+        reasons = set()
+        for x in inside:
+            reasons |= x[3]
+        mxs = [x[2] for x in inside if x[2] is not None]
+        return {"sm_mhz": statistics.median(x[1] for x in inside),
+                "sm_max_mhz": max(mxs) if mxs else None,
+                "reasons": sorted(reasons), "samples": len(inside), "source": self.source}
 
 
 # ---------------------------------------------------------------- helpers
@@ -265,10 +328,12 @@ def bench_prefill(cfg, args, rank, world, torch):
     assert hm.hm_get_device_error() == hm.HM_OK
     barrier(world)
     torch.cuda.synchronize()
+    sampler.mark_start()
     for i in range(K):
         flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
+    sampler.mark_stop()
     launches = launches_per_step * K
     barrier(world)
     torch.cuda.synchronize()
@@ -456,11 +521,13 @@ def bench_decode(cfg, args, rank, world, torch):
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
     e0.record(stream)
     for i in range(steps):
         graphs[i % nstep_tokens].replay()
     e1.record(stream)
     torch.cuda.synchronize()
+    sampler.mark_stop()
     sampler.stop()
     assert hm.hm_get_device_error() == hm.HM_OK
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, torch)
@@ -514,6 +581,7 @@ def bench_mixer(cfg, args, rank, world, torch):
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
     evs = []
+    sampler.mark_start()
     for _ in range(args.steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -521,6 +589,7 @@ def bench_mixer(cfg, args, rank, world, torch):
         e1.record(stream)
         evs.append((e0, e1))
     torch.cuda.synchronize()
+    sampler.mark_stop()
     sampler.stop()
     assert hm.hm_get_device_error() == hm.HM_OK
     ms = max_over_ranks(sum(x.elapsed_time(y) for x, y in evs) / args.steps, world, torch)

@@ -15,6 +15,8 @@
 //   O        = Pt V + diag(exp(cum)) phiQ S_prev               (tensor cores)
 //   den      = rowsum(Pt) + exp(cum) (phiQ z_prev)
 //   S        = gamma S_prev + (w phiK)^T V,  w_j = exp(cum_last - cum_j) <= 1
+//            = gamma S_prev + phiK^T (w V)   (the output kernel weights the
+//              128 value channels of its CTA rather than the 256 features)
 //   z        = gamma z_prev + sum_j w_j phik_j
 // These are exact rewrites of the recurrence.  The state is kept transposed
 // (S^T, value channel x feature) in TMEM: the state update V^T (w phiK) and the
@@ -348,20 +350,24 @@ constexpr uint32_t kColSB = 256; // S^T bf16 pairs  [128 x 128]
 constexpr uint32_t kColO = 384;  // O^T fp32        [128 x 64 tokens]
 constexpr uint32_t kColP = 448;  // [phiQ; phiK] phiK^T fp32 [128 x 64]; lanes 0..63 = P
 
+constexpr int kZGroups = 5;      // token groups of the weighted key-feature sums (13 tokens)
+constexpr int kZTok = 13;
+constexpr int kHelpers = 160;    // threads of the five helper warps
+
 struct CAux {
     float cum[2][kC];
     float qs[2][kC];
     float w[2][kC];
     float rden[2][kC];   // 1 / den
-    float den_intra[kC];
+    float dint[2][kC];   // row sums of Pt: [0] columns 0..31, [1] columns 32..63
+    float dotq[4][kC];   // phiq_i . z_prev over each quarter of the features
     float z[kF];
-    alignas(16) float zred[4][kF];   // per token-group partial sums of the weighted features
+    alignas(16) float zred[kZGroups][kF];
     float gam[2];
     float redb[4];
     float redd[4];
     uint64_t full[2], empty[2];
-    uint64_t p_full, p_empty, epib_done, o_full, o_empty, s_full, sbf_ready;
-    uint64_t den_ready[2];
+    uint64_t p_full, epib_done, o_full, o_empty, s_full, sbf_ready;
     uint32_t tmem;
     int abort;
 };
@@ -373,10 +379,12 @@ struct CAux {
 // phiK phiK^T, which is not used).
 constexpr int kQKBlk = 2 * kBlk;                       // [Q | K] of one feature block
 constexpr int kCStage = 4 * kQKBlk + kTileV;           // Q, K, V of one chunk
-constexpr int kCPBytes = 2 * kC * 128;             // Pt as bf16 hi (8 KB) then lo (8 KB)
-constexpr int kCOffP = 2 * kCStage;               // one Pt buffer per stage
-constexpr int kCOffAux = kCOffP + 2 * kCPBytes;
+constexpr int kCPBytes = 2 * kC * 128;                 // Pt as bf16 hi (8 KB) then lo (8 KB)
+constexpr int kCOffP = 2 * kCStage;                    // one Pt buffer per stage
+constexpr int kCOffVt = kCOffP + 2 * kCPBytes;         // w (.) V of the current chunk
+constexpr int kCOffAux = kCOffVt + kTileV;
 constexpr int kCSmem = kCOffAux + (int)sizeof(CAux) + 1024;
+static_assert(kCSmem <= 227 * 1024, "phase C shared memory");
 
 struct OutArgs {
     Geo g;
@@ -405,6 +413,20 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
     return tot;
 }
 
+// Warp roles (14 warps):
+//   0      TMA producer (phiQ, phiK, V of each chunk; two stages)
+//   1      MMA issuer
+//   2..9   compute group (256 threads): per chunk the decay prefix sums, the
+//          decayed score tile Pt (three 32 x 32 quadrants: rows 0..31 need
+//          only columns 0..31), w (.) V, the weighted key-feature sums for z,
+//          the scaled queries e^cum (.) phiQ with phiq . z_prev, the
+//          denominators and z; then the outputs of the previous chunk, so
+//          that those loads and stores overlap this chunk's MMAs
+//   10..13 state pass: S^T (fp32, TMEM) -> bf16 copy for the next readout,
+//          and S^T <- gamma S^T before the next state MMA
+// Per chunk the MMA issuer runs: scores of the next chunk, then the readout
+// O^T = S^T (e^cum phiQ)^T, O^T += V^T Pt^T (hi and lo), and the state
+// update S^T += (w V)^T phiK.
 __global__ void __launch_bounds__(448, 1)
 scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, OutArgs a, DevErr err) {
@@ -430,24 +452,25 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     auto sK = [&](int s) { return sbase + s * kCStage + kBlk; };
     auto sV = [&](int s) { return sbase + s * kCStage + 4 * kQKBlk; };
     auto sP = [&](int s) { return sbase + kCOffP + s * kCPBytes; };
-    // generic pointers to the same buffers, for CUDA-core accesses
+    const uint32_t sVt = sbase + kCOffVt;
+    // pointers to the same buffers, for CUDA-core accesses
     auto gQ = [&](int s) { return smem + s * kCStage; };
     auto gK = [&](int s) { return smem + s * kCStage + kBlk; };
+    auto gV = [&](int s) { return smem + s * kCStage + 4 * kQKBlk; };
     auto gP = [&](int s) { return smem + kCOffP + s * kCPBytes; };
+    uint8_t *const gVt = smem + kCOffVt;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&X->full[s], 1);
             mbar_init(&X->empty[s], 1);
-            mbar_init(&X->den_ready[s], 1);
         }
         mbar_init(&X->p_full, 1);
-        mbar_init(&X->p_empty, 4);      // one arrival per warp of the group
         mbar_init(&X->epib_done, 1);
         mbar_init(&X->o_full, 1);
-        mbar_init(&X->o_empty, 4);
+        mbar_init(&X->o_empty, 8);      // one arrival per compute warp
         mbar_init(&X->s_full, 1);
-        mbar_init(&X->sbf_ready, 4);
+        mbar_init(&X->sbf_ready, 4);    // one arrival per state-pass warp
         X->abort = 0;
         mbar_fence_init();
     }
@@ -489,13 +512,13 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             constexpr uint32_t idP = idesc_bf16(128, 64, false, false);    // [phiQ; phiK] phiK^T
             constexpr uint32_t idOi = idesc_bf16(128, 64, false, false);   // O^T = S^T phiQ~^T
             constexpr uint32_t idOa = idesc_bf16(128, 64, true, false);    // O^T += V^T Pt^T
-            constexpr uint32_t idS = idesc_bf16(128, 256, true, true);     // S^T += V^T K~
+            constexpr uint32_t idS = idesc_bf16(128, 256, true, true);     // S^T += (wV)^T phiK
             // score MMA of chunk c: P = [phiQ; phiK] phiK^T into the P columns
+            // (the compute group has read P of chunk c - 1: its epib_done is
+            // complete whenever this runs)
             auto issue_scores = [&](int c) -> bool {
                 const int sc = c & 1;
                 if (!mbar_wait(&X->full[sc], (c >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 2)) return false;
-                // the score warpgroup has read P of chunk c - 1
-                if (!mbar_wait(&X->p_empty, (c & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 3)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kF / 16; ++k) {
@@ -513,8 +536,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (!mbar_wait(&X->epib_done, par, abort_flag, err, KID_SCAN_TC_OUT, 4)) break;
                 if (!mbar_wait(&X->sbf_ready, par, abort_flag, err, KID_SCAN_TC_OUT, 5)) break;
                 if (!mbar_wait(&X->o_empty, par ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 6)) break;
-                // the next chunk's scores go first, so that its score warpgroup
-                // work overlaps this chunk's readout and state update
+                // the next chunk's scores go first, so that the compute group's
+                // work on it overlaps this chunk's readout and state update
                 if (it + 1 < nch && !issue_scores(it + 1)) break;
                 tc_fence_after();
 #pragma unroll
@@ -532,226 +555,269 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 mma_commit(&X->o_full);
 #pragma unroll
                 for (int k = 0; k < kC / 16; ++k)
-                    mma_ss(tmem + kColS, desc_mn_sw128(sV(s) + k * 2048, kBlk, 1024),
+                    mma_ss(tmem + kColS, desc_mn_sw128(sVt + k * 2048, kBlk, 1024),
                            desc_mn_sw128(sK(s) + k * 2048, kQKBlk, 1024), idS, 1u);
                 mma_commit(&X->s_full);
                 mma_commit(&X->empty[s]);
             }
         }
-    } else if (warp < 6) {
-        // ------------------------------------------------------------ WG-B: scores, features
-        const int tb = threadIdx.x - 64;
-        const int q = warp & 3;
+    } else if (warp < 10) {
+        // ------------------------------------------------------------ compute group
+        const int gt = threadIdx.x - 64;   // 0..255
+        const int q = warp & 3;            // TMEM lane quarter of this warp
         {
             const float *zi = nullptr;
             if (seg == 0) zi = a.z0 ? a.z0 + bh * kF : nullptr;
             else zi = a.z_start + (bh * g.G + seg) * kF;
-            for (int f = tb; f < kF; f += 128) X->z[f] = zi ? zi[f] : 0.f;
+            X->z[gt] = zi ? zi[gt] : 0.f;
+            // rows 0..31 x columns 32..63 of Pt (hi and lo, both buffers) are
+            // always zero: written once here
+            const int row = gt & 31, cc = 4 + ((gt >> 5) & 3);
+            uint8_t *pb = gP(gt >> 7);
+            *reinterpret_cast<uint4 *>(pb + sw128_off(row, cc)) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(pb + kC * 128 + sw128_off(row, cc)) = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem();
         }
-        named_sync(1, 128);
+        // outputs of chunk c (TMEM O^T: lane = value channel, column = token);
+        // warps 2..5 take tokens 0..31, warps 6..9 tokens 32..63
+        auto epilogue = [&](int c) -> bool {
+            bool okc = mbar_wait(&X->o_full, c & 1, abort_flag, err, KID_SCAN_TC_OUT, 9);
+            okc = __all_sync(0xffffffffu, okc);
+            const int th = warp >= 6 ? 1 : 0;
+            if (okc) {
+                tc_fence_after();
+                uint32_t r[32];
+                tmem_ld32(tmem + kColO + 32 * th + ((uint32_t)(32 * q) << 16), r);
+                tmem_wait_ld();
+                tc_fence_before();
+                const int ch = 32 * q + lane;
+                const int64_t t0 = (int64_t)(c_begin + c) * kC + 32 * th;
+                const int64_t obase = ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
+                const int64_t tstride = (int64_t)g.H * g.dv;
+                const float *rd = X->rden[c & 1] + 32 * th;
+                if (a.o_f32) {
+                    float *op = (float *)a.o + obase;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (t0 + i < g.L) op[i * tstride] = __uint_as_float(r[i]) * rd[i];
+                } else {
+                    __nv_bfloat16 *op = (__nv_bfloat16 *)a.o + obase;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (t0 + i < g.L) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]) * rd[i]);
+                }
+            }
+            // O^T may be overwritten from here on
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->o_empty);
+            return okc;
+        };
         // log a of the next chunk's tokens is fetched one chunk ahead
-        float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, tb);
-        for (int it = 0; it < nch; ++it) {
+        float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, gt);
+        bool ok = named_sync_and(1, 256, true);
+        // every exit from this loop is taken by the whole group (after a
+        // barrier-AND), so `it` is uniform when it ends
+        int it = 0;
+        for (; it < nch; ++it) {
             const int s = it & 1;
-            // (1) decay of the chunk: cum, exp(cum), weights, gamma
-            {
+            // (1) decay of the chunk (warps 2, 3: thread = token): cum, e^cum,
+            // weights e^(cum_last - cum), gamma
+            if (gt < kC) {
                 const float l = l_next;
-                if (it + 1 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 1) * kC, tb);
+                if (it + 1 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 1) * kC, gt);
                 float x = l;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    float y = __shfl_up_sync(0xffffffffu, x, o);
+                    const float y = __shfl_up_sync(0xffffffffu, x, o);
                     if (lane >= o) x += y;
                 }
-                if (tb == 31) X->redb[0] = x;
-                named_sync(1, 128);
-                if (tb >= 32 && tb < kC) x += X->redb[0];
-                if (tb == kC - 1) X->redb[1] = x;
-                named_sync(1, 128);
+                if (gt == 31) X->redb[0] = x;
+                named_sync(3, 64);
+                if (gt >= 32) x += X->redb[0];
+                if (gt == kC - 1) X->redb[1] = x;
+                named_sync(3, 64);
                 const float total = X->redb[1];
-                if (tb < kC) {
-                    X->cum[s][tb] = x;
-                    X->qs[s][tb] = fexp(x);
-                    X->w[s][tb] = fexp(total - x);
-                }
-                if (tb == 0) X->gam[s] = fexp(total);
-                named_sync(1, 128);
+                X->cum[s][gt] = x;
+                X->qs[s][gt] = fexp(x);
+                X->w[s][gt] = fexp(total - x);
+                if (gt == 0) X->gam[s] = fexp(total);
             }
-            // (2) once P is in TMEM (MMA1 done, so phiK is free): warps 4, 5 (the
-            // owners of TMEM lanes 0..63) form the decayed scores Pt while warps
-            // 2, 3 rebuild the weighted features w_j phik_j in place.
-            if (!mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7)) break;
-            if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8)) break;
+            ok = named_sync_and(1, 256, ok);
+            if (!ok) break;
+            // (2) once the chunk's scores are in TMEM
+            bool okw = mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7) &&
+                       mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8);
+            okw = __all_sync(0xffffffffu, okw);
             tc_fence_after();
-            if (q < 2) {
-                // Pt = P * exp(cum_i - cum_j) on j <= i, row sums; Pt -> smem as bf16
-                // hi + lo (the PV product runs twice: a few-token weighted average
-                // would otherwise carry the 2^-9 rounding of each weight)
-                const uint32_t ta = tmem + kColP + ((uint32_t)(32 * q) << 16);
+            if (warp == 4 || warp == 5 || warp == 9) {
+                // Pt = P * exp(cum_i - cum_j) on j <= i, as bf16 hi + lo (the PV
+                // product runs on both: a few-token weighted average would
+                // otherwise carry the 2^-9 rounding of each weight), and row sums.
+                // warp 4: rows 0..31 x columns 0..31; warp 5: rows 32..63 x
+                // columns 0..31 (all below the diagonal); warp 9: rows 32..63 x
+                // columns 32..63.
                 const int i = 32 * q + lane;
-                const float *__restrict__ cum = X->cum[s];
-                const float ci = cum[i];
-                uint8_t *__restrict__ prow = gP(s);
-                float rs = 0.f;
-#pragma unroll
-                for (int hcol = 0; hcol < 2; ++hcol) {
+                const int jc = warp == 9 ? 32 : 0;
+                const bool masked = warp != 5;
+                if (okw) {
                     uint32_t pr[32];
-                    tmem_ld32(ta + 32 * hcol, pr);
+                    tmem_ld32(tmem + kColP + jc + ((uint32_t)(32 * q) << 16), pr);
                     tmem_wait_ld();
+                    const float ci = X->cum[s][i];
+                    const float *__restrict__ cj = X->cum[s] + jc;
+                    uint8_t *__restrict__ prow = gP(s);
+                    float rs = 0.f;
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
-                        const int cc = 4 * hcol + c4;
                         uint4 hi, lo;
                         uint32_t *pk = reinterpret_cast<uint32_t *>(&hi);
                         uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+                        const float4 ca = *reinterpret_cast<const float4 *>(cj + c4 * 8);
+                        const float4 cb = *reinterpret_cast<const float4 *>(cj + c4 * 8 + 4);
+                        const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int jl = c4 * 8 + 2 * e;      // column within this half
-                            const int j = 32 * hcol + jl;
-                            const float e0 = (j <= i) ? __uint_as_float(pr[jl]) * fexp(ci - cum[j]) : 0.f;
-                            const float e1 = (j + 1 <= i) ? __uint_as_float(pr[jl + 1]) * fexp(ci - cum[j + 1]) : 0.f;
+                            const int jl = c4 * 8 + 2 * e;
+                            const int j = jc + jl;
+                            const float e0 = (!masked || j <= i) ? __uint_as_float(pr[jl]) * fexp(ci - cv[2 * e]) : 0.f;
+                            const float e1 =
+                                (!masked || j + 1 <= i) ? __uint_as_float(pr[jl + 1]) * fexp(ci - cv[2 * e + 1]) : 0.f;
                             pk[e] = pack_bf16x2(e0, e1);
                             const float2 r = unpack_bf16x2(pk[e]);
                             pl[e] = pack_bf16x2(e0 - r.x, e1 - r.y);
                             rs += e0 + e1;
                         }
+                        const int cc = (jc >> 3) + c4;
                         *reinterpret_cast<uint4 *>(prow + sw128_off(i, cc)) = hi;
                         *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, cc)) = lo;
                     }
+                    X->dint[jc ? 1 : 0][i] = rs;
+                    tc_fence_before();
                 }
-                X->den_intra[i] = rs;
-                tc_fence_before();
             } else {
-                // weighted features in place (bf16): thread = one 16-byte chunk
-                // (8 features) of the row for the 32 tokens of its warp, 8 rows
-                // loaded at a time
-                const int bb = lane >> 3, cc = lane & 7;
-                const int tg = q - 2;
-                uint8_t *__restrict__ base = gK(s) + bb * kQKBlk;
+                // helpers (warps 2, 3, 6, 7, 8)
+                const int hx = (warp < 4 ? warp - 2 : warp - 4) * 32 + lane;   // 0..159
                 const float *__restrict__ wv = X->w[s];
-                float za[8];
+                // weighted key-feature sums sum_j w_j phik_j: thread = one
+                // 16-byte chunk (8 features) over a group of 13 tokens
+                {
+                    const int cc = hx & 31, tg = hx >> 5;
+                    const uint8_t *__restrict__ base = gK(s) + (cc >> 3) * kQKBlk;
+                    const int j0 = tg * kZTok;
+                    uint4 kv[kZTok];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) za[e] = 0.f;
-#pragma unroll 1
-                for (int j0 = tg * 32; j0 < tg * 32 + 32; j0 += 8) {
-                    uint4 v[8];
+                    for (int jj = 0; jj < kZTok; ++jj)
+                        kv[jj] = (j0 + jj < kC) ? *reinterpret_cast<const uint4 *>(base + sw128_off(j0 + jj, cc & 7))
+                                                : make_uint4(0u, 0u, 0u, 0u);
+                    float2 za[4];
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj)
-                        v[jj] = *reinterpret_cast<const uint4 *>(base + sw128_off(j0 + jj, cc));
+                    for (int e = 0; e < 4; ++e) za[e] = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        uint32_t *pv = reinterpret_cast<uint32_t *>(&v[jj]);
-                        const float wj = wv[j0 + jj];
+                    for (int jj = 0; jj < kZTok; ++jj) {
+                        const float wj = (j0 + jj < kC) ? wv[j0 + jj] : 0.f;
+                        const float2 w2 = make_float2(wj, wj);
+                        const uint32_t *pv = reinterpret_cast<const uint32_t *>(&kv[jj]);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 k = unpack_bf16x2(pv[e]);
-                            pv[e] = pack_bf16x2(wj * k.x, wj * k.y);
-                            const float2 r = unpack_bf16x2(pv[e]);
-                            za[2 * e] += r.x;
-                            za[2 * e + 1] += r.y;
-                        }
+                        for (int e = 0; e < 4; ++e) za[e] = fma2(unpack_bf16x2(pv[e]), w2, za[e]);
+                    }
+                    float *zr = &X->zred[tg][cc * 8];
+                    *reinterpret_cast<float4 *>(zr) = make_float4(za[0].x, za[0].y, za[1].x, za[1].y);
+                    *reinterpret_cast<float4 *>(zr + 4) = make_float4(za[2].x, za[2].y, za[3].x, za[3].y);
+                }
+                // w (.) V into its own tile, once the previous chunk's state MMA
+                // has read that tile
+                if (it > 0) okw = mbar_wait(&X->s_full, (it - 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 13) && okw;
+                okw = __all_sync(0xffffffffu, okw);
+                if (okw) {
+                    const uint8_t *__restrict__ vsrc = gV(s);
+                    uint4 vv[7];
+                    uint32_t offs[7];
+#pragma unroll
+                    for (int r = 0; r < 7; ++r) {
+                        const int u = hx + r * kHelpers;
+                        const int j = (u >> 4) & (kC - 1), ci = u & 15;
+                        offs[r] = (uint32_t)((ci >> 3) * kBlk) + sw128_off(j, ci & 7);
+                        if (u < kC * 16) vv[r] = *reinterpret_cast<const uint4 *>(vsrc + offs[r]);
                     }
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj)
-                        *reinterpret_cast<uint4 *>(base + sw128_off(j0 + jj, cc)) = v[jj];
+                    for (int r = 0; r < 7; ++r) {
+                        const int u = hx + r * kHelpers;
+                        if (u < kC * 16) {
+                            const float wj = wv[u >> 4];
+                            const float2 w2 = make_float2(wj, wj);
+                            uint32_t *pv = reinterpret_cast<uint32_t *>(&vv[r]);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 x = mul2(unpack_bf16x2(pv[e]), w2);
+                                pv[e] = pack_bf16x2(x.x, x.y);
+                            }
+                            *reinterpret_cast<uint4 *>(gVt + offs[r]) = vv[r];
+                        }
+                    }
                 }
-                const int f0 = bb * 64 + cc * 8;
-                *reinterpret_cast<float4 *>(&X->zred[tg][f0]) = make_float4(za[0], za[1], za[2], za[3]);
-                *reinterpret_cast<float4 *>(&X->zred[tg][f0 + 4]) = make_float4(za[4], za[5], za[6], za[7]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&X->p_empty);
-            named_sync(1, 128);   // den_intra and the z partial sums are complete
-            // (3) phiQ rows scaled by exp(cum_i) in place; den = rowsum + e^cum phiq . z
-            {
-                const int i = tb >> 1, hf = tb & 1;
+            // (3) every thread: the query row scaled by e^cum_i, in place, and
+            // phiq_i . z_prev over one quarter of the features (on the unscaled
+            // bf16 values; the scale is applied to the sum)
+            if (okw) {
+                const int i = gt & 63, qf = gt >> 6;
                 const float qsi = X->qs[s][i];
-                uint8_t *__restrict__ qrow = gQ(s) + (2 * hf) * kQKBlk;
-                const float *__restrict__ zv = X->z;
-                uint4 v[16];
+                const float2 q2 = make_float2(qsi, qsi);
+                uint8_t *__restrict__ qb = gQ(s) + qf * kQKBlk;
+                const float *__restrict__ zq = X->z + qf * 64;
+                uint4 v[8];
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    v[k] = *reinterpret_cast<const uint4 *>(qrow + (k >> 3) * kQKBlk + sw128_off(i, k & 7));
-                float dot = 0.f;
+                for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const uint4 *>(qb + sw128_off(i, k));
+                float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
+                for (int k = 0; k < 8; ++k) {
                     uint32_t *pv = reinterpret_cast<uint32_t *>(&v[k]);
-                    const int f = (2 * hf + (k >> 3)) * 64 + (k & 7) * 8;
-                    const float4 za = *reinterpret_cast<const float4 *>(zv + f);
-                    const float4 zb = *reinterpret_cast<const float4 *>(zv + f + 4);
-                    const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+                    const float4 za = *reinterpret_cast<const float4 *>(zq + k * 8);
+                    const float4 zb = *reinterpret_cast<const float4 *>(zq + k * 8 + 4);
+                    const float2 zz[4] = {make_float2(za.x, za.y), make_float2(za.z, za.w), make_float2(zb.x, zb.y),
+                                          make_float2(zb.z, zb.w)};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = unpack_bf16x2(pv[e]);
-                        pv[e] = pack_bf16x2(x.x * qsi, x.y * qsi);
-                        const float2 r = unpack_bf16x2(pv[e]);
-                        dot = fmaf(r.x, zz[2 * e], dot);
-                        dot = fmaf(r.y, zz[2 * e + 1], dot);
+                        d2 = fma2(x, zz[e], d2);
+                        const float2 y = mul2(x, q2);
+                        pv[e] = pack_bf16x2(y.x, y.y);
                     }
                 }
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    *reinterpret_cast<uint4 *>(qrow + (k >> 3) * kQKBlk + sw128_off(i, k & 7)) = v[k];
-                dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-                if (hf == 0) X->rden[s][i] = 1.f / (X->den_intra[i] + dot);
-            }
-            named_sync(1, 128);   // every reader of z in step (3) is done
-            // (4) z <- gamma z + sum_j w_j phik_j
-            {
-                const float gm = X->gam[s];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int f = 2 * tb + e;
-                    X->z[f] = fmaf(gm, X->z[f], X->zred[0][f] + X->zred[1][f]);
-                }
+                for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4 *>(qb + sw128_off(i, k)) = v[k];
+                X->dotq[qf][i] = d2.x + d2.y;
             }
             fence_proxy_async_smem();
-            named_sync(1, 128);
-            if (tb == 0) {
-                mbar_arrive(&X->epib_done);
-                mbar_arrive(&X->den_ready[s]);
+            ok = named_sync_and(1, 256, okw);
+            if (!ok) break;
+            if (gt == 0) mbar_arrive(&X->epib_done);
+            // (4) denominators and z (the chunk's MMAs run meanwhile)
+            if (gt < kC) {
+                const int i = gt;
+                const float dq = (X->dotq[0][i] + X->dotq[1][i]) + (X->dotq[2][i] + X->dotq[3][i]);
+                const float den = X->dint[0][i] + (i >= 32 ? X->dint[1][i] : 0.f) + X->qs[s][i] * dq;
+                X->rden[s][i] = 1.f / den;
             }
+            {
+                float acc = 0.f;
+#pragma unroll
+                for (int tg = 0; tg < kZGroups; ++tg) acc += X->zred[tg][gt];
+                X->z[gt] = fmaf(X->gam[s], X->z[gt], acc);
+            }
+            // (5) outputs of the previous chunk
+            if (it > 0 && !epilogue(it - 1)) ok = false;
         }
-    } else if (warp < 10) {
-        // ------------------------------------------------------------ WG-C: outputs
-        const int q = warp & 3;
-        const int ch = 32 * q + lane;
-        for (int it = 0; it < nch; ++it) {
-            const int s = it & 1;
-            if (!mbar_wait(&X->o_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 9)) break;
-            if (!mbar_wait(&X->den_ready[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 10)) break;
-            tc_fence_after();
-            uint32_t r[64];
-            const uint32_t ta = tmem + kColO + ((uint32_t)(32 * q) << 16);
-            tmem_ld32(ta, r);
-            tmem_ld32(ta + 32, r + 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            const int64_t t0 = (int64_t)(c_begin + it) * kC;
-            const int64_t obase = ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
-            const int64_t tstride = (int64_t)g.H * g.dv;
-            if (a.o_f32) {
-                float *op = (float *)a.o + obase;
-#pragma unroll
-                for (int i = 0; i < kC; ++i)
-                    if (t0 + i < g.L) op[i * tstride] = __uint_as_float(r[i]) * X->rden[s][i];
-            } else {
-                __nv_bfloat16 *op = (__nv_bfloat16 *)a.o + obase;
-#pragma unroll
-                for (int i = 0; i < kC; ++i)
-                    if (t0 + i < g.L) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]) * X->rden[s][i]);
-            }
-            // O^T may be overwritten, and rden of this stage reused, from here on
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&X->o_empty);
+        if (it == nch && nch > 0) {
+            // 1 / den of the last chunk is complete
+            if (named_sync_and(1, 256, ok)) epilogue(nch - 1);
         }
     } else {
-        // ------------------------------------------------------------ WG-D: state pass
+        // ------------------------------------------------------------ state pass
         const int td = threadIdx.x - 320;
         const int q = warp & 3;
         const int ch = 32 * q + lane;
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
-        bool ok = true;
         // prologue: start state -> bf16 copy (for the first readout) and fp32 x gamma_0
         float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, td);
         {
@@ -770,34 +836,38 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
-                tmem_st16(tmem + kColS + c0 + lanebase, v);
-                tmem_st16(tmem + kColS + c0 + 16 + lanebase, v + 16);
+                tmem_st32(tmem + kColS + c0 + lanebase, v);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
-        for (int it = 0; ok && it + 1 < nch; ++it) {
+        bool ok = true;
+        for (int it = 0; it + 1 < nch; ++it) {
             const float gn = fexp(chunk_total(l_next, td, X->redd, 2));
             if (it + 2 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 2) * kC, td);
-            if (!mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11)) {
-                ok = false;
-                break;
-            }
+            ok = named_sync_and(2, 128, ok && mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11));
+            if (!ok) break;
             tc_fence_after();
-#pragma unroll 2
-            for (int c0 = 0; c0 < kF; c0 += 32) {
-                uint32_t v[32], pk[16];
-                tmem_ld32(tmem + kColS + c0 + lanebase, v);
+            // 32-column blocks, the next block's load in flight while this one
+            // is converted and stored
+            const float2 g2 = make_float2(gn, gn);
+#pragma unroll 1
+            for (int blk = 0; blk < kF / 32; ++blk) {
+                uint32_t cur[32], pk[16];
+                tmem_ld32(tmem + kColS + 32 * blk + lanebase, cur);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-                tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gn);
-                tmem_st16(tmem + kColS + c0 + lanebase, v);
-                tmem_st16(tmem + kColS + c0 + 16 + lanebase, v + 16);
+                for (int j = 0; j < 16; ++j) {
+                    const float2 x = make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1]));
+                    pk[j] = pack_bf16x2(x.x, x.y);
+                    const float2 y = mul2(x, g2);
+                    cur[2 * j] = __float_as_uint(y.x);
+                    cur[2 * j + 1] = __float_as_uint(y.y);
+                }
+                tmem_st16(tmem + kColSB + 16 * blk + lanebase, pk);
+                tmem_st32(tmem + kColS + 32 * blk + lanebase, cur);
             }
             tmem_wait_st();
             tc_fence_before();
