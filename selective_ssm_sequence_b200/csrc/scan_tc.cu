@@ -52,7 +52,9 @@ constexpr int kBlk = kC * 128;  // one [64 rows x 128 B] block = 8 KB
 constexpr int kTileF = 4 * kBlk;   // [64 x 256] bf16 tile = 32 KB
 constexpr int kTileV = 2 * kBlk;   // [64 x 128] bf16 tile = 16 KB
 
-__device__ __forceinline__ float fexp(float x) { return exp2f(x * 1.4426950408889634f); }
+// e^x for the decay factors (arguments <= 0 except the log-space prefix sums
+// of a chunk; results are used at bf16 / fp32-accumulate precision)
+__device__ __forceinline__ float fexp(float x) { return ex2_approx(x * 1.4426950408889634f); }
 
 struct Geo {
     int64_t B, L;
@@ -368,6 +370,7 @@ struct CAux {
     float redd[4];
     uint64_t full[2], empty[2];
     uint64_t p_full, epib_done, o_full, o_empty, s_full, sbf_ready;
+    uint64_t den_ready[2], den_free[2];   // 1 / den of a stage written / read
     uint32_t tmem;
     int abort;
 };
@@ -420,10 +423,10 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
 //          decayed score tile Pt (three 32 x 32 quadrants: rows 0..31 need
 //          only columns 0..31), w (.) V, the weighted key-feature sums for z,
 //          the scaled queries e^cum (.) phiQ with phiq . z_prev, the
-//          denominators and z; then the outputs of the previous chunk, so
-//          that those loads and stores overlap this chunk's MMAs
-//   10..13 state pass: S^T (fp32, TMEM) -> bf16 copy for the next readout,
-//          and S^T <- gamma S^T before the next state MMA
+//          denominators and z
+//   10..13 outputs and state pass: o = O^T / den for the chunk, then S^T
+//          (fp32, TMEM) -> bf16 copy for the next readout and
+//          S^T <- gamma S^T before the next state MMA
 // Per chunk the MMA issuer runs: scores of the next chunk, then the readout
 // O^T = S^T (e^cum phiQ)^T, O^T += V^T Pt^T (hi and lo), and the state
 // update S^T += (w V)^T phiK.
@@ -468,9 +471,13 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         mbar_init(&X->p_full, 1);
         mbar_init(&X->epib_done, 1);
         mbar_init(&X->o_full, 1);
-        mbar_init(&X->o_empty, 8);      // one arrival per compute warp
+        mbar_init(&X->o_empty, 4);      // one arrival per output / state-pass warp
         mbar_init(&X->s_full, 1);
-        mbar_init(&X->sbf_ready, 4);    // one arrival per state-pass warp
+        mbar_init(&X->sbf_ready, 4);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&X->den_ready[s], 1);
+            mbar_init(&X->den_free[s], 4);
+        }
         X->abort = 0;
         mbar_fence_init();
     }
@@ -534,11 +541,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 const int s = it & 1;
                 const uint32_t par = it & 1;
                 if (!mbar_wait(&X->epib_done, par, abort_flag, err, KID_SCAN_TC_OUT, 4)) break;
+                // the next chunk's scores go first (P of this chunk has been
+                // read), so that the compute group's work on it overlaps this
+                // chunk's readout, state update and outputs
+                if (it + 1 < nch && !issue_scores(it + 1)) break;
                 if (!mbar_wait(&X->sbf_ready, par, abort_flag, err, KID_SCAN_TC_OUT, 5)) break;
                 if (!mbar_wait(&X->o_empty, par ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 6)) break;
-                // the next chunk's scores go first, so that the compute group's
-                // work on it overlaps this chunk's readout and state update
-                if (it + 1 < nch && !issue_scores(it + 1)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kF / 16; ++k) {
@@ -578,47 +586,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             *reinterpret_cast<uint4 *>(pb + kC * 128 + sw128_off(row, cc)) = make_uint4(0u, 0u, 0u, 0u);
             fence_proxy_async_smem();
         }
-        // outputs of chunk c (TMEM O^T: lane = value channel, column = token);
-        // warps 2..5 take tokens 0..31, warps 6..9 tokens 32..63
-        auto epilogue = [&](int c) -> bool {
-            bool okc = mbar_wait(&X->o_full, c & 1, abort_flag, err, KID_SCAN_TC_OUT, 9);
-            okc = __all_sync(0xffffffffu, okc);
-            const int th = warp >= 6 ? 1 : 0;
-            if (okc) {
-                tc_fence_after();
-                uint32_t r[32];
-                tmem_ld32(tmem + kColO + 32 * th + ((uint32_t)(32 * q) << 16), r);
-                tmem_wait_ld();
-                tc_fence_before();
-                const int ch = 32 * q + lane;
-                const int64_t t0 = (int64_t)(c_begin + c) * kC + 32 * th;
-                const int64_t obase = ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
-                const int64_t tstride = (int64_t)g.H * g.dv;
-                const float *rd = X->rden[c & 1] + 32 * th;
-                if (a.o_f32) {
-                    float *op = (float *)a.o + obase;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (t0 + i < g.L) op[i * tstride] = __uint_as_float(r[i]) * rd[i];
-                } else {
-                    __nv_bfloat16 *op = (__nv_bfloat16 *)a.o + obase;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (t0 + i < g.L) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]) * rd[i]);
-                }
-            }
-            // O^T may be overwritten from here on
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&X->o_empty);
-            return okc;
-        };
         // log a of the next chunk's tokens is fetched one chunk ahead
         float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, gt);
-        bool ok = named_sync_and(1, 256, true);
         // every exit from this loop is taken by the whole group (after a
-        // barrier-AND), so `it` is uniform when it ends
-        int it = 0;
-        for (; it < nch; ++it) {
+        // barrier-AND), so no thread is left waiting at a named barrier
+        bool ok = named_sync_and(1, 256, true);
+        for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
             // (1) decay of the chunk (warps 2, 3: thread = token): cum, e^cum,
             // weights e^(cum_last - cum), gamma
@@ -792,12 +765,18 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             ok = named_sync_and(1, 256, okw);
             if (!ok) break;
             if (gt == 0) mbar_arrive(&X->epib_done);
-            // (4) denominators and z (the chunk's MMAs run meanwhile)
+            // (4) denominators (once the outputs of chunk it - 2 have read this
+            // stage's 1 / den) and z; the chunk's MMAs run meanwhile
             if (gt < kC) {
                 const int i = gt;
+                const bool okd =
+                    mbar_wait(&X->den_free[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 14);
                 const float dq = (X->dotq[0][i] + X->dotq[1][i]) + (X->dotq[2][i] + X->dotq[3][i]);
                 const float den = X->dint[0][i] + (i >= 32 ? X->dint[1][i] : 0.f) + X->qs[s][i] * dq;
                 X->rden[s][i] = 1.f / den;
+                named_sync(3, 64);
+                if (gt == 0) mbar_arrive(&X->den_ready[s]);
+                if (!okd) ok = false;
             }
             {
                 float acc = 0.f;
@@ -805,12 +784,6 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 for (int tg = 0; tg < kZGroups; ++tg) acc += X->zred[tg][gt];
                 X->z[gt] = fmaf(X->gam[s], X->z[gt], acc);
             }
-            // (5) outputs of the previous chunk
-            if (it > 0 && !epilogue(it - 1)) ok = false;
-        }
-        if (it == nch && nch > 0) {
-            // 1 / den of the last chunk is complete
-            if (named_sync_and(1, 256, ok)) epilogue(nch - 1);
         }
     } else {
         // ------------------------------------------------------------ state pass
@@ -844,10 +817,65 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
         bool ok = true;
-        for (int it = 0; it + 1 < nch; ++it) {
-            const float gn = fexp(chunk_total(l_next, td, X->redd, 2));
-            if (it + 2 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 2) * kC, td);
-            ok = named_sync_and(2, 128, ok && mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11));
+        const int64_t tstride = (int64_t)g.H * g.dv;
+        for (int it = 0; it < nch; ++it) {
+            const int s = it & 1;
+            const bool more = it + 1 < nch;
+            float gn = 0.f;
+            if (more) {
+                gn = fexp(chunk_total(l_next, td, X->redd, 2));
+                if (it + 2 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 2) * kC, td);
+            }
+            // outputs of the chunk: o = O^T / den (lane = value channel, column = token)
+            bool okc = ok && mbar_wait(&X->o_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 9) &&
+                       mbar_wait(&X->den_ready[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 10);
+            okc = __all_sync(0xffffffffu, okc);
+            if (okc) {
+                tc_fence_after();
+                const float *rd = X->rden[s];
+#pragma unroll 1
+                for (int th = 0; th < 2; ++th) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + kColO + 32 * th + lanebase, r);
+                    tmem_wait_ld();
+                    const int64_t t0 = (int64_t)(c_begin + it) * kC + 32 * th;
+                    const int64_t obase = ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
+                    // every 1 / den is read before the first store, so that no
+                    // store waits on a shared-memory load behind it
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 d4 = *reinterpret_cast<const float4 *>(rd + 32 * th + 4 * i4);
+                        r[4 * i4 + 0] = __float_as_uint(__uint_as_float(r[4 * i4 + 0]) * d4.x);
+                        r[4 * i4 + 1] = __float_as_uint(__uint_as_float(r[4 * i4 + 1]) * d4.y);
+                        r[4 * i4 + 2] = __float_as_uint(__uint_as_float(r[4 * i4 + 2]) * d4.z);
+                        r[4 * i4 + 3] = __float_as_uint(__uint_as_float(r[4 * i4 + 3]) * d4.w);
+                    }
+                    const int nvalid = g.L - t0 < 32 ? (int)(g.L - t0) : 32;
+                    if (a.o_f32) {
+                        float *__restrict__ op = (float *)a.o + obase;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < nvalid) op[i * tstride] = __uint_as_float(r[i]);
+                    } else {
+                        __nv_bfloat16 *__restrict__ op = (__nv_bfloat16 *)a.o + obase;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < nvalid) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                    }
+                }
+            }
+            // O^T may be overwritten, and this stage's 1 / den rewritten, from here on
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&X->den_free[s]);
+                mbar_arrive(&X->o_empty);
+            }
+            if (!more) {
+                ok = ok && okc;
+                break;
+            }
+            ok = named_sync_and(2, 128, okc && mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11));
             if (!ok) break;
             tc_fence_after();
             // 32-column blocks, the next block's load in flight while this one

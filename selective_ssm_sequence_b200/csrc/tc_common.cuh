@@ -164,6 +164,14 @@ __device__ __forceinline__ bool named_sync_and(int id, int count, bool pred) {
     return r != 0;
 }
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32: a few ulp,
+// results below the normal range flushed to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Packed fp32 pair arithmetic (one instruction for two lanes of work).
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     uint64_t ra, rb, rc, rd;
