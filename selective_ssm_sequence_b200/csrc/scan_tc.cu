@@ -69,9 +69,11 @@ struct Geo {
 
 // ------------------------------------------------------------------ phase A
 
+constexpr int kABuild = 8;    // builder warps of the state kernel (8 tokens each)
+
 struct AAux {
     float w[2][kC];
-    alignas(16) float zred[4][kF];
+    alignas(16) float zred[kABuild][kF];
     float red[4];
     float suf;         // sum of log a over the chunks already processed (later ones)
     uint64_t full[2], empty[2], built, done;
@@ -85,7 +87,7 @@ constexpr int kASmem = kAOffAux + (int)sizeof(AAux) + 1024;
 // One CTA: (batch, head, value half, part).  Chunks of the part run from the
 // last to the first so that the suffix sums of log a (the weights relative to
 // the part end) are accumulated from small to large magnitudes.
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(64 + 32 * kABuild, 1)
 scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constant__ CUtensorMap tmkl,
                   const __grid_constant__ CUtensorMap tmv, Geo g, const float *__restrict__ dt,
                   const float *__restrict__ A_log, int split, int add_lo, float *__restrict__ S_part,
@@ -171,9 +173,11 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
             mma_commit(&X->done);
         }
     } else {
-        // builders: warps 2..5 (128 threads).  Thread: one 16-byte chunk (8
-        // features) of the 256-feature row (lane -> block, chunk) for the 16
+        // builders: warps 2..9 (256 threads).  Thread: one 16-byte chunk (8
+        // features) of the 256-feature row (lane -> block, chunk) for the 8
         // tokens of its warp's group.
+        constexpr int kNB = 32 * kABuild;
+        constexpr int kTok = kC / kABuild;
         const int tb = threadIdx.x - 64;
         const int bb = lane >> 3, cc = lane & 7;
         const int tg = tb >> 5;
@@ -181,15 +185,17 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
         float za[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) za[e] = 0.f;
-        auto token_l = [&](int t0) {
-            return (tb < kC && dt && t0 + tb < g.L) ? hm_log_decay(dt[(b * g.L + t0 + tb) * g.H + h], alog) : 0.f;
+        // dt is fetched a chunk ahead and turned into log a when used (-inf:
+        // log a = 0 past the end of the sequence or without dt)
+        auto token_dt = [&](int t0) {
+            return (tb < kC && dt && t0 + tb < g.L) ? dt[(b * g.L + t0 + tb) * g.H + h] : -INFINITY;
         };
-        float l_next = token_l(c_last * kC);
+        float dt_next = token_dt(c_last * kC);
         bool ok = true;
         for (int it = 0; it < n; ++it) {
             const int s = it & 1;
-            const float l = l_next;
-            if (it + 1 < n) l_next = token_l((c_last - it - 1) * kC);
+            const float l = hm_log_decay(dt_next, alog);
+            if (it + 1 < n) dt_next = token_dt((c_last - it - 1) * kC);
             // exclusive suffix sums of log a within the chunk
             float x = l;  // inclusive suffix sum within the warp
 #pragma unroll
@@ -198,7 +204,7 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
                 if (lane + o < 32) x += y;
             }
             if (tb == 32) X->red[0] = x;       // sum over tokens 32..63
-            named_sync(1, 128);
+            named_sync(1, kNB);
             if (tb < 32) x += X->red[0];
             // exclusive suffix: the inclusive value of the next token
             float ex = __shfl_down_sync(0xffffffffu, x, 1);
@@ -206,7 +212,7 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
             if (tb == 0) X->red[2] = x;        // chunk total
             const float suf = X->suf;
             if (tb < kC) X->w[s][tb] = fexp(suf + ex);
-            named_sync(1, 128);
+            named_sync(1, kNB);
             if (tb == 0) X->suf = suf + X->red[2];
             if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_STATE, 4)) {
                 ok = false;
@@ -218,7 +224,7 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
             uint8_t *__restrict__ kl = kh + kTileF;
             const float *__restrict__ wv = X->w[s];
 #pragma unroll 1
-            for (int j0 = tg * 16; j0 < tg * 16 + 16; j0 += 8) {
+            for (int j0 = tg * kTok; j0 < tg * kTok + kTok; j0 += 8) {
                 uint4 vh[8], vl[8];
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
@@ -260,21 +266,23 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
                 }
             }
             fence_proxy_async_smem();
-            named_sync(1, 128);
+            named_sync(1, kNB);
             if (tb == 0) mbar_arrive(&X->built);
         }
         // z of the part: reduce the four token groups' partial sums
         const int f0 = bb * 64 + cc * 8;
         *reinterpret_cast<float4 *>(&X->zred[tg][f0]) = make_float4(za[0], za[1], za[2], za[3]);
         *reinterpret_cast<float4 *>(&X->zred[tg][f0 + 4]) = make_float4(za[4], za[5], za[6], za[7]);
-        named_sync(1, 128);
+        named_sync(1, kNB);
         if (ok && mbar_wait(&X->done, 0, abort_flag, err, KID_SCAN_TC_STATE, 5)) {
             tc_fence_after();
+            // two warps per TMEM lane quarter: features 0..127 and 128..255
             const int q = warp & 3;
             const int ch = 32 * q + lane;
+            const int fh = (warp - 2) >> 2;
             const int64_t pidx = bh * g.NPc + part;
             float *Sp = S_part + pidx * (int64_t)kF * g.dv + dv0 + ch;
-            for (int c0 = 0; c0 < kF; c0 += 32) {
+            for (int c0 = fh * 128; c0 < fh * 128 + 128; c0 += 32) {
                 uint32_t r[32];
                 tmem_ld32(tmem + c0 + ((uint32_t)(32 * q) << 16), r);
                 tmem_wait_ld();
@@ -282,11 +290,10 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
                 for (int j = 0; j < 32; ++j) Sp[(int64_t)(c0 + j) * g.dv] = __uint_as_float(r[j]);
             }
             if (half == 0) {
+                float zs = 0.f;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int f = 2 * tb + e;
-                    z_part[pidx * kF + f] = X->zred[0][f] + X->zred[1][f] + X->zred[2][f] + X->zred[3][f];
-                }
+                for (int t = 0; t < kABuild; ++t) zs += X->zred[t][tb];
+                z_part[pidx * kF + tb] = zs;
                 if (tb == 0) lsum_part[pidx] = X->suf;
             }
         }
@@ -302,45 +309,55 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
 
 // ------------------------------------------------------------------ phase B
 
-// Per (batch, head) and state element: walks the parts in order,
+// Per (batch, head) and group of 4 state elements: walks the parts in order,
 //   acc <- exp(lsum_p) acc + part_p,
 // storing the state at each segment start and, when every part was
 // computed, the final state.  Elements [0, F*dv) are S, [F*dv, F*dv + F) are z.
-__global__ void scan_carry_kernel(Geo g, const float *__restrict__ S_part, const float *__restrict__ z_part,
-                                  const float *__restrict__ lsum_part, const float *__restrict__ S0,
-                                  const float *__restrict__ z0, float *__restrict__ S_start,
-                                  float *__restrict__ z_start, float *__restrict__ S_out,
-                                  float *__restrict__ z_out) {
+// The parts' values are loaded 8 at a time ahead of the dependent chain.
+__global__ void __launch_bounds__(256)
+scan_carry_kernel(Geo g, const float *__restrict__ S_part, const float *__restrict__ z_part,
+                  const float *__restrict__ lsum_part, const float *__restrict__ S0, const float *__restrict__ z0,
+                  float *__restrict__ S_start, float *__restrict__ z_start, float *__restrict__ S_out,
+                  float *__restrict__ z_out) {
     const int64_t bh = blockIdx.y;
     const int64_t nS = (int64_t)kF * g.dv;
-    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (e >= nS + kF) return;
     const bool isz = e >= nS;
     const int64_t idx = isz ? e - nS : e;
-    float acc = 0.f;
-    if (isz) {
-        if (z0) acc = z0[bh * kF + idx];
-    } else if (S0) {
-        acc = S0[bh * nS + idx];
-    }
+    const int64_t pstride = isz ? kF : nS;
+    const float *part = (isz ? z_part + bh * g.NPc * (int64_t)kF : S_part + bh * g.NPc * nS) + idx;
+    float *start = (isz ? z_start + bh * g.G * (int64_t)kF : S_start + bh * g.G * nS) + idx;
+    const float *init = isz ? (z0 ? z0 + bh * kF + idx : nullptr) : (S0 ? S0 + bh * nS + idx : nullptr);
+    float4 acc = init ? *reinterpret_cast<const float4 *>(init) : make_float4(0.f, 0.f, 0.f, 0.f);
     const int pps = g.seg_chunks / g.part_chunks;
-    for (int p = 0; p <= g.NPc; ++p) {
-        if (p > 0 && p % pps == 0 && p / pps < g.G) {
-            const int seg = p / pps;
-            if (isz) z_start[(bh * g.G + seg) * kF + idx] = acc;
-            else S_start[(bh * g.G + seg) * nS + idx] = acc;
+    for (int p0 = 0; p0 <= g.NPc; p0 += 8) {
+        float4 v[8];
+        float lg[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int p = p0 + u;
+            if (p < g.NPc) {
+                v[u] = *reinterpret_cast<const float4 *>(part + (int64_t)p * pstride);
+                lg[u] = lsum_part[bh * g.NPc + p];
+            }
         }
-        if (p == g.NPc) break;
-        const float gam = expf(lsum_part[bh * g.NPc + p]);
-        const float add = isz ? z_part[(bh * g.NPc + p) * kF + idx] : S_part[(bh * g.NPc + p) * nS + idx];
-        acc = fmaf(gam, acc, add);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int p = p0 + u;
+            if (p > g.NPc) break;
+            if (p > 0 && p % pps == 0 && p / pps < g.G)
+                *reinterpret_cast<float4 *>(start + (int64_t)(p / pps) * pstride) = acc;
+            if (p < g.NPc) {
+                const float gam = expf(lg[u]);
+                acc = make_float4(fmaf(gam, acc.x, v[u].x), fmaf(gam, acc.y, v[u].y), fmaf(gam, acc.z, v[u].z),
+                                  fmaf(gam, acc.w, v[u].w));
+            }
+        }
     }
     if (g.NPc == g.NP) {
-        if (isz) {
-            if (z_out) z_out[bh * kF + idx] = acc;
-        } else if (S_out) {
-            S_out[bh * nS + idx] = acc;
-        }
+        float *out = isz ? (z_out ? z_out + bh * kF + idx : nullptr) : (S_out ? S_out + bh * nS + idx : nullptr);
+        if (out) *reinterpret_cast<float4 *>(out) = acc;
     }
 }
 
@@ -350,10 +367,10 @@ __global__ void scan_carry_kernel(Geo g, const float *__restrict__ S_part, const
 constexpr uint32_t kColS = 0;    // S^T fp32        [128 value lanes x 256 features]
 constexpr uint32_t kColSB = 256; // S^T bf16 pairs  [128 x 128]
 constexpr uint32_t kColO = 384;  // O^T fp32        [128 x 64 tokens]
-constexpr uint32_t kColP = 448;  // [phiQ; phiK] phiK^T fp32 [128 x 64]; lanes 0..63 = P
+constexpr uint32_t kColP = 448;  // [phiK; phiQ] phiK^T fp32 [128 x 64]; lanes 64..127 = P
 
-constexpr int kZGroups = 5;      // token groups of the weighted key-feature sums (13 tokens)
-constexpr int kZTok = 13;
+constexpr int kZGroups = 8;      // token groups of the weighted key-feature sums (8 tokens)
+constexpr int kZTok = kC / kZGroups;
 constexpr int kHelpers = 160;    // threads of the five helper warps
 
 struct CAux {
@@ -368,19 +385,23 @@ struct CAux {
     float gam[2];
     float redb[4];
     float redd[4];
-    uint64_t full[2], empty[2];
-    uint64_t p_full, epib_done, o_full, o_empty, s_full, sbf_ready;
+    // per stage: the phiQ blocks and the phiK + V blocks are loaded and
+    // released separately
+    uint64_t fullq[2], fullkv[2], emptyq[2], emptykv[2];
+    uint64_t stg_free[2];   // the stage's Pt buffer, used to stage outputs, has been read out
+    uint64_t p_full, p_consumed, epib_done, o_full, o_empty, s_full, sbf_ready;
     uint64_t den_ready[2], den_free[2];   // 1 / den of a stage written / read
     uint32_t tmem;
     int abort;
 };
 
-// Phase C stage: for each 64-feature block bb, the 64 phiQ rows and the 64
-// phiK rows are stored back to back ([Q | K], 16 KB), so that one M = 128
-// operand [phiQ; phiK] gives the score tile P = phiQ phiK^T in TMEM lanes
-// 0..63 with the plain 128-lane accumulator layout (lanes 64..127 hold
-// phiK phiK^T, which is not used).
-constexpr int kQKBlk = 2 * kBlk;                       // [Q | K] of one feature block
+// Phase C stage: for each 64-feature block bb, the 64 phiK rows and the 64
+// phiQ rows are stored back to back ([K | Q], 16 KB), so that one M = 128
+// operand [phiK; phiQ] gives the score tile P = phiQ phiK^T in TMEM lanes
+// 64..127 with the plain 128-lane accumulator layout (lanes 0..63 hold
+// phiK phiK^T, which is not used).  Lanes 64..127 are read by warps 2, 3, 6,
+// 7, which share no SM sub-partition with the TMA and MMA warps.
+constexpr int kQKBlk = 2 * kBlk;                       // [K | Q] of one feature block
 constexpr int kCStage = 4 * kQKBlk + kTileV;           // Q, K, V of one chunk
 constexpr int kCPBytes = 2 * kC * 128;                 // Pt as bf16 hi (8 KB) then lo (8 KB)
 constexpr int kCOffP = 2 * kCStage;                    // one Pt buffer per stage
@@ -398,11 +419,13 @@ struct OutArgs {
     const float *S_start, *z_start;  // segments >= 1: [BH][G][F*dv], [BH][G][F]
 };
 
-// log a of token t0 + tg for the first 64 threads of a group (0 otherwise)
-__device__ __forceinline__ float token_log_decay(const OutArgs &a, int64_t b, int h, float alog,
-                                                 int64_t t0, int tg) {
-    if (tg < kC && a.dt && t0 + tg < a.g.L) return hm_log_decay(a.dt[(b * a.g.L + t0 + tg) * a.g.H + h], alog);
-    return 0.f;
+// dt of token t0 + tg for the first 64 threads of a group; -inf (log a = 0)
+// past the end of the sequence, for the other threads, or without dt.  The
+// raw value is fetched a chunk ahead and turned into log a when it is used,
+// so the load's latency is never waited for.
+__device__ __forceinline__ float token_dt(const OutArgs &a, int64_t b, int h, int64_t t0, int tg) {
+    if (tg < kC && a.dt && t0 + tg < a.g.L) return a.dt[(b * a.g.L + t0 + tg) * a.g.H + h];
+    return -INFINITY;
 }
 
 // sum of the 64 per-token values l over the first two warps of a 128-thread
@@ -424,15 +447,17 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
 //          only columns 0..31), w (.) V, the weighted key-feature sums for z,
 //          the scaled queries e^cum (.) phiQ with phiq . z_prev, the
 //          denominators and z
-//   10..13 outputs and state pass: o = O^T / den for the chunk, then S^T
-//          (fp32, TMEM) -> bf16 copy for the next readout and
-//          S^T <- gamma S^T before the next state MMA
+//   10..13 outputs and state pass: o = O^T / den for the chunk, staged in the
+//          chunk's Pt buffer (dead once the PV product is complete) and written
+//          by TMA bulk stores; then S^T (fp32, TMEM) -> bf16 copy for the next
+//          readout and S^T <- gamma S^T before the next state MMA
 // Per chunk the MMA issuer runs: scores of the next chunk, then the readout
 // O^T = S^T (e^cum phiQ)^T, O^T += V^T Pt^T (hi and lo), and the state
 // update S^T += (w V)^T phiK.
 __global__ void __launch_bounds__(448, 1)
 scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                const __grid_constant__ CUtensorMap tmv, OutArgs a, DevErr err) {
+                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo, OutArgs a,
+                DevErr err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
     CAux *X = (CAux *)(smem + kCOffAux);
@@ -450,25 +475,30 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     const float alog = a.dt ? a.A_log[h] : 0.f;
     volatile int *abort_flag = &X->abort;
     const uint32_t sbase = smem_u32(smem);
-    // block bb of phiQ at sQ(s) + bb * kQKBlk, of phiK at sK(s) + bb * kQKBlk
-    auto sQ = [&](int s) { return sbase + s * kCStage; };
-    auto sK = [&](int s) { return sbase + s * kCStage + kBlk; };
+    // block bb of phiK at sK(s) + bb * kQKBlk, of phiQ at sQ(s) + bb * kQKBlk
+    auto sQ = [&](int s) { return sbase + s * kCStage + kBlk; };
+    auto sK = [&](int s) { return sbase + s * kCStage; };
     auto sV = [&](int s) { return sbase + s * kCStage + 4 * kQKBlk; };
     auto sP = [&](int s) { return sbase + kCOffP + s * kCPBytes; };
     const uint32_t sVt = sbase + kCOffVt;
     // pointers to the same buffers, for CUDA-core accesses
-    auto gQ = [&](int s) { return smem + s * kCStage; };
-    auto gK = [&](int s) { return smem + s * kCStage + kBlk; };
+    auto gQ = [&](int s) { return smem + s * kCStage + kBlk; };
+    auto gK = [&](int s) { return smem + s * kCStage; };
     auto gV = [&](int s) { return smem + s * kCStage + 4 * kQKBlk; };
     auto gP = [&](int s) { return smem + kCOffP + s * kCPBytes; };
     uint8_t *const gVt = smem + kCOffVt;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&X->full[s], 1);
-            mbar_init(&X->empty[s], 1);
+            mbar_init(&X->fullq[s], 1);
+            mbar_init(&X->fullkv[s], 1);
+            mbar_init(&X->emptyq[s], 1);
+            mbar_init(&X->stg_free[s], 1);
+            // phiK + V: the chunk's MMAs and the compute group's key-feature sums
+            mbar_init(&X->emptykv[s], 2);
         }
         mbar_init(&X->p_full, 1);
+        mbar_init(&X->p_consumed, 1);   // the compute group has loaded P
         mbar_init(&X->epib_done, 1);
         mbar_init(&X->o_full, 1);
         mbar_init(&X->o_empty, 4);      // one arrival per output / state-pass warp
@@ -493,44 +523,55 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             tma_prefetch_desc(&tmq);
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
-            int it = 0;
-            for (; it < nch; ++it) {
+            int nkv = 0, nq = 0;   // chunks whose phiK + V / phiQ loads were issued
+            for (int it = 0; it < nch; ++it) {
                 const int s = it & 1;
-                if (!mbar_wait(&X->empty[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 1)) break;
+                const uint32_t par = ((it >> 1) & 1) ^ 1;
                 const int t0 = (c_begin + it) * kC;
-                mbar_arrive_expect_tx(&X->full[s], kCStage);
                 uint8_t *q = smem + s * kCStage;
-                for (int bb = 0; bb < 4; ++bb) {
-                    tma_load_4d(q + bb * kQKBlk, &tmq, &X->full[s], bb * 64, h, t0, (int)b);
-                    tma_load_4d(q + bb * kQKBlk + kBlk, &tmk, &X->full[s], bb * 64, h, t0, (int)b);
-                }
+                if (!mbar_wait(&X->emptykv[s], par, abort_flag, err, KID_SCAN_TC_OUT, 1)) break;
+                mbar_arrive_expect_tx(&X->fullkv[s], 4 * kBlk + kTileV);
+                for (int bb = 0; bb < 4; ++bb)
+                    tma_load_4d(q + bb * kQKBlk, &tmk, &X->fullkv[s], bb * 64, h, t0, (int)b);
                 for (int bb = 0; bb < 2; ++bb)
-                    tma_load_4d(q + 4 * kQKBlk + bb * kBlk, &tmv, &X->full[s], dv0 + bb * 64, h, t0, (int)b);
+                    tma_load_4d(q + 4 * kQKBlk + bb * kBlk, &tmv, &X->fullkv[s], dv0 + bb * 64, h, t0, (int)b);
+                ++nkv;
+                if (!mbar_wait(&X->emptyq[s], par, abort_flag, err, KID_SCAN_TC_OUT, 15)) break;
+                mbar_arrive_expect_tx(&X->fullq[s], 4 * kBlk);
+                for (int bb = 0; bb < 4; ++bb)
+                    tma_load_4d(q + bb * kQKBlk + kBlk, &tmq, &X->fullq[s], bb * 64, h, t0, (int)b);
+                ++nq;
             }
-            for (int j = it - 2; j < it; ++j) {
+            // no copy may still be landing when the CTA exits
+            for (int j = nkv - 2; j < nkv; ++j) {
                 if (j < 0) continue;
                 for (uint32_t i = 0; i < kWaitPolls; ++i)
-                    if (mbar_try_wait(&X->full[j & 1], (j >> 1) & 1)) break;
+                    if (mbar_try_wait(&X->fullkv[j & 1], (j >> 1) & 1)) break;
+            }
+            for (int j = nq - 2; j < nq; ++j) {
+                if (j < 0) continue;
+                for (uint32_t i = 0; i < kWaitPolls; ++i)
+                    if (mbar_try_wait(&X->fullq[j & 1], (j >> 1) & 1)) break;
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (elect_one()) {
-            constexpr uint32_t idP = idesc_bf16(128, 64, false, false);    // [phiQ; phiK] phiK^T
+            constexpr uint32_t idP = idesc_bf16(128, 64, false, false);    // [phiK; phiQ] phiK^T
             constexpr uint32_t idOi = idesc_bf16(128, 64, false, false);   // O^T = S^T phiQ~^T
             constexpr uint32_t idOa = idesc_bf16(128, 64, true, false);    // O^T += V^T Pt^T
             constexpr uint32_t idS = idesc_bf16(128, 256, true, true);     // S^T += (wV)^T phiK
-            // score MMA of chunk c: P = [phiQ; phiK] phiK^T into the P columns
-            // (the compute group has read P of chunk c - 1: its epib_done is
-            // complete whenever this runs)
+            // score MMA of chunk c: [phiK; phiQ] phiK^T into the P columns,
+            // once the compute group has loaded P of chunk c - 1
             auto issue_scores = [&](int c) -> bool {
                 const int sc = c & 1;
-                if (!mbar_wait(&X->full[sc], (c >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 2)) return false;
+                if (!mbar_wait(&X->fullkv[sc], (c >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 2)) return false;
+                if (!mbar_wait(&X->fullq[sc], (c >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 16)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < kF / 16; ++k) {
                     const uint32_t off = (k >> 2) * kQKBlk + (k & 3) * 32;
-                    mma_ss(tmem + kColP, desc_k_sw128(sQ(sc) + off), desc_k_sw128(sK(sc) + off), idP,
+                    mma_ss(tmem + kColP, desc_k_sw128(sK(sc) + off), desc_k_sw128(sK(sc) + off), idP,
                            k > 0 ? 1u : 0u);
                 }
                 mma_commit(&X->p_full);
@@ -540,11 +581,14 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int it = 0; ok && it < nch; ++it) {
                 const int s = it & 1;
                 const uint32_t par = it & 1;
+                // the next chunk's scores go as soon as this chunk's P has been
+                // loaded into registers, so that they run under the compute
+                // group's work on this chunk
+                if (it + 1 < nch) {
+                    if (!mbar_wait(&X->p_consumed, par, abort_flag, err, KID_SCAN_TC_OUT, 3)) break;
+                    if (!issue_scores(it + 1)) break;
+                }
                 if (!mbar_wait(&X->epib_done, par, abort_flag, err, KID_SCAN_TC_OUT, 4)) break;
-                // the next chunk's scores go first (P of this chunk has been
-                // read), so that the compute group's work on it overlaps this
-                // chunk's readout, state update and outputs
-                if (it + 1 < nch && !issue_scores(it + 1)) break;
                 if (!mbar_wait(&X->sbf_ready, par, abort_flag, err, KID_SCAN_TC_OUT, 5)) break;
                 if (!mbar_wait(&X->o_empty, par ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 6)) break;
                 tc_fence_after();
@@ -566,7 +610,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     mma_ss(tmem + kColS, desc_mn_sw128(sVt + k * 2048, kBlk, 1024),
                            desc_mn_sw128(sK(s) + k * 2048, kQKBlk, 1024), idS, 1u);
                 mma_commit(&X->s_full);
-                mma_commit(&X->empty[s]);
+                mma_commit(&X->emptykv[s]);
+                mma_commit(&X->emptyq[s]);
             }
         }
     } else if (warp < 10) {
@@ -578,16 +623,9 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (seg == 0) zi = a.z0 ? a.z0 + bh * kF : nullptr;
             else zi = a.z_start + (bh * g.G + seg) * kF;
             X->z[gt] = zi ? zi[gt] : 0.f;
-            // rows 0..31 x columns 32..63 of Pt (hi and lo, both buffers) are
-            // always zero: written once here
-            const int row = gt & 31, cc = 4 + ((gt >> 5) & 3);
-            uint8_t *pb = gP(gt >> 7);
-            *reinterpret_cast<uint4 *>(pb + sw128_off(row, cc)) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(pb + kC * 128 + sw128_off(row, cc)) = make_uint4(0u, 0u, 0u, 0u);
-            fence_proxy_async_smem();
         }
-        // log a of the next chunk's tokens is fetched one chunk ahead
-        float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, gt);
+        // dt of the next chunk's tokens is fetched one chunk ahead
+        float dt_next = token_dt(a, b, h, (int64_t)c_begin * kC, gt);
         // every exit from this loop is taken by the whole group (after a
         // barrier-AND), so no thread is left waiting at a named barrier
         bool ok = named_sync_and(1, 256, true);
@@ -596,8 +634,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             // (1) decay of the chunk (warps 2, 3: thread = token): cum, e^cum,
             // weights e^(cum_last - cum), gamma
             if (gt < kC) {
-                const float l = l_next;
-                if (it + 1 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 1) * kC, gt);
+                const float l = hm_log_decay(dt_next, alog);
+                if (it + 1 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + it + 1) * kC, gt);
                 float x = l;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -619,23 +657,36 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (!ok) break;
             // (2) once the chunk's scores are in TMEM
             bool okw = mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7) &&
-                       mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8);
+                       mbar_wait(&X->fullkv[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8) &&
+                       mbar_wait(&X->fullq[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 17);
             okw = __all_sync(0xffffffffu, okw);
             tc_fence_after();
-            if (warp == 4 || warp == 5 || warp == 9) {
+            const bool pwarp = warp == 2 || warp == 3 || warp == 7;
+            // score-quadrant warps (P rows 0..31 in TMEM lanes 64..95, rows
+            // 32..63 in lanes 96..127): warp 2: rows 0..31 x columns 0..31 (and
+            // the zeros of columns 32..63); warp 3: rows 32..63 x columns 0..31
+            // (all below the diagonal); warp 7: rows 32..63 x columns 32..63
+            const int i = 32 * (q - 2) + lane;
+            const int jc = warp == 7 ? 32 : 0;
+            uint32_t pr[32];
+            if (pwarp && okw) {
+                tmem_ld32(tmem + kColP + jc + ((uint32_t)(32 * q) << 16), pr);
+                tmem_wait_ld();
+            }
+            // every compute thread is past its wait on this chunk's scores and P
+            // is in registers: the next chunk's scores may overwrite it
+            tc_fence_before();
+            named_sync(4, 256);
+            if (gt == 0) mbar_arrive(&X->p_consumed);
+            if (pwarp) {
                 // Pt = P * exp(cum_i - cum_j) on j <= i, as bf16 hi + lo (the PV
                 // product runs on both: a few-token weighted average would
-                // otherwise carry the 2^-9 rounding of each weight), and row sums.
-                // warp 4: rows 0..31 x columns 0..31; warp 5: rows 32..63 x
-                // columns 0..31 (all below the diagonal); warp 9: rows 32..63 x
-                // columns 32..63.
-                const int i = 32 * q + lane;
-                const int jc = warp == 9 ? 32 : 0;
-                const bool masked = warp != 5;
+                // otherwise carry the 2^-9 rounding of each weight), and row sums
+                const bool masked = warp != 3;
+                // the buffer staged chunk it - 2's outputs
+                okw = __all_sync(0xffffffffu, okw && mbar_wait(&X->stg_free[s], ((it >> 1) & 1) ^ 1, abort_flag,
+                                                                   err, KID_SCAN_TC_OUT, 18));
                 if (okw) {
-                    uint32_t pr[32];
-                    tmem_ld32(tmem + kColP + jc + ((uint32_t)(32 * q) << 16), pr);
-                    tmem_wait_ld();
                     const float ci = X->cum[s][i];
                     const float *__restrict__ cj = X->cum[s] + jc;
                     uint8_t *__restrict__ prow = gP(s);
@@ -663,40 +714,20 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         const int cc = (jc >> 3) + c4;
                         *reinterpret_cast<uint4 *>(prow + sw128_off(i, cc)) = hi;
                         *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, cc)) = lo;
+                        if (warp == 2) {
+                            // rows 0..31 x columns 32..63 are zero
+                            *reinterpret_cast<uint4 *>(prow + sw128_off(i, 4 + c4)) = make_uint4(0u, 0u, 0u, 0u);
+                            *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, 4 + c4)) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
                     }
                     X->dint[jc ? 1 : 0][i] = rs;
                     tc_fence_before();
                 }
             } else {
-                // helpers (warps 2, 3, 6, 7, 8)
-                const int hx = (warp < 4 ? warp - 2 : warp - 4) * 32 + lane;   // 0..159
+                // helpers (warps 4, 5, 6, 8, 9)
+                const int hx = (warp < 7 ? warp - 4 : warp - 5) * 32 + lane;   // 0..159
                 const float *__restrict__ wv = X->w[s];
-                // weighted key-feature sums sum_j w_j phik_j: thread = one
-                // 16-byte chunk (8 features) over a group of 13 tokens
-                {
-                    const int cc = hx & 31, tg = hx >> 5;
-                    const uint8_t *__restrict__ base = gK(s) + (cc >> 3) * kQKBlk;
-                    const int j0 = tg * kZTok;
-                    uint4 kv[kZTok];
-#pragma unroll
-                    for (int jj = 0; jj < kZTok; ++jj)
-                        kv[jj] = (j0 + jj < kC) ? *reinterpret_cast<const uint4 *>(base + sw128_off(j0 + jj, cc & 7))
-                                                : make_uint4(0u, 0u, 0u, 0u);
-                    float2 za[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) za[e] = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int jj = 0; jj < kZTok; ++jj) {
-                        const float wj = (j0 + jj < kC) ? wv[j0 + jj] : 0.f;
-                        const float2 w2 = make_float2(wj, wj);
-                        const uint32_t *pv = reinterpret_cast<const uint32_t *>(&kv[jj]);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) za[e] = fma2(unpack_bf16x2(pv[e]), w2, za[e]);
-                    }
-                    float *zr = &X->zred[tg][cc * 8];
-                    *reinterpret_cast<float4 *>(zr) = make_float4(za[0].x, za[0].y, za[1].x, za[1].y);
-                    *reinterpret_cast<float4 *>(zr + 4) = make_float4(za[2].x, za[2].y, za[3].x, za[3].y);
-                }
                 // w (.) V into its own tile, once the previous chunk's state MMA
                 // has read that tile
                 if (it > 0) okw = mbar_wait(&X->s_full, (it - 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 13) && okw;
@@ -738,27 +769,30 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 const float2 q2 = make_float2(qsi, qsi);
                 uint8_t *__restrict__ qb = gQ(s) + qf * kQKBlk;
                 const float *__restrict__ zq = X->z + qf * 64;
-                uint4 v[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const uint4 *>(qb + sw128_off(i, k));
                 float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll 1
+                for (int k0 = 0; k0 < 8; k0 += 4) {
+                    uint4 v[4];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    uint32_t *pv = reinterpret_cast<uint32_t *>(&v[k]);
-                    const float4 za = *reinterpret_cast<const float4 *>(zq + k * 8);
-                    const float4 zb = *reinterpret_cast<const float4 *>(zq + k * 8 + 4);
-                    const float2 zz[4] = {make_float2(za.x, za.y), make_float2(za.z, za.w), make_float2(zb.x, zb.y),
-                                          make_float2(zb.z, zb.w)};
+                    for (int k = 0; k < 4; ++k) v[k] = *reinterpret_cast<const uint4 *>(qb + sw128_off(i, k0 + k));
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 x = unpack_bf16x2(pv[e]);
-                        d2 = fma2(x, zz[e], d2);
-                        const float2 y = mul2(x, q2);
-                        pv[e] = pack_bf16x2(y.x, y.y);
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t *pv = reinterpret_cast<uint32_t *>(&v[k]);
+                        const float4 za = *reinterpret_cast<const float4 *>(zq + (k0 + k) * 8);
+                        const float4 zb = *reinterpret_cast<const float4 *>(zq + (k0 + k) * 8 + 4);
+                        const float2 zz[4] = {make_float2(za.x, za.y), make_float2(za.z, za.w),
+                                              make_float2(zb.x, zb.y), make_float2(zb.z, zb.w)};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = unpack_bf16x2(pv[e]);
+                            d2 = fma2(x, zz[e], d2);
+                            const float2 y = mul2(x, q2);
+                            pv[e] = pack_bf16x2(y.x, y.y);
+                        }
                     }
-                }
 #pragma unroll
-                for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4 *>(qb + sw128_off(i, k)) = v[k];
+                    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4 *>(qb + sw128_off(i, k0 + k)) = v[k];
+                }
                 X->dotq[qf][i] = d2.x + d2.y;
             }
             fence_proxy_async_smem();
@@ -778,6 +812,34 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (gt == 0) mbar_arrive(&X->den_ready[s]);
                 if (!okd) ok = false;
             }
+            // (5) weighted key-feature sums sum_j w_j phik_j (needed only for the
+            // next chunk's denominators, so after the MMAs were released):
+            // thread = one 16-byte chunk (8 features) over a group of 8 tokens
+            {
+                const int cc = gt & 31, tg = gt >> 5;
+                const uint8_t *__restrict__ base = gK(s) + (cc >> 3) * kQKBlk;
+                const float *__restrict__ wv = X->w[s] + tg * kZTok;
+                uint4 kv[kZTok];
+#pragma unroll
+                for (int jj = 0; jj < kZTok; ++jj)
+                    kv[jj] = *reinterpret_cast<const uint4 *>(base + sw128_off(tg * kZTok + jj, cc & 7));
+                float2 za[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) za[e] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int jj = 0; jj < kZTok; ++jj) {
+                    const float2 w2 = make_float2(wv[jj], wv[jj]);
+                    const uint32_t *pv = reinterpret_cast<const uint32_t *>(&kv[jj]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) za[e] = fma2(unpack_bf16x2(pv[e]), w2, za[e]);
+                }
+                float *zr = &X->zred[tg][cc * 8];
+                *reinterpret_cast<float4 *>(zr) = make_float4(za[0].x, za[0].y, za[1].x, za[1].y);
+                *reinterpret_cast<float4 *>(zr + 4) = make_float4(za[2].x, za[2].y, za[3].x, za[3].y);
+            }
+            named_sync(1, 256);
+            if (gt == 0) mbar_arrive(&X->emptykv[s]);   // phiK and V of the stage have been read
+            // (6) z <- gamma z + sum_j w_j phik_j
             {
                 float acc = 0.f;
 #pragma unroll
@@ -792,10 +854,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         const int ch = 32 * q + lane;
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
         // prologue: start state -> bf16 copy (for the first readout) and fp32 x gamma_0
-        float l_next = token_log_decay(a, b, h, alog, (int64_t)c_begin * kC, td);
+        float dt_next = token_dt(a, b, h, (int64_t)c_begin * kC, td);
         {
-            const float gam0 = fexp(chunk_total(l_next, td, X->redd, 2));
-            if (nch > 1) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + 1) * kC, td);
+            const float gam0 = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 2));
+            if (nch > 1) dt_next = token_dt(a, b, h, (int64_t)(c_begin + 1) * kC, td);
             const float *src = nullptr;
             if (seg == 0) src = a.S0 ? a.S0 + bh * (int64_t)kF * g.dv : nullptr;
             else src = a.S_start + (bh * g.G + seg) * (int64_t)kF * g.dv;
@@ -817,31 +879,34 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
         bool ok = true;
-        const int64_t tstride = (int64_t)g.H * g.dv;
         for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
             const bool more = it + 1 < nch;
             float gn = 0.f;
             if (more) {
-                gn = fexp(chunk_total(l_next, td, X->redd, 2));
-                if (it + 2 < nch) l_next = token_log_decay(a, b, h, alog, (int64_t)(c_begin + it + 2) * kC, td);
+                gn = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 2));
+                if (it + 2 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + it + 2) * kC, td);
             }
             // outputs of the chunk: o = O^T / den (lane = value channel, column = token)
             bool okc = ok && mbar_wait(&X->o_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 9) &&
                        mbar_wait(&X->den_ready[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 10);
             okc = __all_sync(0xffffffffu, okc);
-            if (okc) {
-                tc_fence_after();
-                const float *rd = X->rden[s];
+            // staging in the chunk's Pt buffer (16 KB), in two rounds of 32
+            // tokens: box cb = channels 64 cb.. of the CTA's value half, rows of
+            // 64 channels, no swizzle.  bf16 boxes are 4 KB (round th at 8 KB
+            // th); fp32 boxes 8 KB, both rounds at offset 0 (round 1 waits
+            // until round 0 has been read out).
+            uint8_t *const stg = gP(s);
+            const int cb = ch >> 6, cl = ch & 63;
+            const float *rd = X->rden[s];
+            const int t0c = (c_begin + it) * kC;
 #pragma unroll 1
-                for (int th = 0; th < 2; ++th) {
+            for (int th = 0; th < 2; ++th) {
+                if (okc) {
+                    tc_fence_after();
                     uint32_t r[32];
                     tmem_ld32(tmem + kColO + 32 * th + lanebase, r);
                     tmem_wait_ld();
-                    const int64_t t0 = (int64_t)(c_begin + it) * kC + 32 * th;
-                    const int64_t obase = ((b * g.L + t0) * g.H + h) * (int64_t)g.dv + dv0 + ch;
-                    // every 1 / den is read before the first store, so that no
-                    // store waits on a shared-memory load behind it
 #pragma unroll
                     for (int i4 = 0; i4 < 8; ++i4) {
                         const float4 d4 = *reinterpret_cast<const float4 *>(rd + 32 * th + 4 * i4);
@@ -850,27 +915,38 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         r[4 * i4 + 2] = __float_as_uint(__uint_as_float(r[4 * i4 + 2]) * d4.z);
                         r[4 * i4 + 3] = __float_as_uint(__uint_as_float(r[4 * i4 + 3]) * d4.w);
                     }
-                    const int nvalid = g.L - t0 < 32 ? (int)(g.L - t0) : 32;
                     if (a.o_f32) {
-                        float *__restrict__ op = (float *)a.o + obase;
+                        float *box = reinterpret_cast<float *>(stg + cb * 8192) + cl;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i < nvalid) op[i * tstride] = __uint_as_float(r[i]);
+                        for (int i = 0; i < 32; ++i) box[i * 64] = __uint_as_float(r[i]);
                     } else {
-                        __nv_bfloat16 *__restrict__ op = (__nv_bfloat16 *)a.o + obase;
+                        __nv_bfloat16 *box = reinterpret_cast<__nv_bfloat16 *>(stg + th * 8192 + cb * 4096) + cl;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i < nvalid) op[i * tstride] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                        for (int i = 0; i < 32; ++i) box[i * 64] = __float2bfloat16_rn(__uint_as_float(r[i]));
                     }
                 }
+                if (th == 1) {
+                    // O^T may be overwritten, and this stage's 1 / den rewritten
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&X->den_free[s]);
+                        mbar_arrive(&X->o_empty);
+                    }
+                }
+                fence_proxy_async_smem();
+                okc = named_sync_and(2, 128, okc);
+                if (td == 0 && okc && t0c + 32 * th < g.L) {
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        const uint8_t *src = a.o_f32 ? stg + c2 * 8192 : stg + th * 8192 + c2 * 4096;
+                        tma_store_4d(&tmo, src, dv0 + 64 * c2, h, t0c + 32 * th, (int)b);
+                    }
+                    bulk_commit();
+                    if (a.o_f32 || th == 1) bulk_wait_read_all();
+                }
+                if (a.o_f32 && th == 0) named_sync(2, 128);   // round 0 has been read out
             }
-            // O^T may be overwritten, and this stage's 1 / den rewritten, from here on
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&X->den_free[s]);
-                mbar_arrive(&X->o_empty);
-            }
+            if (td == 0) mbar_arrive(&X->stg_free[s]);   // the Pt buffer may be rewritten
             if (!more) {
                 ok = ok && okc;
                 break;
@@ -902,8 +978,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
-        // the MMAs of the last chunk must be complete before TMEM is released
+        // the MMAs of the last chunk must be complete before TMEM is released,
+        // and the output stores before the CTA's shared memory goes away
         if (ok && nch > 0) mbar_wait(&X->s_full, (nch - 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 12);
+        if (td == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -1036,11 +1114,11 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
         e = ensure_smem_limit(scan_state_kernel, kASmem);
         if (e != cudaSuccess) return e;
         const unsigned grid = (unsigned)(2 * g.NPc * BH);
-        scan_state_kernel<<<grid, 192, kASmem, s>>>(tk, tkl, tv, g, c.dt, c.A_log, split ? 1 : 0,
+        scan_state_kernel<<<grid, 64 + 32 * kABuild, kASmem, s>>>(tk, tkl, tv, g, c.dt, c.A_log, split ? 1 : 0,
                                                     add_lo ? 1 : 0, S_part, z_part, lsum, err);
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        dim3 gb((unsigned)((nS + kF + 255) / 256), (unsigned)BH);
+        dim3 gb((unsigned)(((nS + kF) / 4 + 255) / 256), (unsigned)BH);
         scan_carry_kernel<<<gb, 256, 0, s>>>(g, S_part, z_part, lsum, c.S0, c.z0, S_start, z_start,
                                              c.S_out, c.z_out);
         count_launches(1);
@@ -1056,9 +1134,20 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
     oa.z0 = c.z0;
     oa.S_start = S_start;
     oa.z_start = z_start;
+    // output tiles: boxes of 64 channels x 32 tokens, stored from unswizzled staging rows
+    CUtensorMap to;
+    {
+        const uint64_t es = c.o_f32 ? 4 : 2;
+        uint64_t dims[4] = {(uint64_t)c.dv, (uint64_t)c.H, (uint64_t)c.L, (uint64_t)c.B};
+        uint64_t strides[3] = {(uint64_t)c.dv * es, (uint64_t)c.H * c.dv * es, (uint64_t)c.L * c.H * c.dv * es};
+        uint32_t box[4] = {64, 1, 32, 1};
+        if (!make_tmap(&to, c.o_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.o, 4,
+                       dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
     e = ensure_smem_limit(scan_out_kernel, kCSmem);
     if (e != cudaSuccess) return e;
-    scan_out_kernel<<<(unsigned)(2 * g.G * BH), 448, kCSmem, s>>>(tq, tk, tv, oa, err);
+    scan_out_kernel<<<(unsigned)(2 * g.G * BH), 448, kCSmem, s>>>(tq, tk, tv, to, oa, err);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -142,6 +142,25 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Tiled TMA store of a shared-memory box to global memory (bulk async group
+// of the issuing thread).  Coordinates must be >= 0 with x * element size a
+// multiple of 16 bytes; rows outside the tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            (uint64_t)map),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the issuing thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// the issuing thread's bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Named barrier over `count` threads (a warpgroup-sized subset of the CTA).
 __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -366,6 +385,11 @@ cudaError_t ensure_smem_limit(Kern kern, int bytes) {
 // dims 1..rank-1) with 128-byte swizzle.  Returns false on failure.
 bool make_tmap_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                     const uint64_t *strides_bytes, const uint32_t *box);
+
+// Same, for any element type and swizzle mode.
+bool make_tmap(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, int rank,
+               const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+               CUtensorMapSwizzle swizzle);
 
 }  // namespace tc
 }  // namespace hm

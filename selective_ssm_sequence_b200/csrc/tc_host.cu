@@ -27,6 +27,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool make_tmap_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                     const uint64_t *strides_bytes, const uint32_t *box) {
+    return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool make_tmap(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, int rank,
+               const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+               CUtensorMapSwizzle swizzle) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t gdim[5];
@@ -38,9 +45,8 @@ bool make_tmap_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t
         estride[i] = 1;
     }
     for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_bytes[i];
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base),
-                    gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstride, bdim, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
