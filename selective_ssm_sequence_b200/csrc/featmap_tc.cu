@@ -12,7 +12,10 @@
 //   warps 2..9  two epilogue warpgroups taking alternate tiles: one
 //               accumulator row per thread, read from TMEM in two passes (a
 //               running max / normaliser, then the normalised features), the
-//               negate / concatenate / softmax in registers, and the store.
+//               negate / concatenate / softmax in registers.  bf16 features
+//               are staged per warp (boxes of 32 rows x 32 features, two 2 KB
+//               buffers used in turn) and written by TMA bulk stores; fp32
+//               features and the bf16 remainder plane are stored directly.
 // Four TMEM accumulators let the MMAs run ahead of both epilogue warpgroups.
 // The kernel is bound by HBM (x in, phi out); MMA and exp work hide under it.
 #include "tc_common.cuh"
@@ -36,7 +39,9 @@ struct FmLayout {
     static constexpr int kXBytes = kChunks * kXChunkBytes;  // one x tile
     static constexpr int kOffW = 0;
     static constexpr int kOffX = kWBytes;
-    static constexpr int kOffBar = kOffX + kStages * kXBytes;
+    static constexpr int kOffStg = kOffX + kStages * kXBytes;     // 8 warps x 2 x 2 KB staging
+    static constexpr int kStgBytes = 8 * 2 * 2048;
+    static constexpr int kOffBar = kOffStg + kStgBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;      // + barriers, + alignment slack
     static constexpr int kAcc = 512 / P >= 4 ? 4 : 2;       // TMEM accumulators
     static constexpr int kTmemCols = kAcc * P <= 256 ? 256 : 512;
@@ -57,8 +62,8 @@ __device__ __forceinline__ float fexp(float x) { return exp2f(x * 1.442695040888
 template <int D, int P, typename TP>
 __global__ void __launch_bounds__(kThreads, 1)
 featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-                  int64_t Tv, int Hv, const float *__restrict__ bias, int bias_per_head,
-                  TP *__restrict__ phi, __nv_bfloat16 *__restrict__ phi_lo, DevErr err) {
+                  const __grid_constant__ CUtensorMap tmo, int64_t Tv, int Hv, const float *__restrict__ bias,
+                  int bias_per_head, TP *__restrict__ phi, __nv_bfloat16 *__restrict__ phi_lo, DevErr err) {
     using Lay = FmLayout<D, P>;
     constexpr int NA = Lay::kAcc;
     extern __shared__ uint8_t smem_raw[];
@@ -157,6 +162,10 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
         const int row_in_tile = q * 32 + lane;
         constexpr int F = 2 * P;
         const float *bh = bias ? bias + (bias_per_head ? (int64_t)h * P : 0) : nullptr;
+        // bf16 features without a remainder plane leave through TMA stores
+        const bool via_tma = sizeof(TP) == 2 && phi_lo == nullptr;
+        uint8_t *const stg = smem + Lay::kOffStg + (warp - 2) * 2 * 2048;
+        int nbox = 0;   // boxes this warp has issued (buffer nbox & 1)
         int it = e;
         for (int64_t tile = blockIdx.x + (int64_t)e * gridDim.x; tile < ntiles;
              tile += (int64_t)kEpiWG * gridDim.x, it += kEpiWG) {
@@ -188,6 +197,7 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
             const float inv = 1.f / Z;
             const int64_t t = tile * kBM + row_in_tile;
             const bool valid = t < Tv;
+            const int64_t t_warp = tile * kBM + q * 32;   // first row of this warp's slice
             TP *out = phi + (t * Hv + h) * (int64_t)F;
             __nv_bfloat16 *lo = phi_lo ? phi_lo + (t * Hv + h) * (int64_t)F : nullptr;
             // pass 2: normalised features, stored
@@ -200,6 +210,41 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->acce[b]);   // last read of this accumulator
+                }
+                if (via_tma) {
+                    // "+" features c..c+31, then "-" features P+c..P+c+31: 64-byte
+                    // rows (one per lane), 16-byte chunks swizzled by (row / 2) % 4
+#pragma unroll
+                    for (int sg = 0; sg < 2; ++sg) {
+                        uint8_t *buf = stg + (nbox & 1) * 2048;
+                        if (nbox >= 2) {
+                            if (lane == 0) bulk_wait_read_le1();
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            float ev[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float u = __uint_as_float(r[8 * k + j]) + (bh ? bh[c + 8 * k + j] : 0.f);
+                                ev[j] = fexp((sg ? -u : u) - m) * inv;
+                            }
+                            uint4 v;
+                            v.x = pack_bf16x2(ev[0], ev[1]);
+                            v.y = pack_bf16x2(ev[2], ev[3]);
+                            v.z = pack_bf16x2(ev[4], ev[5]);
+                            v.w = pack_bf16x2(ev[6], ev[7]);
+                            *reinterpret_cast<uint4 *>(buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = v;
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0 && t_warp < Tv) {
+                            tma_store_3d(&tmo, buf, sg * P + c, h, (int)t_warp);
+                            bulk_commit();
+                        }
+                        ++nbox;
+                    }
+                    continue;
                 }
                 if (!valid) continue;
 #pragma unroll
@@ -249,6 +294,8 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
         }
     }
 
+    // the epilogue warps' bulk stores must be complete before the CTA exits
+    if (warp >= 2 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -279,6 +326,17 @@ cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head
         uint32_t box[2] = {64, (uint32_t)P};
         if (!tc::make_tmap_bf16(&tmw, W, 2, dims, strides, box)) return cudaErrorInvalidValue;
     }
+    // output boxes of 32 features x 32 rows (bf16, 64-byte rows, 64-byte swizzle)
+    CUtensorMap tmo;
+    {
+        uint64_t dims[3] = {(uint64_t)(2 * P), (uint64_t)Hv, (uint64_t)Tv};
+        uint64_t strides[2] = {(uint64_t)(2 * P) * sizeof(TP), (uint64_t)Hv * (2 * P) * sizeof(TP)};
+        uint32_t box[3] = {32, 1, 32};
+        if (sizeof(TP) == 2 && !tc::make_tmap(&tmo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, phi, 3, dims, strides, box,
+                                              CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
+        if (sizeof(TP) != 2) memset(&tmo, 0, sizeof(tmo));
+    }
     auto kern = featmap_tc_kernel<D, P, TP>;
     cudaError_t e = ensure_smem_limit(kern, Lay::kSmem);
     if (e != cudaSuccess) return e;
@@ -290,7 +348,7 @@ cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head
     if (per_head_ctas > ntiles) per_head_ctas = ntiles;
     if (per_head_ctas < 1) per_head_ctas = 1;
     dim3 grid((unsigned)per_head_ctas, (unsigned)Hv);
-    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx, tmw, Tv, Hv, bias, per_head ? 1 : 0, (TP *)phi,
+    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx, tmw, tmo, Tv, Hv, bias, per_head ? 1 : 0, (TP *)phi,
                                             (__nv_bfloat16 *)phi_lo, err);
     count_launches(1);
     return cudaGetLastError();

@@ -375,6 +375,7 @@ constexpr int kHelpers = 160;    // threads of the five helper warps
 
 struct CAux {
     float cum[2][kC];
+    float bq[2][32];     // e^(cum_(j|7) - cum_j), j < 32: column factors of the below-diagonal quadrant
     float qs[2][kC];
     float w[2][kC];
     float rden[2][kC];   // 1 / den
@@ -648,6 +649,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (gt == kC - 1) X->redb[1] = x;
                 named_sync(3, 64);
                 const float total = X->redb[1];
+                const float xe = __shfl_sync(0xffffffffu, x, lane | 7);   // cum at the end of j's 8-block
+                if (gt < 32) X->bq[s][gt] = fexp(xe - x);
                 X->cum[s][gt] = x;
                 X->qs[s][gt] = fexp(x);
                 X->w[s][gt] = fexp(total - x);
@@ -686,7 +689,38 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 // the buffer staged chunk it - 2's outputs
                 okw = __all_sync(0xffffffffu, okw && mbar_wait(&X->stg_free[s], ((it >> 1) & 1) ^ 1, abort_flag,
                                                                    err, KID_SCAN_TC_OUT, 18));
-                if (okw) {
+                if (okw && !masked) {
+                    // every 8-column block lies below the diagonal:
+                    // e^(cum_i - cum_j) = e^(cum_i - cum_b) e^(cum_b - cum_j), b the
+                    // block's last column, both factors <= 1
+                    const float ci = X->cum[s][i];
+                    uint8_t *__restrict__ prow = gP(s);
+                    float rs = 0.f;
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const float ai = fexp(ci - X->cum[s][8 * c4 + 7]);
+                        const float4 ba = *reinterpret_cast<const float4 *>(&X->bq[s][8 * c4]);
+                        const float4 bb = *reinterpret_cast<const float4 *>(&X->bq[s][8 * c4 + 4]);
+                        const float bv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+                        uint4 hi, lo;
+                        uint32_t *pk = reinterpret_cast<uint32_t *>(&hi);
+                        uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int jl = c4 * 8 + 2 * e;
+                            const float e0 = __uint_as_float(pr[jl]) * (ai * bv[2 * e]);
+                            const float e1 = __uint_as_float(pr[jl + 1]) * (ai * bv[2 * e + 1]);
+                            pk[e] = pack_bf16x2(e0, e1);
+                            const float2 r = unpack_bf16x2(pk[e]);
+                            pl[e] = pack_bf16x2(e0 - r.x, e1 - r.y);
+                            rs += e0 + e1;
+                        }
+                        *reinterpret_cast<uint4 *>(prow + sw128_off(i, c4)) = hi;
+                        *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, c4)) = lo;
+                    }
+                    X->dint[0][i] = rs;
+                    tc_fence_before();
+                } else if (okw) {
                     const float ci = X->cum[s][i];
                     const float *__restrict__ cj = X->cum[s] + jc;
                     uint8_t *__restrict__ prow = gP(s);
