@@ -9,13 +9,13 @@
 // x stream through a 2-stage TMA ring.  Warp roles:
 //   warp 0      TMA producer (one elected lane)
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2..9  two epilogue warpgroups taking alternate tiles: one
+//   warps 2..13 three epilogue warpgroups taking tiles in turn: one
 //               accumulator row per thread, read from TMEM in two passes (a
 //               running max / normaliser, then the normalised features), the
-//               negate / concatenate / softmax in registers.  bf16 features
-//               are staged per warp (boxes of 32 rows x 32 features, two 2 KB
-//               buffers used in turn) and written by TMA bulk stores; fp32
-//               features and the bf16 remainder plane are stored directly.
+//               negate / concatenate / softmax in registers, and the store.
+//               The epilogue is latency-bound (exponentials and TMEM loads of
+//               one row per thread), so three warps per SM sub-partition
+//               share the work.
 // Four TMEM accumulators let the MMAs run ahead of both epilogue warpgroups.
 // The kernel is bound by HBM (x in, phi out); MMA and exp work hide under it.
 #include "tc_common.cuh"
@@ -28,7 +28,7 @@ using namespace tc;
 
 constexpr int kBM = 128;     // rows per tile (MMA M)
 constexpr int kStages = 2;   // x tiles in flight
-constexpr int kEpiWG = 2;    // epilogue warpgroups (alternate tiles)
+constexpr int kEpiWG = 3;    // epilogue warpgroups (tiles in turn)
 constexpr int kThreads = 64 + 128 * kEpiWG;
 
 template <int D, int P>
@@ -39,9 +39,7 @@ struct FmLayout {
     static constexpr int kXBytes = kChunks * kXChunkBytes;  // one x tile
     static constexpr int kOffW = 0;
     static constexpr int kOffX = kWBytes;
-    static constexpr int kOffStg = kOffX + kStages * kXBytes;     // 8 warps x 2 x 2 KB staging
-    static constexpr int kStgBytes = 8 * 2 * 2048;
-    static constexpr int kOffBar = kOffStg + kStgBytes;
+    static constexpr int kOffBar = kOffX + kStages * kXBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;      // + barriers, + alignment slack
     static constexpr int kAcc = 512 / P >= 4 ? 4 : 2;       // TMEM accumulators
     static constexpr int kTmemCols = kAcc * P <= 256 ? 256 : 512;
@@ -61,9 +59,19 @@ __device__ __forceinline__ float fexp(float x) { return exp2f(x * 1.442695040888
 
 template <int D, int P, typename TP>
 __global__ void __launch_bounds__(kThreads, 1)
-featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-                  const __grid_constant__ CUtensorMap tmo, int64_t Tv, int Hv, const float *__restrict__ bias,
-                  int bias_per_head, TP *__restrict__ phi, __nv_bfloat16 *__restrict__ phi_lo, DevErr err) {
+featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constant__ CUtensorMap tmw0,
+                  const __grid_constant__ CUtensorMap tmx1, const __grid_constant__ CUtensorMap tmw1,
+                  int64_t Tv, int Hv, const float *__restrict__ bias0, const float *__restrict__ bias1,
+                  int bias_per_head, TP *__restrict__ phi0, TP *__restrict__ phi1,
+                  __nv_bfloat16 *__restrict__ phi_lo0, __nv_bfloat16 *__restrict__ phi_lo1, DevErr err) {
+    // blockIdx.z selects one of two independent inputs of the same shape (the
+    // q and k maps of a scan run in one launch)
+    const bool second = blockIdx.z != 0;
+    const CUtensorMap &tmx = second ? tmx1 : tmx0;
+    const CUtensorMap &tmw = second ? tmw1 : tmw0;
+    const float *__restrict__ bias = second ? bias1 : bias0;
+    TP *__restrict__ phi = second ? phi1 : phi0;
+    __nv_bfloat16 *__restrict__ phi_lo = second ? phi_lo1 : phi_lo0;
     using Lay = FmLayout<D, P>;
     constexpr int NA = Lay::kAcc;
     extern __shared__ uint8_t smem_raw[];
@@ -162,10 +170,6 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
         const int row_in_tile = q * 32 + lane;
         constexpr int F = 2 * P;
         const float *bh = bias ? bias + (bias_per_head ? (int64_t)h * P : 0) : nullptr;
-        // bf16 features without a remainder plane leave through TMA stores
-        const bool via_tma = sizeof(TP) == 2 && phi_lo == nullptr;
-        uint8_t *const stg = smem + Lay::kOffStg + (warp - 2) * 2 * 2048;
-        int nbox = 0;   // boxes this warp has issued (buffer nbox & 1)
         int it = e;
         for (int64_t tile = blockIdx.x + (int64_t)e * gridDim.x; tile < ntiles;
              tile += (int64_t)kEpiWG * gridDim.x, it += kEpiWG) {
@@ -197,7 +201,6 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
             const float inv = 1.f / Z;
             const int64_t t = tile * kBM + row_in_tile;
             const bool valid = t < Tv;
-            const int64_t t_warp = tile * kBM + q * 32;   // first row of this warp's slice
             TP *out = phi + (t * Hv + h) * (int64_t)F;
             __nv_bfloat16 *lo = phi_lo ? phi_lo + (t * Hv + h) * (int64_t)F : nullptr;
             // pass 2: normalised features, stored
@@ -210,41 +213,6 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->acce[b]);   // last read of this accumulator
-                }
-                if (via_tma) {
-                    // "+" features c..c+31, then "-" features P+c..P+c+31: 64-byte
-                    // rows (one per lane), 16-byte chunks swizzled by (row / 2) % 4
-#pragma unroll
-                    for (int sg = 0; sg < 2; ++sg) {
-                        uint8_t *buf = stg + (nbox & 1) * 2048;
-                        if (nbox >= 2) {
-                            if (lane == 0) bulk_wait_read_le1();
-                            __syncwarp();
-                        }
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            float ev[8];
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const float u = __uint_as_float(r[8 * k + j]) + (bh ? bh[c + 8 * k + j] : 0.f);
-                                ev[j] = fexp((sg ? -u : u) - m) * inv;
-                            }
-                            uint4 v;
-                            v.x = pack_bf16x2(ev[0], ev[1]);
-                            v.y = pack_bf16x2(ev[2], ev[3]);
-                            v.z = pack_bf16x2(ev[4], ev[5]);
-                            v.w = pack_bf16x2(ev[6], ev[7]);
-                            *reinterpret_cast<uint4 *>(buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = v;
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0 && t_warp < Tv) {
-                            tma_store_3d(&tmo, buf, sg * P + c, h, (int)t_warp);
-                            bulk_commit();
-                        }
-                        ++nbox;
-                    }
-                    continue;
                 }
                 if (!valid) continue;
 #pragma unroll
@@ -294,8 +262,6 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
         }
     }
 
-    // the epilogue warps' bulk stores must be complete before the CTA exits
-    if (warp >= 2 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -305,37 +271,35 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant
     }
 }
 
+// One launch for up to two inputs (x1 == nullptr: one).
 template <int D, int P, typename TP>
-cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head_stride,
-               const float *bias, void *phi, void *phi_lo, DevErr err, cudaStream_t s) {
+cudaError_t go(const void *x0, const void *W0, const float *bias0, void *phi0, void *lo0, const void *x1,
+               const void *W1, const float *bias1, void *phi1, void *lo1, int64_t rows, int H,
+               int64_t w_head_stride, DevErr err, cudaStream_t s) {
     using Lay = FmLayout<D, P>;
     const bool per_head = w_head_stride != 0;
     const int Hv = per_head ? H : 1;
     const int64_t Tv = rows / Hv;
-    CUtensorMap tmx, tmw;
-    {
-        uint64_t dims[3] = {(uint64_t)D, (uint64_t)Hv, (uint64_t)Tv};
-        uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)Hv * D * 2};
-        uint32_t box[3] = {64, 1, kBM};
-        if (!tc::make_tmap_bf16(&tmx, x, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    const int nz = x1 ? 2 : 1;
+    CUtensorMap tmx[2], tmw[2];
+    for (int z = 0; z < nz; ++z) {
+        {
+            uint64_t dims[3] = {(uint64_t)D, (uint64_t)Hv, (uint64_t)Tv};
+            uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)Hv * D * 2};
+            uint32_t box[3] = {64, 1, kBM};
+            if (!tc::make_tmap_bf16(&tmx[z], z ? x1 : x0, 3, dims, strides, box)) return cudaErrorInvalidValue;
+        }
+        {
+            // W rows: head h's [P, D] starts at row h * P when the stride is P * D
+            uint64_t dims[2] = {(uint64_t)D, (uint64_t)Hv * P};
+            uint64_t strides[1] = {(uint64_t)D * 2};
+            uint32_t box[2] = {64, (uint32_t)P};
+            if (!tc::make_tmap_bf16(&tmw[z], z ? W1 : W0, 2, dims, strides, box)) return cudaErrorInvalidValue;
+        }
     }
-    {
-        // W rows: head h's [P, D] starts at row h * P when the stride is P * D
-        uint64_t dims[2] = {(uint64_t)D, (uint64_t)Hv * P};
-        uint64_t strides[1] = {(uint64_t)D * 2};
-        uint32_t box[2] = {64, (uint32_t)P};
-        if (!tc::make_tmap_bf16(&tmw, W, 2, dims, strides, box)) return cudaErrorInvalidValue;
-    }
-    // output boxes of 32 features x 32 rows (bf16, 64-byte rows, 64-byte swizzle)
-    CUtensorMap tmo;
-    {
-        uint64_t dims[3] = {(uint64_t)(2 * P), (uint64_t)Hv, (uint64_t)Tv};
-        uint64_t strides[2] = {(uint64_t)(2 * P) * sizeof(TP), (uint64_t)Hv * (2 * P) * sizeof(TP)};
-        uint32_t box[3] = {32, 1, 32};
-        if (sizeof(TP) == 2 && !tc::make_tmap(&tmo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, phi, 3, dims, strides, box,
-                                              CU_TENSOR_MAP_SWIZZLE_64B))
-            return cudaErrorInvalidValue;
-        if (sizeof(TP) != 2) memset(&tmo, 0, sizeof(tmo));
+    if (nz == 1) {
+        tmx[1] = tmx[0];
+        tmw[1] = tmw[0];
     }
     auto kern = featmap_tc_kernel<D, P, TP>;
     cudaError_t e = ensure_smem_limit(kern, Lay::kSmem);
@@ -344,12 +308,13 @@ cudaError_t go(const void *x, int64_t rows, int H, const void *W, int64_t w_head
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t per_head_ctas = (sms + Hv - 1) / Hv;
+    int64_t per_head_ctas = (sms + Hv * nz - 1) / (Hv * nz);
     if (per_head_ctas > ntiles) per_head_ctas = ntiles;
     if (per_head_ctas < 1) per_head_ctas = 1;
-    dim3 grid((unsigned)per_head_ctas, (unsigned)Hv);
-    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx, tmw, tmo, Tv, Hv, bias, per_head ? 1 : 0, (TP *)phi,
-                                            (__nv_bfloat16 *)phi_lo, err);
+    dim3 grid((unsigned)per_head_ctas, (unsigned)Hv, (unsigned)nz);
+    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx[0], tmw[0], tmx[1], tmw[1], Tv, Hv, bias0, bias1, per_head ? 1 : 0,
+                                            (TP *)phi0, (TP *)phi1, (__nv_bfloat16 *)lo0, (__nv_bfloat16 *)lo1,
+                                            err);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -366,16 +331,18 @@ bool featmap_tc_supported(int64_t rows, int H, int d, int p, int64_t w_head_stri
     return true;
 }
 
-cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, const void *W,
-                              int64_t w_head_stride, const float *bias, void *phi, hm_dtype pt,
-                              DevErr err, cudaStream_t s, void *phi_lo) {
+cudaError_t launch_featmap_tc2(const void *x0, const void *W0, const float *bias0, void *phi0, void *lo0,
+                               const void *x1, const void *W1, const float *bias1, void *phi1, void *lo1,
+                               int64_t rows, int H, int d, int p, int64_t w_head_stride, hm_dtype pt, DevErr err,
+                               cudaStream_t s) {
     if (!featmap_tc_supported(rows, H, d, p, w_head_stride)) return cudaErrorNotSupported;
-    if (phi_lo && pt != HM_BF16) return cudaErrorInvalidValue;
-#define HM_FM_CASE(DD, PP)                                                                  \
-    if (d == DD && p == PP)                                                                 \
-        return pt == HM_BF16                                                                \
-                   ? go<DD, PP, __nv_bfloat16>(x, rows, H, W, w_head_stride, bias, phi, phi_lo, err, s) \
-                   : go<DD, PP, float>(x, rows, H, W, w_head_stride, bias, phi, nullptr, err, s);
+    if ((lo0 || lo1) && pt != HM_BF16) return cudaErrorInvalidValue;
+#define HM_FM_CASE(DD, PP)                                                                              \
+    if (d == DD && p == PP)                                                                             \
+        return pt == HM_BF16 ? go<DD, PP, __nv_bfloat16>(x0, W0, bias0, phi0, lo0, x1, W1, bias1, phi1, lo1, \
+                                                         rows, H, w_head_stride, err, s)                  \
+                             : go<DD, PP, float>(x0, W0, bias0, phi0, nullptr, x1, W1, bias1, phi1, nullptr, \
+                                                 rows, H, w_head_stride, err, s);
     HM_FM_CASE(64, 64)
     HM_FM_CASE(64, 128)
     HM_FM_CASE(128, 64)
@@ -384,6 +351,13 @@ cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, 
     HM_FM_CASE(256, 128)
 #undef HM_FM_CASE
     return cudaErrorNotSupported;
+}
+
+cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, const void *W,
+                              int64_t w_head_stride, const float *bias, void *phi, hm_dtype pt,
+                              DevErr err, cudaStream_t s, void *phi_lo) {
+    return launch_featmap_tc2(x, W, bias, phi, phi_lo, nullptr, nullptr, nullptr, nullptr, nullptr, rows, H, d, p,
+                              w_head_stride, pt, err, s);
 }
 
 }  // namespace hm

@@ -85,6 +85,19 @@ cudaError_t run_featmap(const void *x, hm_dtype xt, int64_t rows, int H, int d, 
     return launch_featmap_simt(x, xt, rows, H, d, p, W, wstride, bias, phi, pt, s, phi_lo);
 }
 
+// phi(q) and phi(k): one tensor-core launch when the shape has a kernel.
+cudaError_t run_featmap_qk(const void *q, const void *k, hm_dtype xt, int64_t rows, int H, int d, int p,
+                           const void *W_q, const void *W_k, int64_t wstride, const float *b_q,
+                           const float *b_k, void *phq, void *phk, hm_dtype pt, cudaStream_t s,
+                           void *phk_lo = nullptr) {
+    if (xt == HM_BF16 && featmap_tc_supported(rows, H, d, p, wstride))
+        return launch_featmap_tc2(q, W_q, b_q, phq, nullptr, k, W_k, b_k, phk, phk_lo, rows, H, d, p, wstride, pt,
+                                  DevErr{device_error_word()}, s);
+    cudaError_t e = launch_featmap_simt(q, xt, rows, H, d, p, W_q, wstride, b_q, phq, pt, s, nullptr);
+    if (e != cudaSuccess) return e;
+    return launch_featmap_simt(k, xt, rows, H, d, p, W_k, wstride, b_k, phk, pt, s, phk_lo);
+}
+
 // ------------------------------------------------------------------ scan
 
 struct ScanPlan {
@@ -333,12 +346,9 @@ hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
     if (a->W_q && rows > 0) {
         void *wq = ws, *wk = ws + pl.phi_bytes;
         void *wkl = pl.lo_bytes ? ws + 2 * pl.phi_bytes : nullptr;
-        e = run_featmap(a->q, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->w_head_stride, a->b_q,
-                        wq, pl.feat, s);
-        if (e != cudaSuccess) return cuda_fail(e, "scan: featmap(q)");
-        e = run_featmap(a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_k, a->w_head_stride, a->b_k,
-                        wk, pl.feat, s, wkl);
-        if (e != cudaSuccess) return cuda_fail(e, "scan: featmap(k)");
+        e = run_featmap_qk(a->q, a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->W_k, a->w_head_stride,
+                           a->b_q, a->b_k, wq, wk, pl.feat, s, wkl);
+        if (e != cudaSuccess) return cuda_fail(e, "scan: feature maps");
         phq = wq;
         phk = wk;
         phk_lo = wkl;
@@ -398,12 +408,9 @@ hm_status hm_step_decode(const hm_decode_args *a, hm_stream_t stream) {
     cudaError_t e;
     if (a->W_q && rows > 0) {
         char *ws = (char *)a->workspace;
-        e = run_featmap(a->q, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->w_head_stride, a->b_q,
-                        ws, HM_F32, s);
-        if (e != cudaSuccess) return cuda_fail(e, "decode: featmap(q)");
-        e = run_featmap(a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_k, a->w_head_stride, a->b_k,
-                        ws + pl.phi_bytes, HM_F32, s);
-        if (e != cudaSuccess) return cuda_fail(e, "decode: featmap(k)");
+        e = run_featmap_qk(a->q, a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->W_k, a->w_head_stride,
+                           a->b_q, a->b_k, ws, ws + pl.phi_bytes, HM_F32, s);
+        if (e != cudaSuccess) return cuda_fail(e, "decode: feature maps");
         phq = ws;
         phk = ws + pl.phi_bytes;
         ft = HM_F32;

@@ -89,6 +89,11 @@ cudaError_t launch_featmap_tc(const void *x, int64_t rows, int H, int d, int p, 
                               int64_t w_head_stride, const float *bias, void *phi, hm_dtype pt,
                               DevErr err, cudaStream_t s, void *phi_lo = nullptr);
 bool featmap_tc_supported(int64_t rows, int H, int d, int p, int64_t w_head_stride);
+// Two feature maps of the same shape (e.g. q and k) in one launch.
+cudaError_t launch_featmap_tc2(const void *x0, const void *W0, const float *bias0, void *phi0, void *lo0,
+                               const void *x1, const void *W1, const float *bias1, void *phi1, void *lo1,
+                               int64_t rows, int H, int d, int p, int64_t w_head_stride, hm_dtype pt, DevErr err,
+                               cudaStream_t s);
 
 // Generic SIMT chunk-free scan over precomputed features (fp32 state).
 struct ScanCore {
