@@ -392,6 +392,7 @@ struct CAux {
     uint64_t stg_free[2];   // the stage's Pt buffer, used to stage outputs, has been read out
     uint64_t p_full, p_consumed, epib_done, o_full, o_empty, s_full, sbf_ready;
     uint64_t den_ready[2], den_free[2];   // 1 / den of a stage written / read
+    uint64_t pro_full[3];                 // start-state rounds landed (prologue staging)
     uint32_t tmem;
     int abort;
 };
@@ -457,8 +458,8 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
 // update S^T += (w V)^T phiK.
 __global__ void __launch_bounds__(448, 1)
 scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo, OutArgs a,
-                DevErr err) {
+                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                const __grid_constant__ CUtensorMap tms, OutArgs a, DevErr err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
     CAux *X = (CAux *)(smem + kCOffAux);
@@ -509,6 +510,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_init(&X->den_ready[s], 1);
             mbar_init(&X->den_free[s], 4);
         }
+        for (int r = 0; r < 3; ++r) mbar_init(&X->pro_full[r], 1);
         X->abort = 0;
         mbar_fence_init();
     }
@@ -656,7 +658,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 X->w[s][gt] = fexp(total - x);
                 if (gt == 0) X->gam[s] = fexp(total);
             }
-            ok = named_sync_and(1, 256, ok);
+            // (chunk 0: the state prologue, which stages in the Pt and w V buffers,
+            // must be complete before they are written)
+            ok = named_sync_and(1, 256, ok && (it > 0 || mbar_wait(&X->sbf_ready, 0, abort_flag, err,
+                                                                    KID_SCAN_TC_OUT, 21)));
             if (!ok) break;
             // (2) once the chunk's scores are in TMEM
             bool okw = mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7) &&
@@ -892,20 +897,54 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         {
             const float gam0 = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 2));
             if (nch > 1) dt_next = token_dt(a, b, h, (int64_t)(c_begin + 1) * kC, td);
-            const float *src = nullptr;
-            if (seg == 0) src = a.S0 ? a.S0 + bh * (int64_t)kF * g.dv : nullptr;
-            else src = a.S_start + (bh * g.G + seg) * (int64_t)kF * g.dv;
-            for (int c0 = 0; c0 < kF; c0 += 32) {
-                uint32_t v[32], pk[16];
+            if (seg > 0) {
+                // segment start state [F][dv] (fp32, in L2): rounds of 32 feature rows
+                // x the CTA's 128 channels (16 KB) land by TMA in three rotating
+                // buffers (the Pt and w V tiles, unused until the first chunk)
+                const int row0 = (int)((bh * g.G + seg) * kF);
+                uint8_t *const pbuf = gP(0);
+                if (td == 0)
+                    for (int r = 0; r < 3; ++r) {
+                        mbar_arrive_expect_tx(&X->pro_full[r], 32 * kN * 4);
+                        tma_load_2d(pbuf + r * 32 * kN * 4, &tms, &X->pro_full[r], dv0, row0 + 32 * r);
+                    }
+#pragma unroll 1
+                for (int r = 0; r < kF / 32; ++r) {
+                    mbar_wait(&X->pro_full[r % 3], (r / 3) & 1, abort_flag, err, KID_SCAN_TC_OUT, 22);
+                    const float *buf = reinterpret_cast<const float *>(pbuf + (r % 3) * 32 * kN * 4) + ch;
+                    uint32_t v[32], pk[16];
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    v[j] = __float_as_uint(src ? src[(int64_t)(c0 + j) * g.dv + dv0 + ch] : 0.f);
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(buf[j * kN]);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-                tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
+                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                    tmem_st16(tmem + kColSB + 16 * r + lanebase, pk);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
-                tmem_st32(tmem + kColS + c0 + lanebase, v);
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
+                    tmem_st32(tmem + kColS + 32 * r + lanebase, v);
+                    named_sync(2, 128);   // every thread has read this buffer
+                    if (td == 0 && r + 3 < kF / 32) {
+                        mbar_arrive_expect_tx(&X->pro_full[r % 3], 32 * kN * 4);
+                        tma_load_2d(pbuf + (r % 3) * 32 * kN * 4, &tms, &X->pro_full[r % 3], dv0, row0 + 32 * (r + 3));
+                    }
+                }
+            } else {
+                const float *src = a.S0 ? a.S0 + bh * (int64_t)kF * g.dv : nullptr;
+                for (int c0 = 0; c0 < kF; c0 += 32) {
+                    uint32_t v[32], pk[16];
+                    if (src) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(src[(int64_t)(c0 + j) * g.dv + dv0 + ch]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = 0u;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                    tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
+                    tmem_st32(tmem + kColS + c0 + lanebase, v);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -1179,9 +1218,19 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
                        dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
+    // segment start states [BH * G * F][dv] fp32: boxes of 32 feature rows x 128 channels
+    CUtensorMap tss;
+    {
+        uint64_t dims[2] = {(uint64_t)c.dv, (uint64_t)BH * g.G * kF};
+        uint64_t strides[1] = {(uint64_t)c.dv * 4};
+        uint32_t box[2] = {(uint32_t)kN, 32};
+        if (!make_tmap(&tss, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, S_start, 2, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
     e = ensure_smem_limit(scan_out_kernel, kCSmem);
     if (e != cudaSuccess) return e;
-    scan_out_kernel<<<(unsigned)(2 * g.G * BH), 448, kCSmem, s>>>(tq, tk, tv, to, oa, err);
+    scan_out_kernel<<<(unsigned)(2 * g.G * BH), 448, kCSmem, s>>>(tq, tk, tv, to, tss, oa, err);
     count_launches(1);
     return cudaGetLastError();
 }
