@@ -241,6 +241,15 @@ HM_API uint64_t hm_launch_count(void);
  * word: HM_OK, HM_ERR_TIMEOUT (a bounded wait expired) or HM_ERR_DEVICE. */
 HM_API hm_status hm_get_device_error(hm_stream_t stream);
 
+/* Diagnostic with no counterpart in the method: enqueues one thread block on
+ * `stream` that waits on a barrier nothing ever signals, polling it at most
+ * `polls` times (1 .. 2^20) with the same bounded wait the library's
+ * pipelined kernels use, then records HM_ERR_TIMEOUT in the device error
+ * word, as a stalled pipeline would.  Returns HM_OK once enqueued,
+ * HM_ERR_INVALID_ARG for a bad poll count.  Read the recorded status with
+ * hm_get_device_error; the context remains usable afterwards. */
+HM_API hm_status hm_selftest_wait_timeout(uint32_t polls, hm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

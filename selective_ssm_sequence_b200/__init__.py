@@ -20,7 +20,7 @@ HM_F32, HM_BF16 = 0, 1
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libhm.so is not built (%s); run __graft_entry__.build() or "
-                      "python -m selective_ssm_sequence_b200._build" % LIB_PATH)
+                      "python selective_ssm_sequence_b200/_build.py" % LIB_PATH)
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -80,11 +80,13 @@ lib.hm_launch_count.restype = ctypes.c_uint64
 lib.hm_launch_count.argtypes = []
 lib.hm_get_device_error.restype = _I
 lib.hm_get_device_error.argtypes = [_P]
+lib.hm_selftest_wait_timeout.restype = _I
+lib.hm_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
 
 EXPORTED = ("hm_status_string", "hm_last_error_detail", "hm_version", "hm_featmap",
             "hm_scan_workspace_size", "hm_scan_chunked_fwd", "hm_decode_workspace_size",
             "hm_step_decode", "hm_mixer_workspace_size", "hm_mixer_fwd", "hm_get_device_error",
-            "hm_launch_count", "hm_step_decode_noalloc")
+            "hm_launch_count", "hm_step_decode_noalloc", "hm_selftest_wait_timeout")
 
 
 class HMError(RuntimeError):
@@ -257,6 +259,11 @@ def hm_launch_count() -> int:
 def hm_get_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error word status."""
     return int(lib.hm_get_device_error(_stream(stream)))
+
+
+def hm_selftest_wait_timeout(polls: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test (records HM_ERR_TIMEOUT on the device)."""
+    _check(lib.hm_selftest_wait_timeout(int(polls), _stream(stream)), "hm_selftest_wait_timeout")
 
 
 def alloc_workspace(nbytes: int, device=None):

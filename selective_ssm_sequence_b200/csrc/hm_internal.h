@@ -27,6 +27,7 @@ enum KernelId : unsigned int {
     KID_DECODE = 7,
     KID_GEMM_TC = 8,
     KID_CONV = 9,
+    KID_SELFTEST = 10,
 };
 
 unsigned int *device_error_word();  // address of this device's error word (host)

@@ -16,8 +16,7 @@ HEADER = os.path.join(ROOT, "include", "hm.h")
 @pytest.fixture(scope="module")
 def hm():
     import __graft_entry__
-    from selective_ssm_sequence_b200 import _build
-    _build.build()
+    __graft_entry__._build_module().build()
     import selective_ssm_sequence_b200 as mod
     return mod
 
