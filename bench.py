@@ -54,10 +54,13 @@ def load_peaks():
         return dict(_FALLBACK_PEAKS), "fallback"
 
 
-# DRAM bytes per launch of the dominant kernel from an ncu capture of the
-# current kernel version (dram__bytes_read.sum + dram__bytes_write.sum), or
-# None when the kernel changed since the counters were taken.
-NCU_TRAFFIC_BYTES = {}
+# DRAM bytes per launch of the dominant call from an ncu capture of the
+# current kernel versions (dram__bytes_read.sum + dram__bytes_write.sum,
+# summed over the call's kernels; ncu runs each kernel with cold caches), or
+# None when a kernel changed since the counters were taken.  Prefill
+# B4 H8 L2048: scan_state 33,745,408 + scan_carry 16,856,576 + scan_out
+# 109,500,928 + 9,899,776 (profiles/scan_call_traffic_prefill_B4_H8_L2048.md).
+NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 170002688}
 
 # ---------------------------------------------------------------- clocks
 
@@ -375,7 +378,7 @@ def bench_prefill(cfg, args, rank, world, torch):
     else:
         roof = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": bw, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = NCU_TRAFFIC_BYTES.get(name)
+    roof["traffic"] = NCU_TRAFFIC_BYTES.get((name, cfg.name))
     roof["kernel"] = name
     roof["peak_source"] = peak_kind
     roof["ms_per_launch"] = ms
