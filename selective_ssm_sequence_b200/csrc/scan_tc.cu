@@ -687,6 +687,9 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             named_sync(4, 256);
             if (gt == 0) mbar_arrive(&X->p_consumed);
             if (pwarp) {
+                // (The 8-column block loops below stay rolled: the kernel's roles
+                // together run more code per chunk than the instruction cache
+                // holds, and rolling them measured faster.)
                 // Pt = P * exp(cum_i - cum_j) on j <= i, as bf16 hi + lo (the PV
                 // product runs on both: a few-token weighted average would
                 // otherwise carry the 2^-9 rounding of each weight), and row sums
@@ -701,7 +704,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     const float ci = X->cum[s][i];
                     uint8_t *__restrict__ prow = gP(s);
                     float rs = 0.f;
-#pragma unroll
+#pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
                         const float ai = fexp(ci - X->cum[s][8 * c4 + 7]);
                         const float4 ba = *reinterpret_cast<const float4 *>(&X->bq[s][8 * c4]);
@@ -730,7 +733,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     const float *__restrict__ cj = X->cum[s] + jc;
                     uint8_t *__restrict__ prow = gP(s);
                     float rs = 0.f;
-#pragma unroll
+#pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
                         uint4 hi, lo;
                         uint32_t *pk = reinterpret_cast<uint32_t *>(&hi);
