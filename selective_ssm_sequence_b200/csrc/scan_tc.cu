@@ -426,7 +426,7 @@ struct OutArgs {
 // raw value is fetched a chunk ahead and turned into log a when it is used,
 // so the load's latency is never waited for.
 __device__ __forceinline__ float token_dt(const OutArgs &a, int64_t b, int h, int64_t t0, int tg) {
-    if (tg < kC && a.dt && t0 + tg < a.g.L) return a.dt[(b * a.g.L + t0 + tg) * a.g.H + h];
+    if (tg >= 0 && tg < kC && a.dt && t0 + tg < a.g.L) return a.dt[(b * a.g.L + t0 + tg) * a.g.H + h];
     return -INFINITY;
 }
 
@@ -444,11 +444,12 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
 // Warp roles (14 warps):
 //   0      TMA producer (phiQ, phiK, V of each chunk; two stages)
 //   1      MMA issuer
-//   2..9   compute group (256 threads): per chunk the decay prefix sums, the
-//          decayed score tile Pt (three 32 x 32 quadrants: rows 0..31 need
-//          only columns 0..31), w (.) V, the weighted key-feature sums for z,
-//          the scaled queries e^cum (.) phiQ with phiq . z_prev, the
-//          denominators and z
+//   2..9   compute group (256 threads): per chunk the decayed score tile Pt
+//          (three 32 x 32 quadrants: rows 0..31 need only columns 0..31),
+//          w (.) V and the decay vectors of the next chunk (prefix sums of
+//          log a, e^cum, e^(cum_last - cum), gamma), the scaled queries
+//          e^cum (.) phiQ with phiq . z_prev, the denominators, the weighted
+//          key-feature sums and z
 //   10..13 outputs and state pass: o = O^T / den for the chunk, staged in the
 //          chunk's Pt buffer (dead once the PV product is complete) and written
 //          by TMA bulk stores; then S^T (fp32, TMEM) -> bf16 copy for the next
@@ -628,36 +629,44 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             X->z[gt] = zi ? zi[gt] : 0.f;
         }
         // dt of the next chunk's tokens is fetched one chunk ahead
-        float dt_next = token_dt(a, b, h, (int64_t)c_begin * kC, gt);
+        // decay of chunk c (warps 4, 5: thread = token tk): cum, e^cum, weights
+        // e^(cum_last - cum), the below-diagonal column factors and gamma, into
+        // the buffers of c's parity.  Chunk c + 1's is computed during chunk c,
+        // while those warps wait for the score quadrants.
+        const bool dwarp = warp == 4 || warp == 5;
+        const int tk = gt - 64;   // 0..63 on the decay warps
+        float dt_next = dwarp ? token_dt(a, b, h, (int64_t)c_begin * kC, tk) : -INFINITY;
+        auto decay = [&](int c) {
+            const int sc = c & 1;
+            const float l = hm_log_decay(dt_next, alog);
+            if (c + 1 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + c + 1) * kC, tk);
+            float x = l;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (tk == 31) X->redb[0] = x;
+            named_sync(5, 64);
+            if (tk >= 32) x += X->redb[0];
+            if (tk == kC - 1) X->redb[1] = x;
+            named_sync(5, 64);
+            const float total = X->redb[1];
+            const float xe = __shfl_sync(0xffffffffu, x, lane | 7);   // cum at the end of j's 8-block
+            if (tk < 32) X->bq[sc][tk] = fexp(xe - x);
+            X->cum[sc][tk] = x;
+            X->qs[sc][tk] = fexp(x);
+            X->w[sc][tk] = fexp(total - x);
+            if (tk == 0) X->gam[sc] = fexp(total);
+            named_sync(5, 64);   // redb free again
+        };
+        if (dwarp) decay(0);
         // every exit from this loop is taken by the whole group (after a
         // barrier-AND), so no thread is left waiting at a named barrier
         bool ok = named_sync_and(1, 256, true);
         for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
-            // (1) decay of the chunk (warps 2, 3: thread = token): cum, e^cum,
-            // weights e^(cum_last - cum), gamma
-            if (gt < kC) {
-                const float l = hm_log_decay(dt_next, alog);
-                if (it + 1 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + it + 1) * kC, gt);
-                float x = l;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, o);
-                    if (lane >= o) x += y;
-                }
-                if (gt == 31) X->redb[0] = x;
-                named_sync(3, 64);
-                if (gt >= 32) x += X->redb[0];
-                if (gt == kC - 1) X->redb[1] = x;
-                named_sync(3, 64);
-                const float total = X->redb[1];
-                const float xe = __shfl_sync(0xffffffffu, x, lane | 7);   // cum at the end of j's 8-block
-                if (gt < 32) X->bq[s][gt] = fexp(xe - x);
-                X->cum[s][gt] = x;
-                X->qs[s][gt] = fexp(x);
-                X->w[s][gt] = fexp(total - x);
-                if (gt == 0) X->gam[s] = fexp(total);
-            }
+            // (1) the chunk's decay vectors were computed during the previous chunk
             // (chunk 0: the state prologue, which stages in the Pt and w V buffers,
             // must be complete before they are written)
             ok = named_sync_and(1, 256, ok && (it > 0 || mbar_wait(&X->sbf_ready, 0, abort_flag, err,
@@ -776,31 +785,25 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 okw = __all_sync(0xffffffffu, okw);
                 if (okw) {
                     const uint8_t *__restrict__ vsrc = gV(s);
-                    uint4 vv[7];
-                    uint32_t offs[7];
+#pragma unroll 1
+                    for (int u = hx; u < kC * 16; u += kHelpers) {
+                        const int j = u >> 4, ci = u & 15;
+                        const uint32_t off = (uint32_t)((ci >> 3) * kBlk) + sw128_off(j, ci & 7);
+                        uint4 vv = *reinterpret_cast<const uint4 *>(vsrc + off);
+                        const float wj = wv[j];
+                        const float2 w2 = make_float2(wj, wj);
+                        uint32_t *pv = reinterpret_cast<uint32_t *>(&vv);
 #pragma unroll
-                    for (int r = 0; r < 7; ++r) {
-                        const int u = hx + r * kHelpers;
-                        const int j = (u >> 4) & (kC - 1), ci = u & 15;
-                        offs[r] = (uint32_t)((ci >> 3) * kBlk) + sw128_off(j, ci & 7);
-                        if (u < kC * 16) vv[r] = *reinterpret_cast<const uint4 *>(vsrc + offs[r]);
-                    }
-#pragma unroll
-                    for (int r = 0; r < 7; ++r) {
-                        const int u = hx + r * kHelpers;
-                        if (u < kC * 16) {
-                            const float wj = wv[u >> 4];
-                            const float2 w2 = make_float2(wj, wj);
-                            uint32_t *pv = reinterpret_cast<uint32_t *>(&vv[r]);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 x = mul2(unpack_bf16x2(pv[e]), w2);
-                                pv[e] = pack_bf16x2(x.x, x.y);
-                            }
-                            *reinterpret_cast<uint4 *>(gVt + offs[r]) = vv[r];
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = mul2(unpack_bf16x2(pv[e]), w2);
+                            pv[e] = pack_bf16x2(x.x, x.y);
                         }
+                        *reinterpret_cast<uint4 *>(gVt + off) = vv;
                     }
                 }
+                // the next chunk's decay vectors (its parity's buffers were last
+                // read during chunk it - 1)
+                if (dwarp && it + 1 < nch) decay(it + 1);
             }
             // (3) every thread: the query row scaled by e^cum_i, in place, and
             // phiq_i . z_prev over one quarter of the features (on the unscaled
