@@ -224,8 +224,10 @@ def scan_fwd(q, k, v, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=Non
     if W_q is None:
         phq, phk = q, k
     else:
-        phq = featmap(q, W_q, b_q, H=H, w_head_stride=w_head_stride)
-        phk = featmap(k, W_k, b_k, H=H, w_head_stride=w_head_stride)
+        # biases are per head exactly when the weights are (one [p] row per head)
+        bstride = W_q.shape[-2] if w_head_stride else 0
+        phq = featmap(q, W_q, b_q, H=H, w_head_stride=w_head_stride, b_head_stride=bstride)
+        phk = featmap(k, W_k, b_k, H=H, w_head_stride=w_head_stride, b_head_stride=bstride)
     la = None if dt is None else log_decay(dt, A_log)
     return scan_recurrent(phq, phk, v, la, S0, z0, return_state=return_state)
 

@@ -34,7 +34,8 @@ def to_np(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def run_scan(hm, inp, io, with_W=True, S0=None, z0=None, want_state=False, decay=True):
+def run_scan(hm, inp, io, with_W=True, S0=None, z0=None, want_state=False, decay=True,
+             w_head_stride=0, b_q=None, b_k=None):
     """Prefill through hm_scan_chunked_fwd; returns (o, S, z) as float64."""
     import torch
     q = dev_tensor(inp["q"], io)
@@ -46,7 +47,7 @@ def run_scan(hm, inp, io, with_W=True, S0=None, z0=None, want_state=False, decay
     A_log = dev_tensor(inp["A_log"], "f32") if (decay and "A_log" in inp) else None
     o = torch.empty_like(v)
     B, L, H, d = inp["q"].shape
-    F = 2 * inp["W_q"].shape[0] if with_W else d
+    F = 2 * inp["W_q"].shape[-2] if with_W else d
     dv = inp["v"].shape[-1]
     S = z = None
     if want_state:
@@ -54,8 +55,10 @@ def run_scan(hm, inp, io, with_W=True, S0=None, z0=None, want_state=False, decay
         z = torch.full((B, H, F), float("nan"), device="cuda")
     tS0 = dev_tensor(S0, "f32") if S0 is not None else None
     tz0 = dev_tensor(z0, "f32") if z0 is not None else None
+    tbq = dev_tensor(b_q, "f32") if b_q is not None else None
+    tbk = dev_tensor(b_k, "f32") if b_k is not None else None
     args = hm.scan_args(q, k, v, o, W_q=Wq, W_k=Wk, dt=dt, A_log=A_log, S0=tS0, z0=tz0,
-                        S_out=S, z_out=z)
+                        S_out=S, z_out=z, b_q=tbq, b_k=tbk, w_head_stride=w_head_stride)
     ws = hm.alloc_workspace(hm.hm_scan_workspace_size(args))
     args.workspace, args.workspace_bytes = ws.data_ptr(), ws.numel()
     hm.hm_scan_chunked_fwd(args)

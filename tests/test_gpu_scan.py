@@ -209,3 +209,33 @@ def test_precomputed_features_path(hm):
     o, _, _ = run_scan(hm, feat, "bf16", with_W=False)
     o_ref = oracle.scan_recurrent(phq, phk, inp["v"], oracle.log_decay(inp["dt"], inp["A_log"]))
     assert rel_err(o, o_ref) <= TOL_BF16
+
+
+def test_per_head_weights_and_biases(hm):
+    # one Hedgehog projection (and bias) per head: the q and k maps run in one
+    # launch with one CTA column per head
+    cfg = wl.PREFILL_PYTHIA
+    inp = wl.scan_inputs(cfg, B=2, L=200, seed=27)
+    H, p, d = cfg.H, cfg.p, cfg.d
+    Wq = wl.round_bf16(wl.normal(27, "Wq_heads", (H, p, d), 1 / d))
+    Wk = wl.round_bf16(wl.normal(27, "Wk_heads", (H, p, d), 1 / d))
+    bq = wl.round_f32(wl.normal(27, "bq_heads", (H, p), 0.25))
+    bk = wl.round_f32(wl.normal(27, "bk_heads", (H, p), 0.25))
+    heads = dict(inp, W_q=Wq, W_k=Wk)
+    o, S, z = run_scan(hm, heads, "bf16", want_state=True, w_head_stride=p * d, b_q=bq, b_k=bk)
+    o_ref, S_ref, z_ref = oracle.scan_fwd(inp["q"], inp["k"], inp["v"], Wq, Wk, dt=inp["dt"], A_log=inp["A_log"],
+                                          b_q=bq, b_k=bk, w_head_stride=p * d, return_state=True)
+    assert rel_err(o, o_ref) <= TOL_BF16
+    assert rel_err(S, S_ref) <= TOL_BF16
+    assert rel_err(z, z_ref) <= TOL_BF16
+
+
+def test_shared_weights_with_biases(hm):
+    cfg = wl.PREFILL_PYTHIA
+    inp = wl.scan_inputs(cfg, B=1, L=333, seed=28)
+    bq = wl.round_f32(wl.normal(28, "bq", (cfg.p,), 0.25))
+    bk = wl.round_f32(wl.normal(28, "bk", (cfg.p,), 0.25))
+    o, _, _ = run_scan(hm, inp, "bf16", b_q=bq, b_k=bk)
+    o_ref = oracle.scan_fwd(inp["q"], inp["k"], inp["v"], inp["W_q"], inp["W_k"], dt=inp["dt"],
+                            A_log=inp["A_log"], b_q=bq, b_k=bk)
+    assert rel_err(o, o_ref) <= TOL_BF16
