@@ -58,9 +58,10 @@ def load_peaks():
 # current kernel versions (dram__bytes_read.sum + dram__bytes_write.sum,
 # summed over the call's kernels; ncu runs each kernel with cold caches), or
 # None when a kernel changed since the counters were taken.  Prefill
-# B4 H8 L2048: scan_state 33,745,408 + scan_carry 16,856,576 + scan_out
-# 109,500,928 + 9,899,776 (profiles/scan_call_traffic_prefill_B4_H8_L2048.md).
-NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 170002688}
+# B4 H8 L2048: scan_state 33,745,664 + 2,048 + scan_carry 16,856,576 +
+# scan_out 109,442,304 + 10,339,072
+# (profiles/scan_call_traffic_prefill_B4_H8_L2048.md).
+NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 170385664}
 
 # ---------------------------------------------------------------- clocks
 
@@ -423,9 +424,17 @@ def bench_prefill(cfg, args, rank, world, torch):
 
 
 def bench_prefill_e2e(cfg, inp, Wq, Wk, A_log, args, world, torch, hm, flush):
-    """Same metric through one hm_scan_chunked_fwd call per step with the
-    step's inputs copied from pinned host memory and the output copied back."""
+    """Same metric through the C ABI with the step's inputs copied from pinned
+    host memory and the outputs copied back, all inside the timed region.
+
+    The batch is cut into pieces (one sequence each; a single sequence is cut
+    into 8 runs of tokens whose final state starts the next run), and the
+    pieces are pipelined on three streams: the upload of piece i + 1 and the
+    download of piece i - 1 overlap the scan of piece i (PCIe is full duplex).
+    The timed region runs from an event before the first upload to an event
+    after the last download, on the device timeline."""
     B, L, H, d, p, dv = cfg.B, cfg.L, cfg.H, cfg.d, cfg.p, cfg.dv
+    F = 2 * p
     hq, hk, hv = (torch.from_numpy(inp[n].astype(np.float32)).to(torch.bfloat16).pin_memory()
                   for n in ("q", "k", "v"))
     hdt = torch.from_numpy(inp["dt"].astype(np.float32)).pin_memory()
@@ -435,41 +444,79 @@ def bench_prefill_e2e(cfg, inp, Wq, Wk, A_log, args, world, torch, hm, flush):
     v = torch.empty(hv.shape, dtype=torch.bfloat16, device="cuda")
     dtt = torch.empty(hdt.shape, dtype=torch.float32, device="cuda")
     o = torch.empty_like(v)
-    a = hm.scan_args(q, k, v, o, W_q=Wq, W_k=Wk, dt=dtt, A_log=A_log)
-    ws = hm.alloc_workspace(hm.hm_scan_workspace_size(a))
-    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
-    stream = torch.cuda.current_stream()
+    if B > 1:
+        pieces = [(b, b + 1, 0, L) for b in range(B)]
+    else:
+        n = 8 if L % (8 * 64) == 0 else 1
+        pieces = [(0, 1, i * (L // n), (i + 1) * (L // n)) for i in range(n)]
+    chained = B == 1 and len(pieces) > 1
+    # state carried between the runs of one sequence (two buffers, alternating)
+    Sbuf = [torch.empty(1, H, F, dv, device="cuda") for _ in range(2)] if chained else None
+    zbuf = [torch.empty(1, H, F, device="cuda") for _ in range(2)] if chained else None
+    args_list = []
+    for i, (b0, b1, t0, t1) in enumerate(pieces):
+        sl = (slice(b0, b1), slice(t0, t1))
+        S0 = Sbuf[(i - 1) % 2] if chained and i > 0 else None
+        z0 = zbuf[(i - 1) % 2] if chained and i > 0 else None
+        So = Sbuf[i % 2] if chained and i + 1 < len(pieces) else None
+        zo = zbuf[i % 2] if chained and i + 1 < len(pieces) else None
+        a = hm.scan_args(q[sl], k[sl], v[sl], o[sl], W_q=Wq, W_k=Wk, dt=dtt[sl], A_log=A_log,
+                         S0=S0, z0=z0, S_out=So, z_out=zo)
+        args_list.append(a)
+    ws = hm.alloc_workspace(max(hm.hm_scan_workspace_size(a) for a in args_list))
+    for a in args_list:
+        a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    main = torch.cuda.current_stream()
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdt))
     d2h = ho.numel() * ho.element_size()
 
-    def step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        dtt.copy_(hdt, non_blocking=True)
-        hm.hm_scan_chunked_fwd(a, stream)
-        ho.copy_(o, non_blocking=True)
+    def step(e0, e1):
+        e0.record(main)
+        for st in (s_in, s_comp, s_out):
+            st.wait_event(e0)
+        done_in, done_comp = [], []
+        for i, (b0, b1, t0, t1) in enumerate(pieces):
+            sl = (slice(b0, b1), slice(t0, t1))
+            with torch.cuda.stream(s_in):
+                for dst, src in ((q, hq), (k, hk), (v, hv), (dtt, hdt)):
+                    dst[sl].copy_(src[sl], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(s_in)
+                done_in.append(ev)
+            s_comp.wait_event(done_in[i])
+            hm.hm_scan_chunked_fwd(args_list[i], s_comp)
+            ev = torch.cuda.Event()
+            ev.record(s_comp)
+            done_comp.append(ev)
+            s_out.wait_event(ev)
+            with torch.cuda.stream(s_out):
+                ho[sl].copy_(o[sl], non_blocking=True)
+        main.wait_stream(s_out)
+        main.wait_stream(s_comp)
+        e1.record(main)
 
     for _ in range(max(1, args.warmup)):
         flush.zero_()
-        step()
+        step(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     torch.cuda.synchronize()
+    assert hm.hm_get_device_error() == hm.HM_OK
     barrier(world)
     K = max(1, min(args.steps, 50))
     ts = []
     for _ in range(K):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        step()
-        e1.record(stream)
+        step(e0, e1)
         ts.append((e0, e1))
     torch.cuda.synchronize()
+    assert hm.hm_get_device_error() == hm.HM_OK
     barrier(world)
     ms = max_over_ranks(sum(x.elapsed_time(y) for x, y in ts) / K, world, torch)
     return {"value": B * L * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": K,
-            "call": "hm_scan_chunked_fwd (feature maps + scan) with pinned-host copies"}
+            "call": "hm_scan_chunked_fwd (feature maps + scan) per piece of %d, pinned-host copies "
+                    "pipelined on three streams" % len(pieces)}
 
 
 # ---------------------------------------------------------------- decode workload
