@@ -69,25 +69,59 @@ struct Geo {
 
 // ------------------------------------------------------------------ phase A
 
-constexpr int kABuild = 8;    // builder warps of the state kernel (8 tokens each)
+constexpr int kABuild = 8;              // builder warps of the state kernel
+constexpr int kAWB = 16 * 128;          // weight rows for z: [16 rows x 64 tokens] bf16, K-major
+constexpr int kAStageBudget = 200 * 1024;
 
 struct AAux {
-    float w[2][kC];
-    alignas(16) float zred[kABuild][kF];
-    float red[4];
-    float suf;         // sum of log a over the chunks already processed (later ones)
-    uint64_t full[2], empty[2], built, done;
+    float w[4][kC];    // weights of the chunk in each stage
+    uint64_t full[4], empty[4], built[4], wfull[4], done;
     uint32_t tmem;
     int abort;
 };
 
-constexpr int kAOffAux = 2 * (2 * kTileF + kTileV);
+// Stage layout of the state kernel: phiK (hi) [64 x 256], phiK lo when the
+// caller passes it, V [64 x 128] (overwritten by w (.) V, bf16 hi), the lo
+// part of w (.) V when the state is returned, and the weight rows of the z
+// product.  As many stages as fit the budget, at most 4.
+struct ALay {
+    int kl, v, vl, wb, stage, nst;
+};
+__host__ __device__ constexpr ALay a_layout(int split, int add_lo) {
+    ALay l{};
+    int o = kTileF;
+    l.kl = add_lo ? o : 0;
+    o += add_lo ? kTileF : 0;
+    l.v = o;
+    o += kTileV;
+    l.vl = split ? o : 0;
+    o += split ? kTileV : 0;
+    l.wb = o;
+    o += kAWB;
+    l.stage = o;
+    l.nst = kAStageBudget / o < 4 ? kAStageBudget / o : 4;
+    return l;
+}
+static_assert(a_layout(1, 1).nst >= 2 && a_layout(0, 0).nst == 4, "state kernel stages");
+
+constexpr int kAOffAux = kAStageBudget;
 constexpr int kASmem = kAOffAux + (int)sizeof(AAux) + 1024;
+static_assert(kASmem <= 227 * 1024, "phase A shared memory");
 
 // One CTA: (batch, head, value half, part).  Chunks of the part run from the
 // last to the first so that the suffix sums of log a (the weights relative to
-// the part end) are accumulated from small to large magnitudes.
-__global__ void __launch_bounds__(64 + 32 * kABuild, 1)
+// the part end) are accumulated from small to large magnitudes.  Per chunk:
+//   S_part^T += (w (.) V)^T phiK     (M = 128 value channels, N = 256 features)
+//   z_part   += phiK^T w             (M = the 128 features of the CTA's value
+//                                     half's index, N = 16: the weight rows
+//                                     w_hi, w_lo and 14 zero rows)
+// The builder warps only weight the CTA's 128 value channels; the z sums run
+// on the tensor cores, each value half taking half of the features; the
+// weights of the chunks come from one more warp that runs ahead of the
+// builders.
+constexpr int kAThreads = 64 + 32 * kABuild + 32;
+
+__global__ void __launch_bounds__(kAThreads, 1)
 scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constant__ CUtensorMap tmkl,
                   const __grid_constant__ CUtensorMap tmv, Geo g, const float *__restrict__ dt,
                   const float *__restrict__ A_log, int split, int add_lo, float *__restrict__ S_part,
@@ -105,21 +139,23 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
     const int c_first = part * g.part_chunks;
     const int c_last = min(g.nchunks, c_first + g.part_chunks) - 1;
     const int n = c_last - c_first + 1;
+    const ALay lay = a_layout(split, add_lo);
+    const int nst = lay.nst;
     volatile int *abort_flag = &X->abort;
-    auto stage = [&](int s) { return smem + s * (2 * kTileF + kTileV); };
+    auto stage = [&](int s) { return smem + s * lay.stage; };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < nst; ++s) {
             mbar_init(&X->full[s], 1);
             mbar_init(&X->empty[s], 1);
+            mbar_init(&X->built[s], kABuild);   // one arrival per builder warp
+            mbar_init(&X->wfull[s], 1);
         }
-        mbar_init(&X->built, 1);
         mbar_init(&X->done, 1);
         X->abort = 0;
-        X->suf = 0.f;
         mbar_fence_init();
     }
-    if (warp == 1) tmem_alloc(&X->tmem, 256);
+    if (warp == 1) tmem_alloc(&X->tmem, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -130,150 +166,188 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
             tma_prefetch_desc(&tmkh);
             tma_prefetch_desc(&tmkl);
             tma_prefetch_desc(&tmv);
-            int it = 0;
+            const uint32_t tx = kTileF + kTileV + (add_lo ? kTileF : 0);
+            int it = 0, s = 0;
+            uint32_t ph = 0;
             for (; it < n; ++it) {
-                const int s = it & 1;
-                if (!mbar_wait(&X->empty[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_STATE, 1)) break;
+                if (!mbar_wait(&X->empty[s], ph ^ 1, abort_flag, err, KID_SCAN_TC_STATE, 1)) break;
                 const int t0 = (c_last - it) * kC;
                 uint8_t *st = stage(s);
-                mbar_arrive_expect_tx(&X->full[s], add_lo ? 2 * kTileF + kTileV : kTileF + kTileV);
+                mbar_arrive_expect_tx(&X->full[s], tx);
                 for (int bb = 0; bb < 4; ++bb)
                     tma_load_4d(st + bb * kBlk, &tmkh, &X->full[s], bb * 64, h, t0, (int)b);
                 if (add_lo)
                     for (int bb = 0; bb < 4; ++bb)
-                        tma_load_4d(st + kTileF + bb * kBlk, &tmkl, &X->full[s], bb * 64, h, t0, (int)b);
+                        tma_load_4d(st + lay.kl + bb * kBlk, &tmkl, &X->full[s], bb * 64, h, t0, (int)b);
                 for (int bb = 0; bb < 2; ++bb)
-                    tma_load_4d(st + 2 * kTileF + bb * kBlk, &tmv, &X->full[s], dv0 + bb * 64, h, t0, (int)b);
+                    tma_load_4d(st + lay.v + bb * kBlk, &tmv, &X->full[s], dv0 + bb * 64, h, t0, (int)b);
+                if (++s == nst) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
-            for (int j = it - 2; j < it; ++j) {
-                if (j < 0) continue;
+            // on an early exit, the loads still in flight land before the CTA ends
+            for (int j = max(0, it - nst); j < it; ++j) {
                 for (uint32_t i = 0; i < kWaitPolls; ++i)
-                    if (mbar_try_wait(&X->full[j & 1], (j >> 1) & 1)) break;
+                    if (mbar_try_wait(&X->full[j % nst], (j / nst) & 1)) break;
             }
         }
     } else if (warp == 1) {
         if (elect_one()) {
-            constexpr uint32_t idesc = idesc_bf16(128, 256, true, true);
+            constexpr uint32_t idS = idesc_bf16(128, 256, true, true);
+            constexpr uint32_t idZ = idesc_bf16(128, 16, true, false);
+            int s = 0;
+            uint32_t ph = 0;
             for (int it = 0; it < n; ++it) {
-                const int s = it & 1;
-                if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_STATE, 2)) break;
-                if (!mbar_wait(&X->built, it & 1, abort_flag, err, KID_SCAN_TC_STATE, 3)) break;
+                if (!mbar_wait(&X->full[s], ph, abort_flag, err, KID_SCAN_TC_STATE, 2)) break;
+                if (!mbar_wait(&X->built[s], ph, abort_flag, err, KID_SCAN_TC_STATE, 3)) break;
                 tc_fence_after();
                 const uint32_t kh = smem_u32(stage(s));
-                const uint32_t kl = kh + kTileF;
-                const uint32_t vv = kh + 2 * kTileF;
+                const uint32_t kl = kh + lay.kl, vv = kh + lay.v, vl = kh + lay.vl, wb = kh + lay.wb;
                 for (int k = 0; k < kC / 16; ++k) {
-                    const uint64_t ad = desc_mn_sw128(vv + k * 2048, kBlk, 1024);
-                    mma_ss(tmem, ad, desc_mn_sw128(kh + k * 2048, kBlk, 1024), idesc,
-                           (it > 0 || k > 0) ? 1u : 0u);
-                    if (split) mma_ss(tmem, ad, desc_mn_sw128(kl + k * 2048, kBlk, 1024), idesc, 1u);
+                    const uint32_t acc = (it > 0 || k > 0) ? 1u : 0u;
+                    const uint64_t bk = desc_mn_sw128(kh + k * 2048, kBlk, 1024);
+                    const uint64_t av = desc_mn_sw128(vv + k * 2048, kBlk, 1024);
+                    mma_ss(tmem, av, bk, idS, acc);
+                    if (split) mma_ss(tmem, desc_mn_sw128(vl + k * 2048, kBlk, 1024), bk, idS, 1u);
+                    if (add_lo) mma_ss(tmem, av, desc_mn_sw128(kl + k * 2048, kBlk, 1024), idS, 1u);
+                    const uint64_t bw = desc_k_sw128(wb + k * 32);
+                    mma_ss(tmem + 256, desc_mn_sw128(kh + half * 2 * kBlk + k * 2048, kBlk, 1024), bw, idZ, acc);
+                    if (add_lo)
+                        mma_ss(tmem + 256, desc_mn_sw128(kl + half * 2 * kBlk + k * 2048, kBlk, 1024), bw, idZ, 1u);
                 }
                 mma_commit(&X->empty[s]);
+                if (++s == nst) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
             mma_commit(&X->done);
+            // TMEM is released only after the issued MMAs have completed
+            for (uint32_t i = 0; i < kWaitPolls; ++i)
+                if (mbar_try_wait(&X->done, 0)) break;
         }
-    } else {
-        // builders: warps 2..9 (256 threads).  Thread: one 16-byte chunk (8
-        // features) of the 256-feature row (lane -> block, chunk) for the 8
-        // tokens of its warp's group.
-        constexpr int kNB = 32 * kABuild;
-        constexpr int kTok = kC / kABuild;
-        const int tb = threadIdx.x - 64;
-        const int bb = lane >> 3, cc = lane & 7;
-        const int tg = tb >> 5;
+    } else if (warp == 2 + kABuild) {
+        // weights: w_j = exp(sum of log a over the tokens after j up to the
+        // part end); lane: tokens 2 lane and 2 lane + 1 of each chunk
         const float alog = dt ? A_log[h] : 0.f;
-        float za[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) za[e] = 0.f;
-        // dt is fetched a chunk ahead and turned into log a when used (-inf:
-        // log a = 0 past the end of the sequence or without dt)
-        auto token_dt = [&](int t0) {
-            return (tb < kC && dt && t0 + tb < g.L) ? dt[(b * g.L + t0 + tb) * g.H + h] : -INFINITY;
+        // dt of the chunk it + i in da[i], db[i] (fetched four chunks ahead)
+        auto token_dt = [&](int it, int j) {
+            const int64_t t = (int64_t)(c_last - it) * kC + j;
+            return (dt && it < n && t < g.L) ? dt[(b * g.L + t) * g.H + h] : -INFINITY;
         };
-        float dt_next = token_dt(c_last * kC);
-        bool ok = true;
+        float da[4], db[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            da[i] = token_dt(i, 2 * lane);
+            db[i] = token_dt(i, 2 * lane + 1);
+        }
+        float suf = 0.f;
+        int s = 0;
+        uint32_t ph = 0;
+        bool okw = true;
         for (int it = 0; it < n; ++it) {
-            const int s = it & 1;
-            const float l = hm_log_decay(dt_next, alog);
-            if (it + 1 < n) dt_next = token_dt((c_last - it - 1) * kC);
-            // exclusive suffix sums of log a within the chunk
-            float x = l;  // inclusive suffix sum within the warp
+            const float l0 = hm_log_decay(da[0], alog), l1 = hm_log_decay(db[0], alog);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                da[i] = da[i + 1];
+                db[i] = db[i + 1];
+            }
+            da[3] = token_dt(it + 4, 2 * lane);
+            db[3] = token_dt(it + 4, 2 * lane + 1);
+            // inclusive suffix sums of the token pairs over the lanes
+            const float pair = l0 + l1;
+            float x = pair;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                float y = __shfl_down_sync(0xffffffffu, x, o);
+                const float y = __shfl_down_sync(0xffffffffu, x, o);
                 if (lane + o < 32) x += y;
             }
-            if (tb == 32) X->red[0] = x;       // sum over tokens 32..63
-            named_sync(1, kNB);
-            if (tb < 32) x += X->red[0];
-            // exclusive suffix: the inclusive value of the next token
-            float ex = __shfl_down_sync(0xffffffffu, x, 1);
-            if (lane == 31) ex = (tb == 31) ? X->red[0] : 0.f;
-            if (tb == 0) X->red[2] = x;        // chunk total
-            const float suf = X->suf;
-            if (tb < kC) X->w[s][tb] = fexp(suf + ex);
-            named_sync(1, kNB);
-            if (tb == 0) X->suf = suf + X->red[2];
-            if (!mbar_wait(&X->full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_STATE, 4)) {
+            const float tot = __shfl_sync(0xffffffffu, x, 0);
+            const float ex1 = x - pair;   // tokens after 2 lane + 1
+            const float ex0 = ex1 + l1;   // tokens after 2 lane
+            // the stage's weights were last read by the build of chunk it - nst
+            if (it >= nst) okw = mbar_wait(&X->built[s], ph ^ 1, abort_flag, err, KID_SCAN_TC_STATE, 6);
+            okw = __all_sync(0xffffffffu, okw);
+            if (!okw) break;
+            *reinterpret_cast<float2 *>(&X->w[s][2 * lane]) = make_float2(fexp(suf + ex0), fexp(suf + ex1));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->wfull[s]);
+            suf += tot;
+            if (++s == nst) {
+                s = 0;
+                ph ^= 1;
+            }
+        }
+        if (okw && half == 0 && lane == 0) lsum_part[bh * g.NPc + part] = suf;
+    } else {
+        // builders: warps 2..9 (256 threads).  Thread: one 16-byte chunk (8
+        // channels) of four consecutive token rows of V.
+        constexpr int kNB = 32 * kABuild;
+        const int tb = threadIdx.x - 64;
+        const int vb = (tb >> 3) & 1, vc = tb & 7, r0 = (tb >> 4) * 4;
+        // zero rows 2..15 of every stage's weight tile (rows 0 and 1 are
+        // rewritten for each chunk)
+        for (int i = tb; i < nst * (kAWB - 256) / 16; i += kNB) {
+            const int st = i / ((kAWB - 256) / 16), r = i % ((kAWB - 256) / 16);
+            *reinterpret_cast<uint4 *>(stage(st) + lay.wb + 256 + r * 16) = make_uint4(0, 0, 0, 0);
+        }
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int it = 0; it < n; ++it) {
+            // each builder warp runs on its own (no named barrier in the loop)
+            bool okw = mbar_wait(&X->wfull[s], ph, abort_flag, err, KID_SCAN_TC_STATE, 7) &&
+                       mbar_wait(&X->full[s], ph, abort_flag, err, KID_SCAN_TC_STATE, 4);
+            if (!__all_sync(0xffffffffu, okw)) {
                 ok = false;
                 break;
             }
-            // weighted features, split into bf16 hi + lo, written back in place
-            // (8 rows loaded at a time)
-            uint8_t *__restrict__ kh = stage(s) + bb * kBlk;
-            uint8_t *__restrict__ kl = kh + kTileF;
+            uint8_t *const st = stage(s);
             const float *__restrict__ wv = X->w[s];
-#pragma unroll 1
-            for (int j0 = tg * kTok; j0 < tg * kTok + kTok; j0 += 8) {
-                uint4 vh[8], vl[8];
+            // weight rows of the z product: row 0 = bf16(w), row 1 = the remainder
+            if (tb < kC) {
+                const float wmine = wv[tb];
+                const __nv_bfloat16 wh = __float2bfloat16_rn(wmine);
+                const __nv_bfloat16 wl = __float2bfloat16_rn(wmine - __bfloat162float(wh));
+                const int c8 = tb >> 3, e = tb & 7;
+                *reinterpret_cast<__nv_bfloat16 *>(st + lay.wb + (c8 << 4) + 2 * e) = wh;
+                *reinterpret_cast<__nv_bfloat16 *>(st + lay.wb + 128 + ((c8 ^ 1) << 4) + 2 * e) = wl;
+            }
+            // w (.) V in place as bf16, the rounding remainder into its own tile
+            uint8_t *__restrict__ vt = st + lay.v + vb * kBlk;
+            uint8_t *__restrict__ vlt = st + lay.vl + vb * kBlk;
+            uint4 xv[4];
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const uint32_t off = sw128_off(j0 + jj, cc);
-                    vh[jj] = *reinterpret_cast<const uint4 *>(kh + off);
-                    vl[jj] = add_lo ? *reinterpret_cast<const uint4 *>(kl + off) : make_uint4(0, 0, 0, 0);
-                }
+            for (int jj = 0; jj < 4; ++jj) xv[jj] = *reinterpret_cast<const uint4 *>(vt + sw128_off(r0 + jj, vc));
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    uint32_t *ph = reinterpret_cast<uint32_t *>(&vh[jj]);
-                    uint32_t *pl = reinterpret_cast<uint32_t *>(&vl[jj]);
-                    const float wj = wv[j0 + jj];
+            for (int jj = 0; jj < 4; ++jj) {
+                uint32_t *ph32 = reinterpret_cast<uint32_t *>(&xv[jj]);
+                uint4 lo;
+                uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+                const float wj = wv[r0 + jj];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float2 k = unpack_bf16x2(ph[e]);
-                        if (add_lo) {
-                            const float2 k2 = unpack_bf16x2(pl[e]);
-                            k.x += k2.x;
-                            k.y += k2.y;
-                        }
-                        const float kt0 = wj * k.x, kt1 = wj * k.y;
-                        ph[e] = pack_bf16x2(kt0, kt1);
-                        const float2 hf = unpack_bf16x2(ph[e]);
-                        if (split) {
-                            pl[e] = pack_bf16x2(kt0 - hf.x, kt1 - hf.y);
-                            za[2 * e] += kt0;
-                            za[2 * e + 1] += kt1;
-                        } else {
-                            za[2 * e] += hf.x;
-                            za[2 * e + 1] += hf.y;
-                        }
+                for (int e = 0; e < 4; ++e) {
+                    const float2 vv = unpack_bf16x2(ph32[e]);
+                    const float t0 = wj * vv.x, t1 = wj * vv.y;
+                    ph32[e] = pack_bf16x2(t0, t1);
+                    if (split) {
+                        const float2 hf = unpack_bf16x2(ph32[e]);
+                        pl[e] = pack_bf16x2(t0 - hf.x, t1 - hf.y);
                     }
                 }
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const uint32_t off = sw128_off(j0 + jj, cc);
-                    *reinterpret_cast<uint4 *>(kh + off) = vh[jj];
-                    if (split) *reinterpret_cast<uint4 *>(kl + off) = vl[jj];
-                }
+                const uint32_t off = sw128_off(r0 + jj, vc);
+                *reinterpret_cast<uint4 *>(vt + off) = xv[jj];
+                if (split) *reinterpret_cast<uint4 *>(vlt + off) = lo;
             }
             fence_proxy_async_smem();
-            named_sync(1, kNB);
-            if (tb == 0) mbar_arrive(&X->built);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->built[s]);
+            if (++s == nst) {
+                s = 0;
+                ph ^= 1;
+            }
         }
-        // z of the part: reduce the four token groups' partial sums
-        const int f0 = bb * 64 + cc * 8;
-        *reinterpret_cast<float4 *>(&X->zred[tg][f0]) = make_float4(za[0], za[1], za[2], za[3]);
-        *reinterpret_cast<float4 *>(&X->zred[tg][f0 + 4]) = make_float4(za[4], za[5], za[6], za[7]);
-        named_sync(1, kNB);
         if (ok && mbar_wait(&X->done, 0, abort_flag, err, KID_SCAN_TC_STATE, 5)) {
             tc_fence_after();
             // two warps per TMEM lane quarter: features 0..127 and 128..255
@@ -289,12 +363,12 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
 #pragma unroll
                 for (int j = 0; j < 32; ++j) Sp[(int64_t)(c0 + j) * g.dv] = __uint_as_float(r[j]);
             }
-            if (half == 0) {
-                float zs = 0.f;
-#pragma unroll
-                for (int t = 0; t < kABuild; ++t) zs += X->zred[t][tb];
-                z_part[pidx * kF + tb] = zs;
-                if (tb == 0) lsum_part[pidx] = X->suf;
+            if (fh == 0) {
+                // z: TMEM lane = feature within the CTA's half, columns 0 (w hi) and 1 (w lo)
+                uint32_t r[16];
+                tmem_ld16(tmem + 256 + ((uint32_t)(32 * q) << 16), r);
+                tmem_wait_ld();
+                z_part[pidx * kF + half * 128 + ch] = __uint_as_float(r[0]) + __uint_as_float(r[1]);
             }
         }
     }
@@ -303,61 +377,84 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
 // ------------------------------------------------------------------ phase B
 
-// Per (batch, head) and group of 4 state elements: walks the parts in order,
+// Per (batch, head) and 4-element groups of the state: walks the parts in
+// order,
 //   acc <- exp(lsum_p) acc + part_p,
 // storing the state at each segment start and, when every part was
 // computed, the final state.  Elements [0, F*dv) are S, [F*dv, F*dv + F) are z.
-// The parts' values are loaded 8 at a time ahead of the dependent chain.
-__global__ void __launch_bounds__(256)
+// A thread owns kCarryCols groups, 256 apart (coalesced), and loads the next
+// part of all of them while it combines the current one, so that enough bytes
+// are in flight to stream the parts at HBM speed.
+constexpr int kCarryCols = 4;
+
+__global__ void __launch_bounds__(256, 4)
 scan_carry_kernel(Geo g, const float *__restrict__ S_part, const float *__restrict__ z_part,
                   const float *__restrict__ lsum_part, const float *__restrict__ S0, const float *__restrict__ z0,
                   float *__restrict__ S_start, float *__restrict__ z_start, float *__restrict__ S_out,
                   float *__restrict__ z_out) {
     const int64_t bh = blockIdx.y;
-    const int64_t nS = (int64_t)kF * g.dv;
-    const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-    if (e >= nS + kF) return;
-    const bool isz = e >= nS;
-    const int64_t idx = isz ? e - nS : e;
-    const int64_t pstride = isz ? kF : nS;
-    const float *part = (isz ? z_part + bh * g.NPc * (int64_t)kF : S_part + bh * g.NPc * nS) + idx;
-    float *start = (isz ? z_start + bh * g.G * (int64_t)kF : S_start + bh * g.G * nS) + idx;
-    const float *init = isz ? (z0 ? z0 + bh * kF + idx : nullptr) : (S0 ? S0 + bh * nS + idx : nullptr);
-    float4 acc = init ? *reinterpret_cast<const float4 *>(init) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int nS = kF * g.dv;
     const int pps = g.seg_chunks / g.part_chunks;
-    for (int p0 = 0; p0 <= g.NPc; p0 += 8) {
-        float4 v[8];
-        float lg[8];
+    // group j: element e = 4 * col; S element e, or z element e - nS
+    int col[kCarryCols];
+    float4 acc[kCarryCols], cur[kCarryCols];
+    auto elem = [&](const float *S, const float *z, int64_t blk, int c) -> const float * {
+        const int e = 4 * c;
+        return e < nS ? S + blk * nS + e : z + blk * kF + (e - nS);
+    };
+    auto elem_w = [&](float *S, float *z, int64_t blk, int c) -> float * {
+        const int e = 4 * c;
+        return e < nS ? S + blk * nS + e : z + blk * kF + (e - nS);
+    };
+    const int ncol = (nS + kF) / 4;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int p = p0 + u;
-            if (p < g.NPc) {
-                v[u] = *reinterpret_cast<const float4 *>(part + (int64_t)p * pstride);
-                lg[u] = lsum_part[bh * g.NPc + p];
-            }
+    for (int j = 0; j < kCarryCols; ++j) {
+        col[j] = (blockIdx.x * kCarryCols + j) * blockDim.x + threadIdx.x;
+        acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        cur[j] = acc[j];
+        if (col[j] < ncol) {
+            const bool isz = 4 * col[j] >= nS;
+            if (isz ? z0 != nullptr : S0 != nullptr)
+                acc[j] = *reinterpret_cast<const float4 *>(elem(S0, z0, bh, col[j]));
+            if (g.NPc > 0) cur[j] = *reinterpret_cast<const float4 *>(elem(S_part, z_part, bh * g.NPc, col[j]));
         }
+    }
+    for (int p = 0; p <= g.NPc; ++p) {
+        if (p > 0 && p % pps == 0 && p / pps < g.G) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int p = p0 + u;
-            if (p > g.NPc) break;
-            if (p > 0 && p % pps == 0 && p / pps < g.G)
-                *reinterpret_cast<float4 *>(start + (int64_t)(p / pps) * pstride) = acc;
-            if (p < g.NPc) {
-                const float gam = expf(lg[u]);
-                acc = make_float4(fmaf(gam, acc.x, v[u].x), fmaf(gam, acc.y, v[u].y), fmaf(gam, acc.z, v[u].z),
-                                  fmaf(gam, acc.w, v[u].w));
-            }
+            for (int j = 0; j < kCarryCols; ++j)
+                if (col[j] < ncol)
+                    *reinterpret_cast<float4 *>(elem_w(S_start, z_start, bh * g.G + p / pps, col[j])) = acc[j];
+        }
+        if (p == g.NPc) break;
+        float4 nxt[kCarryCols];
+#pragma unroll
+        for (int j = 0; j < kCarryCols; ++j)
+            nxt[j] = (col[j] < ncol && p + 1 < g.NPc)
+                         ? *reinterpret_cast<const float4 *>(elem(S_part, z_part, bh * g.NPc + p + 1, col[j]))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float gam = expf(lsum_part[bh * g.NPc + p]);
+#pragma unroll
+        for (int j = 0; j < kCarryCols; ++j) {
+            acc[j] = make_float4(fmaf(gam, acc[j].x, cur[j].x), fmaf(gam, acc[j].y, cur[j].y),
+                                 fmaf(gam, acc[j].z, cur[j].z), fmaf(gam, acc[j].w, cur[j].w));
+            cur[j] = nxt[j];
         }
     }
     if (g.NPc == g.NP) {
-        float *out = isz ? (z_out ? z_out + bh * kF + idx : nullptr) : (S_out ? S_out + bh * nS + idx : nullptr);
-        if (out) *reinterpret_cast<float4 *>(out) = acc;
+#pragma unroll
+        for (int j = 0; j < kCarryCols; ++j) {
+            if (col[j] >= ncol) continue;
+            const bool isz = 4 * col[j] >= nS;
+            if (isz ? z_out != nullptr : S_out != nullptr)
+                *reinterpret_cast<float4 *>(elem_w(S_out, z_out, bh, col[j])) = acc[j];
+        }
     }
 }
 
@@ -1193,11 +1290,11 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
         e = ensure_smem_limit(scan_state_kernel, kASmem);
         if (e != cudaSuccess) return e;
         const unsigned grid = (unsigned)(2 * g.NPc * BH);
-        scan_state_kernel<<<grid, 64 + 32 * kABuild, kASmem, s>>>(tk, tkl, tv, g, c.dt, c.A_log, split ? 1 : 0,
+        scan_state_kernel<<<grid, kAThreads, kASmem, s>>>(tk, tkl, tv, g, c.dt, c.A_log, split ? 1 : 0,
                                                     add_lo ? 1 : 0, S_part, z_part, lsum, err);
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        dim3 gb((unsigned)(((nS + kF) / 4 + 255) / 256), (unsigned)BH);
+        dim3 gb((unsigned)(((nS + kF) / 4 + 256 * kCarryCols - 1) / (256 * kCarryCols)), (unsigned)BH);
         scan_carry_kernel<<<gb, 256, 0, s>>>(g, S_part, z_part, lsum, c.S0, c.z0, S_start, z_start,
                                              c.S_out, c.z_out);
         count_launches(1);

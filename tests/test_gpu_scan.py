@@ -118,6 +118,9 @@ def test_bf16_initial_state_and_split_invariance(hm):
 
 
 def test_bf16_pythia_full_size(hm):
+    # with the final state returned (the state phase covers every part, with
+    # hi / lo splits) and without it (the timed prefill call: the state phase
+    # covers the first segment only)
     cfg = wl.PREFILL_PYTHIA
     inp = wl.scan_inputs(cfg)
     o, S, z = run_scan(hm, inp, "bf16", want_state=True)
@@ -125,6 +128,23 @@ def test_bf16_pythia_full_size(hm):
     assert rel_err(o, o_ref) <= TOL_BF16
     assert rel_err(S, S_ref) <= TOL_BF16
     assert rel_err(z, z_ref) <= TOL_BF16
+    o2, _, _ = run_scan(hm, inp, "bf16")
+    assert rel_err(o2, o_ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("L", [512, 1000])
+def test_bf16_two_segments_with_initial_state(hm, L):
+    # 32 heads: two output segments; the initial state enters segment 0
+    # directly and segment 1 through the state parts and the carry
+    cfg = wl.PREFILL_PYTHIA
+    inp = wl.scan_inputs(cfg, L=L, seed=300 + L)
+    B = inp["q"].shape[0]
+    F = 2 * cfg.p
+    S0 = wl.round_f32(wl.normal(300 + L, "S0", (B, cfg.H, F, cfg.dv)) * 0.5)
+    z0 = wl.round_f32(np.abs(wl.normal(300 + L, "z0", (B, cfg.H, F))) + 0.1)
+    o, _, _ = run_scan(hm, inp, "bf16", S0=S0, z0=z0)
+    o_ref, _, _ = _oracle(inp, S0=S0, z0=z0)
+    assert rel_err(o, o_ref) <= TOL_BF16
 
 
 def test_bf16_long_context_full_size_sampled_heads(hm):
@@ -132,6 +152,7 @@ def test_bf16_long_context_full_size_sampled_heads(hm):
     cfg = wl.PREFILL_LONG
     inp = wl.scan_inputs(cfg)
     o, S, z = run_scan(hm, inp, "bf16", want_state=True)
+    o2, _, _ = run_scan(hm, inp, "bf16")   # the timed call: no returned state
     for h in (0, 5):
         sub = {k: (v[:, :, h:h + 1] if k in ("q", "k", "v", "dt") else
                    (v[h:h + 1] if k == "A_log" else v)) for k, v in inp.items()}
@@ -139,6 +160,7 @@ def test_bf16_long_context_full_size_sampled_heads(hm):
         assert rel_err(o[:, :, h:h + 1], o_ref) <= TOL_BF16
         assert rel_err(S[:, h:h + 1], S_ref) <= TOL_BF16
         assert rel_err(z[:, h:h + 1], z_ref) <= TOL_BF16
+        assert rel_err(o2[:, :, h:h + 1], o_ref) <= TOL_BF16
 
 
 # ------------------------------------------------------------------ closed forms and degenerate cases
