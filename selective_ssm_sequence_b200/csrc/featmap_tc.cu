@@ -12,12 +12,12 @@
 //   warps 2..13 three epilogue warpgroups taking tiles in turn: one
 //               accumulator row per thread, read from TMEM in two passes (a
 //               running max / normaliser, then the normalised features), the
-//               negate / concatenate / softmax in registers, and the store.
-//               The epilogue is latency-bound (exponentials and TMEM loads of
-//               one row per thread), so three warps per SM sub-partition
-//               share the work.
-// Four TMEM accumulators let the MMAs run ahead of both epilogue warpgroups.
-// The kernel is bound by HBM (x in, phi out); MMA and exp work hide under it.
+//               negate / concatenate / softmax in registers in the log2
+//               domain (one FMA-free exp2 per feature).  bf16 features leave
+//               through a per-warpgroup staging buffer and TMA stores of 128
+//               rows x 64 bytes: a thread owns a row, so direct stores would
+//               touch 32 rows (4 KB apart) per instruction.
+// Four TMEM accumulators let the MMAs run ahead of the epilogue warpgroups.
 #include "tc_common.cuh"
 
 namespace hm {
@@ -39,8 +39,11 @@ struct FmLayout {
     static constexpr int kXBytes = kChunks * kXChunkBytes;  // one x tile
     static constexpr int kOffW = 0;
     static constexpr int kOffX = kWBytes;
-    static constexpr int kOffBar = kOffX + kStages * kXBytes;
+    static constexpr int kStgBytes = kBM * 64;               // output staging: 128 rows x 32 bf16
+    static constexpr int kOffStg = kOffX + kStages * kXBytes;
+    static constexpr int kOffBar = kOffStg + kEpiWG * kStgBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;      // + barriers, + alignment slack
+    static_assert(kSmem <= 227 * 1024, "feature-map shared memory");
     static constexpr int kAcc = 512 / P >= 4 ? 4 : 2;       // TMEM accumulators
     static constexpr int kTmemCols = kAcc * P <= 256 ? 256 : 512;
 };
@@ -55,12 +58,13 @@ struct FmBars {
     int abort;
 };
 
-__device__ __forceinline__ float fexp(float x) { return exp2f(x * 1.4426950408889634f); }
+constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D, int P, typename TP>
+template <int D, int P, typename TP, bool kHasBias>
 __global__ void __launch_bounds__(kThreads, 1)
 featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constant__ CUtensorMap tmw0,
                   const __grid_constant__ CUtensorMap tmx1, const __grid_constant__ CUtensorMap tmw1,
+                  const __grid_constant__ CUtensorMap tmo0, const __grid_constant__ CUtensorMap tmo1,
                   int64_t Tv, int Hv, const float *__restrict__ bias0, const float *__restrict__ bias1,
                   int bias_per_head, TP *__restrict__ phi0, TP *__restrict__ phi1,
                   __nv_bfloat16 *__restrict__ phi_lo0, __nv_bfloat16 *__restrict__ phi_lo1, DevErr err) {
@@ -69,6 +73,7 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constan
     const bool second = blockIdx.z != 0;
     const CUtensorMap &tmx = second ? tmx1 : tmx0;
     const CUtensorMap &tmw = second ? tmw1 : tmw0;
+    const CUtensorMap &tmo = second ? tmo1 : tmo0;   // phi as (F, H, rows), 64-byte swizzle (bf16 phi)
     const float *__restrict__ bias = second ? bias1 : bias0;
     TP *__restrict__ phi = second ? phi1 : phi0;
     __nv_bfloat16 *__restrict__ phi_lo = second ? phi_lo1 : phi_lo0;
@@ -168,6 +173,8 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constan
         const int e = (warp - 2) >> 2;
         const int q = warp & 3;              // TMEM lane quarter of this warp
         const int row_in_tile = q * 32 + lane;
+        const int wt = threadIdx.x - 64 - 128 * e;   // thread within the warpgroup
+        uint8_t *const stg = smem + Lay::kOffStg + e * Lay::kStgBytes;
         constexpr int F = 2 * P;
         const float *bh = bias ? bias + (bias_per_head ? (int64_t)h * P : 0) : nullptr;
         int it = e;
@@ -175,91 +182,142 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constan
              tile += (int64_t)kEpiWG * gridDim.x, it += kEpiWG) {
             const int b = it % NA;
             const uint32_t bph = (it / NA) & 1;
-            if (!mbar_wait(&bars->accf[b], bph, abort_flag, err, KID_FEATMAP_TC, 5)) break;
+            const bool okw = mbar_wait(&bars->accf[b], bph, abort_flag, err, KID_FEATMAP_TC, 5);
+            // the warpgroup leaves together (its threads meet at named barriers)
+            if (!named_sync_and(1 + e, 128, okw)) break;
             tc_fence_after();
             const uint32_t tbase = tmem + b * P + ((uint32_t)(q * 32) << 16);
-            // pass 1: running max m of |u| and normaliser Z = sum exp(u - m) + exp(-u - m),
-            // rescaled whenever m grows (one extra exp per 32 columns)
-            float m = 0.f, Z = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < P; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tbase + c, r);
-                tmem_wait_ld();
-                float mc = m;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) mc = fmaxf(mc, fabsf(__uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f)));
-                float zc = 0.f;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float u = __uint_as_float(r[j]) + (bh ? bh[c + j] : 0.f);
-                    zc += fexp(u - mc) + fexp(-u - mc);
-                }
-                Z = Z * fexp(m - mc) + zc;
-                m = mc;
-            }
-            const float inv = 1.f / Z;
             const int64_t t = tile * kBM + row_in_tile;
             const bool valid = t < Tv;
             TP *out = phi + (t * Hv + h) * (int64_t)F;
-            __nv_bfloat16 *lo = phi_lo ? phi_lo + (t * Hv + h) * (int64_t)F : nullptr;
-            // pass 2: normalised features, stored
-#pragma unroll 1
-            for (int c = 0; c < P; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tbase + c, r);
-                tmem_wait_ld();
-                if (c + 32 >= P) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->acce[b]);   // last read of this accumulator
+            __nv_bfloat16 *lo = (phi_lo && valid) ? phi_lo + (t * Hv + h) * (int64_t)F : nullptr;
+            // Everything in the log2 domain: y = u log2(e).  Pass 1: running max
+            // m of |y| and normaliser Z = sum 2^(y - m) + 2^(-y - m), rescaled
+            // when m grows.  Pass 2: phi = 2^(+-y - sh) with sh = m + log2 Z, so
+            // the normalisation costs nothing per feature.  The TMEM load of
+            // the next 32 columns is in flight while a block is processed.
+            auto yv = [&](const uint32_t *r, int c, int j) {
+                return (__uint_as_float(r[j]) + ((kHasBias && bh) ? bh[c + j] : 0.f)) * kLog2e;
+            };
+            float m = 0.f, Z = 0.f;
+            auto pass1 = [&](const uint32_t *r, int c) {
+                float mc = m;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mc = fmaxf(mc, fabsf(yv(r, c, j)));
+                float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const float y0 = yv(r, c, j), y1 = yv(r, c, j + 1);
+                    z0 += ex2_approx(y0 - mc) + ex2_approx(-y0 - mc);
+                    z1 += ex2_approx(y1 - mc) + ex2_approx(-y1 - mc);
                 }
-                if (!valid) continue;
+                Z = Z * ex2_approx(m - mc) + (z0 + z1);
+                m = mc;
+            };
+            {
+                uint32_t ra[32], rb[32];
+                tmem_ld32(tbase, ra);
+                tmem_wait_ld();
+#pragma unroll 1
+                for (int c = 0; c < P; c += 64) {
+                    tmem_ld32(tbase + c + 32, rb);
+                    pass1(ra, c);
+                    tmem_wait_ld();
+                    if (c + 64 < P) tmem_ld32(tbase + c + 64, ra);
+                    pass1(rb, c + 32);
+                    tmem_wait_ld();
+                }
+            }
+            const float sh = m + lg2_approx(Z);
+            if constexpr (sizeof(TP) == 2) {
+                // bf16 phi: each half of a 32-column block (32 features of one
+                // row per thread) goes through the warpgroup's staging buffer
+                // (64-byte rows, 64-byte swizzle: conflict-free 16-byte writes)
+                // and leaves by one TMA store of 128 rows x 64 bytes
+                auto stage_half = [&](const uint32_t *r, int c, int hf) {
+                    uint32_t pk[16];
+                    const float sg = hf ? -1.f : 1.f;
+                    uint32_t lw[4];
 #pragma unroll
-                for (int j0 = 0; j0 < 32; j0 += 8) {
-                    float e1[8], e2[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float u = __uint_as_float(r[j0 + j]) + (bh ? bh[c + j0 + j] : 0.f);
-                        e1[j] = fexp(u - m) * inv;
-                        e2[j] = fexp(-u - m) * inv;
-                    }
-                    if constexpr (sizeof(TP) == 2) {
-                        uint4 v1, v2;
-                        uint32_t *p1 = reinterpret_cast<uint32_t *>(&v1);
-                        uint32_t *p2 = reinterpret_cast<uint32_t *>(&v2);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            p1[j] = pack_bf16x2(e1[2 * j], e1[2 * j + 1]);
-                            p2[j] = pack_bf16x2(e2[2 * j], e2[2 * j + 1]);
-                        }
-                        *reinterpret_cast<uint4 *>(out + c + j0) = v1;
-                        *reinterpret_cast<uint4 *>(out + P + c + j0) = v2;
+                    for (int j = 0; j < 16; ++j) {
+                        const float y0 = sg * yv(r, c, 2 * j), y1 = sg * yv(r, c, 2 * j + 1);
+                        const float p0 = ex2_approx(y0 - sh), p1 = ex2_approx(y1 - sh);
+                        pk[j] = pack_bf16x2(p0, p1);
                         if (lo) {
                             // remainder phi - bf16(phi), so that hi + lo carries ~16 bits
-                            uint4 l1, l2;
-                            uint32_t *q1 = reinterpret_cast<uint32_t *>(&l1);
-                            uint32_t *q2 = reinterpret_cast<uint32_t *>(&l2);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float2 h1 = unpack_bf16x2(p1[j]), h2 = unpack_bf16x2(p2[j]);
-                                q1[j] = pack_bf16x2(e1[2 * j] - h1.x, e1[2 * j + 1] - h1.y);
-                                q2[j] = pack_bf16x2(e2[2 * j] - h2.x, e2[2 * j + 1] - h2.y);
-                            }
-                            *reinterpret_cast<uint4 *>(lo + c + j0) = l1;
-                            *reinterpret_cast<uint4 *>(lo + P + c + j0) = l2;
+                            const float2 hv = unpack_bf16x2(pk[j]);
+                            lw[j & 3] = pack_bf16x2(p0 - hv.x, p1 - hv.y);
+                            if ((j & 3) == 3)
+                                *reinterpret_cast<uint4 *>(lo + hf * P + c + 2 * (j - 3)) =
+                                    make_uint4(lw[0], lw[1], lw[2], lw[3]);
                         }
-                    } else {
-                        float4 *o1 = reinterpret_cast<float4 *>(out + c + j0);
-                        float4 *o2 = reinterpret_cast<float4 *>(out + P + c + j0);
-                        o1[0] = make_float4(e1[0], e1[1], e1[2], e1[3]);
-                        o1[1] = make_float4(e1[4], e1[5], e1[6], e1[7]);
-                        o2[0] = make_float4(e2[0], e2[1], e2[2], e2[3]);
-                        o2[1] = make_float4(e2[4], e2[5], e2[6], e2[7]);
                     }
+                    if (wt == 0) bulk_wait_read_all();   // the previous store has read the buffer
+                    named_sync(1 + e, 128);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int pc = j ^ ((row_in_tile >> 1) & 3);
+                        *reinterpret_cast<uint4 *>(stg + row_in_tile * 64 + pc * 16) =
+                            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    named_sync(1 + e, 128);
+                    if (wt == 0) {
+                        tma_store_3d(&tmo, stg, hf * P + c, h, (int)(tile * kBM));
+                        bulk_commit();
+                    }
+                };
+#pragma unroll 1
+                for (int c = 0; c < P; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c, r);
+                    tmem_wait_ld();
+                    if (c + 32 >= P) {
+                        // the last read of this accumulator has landed
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars->acce[b]);
+                    }
+                    stage_half(r, c, 0);
+                    stage_half(r, c, 1);
+                }
+            } else {
+                // fp32 phi: direct 16-byte stores of each row
+                auto pass2 = [&](const uint32_t *r, int c) {
+#pragma unroll
+                    for (int j0 = 0; j0 < 32; j0 += 4) {
+                        float e1[4], e2[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float y = yv(r, c, j0 + j);
+                            e1[j] = ex2_approx(y - sh);
+                            e2[j] = ex2_approx(-y - sh);
+                        }
+                        *reinterpret_cast<float4 *>(out + c + j0) = make_float4(e1[0], e1[1], e1[2], e1[3]);
+                        *reinterpret_cast<float4 *>(out + P + c + j0) = make_float4(e2[0], e2[1], e2[2], e2[3]);
+                    }
+                };
+                uint32_t ra[32], rb[32];
+                tmem_ld32(tbase, ra);
+                tmem_wait_ld();
+#pragma unroll 1
+                for (int c = 0; c < P; c += 64) {
+                    tmem_ld32(tbase + c + 32, rb);
+                    if (valid) pass2(ra, c);
+                    tmem_wait_ld();
+                    if (c + 64 < P) tmem_ld32(tbase + c + 64, ra);
+                    if (c + 64 >= P) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars->acce[b]);
+                    }
+                    if (valid) pass2(rb, c + 32);
+                    tmem_wait_ld();
                 }
             }
         }
+        // the staging buffer is read (and the stores issued) before the CTA ends
+        if (wt == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -281,8 +339,17 @@ cudaError_t go(const void *x0, const void *W0, const float *bias0, void *phi0, v
     const int Hv = per_head ? H : 1;
     const int64_t Tv = rows / Hv;
     const int nz = x1 ? 2 : 1;
-    CUtensorMap tmx[2], tmw[2];
+    CUtensorMap tmx[2], tmw[2], tmo[2];
     for (int z = 0; z < nz; ++z) {
+        if constexpr (sizeof(TP) == 2) {
+            // phi [rows, F] bf16 viewed as (F, Hv, Tv); boxes of 32 features x 128 rows
+            uint64_t dims[3] = {(uint64_t)(2 * P), (uint64_t)Hv, (uint64_t)Tv};
+            uint64_t strides[2] = {(uint64_t)(2 * P) * 2, (uint64_t)Hv * (2 * P) * 2};
+            uint32_t box[3] = {32, 1, kBM};
+            if (!tc::make_tmap(&tmo[z], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, z ? phi1 : phi0, 3, dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
+        }
         {
             uint64_t dims[3] = {(uint64_t)D, (uint64_t)Hv, (uint64_t)Tv};
             uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)Hv * D * 2};
@@ -297,11 +364,16 @@ cudaError_t go(const void *x0, const void *W0, const float *bias0, void *phi0, v
             if (!tc::make_tmap_bf16(&tmw[z], z ? W1 : W0, 2, dims, strides, box)) return cudaErrorInvalidValue;
         }
     }
+    if constexpr (sizeof(TP) != 2) {
+        tmo[0] = tmx[0];   // unused: fp32 phi is stored directly
+        tmo[1] = tmx[nz - 1];
+    }
     if (nz == 1) {
         tmx[1] = tmx[0];
         tmw[1] = tmw[0];
+        tmo[1] = tmo[0];
     }
-    auto kern = featmap_tc_kernel<D, P, TP>;
+    auto kern = (bias0 || bias1) ? featmap_tc_kernel<D, P, TP, true> : featmap_tc_kernel<D, P, TP, false>;
     cudaError_t e = ensure_smem_limit(kern, Lay::kSmem);
     if (e != cudaSuccess) return e;
     const int64_t ntiles = (Tv + kBM - 1) / kBM;
@@ -312,7 +384,7 @@ cudaError_t go(const void *x0, const void *W0, const float *bias0, void *phi0, v
     if (per_head_ctas > ntiles) per_head_ctas = ntiles;
     if (per_head_ctas < 1) per_head_ctas = 1;
     dim3 grid((unsigned)per_head_ctas, (unsigned)Hv, (unsigned)nz);
-    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx[0], tmw[0], tmx[1], tmw[1], Tv, Hv, bias0, bias1, per_head ? 1 : 0,
+    kern<<<grid, kThreads, Lay::kSmem, s>>>(tmx[0], tmw[0], tmx[1], tmw[1], tmo[0], tmo[1], Tv, Hv, bias0, bias1, per_head ? 1 : 0,
                                             (TP *)phi0, (TP *)phi1, (__nv_bfloat16 *)lo0, (__nv_bfloat16 *)lo1,
                                             err);
     count_launches(1);

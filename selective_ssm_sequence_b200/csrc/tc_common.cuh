@@ -202,6 +202,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// log2(x) by the hardware approximation (PTX lg2.approx.ftz.f32).
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Packed fp32 pair arithmetic (one instruction for two lanes of work).
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     uint64_t ra, rb, rc, rd;

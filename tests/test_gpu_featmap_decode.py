@@ -51,21 +51,23 @@ def test_featmap_fp32_tiny_config(hm):
     assert rel_err(phi, ref) <= TOL_F32
 
 
-def test_featmap_per_head_weights_and_bias(hm):
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_featmap_per_head_weights_and_bias(hm, out_dtype):
     H, d, p, rows = 4, 256, 128, 4 * 300
     x = wl.round_bf16(wl.normal(3, "x", (rows, d)))
     W = wl.round_bf16(wl.normal(3, "W", (H, p, d), 1 / 16))
     b = wl.round_f32(wl.normal(3, "b", (H, p), 0.5))
-    phi = _featmap_gpu(hm, x, W, "bf16", "f32", H=H, bias=b, w_head_stride=p * d)
+    phi = _featmap_gpu(hm, x, W, "bf16", out_dtype, H=H, bias=b, w_head_stride=p * d)
     ref = oracle.featmap(x, W, bias=b, H=H, w_head_stride=p * d, b_head_stride=p)
     assert rel_err(phi, ref) <= TOL_BF16
 
 
-def test_featmap_large_logits_stay_finite(hm):
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_featmap_large_logits_stay_finite(hm, out_dtype):
     # |u| up to ~60: the max subtraction keeps exp in range
     x = wl.round_bf16(wl.normal(4, "x", (300, 256), 4.0))
     W = wl.round_bf16(wl.normal(4, "W", (128, 256), 1.0))
-    phi = _featmap_gpu(hm, x, W, "bf16", "f32")
+    phi = _featmap_gpu(hm, x, W, "bf16", out_dtype)
     assert np.isfinite(phi).all()
     assert rel_err(phi, oracle.featmap(x, W)) <= TOL_BF16
 
