@@ -10,7 +10,8 @@
 // 256-byte row segments per access.  All row loads of a thread are issued
 // before any arithmetic (16 x 16 B in flight per thread) with streaming
 // cache hints, the update is done in registers and written back in place;
-// the 16 row-group partial numerators are reduced through shared memory.
+// the 16 row-group partial numerators are reduced through shared memory
+// while the next tile's loads are already in flight.
 // One CTA walks all column tiles of its head, so z (shared by every column)
 // is read and rewritten by the same thread with no cross-CTA race.
 #include "hm_internal.h"
@@ -91,13 +92,6 @@ decode_kernel(int H, int F, int dv, const TF *__restrict__ phq, const TF *__rest
     for (int tile = 0; tile * kCols < dv; ++tile) {
         const int c0 = tile * kCols + cg * 4;
         const bool cols_ok = c0 < dv;  // dv % 4 == 0 (host-checked)
-        if (tile > 0) {
-#pragma unroll
-            for (int m = 0; m < kMaxRowsPerThread; ++m) {
-                int f = rg + kRowGroups * m;
-                if (f < F && cols_ok) s[m] = ld_stream(Sbh + ((int64_t)f * dv + c0) / 4);
-            }
-        }
         float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
         if (cols_ok) {
             vv.x = hm_ld(v, bh * dv + c0 + 0);
@@ -121,6 +115,17 @@ decode_kernel(int H, int F, int dv, const TF *__restrict__ phq, const TF *__rest
                 num.y = fmaf(qf, t.y, num.y);
                 num.z = fmaf(qf, t.z, num.z);
                 num.w = fmaf(qf, t.w, num.w);
+            }
+        }
+        // the next tile's state rows go out before the reduction of this one
+        {
+            const int cn = c0 + kCols;
+            if (cn < dv) {
+#pragma unroll
+                for (int m = 0; m < kMaxRowsPerThread; ++m) {
+                    int f = rg + kRowGroups * m;
+                    if (f < F) s[m] = ld_stream(Sbh + ((int64_t)f * dv + cn) / 4);
+                }
             }
         }
         snum[rg][cg * 4 + 0] = num.x;
