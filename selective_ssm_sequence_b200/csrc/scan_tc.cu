@@ -55,6 +55,7 @@ constexpr int kTileV = 2 * kBlk;   // [64 x 128] bf16 tile = 16 KB
 // e^x for the decay factors (arguments <= 0 except the log-space prefix sums
 // of a chunk; results are used at bf16 / fp32-accumulate precision)
 __device__ __forceinline__ float fexp(float x) { return ex2_approx(x * 1.4426950408889634f); }
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct Geo {
     int64_t B, L;
@@ -481,7 +482,6 @@ struct CAux {
     float z[kF];
     alignas(16) float zred[kZGroups][kF];
     float gam[2];
-    float redb[4];
     float redd[4];
     // per stage: the phiQ blocks and the phiK + V blocks are loaded and
     // released separately
@@ -490,6 +490,7 @@ struct CAux {
     uint64_t p_full, p_consumed, epib_done, o_full, o_empty, s_full, sbf_ready;
     uint64_t den_ready[2], den_free[2];   // 1 / den of a stage written / read
     uint64_t pro_full[3];                 // start-state rounds landed (prologue staging)
+    uint64_t dec_full[2], dec_free[2];    // decay vectors of a parity written / read
     uint32_t tmem;
     int abort;
 };
@@ -538,23 +539,26 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
     return tot;
 }
 
-// Warp roles (14 warps):
+// Warp roles (15 warps):
 //   0      TMA producer (phiQ, phiK, V of each chunk; two stages)
 //   1      MMA issuer
 //   2..9   compute group (256 threads): per chunk the decayed score tile Pt
 //          (three 32 x 32 quadrants: rows 0..31 need only columns 0..31),
-//          w (.) V and the decay vectors of the next chunk (prefix sums of
-//          log a, e^cum, e^(cum_last - cum), gamma), the scaled queries
-//          e^cum (.) phiQ with phiq . z_prev, the denominators, the weighted
-//          key-feature sums and z
+//          w (.) V, the scaled queries e^cum (.) phiQ with phiq . z_prev, the
+//          denominators, the weighted key-feature sums and z
 //   10..13 outputs and state pass: o = O^T / den for the chunk, staged in the
 //          chunk's Pt buffer (dead once the PV product is complete) and written
 //          by TMA bulk stores; then S^T (fp32, TMEM) -> bf16 copy for the next
 //          readout and S^T <- gamma S^T before the next state MMA
+//   14     decay vectors, one chunk ahead of the compute group (prefix sums
+//          of log a, e^cum, e^(cum_last - cum), the below-diagonal column
+//          factors, gamma), two tokens per lane
 // Per chunk the MMA issuer runs: scores of the next chunk, then the readout
 // O^T = S^T (e^cum phiQ)^T, O^T += V^T Pt^T (hi and lo), and the state
 // update S^T += (w V)^T phiK.
-__global__ void __launch_bounds__(448, 1)
+constexpr int kCThreads = 480;
+
+__global__ void __launch_bounds__(kCThreads, 1)
 scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                 const __grid_constant__ CUtensorMap tms, OutArgs a, DevErr err) {
@@ -609,6 +613,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_init(&X->den_free[s], 4);
         }
         for (int r = 0; r < 3; ++r) mbar_init(&X->pro_full[r], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&X->dec_full[s], 1);
+            mbar_init(&X->dec_free[s], 1);
+        }
         X->abort = 0;
         mbar_fence_init();
     }
@@ -725,50 +733,21 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             else zi = a.z_start + (bh * g.G + seg) * kF;
             X->z[gt] = zi ? zi[gt] : 0.f;
         }
-        // dt of the next chunk's tokens is fetched one chunk ahead
-        // decay of chunk c (warps 4, 5: thread = token tk): cum, e^cum, weights
-        // e^(cum_last - cum), the below-diagonal column factors and gamma, into
-        // the buffers of c's parity.  Chunk c + 1's is computed during chunk c,
-        // while those warps wait for the score quadrants.
-        const bool dwarp = warp == 4 || warp == 5;
-        const int tk = gt - 64;   // 0..63 on the decay warps
-        float dt_next = dwarp ? token_dt(a, b, h, (int64_t)c_begin * kC, tk) : -INFINITY;
-        auto decay = [&](int c) {
-            const int sc = c & 1;
-            const float l = hm_log_decay(dt_next, alog);
-            if (c + 1 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + c + 1) * kC, tk);
-            float x = l;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (tk == 31) X->redb[0] = x;
-            named_sync(5, 64);
-            if (tk >= 32) x += X->redb[0];
-            if (tk == kC - 1) X->redb[1] = x;
-            named_sync(5, 64);
-            const float total = X->redb[1];
-            const float xe = __shfl_sync(0xffffffffu, x, lane | 7);   // cum at the end of j's 8-block
-            if (tk < 32) X->bq[sc][tk] = fexp(xe - x);
-            X->cum[sc][tk] = x;
-            X->qs[sc][tk] = fexp(x);
-            X->w[sc][tk] = fexp(total - x);
-            if (tk == 0) X->gam[sc] = fexp(total);
-            named_sync(5, 64);   // redb free again
-        };
-        if (dwarp) decay(0);
         // every exit from this loop is taken by the whole group (after a
         // barrier-AND), so no thread is left waiting at a named barrier
         bool ok = named_sync_and(1, 256, true);
         for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
-            // (1) the chunk's decay vectors were computed during the previous chunk
-            // (chunk 0: the state prologue, which stages in the Pt and w V buffers,
-            // must be complete before they are written)
-            ok = named_sync_and(1, 256, ok && (it > 0 || mbar_wait(&X->sbf_ready, 0, abort_flag, err,
-                                                                    KID_SCAN_TC_OUT, 21)));
+            // (1) the chunk's decay vectors (from the decay warp; chunk 0: the
+            // state prologue, which stages in the Pt and w V buffers, must also
+            // be complete before they are written)
+            const bool okd = mbar_wait(&X->dec_full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 22) &&
+                             (it > 0 || mbar_wait(&X->sbf_ready, 0, abort_flag, err, KID_SCAN_TC_OUT, 21));
+            ok = named_sync_and(1, 256, ok && okd);
             if (!ok) break;
+            // every thread is past chunk it - 1, the last reader of the other
+            // parity's decay vectors
+            if (gt == 0 && it > 0) mbar_arrive(&X->dec_free[(it - 1) & 1]);
             // (2) once the chunk's scores are in TMEM
             bool okw = mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7) &&
                        mbar_wait(&X->fullkv[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8) &&
@@ -809,36 +788,39 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     // block's last column, both factors <= 1
                     const float ci = X->cum[s][i];
                     uint8_t *__restrict__ prow = gP(s);
-                    float rs = 0.f;
+                    float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
-                        const float ai = fexp(ci - X->cum[s][8 * c4 + 7]);
+                        const float ai = ex2_approx(ci - X->cum[s][8 * c4 + 7]);
+                        const float2 a2 = make_float2(ai, ai);
                         const float4 ba = *reinterpret_cast<const float4 *>(&X->bq[s][8 * c4]);
                         const float4 bb = *reinterpret_cast<const float4 *>(&X->bq[s][8 * c4 + 4]);
-                        const float bv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+                        const float2 bv[4] = {make_float2(ba.x, ba.y), make_float2(ba.z, ba.w),
+                                              make_float2(bb.x, bb.y), make_float2(bb.z, bb.w)};
                         uint4 hi, lo;
                         uint32_t *pk = reinterpret_cast<uint32_t *>(&hi);
                         uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int jl = c4 * 8 + 2 * e;
-                            const float e0 = __uint_as_float(pr[jl]) * (ai * bv[2 * e]);
-                            const float e1 = __uint_as_float(pr[jl + 1]) * (ai * bv[2 * e + 1]);
-                            pk[e] = pack_bf16x2(e0, e1);
-                            const float2 r = unpack_bf16x2(pk[e]);
-                            pl[e] = pack_bf16x2(e0 - r.x, e1 - r.y);
-                            rs += e0 + e1;
+                            const float2 ev = mul2(make_float2(__uint_as_float(pr[jl]), __uint_as_float(pr[jl + 1])),
+                                                   mul2(a2, bv[e]));
+                            pk[e] = pack_bf16x2(ev.x, ev.y);
+                            const float2 r = sub2(ev, unpack_bf16x2(pk[e]));
+                            pl[e] = pack_bf16x2(r.x, r.y);
+                            rs2 = add2(rs2, ev);
                         }
                         *reinterpret_cast<uint4 *>(prow + sw128_off(i, c4)) = hi;
                         *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, c4)) = lo;
                     }
-                    X->dint[0][i] = rs;
+                    X->dint[0][i] = rs2.x + rs2.y;
                     tc_fence_before();
                 } else if (okw) {
                     const float ci = X->cum[s][i];
+                    const float2 ci2 = make_float2(ci, ci);
                     const float *__restrict__ cj = X->cum[s] + jc;
                     uint8_t *__restrict__ prow = gP(s);
-                    float rs = 0.f;
+                    float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
                         uint4 hi, lo;
@@ -846,18 +828,21 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
                         const float4 ca = *reinterpret_cast<const float4 *>(cj + c4 * 8);
                         const float4 cb = *reinterpret_cast<const float4 *>(cj + c4 * 8 + 4);
-                        const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                        const float2 cv[4] = {make_float2(ca.x, ca.y), make_float2(ca.z, ca.w),
+                                              make_float2(cb.x, cb.y), make_float2(cb.z, cb.w)};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int jl = c4 * 8 + 2 * e;
                             const int j = jc + jl;
-                            const float e0 = (!masked || j <= i) ? __uint_as_float(pr[jl]) * fexp(ci - cv[2 * e]) : 0.f;
-                            const float e1 =
-                                (!masked || j + 1 <= i) ? __uint_as_float(pr[jl + 1]) * fexp(ci - cv[2 * e + 1]) : 0.f;
-                            pk[e] = pack_bf16x2(e0, e1);
-                            const float2 r = unpack_bf16x2(pk[e]);
-                            pl[e] = pack_bf16x2(e0 - r.x, e1 - r.y);
-                            rs += e0 + e1;
+                            const float2 d = sub2(ci2, cv[e]);
+                            float2 ev = mul2(make_float2(__uint_as_float(pr[jl]), __uint_as_float(pr[jl + 1])),
+                                             make_float2(ex2_approx(d.x), ex2_approx(d.y)));
+                            if (masked && j > i) ev.x = 0.f;
+                            if (masked && j + 1 > i) ev.y = 0.f;
+                            pk[e] = pack_bf16x2(ev.x, ev.y);
+                            const float2 r = sub2(ev, unpack_bf16x2(pk[e]));
+                            pl[e] = pack_bf16x2(r.x, r.y);
+                            rs2 = add2(rs2, ev);
                         }
                         const int cc = (jc >> 3) + c4;
                         *reinterpret_cast<uint4 *>(prow + sw128_off(i, cc)) = hi;
@@ -869,7 +854,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                                 make_uint4(0u, 0u, 0u, 0u);
                         }
                     }
-                    X->dint[jc ? 1 : 0][i] = rs;
+                    X->dint[jc ? 1 : 0][i] = rs2.x + rs2.y;
                     tc_fence_before();
                 }
             } else {
@@ -898,9 +883,6 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         *reinterpret_cast<uint4 *>(gVt + off) = vv;
                     }
                 }
-                // the next chunk's decay vectors (its parity's buffers were last
-                // read during chunk it - 1)
-                if (dwarp && it + 1 < nch) decay(it + 1);
             }
             // (3) every thread: the query row scaled by e^cum_i, in place, and
             // phiq_i . z_prev over one quarter of the features (on the unscaled
@@ -988,6 +970,47 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 for (int tg = 0; tg < kZGroups; ++tg) acc += X->zred[tg][gt];
                 X->z[gt] = fmaf(X->gam[s], X->z[gt], acc);
             }
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------------------ decay vectors
+        // lane: tokens 2 lane and 2 lane + 1 of the chunk; dt two chunks ahead
+        float da[2], db[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            da[i] = i < nch ? token_dt(a, b, h, (int64_t)(c_begin + i) * kC, 2 * lane) : -INFINITY;
+            db[i] = i < nch ? token_dt(a, b, h, (int64_t)(c_begin + i) * kC, 2 * lane + 1) : -INFINITY;
+        }
+        for (int c = 0; c < nch; ++c) {
+            const int sc = c & 1;
+            const float l0 = hm_log_decay(da[0], alog) * kLog2e, l1 = hm_log_decay(db[0], alog) * kLog2e;
+            da[0] = da[1];
+            db[0] = db[1];
+            da[1] = c + 2 < nch ? token_dt(a, b, h, (int64_t)(c_begin + c + 2) * kC, 2 * lane) : -INFINITY;
+            db[1] = c + 2 < nch ? token_dt(a, b, h, (int64_t)(c_begin + c + 2) * kC, 2 * lane + 1) : -INFINITY;
+            // inclusive prefix sums of the token pairs over the lanes: x = cum
+            // at token 2 lane + 1
+            float x = l0 + l1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            const float x0 = x - l1;                                   // cum at token 2 lane
+            const float total = __shfl_sync(0xffffffffu, x, 31);
+            const float xe = __shfl_sync(0xffffffffu, x, lane | 3);   // cum at the end of the 8-block
+            // the parity's buffers were last read during chunk c - 2
+            bool okw = c < 2 || mbar_wait(&X->dec_free[sc], ((c >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 23);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            if (lane < 16)
+                *reinterpret_cast<float2 *>(&X->bq[sc][2 * lane]) =
+                    make_float2(ex2_approx(xe - x0), ex2_approx(xe - x));
+            *reinterpret_cast<float2 *>(&X->cum[sc][2 * lane]) = make_float2(x0, x);
+            *reinterpret_cast<float2 *>(&X->qs[sc][2 * lane]) = make_float2(ex2_approx(x0), ex2_approx(x));
+            *reinterpret_cast<float2 *>(&X->w[sc][2 * lane]) =
+                make_float2(ex2_approx(total - x0), ex2_approx(total - x));
+            if (lane == 0) X->gam[sc] = ex2_approx(total);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->dec_full[sc]);
         }
     } else {
         // ------------------------------------------------------------ state pass
@@ -1333,7 +1356,7 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
     }
     e = ensure_smem_limit(scan_out_kernel, kCSmem);
     if (e != cudaSuccess) return e;
-    scan_out_kernel<<<(unsigned)(2 * g.G * BH), 448, kCSmem, s>>>(tq, tk, tv, to, tss, oa, err);
+    scan_out_kernel<<<(unsigned)(2 * g.G * BH), kCThreads, kCSmem, s>>>(tq, tk, tv, to, tss, oa, err);
     count_launches(1);
     return cudaGetLastError();
 }
