@@ -57,11 +57,8 @@ def load_peaks():
 # DRAM bytes per launch of the dominant call from an ncu capture of the
 # current kernel versions (dram__bytes_read.sum + dram__bytes_write.sum,
 # summed over the call's kernels; ncu runs each kernel with cold caches), or
-# None when a kernel changed since the counters were taken.  Prefill
-# B4 H8 L2048: scan_state 33,745,664 + 2,048 + scan_carry 16,856,576 +
-# scan_out 109,442,304 + 10,339,072
-# (profiles/scan_call_traffic_prefill_B4_H8_L2048.md).
-NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 170385664}
+# None when a kernel changed since the counters were taken.
+NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): None}
 
 # ---------------------------------------------------------------- clocks
 
