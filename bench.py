@@ -57,8 +57,11 @@ def load_peaks():
 # DRAM bytes per launch of the dominant call from an ncu capture of the
 # current kernel versions (dram__bytes_read.sum + dram__bytes_write.sum,
 # summed over the call's kernels; ncu runs each kernel with cold caches), or
-# None when a kernel changed since the counters were taken.
-NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): None}
+# None when a kernel changed since the counters were taken.  Prefill
+# B4 H8 L2048: scan_state 33,730,816 + 2,048 + scan_carry 16,865,280 +
+# scan_out 109,435,392 + 10,352,896
+# (profiles/scan_call_traffic_prefill_B4_H8_L2048.md).
+NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 170386432}
 
 # ---------------------------------------------------------------- clocks
 
@@ -598,7 +601,7 @@ def bench_decode(cfg, args, rank, world, torch):
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
                      "bytes_per_step": state_bytes + io_bytes, "peak_source": peak_kind,
-                     "kernel": "whole step (2 featmap + 1 decode launch)"},
+                     "kernel": "whole step (the q and k feature maps in one launch + the decode launch)"},
         "gpu_launches": per_step * steps,
         "clocks": sampler.summary(),
     }

@@ -389,11 +389,11 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
 //   acc <- exp(lsum_p) acc + part_p,
 // storing the state at each segment start and, when every part was
 // computed, the final state.  Elements [0, F*dv) are S, [F*dv, F*dv + F) are z.
-// A thread owns kCarryCols groups, 256 apart (coalesced), and loads the next
-// part of all of them while it combines the current one, so that enough bytes
-// are in flight to stream the parts at HBM speed.
-constexpr int kCarryCols = 4;
-
+// A thread owns COLS groups, 256 apart (coalesced), and loads PF parts of all
+// of them before combining them, so that enough bytes are in flight to stream
+// the parts at HBM speed: many heads take COLS = 2, PF = 2; few heads (and
+// then many parts) COLS = 1, PF = 8 (more CTAs, deeper prefetch).
+template <int COLS, int PF>
 __global__ void __launch_bounds__(256, 4)
 scan_carry_kernel(Geo g, const float *__restrict__ S_part, const float *__restrict__ z_part,
                   const float *__restrict__ lsum_part, const float *__restrict__ S0, const float *__restrict__ z0,
@@ -403,8 +403,6 @@ scan_carry_kernel(Geo g, const float *__restrict__ S_part, const float *__restri
     const int nS = kF * g.dv;
     const int pps = g.seg_chunks / g.part_chunks;
     // group j: element e = 4 * col; S element e, or z element e - nS
-    int col[kCarryCols];
-    float4 acc[kCarryCols], cur[kCarryCols];
     auto elem = [&](const float *S, const float *z, int64_t blk, int c) -> const float * {
         const int e = 4 * c;
         return e < nS ? S + blk * nS + e : z + blk * kF + (e - nS);
@@ -414,43 +412,53 @@ scan_carry_kernel(Geo g, const float *__restrict__ S_part, const float *__restri
         return e < nS ? S + blk * nS + e : z + blk * kF + (e - nS);
     };
     const int ncol = (nS + kF) / 4;
+    int col[COLS];
+    float4 acc[COLS];
 #pragma unroll
-    for (int j = 0; j < kCarryCols; ++j) {
-        col[j] = (blockIdx.x * kCarryCols + j) * blockDim.x + threadIdx.x;
+    for (int j = 0; j < COLS; ++j) {
+        col[j] = (blockIdx.x * COLS + j) * blockDim.x + threadIdx.x;
         acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        cur[j] = acc[j];
         if (col[j] < ncol) {
             const bool isz = 4 * col[j] >= nS;
             if (isz ? z0 != nullptr : S0 != nullptr)
                 acc[j] = *reinterpret_cast<const float4 *>(elem(S0, z0, bh, col[j]));
-            if (g.NPc > 0) cur[j] = *reinterpret_cast<const float4 *>(elem(S_part, z_part, bh * g.NPc, col[j]));
         }
     }
-    for (int p = 0; p <= g.NPc; ++p) {
-        if (p > 0 && p % pps == 0 && p / pps < g.G) {
+    for (int p0 = 0; p0 <= g.NPc; p0 += PF) {
+        float4 v[PF][COLS];
+        float lg[PF];
 #pragma unroll
-            for (int j = 0; j < kCarryCols; ++j)
-                if (col[j] < ncol)
-                    *reinterpret_cast<float4 *>(elem_w(S_start, z_start, bh * g.G + p / pps, col[j])) = acc[j];
+        for (int u = 0; u < PF; ++u) {
+            const int p = p0 + u;
+            lg[u] = p < g.NPc ? lsum_part[bh * g.NPc + p] : 0.f;
+#pragma unroll
+            for (int j = 0; j < COLS; ++j)
+                v[u][j] = (p < g.NPc && col[j] < ncol)
+                              ? *reinterpret_cast<const float4 *>(elem(S_part, z_part, bh * g.NPc + p, col[j]))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        if (p == g.NPc) break;
-        float4 nxt[kCarryCols];
 #pragma unroll
-        for (int j = 0; j < kCarryCols; ++j)
-            nxt[j] = (col[j] < ncol && p + 1 < g.NPc)
-                         ? *reinterpret_cast<const float4 *>(elem(S_part, z_part, bh * g.NPc + p + 1, col[j]))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float gam = expf(lsum_part[bh * g.NPc + p]);
+        for (int u = 0; u < PF; ++u) {
+            const int p = p0 + u;
+            if (p > g.NPc) break;
+            if (p > 0 && p % pps == 0 && p / pps < g.G) {
 #pragma unroll
-        for (int j = 0; j < kCarryCols; ++j) {
-            acc[j] = make_float4(fmaf(gam, acc[j].x, cur[j].x), fmaf(gam, acc[j].y, cur[j].y),
-                                 fmaf(gam, acc[j].z, cur[j].z), fmaf(gam, acc[j].w, cur[j].w));
-            cur[j] = nxt[j];
+                for (int j = 0; j < COLS; ++j)
+                    if (col[j] < ncol)
+                        *reinterpret_cast<float4 *>(elem_w(S_start, z_start, bh * g.G + p / pps, col[j])) = acc[j];
+            }
+            if (p < g.NPc) {
+                const float gam = expf(lg[u]);
+#pragma unroll
+                for (int j = 0; j < COLS; ++j)
+                    acc[j] = make_float4(fmaf(gam, acc[j].x, v[u][j].x), fmaf(gam, acc[j].y, v[u][j].y),
+                                         fmaf(gam, acc[j].z, v[u][j].z), fmaf(gam, acc[j].w, v[u][j].w));
+            }
         }
     }
     if (g.NPc == g.NP) {
 #pragma unroll
-        for (int j = 0; j < kCarryCols; ++j) {
+        for (int j = 0; j < COLS; ++j) {
             if (col[j] >= ncol) continue;
             const bool isz = 4 * col[j] >= nS;
             if (isz ? z_out != nullptr : S_out != nullptr)
@@ -1317,9 +1325,17 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
                                                     add_lo ? 1 : 0, S_part, z_part, lsum, err);
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        dim3 gb((unsigned)(((nS + kF) / 4 + 256 * kCarryCols - 1) / (256 * kCarryCols)), (unsigned)BH);
-        scan_carry_kernel<<<gb, 256, 0, s>>>(g, S_part, z_part, lsum, c.S0, c.z0, S_start, z_start,
-                                             c.S_out, c.z_out);
+        const int64_t ncol = (int64_t)(nS + kF) / 4;
+        const int64_t wide_ctas = BH * ((ncol + 511) / 512);
+        if (wide_ctas >= 2 * (int64_t)num_sms()) {
+            dim3 gb((unsigned)((ncol + 511) / 512), (unsigned)BH);
+            scan_carry_kernel<2, 2><<<gb, 256, 0, s>>>(g, S_part, z_part, lsum, c.S0, c.z0, S_start, z_start,
+                                                       c.S_out, c.z_out);
+        } else {
+            dim3 gb((unsigned)((ncol + 255) / 256), (unsigned)BH);
+            scan_carry_kernel<1, 8><<<gb, 256, 0, s>>>(g, S_part, z_part, lsum, c.S0, c.z0, S_start, z_start,
+                                                       c.S_out, c.z_out);
+        }
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
