@@ -10,13 +10,13 @@
 // chunk up to token i; gamma = exp(cum_last)):
 //   P        = phiQ phiK^T                                     (tensor cores)
 //   Pt_ij    = P_ij exp(cum_i - cum_j) [j <= i]                (registers; the
-//              decay is applied elementwise, never factorised, so no term
-//              overflows)
+//              decay is applied elementwise, or as a product of two factors
+//              that are both <= 1, so no term overflows)
 //   O        = Pt V + diag(exp(cum)) phiQ S_prev               (tensor cores)
 //   den      = rowsum(Pt) + exp(cum) (phiQ z_prev)
 //   S        = gamma S_prev + (w phiK)^T V,  w_j = exp(cum_last - cum_j) <= 1
-//            = gamma S_prev + phiK^T (w V)   (the output kernel weights the
-//              128 value channels of its CTA rather than the 256 features)
+//            = gamma S_prev + phiK^T (w V)   (the kernels weight the 128 value
+//              channels of their CTA rather than the 256 features)
 //   z        = gamma z_prev + sum_j w_j phik_j
 // These are exact rewrites of the recurrence.  The state is kept transposed
 // (S^T, value channel x feature) in TMEM: the state update V^T (w phiK) and the
@@ -27,8 +27,9 @@
 // Long sequences are cut into segments that run in parallel.  Three kernels:
 //   A  scan_state_kernel  local end state of each part (a run of chunks) from a
 //                         zero start, weights relative to the part end; with
-//                         hi / lo bf16 splits of w * phik the state update is
-//                         accurate to ~16 bits (used for the returned state).
+//                         hi / lo bf16 splits of w (.) v and of phik the state
+//                         update is accurate to ~16 bits (used for the
+//                         returned state).
 //   B  scan_carry_kernel  composes the parts' affine maps (S -> g S + S_part,
 //                         SSM article sec. 4.2) in fp32 to get each segment's
 //                         start state and the final state.
