@@ -408,12 +408,15 @@ hm_status hm_step_decode(const hm_decode_args *a, hm_stream_t stream) {
     cudaError_t e;
     if (a->W_q && rows > 0) {
         char *ws = (char *)a->workspace;
+        // bf16 io: bf16 features, as in the prefill (the tensor-core map then
+        // writes them through its TMA-staged epilogue); fp32 io: fp32 features
+        const hm_dtype pt = a->io_dtype == HM_BF16 ? HM_BF16 : HM_F32;
         e = run_featmap_qk(a->q, a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->W_k, a->w_head_stride,
-                           a->b_q, a->b_k, ws, ws + pl.phi_bytes, HM_F32, s);
+                           a->b_q, a->b_k, ws, ws + pl.phi_bytes, pt, s);
         if (e != cudaSuccess) return cuda_fail(e, "decode: feature maps");
         phq = ws;
         phk = ws + pl.phi_bytes;
-        ft = HM_F32;
+        ft = pt;
     }
     DecodeCore c{};
     c.B = a->B; c.H = a->H; c.F = pl.F; c.dv = a->dv;
