@@ -233,6 +233,22 @@ def test_precomputed_features_path(hm):
     assert rel_err(o, o_ref) <= TOL_BF16
 
 
+def test_precomputed_features_with_returned_state(hm):
+    # W_q = NULL and S_out requested: the state phase covers every part with
+    # the hi / lo split of w (.) v and no phik remainder plane (three stages)
+    cfg = wl.PREFILL_PYTHIA
+    inp = wl.scan_inputs(cfg, B=1, L=700, seed=28)
+    phq = wl.round_bf16(oracle.featmap(inp["q"], inp["W_q"]))
+    phk = wl.round_bf16(oracle.featmap(inp["k"], inp["W_k"]))
+    feat = dict(inp, q=phq, k=phk)
+    o, S, z = run_scan(hm, feat, "bf16", with_W=False, want_state=True)
+    o_ref, S_ref, z_ref = oracle.scan_recurrent(phq, phk, inp["v"], oracle.log_decay(inp["dt"], inp["A_log"]),
+                                                return_state=True)
+    assert rel_err(o, o_ref) <= TOL_BF16
+    assert rel_err(S, S_ref) <= TOL_BF16
+    assert rel_err(z, z_ref) <= TOL_BF16
+
+
 def test_per_head_weights_and_biases(hm):
     # one Hedgehog projection (and bias) per head: the q and k maps run in one
     # launch with one CTA column per head
