@@ -44,12 +44,19 @@ def _key(seed: int, name: str) -> np.uint64:
 
 
 def splitmix64_at(key: np.uint64, ctr: np.ndarray) -> np.ndarray:
-    """splitmix64 outputs for the given counters (uint64 array) under ``key``."""
+    """splitmix64 outputs for the given counters (uint64 array) under ``key``
+    (computed in place: one output array, one temporary)."""
     with np.errstate(over="ignore"):
-        z = key + ctr.astype(np.uint64) * _GOLD
-        z = (z ^ (z >> np.uint64(30))) * _M1
-        z = (z ^ (z >> np.uint64(27))) * _M2
-        z = z ^ (z >> np.uint64(31))
+        z = np.multiply(ctr, _GOLD, dtype=np.uint64)
+        z += key
+        t = np.right_shift(z, np.uint64(30))
+        z ^= t
+        z *= _M1
+        np.right_shift(z, np.uint64(27), out=t)
+        z ^= t
+        z *= _M2
+        np.right_shift(z, np.uint64(31), out=t)
+        z ^= t
     return z
 
 
@@ -59,7 +66,10 @@ def splitmix64(key: np.uint64, n: int) -> np.ndarray:
 
 
 def _u01(bits: np.ndarray) -> np.ndarray:
-    return ((bits >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+    u = np.right_shift(bits, np.uint64(11)).astype(np.float64)
+    u += 0.5
+    u *= 2.0 ** -53
+    return u
 
 
 def _flat_index(shape, index):
@@ -89,12 +99,38 @@ def uniform(seed: int, name: str, shape, lo: float = 0.0, hi: float = 1.0, index
     return lo + (hi - lo) * u
 
 
+def _contiguous_block(shape, index):
+    """(start, count, block shape) when the sub-block ``index`` (leading ints,
+    then at most one unit-step slice as its last entry) is one contiguous run
+    of the flat C-order array; None otherwise."""
+    shape = tuple(int(x) for x in shape)
+    if index is None:
+        return 0, int(np.prod(shape)), shape
+    index = tuple(index)
+    start = 0
+    for i, ix in enumerate(index):
+        st = int(np.prod(shape[i + 1:]))
+        if isinstance(ix, slice):
+            a, b, step = ix.indices(shape[i])
+            if step != 1 or i != len(index) - 1:
+                return None
+            n = max(0, b - a)
+            return start + a * st, n * st, (n,) + shape[i + 1:]
+        j = int(ix)
+        if j < 0:
+            j += shape[i]
+        start += j * st
+    return start, int(np.prod(shape[len(index):])), shape[len(index):]
+
+
 def normal(seed: int, name: str, shape, std: float = 1.0, index=None) -> np.ndarray:
     """N(0, std^2) array of ``shape`` (or its sub-block ``index``).  Element n
     is the cosine (n even) or sine (n odd) branch of Box-Muller on the uniform
     pair with counters 2*(n//2) + 1 and 2*(n//2) + 2."""
-    if index is None and int(np.prod(shape)) > (1 << 22):
-        return _normal_chunked(seed, name, shape, std)
+    blk = _contiguous_block(shape, index)
+    if blk is not None and blk[1] > (1 << 16):
+        start, count, bshape = blk
+        return _normal_range(seed, name, start, count, std).reshape(bshape)
     idx = _flat_index(shape, index)
     m = (idx // 2).astype(np.uint64)
     key = _key(seed, name)
@@ -105,13 +141,14 @@ def normal(seed: int, name: str, shape, std: float = 1.0, index=None) -> np.ndar
     return std * np.where((idx & 1) == 0, r * np.cos(ang), r * np.sin(ang))
 
 
-def _normal_chunked(seed, name, shape, std):
-    n = int(np.prod(shape))
-    out = np.empty(n, dtype=np.float64)
+def _normal_range(seed, name, start, count, std):
+    """Elements start .. start + count - 1 of the flat normal stream, in chunks,
+    each Box-Muller pair computed once."""
+    out = np.empty(count, dtype=np.float64)
     key = _key(seed, name)
     step = 1 << 22
-    for s0 in range(0, n, step):
-        s1 = min(n, s0 + step)
+    for s0 in range(start, start + count, step):
+        s1 = min(start + count, s0 + step)
         m0, m1 = s0 // 2, (s1 + 1) // 2
         mm = np.arange(m0, m1, dtype=np.uint64)
         u1 = _u01(splitmix64_at(key, 2 * mm + np.uint64(1)))
@@ -121,8 +158,8 @@ def _normal_chunked(seed, name, shape, std):
         z = np.empty(2 * (m1 - m0), dtype=np.float64)
         z[0::2] = r * np.cos(ang)
         z[1::2] = r * np.sin(ang)
-        out[s0:s1] = z[s0 - 2 * m0:s1 - 2 * m0]
-    return std * out.reshape(shape)
+        out[s0 - start:s1 - start] = z[s0 - 2 * m0:s1 - 2 * m0]
+    return std * out
 
 
 # --------------------------------------------------------------------------
