@@ -49,3 +49,16 @@ def test_scan_inputs_shapes():
     assert inp["A_log"].shape == (8,)
     # values are already bf16-representable
     np.testing.assert_array_equal(wl.round_bf16(inp["q"]), inp["q"])
+
+
+def test_sub_blocks_equal_slices_of_the_full_draw():
+    # contiguous sub-blocks (drawn pair by pair over a flat range) and strided
+    # ones (drawn element by element) both equal the same slice of the full array
+    shape = (6, 70, 4, 64)
+    full = wl.normal(9, "v", shape, std=0.5)
+    np.testing.assert_array_equal(wl.normal(9, "v", shape, std=0.5, index=(slice(1, 5),)), full[1:5])
+    np.testing.assert_array_equal(wl.normal(9, "v", shape, std=0.5, index=(3, slice(7, 60))), full[3, 7:60])
+    np.testing.assert_array_equal(wl.normal(9, "v", shape, std=0.5, index=(slice(0, 6, 2),)), full[0:6:2])
+    np.testing.assert_array_equal(wl.normal(9, "v", shape, std=0.5, index=(-1,)), full[-1])
+    u = wl.uniform(9, "a", shape)
+    np.testing.assert_array_equal(wl.uniform(9, "a", shape, index=(slice(2, 4),)), u[2:4])
