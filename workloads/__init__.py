@@ -87,7 +87,8 @@ def _flat_index(shape, index):
             r = np.arange(n, dtype=np.int64)[ix]
             out = out[..., None] + r * st
         else:
-            out = out + int(ix) * st
+            j = int(ix)
+            out = out + (j + n if j < 0 else j) * st
     return out
 
 
