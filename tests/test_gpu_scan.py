@@ -233,6 +233,20 @@ def test_precomputed_features_path(hm):
     assert rel_err(o, o_ref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("want_state", [False, True])
+def test_more_heads_than_sms(hm, want_state):
+    # 80 heads x 2 value halves = 160 CTAs per segment: one segment, and the
+    # output (and state) grids take a second wave
+    cfg = wl.PREFILL_PYTHIA
+    inp = wl.scan_inputs(cfg, B=10, L=300, seed=29)
+    o, S, z = run_scan(hm, inp, "bf16", want_state=want_state)
+    o_ref, S_ref, z_ref = _oracle(inp)
+    assert rel_err(o, o_ref) <= TOL_BF16
+    if want_state:
+        assert rel_err(S, S_ref) <= TOL_BF16
+        assert rel_err(z, z_ref) <= TOL_BF16
+
+
 def test_precomputed_features_with_returned_state(hm):
     # W_q = NULL and S_out requested: the state phase covers every part with
     # the hi / lo split of w (.) v and no phik remainder plane (three stages)
