@@ -17,11 +17,12 @@ Page citations (see ``hm_oracle.c`` for the full list):
   [LA]  Linear-attention tutorial (cnblogs 22790249): sec. 2 kernel form and
         associativity, sec. 3 recurrent form, sec. 4.3 RetNet decay.
   [SSM] SSM article (quant67 56-ssm): sec. 3.2 softplus dt, sec. 4.2 affine
-        composition.
+        composition, sec. 4.3 states recomputed in the backward pass.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-against closed forms, invariants, a brute-force rational-arithmetic evaluation
-or an independent formulation.  End-to-end numeric values are not printed on
+(forward) and ``tests/test_oracle_backward_pins.py`` (backward) against closed
+forms, invariants, finite differences, a brute-force rational-arithmetic
+evaluation or an independent formulation.  End-to-end numeric values are not printed on
 the pages (no worked example), so absolute values rest on those pins.
 """
 from __future__ import annotations
@@ -230,6 +231,112 @@ def scan_fwd(q, k, v, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=Non
         phk = featmap(k, W_k, b_k, H=H, w_head_stride=w_head_stride, b_head_stride=bstride)
     la = None if dt is None else log_decay(dt, A_log)
     return scan_recurrent(phq, phk, v, la, S0, z0, return_state=return_state)
+
+
+# --------------------------------------------------------------------------
+# backward (the derivative of the forward definition above, by the chain rule;
+# the pages train the mixer by distillation, [HM] sec. 3, and Mamba's kernels
+# recompute the states in the backward pass, [SSM] sec. 4.3)
+# --------------------------------------------------------------------------
+
+def scan_recurrent_bwd(phq, phk, v, do, log_a=None, S0=None, z0=None):
+    """Gradients of sum(do * o) for o = scan_recurrent(phq, phk, v, log_a, S0, z0).
+
+    Reverse-mode form of the recurrence, with n_t = S_t^T phq_t, d_t = phq_t . z_t,
+    o_t = n_t / d_t and G_t, g_t the total gradients of S_t, z_t:
+      dn_t = do_t / d_t,  dd_t = -(do_t . o_t) / d_t
+      G_t = phq_t dn_t^T + a_{t+1} G_{t+1},   g_t = phq_t dd_t + a_{t+1} g_{t+1}
+      dphq_t = S_t dn_t + z_t dd_t
+      dphk_t = G_t v_t + g_t,   dv_t = G_t^T phk_t
+      dlog_a_t = a_t (<G_t, S_{t-1}> + g_t . z_{t-1})
+      dS0 = a_1 G_1,  dz0 = a_1 g_1
+    The forward states are kept for the whole sequence (small cases only).
+    Returns (dphq, dphk, dv, dlog_a, dS0, dz0); dlog_a is None without log_a."""
+    phq, phk, v, do = _f64(phq), _f64(phk), _f64(v), _f64(do)
+    B, L, H, F = phq.shape
+    dv_ = v.shape[-1]
+    la = None if log_a is None else _f64(log_a)
+    a = np.ones((B, L, H)) if la is None else np.exp(la)
+    S = np.zeros((B, H, F, dv_)) if S0 is None else _f64(S0).copy()
+    z = np.zeros((B, H, F)) if z0 is None else _f64(z0).copy()
+    Ss = np.empty((L + 1, B, H, F, dv_))
+    zs = np.empty((L + 1, B, H, F))
+    Ss[0], zs[0] = S, z
+    for t in range(L):
+        S = a[:, t, :, None, None] * S + phk[:, t, :, :, None] * v[:, t, :, None, :]
+        z = a[:, t, :, None] * z + phk[:, t]
+        Ss[t + 1], zs[t + 1] = S, z
+    dphq = np.empty_like(phq)
+    dphk = np.empty_like(phk)
+    dv = np.empty_like(v)
+    dla = np.empty((B, L, H))
+    G = np.zeros((B, H, F, dv_))
+    g = np.zeros((B, H, F))
+    for t in range(L - 1, -1, -1):
+        St, zt = Ss[t + 1], zs[t + 1]
+        num = np.einsum("bhfv,bhf->bhv", St, phq[:, t])
+        den = np.einsum("bhf,bhf->bh", zt, phq[:, t])
+        if np.any(den <= 0):
+            raise FloatingPointError("oracle: a denominator was not > 0")
+        o = num / den[..., None]
+        dn = do[:, t] / den[..., None]
+        dd = -np.einsum("bhv,bhv->bh", do[:, t], o) / den
+        if t + 1 < L:
+            G = a[:, t + 1, :, None, None] * G
+            g = a[:, t + 1, :, None] * g
+        G = G + phq[:, t, :, :, None] * dn[:, :, None, :]
+        g = g + phq[:, t] * dd[..., None]
+        dphq[:, t] = np.einsum("bhfv,bhv->bhf", St, dn) + zt * dd[..., None]
+        dphk[:, t] = np.einsum("bhfv,bhv->bhf", G, v[:, t]) + g
+        dv[:, t] = np.einsum("bhfv,bhf->bhv", G, phk[:, t])
+        dla[:, t] = a[:, t] * (np.einsum("bhfv,bhfv->bh", G, Ss[t]) + np.einsum("bhf,bhf->bh", g, zs[t]))
+    dS0 = a[:, 0, :, None, None] * G
+    dz0 = a[:, 0, :, None] * g
+    return dphq, dphk, dv, (None if la is None else dla), dS0, dz0
+
+
+def log_decay_bwd(dt, A_log, dlog_a):
+    """Gradients of sum(dlog_a * l) for l = log_decay(dt, A_log):
+    dl/ddt = -sigmoid(dt) exp(A_log) and dl/dA_log = l.  Returns (ddt, dA_log)."""
+    dt, A_log, g = _f64(dt), _f64(A_log), _f64(dlog_a)
+    sig = 1.0 / (1.0 + np.exp(-dt))
+    ddt = -g * sig * np.exp(A_log)
+    dA = np.sum(g * log_decay(dt, A_log), axis=tuple(range(g.ndim - 1)))
+    return ddt, dA
+
+
+def featmap_bwd(x, W, dphi, bias=None):
+    """Gradients of sum(dphi * phi) for phi = featmap(x, W, bias) with one W
+    shared by every row: with e = [u, -u], u = W x + b and phi = softmax(e),
+      de = phi * (dphi - sum(dphi * phi)),  du = de[:p] - de[p:]
+      dx = W^T du,  dW = sum over rows du x^T,  db = sum over rows du.
+    Returns (dx, dW, db)."""
+    x, W, dphi = _f64(x), _f64(W), _f64(dphi)
+    p = W.shape[0]
+    phi = featmap(x, W, bias)
+    de = phi * (dphi - np.sum(dphi * phi, axis=-1, keepdims=True))
+    du = de[..., :p] - de[..., p:]
+    dx = du @ W
+    du2 = du.reshape(-1, p)
+    dW = du2.T @ x.reshape(-1, x.shape[-1])
+    db = du2.sum(axis=0)
+    return dx, dW, db
+
+
+def scan_bwd(q, k, v, W_q, W_k, do, dt=None, A_log=None):
+    """Gradients of sum(do * o) for o = scan_fwd(q, k, v, W_q, W_k, dt, A_log)
+    (shared Hedgehog weights, no bias, zero initial state).
+    Returns dict with dq, dk, dv, dW_q, dW_k and, with decay, ddt and dA_log."""
+    phq = featmap(q, W_q)
+    phk = featmap(k, W_k)
+    la = None if dt is None else log_decay(dt, A_log)
+    dphq, dphk, dv, dla, _, _ = scan_recurrent_bwd(phq, phk, v, do, la)
+    dq, dWq, _ = featmap_bwd(q, W_q, dphq)
+    dk, dWk, _ = featmap_bwd(k, W_k, dphk)
+    out = {"dq": dq, "dk": dk, "dv": dv, "dW_q": dWq, "dW_k": dWk}
+    if dt is not None:
+        out["ddt"], out["dA_log"] = log_decay_bwd(dt, A_log, dla)
+    return out
 
 
 def mixer_fwd(x, W_q, W_k, W_v, W_g, W_dt, conv_w, W_hq, W_hk, A_log, W_o,
