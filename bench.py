@@ -1,14 +1,15 @@
 #!/usr/bin/env python
 """Benchmark of the HedgeMamba mixer scan on B200 (prints one JSON line).
 
-Default workload: the Pythia-1B-shaped single-layer prefill (B=4, H=8,
-L=2048, d = dv = 256, Hedgehog 256->128 so F = 256, bf16 q/k/v, fp32
-state and accumulation, dt ~ N(0,1), A_log ~ U(0, log 16)).  One step is one
-pass of the whole hot path over one batch: the Hedgehog map on q and on k,
-then the decayed normalised chunked scan, each through the C ABI.
+Default workload: the long-context prefill (B=1, H=8, L=32768, d = dv = 256,
+Hedgehog 256->128 so F = 256, bf16 q/k/v, fp32 state and accumulation,
+dt ~ N(0,1), A_log ~ U(0, log 16)), the largest single-GPU scan workload;
+`--workload prefill` runs the Pythia-1B-shaped B=4, L=2048 case.  One step is
+one pass of the whole hot path over one batch: the Hedgehog map on q and on k,
+then the decayed normalised chunked scan, through one C-ABI call.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill|long|decode|mixer]
+                    [--workload long|prefill|decode|mixer] [--batch B]
 
 Multi-GPU (N > 1, launched by torchrun): every rank runs its own batch (its
 own seed); there is no data-path collective ("weak" scaling).  Times are
@@ -24,6 +25,7 @@ on bounded samples of the same workload on the host cores; rank 0 only.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -156,8 +158,35 @@ class ClockSampler:
             rs = {n for n, val in zip(names, parts[5:9]) if val.lower().startswith("active")}
             self.samples.append((time.perf_counter(), sm, mx, rs))
 
+    def sample_now(self):
+        """One synchronous read (NVML only), so that a timed region shorter
+        than the polling period still has samples."""
+        if self.handle is None:
+            return
+        nv, hd = self.nv, self.handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        try:
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(hd, nv.NVML_CLOCK_SM))
+        except Exception:
+            mx = None
+        try:
+            t = time.perf_counter()
+            sm = float(nv.nvmlDeviceGetClockInfo(hd, nv.NVML_CLOCK_SM))
+            bits = int(get_reasons(hd))
+            self.samples.append((t, sm, mx, {n for n, attr in self.REASONS
+                                             if getattr(nv, attr, 0) and bits & getattr(nv, attr, 0)}))
+        except Exception:
+            pass
+
     def mark_start(self):
         self.t0 = time.perf_counter()
+        self.sample_now()
+
+    def in_flight(self):
+        """Call once the timed work is enqueued and before waiting for it:
+        one more synchronous sample while the GPU runs it."""
+        self.sample_now()
 
     def mark_stop(self):
         self.t1 = time.perf_counter()
@@ -337,6 +366,7 @@ def bench_prefill(cfg, args, rank, world, torch):
     torch.cuda.synchronize()
     sampler.mark_start()
     timed(graphs[0], evs)
+    sampler.in_flight()
     torch.cuda.synchronize()
     sampler.mark_stop()
     launches = launches_per_step * K
@@ -529,6 +559,8 @@ def bench_decode(cfg, args, rank, world, torch):
     CUDA graph (one featmap launch per q / k and one decode launch)."""
     import selective_ssm_sequence_b200 as hm
     peaks, peak_kind = load_peaks()
+    if args.batch:
+        cfg = dataclasses.replace(cfg, B=args.batch, name=cfg.name + "_batch%d" % args.batch)
     w = wl.decode_weights(cfg)
     B, H, F, dv = cfg.B, cfg.H, cfg.F, cfg.dv
     tWq, tWk = to_dev(w["W_q"], "bf16", torch), to_dev(w["W_k"], "bf16", torch)
@@ -583,6 +615,7 @@ def bench_decode(cfg, args, rank, world, torch):
     for i in range(steps):
         graphs[i % nstep_tokens].replay()
     e1.record(stream)
+    sampler.in_flight()
     torch.cuda.synchronize()
     sampler.mark_stop()
     sampler.stop()
@@ -614,6 +647,8 @@ def bench_mixer(cfg, args, rank, world, torch):
     replayed from a CUDA graph."""
     import selective_ssm_sequence_b200 as hm
     peaks, peak_kind = load_peaks()
+    if args.batch:
+        cfg = dataclasses.replace(cfg, B=args.batch, name=cfg.name + "_batch%d" % args.batch)
     w = wl.mixer_weights(cfg)
     t = {k: to_dev(v, "f32" if k in ("conv_w", "A_log") else "bf16", torch) for k, v in w.items()}
     x = to_dev(wl.mixer_x(cfg), "bf16", torch)
@@ -645,6 +680,7 @@ def bench_mixer(cfg, args, rank, world, torch):
         g.replay()
         e1.record(stream)
         evs.append((e0, e1))
+    sampler.in_flight()
     torch.cuda.synchronize()
     sampler.mark_stop()
     sampler.stop()
@@ -674,7 +710,7 @@ def run_reference(args, rank, world):
         return None
     import oracle
     oracle.build()
-    cfg = wl.PREFILL_PYTHIA
+    cfg = {"prefill": wl.PREFILL_PYTHIA}.get(args.workload, wl.PREFILL_LONG)
     # each step: the oracle on every (batch, head) pair for a 64-token slice of
     # the sequence (a bounded sample of the workload)
     T = 64
@@ -714,7 +750,13 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "long", "decode", "mixer"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "long", "decode", "mixer"], default="long",
+                    help="long: B1 H8 L32768 prefill (default, the largest single-GPU scan "
+                         "workload); prefill: B4 H8 L2048; decode: 256 x 8 heads, 512 steps; "
+                         "mixer: B8 L4096 D2048")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (decode: sequences, mixer: B) for small "
+                         "profiling captures; the reported config says so")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

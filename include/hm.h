@@ -220,16 +220,18 @@ HM_API hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t wo
  * device memory (for example a plugin whose host application owns all device
  * memory and offers no allocator, or a serving loop that must not allocate
  * after start-up).  There is no counterpart in the paper; it is a deployment
- * convenience.  Same arguments and results as hm_step_decode, except that
- * workspace / workspace_bytes are ignored: the feature vectors live in a fixed
- * device array inside the library (two planes of 524,288 fp32 values, 4 MiB,
- * held by every GPU that loads the library until the process exits).
+ * convenience.  Same arguments, checks and results (bit-identical) as
+ * hm_step_decode, except that workspace / workspace_bytes are ignored: the
+ * fp32 feature vectors live in a fixed device array inside the library (two
+ * planes of 524,288 fp32 values, 4 MiB, held by every GPU that loads the
+ * library until the process exits).
  * Limit: when W_q != NULL, B * H * F must not exceed 524,288; larger calls
  * return HM_ERR_INVALID_ARG before anything is enqueued (use hm_step_decode).
  * All calls share that array, so calls whose kernels may overlap on a GPU
  * (several streams or host threads on one device) race and must be serialised
  * by the caller.  The first call on each device looks up the array's device
- * address; make that first call before any stream capture.
+ * address and caches it for the process; make that first call before any
+ * stream capture, and do not call this entry point after cudaDeviceReset.
  */
 HM_API hm_status hm_step_decode_noalloc(const hm_decode_args *a, hm_stream_t stream);
 

@@ -157,12 +157,6 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
 
 // ------------------------------------------------------------------ decode
 
-struct DecodePlan {
-    int F;
-    size_t phi_bytes;
-    size_t total;
-};
-
 hm_status check_decode(const hm_decode_args *a, DecodePlan *plan) {
     if (!a) return fail(HM_ERR_INVALID_ARG, "decode: null args");
     if (!valid_dtype(a->io_dtype)) return fail(HM_ERR_INVALID_ARG, "decode: bad io dtype");
@@ -176,7 +170,8 @@ hm_status check_decode(const hm_decode_args *a, DecodePlan *plan) {
     if (F > 256) return fail(HM_ERR_UNSUPPORTED, "decode: feature dim F=%d > 256", F);
     if (a->d > 512) return fail(HM_ERR_UNSUPPORTED, "decode: d=%d > 512", a->d);
     if (a->dv % 4 != 0) return fail(HM_ERR_UNSUPPORTED, "decode: dv must be a multiple of 4");
-    if (a->B * a->H > 0x7fffffffLL) return fail(HM_ERR_UNSUPPORTED, "decode: B*H too large");
+    if (a->B > 0x7fffffffLL || a->B * a->H > 0x7fffffffLL)
+        return fail(HM_ERR_UNSUPPORTED, "decode: B*H too large");
     if (a->B > 0 && (!a->q || !a->k || !a->v || !a->o || !a->S || !a->z))
         return fail(HM_ERR_INVALID_ARG, "decode: null q/k/v/o/S/z");
     const void *ptrs[] = {a->q, a->k, a->v, a->W_q, a->W_k, a->b_q, a->b_k, a->dt, a->A_log,
@@ -185,11 +180,48 @@ hm_status check_decode(const hm_decode_args *a, DecodePlan *plan) {
         if (!aligned16(p)) return fail(HM_ERR_INVALID_ARG, "decode: pointers must be 16-byte aligned");
     DecodePlan pl{};
     pl.F = F;
-    pl.phi_bytes = a->W_q ? round_up((size_t)a->B * a->H * F * sizeof(float), 256) : 0;
+    pl.feat_values = a->W_q ? a->B * a->H * F : 0;
+    pl.phi_bytes = a->W_q ? round_up((size_t)pl.feat_values * sizeof(float), 256) : 0;
     pl.total = 2 * pl.phi_bytes;
     *plan = pl;
     return HM_OK;
 }
+
+}  // namespace
+
+hm_status check_decode_args(const hm_decode_args *a, DecodePlan *plan) { return check_decode(a, plan); }
+
+// The decode step after its arguments were checked: per-token feature maps
+// into phq_buf / phk_buf (fp32, pl.feat_values each; unused when W_q == NULL),
+// then the state update.  Both decode entry points enqueue through here, so
+// they produce identical results.  The features are fp32 whatever the io
+// dtype: the state adds phi(k) v^T at every step, and a bf16 phi(k) would put
+// a 2^-9 relative error on each increment of S.
+hm_status decode_enqueue(const hm_decode_args *a, const DecodePlan &pl, void *phq_buf, void *phk_buf,
+                         cudaStream_t s) {
+    const int64_t rows = a->B * a->H;
+    if (rows == 0) return HM_OK;
+    const void *phq = a->q, *phk = a->k;
+    hm_dtype ft = a->io_dtype;
+    cudaError_t e;
+    if (a->W_q) {
+        e = run_featmap_qk(a->q, a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->W_k, a->w_head_stride,
+                           a->b_q, a->b_k, phq_buf, phk_buf, HM_F32, s);
+        if (e != cudaSuccess) return cuda_fail(e, "decode: feature maps");
+        phq = phq_buf;
+        phk = phk_buf;
+        ft = HM_F32;
+    }
+    DecodeCore c{};
+    c.B = a->B; c.H = a->H; c.F = pl.F; c.dv = a->dv;
+    c.feat_dtype = ft; c.io_dtype = a->io_dtype;
+    c.phq = phq; c.phk = phk; c.v = a->v; c.dt = a->dt; c.A_log = a->A_log;
+    c.S = a->S; c.z = a->z; c.o = a->o;
+    e = launch_decode(c, s);
+    return e == cudaSuccess ? HM_OK : cuda_fail(e, "decode launch");
+}
+
+namespace {
 
 // ------------------------------------------------------------------ mixer
 
@@ -401,30 +433,8 @@ hm_status hm_step_decode(const hm_decode_args *a, hm_stream_t stream) {
                     a->workspace_bytes, pl.total);
     if (((uintptr_t)a->workspace & 255u) != 0)
         return fail(HM_ERR_INVALID_ARG, "decode: workspace must be 256-byte aligned");
-    cudaStream_t s = (cudaStream_t)stream;
-    const int64_t rows = a->B * a->H;
-    const void *phq = a->q, *phk = a->k;
-    hm_dtype ft = a->io_dtype;
-    cudaError_t e;
-    if (a->W_q && rows > 0) {
-        char *ws = (char *)a->workspace;
-        // bf16 io: bf16 features, as in the prefill (the tensor-core map then
-        // writes them through its TMA-staged epilogue); fp32 io: fp32 features
-        const hm_dtype pt = a->io_dtype == HM_BF16 ? HM_BF16 : HM_F32;
-        e = run_featmap_qk(a->q, a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->W_k, a->w_head_stride,
-                           a->b_q, a->b_k, ws, ws + pl.phi_bytes, pt, s);
-        if (e != cudaSuccess) return cuda_fail(e, "decode: feature maps");
-        phq = ws;
-        phk = ws + pl.phi_bytes;
-        ft = pt;
-    }
-    DecodeCore c{};
-    c.B = a->B; c.H = a->H; c.F = pl.F; c.dv = a->dv;
-    c.feat_dtype = ft; c.io_dtype = a->io_dtype;
-    c.phq = phq; c.phk = phk; c.v = a->v; c.dt = a->dt; c.A_log = a->A_log;
-    c.S = a->S; c.z = a->z; c.o = a->o;
-    e = launch_decode(c, s);
-    return e == cudaSuccess ? HM_OK : cuda_fail(e, "decode launch");
+    char *ws = (char *)a->workspace;
+    return decode_enqueue(a, pl, ws, ws + pl.phi_bytes, (cudaStream_t)stream);
 }
 
 size_t hm_mixer_workspace_size(const hm_mixer_args *a) {

@@ -130,6 +130,23 @@ struct DecodeCore {
 };
 cudaError_t launch_decode(const DecodeCore &c, cudaStream_t s);
 
+// Checked shape of a decode call: F, and the size of each per-token feature
+// plane (B * H * F values when W_q != NULL, else 0) and of the workspace.
+struct DecodePlan {
+    int F;
+    int64_t feat_values;
+    size_t phi_bytes;   // one feature plane, fp32, rounded up to 256 bytes
+    size_t total;       // workspace bytes of hm_step_decode
+};
+
+// Argument check shared by every decode entry point (sets the error detail).
+hm_status check_decode_args(const hm_decode_args *a, DecodePlan *plan);
+
+// Enqueues a checked decode step with its feature planes at phq_buf / phk_buf
+// (fp32, plan.feat_values each; ignored when W_q == NULL).
+hm_status decode_enqueue(const hm_decode_args *a, const DecodePlan &plan, void *phq_buf, void *phk_buf,
+                         cudaStream_t s);
+
 // bf16 GEMM C[M,N] = A[M,K] B[N,K]^T on tcgen05 with a fused epilogue.
 enum GemmEpi : int {
     EPI_STORE_BF16 = 0,  // C bf16

@@ -101,10 +101,14 @@ constexpr uint32_t kWaitPolls = 1u << 22;
 
 // Bounded wait on phase `parity` of `bar`.  Returns false (after recording a
 // timeout in the device error word and raising the CTA's abort flag) if the
-// phase does not complete, or if another thread of the CTA already aborted.
+// phase does not complete within `max_polls` polls, or if another thread of
+// the CTA already aborted.  Every pipelined kernel waits through this
+// function with the default limit; the library's self-test calls it with a
+// small limit on a barrier that is never signalled.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          DevErr err, unsigned kid, unsigned site) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+                                          DevErr err, unsigned kid, unsigned site,
+                                          uint32_t max_polls = kWaitPolls) {
+    for (uint32_t i = 0; i < max_polls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 63u && *abort_flag) return false;
     }

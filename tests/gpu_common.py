@@ -24,6 +24,28 @@ def rel_err(x, r):
     return float(np.max(np.abs(x - r) / np.maximum(np.abs(r), scale)))
 
 
+def rel_err_rows(x, r):
+    """max_i |x_i - r_i| / max(|r_i|, rms of r's row) over rows of the last axis.
+
+    For outputs whose scale varies by orders of magnitude from token to token
+    (with a = 1 the mixer's output at token t is a t-token average, ~1/sqrt(t)
+    of the first token's), the floor is the token's own output scale instead
+    of the whole tensor's."""
+    x = np.asarray(x, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    if r.size == 0:
+        return 0.0
+    scale = np.maximum(np.sqrt(np.mean(r * r, axis=-1, keepdims=True)), 1e-30)
+    return float(np.max(np.abs(x - r) / np.maximum(np.abs(r), scale)))
+
+
+def rel_err_norm(x, r):
+    """Normwise relative error ||x - r||_2 / ||r||_2."""
+    x = np.asarray(x, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    return float(np.linalg.norm(x - r) / max(np.linalg.norm(r), 1e-300))
+
+
 def dev_tensor(a, dtype, device="cuda"):
     import torch
     t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)

@@ -6,6 +6,8 @@ import os
 import subprocess
 import sys
 
+import workloads as wl  # noqa: E402
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -22,7 +24,7 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
     assert d["warmup"] >= 3 and d["steps"] == 1 and d["higher_is_better"] is True
-    assert d["config"]["workload"] == "prefill_B4_H8_L2048_d256_F256_bf16"
+    assert d["config"]["workload"] == wl.PREFILL_LONG.name   # the default workload
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

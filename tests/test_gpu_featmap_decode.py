@@ -149,6 +149,40 @@ def test_decode_steps_full_size_sampled_heads(hm):
     assert hm.hm_get_device_error() == hm.HM_OK
 
 
+def test_decode_all_heads_16_steps_against_oracle(hm):
+    """Every one of the 256 x 8 heads, 16 consecutive hm_step_decode calls,
+    from a small seeded state (so that the per-step increments phi(k) v^T,
+    not the initial state, make up S): o at every step and the final S and z
+    against the oracle's own decode steps."""
+    import torch
+    cfg = wl.DECODE
+    steps = 16
+    w = wl.decode_weights(cfg)
+    B, H, F, dv = cfg.B, cfg.H, cfg.F, cfg.dv
+    S_ref = wl.round_f32(np.abs(wl.normal(cfg.seed, "S_all", (B, H, F, dv), 0.01)))
+    z_ref = wl.round_f32(np.abs(wl.normal(cfg.seed, "z_all", (B, H, F), 0.01)) + 1e-3)
+    tS, tz = dev_tensor(S_ref, "f32"), dev_tensor(z_ref, "f32")
+    tWq, tWk = dev_tensor(w["W_q"], "bf16"), dev_tensor(w["W_k"], "bf16")
+    tA = dev_tensor(w["A_log"], "f32")
+    for t in range(steps):
+        tok = wl.decode_step_tokens(cfg, 300 + t)
+        tq, tk, tv = (dev_tensor(tok[n], "bf16") for n in ("q", "k", "v"))
+        o = torch.empty_like(tv)
+        args = hm.decode_args(tq, tk, tv, o, tS, tz, W_q=tWq, W_k=tWk,
+                              dt=dev_tensor(tok["dt"], "f32"), A_log=tA)
+        ws = hm.alloc_workspace(hm.hm_decode_workspace_size(args))
+        args.workspace, args.workspace_bytes = ws.data_ptr(), ws.numel()
+        hm.hm_step_decode(args)
+        phq = oracle.featmap(tok["q"], w["W_q"])
+        phk = oracle.featmap(tok["k"], w["W_k"])
+        la = oracle.log_decay(tok["dt"], w["A_log"])
+        o_ref, S_ref, z_ref = oracle.decode_step(phq, phk, tok["v"], S_ref, z_ref, la)
+        assert rel_err(to_np(o), o_ref) <= TOL_BF16, t
+    assert hm.hm_get_device_error() == hm.HM_OK
+    assert rel_err(to_np(tS), S_ref) <= TOL_BF16
+    assert rel_err(to_np(tz), z_ref) <= TOL_BF16
+
+
 def test_decode_continues_gpu_prefill(hm):
     """prefill(L) then n decode steps = prefill(L + n) (both on the GPU and
     compared with the oracle's single prefill)."""

@@ -110,6 +110,21 @@ def test_featmap_per_head_weights(oracle_mod):
         np.testing.assert_allclose(phi[:, :, h], ref, rtol=1e-14)
 
 
+def test_featmap_per_head_bias_log_ratio(oracle_mod):
+    # per-head weights and biases (a bias has the per-head layout of its
+    # weights: one [p] row per head): for each head h,
+    # log(phi_f / phi_{f+p}) = 2 (W_h x + b_h)_f, against a library matmul
+    H, d, p = 3, 10, 4
+    x = rng.normal(size=(2, 7, H, d))
+    W = rng.normal(size=(H, p, d)) / 3
+    b = rng.normal(size=(H, p))
+    phi = oracle_mod.featmap(x, W, bias=b, H=H, w_head_stride=p * d, b_head_stride=p)
+    for h in range(H):
+        u = x[:, :, h] @ W[h].T + b[h]
+        np.testing.assert_allclose(np.log(phi[:, :, h, :p] / phi[:, :, h, p:]), 2 * u,
+                                   rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- the scan
 
 def _tiny_case(B=2, L=13, H=2, F=6, dv=3, decay=True, zero_at=None):
