@@ -74,6 +74,14 @@ def _load():
         lib.hmo_scan_quadratic.argtypes = [I64, I64, I, I, I, P, P, P, P, P]
         lib.hmo_decode_step.restype = I64
         lib.hmo_decode_step.argtypes = [I64, I, I, I, P, P, P, P, P, P, P]
+        lib.hmo_scan_recurrent_ext.restype = I64
+        lib.hmo_scan_recurrent_ext.argtypes = [I64, I64, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
+        lib.hmo_scan_quadratic_ext.restype = None
+        lib.hmo_scan_quadratic_ext.argtypes = [I64, I64, I, I, I, P, P, P, P, P, P, P]
+        lib.hmo_log_decay_f.restype = None
+        lib.hmo_log_decay_f.argtypes = [P, I64, I, I, P, P]
+        lib.hmo_step_size.restype = None
+        lib.hmo_step_size.argtypes = [P, I64, P]
         lib.hmo_causal_conv.restype = None
         lib.hmo_causal_conv.argtypes = [I64, I64, I, I, P, P, P, P]
         _lib = lib
@@ -159,6 +167,64 @@ def scan_recurrent(phq, phk, v, log_a=None, S0=None, z0=None, return_state=False
     return o
 
 
+def log_decay_per_feature(dt, A_log_f):
+    """l[b,t,h,f] = -softplus(dt[b,t,h]) * exp(A_log_f[h,f]) (the per-feature
+    decay variant; [LA] sec. 4.4).  dt: [..., H]; A_log_f: [H, F]."""
+    dt = _f64(dt)
+    A = _f64(A_log_f)
+    H, F = A.shape
+    assert dt.shape[-1] == H
+    out = np.empty(dt.shape + (F,), dtype=np.float64)
+    _load().hmo_log_decay_f(_ptr(dt), dt.size // H, H, F, _ptr(A), _ptr(out))
+    return out
+
+
+def step_size(dt):
+    """Delta = softplus(dt) ([SSM] sec. 3.2), elementwise."""
+    dt = _f64(dt)
+    out = np.empty_like(dt)
+    _load().hmo_step_size(_ptr(dt), dt.size, _ptr(out))
+    return out
+
+
+def scan_recurrent_ext(phq, phk, v, log_a=None, log_a_f=None, in_scale=None, S0=None, z0=None,
+                       return_state=False):
+    """The recurrence with the step-scaled input (in_scale = Delta, [HM]
+    sec. 5.2 / [SSM] sec. 3.2) and/or a per-feature decay (log_a_f
+    [B, L, H, F], [LA] sec. 4.4); see hmo_scan_recurrent_ext."""
+    phq, phk, v = _f64(phq), _f64(phk), _f64(v)
+    B, L, H, F = phq.shape
+    dv = v.shape[-1]
+    la = None if log_a is None else _f64(log_a)
+    laf = None if log_a_f is None else _f64(log_a_f)
+    sc = None if in_scale is None else _f64(in_scale)
+    S0 = None if S0 is None else _f64(S0)
+    z0 = None if z0 is None else _f64(z0)
+    o = np.empty((B, L, H, dv), dtype=np.float64)
+    S = np.empty((B, H, F, dv), dtype=np.float64) if return_state else None
+    z = np.empty((B, H, F), dtype=np.float64) if return_state else None
+    bad = _load().hmo_scan_recurrent_ext(B, L, H, F, dv, _ptr(phq), _ptr(phk), _ptr(v), _ptr(la),
+                                         _ptr(laf), _ptr(sc), _ptr(S0), _ptr(z0), _ptr(o), _ptr(S),
+                                         _ptr(z))
+    if bad:
+        raise FloatingPointError("oracle: %d denominators were not > 0" % bad)
+    return (o, S, z) if return_state else o
+
+
+def scan_quadratic_ext(phq, phk, v, log_a=None, log_a_f=None, in_scale=None):
+    """O(L^2) masked form of scan_recurrent_ext (zero initial state)."""
+    phq, phk, v = _f64(phq), _f64(phk), _f64(v)
+    B, L, H, F = phq.shape
+    dv = v.shape[-1]
+    la = None if log_a is None else _f64(log_a)
+    laf = None if log_a_f is None else _f64(log_a_f)
+    sc = None if in_scale is None else _f64(in_scale)
+    o = np.empty((B, L, H, dv), dtype=np.float64)
+    _load().hmo_scan_quadratic_ext(B, L, H, F, dv, _ptr(phq), _ptr(phk), _ptr(v), _ptr(la), _ptr(laf),
+                                   _ptr(sc), _ptr(o))
+    return o
+
+
 def scan_quadratic(phq, phk, v, log_a=None):
     """O(L^2) masked form ([LA] sec. 2): o_i = sum_{j<=i} w_ij v_j / sum_j w_ij,
     w_ij = exp(sum_{j<t<=i} l_t) phiq_i . phik_j.  Zero initial state."""
@@ -214,12 +280,14 @@ def silu(x):
 # --------------------------------------------------------------------------
 
 def scan_fwd(q, k, v, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=None,
-             S0=None, z0=None, w_head_stride=0, return_state=False):
+             S0=None, z0=None, w_head_stride=0, return_state=False, dt_scaled_input=False):
     """Feature map on q and k, then the decayed normalised recurrence.
 
     q, k: [B, L, H, d]; v: [B, L, H, dv]; W_q, W_k: [p, d] (or per-head); if
     W_q is None, q and k are taken as feature vectors already (F = d).
-    dt: [B, L, H] or None (a = 1); A_log: [H]."""
+    dt: [B, L, H] or None (a = 1); A_log: [H], or [H, F] for a decay per
+    feature.  dt_scaled_input: the input term is multiplied by Delta =
+    softplus(dt) (Mamba's discretised input)."""
     q, k = _f64(q), _f64(k)
     B, L, H, d = q.shape
     if W_q is None:
@@ -229,8 +297,16 @@ def scan_fwd(q, k, v, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=Non
         bstride = W_q.shape[-2] if w_head_stride else 0
         phq = featmap(q, W_q, b_q, H=H, w_head_stride=w_head_stride, b_head_stride=bstride)
         phk = featmap(k, W_k, b_k, H=H, w_head_stride=w_head_stride, b_head_stride=bstride)
-    la = None if dt is None else log_decay(dt, A_log)
-    return scan_recurrent(phq, phk, v, la, S0, z0, return_state=return_state)
+    per_feature = A_log is not None and np.ndim(A_log) == 2
+    if not per_feature and not dt_scaled_input:
+        la = None if dt is None else log_decay(dt, A_log)
+        return scan_recurrent(phq, phk, v, la, S0, z0, return_state=return_state)
+    assert dt is not None, "the variants are functions of dt"
+    la = None if per_feature else log_decay(dt, A_log)
+    laf = log_decay_per_feature(dt, A_log) if per_feature else None
+    sc = step_size(dt) if dt_scaled_input else None
+    return scan_recurrent_ext(phq, phk, v, log_a=la, log_a_f=laf, in_scale=sc, S0=S0, z0=z0,
+                              return_state=return_state)
 
 
 # --------------------------------------------------------------------------

@@ -59,6 +59,27 @@ HMO_EXPORT void hmo_log_decay(const double *dt, int64_t BL, int H,
         }
 }
 
+/* Per-feature log decay (the per-dimension decay variant, see
+ * hmo_scan_recurrent_ext):  l[b,t,h,f] = -softplus(dt[b,t,h]) * exp(A_log_f[h,f]).
+ * BL = B*L; A_log_f is [H, F]; log_a_f is [BL, H, F]. */
+HMO_EXPORT void hmo_log_decay_f(const double *dt, int64_t BL, int H, int F,
+                                const double *A_log_f, double *log_a_f) {
+    for (int64_t r = 0; r < BL; ++r)
+        for (int h = 0; h < H; ++h) {
+            double sp = hmo_softplus(dt[r * H + h]);
+            for (int f = 0; f < F; ++f) {
+                double rate = exp(A_log_f[(int64_t)h * F + f]);
+                log_a_f[(r * H + h) * F + f] = (rate == 0.0) ? 0.0 : -sp * rate;
+            }
+        }
+}
+
+/* Step size Delta = softplus(dt) ([SSM] sec. 3.2), the factor of the input
+ * term in the step-scaled variant; n values. */
+HMO_EXPORT void hmo_step_size(const double *dt, int64_t n, double *delta) {
+    for (int64_t i = 0; i < n; ++i) delta[i] = hmo_softplus(dt[i]);
+}
+
 /* Hedgehog feature map, [HM] sec. 2.1 and sec. 5.3:
  *   u   = W x + b                      (one Linear layer, W is [p, d])
  *   phi = softmax([u, -u])             over the 2p feature axis
@@ -186,6 +207,108 @@ HMO_EXPORT void hmo_scan_quadratic(int64_t B, int64_t L, int H, int F, int dv,
             }
             for (int c = 0; c < dv; ++c) oo[c] /= den;
         }
+    }
+}
+
+/* The recurrence with the two variants of the pages that the plain form
+ * leaves out (both off gives exactly hmo_scan_recurrent):
+ *
+ *  - input scaled by the step size ([HM] sec. 5.2: the mixer calls Mamba's
+ *    selective scan, whose discretised input is B-bar = Delta B; [SSM] sec.
+ *    3.2: Delta = softplus(dt)).  With in_scale[b,t,h] = Delta_t:
+ *        S_t = a_t S_{t-1} + Delta_t phik_t v_t^T,  z_t = a_t z_{t-1} + Delta_t phik_t
+ *  - a decay per feature ([LA] sec. 4.4, gated linear attention's
+ *    S_i = diag(alpha_i) S_{i-1} + k_i v_i^T; Mamba-1 keeps one A per state
+ *    dimension).  With log_a_f[b,t,h,f]:
+ *        S_t[f,:] = a_{t,f} S_{t-1}[f,:] + ...,  z_t[f] = a_{t,f} z_{t-1}[f] + ...
+ *    replacing the scalar log_a.
+ * in_scale [B,L,H] or NULL (1); log_a [B,L,H] or NULL; log_a_f [B,L,H,F] or
+ * NULL (when given, log_a is ignored).  Other arguments and the return value
+ * as hmo_scan_recurrent. */
+HMO_EXPORT int64_t hmo_scan_recurrent_ext(int64_t B, int64_t L, int H, int F, int dv,
+                                          const double *phq, const double *phk,
+                                          const double *v, const double *log_a,
+                                          const double *log_a_f, const double *in_scale,
+                                          const double *S0, const double *z0,
+                                          double *o, double *S_out, double *z_out) {
+    int64_t bad = 0;
+    #pragma omp parallel for schedule(dynamic) reduction(+ : bad)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        int64_t b = bh / H;
+        int h = (int)(bh % H);
+        double *S = (double *)calloc((size_t)F * dv, sizeof(double));
+        double *z = (double *)calloc((size_t)F, sizeof(double));
+        if (S0) memcpy(S, S0 + bh * F * dv, sizeof(double) * (size_t)F * dv);
+        if (z0) memcpy(z, z0 + bh * F, sizeof(double) * (size_t)F);
+        for (int64_t t = 0; t < L; ++t) {
+            int64_t row = (b * L + t) * H + h;
+            double sc = in_scale ? in_scale[row] : 1.0;
+            const double *qk = phq + row * F;
+            const double *kk = phk + row * F;
+            const double *vv = v + row * dv;
+            for (int f = 0; f < F; ++f) {
+                double a = log_a_f ? exp(log_a_f[row * F + f]) : (log_a ? exp(log_a[row]) : 1.0);
+                double kf = sc * kk[f];
+                z[f] = a * z[f] + kf;
+                for (int c = 0; c < dv; ++c)
+                    S[(int64_t)f * dv + c] = a * S[(int64_t)f * dv + c] + kf * vv[c];
+            }
+            double den = 0.0;
+            for (int f = 0; f < F; ++f) den += qk[f] * z[f];
+            if (!(den > 0.0)) bad += 1;
+            double *oo = o + row * dv;
+            for (int c = 0; c < dv; ++c) {
+                double num = 0.0;
+                for (int f = 0; f < F; ++f) num += qk[f] * S[(int64_t)f * dv + c];
+                oo[c] = num / den;
+            }
+        }
+        if (S_out) memcpy(S_out + bh * F * dv, S, sizeof(double) * (size_t)F * dv);
+        if (z_out) memcpy(z_out + bh * F, z, sizeof(double) * (size_t)F);
+        free(S);
+        free(z);
+    }
+    return bad;
+}
+
+/* The O(L^2) masked form of hmo_scan_recurrent_ext (zero initial state):
+ *   w_ij = Delta_j * sum_f phiq_if phik_jf exp( sum_{j < t <= i} l_{t,f} ),  j <= i
+ *   o_i  = sum_j w_ij v_j / sum_j w_ij
+ * with l_{t,f} = log_a_f[t,f] (or log_a[t] for every f, or 0) and Delta_j =
+ * in_scale[j] (or 1).  Each feature's decay sum is accumulated directly, as in
+ * hmo_scan_quadratic.  Tiny sizes only. */
+HMO_EXPORT void hmo_scan_quadratic_ext(int64_t B, int64_t L, int H, int F, int dv,
+                                       const double *phq, const double *phk,
+                                       const double *v, const double *log_a,
+                                       const double *log_a_f, const double *in_scale,
+                                       double *o) {
+    #pragma omp parallel for schedule(dynamic)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        int64_t b = bh / H;
+        int h = (int)(bh % H);
+        double *logw = (double *)malloc(sizeof(double) * (size_t)F);
+        for (int64_t i = 0; i < L; ++i) {
+            int64_t ri = (b * L + i) * H + h;
+            double *oo = o + ri * dv;
+            for (int c = 0; c < dv; ++c) oo[c] = 0.0;
+            for (int f = 0; f < F; ++f) logw[f] = 0.0;
+            double den = 0.0;
+            for (int64_t j = i; j >= 0; --j) {
+                int64_t rj = (b * L + j) * H + h;
+                if (j < i) {
+                    int64_t rt = (b * L + (j + 1)) * H + h;
+                    for (int f = 0; f < F; ++f)
+                        logw[f] += log_a_f ? log_a_f[rt * F + f] : (log_a ? log_a[rt] : 0.0);
+                }
+                double w = 0.0;
+                for (int f = 0; f < F; ++f) w += phq[ri * F + f] * phk[rj * F + f] * exp(logw[f]);
+                if (in_scale) w *= in_scale[rj];
+                den += w;
+                for (int c = 0; c < dv; ++c) oo[c] += w * v[rj * dv + c];
+            }
+            for (int c = 0; c < dv; ++c) oo[c] /= den;
+        }
+        free(logw);
     }
 }
 
