@@ -79,6 +79,27 @@ typedef enum {
 
 typedef enum { HM_F32 = 0, HM_BF16 = 1 } hm_dtype;
 
+/*
+ * Variant flags of the scan and the decode step (the `flags` field of
+ * hm_scan_args / hm_decode_args; 0 = the plain recurrence above).
+ *
+ * HM_FLAG_DT_SCALED_INPUT  the input term is multiplied by the step size
+ *     Delta_t = softplus(dt_t), as in Mamba's discretised input B-bar = Delta B
+ *     (HedgeMamba explainer sec. 5.2: the mixer calls Mamba's selective scan;
+ *     SSM article sec. 3.2):
+ *         S_t = a_t S_{t-1} + Delta_t phi(k_t) v_t^T,  z_t = a_t z_{t-1} + Delta_t phi(k_t)
+ *     Requires dt.
+ * HM_FLAG_PER_FEATURE_DECAY  one decay rate per (head, feature): A_log is
+ *     [H, F] and a_{t,f} = exp(-softplus(dt_t) * exp(A_log[h, f])) scales row
+ *     f of S and entry f of z (gated linear attention's diag(alpha) S,
+ *     linear-attention tutorial sec. 4.4; Mamba-1's A per state dimension).
+ *     Requires dt.  Runs on the CUDA-core scan (no tensor-core kernel).
+ */
+typedef enum {
+    HM_FLAG_DT_SCALED_INPUT = 1u,
+    HM_FLAG_PER_FEATURE_DECAY = 2u
+} hm_flag;
+
 /* Static description of a status code.  Never NULL. */
 HM_API const char *hm_status_string(hm_status s);
 
@@ -133,14 +154,20 @@ typedef struct {
     const float *b_q;      /* [p] bias of the q map (per head like W) or NULL */
     const float *b_k;      /* [p] bias of the k map or NULL */
     const float *dt;       /* [B, L, H] fp32, or NULL: a_t = 1 (no decay) */
-    const float *A_log;    /* [H] fp32; required when dt != NULL */
+    const float *A_log;    /* [H] fp32 ([H, F] with HM_FLAG_PER_FEATURE_DECAY); required with dt */
     const float *S0;       /* [B, H, F, dv] initial state, or NULL (zero) */
     const float *z0;       /* [B, H, F] initial state, or NULL (zero); NULL iff S0 NULL */
-    void *o;               /* [B, L, H, dv] of io_dtype (written) */
+    void *o;               /* [B, L, H, dv] of io_dtype (written), or NULL for a state-only
+                              call (S_out required): only the final state is computed */
     float *S_out;          /* [B, H, F, dv] final state, or NULL; may alias S0 */
     float *z_out;          /* [B, H, F] final state, or NULL; may alias z0 */
     void *workspace;       /* device scratch of >= hm_scan_workspace_size() bytes, 256-B aligned */
     size_t workspace_bytes;
+    unsigned int flags;    /* hm_flag bits (0: the plain recurrence); unknown bits are rejected */
+    float *log_decay_out;  /* [B, H] (per-feature decay: [B, H, F]) sum over the call's tokens of
+                              log a_t, i.e. the log of the decay the whole call applies to the
+                              state it starts from; or NULL.  With S_out of a zero-start call
+                              it is the call's affine map S -> exp(.) S + S_out (hm_scan_combine). */
 } hm_scan_args;
 
 /* Bytes of workspace hm_scan_chunked_fwd needs for these arguments (0 on
@@ -148,6 +175,45 @@ typedef struct {
 HM_API size_t hm_scan_workspace_size(const hm_scan_args *a);
 
 HM_API hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stream);
+
+/*
+ * hm_scan_combine -- start states of consecutive sequence segments from their
+ * own zero-start results (SSM article sec. 4.2: the maps S -> A S + b compose
+ * associatively, (A2, b2) o (A1, b1) = (A2 A1, A2 b1 + b2); here A is the
+ * diagonal decay exp(log_decay) and b the segment's zero-start end state).
+ *
+ * A sequence cut into n_parts consecutive segments (for example one per GPU)
+ * is scanned segment by segment with S0 = NULL, S_out, z_out and log_decay_out
+ * (o may be NULL).  Part r's results sit in one flat fp32 record at
+ * parts + r * part_len, laid out [log_decay | S | z]:
+ *     log_decay  BH values (BH * F with per_feature), padded with unread
+ *                values to a multiple of 4
+ *     S          BH * F * dv values ([BH][F][dv])
+ *     z          BH * F values
+ * (part_len >= their total; the layout an all-gather of per-rank records
+ * produces).  The start state of part r is then
+ *     start_0 = (S0, z0) or zero,   start_{r+1} = exp(log_decay_r) (.) start_r + (S_r, z_r)
+ * and the segment's outputs are those of a scan with S0 = start_r.
+ * only_part = -1 writes every part's start to S_start [n_parts][BH][F][dv] and
+ * z_start [n_parts][BH][F]; only_part = r writes just part r's start (one
+ * [BH][F][dv] / [BH][F] block).  S_end / z_end (nullable) receive start_{n_parts},
+ * the state after the whole sequence.  All pointers device, fp32, 16-byte
+ * aligned; part_len a multiple of 4.
+ */
+typedef struct {
+    int64_t n_parts;       /* segments, in sequence order */
+    int64_t BH;            /* batch x heads */
+    int F, dv;             /* state shape per head */
+    int per_feature;       /* log_decay has F values per head (HM_FLAG_PER_FEATURE_DECAY) */
+    const float *parts;    /* n_parts records of part_len floats */
+    int64_t part_len;
+    const float *S0, *z0;  /* start of part 0 ([BH][F][dv], [BH][F]) or NULL (zero) */
+    int64_t only_part;     /* -1: all parts' starts; else the one part whose start is written */
+    float *S_start, *z_start;
+    float *S_end, *z_end;  /* nullable */
+} hm_combine_args;
+
+HM_API hm_status hm_scan_combine(const hm_combine_args *a, hm_stream_t stream);
 
 /*
  * hm_step_decode -- one recurrent step per (batch, head) (linear-attention
@@ -166,12 +232,13 @@ typedef struct {
     int64_t w_head_stride;
     const float *b_q, *b_k;
     const float *dt;       /* [B, H] fp32 or NULL (a = 1) */
-    const float *A_log;    /* [H] fp32 */
+    const float *A_log;    /* [H] fp32 ([H, F] with HM_FLAG_PER_FEATURE_DECAY) */
     float *S;              /* [B, H, F, dv] fp32, read and written */
     float *z;              /* [B, H, F] fp32, read and written */
     void *o;               /* [B, H, dv] of io_dtype (written) */
     void *workspace;       /* >= hm_decode_workspace_size() bytes, 256-B aligned */
     size_t workspace_bytes;
+    unsigned int flags;    /* hm_flag bits, as in hm_scan_args */
 } hm_decode_args;
 
 HM_API size_t hm_decode_workspace_size(const hm_decode_args *a);

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libhm.so")
 
 HM_OK, HM_ERR_INVALID_ARG, HM_ERR_UNSUPPORTED, HM_ERR_CUDA, HM_ERR_TIMEOUT, HM_ERR_DEVICE = range(6)
 HM_F32, HM_BF16 = 0, 1
+HM_FLAG_DT_SCALED_INPUT, HM_FLAG_PER_FEATURE_DECAY = 1, 2
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libhm.so is not built (%s); run __graft_entry__.build() or "
@@ -36,7 +37,15 @@ class ScanArgs(ctypes.Structure):
                 ("io_dtype", _I), ("q", _P), ("k", _P), ("v", _P), ("W_q", _P), ("W_k", _P),
                 ("w_head_stride", _I64), ("b_q", _P), ("b_k", _P), ("dt", _P), ("A_log", _P),
                 ("S0", _P), ("z0", _P), ("o", _P), ("S_out", _P), ("z_out", _P),
-                ("workspace", _P), ("workspace_bytes", _SZ)]
+                ("workspace", _P), ("workspace_bytes", _SZ), ("flags", ctypes.c_uint),
+                ("log_decay_out", _P)]
+
+
+class CombineArgs(ctypes.Structure):
+    """Mirror of hm_combine_args."""
+    _fields_ = [("n_parts", _I64), ("BH", _I64), ("F", _I), ("dv", _I), ("per_feature", _I),
+                ("parts", _P), ("part_len", _I64), ("S0", _P), ("z0", _P), ("only_part", _I64),
+                ("S_start", _P), ("z_start", _P), ("S_end", _P), ("z_end", _P)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -44,7 +53,8 @@ class DecodeArgs(ctypes.Structure):
     _fields_ = [("B", _I64), ("H", _I), ("d", _I), ("p", _I), ("dv", _I), ("io_dtype", _I),
                 ("q", _P), ("k", _P), ("v", _P), ("W_q", _P), ("W_k", _P),
                 ("w_head_stride", _I64), ("b_q", _P), ("b_k", _P), ("dt", _P), ("A_log", _P),
-                ("S", _P), ("z", _P), ("o", _P), ("workspace", _P), ("workspace_bytes", _SZ)]
+                ("S", _P), ("z", _P), ("o", _P), ("workspace", _P), ("workspace_bytes", _SZ),
+                ("flags", ctypes.c_uint)]
 
 
 class MixerArgs(ctypes.Structure):
@@ -76,6 +86,8 @@ lib.hm_mixer_workspace_size.restype = _SZ
 lib.hm_mixer_workspace_size.argtypes = [ctypes.POINTER(MixerArgs)]
 lib.hm_mixer_fwd.restype = _I
 lib.hm_mixer_fwd.argtypes = [ctypes.POINTER(MixerArgs), _P, _SZ, _P]
+lib.hm_scan_combine.restype = _I
+lib.hm_scan_combine.argtypes = [ctypes.POINTER(CombineArgs), _P]
 lib.hm_launch_count.restype = ctypes.c_uint64
 lib.hm_launch_count.argtypes = []
 lib.hm_get_device_error.restype = _I
@@ -86,7 +98,7 @@ lib.hm_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
 EXPORTED = ("hm_status_string", "hm_last_error_detail", "hm_version", "hm_featmap",
             "hm_scan_workspace_size", "hm_scan_chunked_fwd", "hm_decode_workspace_size",
             "hm_step_decode", "hm_mixer_workspace_size", "hm_mixer_fwd", "hm_get_device_error",
-            "hm_launch_count", "hm_step_decode_noalloc", "hm_selftest_wait_timeout")
+            "hm_launch_count", "hm_step_decode_noalloc", "hm_selftest_wait_timeout", "hm_scan_combine")
 
 
 class HMError(RuntimeError):
@@ -159,24 +171,27 @@ def hm_featmap(x, W, phi, H: int = 1, bias=None, w_head_stride: int = 0, stream=
 
 def scan_args(q, k, v, o, W_q=None, W_k=None, dt=None, A_log=None, S0=None, z0=None,
               S_out=None, z_out=None, b_q=None, b_k=None, w_head_stride: int = 0,
-              workspace=None) -> ScanArgs:
-    """Fill an hm_scan_args from tensors (q, k: [B, L, H, d]; v, o: [B, L, H, dv])."""
-    B, L, H, d = q.shape
+              workspace=None, flags: int = 0, log_decay_out=None) -> ScanArgs:
+    """Fill an hm_scan_args from tensors (q, k: [B, L, H, d]; v, o: [B, L, H, dv]).
+    o = None (with S_out) makes a state-only call; q may then be None too."""
+    B, L, H, d = k.shape
     dv = v.shape[-1]
     a = ScanArgs()
     a.B, a.L, a.H, a.d, a.dv = B, L, H, d, dv
     a.p = W_q.shape[-2] if W_q is not None else 0
-    a.io_dtype = _dtype_code(q)
+    a.io_dtype = _dtype_code(k)
     a.q, a.k, a.v, a.o = _ptr(q), _ptr(k), _ptr(v), _ptr(o)
     a.W_q, a.W_k, a.w_head_stride = _ptr(W_q), _ptr(W_k), int(w_head_stride)
     a.b_q, a.b_k = _ptr(b_q), _ptr(b_k)
     a.dt, a.A_log = _ptr(dt), _ptr(A_log)
     a.S0, a.z0, a.S_out, a.z_out = _ptr(S0), _ptr(z0), _ptr(S_out), _ptr(z_out)
+    a.flags = int(flags)
+    a.log_decay_out = _ptr(log_decay_out)
     if workspace is not None:
         a.workspace = _ptr(workspace)
         a.workspace_bytes = workspace.numel() * workspace.element_size()
     # the struct holds raw addresses: keep the tensors alive as long as it lives
-    a._refs = (q, k, v, o, W_q, W_k, dt, A_log, S0, z0, S_out, z_out, b_q, b_k, workspace)
+    a._refs = (q, k, v, o, W_q, W_k, dt, A_log, S0, z0, S_out, z_out, b_q, b_k, workspace, log_decay_out)
     return a
 
 
@@ -188,8 +203,32 @@ def hm_scan_chunked_fwd(args: ScanArgs, stream=None) -> None:
     _check(lib.hm_scan_chunked_fwd(ctypes.byref(args), _stream(stream)), "hm_scan_chunked_fwd")
 
 
+def combine_args(parts, n_parts: int, BH: int, F: int, dv: int, part_len: int, S_start, z_start,
+                 per_feature: bool = False, S0=None, z0=None, only_part: int = -1, S_end=None,
+                 z_end=None) -> CombineArgs:
+    """Fill an hm_combine_args: `parts` holds n_parts records of part_len fp32
+    values, each [log_decay (padded to 4) | S | z] of one sequence segment."""
+    a = CombineArgs()
+    a.n_parts, a.BH, a.F, a.dv, a.per_feature = int(n_parts), int(BH), int(F), int(dv), int(per_feature)
+    a.parts, a.part_len = _ptr(parts), int(part_len)
+    a.S0, a.z0, a.only_part = _ptr(S0), _ptr(z0), int(only_part)
+    a.S_start, a.z_start, a.S_end, a.z_end = _ptr(S_start), _ptr(z_start), _ptr(S_end), _ptr(z_end)
+    a._refs = (parts, S0, z0, S_start, z_start, S_end, z_end)
+    return a
+
+
+def hm_scan_combine(args: CombineArgs, stream=None) -> None:
+    _check(lib.hm_scan_combine(ctypes.byref(args), _stream(stream)), "hm_scan_combine")
+
+
+def combine_record_len(BH: int, F: int, dv: int, per_feature: bool = False) -> int:
+    """fp32 values of one [log_decay | S | z] record (the log-decay part padded to 4)."""
+    nl = BH * F if per_feature else BH
+    return (nl + 3) // 4 * 4 + BH * F * dv + BH * F
+
+
 def decode_args(q, k, v, o, S, z, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=None,
-                w_head_stride: int = 0, workspace=None) -> DecodeArgs:
+                w_head_stride: int = 0, workspace=None, flags: int = 0) -> DecodeArgs:
     """Fill an hm_decode_args (q, k: [B, H, d]; v, o: [B, H, dv]; S: [B, H, F, dv])."""
     B, H, d = q.shape
     a = DecodeArgs()
@@ -201,6 +240,7 @@ def decode_args(q, k, v, o, S, z, W_q=None, W_k=None, dt=None, A_log=None, b_q=N
     a.b_q, a.b_k = _ptr(b_q), _ptr(b_k)
     a.dt, a.A_log = _ptr(dt), _ptr(A_log)
     a.S, a.z = _ptr(S), _ptr(z)
+    a.flags = int(flags)
     if workspace is not None:
         a.workspace = _ptr(workspace)
         a.workspace_bytes = workspace.numel() * workspace.element_size()

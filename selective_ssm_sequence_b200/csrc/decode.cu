@@ -14,6 +14,8 @@
 // while the next tile's loads are already in flight.
 // One CTA walks all column tiles of its head, so z (shared by every column)
 // is read and rewritten by the same thread with no cross-CTA race.
+// The scan's variants are supported: phik times softplus(dt) for the
+// step-scaled input, and one decay per feature row with A_log [H, F].
 #include "hm_internal.h"
 
 namespace hm {
@@ -43,8 +45,8 @@ __global__ void __launch_bounds__(kThreads)
 decode_kernel(int H, int F, int dv, const TF *__restrict__ phq, const TF *__restrict__ phk,
               const TIO *__restrict__ v, const float *__restrict__ dt,
               const float *__restrict__ A_log, float *__restrict__ S, float *__restrict__ z,
-              TIO *__restrict__ o) {
-    __shared__ float sq[256], sk[256];
+              TIO *__restrict__ o, int dt_scaled, int per_feature) {
+    __shared__ float sq[256], sk[256], sa[256];
     __shared__ float snum[kRowGroups][kCols];
     __shared__ float sden[kThreads / 32];
 
@@ -55,7 +57,10 @@ decode_kernel(int H, int F, int dv, const TF *__restrict__ phq, const TF *__rest
     const int rg = tid / kColThreads;   // row group
     float4 *Sbh = reinterpret_cast<float4 *>(S + bh * (int64_t)F * dv);
 
-    const float a = dt ? expf(hm_log_decay(dt[bh], A_log[h])) : 1.f;
+    // variants: the step-scaled input multiplies phik by softplus(dt); the
+    // per-feature decay takes one rate per (head, feature) from A_log [H, F]
+    const float a = (dt && !per_feature) ? expf(hm_log_decay(dt[bh], A_log[h])) : 1.f;
+    const float delta = dt_scaled ? hm_step_size(dt[bh]) : 1.f;
 
     // first tile's state loads go out before anything else
     float4 s[kMaxRowsPerThread];
@@ -69,7 +74,8 @@ decode_kernel(int H, int F, int dv, const TF *__restrict__ phq, const TF *__rest
     }
     for (int f = tid; f < F; f += kThreads) {
         sq[f] = hm_ld(phq, bh * F + f);
-        sk[f] = hm_ld(phk, bh * F + f);
+        sk[f] = hm_ld(phk, bh * F + f) * delta;
+        sa[f] = per_feature ? expf(hm_log_decay(dt[bh], A_log[(int64_t)h * F + f])) : a;
     }
     __syncthreads();
 
@@ -77,7 +83,7 @@ decode_kernel(int H, int F, int dv, const TF *__restrict__ phq, const TF *__rest
     // den = phiq . z'
     float dpart = 0.f;
     for (int f = tid; f < F; f += kThreads) {
-        float zf = fmaf(a, z[bh * F + f], sk[f]);
+        float zf = fmaf(sa[f], z[bh * F + f], sk[f]);
         dpart = fmaf(sq[f], zf, dpart);
         z[bh * F + f] = zf;
     }
@@ -104,12 +110,12 @@ decode_kernel(int H, int F, int dv, const TF *__restrict__ phq, const TF *__rest
         for (int m = 0; m < kMaxRowsPerThread; ++m) {
             int f = rg + kRowGroups * m;
             if (f < F && cols_ok) {
-                const float kf = sk[f], qf = sq[f];
+                const float kf = sk[f], qf = sq[f], af = sa[f];
                 float4 t = s[m];
-                t.x = fmaf(a, t.x, kf * vv.x);
-                t.y = fmaf(a, t.y, kf * vv.y);
-                t.z = fmaf(a, t.z, kf * vv.z);
-                t.w = fmaf(a, t.w, kf * vv.w);
+                t.x = fmaf(af, t.x, kf * vv.x);
+                t.y = fmaf(af, t.y, kf * vv.y);
+                t.z = fmaf(af, t.z, kf * vv.z);
+                t.w = fmaf(af, t.w, kf * vv.w);
                 st_stream(Sbh + ((int64_t)f * dv + c0) / 4, t);
                 num.x = fmaf(qf, t.x, num.x);
                 num.y = fmaf(qf, t.y, num.y);
@@ -149,7 +155,8 @@ cudaError_t go(const DecodeCore &c, cudaStream_t s) {
     dim3 grid((unsigned)(c.B * c.H));
     decode_kernel<TF, TIO><<<grid, kThreads, 0, s>>>(c.H, c.F, c.dv, (const TF *)c.phq,
                                                      (const TF *)c.phk, (const TIO *)c.v, c.dt,
-                                                     c.A_log, c.S, c.z, (TIO *)c.o);
+                                                     c.A_log, c.S, c.z, (TIO *)c.o, c.dt_scaled ? 1 : 0,
+                                                     c.per_feature ? 1 : 0);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -123,6 +123,9 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
     if ((a->S_out == nullptr) != (a->z_out == nullptr))
         return fail(HM_ERR_INVALID_ARG, "scan: S_out and z_out must both be given or both NULL");
     if (a->dt && !a->A_log) return fail(HM_ERR_INVALID_ARG, "scan: dt given without A_log");
+    if (a->flags & ~(unsigned)(HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY))
+        return fail(HM_ERR_INVALID_ARG, "scan: unknown flag bits 0x%x", a->flags);
+    if (a->flags && !a->dt) return fail(HM_ERR_INVALID_ARG, "scan: the variant flags need dt");
     const int F = a->W_q ? 2 * a->p : a->d;
     if (a->W_q && (a->p < 1 || a->p > 256)) return fail(HM_ERR_UNSUPPORTED, "scan: need 1 <= p <= 256");
     if (F > 256) return fail(HM_ERR_UNSUPPORTED, "scan: feature dim F=%d > 256", F);
@@ -130,10 +133,12 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
     if (a->dv % 4 != 0) return fail(HM_ERR_UNSUPPORTED, "scan: dv must be a multiple of 4");
     if (a->B * a->H > 65535) return fail(HM_ERR_UNSUPPORTED, "scan: B*H > 65535");
     const int64_t rows = a->B * a->L * a->H;
-    if (rows > 0 && (!a->q || !a->k || !a->v || !a->o))
-        return fail(HM_ERR_INVALID_ARG, "scan: null q/k/v/o");
+    // o == NULL: a state-only call (the final state, and the log decay, are its results)
+    if (!a->o && !a->S_out) return fail(HM_ERR_INVALID_ARG, "scan: o may be NULL only when S_out is given");
+    if (rows > 0 && (!a->k || !a->v || (a->o && !a->q)))
+        return fail(HM_ERR_INVALID_ARG, "scan: null q/k/v");
     const void *ptrs[] = {a->q, a->k, a->v, a->W_q, a->W_k, a->b_q, a->b_k, a->dt, a->A_log,
-                          a->S0, a->z0, a->o, a->S_out, a->z_out};
+                          a->S0, a->z0, a->o, a->S_out, a->z_out, a->log_decay_out};
     for (const void *p : ptrs)
         if (!aligned16(p)) return fail(HM_ERR_INVALID_ARG, "scan: pointers must be 16-byte aligned");
     ScanPlan pl{};
@@ -141,6 +146,8 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
     ScanCore c{};
     c.B = a->B; c.L = a->L; c.H = a->H; c.F = F; c.dv = a->dv;
     c.feat_dtype = a->io_dtype; c.io_dtype = a->io_dtype;
+    c.dt_scaled = (a->flags & HM_FLAG_DT_SCALED_INPUT) != 0;
+    c.per_feature = (a->flags & HM_FLAG_PER_FEATURE_DECAY) != 0;
     pl.tc = scan_tc_supported(c);
     // Features computed here are kept in fp32 for the CUDA-core path: its state
     // update then adds exact products instead of bf16-rounded ones.  When
@@ -165,6 +172,9 @@ hm_status check_decode(const hm_decode_args *a, DecodePlan *plan) {
     if ((a->W_q == nullptr) != (a->W_k == nullptr))
         return fail(HM_ERR_INVALID_ARG, "decode: W_q and W_k must both be given or both NULL");
     if (a->dt && !a->A_log) return fail(HM_ERR_INVALID_ARG, "decode: dt given without A_log");
+    if (a->flags & ~(unsigned)(HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY))
+        return fail(HM_ERR_INVALID_ARG, "decode: unknown flag bits 0x%x", a->flags);
+    if (a->flags && !a->dt) return fail(HM_ERR_INVALID_ARG, "decode: the variant flags need dt");
     const int F = a->W_q ? 2 * a->p : a->d;
     if (a->W_q && (a->p < 1 || a->p > 256)) return fail(HM_ERR_UNSUPPORTED, "decode: need 1 <= p <= 256");
     if (F > 256) return fail(HM_ERR_UNSUPPORTED, "decode: feature dim F=%d > 256", F);
@@ -217,6 +227,8 @@ hm_status decode_enqueue(const hm_decode_args *a, const DecodePlan &pl, void *ph
     c.feat_dtype = ft; c.io_dtype = a->io_dtype;
     c.phq = phq; c.phk = phk; c.v = a->v; c.dt = a->dt; c.A_log = a->A_log;
     c.S = a->S; c.z = a->z; c.o = a->o;
+    c.dt_scaled = (a->flags & HM_FLAG_DT_SCALED_INPUT) != 0;
+    c.per_feature = (a->flags & HM_FLAG_PER_FEATURE_DECAY) != 0;
     e = launch_decode(c, s);
     return e == cudaSuccess ? HM_OK : cuda_fail(e, "decode launch");
 }
@@ -378,12 +390,25 @@ hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
     if (a->W_q && rows > 0) {
         void *wq = ws, *wk = ws + pl.phi_bytes;
         void *wkl = pl.lo_bytes ? ws + 2 * pl.phi_bytes : nullptr;
-        e = run_featmap_qk(a->q, a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->W_k, a->w_head_stride,
-                           a->b_q, a->b_k, wq, wk, pl.feat, s, wkl);
+        if (a->o) {
+            e = run_featmap_qk(a->q, a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_q, a->W_k,
+                               a->w_head_stride, a->b_q, a->b_k, wq, wk, pl.feat, s, wkl);
+            phq = wq;
+        } else {
+            // state only: phi(q) is not needed
+            e = run_featmap(a->k, a->io_dtype, rows, a->H, a->d, a->p, a->W_k, a->w_head_stride, a->b_k, wk,
+                            pl.feat, s, wkl);
+            phq = nullptr;
+        }
         if (e != cudaSuccess) return cuda_fail(e, "scan: feature maps");
-        phq = wq;
         phk = wk;
         phk_lo = wkl;
+    }
+    if (!a->o) phq = nullptr;
+    if (a->log_decay_out) {
+        e = launch_logdecay_sum(a->B, a->L, a->H, pl.F, (a->flags & HM_FLAG_PER_FEATURE_DECAY) != 0, a->dt,
+                                a->A_log, a->log_decay_out, s);
+        if (e != cudaSuccess) return cuda_fail(e, "scan: log decay sum");
     }
     ScanCore c{};
     c.B = a->B; c.L = a->L; c.H = a->H; c.F = pl.F; c.dv = a->dv;
@@ -392,6 +417,8 @@ hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
     c.dt = a->dt; c.A_log = a->A_log; c.S0 = a->S0; c.z0 = a->z0;
     c.o = a->o; c.S_out = a->S_out; c.z_out = a->z_out;
     c.o_f32 = o_f32 && pl.tc;
+    c.dt_scaled = (a->flags & HM_FLAG_DT_SCALED_INPUT) != 0;
+    c.per_feature = (a->flags & HM_FLAG_PER_FEATURE_DECAY) != 0;
     if (pl.tc)
         e = launch_scan_tc(c, ws + 2 * pl.phi_bytes + pl.lo_bytes, pl.tc_bytes,
                            DevErr{device_error_word()}, s);

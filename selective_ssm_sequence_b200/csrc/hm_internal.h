@@ -109,6 +109,8 @@ struct ScanCore {
     void *o;
     bool o_f32;           // tensor-core path: write o as fp32 instead of io_dtype
     float *S_out, *z_out;
+    bool dt_scaled;       // HM_FLAG_DT_SCALED_INPUT: input term times softplus(dt)
+    bool per_feature;     // HM_FLAG_PER_FEATURE_DECAY: A_log is [H, F]
 };
 cudaError_t launch_scan_simt(const ScanCore &c, cudaStream_t s);
 
@@ -117,6 +119,11 @@ bool scan_tc_supported(const ScanCore &c);
 size_t scan_tc_workspace(const ScanCore &c);
 cudaError_t launch_scan_tc(const ScanCore &c, void *ws, size_t ws_bytes, DevErr err,
                            cudaStream_t s);
+
+// lambda = sum over the L tokens of log a_t per (b, h) ([B, H]) or per
+// (b, h, f) with the per-feature decay ([B, H, F]); zeros when dt is NULL.
+cudaError_t launch_logdecay_sum(int64_t B, int64_t L, int H, int F, bool per_feature, const float *dt,
+                                const float *A_log, float *out, cudaStream_t s);
 
 // Decode step over precomputed features.
 struct DecodeCore {
@@ -127,8 +134,13 @@ struct DecodeCore {
     const float *dt, *A_log;
     float *S, *z;
     void *o;
+    bool dt_scaled;       // as in ScanCore
+    bool per_feature;
 };
 cudaError_t launch_decode(const DecodeCore &c, cudaStream_t s);
+
+// softplus(dt): the step size of the step-scaled input variant.
+__device__ __forceinline__ float hm_step_size(float dt) { return hm_softplus(dt); }
 
 // Checked shape of a decode call: F, and the size of each per-token feature
 // plane (B * H * F values when W_q != NULL, else 0) and of the workspace.

@@ -12,6 +12,12 @@
 // per 16 tokens.  This is the fp32 path (a 1e-4 tolerance rules out bf16 or
 // TF32 tensor-core operands) and the path for shapes without a tensor-core
 // kernel; it performs the recurrence in exactly the order of its definition.
+//
+// Variants (the scan's flags): with the step-scaled input the staged phik of
+// token t is multiplied by Delta_t = softplus(dt_t) (Mamba's B-bar = Delta B);
+// with the per-feature decay a_t is staged per (token, feature) from A_log
+// [H, F] and scales row f of S and entry f of z (gated linear attention's
+// diag(alpha_t)).
 #include "hm_internal.h"
 
 namespace hm {
@@ -28,7 +34,7 @@ scan_simt_kernel(int64_t L, int H, int F, int dv, const TF *__restrict__ phq,
                  const TF *__restrict__ phk, const TIO *__restrict__ v,
                  const float *__restrict__ dt, const float *__restrict__ A_log,
                  const float *__restrict__ S0, const float *__restrict__ z0, TIO *__restrict__ o,
-                 float *__restrict__ S_out, float *__restrict__ z_out) {
+                 float *__restrict__ S_out, float *__restrict__ z_out, int dt_scaled, int per_feature) {
     extern __shared__ float smem[];
     float *sq = smem;                      // [kTB][F]
     float *sk = sq + kTB * F;              // [kTB][F]
@@ -36,6 +42,8 @@ scan_simt_kernel(int64_t L, int H, int F, int dv, const TF *__restrict__ phq,
     float *sa = sv + kTB * 32;             // [kTB]
     float *red = sa + kTB;                 // [kTB][kW][32]
     float *rden = red + kTB * kW * 32;     // [kTB][kW]
+    float *saf = rden + kTB * kW;          // [kTB][F] per-feature decay (per_feature only)
+    float *sdl = saf + (per_feature ? kTB * F : 0);   // [kTB] step sizes
 
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t bh = blockIdx.y;
@@ -43,7 +51,7 @@ scan_simt_kernel(int64_t L, int H, int F, int dv, const TF *__restrict__ phq,
     const int h = (int)(bh % H);
     const int col = blockIdx.x * 32 + lane;
     const bool col_ok = col < dv;
-    const float a_rate = (dt != nullptr) ? A_log[h] : 0.f;
+    const float a_rate = (dt != nullptr && !per_feature) ? A_log[h] : 0.f;
 
     float S[kMaxRows], z[kMaxRows];
 #pragma unroll
@@ -62,7 +70,7 @@ scan_simt_kernel(int64_t L, int H, int F, int dv, const TF *__restrict__ phq,
         for (int i = threadIdx.x; i < nt * F; i += blockDim.x) {
             int t = i / F, f = i % F;
             int64_t row = (b * L + t0 + t) * H + h;
-            sq[t * F + f] = hm_ld(phq, row * F + f);
+            sq[t * F + f] = phq ? hm_ld(phq, row * F + f) : 0.f;   // no phq: state-only call
             sk[t * F + f] = hm_ld(phk, row * F + f);
         }
         for (int i = threadIdx.x; i < nt * 32; i += blockDim.x) {
@@ -72,17 +80,29 @@ scan_simt_kernel(int64_t L, int H, int F, int dv, const TF *__restrict__ phq,
         }
         if (threadIdx.x < nt) {
             int64_t row = (b * L + t0 + threadIdx.x) * H + h;
-            sa[threadIdx.x] = dt ? expf(hm_log_decay(dt[row], a_rate)) : 1.f;
+            sa[threadIdx.x] = (dt && !per_feature) ? expf(hm_log_decay(dt[row], a_rate)) : 1.f;
+            sdl[threadIdx.x] = dt_scaled ? hm_step_size(dt[row]) : 1.f;
         }
+        if (per_feature)
+            for (int i = threadIdx.x; i < nt * F; i += blockDim.x) {
+                int t = i / F, f = i % F;
+                int64_t row = (b * L + t0 + t) * H + h;
+                saf[i] = expf(hm_log_decay(dt[row], A_log[(int64_t)h * F + f]));
+            }
         __syncthreads();
+        if (dt_scaled) {
+            for (int i = threadIdx.x; i < nt * F; i += blockDim.x) sk[i] *= sdl[i / F];
+            __syncthreads();
+        }
         for (int t = 0; t < nt; ++t) {
-            const float a = sa[t];
+            const float at = sa[t];
             const float vv = sv[t * 32 + lane];
             float num = 0.f, den = 0.f;
 #pragma unroll
             for (int m = 0; m < kMaxRows; ++m) {
                 int f = w + kW * m;
                 if (f < F) {
+                    const float a = per_feature ? saf[t * F + f] : at;
                     float kf = sk[t * F + f], qf = sq[t * F + f];
                     S[m] = fmaf(a, S[m], kf * vv);
                     num = fmaf(qf, S[m], num);
@@ -103,7 +123,7 @@ scan_simt_kernel(int64_t L, int H, int F, int dv, const TF *__restrict__ phq,
                 den += rden[t * kW + ww];
             }
             int cc = blockIdx.x * 32 + c;
-            if (cc < dv) {
+            if (cc < dv && o) {
                 int64_t row = (b * L + t0 + t) * H + h;
                 hm_st(o, row * dv + cc, num / den);
             }
@@ -124,7 +144,8 @@ scan_simt_kernel(int64_t L, int H, int F, int dv, const TF *__restrict__ phq,
 template <typename TF, typename TIO>
 cudaError_t go(const ScanCore &c, cudaStream_t s) {
     dim3 grid((unsigned)((c.dv + 31) / 32), (unsigned)(c.B * c.H));
-    size_t smem = sizeof(float) * (size_t)(2 * kTB * c.F + kTB * 32 + kTB + kTB * kW * 32 + kTB * kW);
+    size_t smem = sizeof(float) * (size_t)(2 * kTB * c.F + kTB * 32 + kTB + kTB * kW * 32 + kTB * kW +
+                                           (c.per_feature ? kTB * c.F : 0) + kTB);
     auto kern = scan_simt_kernel<TF, TIO>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -132,7 +153,7 @@ cudaError_t go(const ScanCore &c, cudaStream_t s) {
     }
     kern<<<grid, 32 * kW, smem, s>>>(c.L, c.H, c.F, c.dv, (const TF *)c.phq, (const TF *)c.phk,
                                      (const TIO *)c.v, c.dt, c.A_log, c.S0, c.z0, (TIO *)c.o,
-                                     c.S_out, c.z_out);
+                                     c.S_out, c.z_out, c.dt_scaled ? 1 : 0, c.per_feature ? 1 : 0);
     count_launches(1);
     return cudaGetLastError();
 }

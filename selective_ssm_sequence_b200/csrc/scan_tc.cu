@@ -24,6 +24,12 @@
 // their M dimension, and the readout takes its A operand (a bf16 copy of S^T)
 // straight from TMEM.
 //
+// Step-scaled input (HM_FLAG_DT_SCALED_INPUT, Mamba's B-bar = Delta B): every
+// factor that weights key j -- w_j, the decay of column j of Pt -- also
+// carries Delta_j = softplus(dt_j); the decay warp folds log2(Delta_j) into the
+// key-side prefix sums, so the chunk loop is unchanged.  (The per-feature
+// decay variant has no tensor-core kernel: it runs on the CUDA-core scan.)
+//
 // Long sequences are cut into segments that run in parallel.  Three kernels:
 //   A  scan_state_kernel  local end state of each part (a run of chunks) from a
 //                         zero start, weights relative to the part end; with
@@ -126,7 +132,7 @@ constexpr int kAThreads = 64 + 32 * kABuild + 32;
 __global__ void __launch_bounds__(kAThreads, 1)
 scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constant__ CUtensorMap tmkl,
                   const __grid_constant__ CUtensorMap tmv, Geo g, const float *__restrict__ dt,
-                  const float *__restrict__ A_log, int split, int add_lo, float *__restrict__ S_part,
+                  const float *__restrict__ A_log, int split, int add_lo, int dt_scaled, float *__restrict__ S_part,
                   float *__restrict__ z_part, float *__restrict__ lsum_part, DevErr err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
@@ -250,6 +256,9 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
         bool okw = true;
         for (int it = 0; it < n; ++it) {
             const float l0 = hm_log_decay(da[0], alog), l1 = hm_log_decay(db[0], alog);
+            // step-scaled input: the token's weight also carries softplus(dt)
+            const float d0 = dt_scaled ? hm_step_size(da[0]) : 1.f;
+            const float d1 = dt_scaled ? hm_step_size(db[0]) : 1.f;
 #pragma unroll
             for (int i = 0; i < 3; ++i) {
                 da[i] = da[i + 1];
@@ -272,7 +281,8 @@ scan_state_kernel(const __grid_constant__ CUtensorMap tmkh, const __grid_constan
             if (it >= nst) okw = mbar_wait(&X->built[s], ph ^ 1, abort_flag, err, KID_SCAN_TC_STATE, 6);
             okw = __all_sync(0xffffffffu, okw);
             if (!okw) break;
-            *reinterpret_cast<float2 *>(&X->w[s][2 * lane]) = make_float2(fexp(suf + ex0), fexp(suf + ex1));
+            *reinterpret_cast<float2 *>(&X->w[s][2 * lane]) =
+                make_float2(fexp(suf + ex0) * d0, fexp(suf + ex1) * d1);
             __syncwarp();
             if (lane == 0) mbar_arrive(&X->wfull[s]);
             suf += tot;
@@ -482,6 +492,7 @@ constexpr int kHelpers = 160;    // threads of the five helper warps
 
 struct CAux {
     float cum[2][kC];
+    float ck[2][kC];     // key-side cums: cum_j - log2(Delta_j) (= cum_j without the step-scaled input)
     float bq[2][32];     // e^(cum_(j|7) - cum_j), j < 32: column factors of the below-diagonal quadrant
     float qs[2][kC];
     float w[2][kC];
@@ -524,6 +535,7 @@ struct OutArgs {
     const float *dt, *A_log;
     void *o;
     int o_f32;                       // o stored as fp32 (else bf16)
+    int dt_scaled;                   // step-scaled input: key j weighted by softplus(dt_j)
     const float *S0, *z0;            // segment 0 start state (caller layout) or null
     const float *S_start, *z_start;  // segments >= 1: [BH][G][F*dv], [BH][G][F]
 };
@@ -827,7 +839,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 } else if (okw) {
                     const float ci = X->cum[s][i];
                     const float2 ci2 = make_float2(ci, ci);
-                    const float *__restrict__ cj = X->cum[s] + jc;
+                    const float *__restrict__ cj = X->ck[s] + jc;
                     uint8_t *__restrict__ prow = gP(s);
                     float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll 1
@@ -992,6 +1004,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         for (int c = 0; c < nch; ++c) {
             const int sc = c & 1;
             const float l0 = hm_log_decay(da[0], alog) * kLog2e, l1 = hm_log_decay(db[0], alog) * kLog2e;
+            // step-scaled input: log2 of softplus(dt) of the two tokens, added
+            // to every factor that weights a key (-inf past the sequence end)
+            const float g0 = a.dt_scaled ? lg2_approx(hm_step_size(da[0])) : 0.f;
+            const float g1 = a.dt_scaled ? lg2_approx(hm_step_size(db[0])) : 0.f;
             da[0] = da[1];
             db[0] = db[1];
             da[1] = c + 2 < nch ? token_dt(a, b, h, (int64_t)(c_begin + c + 2) * kC, 2 * lane) : -INFINITY;
@@ -1012,11 +1028,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (!__all_sync(0xffffffffu, okw)) break;
             if (lane < 16)
                 *reinterpret_cast<float2 *>(&X->bq[sc][2 * lane]) =
-                    make_float2(ex2_approx(xe - x0), ex2_approx(xe - x));
+                    make_float2(ex2_approx(xe - x0 + g0), ex2_approx(xe - x + g1));
             *reinterpret_cast<float2 *>(&X->cum[sc][2 * lane]) = make_float2(x0, x);
+            *reinterpret_cast<float2 *>(&X->ck[sc][2 * lane]) = make_float2(x0 - g0, x - g1);
             *reinterpret_cast<float2 *>(&X->qs[sc][2 * lane]) = make_float2(ex2_approx(x0), ex2_approx(x));
             *reinterpret_cast<float2 *>(&X->w[sc][2 * lane]) =
-                make_float2(ex2_approx(total - x0), ex2_approx(total - x));
+                make_float2(ex2_approx(total - x0 + g0), ex2_approx(total - x + g1));
             if (lane == 0) X->gam[sc] = ex2_approx(total);
             __syncwarp();
             if (lane == 0) mbar_arrive(&X->dec_full[sc]);
@@ -1277,7 +1294,7 @@ bool tmap_tokens(CUtensorMap *m, const void *base, int64_t B, int64_t L, int H, 
 }  // namespace
 
 bool scan_tc_supported(const ScanCore &c) {
-    return c.io_dtype == HM_BF16 && c.feat_dtype == HM_BF16 && c.F == kF && c.dv % kN == 0 &&
+    return !c.per_feature && c.io_dtype == HM_BF16 && c.feat_dtype == HM_BF16 && c.F == kF && c.dv % kN == 0 &&
            c.dv == 2 * kN && c.L < (int64_t)1 << 30 && c.B < 65536 && c.H < 65536;
 }
 
@@ -1308,10 +1325,12 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
         }
         return cudaSuccess;
     }
+    // a state-only call (o == NULL) runs phases A and B and no output kernel
+    const bool outputs = c.o != nullptr;
     CUtensorMap tq, tk, tkl, tv;
-    if (!tmap_tokens(&tq, c.phq, c.B, c.L, c.H, kF, 64) || !tmap_tokens(&tk, c.phk, c.B, c.L, c.H, kF, 64) ||
-        !tmap_tokens(&tv, c.v, c.B, c.L, c.H, c.dv, 64))
+    if (!tmap_tokens(&tk, c.phk, c.B, c.L, c.H, kF, 64) || !tmap_tokens(&tv, c.v, c.B, c.L, c.H, c.dv, 64))
         return cudaErrorInvalidValue;
+    if (outputs && !tmap_tokens(&tq, c.phq, c.B, c.L, c.H, kF, 64)) return cudaErrorInvalidValue;
     // with a returned state, the weighted features of the state phase are split
     // into bf16 hi + lo (and phik's own rounding remainder is added when given)
     const bool split = want_state;
@@ -1323,7 +1342,8 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
         if (e != cudaSuccess) return e;
         const unsigned grid = (unsigned)(2 * g.NPc * BH);
         scan_state_kernel<<<grid, kAThreads, kASmem, s>>>(tk, tkl, tv, g, c.dt, c.A_log, split ? 1 : 0,
-                                                    add_lo ? 1 : 0, S_part, z_part, lsum, err);
+                                                    add_lo ? 1 : 0, c.dt_scaled ? 1 : 0, S_part, z_part,
+                                                    lsum, err);
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int64_t ncol = (int64_t)(nS + kF) / 4;
@@ -1340,12 +1360,14 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if (!outputs) return cudaSuccess;
     OutArgs oa{};
     oa.g = g;
     oa.dt = c.dt;
     oa.A_log = c.A_log;
     oa.o = c.o;
     oa.o_f32 = c.o_f32 ? 1 : 0;
+    oa.dt_scaled = c.dt_scaled ? 1 : 0;
     oa.S0 = c.S0;
     oa.z0 = c.z0;
     oa.S_start = S_start;

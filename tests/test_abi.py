@@ -121,3 +121,22 @@ def test_validation_rejects_bad_calls_before_launch(hm):
     m.B, m.L, m.d_model, m.H, m.E, m.p, m.conv_k = 1, 16, 2048, 8, 2050, 128, 4
     assert hm.lib.hm_mixer_fwd(ctypes.byref(m), None, 0, None) in (hm.HM_ERR_INVALID_ARG,
                                                                    hm.HM_ERR_UNSUPPORTED)
+
+
+def test_variant_flags_are_validated_before_launch(hm):
+    def call(a):
+        return hm.lib.hm_scan_chunked_fwd(ctypes.byref(a), None)
+    assert call(_args(hm, flags=4)) == hm.HM_ERR_INVALID_ARG           # unknown bit
+    assert b"flag" in hm.lib.hm_last_error_detail()
+    assert call(_args(hm, flags=hm.HM_FLAG_DT_SCALED_INPUT, dt=None)) == hm.HM_ERR_INVALID_ARG
+    assert call(_args(hm, flags=hm.HM_FLAG_PER_FEATURE_DECAY, dt=None)) == hm.HM_ERR_INVALID_ARG
+    # valid flags size a workspace like the plain call (CUDA-core path for the per-feature decay)
+    assert hm.hm_scan_workspace_size(_args(hm, flags=hm.HM_FLAG_DT_SCALED_INPUT)) > 0
+    assert hm.hm_scan_workspace_size(_args(hm, flags=hm.HM_FLAG_PER_FEATURE_DECAY)) > 0
+    d = hm.DecodeArgs()
+    d.B, d.H, d.d, d.p, d.dv = 2, 8, 256, 128, 256
+    d.q = d.k = d.v = d.o = d.S = d.z = 1 << 20
+    d.flags = 8
+    assert hm.lib.hm_step_decode(ctypes.byref(d), None) == hm.HM_ERR_INVALID_ARG
+    d.flags = hm.HM_FLAG_DT_SCALED_INPUT                                    # needs dt
+    assert hm.lib.hm_step_decode(ctypes.byref(d), None) == hm.HM_ERR_INVALID_ARG
