@@ -82,6 +82,8 @@ def _load():
         lib.hmo_log_decay_f.argtypes = [P, I64, I, I, P, P]
         lib.hmo_step_size.restype = None
         lib.hmo_step_size.argtypes = [P, I64, P]
+        lib.hmo_rope.restype = None
+        lib.hmo_rope.argtypes = [P, I64, I, P, ctypes.c_double, P]
         lib.hmo_causal_conv.restype = None
         lib.hmo_causal_conv.argtypes = [I64, I64, I, I, P, P, P, P]
         _lib = lib
@@ -165,6 +167,25 @@ def scan_recurrent(phq, phk, v, log_a=None, S0=None, z0=None, return_state=False
     if return_state:
         return o, S_out, z_out
     return o
+
+
+def rope(x, pos, base=10000.0):
+    """Rotary embedding of feature vectors ([HM] sec. 5.2, RoPE on phi(Q),
+    phi(K)); "rotate half" pairing (i, i + F/2), angle pos * base^(-2i/F).
+    x: [..., F]; pos: broadcastable to x.shape[:-1] (absolute positions)."""
+    x = _f64(x)
+    F = x.shape[-1]
+    assert F % 2 == 0
+    p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, dtype=np.float64), x.shape[:-1]))
+    out = np.empty_like(x)
+    _load().hmo_rope(_ptr(x), x.size // F, F, _ptr(p), float(base), _ptr(out))
+    return out
+
+
+def token_positions(B, L, H, pos0=0):
+    """Absolute position of every (b, t, h) row of a [B, L, H, *] tensor: pos0 + t."""
+    t = np.arange(L, dtype=np.float64) + float(pos0)
+    return np.broadcast_to(t[None, :, None], (B, L, H))
 
 
 def log_decay_per_feature(dt, A_log_f):
@@ -280,14 +301,16 @@ def silu(x):
 # --------------------------------------------------------------------------
 
 def scan_fwd(q, k, v, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=None,
-             S0=None, z0=None, w_head_stride=0, return_state=False, dt_scaled_input=False):
+             S0=None, z0=None, w_head_stride=0, return_state=False, dt_scaled_input=False,
+             rope_base=None, pos0=0):
     """Feature map on q and k, then the decayed normalised recurrence.
 
     q, k: [B, L, H, d]; v: [B, L, H, dv]; W_q, W_k: [p, d] (or per-head); if
     W_q is None, q and k are taken as feature vectors already (F = d).
     dt: [B, L, H] or None (a = 1); A_log: [H], or [H, F] for a decay per
     feature.  dt_scaled_input: the input term is multiplied by Delta =
-    softplus(dt) (Mamba's discretised input)."""
+    softplus(dt) (Mamba's discretised input).  rope_base: rotary embedding of
+    phi(q) and phi(k) (rope) at positions pos0 + t; None = off."""
     q, k = _f64(q), _f64(k)
     B, L, H, d = q.shape
     if W_q is None:
@@ -297,6 +320,9 @@ def scan_fwd(q, k, v, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=Non
         bstride = W_q.shape[-2] if w_head_stride else 0
         phq = featmap(q, W_q, b_q, H=H, w_head_stride=w_head_stride, b_head_stride=bstride)
         phk = featmap(k, W_k, b_k, H=H, w_head_stride=w_head_stride, b_head_stride=bstride)
+    if rope_base is not None:
+        pos = token_positions(B, L, H, pos0)
+        phq, phk = rope(phq, pos, rope_base), rope(phk, pos, rope_base)
     per_feature = A_log is not None and np.ndim(A_log) == 2
     if not per_feature and not dt_scaled_input:
         la = None if dt is None else log_decay(dt, A_log)

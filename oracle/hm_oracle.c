@@ -119,6 +119,29 @@ HMO_EXPORT void hmo_featmap(const double *x, int64_t rows, int H, int d, int p,
     }
 }
 
+/* Rotary position embedding on feature vectors ([HM] sec. 5.2: RoPE is
+ * applied to phi(Q) and phi(K) in the mixer).  Reading: the "rotate half"
+ * pairing of the GPT-NeoX / Pythia models the pages distil from -- feature i
+ * pairs with feature i + F/2 -- with angle pos * base^(-2i/F), i < F/2:
+ *   x_i'       = x_i cos(angle) - x_{i+F/2} sin(angle)
+ *   x_{i+F/2}' = x_i sin(angle) + x_{i+F/2} cos(angle)
+ * x, y: [rows, F] (F even; y may alias x); pos: [rows] absolute positions. */
+HMO_EXPORT void hmo_rope(const double *x, int64_t rows, int F, const double *pos,
+                         double base, double *y) {
+    int half = F / 2;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int i = 0; i < half; ++i) {
+            double theta = pow(base, -2.0 * (double)i / (double)F);
+            double ang = pos[r] * theta;
+            double c = cos(ang), s = sin(ang);
+            double a = x[r * F + i], b = x[r * F + i + half];
+            y[r * F + i] = a * c - b * s;
+            y[r * F + i + half] = a * s + b * c;
+        }
+    }
+}
+
 /* Decayed normalised recurrence (spec definition; [HM] sec. 2.3 and
  * 5.2 doubled state; [LA] sec. 3 recurrent form, sec. 4.3 decayed form):
  *   S_t = a_t S_{t-1} + phik_t v_t^T

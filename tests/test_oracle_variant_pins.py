@@ -8,9 +8,14 @@
   attention S_i = diag(alpha_i) S_{i-1} + k_i v_i^T):
       S_t[f, :] = a_{t,f} S_{t-1}[f, :] + phik_t[f] v_t^T
 
-Each is checked against an independent O(L^2) masked form, closed forms on
-one and two tokens, and exact invariances that tie it back to the pinned
-plain recurrence."""
+* the rotary embedding on phi(Q), phi(K) (HedgeMamba explainer sec. 5.2),
+  "rotate half" pairing (i, i + F/2), angle pos * base^(-2i/F).
+
+Each recurrence variant is checked against an independent O(L^2) masked
+form, closed forms on one and two tokens, and exact invariances that tie it
+back to the pinned plain recurrence; the rotation against plane-rotation
+closed forms, composition, relative-position invariance, and a split of the
+sequence with carried state and a position offset."""
 import math
 
 import numpy as np
@@ -140,3 +145,55 @@ def test_scan_fwd_routes_the_variants(oracle_mod):
                                         log_a_f=oracle_mod.log_decay_per_feature(dt, A),
                                         in_scale=oracle_mod.step_size(dt))
     np.testing.assert_array_equal(o, ref)
+
+
+# ---------------------------------------------------------------- rotary embedding on the features
+
+def test_rope_position_zero_is_identity_and_pairs_keep_their_norm(oracle_mod):
+    x = rng.normal(size=(5, 12))
+    np.testing.assert_array_equal(oracle_mod.rope(x, 0.0), x)
+    y = oracle_mod.rope(x, rng.uniform(0, 500, size=5))
+    np.testing.assert_allclose(x[:, :6] ** 2 + x[:, 6:] ** 2, y[:, :6] ** 2 + y[:, 6:] ** 2, rtol=1e-12)
+
+
+def test_rope_closed_forms(oracle_mod):
+    # F = 2: a plane rotation by the position itself (theta_0 = base^0 = 1)
+    x = np.array([[0.3, -1.2]])
+    for t in (0.5, 3.0, 17.0):
+        c, s = math.cos(t), math.sin(t)
+        np.testing.assert_allclose(oracle_mod.rope(x, t), [[0.3 * c + 1.2 * s, 0.3 * s - 1.2 * c]], rtol=1e-14)
+    # F = 4, base 100: pair (0, 2) at angle t, pair (1, 3) at angle t * 100^(-1/2) = t / 10
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    t = 2.0
+    y = oracle_mod.rope(x, t, base=100.0)
+    a0, a1 = t, t / 10
+    ref = [1 * math.cos(a0) - 3 * math.sin(a0), 2 * math.cos(a1) - 4 * math.sin(a1),
+           1 * math.sin(a0) + 3 * math.cos(a0), 2 * math.sin(a1) + 4 * math.cos(a1)]
+    np.testing.assert_allclose(y[0], ref, rtol=1e-14)
+
+
+def test_rope_composes_and_depends_on_relative_position(oracle_mod):
+    x, y = rng.normal(size=(4, 16)), rng.normal(size=(4, 16))
+    t, s, d = 7.0, 3.0, 41.0
+    np.testing.assert_allclose(oracle_mod.rope(oracle_mod.rope(x, t), s), oracle_mod.rope(x, t + s),
+                               rtol=1e-11, atol=1e-12)
+    dot1 = np.sum(oracle_mod.rope(x, t) * oracle_mod.rope(y, s), axis=-1)
+    dot2 = np.sum(oracle_mod.rope(x, t + d) * oracle_mod.rope(y, s + d), axis=-1)
+    np.testing.assert_allclose(dot1, dot2, rtol=1e-11, atol=1e-12)
+
+
+def test_rope_scan_split_with_carried_state_and_position_offset(oracle_mod):
+    # running [0, L1) then [L1, L) from the carried state at positions L1.. equals one pass
+    B, L, H, d, p, dv, L1 = 2, 40, 2, 8, 4, 3, 17
+    q, k = rng.normal(size=(B, L, H, d)), rng.normal(size=(B, L, H, d))
+    v = rng.normal(size=(B, L, H, dv))
+    Wq, Wk = rng.normal(size=(p, d)) / 4, rng.normal(size=(p, d)) / 4
+    dt = rng.normal(size=(B, L, H)) + 2.0       # strong decay keeps the denominators positive
+    A = np.array([0.5, 1.0])
+    kw = dict(W_q=Wq, W_k=Wk, A_log=A, rope_base=10000.0)
+    o = oracle_mod.scan_fwd(q, k, v, dt=dt, **kw)
+    o1, S1, z1 = oracle_mod.scan_fwd(q[:, :L1], k[:, :L1], v[:, :L1], dt=dt[:, :L1], return_state=True, **kw)
+    o2 = oracle_mod.scan_fwd(q[:, L1:], k[:, L1:], v[:, L1:], dt=dt[:, L1:], S0=S1, z0=z1, pos0=L1, **kw)
+    np.testing.assert_allclose(np.concatenate([o1, o2], axis=1), o, rtol=1e-11, atol=1e-12)
+    # and the rotation is really applied: without it the outputs differ
+    assert not np.allclose(oracle_mod.scan_fwd(q, k, v, dt=dt, W_q=Wq, W_k=Wk, A_log=A), o)
