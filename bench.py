@@ -703,6 +703,88 @@ def bench_mixer(cfg, args, rank, world, torch):
     }
 
 
+# ---------------------------------------------------------------- backward workload
+
+def backward_flops_per_token_head(F: int, d: int, p: int, dv: int) -> int:
+    """Algorithmic FLOPs of the scan's backward per (batch, token, head): the
+    forward state recomputed (2 F dv), dphiq = S dn (2 F dv), the adjoint
+    update (2 F dv), dphik = G v (2 F dv) and dv = G^T phik (2 F dv); the
+    feature maps' dx = du W and dW += du x^T for q and k (4 x 2 p d)."""
+    return 10 * F * dv + 8 * p * d
+
+
+def bench_backward(cfg, args, rank, world, torch):
+    """hm_scan_bwd on the Pythia-shaped prefill (B4 H8 L2048): gradients of
+    sum(dout * o) for q, k, v, W_q, W_k, dt and A_log, one call per step,
+    replayed from a CUDA graph."""
+    import selective_ssm_sequence_b200 as hm
+    peaks, peak_kind = load_peaks()
+    inp = wl.scan_inputs(cfg, seed=rank_seed(cfg.seed, rank))
+    B, L, H, d, p, dv = cfg.B, cfg.L, cfg.H, cfg.d, cfg.p, cfg.dv
+    F = 2 * p
+    q, k, v = (to_dev(inp[n], "bf16", torch) for n in ("q", "k", "v"))
+    Wq, Wk = to_dev(inp["W_q"], "bf16", torch), to_dev(inp["W_k"], "bf16", torch)
+    dtt, A_log = to_dev(inp["dt"], "f32", torch), to_dev(inp["A_log"], "f32", torch)
+    dout = to_dev(wl.normal(cfg.seed, "dout", (B, L, H, dv)), "bf16", torch)
+    f32 = lambda *shape: torch.empty(shape, device="cuda")
+    a = hm.scan_bwd_args(q, k, v, dout, f32(B, L, H, d), f32(B, L, H, d), f32(B, L, H, dv), W_q=Wq, W_k=Wk,
+                         grad_W_q=f32(p, d), grad_W_k=f32(p, d), dt=dtt, A_log=A_log, grad_dt=f32(B, L, H),
+                         grad_A_log=f32(H))
+    ws = hm.alloc_workspace(hm.hm_scan_bwd_workspace_size(a))
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    stream = torch.cuda.current_stream()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        hm.hm_scan_bwd(a)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    n0 = hm.hm_launch_count()
+    with torch.cuda.graph(g, stream=cap):
+        hm.hm_scan_bwd(a)
+    per_step = hm.hm_launch_count() - n0
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    evs = []
+    sampler.mark_start()
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        evs.append((e0, e1))
+    sampler.in_flight()
+    torch.cuda.synchronize()
+    sampler.mark_stop()
+    sampler.stop()
+    assert hm.hm_get_device_error() == hm.HM_OK
+    ms = max_over_ranks(sum(x.elapsed_time(y) for x, y in evs) / args.steps, world, torch)
+    fl = backward_flops_per_token_head(F, d, p, dv) * B * L * H
+    # CUDA-core fp32 peak from the unit counts: 148 SMs x 128 FMA lanes x 2 flops x the SM clock
+    clk = sampler.summary().get("sm_max_mhz") or 1965.0
+    alu_peak = 148 * 128 * 2 * clk * 1e6 / 1e12
+    tfs = fl / (ms * 1e-3) / 1e12
+    return {
+        "metric": "backward tokens/sec (gradients of the prefill: q, k, v, W_q, W_k, dt, A_log)",
+        "value": B * L * world / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in, fp32 math", "data": "synthetic",
+        "config": {"workload": "backward_" + cfg.name, "B": B, "L": L, "H": H, "F": F, "dv": dv,
+                   "l2": "512 MiB buffer written between timed steps"},
+        "roofline": {"bound": "alu", "achieved": tfs, "peak": alu_peak, "unit": "TFLOP/s", "frac": tfs / alu_peak,
+                     "flops_per_token_head": backward_flops_per_token_head(F, d, p, dv),
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x max SM clock",
+                     "kernel": "whole backward call"},
+        "gpu_launches": per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -750,10 +832,10 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "long", "decode", "mixer"], default="long",
+    ap.add_argument("--workload", choices=["prefill", "long", "decode", "mixer", "backward"], default="long",
                     help="long: B1 H8 L32768 prefill (default, the largest single-GPU scan "
                          "workload); prefill: B4 H8 L2048; decode: 256 x 8 heads, 512 steps; "
-                         "mixer: B8 L4096 D2048")
+                         "mixer: B8 L4096 D2048; backward: hm_scan_bwd on B4 H8 L2048")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (decode: sequences, mixer: B) for small "
                          "profiling captures; the reported config says so")
@@ -779,6 +861,8 @@ def main():
         res = bench_decode(wl.DECODE, args, rank, world, torch)
     elif args.workload == "mixer":
         res = bench_mixer(wl.MIXER, args, rank, world, torch)
+    elif args.workload == "backward":
+        res = bench_backward(wl.PREFILL_PYTHIA, args, rank, world, torch)
     else:
         cfg = {"prefill": wl.PREFILL_PYTHIA, "long": wl.PREFILL_LONG}[args.workload]
         res = bench_prefill(cfg, args, rank, world, torch)

@@ -94,10 +94,17 @@ typedef enum { HM_F32 = 0, HM_BF16 = 1 } hm_dtype;
  *     f of S and entry f of z (gated linear attention's diag(alpha) S,
  *     linear-attention tutorial sec. 4.4; Mamba-1's A per state dimension).
  *     Requires dt.  Runs on the CUDA-core scan (no tensor-core kernel).
+ * HM_FLAG_ROPE  rotary position embedding on phi(q_t) and phi(k_t) before the
+ *     recurrence (HedgeMamba explainer sec. 5.2: RoPE on phi(Q), phi(K)), with
+ *     the "rotate half" pairing of feature i with feature i + F/2 and angle
+ *     pos_t * rope_base^(-2i/F); pos_t = pos0 + t in a scan, positions[b] in a
+ *     decode step.  Rotated features may be negative, so the denominator is
+ *     no longer positive by construction; no guard is applied (o = num / den).
  */
 typedef enum {
     HM_FLAG_DT_SCALED_INPUT = 1u,
-    HM_FLAG_PER_FEATURE_DECAY = 2u
+    HM_FLAG_PER_FEATURE_DECAY = 2u,
+    HM_FLAG_ROPE = 4u
 } hm_flag;
 
 /* Static description of a status code.  Never NULL. */
@@ -168,6 +175,8 @@ typedef struct {
                               log a_t, i.e. the log of the decay the whole call applies to the
                               state it starts from; or NULL.  With S_out of a zero-start call
                               it is the call's affine map S -> exp(.) S + S_out (hm_scan_combine). */
+    double rope_base;      /* HM_FLAG_ROPE: base of the rotation angles (> 0, e.g. 10000) */
+    int64_t pos0;          /* HM_FLAG_ROPE: position of token 0 of this call (>= 0) */
 } hm_scan_args;
 
 /* Bytes of workspace hm_scan_chunked_fwd needs for these arguments (0 on
@@ -216,6 +225,41 @@ typedef struct {
 HM_API hm_status hm_scan_combine(const hm_combine_args *a, hm_stream_t stream);
 
 /*
+ * hm_scan_bwd -- gradients of a prefill (HedgeMamba explainer sec. 3: the
+ * mixer is trained by distillation; SSM article sec. 4.3: the scan's states
+ * are recomputed in the backward pass, not stored).  For the loss
+ * sum over (b, t, h, c) of dout * o with o = hm_scan_chunked_fwd(...) (plain
+ * recurrence, no variant flags, shared Hedgehog weights without bias), it
+ * writes the gradients with respect to q, k, v, W_q, W_k, dt, A_log and,
+ * when asked, the initial state.  All gradients are fp32.  With W_q == NULL
+ * (q, k are the features, F = d), grad_q and grad_k are the gradients of the
+ * features and grad_W_q, grad_W_k are not written.
+ * Computed on CUDA cores in fp32 from fp32 features recomputed from q, k.
+ */
+typedef struct {
+    int64_t B, L;
+    int H, d, p, dv;       /* as in hm_scan_args */
+    hm_dtype io_dtype;     /* dtype of q, k, v, W_q, W_k and dout */
+    const void *q, *k, *v; /* the forward inputs */
+    const void *W_q, *W_k; /* [p, d] shared by all heads, or NULL */
+    const float *dt, *A_log; /* as in hm_scan_args (dt NULL: a = 1) */
+    const float *S0, *z0;  /* the forward's initial state or NULL */
+    const void *dout;      /* [B, L, H, dv] gradient of the loss with respect to o */
+    float *grad_q, *grad_k;     /* [B, L, H, d] */
+    float *grad_v;              /* [B, L, H, dv] */
+    float *grad_W_q, *grad_W_k; /* [p, d] (W_q != NULL) */
+    float *grad_dt;             /* [B, L, H] (dt != NULL) */
+    float *grad_A_log;          /* [H] (dt != NULL) */
+    float *grad_S0, *grad_z0;   /* [B, H, F, dv], [B, H, F], or NULL */
+    void *workspace;       /* >= hm_scan_bwd_workspace_size() bytes, 256-B aligned */
+    size_t workspace_bytes;
+} hm_scan_bwd_args;
+
+HM_API size_t hm_scan_bwd_workspace_size(const hm_scan_bwd_args *a);
+
+HM_API hm_status hm_scan_bwd(const hm_scan_bwd_args *a, hm_stream_t stream);
+
+/*
  * hm_step_decode -- one recurrent step per (batch, head) (linear-attention
  * tutorial sec. 3 and sec. 5, recurrent mode): feature maps on the new q and
  * k, then S <- a S + phi(k) v^T, z <- a z + phi(k), o = phi(q)^T S / phi(q)^T z.
@@ -239,6 +283,8 @@ typedef struct {
     void *workspace;       /* >= hm_decode_workspace_size() bytes, 256-B aligned */
     size_t workspace_bytes;
     unsigned int flags;    /* hm_flag bits, as in hm_scan_args */
+    double rope_base;      /* HM_FLAG_ROPE: base of the rotation angles (> 0) */
+    const int64_t *positions; /* HM_FLAG_ROPE: [B] device int64, position of each sequence's token */
 } hm_decode_args;
 
 HM_API size_t hm_decode_workspace_size(const hm_decode_args *a);

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libhm.so")
 
 HM_OK, HM_ERR_INVALID_ARG, HM_ERR_UNSUPPORTED, HM_ERR_CUDA, HM_ERR_TIMEOUT, HM_ERR_DEVICE = range(6)
 HM_F32, HM_BF16 = 0, 1
-HM_FLAG_DT_SCALED_INPUT, HM_FLAG_PER_FEATURE_DECAY = 1, 2
+HM_FLAG_DT_SCALED_INPUT, HM_FLAG_PER_FEATURE_DECAY, HM_FLAG_ROPE = 1, 2, 4
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libhm.so is not built (%s); run __graft_entry__.build() or "
@@ -38,7 +38,16 @@ class ScanArgs(ctypes.Structure):
                 ("w_head_stride", _I64), ("b_q", _P), ("b_k", _P), ("dt", _P), ("A_log", _P),
                 ("S0", _P), ("z0", _P), ("o", _P), ("S_out", _P), ("z_out", _P),
                 ("workspace", _P), ("workspace_bytes", _SZ), ("flags", ctypes.c_uint),
-                ("log_decay_out", _P)]
+                ("log_decay_out", _P), ("rope_base", ctypes.c_double), ("pos0", _I64)]
+
+
+class ScanBwdArgs(ctypes.Structure):
+    """Mirror of hm_scan_bwd_args."""
+    _fields_ = [("B", _I64), ("L", _I64), ("H", _I), ("d", _I), ("p", _I), ("dv", _I), ("io_dtype", _I),
+                ("q", _P), ("k", _P), ("v", _P), ("W_q", _P), ("W_k", _P), ("dt", _P), ("A_log", _P),
+                ("S0", _P), ("z0", _P), ("dout", _P), ("grad_q", _P), ("grad_k", _P), ("grad_v", _P),
+                ("grad_W_q", _P), ("grad_W_k", _P), ("grad_dt", _P), ("grad_A_log", _P), ("grad_S0", _P),
+                ("grad_z0", _P), ("workspace", _P), ("workspace_bytes", _SZ)]
 
 
 class CombineArgs(ctypes.Structure):
@@ -54,7 +63,7 @@ class DecodeArgs(ctypes.Structure):
                 ("q", _P), ("k", _P), ("v", _P), ("W_q", _P), ("W_k", _P),
                 ("w_head_stride", _I64), ("b_q", _P), ("b_k", _P), ("dt", _P), ("A_log", _P),
                 ("S", _P), ("z", _P), ("o", _P), ("workspace", _P), ("workspace_bytes", _SZ),
-                ("flags", ctypes.c_uint)]
+                ("flags", ctypes.c_uint), ("rope_base", ctypes.c_double), ("positions", _P)]
 
 
 class MixerArgs(ctypes.Structure):
@@ -86,6 +95,10 @@ lib.hm_mixer_workspace_size.restype = _SZ
 lib.hm_mixer_workspace_size.argtypes = [ctypes.POINTER(MixerArgs)]
 lib.hm_mixer_fwd.restype = _I
 lib.hm_mixer_fwd.argtypes = [ctypes.POINTER(MixerArgs), _P, _SZ, _P]
+lib.hm_scan_bwd_workspace_size.restype = _SZ
+lib.hm_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanBwdArgs)]
+lib.hm_scan_bwd.restype = _I
+lib.hm_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdArgs), _P]
 lib.hm_scan_combine.restype = _I
 lib.hm_scan_combine.argtypes = [ctypes.POINTER(CombineArgs), _P]
 lib.hm_launch_count.restype = ctypes.c_uint64
@@ -98,7 +111,8 @@ lib.hm_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
 EXPORTED = ("hm_status_string", "hm_last_error_detail", "hm_version", "hm_featmap",
             "hm_scan_workspace_size", "hm_scan_chunked_fwd", "hm_decode_workspace_size",
             "hm_step_decode", "hm_mixer_workspace_size", "hm_mixer_fwd", "hm_get_device_error",
-            "hm_launch_count", "hm_step_decode_noalloc", "hm_selftest_wait_timeout", "hm_scan_combine")
+            "hm_launch_count", "hm_step_decode_noalloc", "hm_selftest_wait_timeout", "hm_scan_combine",
+            "hm_scan_bwd_workspace_size", "hm_scan_bwd")
 
 
 class HMError(RuntimeError):
@@ -171,7 +185,8 @@ def hm_featmap(x, W, phi, H: int = 1, bias=None, w_head_stride: int = 0, stream=
 
 def scan_args(q, k, v, o, W_q=None, W_k=None, dt=None, A_log=None, S0=None, z0=None,
               S_out=None, z_out=None, b_q=None, b_k=None, w_head_stride: int = 0,
-              workspace=None, flags: int = 0, log_decay_out=None) -> ScanArgs:
+              workspace=None, flags: int = 0, log_decay_out=None, rope_base: float = 0.0,
+              pos0: int = 0) -> ScanArgs:
     """Fill an hm_scan_args from tensors (q, k: [B, L, H, d]; v, o: [B, L, H, dv]).
     o = None (with S_out) makes a state-only call; q may then be None too."""
     B, L, H, d = k.shape
@@ -187,6 +202,7 @@ def scan_args(q, k, v, o, W_q=None, W_k=None, dt=None, A_log=None, S0=None, z0=N
     a.S0, a.z0, a.S_out, a.z_out = _ptr(S0), _ptr(z0), _ptr(S_out), _ptr(z_out)
     a.flags = int(flags)
     a.log_decay_out = _ptr(log_decay_out)
+    a.rope_base, a.pos0 = float(rope_base), int(pos0)
     if workspace is not None:
         a.workspace = _ptr(workspace)
         a.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -201,6 +217,37 @@ def hm_scan_workspace_size(args: ScanArgs) -> int:
 
 def hm_scan_chunked_fwd(args: ScanArgs, stream=None) -> None:
     _check(lib.hm_scan_chunked_fwd(ctypes.byref(args), _stream(stream)), "hm_scan_chunked_fwd")
+
+
+def scan_bwd_args(q, k, v, dout, grad_q, grad_k, grad_v, W_q=None, W_k=None, grad_W_q=None,
+                  grad_W_k=None, dt=None, A_log=None, grad_dt=None, grad_A_log=None, S0=None, z0=None,
+                  grad_S0=None, grad_z0=None, workspace=None) -> ScanBwdArgs:
+    """Fill an hm_scan_bwd_args (forward inputs, dout [B, L, H, dv] and the fp32
+    gradient buffers)."""
+    B, L, H, d = q.shape
+    a = ScanBwdArgs()
+    a.B, a.L, a.H, a.d, a.dv = B, L, H, d, v.shape[-1]
+    a.p = W_q.shape[-2] if W_q is not None else 0
+    a.io_dtype = _dtype_code(q)
+    a.q, a.k, a.v, a.dout = _ptr(q), _ptr(k), _ptr(v), _ptr(dout)
+    a.W_q, a.W_k, a.dt, a.A_log, a.S0, a.z0 = map(_ptr, (W_q, W_k, dt, A_log, S0, z0))
+    a.grad_q, a.grad_k, a.grad_v = _ptr(grad_q), _ptr(grad_k), _ptr(grad_v)
+    a.grad_W_q, a.grad_W_k, a.grad_dt, a.grad_A_log = map(_ptr, (grad_W_q, grad_W_k, grad_dt, grad_A_log))
+    a.grad_S0, a.grad_z0 = _ptr(grad_S0), _ptr(grad_z0)
+    if workspace is not None:
+        a.workspace = _ptr(workspace)
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
+    a._refs = (q, k, v, dout, grad_q, grad_k, grad_v, W_q, W_k, grad_W_q, grad_W_k, dt, A_log, grad_dt,
+               grad_A_log, S0, z0, grad_S0, grad_z0, workspace)
+    return a
+
+
+def hm_scan_bwd_workspace_size(args: ScanBwdArgs) -> int:
+    return int(lib.hm_scan_bwd_workspace_size(ctypes.byref(args)))
+
+
+def hm_scan_bwd(args: ScanBwdArgs, stream=None) -> None:
+    _check(lib.hm_scan_bwd(ctypes.byref(args), _stream(stream)), "hm_scan_bwd")
 
 
 def combine_args(parts, n_parts: int, BH: int, F: int, dv: int, part_len: int, S_start, z_start,
@@ -228,7 +275,8 @@ def combine_record_len(BH: int, F: int, dv: int, per_feature: bool = False) -> i
 
 
 def decode_args(q, k, v, o, S, z, W_q=None, W_k=None, dt=None, A_log=None, b_q=None, b_k=None,
-                w_head_stride: int = 0, workspace=None, flags: int = 0) -> DecodeArgs:
+                w_head_stride: int = 0, workspace=None, flags: int = 0, rope_base: float = 0.0,
+                positions=None) -> DecodeArgs:
     """Fill an hm_decode_args (q, k: [B, H, d]; v, o: [B, H, dv]; S: [B, H, F, dv])."""
     B, H, d = q.shape
     a = DecodeArgs()
@@ -241,10 +289,11 @@ def decode_args(q, k, v, o, S, z, W_q=None, W_k=None, dt=None, A_log=None, b_q=N
     a.dt, a.A_log = _ptr(dt), _ptr(A_log)
     a.S, a.z = _ptr(S), _ptr(z)
     a.flags = int(flags)
+    a.rope_base, a.positions = float(rope_base), _ptr(positions)
     if workspace is not None:
         a.workspace = _ptr(workspace)
         a.workspace_bytes = workspace.numel() * workspace.element_size()
-    a._refs = (q, k, v, o, S, z, W_q, W_k, dt, A_log, b_q, b_k, workspace)
+    a._refs = (q, k, v, o, S, z, W_q, W_k, dt, A_log, b_q, b_k, workspace, positions)
     return a
 
 

@@ -87,7 +87,7 @@ extern "C" hm_status hm_step_decode_noalloc(const hm_decode_args *a, hm_stream_t
     }
     if (a->B == 0) return HM_OK;
     float *fq = nullptr, *fk = nullptr;
-    if (a->W_q) {
+    if (pl.feat_values > 0) {   // feature planes: the Hedgehog maps, or rotated caller features
         cudaError_t e = cudaSuccess;
         float *scratch = scratch_address(&e);
         if (!scratch) return reject(HM_ERR_CUDA, cudaGetErrorString(e));

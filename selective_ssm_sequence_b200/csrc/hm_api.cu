@@ -98,6 +98,54 @@ cudaError_t run_featmap_qk(const void *q, const void *k, hm_dtype xt, int64_t ro
     return launch_featmap_simt(k, xt, rows, H, d, p, W_k, wstride, b_k, phk, pt, s, phk_lo);
 }
 
+}  // namespace
+
+cudaError_t run_featmap_f32(const void *x, hm_dtype xt, int64_t rows, int H, int d, int p, const void *W,
+                            float *phi, cudaStream_t s) {
+    return run_featmap(x, xt, rows, H, d, p, W, 0, nullptr, phi, HM_F32, s);
+}
+
+namespace {
+
+// ------------------------------------------------------------------ backward
+
+hm_status check_scan_bwd(const hm_scan_bwd_args *a, ScanBwdCore *core) {
+    if (!a) return fail(HM_ERR_INVALID_ARG, "scan_bwd: null args");
+    if (!valid_dtype(a->io_dtype)) return fail(HM_ERR_INVALID_ARG, "scan_bwd: bad io dtype");
+    if (a->B < 0 || a->L < 0 || a->H < 1 || a->d < 1 || a->dv < 1)
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: bad sizes");
+    if ((a->W_q == nullptr) != (a->W_k == nullptr))
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: W_q and W_k must both be given or both NULL");
+    if ((a->S0 == nullptr) != (a->z0 == nullptr))
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: S0 and z0 must both be given or both NULL");
+    if ((a->grad_S0 == nullptr) != (a->grad_z0 == nullptr))
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: grad_S0 and grad_z0 must both be given or both NULL");
+    if (a->dt && (!a->A_log || !a->grad_dt || !a->grad_A_log))
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: dt needs A_log, grad_dt and grad_A_log");
+    const int F = a->W_q ? 2 * a->p : a->d;
+    if (a->W_q && (a->p < 1 || a->p > 256)) return fail(HM_ERR_UNSUPPORTED, "scan_bwd: need 1 <= p <= 256");
+    if (F > 256) return fail(HM_ERR_UNSUPPORTED, "scan_bwd: feature dim F=%d > 256", F);
+    if (a->d > 512) return fail(HM_ERR_UNSUPPORTED, "scan_bwd: d=%d > 512", a->d);
+    if (a->B * a->H > 65535) return fail(HM_ERR_UNSUPPORTED, "scan_bwd: B*H > 65535");
+    const int64_t rows = a->B * a->L * a->H;
+    if (rows > 0 && (!a->q || !a->k || !a->v || !a->dout || !a->grad_q || !a->grad_k || !a->grad_v ||
+                     (a->W_q && (!a->grad_W_q || !a->grad_W_k))))
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: null input or gradient pointer");
+    const void *ptrs[] = {a->q, a->k, a->v, a->W_q, a->W_k, a->dt, a->A_log, a->S0, a->z0, a->dout, a->grad_q,
+                          a->grad_k, a->grad_v, a->grad_W_q, a->grad_W_k, a->grad_dt, a->grad_A_log, a->grad_S0, a->grad_z0};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return fail(HM_ERR_INVALID_ARG, "scan_bwd: pointers must be 16-byte aligned");
+    ScanBwdCore c{};
+    c.B = a->B; c.L = a->L; c.H = a->H; c.d = a->d; c.p = a->p; c.F = F; c.dv = a->dv;
+    c.io_dtype = a->io_dtype;
+    c.q = a->q; c.k = a->k; c.v = a->v; c.dout = a->dout; c.W_q = a->W_q; c.W_k = a->W_k;
+    c.dt = a->dt; c.A_log = a->A_log; c.S0 = a->S0; c.z0 = a->z0;
+    c.dq = a->grad_q; c.dk = a->grad_k; c.dv_out = a->grad_v; c.dW_q = a->grad_W_q; c.dW_k = a->grad_W_k;
+    c.ddt = a->grad_dt; c.dA_log = a->grad_A_log; c.dS0 = a->grad_S0; c.dz0 = a->grad_z0;
+    *core = c;
+    return HM_OK;
+}
+
 // ------------------------------------------------------------------ scan
 
 struct ScanPlan {
@@ -123,10 +171,15 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
     if ((a->S_out == nullptr) != (a->z_out == nullptr))
         return fail(HM_ERR_INVALID_ARG, "scan: S_out and z_out must both be given or both NULL");
     if (a->dt && !a->A_log) return fail(HM_ERR_INVALID_ARG, "scan: dt given without A_log");
-    if (a->flags & ~(unsigned)(HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY))
+    if (a->flags & ~(unsigned)(HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY | HM_FLAG_ROPE))
         return fail(HM_ERR_INVALID_ARG, "scan: unknown flag bits 0x%x", a->flags);
-    if (a->flags && !a->dt) return fail(HM_ERR_INVALID_ARG, "scan: the variant flags need dt");
+    if ((a->flags & (HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY)) && !a->dt)
+        return fail(HM_ERR_INVALID_ARG, "scan: the step-scaled input and the per-feature decay need dt");
+    const bool rope = (a->flags & HM_FLAG_ROPE) != 0;
+    if (rope && (!(a->rope_base > 0.0) || a->pos0 < 0))
+        return fail(HM_ERR_INVALID_ARG, "scan: the rotary embedding needs rope_base > 0 and pos0 >= 0");
     const int F = a->W_q ? 2 * a->p : a->d;
+    if (rope && F % 2 != 0) return fail(HM_ERR_INVALID_ARG, "scan: the rotary embedding needs an even F");
     if (a->W_q && (a->p < 1 || a->p > 256)) return fail(HM_ERR_UNSUPPORTED, "scan: need 1 <= p <= 256");
     if (F > 256) return fail(HM_ERR_UNSUPPORTED, "scan: feature dim F=%d > 256", F);
     if (a->d > 512) return fail(HM_ERR_UNSUPPORTED, "scan: d=%d > 512", a->d);
@@ -154,7 +207,9 @@ hm_status check_scan(const hm_scan_args *a, ScanPlan *plan) {
     // W_q == NULL the caller's q / k are the features and keep their dtype.
     pl.feat = a->W_q ? (pl.tc ? HM_BF16 : HM_F32) : a->io_dtype;
     c.feat_dtype = pl.feat;
-    pl.phi_bytes = a->W_q ? round_up((size_t)rows * F * dsize(pl.feat), 256) : 0;
+    // rotated caller features (W_q == NULL with the rotary embedding) are
+    // written to the workspace too: the caller's q, k are never modified
+    pl.phi_bytes = (a->W_q || rope) ? round_up((size_t)rows * F * dsize(pl.feat), 256) : 0;
     pl.lo_bytes = (pl.tc && a->W_q && a->S_out) ? pl.phi_bytes : 0;
     pl.tc_bytes = pl.tc ? round_up(scan_tc_workspace(c), 256) : 0;
     pl.total = 2 * pl.phi_bytes + pl.lo_bytes + pl.tc_bytes;
@@ -172,10 +227,15 @@ hm_status check_decode(const hm_decode_args *a, DecodePlan *plan) {
     if ((a->W_q == nullptr) != (a->W_k == nullptr))
         return fail(HM_ERR_INVALID_ARG, "decode: W_q and W_k must both be given or both NULL");
     if (a->dt && !a->A_log) return fail(HM_ERR_INVALID_ARG, "decode: dt given without A_log");
-    if (a->flags & ~(unsigned)(HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY))
+    if (a->flags & ~(unsigned)(HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY | HM_FLAG_ROPE))
         return fail(HM_ERR_INVALID_ARG, "decode: unknown flag bits 0x%x", a->flags);
-    if (a->flags && !a->dt) return fail(HM_ERR_INVALID_ARG, "decode: the variant flags need dt");
+    if ((a->flags & (HM_FLAG_DT_SCALED_INPUT | HM_FLAG_PER_FEATURE_DECAY)) && !a->dt)
+        return fail(HM_ERR_INVALID_ARG, "decode: the step-scaled input and the per-feature decay need dt");
+    const bool rope = (a->flags & HM_FLAG_ROPE) != 0;
+    if (rope && (!(a->rope_base > 0.0) || !a->positions || !aligned16(a->positions)))
+        return fail(HM_ERR_INVALID_ARG, "decode: the rotary embedding needs rope_base > 0 and positions");
     const int F = a->W_q ? 2 * a->p : a->d;
+    if (rope && F % 2 != 0) return fail(HM_ERR_INVALID_ARG, "decode: the rotary embedding needs an even F");
     if (a->W_q && (a->p < 1 || a->p > 256)) return fail(HM_ERR_UNSUPPORTED, "decode: need 1 <= p <= 256");
     if (F > 256) return fail(HM_ERR_UNSUPPORTED, "decode: feature dim F=%d > 256", F);
     if (a->d > 512) return fail(HM_ERR_UNSUPPORTED, "decode: d=%d > 512", a->d);
@@ -190,8 +250,8 @@ hm_status check_decode(const hm_decode_args *a, DecodePlan *plan) {
         if (!aligned16(p)) return fail(HM_ERR_INVALID_ARG, "decode: pointers must be 16-byte aligned");
     DecodePlan pl{};
     pl.F = F;
-    pl.feat_values = a->W_q ? a->B * a->H * F : 0;
-    pl.phi_bytes = a->W_q ? round_up((size_t)pl.feat_values * sizeof(float), 256) : 0;
+    pl.feat_values = (a->W_q || rope) ? a->B * a->H * F : 0;
+    pl.phi_bytes = pl.feat_values ? round_up((size_t)pl.feat_values * sizeof(float), 256) : 0;
     pl.total = 2 * pl.phi_bytes;
     *plan = pl;
     return HM_OK;
@@ -221,6 +281,17 @@ hm_status decode_enqueue(const hm_decode_args *a, const DecodePlan &pl, void *ph
         phq = phq_buf;
         phk = phk_buf;
         ft = HM_F32;
+    }
+    if (a->flags & HM_FLAG_ROPE) {
+        // rotary embedding at each sequence's position: in place on the fp32
+        // maps above, or from the caller's features into the fp32 planes
+        e = launch_rope(phq, nullptr, phq_buf, nullptr, ft, a->B, 1, a->H, pl.F, a->rope_base, 0, a->positions, s);
+        if (e == cudaSuccess)
+            e = launch_rope(phk, nullptr, phk_buf, nullptr, ft, a->B, 1, a->H, pl.F, a->rope_base, 0, a->positions,
+                            s);
+        if (e != cudaSuccess) return cuda_fail(e, "decode: rotary embedding");
+        phq = phq_buf;
+        phk = phk_buf;
     }
     DecodeCore c{};
     c.B = a->B; c.H = a->H; c.F = pl.F; c.dv = a->dv;
@@ -405,6 +476,22 @@ hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
         phk_lo = wkl;
     }
     if (!a->o) phq = nullptr;
+    if ((a->flags & HM_FLAG_ROPE) && rows > 0) {
+        // rotary embedding of phi(q), phi(k): in place on the maps computed
+        // above, or from the caller's features into the workspace
+        void *wq = ws, *wk = ws + pl.phi_bytes;
+        void *wkl = pl.lo_bytes ? ws + 2 * pl.phi_bytes : nullptr;
+        if (phq) {
+            e = launch_rope(phq, nullptr, wq, nullptr, pl.feat, a->B, a->L, a->H, pl.F, a->rope_base, a->pos0,
+                            nullptr, s);
+            if (e != cudaSuccess) return cuda_fail(e, "scan: rotary embedding");
+            phq = wq;
+        }
+        e = launch_rope(phk, phk_lo, wk, wkl, pl.feat, a->B, a->L, a->H, pl.F, a->rope_base, a->pos0, nullptr, s);
+        if (e != cudaSuccess) return cuda_fail(e, "scan: rotary embedding");
+        phk = wk;
+        phk_lo = wkl;
+    }
     if (a->log_decay_out) {
         e = launch_logdecay_sum(a->B, a->L, a->H, pl.F, (a->flags & HM_FLAG_PER_FEATURE_DECAY) != 0, a->dt,
                                 a->A_log, a->log_decay_out, s);
@@ -443,6 +530,26 @@ extern "C" hm_status hm_scan_chunked_fwd(const hm_scan_args *a, hm_stream_t stre
 }
 
 extern "C" {
+
+size_t hm_scan_bwd_workspace_size(const hm_scan_bwd_args *a) {
+    ScanBwdCore c;
+    if (check_scan_bwd(a, &c) != HM_OK) return 0;
+    return scan_bwd_workspace(c);
+}
+
+hm_status hm_scan_bwd(const hm_scan_bwd_args *a, hm_stream_t stream) {
+    g_detail[0] = 0;
+    ScanBwdCore c;
+    hm_status st = check_scan_bwd(a, &c);
+    if (st != HM_OK) return st;
+    const size_t need = scan_bwd_workspace(c);
+    if (!a->workspace || a->workspace_bytes < need)
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: workspace too small (%zu < %zu bytes)", a->workspace_bytes, need);
+    if (((uintptr_t)a->workspace & 255u) != 0)
+        return fail(HM_ERR_INVALID_ARG, "scan_bwd: workspace must be 256-byte aligned");
+    cudaError_t e = launch_scan_bwd(c, a->workspace, (cudaStream_t)stream);
+    return e == cudaSuccess ? HM_OK : cuda_fail(e, "scan_bwd launch");
+}
 
 size_t hm_decode_workspace_size(const hm_decode_args *a) {
     DecodePlan pl;

@@ -125,6 +125,29 @@ cudaError_t launch_scan_tc(const ScanCore &c, void *ws, size_t ws_bytes, DevErr 
 cudaError_t launch_logdecay_sum(int64_t B, int64_t L, int H, int F, bool per_feature, const float *dt,
                                 const float *A_log, float *out, cudaStream_t s);
 
+// Rotary embedding of feature rows [B, L, H, F] (ft = fp32 or bf16, with an
+// optional bf16 remainder plane), src -> dst (may alias): pair (i, i + F/2) at
+// angle (positions ? positions[b] : pos0 + t) * base^(-2i/F).
+cudaError_t launch_rope(const void *src, const void *src_lo, void *dst, void *dst_lo, hm_dtype ft, int64_t B,
+                        int64_t L, int H, int F, double base, int64_t pos0, const int64_t *positions,
+                        cudaStream_t s);
+
+// Backward of the scan and of the Hedgehog maps (CUDA cores, fp32).
+struct ScanBwdCore {
+    int64_t B, L;
+    int H, d, p, F, dv;
+    hm_dtype io_dtype;
+    const void *q, *k, *v, *dout;
+    const void *W_q, *W_k;    // shared Hedgehog weights, or null: q, k are the features
+    const float *dt, *A_log, *S0, *z0;
+    float *dq, *dk, *dv_out, *dW_q, *dW_k, *ddt, *dA_log, *dS0, *dz0;
+};
+size_t scan_bwd_workspace(const ScanBwdCore &c);
+cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s);
+// The Hedgehog map into fp32 features (tensor cores when the shape has a kernel).
+cudaError_t run_featmap_f32(const void *x, hm_dtype xt, int64_t rows, int H, int d, int p, const void *W,
+                            float *phi, cudaStream_t s);
+
 // Decode step over precomputed features.
 struct DecodeCore {
     int64_t B;

@@ -1,0 +1,507 @@
+// scan_bwd.cu -- gradients of the decayed normalised scan and of the Hedgehog
+// feature map on CUDA cores, fp32.
+//
+// The mixer is trained (HedgeMamba explainer sec. 3: two-stage distillation),
+// and Mamba-style scans recompute their states in the backward pass instead
+// of storing them (SSM article sec. 4.3).  For L = sum_t do_t . o_t with
+//   S_t = a_t S_{t-1} + phik_t v_t^T,  z_t = a_t z_{t-1} + phik_t,
+//   n_t = S_t^T phiq_t,  d_t = phiq_t . z_t,  o_t = n_t / d_t
+// and dn_t = do_t / d_t, dd_t = -(do_t . o_t) / d_t:
+//   dphiq_t = S_t dn_t + z_t dd_t                          (forward in time)
+//   G_t = phiq_t dn_t^T + a_{t+1} G_{t+1},  g_t likewise   (backward in time)
+//   dphik_t = G_t v_t + g_t,   dv_t = G_t^T phik_t,   dS0 = a_1 G_1, dz0 = a_1 g_1
+//   dlog a_t = -sum_{i >= t} phik_i . dphik_i
+// The last line holds because o_t is normalised: the factors exp(cum_i) that
+// a decay puts on the query side of S_i cancel between n_i and d_i, so only
+// the key side of each pair (j < t <= i) carries the gradient, and that is the
+// key's phik_j . dphik_j.  It needs neither forward nor backward state, so no
+// pass has to hold S and G at once.
+//
+// Passes, each one CTA per (batch, head, 32 value columns) with the state in
+// registers as in the CUDA-core forward scan (warp w holds feature rows w,
+// w + 8, ..., lane = value column):
+//   P0 forward: d_t (slice 0) and the slice's share of sum_c do_t[c] n_t[c]
+//   PA forward: the slice's share of dphiq_t (+ z_t dd_t on slice 0)
+//   PB backward: the slice's share of dphik_t (+ g_t on slice 0), dv_t, dS0, dz0
+// then a reduction of the slices' shares (and the suffix sums of dlog a),
+// the feature-map backward (softmax Jacobian, dx = du W, dW = sum du x^T) and
+// the decay's (d dt = dlog a (-sigmoid(dt) e^A_log), dA_log = sum dlog a * log a).
+#include "hm_internal.h"
+
+namespace hm {
+
+namespace {
+
+constexpr int kW = 8;        // warps
+constexpr int kTB = 16;      // tokens staged per round
+constexpr int kMaxRows = 32; // F <= 256
+
+struct BwdArgs {
+    int64_t B, L;
+    int H, F, dv, ns;        // ns = column slices (dv / 32, rounded up)
+    const float *phq, *phk;  // [B, L, H, F] fp32
+    const void *v;           // [B, L, H, dv] of io dtype
+    const void *dout;        // [B, L, H, dv] of io dtype
+    const float *dt, *A_log;
+    const float *S0, *z0;
+    float *den;              // [B, L, H]
+    float *e_part;           // [ns][B, L, H]: slices' shares of do . n
+    float *dq_part, *dk_part;   // [ns][B, L, H, F]
+    float *dv_out;           // [B, L, H, dv] fp32
+    float *dS0, *dz0;        // nullable
+};
+
+template <int MODE, typename TIO>
+__global__ void __launch_bounds__(32 * kW)
+bwd_pass_kernel(BwdArgs a) {
+    // MODE 0: P0, MODE 1: PA, MODE 2: PB (tokens in reverse order)
+    extern __shared__ float smem[];
+    const int F = a.F, dv = a.dv;
+    float *sq = smem;                      // [kTB][F]
+    float *sk = sq + kTB * F;              // [kTB][F]
+    float *sv = sk + kTB * F;              // [kTB][32]   v
+    float *sg = sv + kTB * 32;             // [kTB][32]   do
+    float *sa = sg + kTB * 32;             // [kTB]       a_t
+    float *sa1 = sa + kTB;                 // [kTB]       a_{t+1} (PB)
+    float *sden = sa1 + kTB;               // [kTB]
+    float *sdd = sden + kTB;               // [kTB]       dd_t
+    float *red = sdd + kTB;                // [kTB][kW][32]
+    float *rden = red + kTB * kW * 32;     // [kTB][kW]
+
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t bh = blockIdx.y;
+    const int64_t b = bh / a.H;
+    const int h = (int)(bh % a.H);
+    const int slice = blockIdx.x;
+    const int col = slice * 32 + lane;
+    const bool col_ok = col < dv;
+    const float alog = a.dt ? a.A_log[h] : 0.f;
+    const TIO *v = (const TIO *)a.v;
+    const TIO *dout = (const TIO *)a.dout;
+    const int64_t L = a.L;
+    auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
+
+    float S[kMaxRows], z[kMaxRows];
+#pragma unroll
+    for (int m = 0; m < kMaxRows; ++m) {
+        const int f = w + kW * m;
+        S[m] = 0.f;
+        z[m] = 0.f;
+        if (MODE < 2 && f < F) {
+            if (a.S0 && col_ok) S[m] = a.S0[(bh * F + f) * dv + col];
+            if (a.z0) z[m] = a.z0[bh * F + f];
+        }
+    }
+    const int64_t nblk = (L + kTB - 1) / kTB;
+    for (int64_t bi = 0; bi < nblk; ++bi) {
+        // PB walks the token blocks from the last to the first
+        const int64_t t0 = (MODE == 2 ? nblk - 1 - bi : bi) * kTB;
+        const int nt = (int)((L - t0) < kTB ? (L - t0) : kTB);
+        for (int i = threadIdx.x; i < nt * F; i += blockDim.x) {
+            const int t = i / F, f = i % F;
+            sq[i] = a.phq[rowi(t0 + t) * F + f];
+            sk[i] = a.phk[rowi(t0 + t) * F + f];
+        }
+        for (int i = threadIdx.x; i < nt * 32; i += blockDim.x) {
+            const int t = i / 32, c = slice * 32 + (i % 32);
+            const bool ok = c < dv;
+            sv[i] = ok ? hm_ld(v, rowi(t0 + t) * dv + c) : 0.f;
+            sg[i] = ok ? hm_ld(dout, rowi(t0 + t) * dv + c) : 0.f;
+        }
+        if (threadIdx.x < nt) {
+            const int t = threadIdx.x;
+            const int64_t r = rowi(t0 + t);
+            sa[t] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
+            // a_{t+1}: the decay that carries G_{t+1} back to token t (none after the last token)
+            sa1[t] = (t0 + t + 1 < L && a.dt) ? expf(hm_log_decay(a.dt[rowi(t0 + t + 1)], alog)) : 1.f;
+            if (MODE >= 1) {
+                const float dn_den = a.den[r];
+                float e = 0.f;
+                for (int s = 0; s < a.ns; ++s) e += a.e_part[(int64_t)s * a.B * L * a.H + r];
+                sden[t] = dn_den;
+                sdd[t] = -e / (dn_den * dn_den);   // dd = -(do . o) / d = -(do . n) / d^2
+            }
+        }
+        __syncthreads();
+        if (MODE < 2) {
+            for (int t = 0; t < nt; ++t) {
+                const float at = sa[t];
+                const float vv = sv[t * 32 + lane];
+                float num = 0.f, den = 0.f;
+#pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) {
+                    const int f = w + kW * m;
+                    if (f < F) {
+                        const float kf = sk[t * F + f], qf = sq[t * F + f];
+                        S[m] = fmaf(at, S[m], kf * vv);
+                        z[m] = fmaf(at, z[m], kf);
+                        num = fmaf(qf, S[m], num);
+                        den = fmaf(qf, z[m], den);
+                    }
+                }
+                if (MODE == 0) {
+                    red[(t * kW + w) * 32 + lane] = num;
+                    if (lane == 0) rden[t * kW + w] = den;
+                } else {
+                    // the slice's share of dphiq_t[f] = sum_c S_t[f, c] dn_t[c] (+ z_t[f] dd_t)
+                    const float dn = sg[t * 32 + lane] / sden[t];
+                    const int64_t r = rowi(t0 + t);
+                    float *dq = a.dq_part + ((int64_t)slice * a.B * L * a.H + r) * F;
+#pragma unroll
+                    for (int m = 0; m < kMaxRows; ++m) {
+                        const int f = w + kW * m;
+                        if (f < F) {
+                            float x = warp_sum(S[m] * dn);
+                            if (lane == (m & 31)) dq[f] = x + (slice == 0 ? z[m] * sdd[t] : 0.f);
+                        }
+                    }
+                }
+            }
+            if (MODE == 0) {
+                __syncthreads();
+                // per token: d_t (slice 0) and the slice's share of do_t . n_t
+                for (int t = w; t < nt; t += kW) {
+                    float n = 0.f, d = 0.f;
+                    for (int ww = 0; ww < kW; ++ww) {
+                        n += red[(t * kW + ww) * 32 + lane];
+                        d += rden[t * kW + ww];
+                    }
+                    const float e = warp_sum(n * sg[t * 32 + lane]);
+                    const int64_t r = rowi(t0 + t);
+                    if (lane == 0) {
+                        a.e_part[(int64_t)slice * a.B * L * a.H + r] = e;
+                        if (slice == 0) a.den[r] = d;
+                    }
+                }
+            }
+        } else {
+            // PB: G_t = phiq_t dn_t^T + a_{t+1} G_{t+1} (S holds G, z holds g)
+            for (int t = nt - 1; t >= 0; --t) {
+                const float a1 = sa1[t];
+                const float dn = sg[t * 32 + lane] / sden[t];
+                const float dd = sdd[t];
+                const float vv = sv[t * 32 + lane];
+                const int64_t r = rowi(t0 + t);
+                float *dk = a.dk_part + ((int64_t)slice * a.B * L * a.H + r) * F;
+                float dvp = 0.f;
+#pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) {
+                    const int f = w + kW * m;
+                    if (f < F) {
+                        const float qf = sq[t * F + f], kf = sk[t * F + f];
+                        S[m] = fmaf(a1, S[m], qf * dn);
+                        z[m] = fmaf(a1, z[m], qf * dd);
+                        dvp = fmaf(S[m], kf, dvp);
+                        const float x = warp_sum(S[m] * vv);
+                        if (lane == (m & 31)) dk[f] = x + (slice == 0 ? z[m] : 0.f);
+                    }
+                }
+                red[(t * kW + w) * 32 + lane] = dvp;
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < nt * 32; i += blockDim.x) {
+                const int t = i / 32, c = i % 32;
+                float acc = 0.f;
+                for (int ww = 0; ww < kW; ++ww) acc += red[(t * kW + ww) * 32 + c];
+                const int cc = slice * 32 + c;
+                if (cc < dv) a.dv_out[rowi(t0 + t) * dv + cc] = acc;
+            }
+            if (t0 == 0) {
+                // dS0 = a_1 G_1, dz0 = a_1 g_1 (a_1 = the first token's decay)
+                const float a0 = sa[0];
+#pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) {
+                    const int f = w + kW * m;
+                    if (f < F) {
+                        if (a.dS0 && col_ok) a.dS0[(bh * F + f) * dv + col] = a0 * S[m];
+                        if (a.dz0 && slice == 0 && lane == 0) a.dz0[bh * F + f] = a0 * z[m];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// dphiq, dphik = sums of the slices' shares, and kd_r = phik_r . dphik_r;
+// one warp per row (lanes over the features).
+__global__ void __launch_bounds__(256)
+bwd_reduce_kernel(BwdArgs a, float *__restrict__ dphq, float *__restrict__ dphk, float *__restrict__ kd) {
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = a.B * a.L * a.H;
+    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (r >= rows) return;
+    const int64_t plane = rows * (int64_t)a.F;
+    float acc = 0.f;
+    for (int f = lane; f < a.F; f += 32) {
+        float sq = 0.f, sk = 0.f;
+        for (int s = 0; s < a.ns; ++s) {
+            sq += a.dq_part[s * plane + r * a.F + f];
+            sk += a.dk_part[s * plane + r * a.F + f];
+        }
+        dphq[r * a.F + f] = sq;
+        dphk[r * a.F + f] = sk;
+        acc = fmaf(a.phk[r * a.F + f], sk, acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) kd[r] = acc;
+}
+
+// dlog a_t = -sum_{i >= t} kd_i per (b, h): one warp per (b, h) walks the
+// tokens from the end in blocks of 32 with a warp suffix scan.
+__global__ void __launch_bounds__(256)
+bwd_suffix_kernel(int64_t B, int64_t L, int H, const float *__restrict__ kd, float *__restrict__ dla) {
+    const int lane = threadIdx.x & 31;
+    const int64_t bh = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (bh >= B * H) return;
+    const int64_t b = bh / H;
+    const int h = (int)(bh % H);
+    float carry = 0.f;
+    for (int64_t tb = L - 1; tb >= 0; tb -= 32) {
+        const int64_t t = tb - lane;   // lane 0 = the latest token of the block
+        float x = t >= 0 ? kd[(b * L + t) * H + h] : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (t >= 0) dla[(b * L + t) * H + h] = -(carry + x);
+        carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+}
+
+// fp32 copy of caller-supplied features (for the passes above).
+template <typename T>
+__global__ void to_f32_kernel(const T *__restrict__ x, int64_t n, float *__restrict__ y) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = hm_ld(x, i);
+}
+
+// Feature-map backward, per row: phi = softmax([u, -u]), so
+// de = phi (.) (dphi - sum(phi (.) dphi)), du = de[:p] - de[p:].  One warp per row.
+__global__ void __launch_bounds__(256)
+featmap_bwd_du_kernel(const float *__restrict__ phi, const float *__restrict__ dphi, int64_t rows, int p,
+                      float *__restrict__ du) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (r >= rows) return;
+    const float *ph = phi + r * 2 * p, *dp = dphi + r * 2 * p;
+    float s = 0.f;
+    for (int f = lane; f < 2 * p; f += 32) s = fmaf(ph[f], dp[f], s);
+    s = warp_sum(s);
+    for (int j = lane; j < p; j += 32)
+        du[r * p + j] = ph[j] * (dp[j] - s) - ph[p + j] * (dp[p + j] - s);
+}
+
+// dx[r, i] = sum_j du[r, j] W[j, i]: one CTA per 32 rows, W read from L2.
+template <typename TW>
+__global__ void __launch_bounds__(256)
+featmap_bwd_dx_kernel(const float *__restrict__ du, const TW *__restrict__ W, int64_t rows, int p, int d,
+                      float *__restrict__ dx) {
+    __shared__ float sdu[32][256];
+    const int64_t r0 = (int64_t)blockIdx.x * 32;
+    for (int i = threadIdx.x; i < 32 * p; i += blockDim.x) {
+        const int rr = i / p, j = i % p;
+        sdu[rr][j] = r0 + rr < rows ? du[(r0 + rr) * p + j] : 0.f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+        float acc[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) acc[rr] = 0.f;
+        for (int j = 0; j < p; ++j) {
+            const float wv = hm_ld(W, (int64_t)j * d + i);
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) acc[rr] = fmaf(sdu[rr][j], wv, acc[rr]);
+        }
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr)
+            if (r0 + rr < rows) dx[(r0 + rr) * d + i] = acc[rr];
+    }
+}
+
+// dW[j, i] += sum over the CTA's rows of du[r, j] x[r, i]: CTA = (1024 rows,
+// 32 x 64 tile of dW); partial sums added to dW (zeroed first) atomically.
+template <typename TX>
+__global__ void __launch_bounds__(256)
+featmap_bwd_dw_kernel(const float *__restrict__ du, const TX *__restrict__ x, int64_t rows, int p, int d,
+                      float *__restrict__ dW) {
+    __shared__ float su[32][32];
+    __shared__ float sx[32][64];
+    const int j0 = blockIdx.y * 32, i0 = blockIdx.z * 64;
+    const int64_t r0 = (int64_t)blockIdx.x * 1024;
+    const int tj = threadIdx.x >> 3, ti = (threadIdx.x & 7) * 8;   // thread: dW[j0 + tj][i0 + ti .. +8]
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int64_t rb = r0; rb < r0 + 1024 && rb < rows; rb += 32) {
+        for (int k = threadIdx.x; k < 32 * 32; k += 256) {
+            const int rr = k / 32, jj = k % 32;
+            su[rr][jj] = (rb + rr < rows && j0 + jj < p) ? du[(rb + rr) * p + j0 + jj] : 0.f;
+        }
+        for (int k = threadIdx.x; k < 32 * 64; k += 256) {
+            const int rr = k / 64, ii = k % 64;
+            sx[rr][ii] = (rb + rr < rows && i0 + ii < d) ? hm_ld(x, (rb + rr) * d + i0 + ii) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int rr = 0; rr < 32; ++rr) {
+            const float uj = su[rr][tj];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(uj, sx[rr][ti + e], acc[e]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        if (j0 + tj < p && i0 + ti + e < d) atomicAdd(&dW[(int64_t)(j0 + tj) * d + i0 + ti + e], acc[e]);
+}
+
+// d dt = dlog a * (-sigmoid(dt) e^A_log);  dA_log[h] += sum dlog a * log a.
+__global__ void __launch_bounds__(256)
+decay_bwd_kernel(const float *__restrict__ dt, const float *__restrict__ A_log, const float *__restrict__ dla,
+                 int64_t BL, int H, float *__restrict__ ddt, float *__restrict__ dA) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    float contrib = 0.f;
+    int h = 0;
+    if (i < BL * H) {
+        h = (int)(i % H);
+        const float x = dt[i], rate = expf(A_log[h]);
+        const float sig = 1.f / (1.f + expf(-x));
+        ddt[i] = dla[i] * (-sig * rate);
+        contrib = dla[i] * hm_log_decay(x, A_log[h]);
+    }
+    // lanes of a warp may hold different heads: one addition per element
+    if (i < BL * H) atomicAdd(&dA[h], contrib);
+}
+
+template <typename TIO>
+cudaError_t run_passes(const BwdArgs &a, cudaStream_t s) {
+    dim3 grid((unsigned)a.ns, (unsigned)(a.B * a.H));
+    const size_t smem = sizeof(float) * (size_t)(2 * kTB * a.F + 2 * kTB * 32 + 4 * kTB + kTB * kW * 32 + kTB * kW);
+    cudaError_t e;
+    auto k0 = bwd_pass_kernel<0, TIO>;
+    auto k1 = bwd_pass_kernel<1, TIO>;
+    auto k2 = bwd_pass_kernel<2, TIO>;
+    for (auto k : {k0, k1, k2}) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k0<<<grid, 32 * kW, smem, s>>>(a);
+    k1<<<grid, 32 * kW, smem, s>>>(a);
+    k2<<<grid, 32 * kW, smem, s>>>(a);
+    count_launches(3);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t scan_bwd_workspace(const ScanBwdCore &c) {
+    const int ns = (c.dv + 31) / 32;
+    const size_t rows = (size_t)c.B * c.L * c.H;
+    auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+    size_t n = 0;
+    n += 2 * r256(rows * c.F * 4);             // phq, phk (fp32)
+    n += r256(rows * 4);                       // den
+    n += r256((size_t)ns * rows * 4);          // e_part
+    n += 2 * r256((size_t)ns * rows * c.F * 4);  // dq_part, dk_part
+    n += 2 * r256(rows * c.F * 4);             // dphq, dphk
+    n += 2 * r256(rows * 4);                   // kd, dlog a
+    if (c.W_q) n += r256(rows * c.p * 4);      // du
+    return n;
+}
+
+cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
+    const int ns = (c.dv + 31) / 32;
+    const int64_t rows = c.B * c.L * c.H;
+    if (rows == 0) return cudaSuccess;
+    auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+    char *w = (char *)ws;
+    auto take = [&](size_t bytes) { char *p = w; w += r256(bytes); return p; };
+    float *phq = (float *)take(rows * c.F * 4), *phk = (float *)take(rows * c.F * 4);
+    BwdArgs a{};
+    a.B = c.B; a.L = c.L; a.H = c.H; a.F = c.F; a.dv = c.dv; a.ns = ns;
+    a.phq = phq; a.phk = phk; a.v = c.v; a.dout = c.dout; a.dt = c.dt; a.A_log = c.A_log;
+    a.S0 = c.S0; a.z0 = c.z0;
+    a.den = (float *)take(rows * 4);
+    a.e_part = (float *)take((size_t)ns * rows * 4);
+    a.dq_part = (float *)take((size_t)ns * rows * c.F * 4);
+    a.dk_part = (float *)take((size_t)ns * rows * c.F * 4);
+    float *dphq = (float *)take(rows * c.F * 4), *dphk = (float *)take(rows * c.F * 4);
+    float *kd = (float *)take(rows * 4);
+    float *dla = (float *)take(rows * 4);
+    float *du = c.W_q ? (float *)take(rows * c.p * 4) : nullptr;
+    a.dv_out = c.dv_out;
+    a.dS0 = c.dS0;
+    a.dz0 = c.dz0;
+    cudaError_t e;
+    // the features in fp32: the Hedgehog maps, or the caller's features
+    if (c.W_q) {
+        e = run_featmap_f32(c.q, c.io_dtype, rows, c.H, c.d, c.p, c.W_q, phq, s);
+        if (e == cudaSuccess) e = run_featmap_f32(c.k, c.io_dtype, rows, c.H, c.d, c.p, c.W_k, phk, s);
+    } else {
+        const int64_t n = rows * c.F;
+        const unsigned nb = (unsigned)((n + 255) / 256);
+        if (c.io_dtype == HM_BF16) {
+            to_f32_kernel<__nv_bfloat16><<<nb, 256, 0, s>>>((const __nv_bfloat16 *)c.q, n, phq);
+            to_f32_kernel<__nv_bfloat16><<<nb, 256, 0, s>>>((const __nv_bfloat16 *)c.k, n, phk);
+        } else {
+            to_f32_kernel<float><<<nb, 256, 0, s>>>((const float *)c.q, n, phq);
+            to_f32_kernel<float><<<nb, 256, 0, s>>>((const float *)c.k, n, phk);
+        }
+        count_launches(2);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return e;
+    e = c.io_dtype == HM_BF16 ? run_passes<__nv_bfloat16>(a, s) : run_passes<float>(a, s);
+    if (e != cudaSuccess) return e;
+    const unsigned wb = (unsigned)((rows * 32 + 255) / 256);
+    bwd_reduce_kernel<<<wb, 256, 0, s>>>(a, dphq, dphk, kd);
+    bwd_suffix_kernel<<<(unsigned)((c.B * c.H * 32 + 255) / 256), 256, 0, s>>>(c.B, c.L, c.H, kd, dla);
+    count_launches(2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (c.W_q) {
+        const unsigned xb = (unsigned)((rows + 31) / 32);
+        dim3 gw((unsigned)((rows + 1023) / 1024), (unsigned)((c.p + 31) / 32), (unsigned)((c.d + 63) / 64));
+        const float *dphis[2] = {dphq, dphk};
+        const float *phis[2] = {phq, phk};
+        const void *xs[2] = {c.q, c.k};
+        const void *Ws[2] = {c.W_q, c.W_k};
+        float *dxs[2] = {c.dq, c.dk};
+        float *dWs[2] = {c.dW_q, c.dW_k};
+        for (int m = 0; m < 2; ++m) {
+            featmap_bwd_du_kernel<<<wb, 256, 0, s>>>(phis[m], dphis[m], rows, c.p, du);
+            if (c.io_dtype == HM_BF16)
+                featmap_bwd_dx_kernel<__nv_bfloat16><<<xb, 256, 0, s>>>(du, (const __nv_bfloat16 *)Ws[m], rows, c.p,
+                                                                         c.d, dxs[m]);
+            else
+                featmap_bwd_dx_kernel<float><<<xb, 256, 0, s>>>(du, (const float *)Ws[m], rows, c.p, c.d, dxs[m]);
+            e = cudaMemsetAsync(dWs[m], 0, sizeof(float) * (size_t)c.p * c.d, s);
+            if (e != cudaSuccess) return e;
+            if (c.io_dtype == HM_BF16)
+                featmap_bwd_dw_kernel<__nv_bfloat16><<<gw, 256, 0, s>>>(du, (const __nv_bfloat16 *)xs[m], rows, c.p,
+                                                                         c.d, dWs[m]);
+            else
+                featmap_bwd_dw_kernel<float><<<gw, 256, 0, s>>>(du, (const float *)xs[m], rows, c.p, c.d, dWs[m]);
+            count_launches(3);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+    } else {
+        // caller features: their gradients are dphiq and dphik
+        e = cudaMemcpyAsync(c.dq, dphq, (size_t)rows * c.F * 4, cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(c.dk, dphk, (size_t)rows * c.F * 4, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return e;
+    }
+    if (c.dt) {
+        e = cudaMemsetAsync(c.dA_log, 0, sizeof(float) * (size_t)c.H, s);
+        if (e != cudaSuccess) return e;
+        const int64_t BL = c.B * c.L;
+        decay_bwd_kernel<<<(unsigned)((BL * c.H + 255) / 256), 256, 0, s>>>(c.dt, c.A_log, dla, BL, c.H, c.ddt,
+                                                                         c.dA_log);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace hm

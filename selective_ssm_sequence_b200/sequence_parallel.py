@@ -22,8 +22,6 @@ the default is the library itself (`LibOps`).
 """
 from __future__ import annotations
 
-from typing import Optional
-
 
 class LibOps:
     """The three compute steps, on CUDA tensors through libhm."""
@@ -56,7 +54,7 @@ class LibOps:
         a = hm.scan_args(None, seg["k"], seg["v"], None, W_q=seg.get("W_q"), W_k=seg.get("W_k"),
                          dt=seg.get("dt"), A_log=seg.get("A_log"), S_out=S, z_out=z, flags=flags,
                          b_q=seg.get("b_q"), b_k=seg.get("b_k"), w_head_stride=seg.get("w_head_stride", 0),
-                         log_decay_out=lam)
+                         log_decay_out=lam, rope_base=seg.get("rope_base", 0.0), pos0=seg.get("pos0", 0))
         ws = self._ws(a)
         hm.hm_scan_chunked_fwd(a)
         del ws
@@ -73,7 +71,8 @@ class LibOps:
         a = hm.scan_args(seg["q"], seg["k"], seg["v"], o, W_q=seg.get("W_q"), W_k=seg.get("W_k"),
                          dt=seg.get("dt"), A_log=seg.get("A_log"), S0=S0, z0=z0, S_out=S_out, z_out=z_out,
                          flags=flags, b_q=seg.get("b_q"), b_k=seg.get("b_k"),
-                         w_head_stride=seg.get("w_head_stride", 0))
+                         w_head_stride=seg.get("w_head_stride", 0), rope_base=seg.get("rope_base", 0.0),
+                         pos0=seg.get("pos0", 0))
         ws = self._ws(a)
         hm.hm_scan_chunked_fwd(a)
         del ws
@@ -91,8 +90,9 @@ def prefill_sequence_parallel(seg: dict, o, F: int, flags: int = 0, S0=None, z0=
 
     seg: this rank's consecutive token range, as tensors q, k [B, Ls, H, d],
     v [B, Ls, H, dv] and optionally W_q, W_k, dt [B, Ls, H], A_log, biases;
-    rank r holds tokens after those of ranks 0..r-1.  o [B, Ls, H, dv] gets
-    this segment's outputs.  S0, z0: the state before rank 0's tokens (only
+    with HM_FLAG_ROPE also "rope_base" and "pos0" (the position of this rank's
+    first token); rank r holds tokens after those of ranks 0..r-1.
+    o [B, Ls, H, dv] gets this segment's outputs.  S0, z0: the state before rank 0's tokens (only
     rank 0's arguments are used; NULL = zero).  S_out, z_out: this rank's end
     state, i.e. on the last rank the state after the whole sequence.
     F is the feature dimension (2p with Hedgehog weights, else d)."""
@@ -114,8 +114,8 @@ def prefill_sequence_parallel(seg: dict, o, F: int, flags: int = 0, S0=None, z0=
     parts = [ops.empty(n, k) for _ in range(world)]
     dist.all_gather(parts, mine, group=group)
     gathered = torch.cat(parts)
-    # the initial state lives on rank 0; the others learn of it only through
-    # this broadcast (a zero-length flag when there is none)
+    # the initial state lives on rank 0; the others learn whether there is one,
+    # and its value, through these broadcasts
     has0 = torch.tensor([1 if (rank == 0 and S0 is not None) else 0], dtype=torch.int32, device=k.device)
     dist.broadcast(has0, src=dist.get_global_rank(group, 0) if group is not None else 0, group=group)
     if int(has0.item()):

@@ -64,7 +64,9 @@ def _c_layout(struct, fields):
 
 @pytest.mark.parametrize("cname,pyname", [("hm_scan_args", "ScanArgs"),
                                           ("hm_decode_args", "DecodeArgs"),
-                                          ("hm_mixer_args", "MixerArgs")])
+                                          ("hm_mixer_args", "MixerArgs"),
+                                          ("hm_scan_bwd_args", "ScanBwdArgs"),
+                                          ("hm_combine_args", "CombineArgs")])
 def test_struct_layouts_match_the_header(hm, cname, pyname):
     cls = getattr(hm, pyname)
     fields = [f[0] for f in cls._fields_]
@@ -126,8 +128,11 @@ def test_validation_rejects_bad_calls_before_launch(hm):
 def test_variant_flags_are_validated_before_launch(hm):
     def call(a):
         return hm.lib.hm_scan_chunked_fwd(ctypes.byref(a), None)
-    assert call(_args(hm, flags=4)) == hm.HM_ERR_INVALID_ARG           # unknown bit
+    assert call(_args(hm, flags=8)) == hm.HM_ERR_INVALID_ARG           # unknown bit
     assert b"flag" in hm.lib.hm_last_error_detail()
+    assert call(_args(hm, flags=hm.HM_FLAG_ROPE)) == hm.HM_ERR_INVALID_ARG   # no rope_base
+    assert call(_args(hm, flags=hm.HM_FLAG_ROPE, rope_base=1e4, pos0=-1)) == hm.HM_ERR_INVALID_ARG
+    assert hm.hm_scan_workspace_size(_args(hm, flags=hm.HM_FLAG_ROPE, rope_base=1e4)) > 0
     assert call(_args(hm, flags=hm.HM_FLAG_DT_SCALED_INPUT, dt=None)) == hm.HM_ERR_INVALID_ARG
     assert call(_args(hm, flags=hm.HM_FLAG_PER_FEATURE_DECAY, dt=None)) == hm.HM_ERR_INVALID_ARG
     # valid flags size a workspace like the plain call (CUDA-core path for the per-feature decay)
@@ -138,5 +143,8 @@ def test_variant_flags_are_validated_before_launch(hm):
     d.q = d.k = d.v = d.o = d.S = d.z = 1 << 20
     d.flags = 8
     assert hm.lib.hm_step_decode(ctypes.byref(d), None) == hm.HM_ERR_INVALID_ARG
+    d.flags, d.rope_base = hm.HM_FLAG_ROPE, 1e4                             # needs positions
+    assert hm.lib.hm_step_decode(ctypes.byref(d), None) == hm.HM_ERR_INVALID_ARG
+    d.rope_base = 0.0
     d.flags = hm.HM_FLAG_DT_SCALED_INPUT                                    # needs dt
     assert hm.lib.hm_step_decode(ctypes.byref(d), None) == hm.HM_ERR_INVALID_ARG
