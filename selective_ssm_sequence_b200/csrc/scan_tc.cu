@@ -486,8 +486,6 @@ constexpr uint32_t kColSB = 256; // S^T bf16 pairs  [128 x 128]
 constexpr uint32_t kColO = 384;  // O^T fp32        [128 x 64 tokens]
 constexpr uint32_t kColP = 448;  // [phiK; phiQ] phiK^T fp32 [128 x 64]; lanes 64..127 = P
 
-constexpr int kZGroups = 8;      // token groups of the weighted key-feature sums (8 tokens)
-constexpr int kZTok = kC / kZGroups;
 constexpr int kHelpers = 160;    // threads of the five helper warps
 
 struct CAux {
@@ -499,8 +497,7 @@ struct CAux {
     float rden[2][kC];   // 1 / den
     float dint[2][kC];   // row sums of Pt: [0] columns 0..31, [1] columns 32..63
     float dotq[4][kC];   // phiq_i . z_prev over each quarter of the features
-    float z[kF];
-    alignas(16) float zred[kZGroups][kF];
+    alignas(16) float zb[2][kF];   // z after chunk c in zb[c & 1]; the start z in zb[1]
     float gam[2];
     float redd[4];
     // per stage: the phiQ blocks and the phiK + V blocks are loaded and
@@ -511,6 +508,8 @@ struct CAux {
     uint64_t den_ready[2], den_free[2];   // 1 / den of a stage written / read
     uint64_t pro_full[3];                 // start-state rounds landed (prologue staging)
     uint64_t dec_full[2], dec_free[2];    // decay vectors of a parity written / read
+    uint64_t zfull[2], zfree[2];          // z buffer of a parity written / read
+    int szero;           // gamma of the next state MMA's chunk is 0: that MMA overwrites S
     uint32_t tmem;
     int abort;
 };
@@ -563,17 +562,18 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
 // Warp roles (15 warps):
 //   0      TMA producer (phiQ, phiK, V of each chunk; two stages)
 //   1      MMA issuer
-//   2..9   compute group (256 threads): per chunk the decayed score tile Pt
-//          (three 32 x 32 quadrants: rows 0..31 need only columns 0..31),
-//          w (.) V, the scaled queries e^cum (.) phiQ with phiq . z_prev, the
-//          denominators, the weighted key-feature sums and z
+//   2, 3, 14, 5..9  compute group (256 threads): per chunk the decayed score
+//          tile Pt (three 32 x 32 quadrants: rows 0..31 need only columns
+//          0..31), w (.) V, the scaled queries e^cum (.) phiQ with
+//          phiq . z_prev, and the denominators
 //   10..13 outputs and state pass: o = O^T / den for the chunk, staged in the
 //          chunk's Pt buffer (dead once the PV product is complete) and written
 //          by TMA bulk stores; then S^T (fp32, TMEM) -> bf16 copy for the next
 //          readout and S^T <- gamma S^T before the next state MMA
-//   14     decay vectors, one chunk ahead of the compute group (prefix sums
+//   4      decay vectors, one chunk ahead of the compute group (prefix sums
 //          of log a, e^cum, e^(cum_last - cum), the below-diagonal column
-//          factors, gamma), two tokens per lane
+//          factors, gamma), two tokens per lane; then the weighted key-feature
+//          sums and z of the chunk before, eight features per lane
 // Per chunk the MMA issuer runs: scores of the next chunk, then the readout
 // O^T = S^T (e^cum phiQ)^T, O^T += V^T Pt^T (hi and lo), and the state
 // update S^T += (w V)^T phiK.
@@ -623,7 +623,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_init(&X->emptykv[s], 2);
         }
         mbar_init(&X->p_full, 1);
-        mbar_init(&X->p_consumed, 1);   // the compute group has loaded P
+        mbar_init(&X->p_consumed, 3);   // the three score-quadrant warps have loaded P
         mbar_init(&X->epib_done, 1);
         mbar_init(&X->o_full, 1);
         mbar_init(&X->o_empty, 4);      // one arrival per output / state-pass warp
@@ -637,6 +637,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         for (int s = 0; s < 2; ++s) {
             mbar_init(&X->dec_full[s], 1);
             mbar_init(&X->dec_free[s], 1);
+            mbar_init(&X->zfull[s], 1);
+            mbar_init(&X->zfree[s], 1);
         }
         X->abort = 0;
         mbar_fence_init();
@@ -735,25 +737,24 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     mma_ss(tmem + kColO, va, desc_k_sw128(sP(s) + kC * 128 + k * 32), idOa, 1u);
                 }
                 mma_commit(&X->o_full);
+                // a chunk whose decay gamma underflowed to 0 forgets the state:
+                // its update overwrites S (the state pass then skipped S <- 0 S)
+                const uint32_t acc0 = X->szero ? 0u : 1u;
 #pragma unroll
                 for (int k = 0; k < kC / 16; ++k)
                     mma_ss(tmem + kColS, desc_mn_sw128(sVt + k * 2048, kBlk, 1024),
-                           desc_mn_sw128(sK(s) + k * 2048, kQKBlk, 1024), idS, 1u);
+                           desc_mn_sw128(sK(s) + k * 2048, kQKBlk, 1024), idS, k == 0 ? acc0 : 1u);
                 mma_commit(&X->s_full);
                 mma_commit(&X->emptykv[s]);
                 mma_commit(&X->emptyq[s]);
             }
         }
-    } else if (warp < 10) {
+    } else if ((warp >= 2 && warp < 10 && warp != 4) || warp == 14) {
         // ------------------------------------------------------------ compute group
-        const int gt = threadIdx.x - 64;   // 0..255
+        // warps 2, 3, 14, 5, 6, 7, 8, 9 (warp 14 stands in for warp 4, which
+        // runs the decay vectors and z on the less busy SM sub-partition 0)
+        const int gt = (warp == 14 ? 2 : warp - 2) * 32 + lane;   // 0..255
         const int q = warp & 3;            // TMEM lane quarter of this warp
-        {
-            const float *zi = nullptr;
-            if (seg == 0) zi = a.z0 ? a.z0 + bh * kF : nullptr;
-            else zi = a.z_start + (bh * g.G + seg) * kF;
-            X->z[gt] = zi ? zi[gt] : 0.f;
-        }
         // every exit from this loop is taken by the whole group (after a
         // barrier-AND), so no thread is left waiting at a named barrier
         bool ok = named_sync_and(1, 256, true);
@@ -769,29 +770,28 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             // every thread is past chunk it - 1, the last reader of the other
             // parity's decay vectors
             if (gt == 0 && it > 0) mbar_arrive(&X->dec_free[(it - 1) & 1]);
-            // (2) once the chunk's scores are in TMEM
-            bool okw = mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7) &&
-                       mbar_wait(&X->fullkv[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8) &&
-                       mbar_wait(&X->fullq[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 17);
-            okw = __all_sync(0xffffffffu, okw);
-            tc_fence_after();
+            // (2) the chunk's stage is loaded and its score MMA has completed:
+            // every thread waits for both -- the score MMA reads phiQ of the
+            // stage, which step (3) scales in place -- and then meets the others
+            // at barrier 4, so that all waiters of this p_full phase are past it
+            // before p_consumed lets the next phase begin.  Score-quadrant warps
+            // (P rows 0..31 in TMEM lanes 64..95, rows 32..63 in lanes 96..127):
+            // warp 2: rows 0..31 x columns 0..31 (and the zeros of columns
+            // 32..63); warp 3: rows 32..63 x columns 0..31 (all below the
+            // diagonal); warp 7: rows 32..63 x columns 32..63.  Each reads its
+            // quadrant from TMEM 8 columns at a time as it goes and then
+            // arrives on p_consumed (count 3), after which the next chunk's
+            // scores may overwrite it.
             const bool pwarp = warp == 2 || warp == 3 || warp == 7;
-            // score-quadrant warps (P rows 0..31 in TMEM lanes 64..95, rows
-            // 32..63 in lanes 96..127): warp 2: rows 0..31 x columns 0..31 (and
-            // the zeros of columns 32..63); warp 3: rows 32..63 x columns 0..31
-            // (all below the diagonal); warp 7: rows 32..63 x columns 32..63
+            bool okw = mbar_wait(&X->fullkv[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8) &&
+                       mbar_wait(&X->fullq[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 17) &&
+                       mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7);
+            okw = __all_sync(0xffffffffu, okw);
+            named_sync(4, 256);
+            tc_fence_after();
             const int i = 32 * (q - 2) + lane;
             const int jc = warp == 7 ? 32 : 0;
-            uint32_t pr[32];
-            if (pwarp && okw) {
-                tmem_ld32(tmem + kColP + jc + ((uint32_t)(32 * q) << 16), pr);
-                tmem_wait_ld();
-            }
-            // every compute thread is past its wait on this chunk's scores and P
-            // is in registers: the next chunk's scores may overwrite it
-            tc_fence_before();
-            named_sync(4, 256);
-            if (gt == 0) mbar_arrive(&X->p_consumed);
+            const uint32_t ptm = tmem + kColP + jc + ((uint32_t)(32 * q) << 16);
             if (pwarp) {
                 // (The 8-column block loops below stay rolled: the kernel's roles
                 // together run more code per chunk than the instruction cache
@@ -812,6 +812,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t pr[8];
+                        tmem_ld8(ptm + 8 * c4, pr);
                         const float ai = ex2_approx(ci - X->cum[s][8 * c4 + 7]);
                         const float2 a2 = make_float2(ai, ai);
                         const float4 ba = *reinterpret_cast<const float4 *>(&X->bq[s][8 * c4]);
@@ -821,10 +823,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         uint4 hi, lo;
                         uint32_t *pk = reinterpret_cast<uint32_t *>(&hi);
                         uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+                        tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int jl = c4 * 8 + 2 * e;
-                            const float2 ev = mul2(make_float2(__uint_as_float(pr[jl]), __uint_as_float(pr[jl + 1])),
+                            const float2 ev = mul2(make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])),
                                                    mul2(a2, bv[e]));
                             pk[e] = pack_bf16x2(ev.x, ev.y);
                             const float2 r = sub2(ev, unpack_bf16x2(pk[e]));
@@ -835,7 +837,6 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, c4)) = lo;
                     }
                     X->dint[0][i] = rs2.x + rs2.y;
-                    tc_fence_before();
                 } else if (okw) {
                     const float ci = X->cum[s][i];
                     const float2 ci2 = make_float2(ci, ci);
@@ -844,6 +845,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t pr[8];
+                        tmem_ld8(ptm + 8 * c4, pr);
                         uint4 hi, lo;
                         uint32_t *pk = reinterpret_cast<uint32_t *>(&hi);
                         uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
@@ -851,12 +854,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         const float4 cb = *reinterpret_cast<const float4 *>(cj + c4 * 8 + 4);
                         const float2 cv[4] = {make_float2(ca.x, ca.y), make_float2(ca.z, ca.w),
                                               make_float2(cb.x, cb.y), make_float2(cb.z, cb.w)};
+                        tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int jl = c4 * 8 + 2 * e;
-                            const int j = jc + jl;
+                            const int j = jc + c4 * 8 + 2 * e;
                             const float2 d = sub2(ci2, cv[e]);
-                            float2 ev = mul2(make_float2(__uint_as_float(pr[jl]), __uint_as_float(pr[jl + 1])),
+                            float2 ev = mul2(make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])),
                                              make_float2(ex2_approx(d.x), ex2_approx(d.y)));
                             if (masked && j > i) ev.x = 0.f;
                             if (masked && j + 1 > i) ev.y = 0.f;
@@ -876,11 +879,14 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         }
                     }
                     X->dint[jc ? 1 : 0][i] = rs2.x + rs2.y;
-                    tc_fence_before();
                 }
+                // P has been read: the next chunk's scores may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&X->p_consumed);
             } else {
-                // helpers (warps 4, 5, 6, 8, 9)
-                const int hx = (warp < 7 ? warp - 4 : warp - 5) * 32 + lane;   // 0..159
+                // helpers (warps 14, 5, 6, 8, 9)
+                const int hx = (warp == 14 ? 0 : (warp < 7 ? warp - 4 : warp - 5)) * 32 + lane;   // 0..159
                 const float *__restrict__ wv = X->w[s];
                 // w (.) V into its own tile, once the previous chunk's state MMA
                 // has read that tile
@@ -894,26 +900,27 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         const uint32_t off = (uint32_t)((ci >> 3) * kBlk) + sw128_off(j, ci & 7);
                         uint4 vv = *reinterpret_cast<const uint4 *>(vsrc + off);
                         const float wj = wv[j];
-                        const float2 w2 = make_float2(wj, wj);
+                        const uint32_t w2 = pack_bf16x2(wj, wj);
                         uint32_t *pv = reinterpret_cast<uint32_t *>(&vv);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 x = mul2(unpack_bf16x2(pv[e]), w2);
-                            pv[e] = pack_bf16x2(x.x, x.y);
-                        }
+                        for (int e = 0; e < 4; ++e) pv[e] = mul_bf16x2(pv[e], w2);
                         *reinterpret_cast<uint4 *>(gVt + off) = vv;
                     }
                 }
             }
             // (3) every thread: the query row scaled by e^cum_i, in place, and
             // phiq_i . z_prev over one quarter of the features (on the unscaled
-            // bf16 values; the scale is applied to the sum)
+            // bf16 values; the scale is applied to the sum).  z_prev = z after
+            // chunk it - 1 (the start z for it = 0), from the z warp: buffer
+            // (it - 1) & 1, whose (it >> 1)-th write it is.
+            okw = __all_sync(0xffffffffu, okw && mbar_wait(&X->zfull[(it - 1) & 1], (it >> 1) & 1, abort_flag,
+                                                               err, KID_SCAN_TC_OUT, 24));
             if (okw) {
                 const int i = gt & 63, qf = gt >> 6;
                 const float qsi = X->qs[s][i];
-                const float2 q2 = make_float2(qsi, qsi);
+                const uint32_t q2 = pack_bf16x2(qsi, qsi);
                 uint8_t *__restrict__ qb = gQ(s) + qf * kQKBlk;
-                const float *__restrict__ zq = X->z + qf * 64;
+                const float *__restrict__ zq = X->zb[(it - 1) & 1] + qf * 64;
                 float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll 1
                 for (int k0 = 0; k0 < 8; k0 += 4) {
@@ -929,10 +936,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                                               make_float2(zb.x, zb.y), make_float2(zb.z, zb.w)};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const float2 x = unpack_bf16x2(pv[e]);
-                            d2 = fma2(x, zz[e], d2);
-                            const float2 y = mul2(x, q2);
-                            pv[e] = pack_bf16x2(y.x, y.y);
+                            d2 = fma2(unpack_bf16x2(pv[e]), zz[e], d2);
+                            pv[e] = mul_bf16x2(pv[e], q2);
                         }
                     }
 #pragma unroll
@@ -943,7 +948,10 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             fence_proxy_async_smem();
             ok = named_sync_and(1, 256, okw);
             if (!ok) break;
-            if (gt == 0) mbar_arrive(&X->epib_done);
+            if (gt == 0) {
+                mbar_arrive(&X->epib_done);
+                mbar_arrive(&X->zfree[(it - 1) & 1]);   // z_prev has been read
+            }
             // (4) denominators (once the outputs of chunk it - 2 have read this
             // stage's 1 / den) and z; the chunk's MMAs run meanwhile
             if (gt < kC) {
@@ -951,57 +959,42 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 const bool okd =
                     mbar_wait(&X->den_free[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 14);
                 const float dq = (X->dotq[0][i] + X->dotq[1][i]) + (X->dotq[2][i] + X->dotq[3][i]);
-                const float den = X->dint[0][i] + (i >= 32 ? X->dint[1][i] : 0.f) + X->qs[s][i] * dq;
+                // the inter-chunk term with the query scale as the readout used it
+                // (rounded to bf16), so that numerator and denominator agree
+                const float qsr = __bfloat162float(__float2bfloat16_rn(X->qs[s][i]));
+                const float den = X->dint[0][i] + (i >= 32 ? X->dint[1][i] : 0.f) + qsr * dq;
                 X->rden[s][i] = 1.f / den;
                 named_sync(3, 64);
                 if (gt == 0) mbar_arrive(&X->den_ready[s]);
                 if (!okd) ok = false;
             }
-            // (5) weighted key-feature sums sum_j w_j phik_j (needed only for the
-            // next chunk's denominators, so after the MMAs were released):
-            // thread = one 16-byte chunk (8 features) over a group of 8 tokens
-            {
-                const int cc = gt & 31, tg = gt >> 5;
-                const uint8_t *__restrict__ base = gK(s) + (cc >> 3) * kQKBlk;
-                const float *__restrict__ wv = X->w[s] + tg * kZTok;
-                uint4 kv[kZTok];
-#pragma unroll
-                for (int jj = 0; jj < kZTok; ++jj)
-                    kv[jj] = *reinterpret_cast<const uint4 *>(base + sw128_off(tg * kZTok + jj, cc & 7));
-                float2 za[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) za[e] = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int jj = 0; jj < kZTok; ++jj) {
-                    const float2 w2 = make_float2(wv[jj], wv[jj]);
-                    const uint32_t *pv = reinterpret_cast<const uint32_t *>(&kv[jj]);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) za[e] = fma2(unpack_bf16x2(pv[e]), w2, za[e]);
-                }
-                float *zr = &X->zred[tg][cc * 8];
-                *reinterpret_cast<float4 *>(zr) = make_float4(za[0].x, za[0].y, za[1].x, za[1].y);
-                *reinterpret_cast<float4 *>(zr + 4) = make_float4(za[2].x, za[2].y, za[3].x, za[3].y);
-            }
-            named_sync(1, 256);
-            if (gt == 0) mbar_arrive(&X->emptykv[s]);   // phiK and V of the stage have been read
-            // (6) z <- gamma z + sum_j w_j phik_j
-            {
-                float acc = 0.f;
-#pragma unroll
-                for (int tg = 0; tg < kZGroups; ++tg) acc += X->zred[tg][gt];
-                X->z[gt] = fmaf(X->gam[s], X->z[gt], acc);
-            }
         }
-    } else if (warp == 14) {
-        // ------------------------------------------------------------ decay vectors
-        // lane: tokens 2 lane and 2 lane + 1 of the chunk; dt two chunks ahead
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ decay vectors and z
+        // Iteration c: the decay vectors of chunk c (one chunk ahead of the
+        // compute group), then z after chunk c - 1:
+        //   z_{c-1} = gamma_{c-1} z_{c-2} + sum_j w_j phik_j  (over chunk c - 1)
+        // into zb[(c - 1) & 1] for the compute group's denominators of chunk c.
+        // Lane: tokens 2 lane and 2 lane + 1 for the decay vectors (dt two
+        // chunks ahead); features 8 lane .. 8 lane + 7 for z.
+        {
+            // the start z, as the first write of buffer 1
+            const float *zi = nullptr;
+            if (seg == 0) zi = a.z0 ? a.z0 + bh * kF : nullptr;
+            else zi = a.z_start + (bh * g.G + seg) * kF;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) X->zb[1][8 * lane + e] = zi ? zi[8 * lane + e] : 0.f;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->zfull[1]);
+        }
         float da[2], db[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             da[i] = i < nch ? token_dt(a, b, h, (int64_t)(c_begin + i) * kC, 2 * lane) : -INFINITY;
             db[i] = i < nch ? token_dt(a, b, h, (int64_t)(c_begin + i) * kC, 2 * lane + 1) : -INFINITY;
         }
-        for (int c = 0; c < nch; ++c) {
+        for (int c = 0; c <= nch; ++c) {
+          if (c < nch) {
             const int sc = c & 1;
             const float l0 = hm_log_decay(da[0], alog) * kLog2e, l1 = hm_log_decay(db[0], alog) * kLog2e;
             // step-scaled input: log2 of softplus(dt) of the two tokens, added
@@ -1037,6 +1030,49 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (lane == 0) X->gam[sc] = ex2_approx(total);
             __syncwarp();
             if (lane == 0) mbar_arrive(&X->dec_full[sc]);
+          }
+          if (c >= 1) {
+            // z after chunk c - 1 (stage s1 holds its phiK; its weights and
+            // gamma are this warp's own decay vectors of parity s1)
+            const int s1 = (c - 1) & 1;
+            bool okz = mbar_wait(&X->fullkv[s1], ((c - 1) >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 25);
+            if (!__all_sync(0xffffffffu, okz)) break;
+            const uint8_t *__restrict__ base = gK(s1) + (lane >> 3) * kQKBlk;
+            const float *__restrict__ wv = X->w[s1];
+            float2 za[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) za[e] = make_float2(0.f, 0.f);
+#pragma unroll 1
+            for (int j0 = 0; j0 < kC; j0 += 8) {
+                uint4 kv[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    kv[jj] = *reinterpret_cast<const uint4 *>(base + sw128_off(j0 + jj, lane & 7));
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float wj = wv[j0 + jj];
+                    const float2 w2 = make_float2(wj, wj);
+                    const uint32_t *pv = reinterpret_cast<const uint32_t *>(&kv[jj]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) za[e] = fma2(unpack_bf16x2(pv[e]), w2, za[e]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->emptykv[s1]);   // this warp's reads of the stage are done
+            // the buffer of z_{c-1} was last read by the compute group in chunk c - 2
+            okz = c < 2 || mbar_wait(&X->zfree[s1], ((c - 2) >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 26);
+            if (!__all_sync(0xffffffffu, okz)) break;
+            const float gm = X->gam[s1];
+            const float *__restrict__ zp = X->zb[(c - 2) & 1] + 8 * lane;
+            float *__restrict__ zn = X->zb[s1] + 8 * lane;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                zn[2 * e] = fmaf(gm, zp[2 * e], za[e].x);
+                zn[2 * e + 1] = fmaf(gm, zp[2 * e + 1], za[e].y);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->zfull[s1]);
+          }
         }
     } else {
         // ------------------------------------------------------------ state pass
@@ -1099,8 +1135,9 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 }
             }
             tmem_wait_st();
+            if (td == 0) X->szero = gam0 == 0.f ? 1 : 0;
             tc_fence_before();
-            __syncwarp();
+            named_sync(2, 128);   // szero is written before any warp's arrival
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
         bool ok = true;
@@ -1179,8 +1216,11 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             ok = named_sync_and(2, 128, okc && mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11));
             if (!ok) break;
             tc_fence_after();
-            // 32-column blocks, the next block's load in flight while this one
-            // is converted and stored
+            // 32-column blocks: S^T -> its bf16 copy for the next readout, and
+            // S^T <- gamma S^T before the next state MMA.  gn is the same in
+            // every thread; when it is 0 the next state MMA overwrites S instead
+            // (szero), so S is only converted.
+            const bool gz = gn == 0.f;
             const float2 g2 = make_float2(gn, gn);
 #pragma unroll 1
             for (int blk = 0; blk < kF / 32; ++blk) {
@@ -1188,19 +1228,23 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 tmem_ld32(tmem + kColS + 32 * blk + lanebase, cur);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float2 x = make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1]));
-                    pk[j] = pack_bf16x2(x.x, x.y);
-                    const float2 y = mul2(x, g2);
-                    cur[2 * j] = __float_as_uint(y.x);
-                    cur[2 * j + 1] = __float_as_uint(y.y);
-                }
+                for (int j = 0; j < 16; ++j)
+                    pk[j] = pack_bf16x2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1]));
                 tmem_st16(tmem + kColSB + 16 * blk + lanebase, pk);
-                tmem_st32(tmem + kColS + 32 * blk + lanebase, cur);
+                if (!gz) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float2 y = mul2(make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])), g2);
+                        cur[2 * j] = __float_as_uint(y.x);
+                        cur[2 * j + 1] = __float_as_uint(y.y);
+                    }
+                    tmem_st32(tmem + kColS + 32 * blk + lanebase, cur);
+                }
             }
             tmem_wait_st();
+            if (td == 0) X->szero = gz ? 1 : 0;
             tc_fence_before();
-            __syncwarp();
+            named_sync(2, 128);   // szero is written before any warp's arrival
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
         // the MMAs of the last chunk must be complete before TMEM is released,
