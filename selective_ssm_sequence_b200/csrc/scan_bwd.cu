@@ -51,6 +51,25 @@ struct BwdArgs {
     float *dS0, *dz0;        // nullable
 };
 
+// v[m] is this lane's contribution to row m (m = 0..31); afterwards v[0] of
+// lane l is the sum over the warp of row l.  Recursive halving: at step `off`
+// each lane keeps the half of its rows selected by its lane bit `off` and
+// adds the partner's copy of that half (31 shuffles instead of 32 reductions
+// of 5).
+__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int j = 0; j < off; ++j) {
+            const float send = upper ? v[j] : v[j + off];
+            const float keep = upper ? v[j + off] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return v[0];
+}
+
 template <int MODE, typename TIO>
 __global__ void __launch_bounds__(32 * kW)
 bwd_pass_kernel(BwdArgs a) {
@@ -67,6 +86,7 @@ bwd_pass_kernel(BwdArgs a) {
     float *sdd = sden + kTB;               // [kTB]       dd_t
     float *red = sdd + kTB;                // [kTB][kW][32]
     float *rden = red + kTB * kW * 32;     // [kTB][kW]
+    float *sout = rden + kTB * kW;         // [kTB][F]: the slice's shares of dphiq / dphik
 
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t bh = blockIdx.y;
@@ -143,19 +163,26 @@ bwd_pass_kernel(BwdArgs a) {
                     red[(t * kW + w) * 32 + lane] = num;
                     if (lane == 0) rden[t * kW + w] = den;
                 } else {
-                    // the slice's share of dphiq_t[f] = sum_c S_t[f, c] dn_t[c] (+ z_t[f] dd_t)
+                    // the slice's share of dphiq_t[f] = sum_c S_t[f, c] dn_t[c] (+ z_t[f] dd_t),
+                    // row f = w + 8 m summed over the warp's lanes (columns)
                     const float dn = sg[t * 32 + lane] / sden[t];
-                    const int64_t r = rowi(t0 + t);
-                    float *dq = a.dq_part + ((int64_t)slice * a.B * L * a.H + r) * F;
+                    float x[kMaxRows];
 #pragma unroll
-                    for (int m = 0; m < kMaxRows; ++m) {
-                        const int f = w + kW * m;
-                        if (f < F) {
-                            float x = warp_sum(S[m] * dn);
-                            if (lane == (m & 31)) dq[f] = x + (slice == 0 ? z[m] * sdd[t] : 0.f);
-                        }
-                    }
+                    for (int m = 0; m < kMaxRows; ++m) x[m] = S[m] * dn;
+                    const float tot = warp_reduce_scatter32(x, lane);
+                    // lane l now holds row w + 8 l; z of that row lives in lane l's z[l]
+                    float zl = 0.f;
+#pragma unroll
+                    for (int m = 0; m < kMaxRows; ++m) zl = lane == m ? z[m] : zl;
+                    const int f = w + kW * lane;
+                    if (f < F) sout[t * F + f] = tot + (slice == 0 ? zl * sdd[t] : 0.f);
                 }
+            }
+            if (MODE == 1) {
+                __syncthreads();
+                float *dq = a.dq_part + (int64_t)slice * a.B * L * a.H * F;
+                for (int i = threadIdx.x; i < nt * F; i += blockDim.x)
+                    dq[rowi(t0 + i / F) * F + (i % F)] = sout[i];
             }
             if (MODE == 0) {
                 __syncthreads();
@@ -181,21 +208,27 @@ bwd_pass_kernel(BwdArgs a) {
                 const float dn = sg[t * 32 + lane] / sden[t];
                 const float dd = sdd[t];
                 const float vv = sv[t * 32 + lane];
-                const int64_t r = rowi(t0 + t);
-                float *dk = a.dk_part + ((int64_t)slice * a.B * L * a.H + r) * F;
                 float dvp = 0.f;
+                float x[kMaxRows];
 #pragma unroll
                 for (int m = 0; m < kMaxRows; ++m) {
                     const int f = w + kW * m;
+                    x[m] = 0.f;
                     if (f < F) {
                         const float qf = sq[t * F + f], kf = sk[t * F + f];
                         S[m] = fmaf(a1, S[m], qf * dn);
                         z[m] = fmaf(a1, z[m], qf * dd);
                         dvp = fmaf(S[m], kf, dvp);
-                        const float x = warp_sum(S[m] * vv);
-                        if (lane == (m & 31)) dk[f] = x + (slice == 0 ? z[m] : 0.f);
+                        x[m] = S[m] * vv;
                     }
                 }
+                // the slice's share of dphik_t[f] = sum_c G_t[f, c] v_t[c] (+ g_t[f])
+                const float tot = warp_reduce_scatter32(x, lane);
+                float zl = 0.f;
+#pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) zl = lane == m ? z[m] : zl;
+                const int fl = w + kW * lane;
+                if (fl < F) sout[t * F + fl] = tot + (slice == 0 ? zl : 0.f);
                 red[(t * kW + w) * 32 + lane] = dvp;
             }
             __syncthreads();
@@ -205,6 +238,11 @@ bwd_pass_kernel(BwdArgs a) {
                 for (int ww = 0; ww < kW; ++ww) acc += red[(t * kW + ww) * 32 + c];
                 const int cc = slice * 32 + c;
                 if (cc < dv) a.dv_out[rowi(t0 + t) * dv + cc] = acc;
+            }
+            {
+                float *dk = a.dk_part + (int64_t)slice * a.B * L * a.H * F;
+                for (int i = threadIdx.x; i < nt * F; i += blockDim.x)
+                    dk[rowi(t0 + i / F) * F + (i % F)] = sout[i];
             }
             if (t0 == 0) {
                 // dS0 = a_1 G_1, dz0 = a_1 g_1 (a_1 = the first token's decay)
@@ -378,7 +416,7 @@ decay_bwd_kernel(const float *__restrict__ dt, const float *__restrict__ A_log, 
 template <typename TIO>
 cudaError_t run_passes(const BwdArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)a.ns, (unsigned)(a.B * a.H));
-    const size_t smem = sizeof(float) * (size_t)(2 * kTB * a.F + 2 * kTB * 32 + 4 * kTB + kTB * kW * 32 + kTB * kW);
+    const size_t smem = sizeof(float) * (size_t)(3 * kTB * a.F + 2 * kTB * 32 + 4 * kTB + kTB * kW * 32 + kTB * kW);
     cudaError_t e;
     auto k0 = bwd_pass_kernel<0, TIO>;
     auto k1 = bwd_pass_kernel<1, TIO>;
