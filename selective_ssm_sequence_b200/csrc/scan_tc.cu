@@ -559,25 +559,30 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
     return tot;
 }
 
-// Warp roles (15 warps):
+// Warp roles (19 warps):
 //   0      TMA producer (phiQ, phiK, V of each chunk; two stages)
 //   1      MMA issuer
 //   2, 3, 14, 5..9  compute group (256 threads): per chunk the decayed score
 //          tile Pt (three 32 x 32 quadrants: rows 0..31 need only columns
 //          0..31), w (.) V, the scaled queries e^cum (.) phiQ with
 //          phiq . z_prev, and the denominators
-//   10..13 outputs and state pass: o = O^T / den for the chunk, staged in the
-//          chunk's Pt buffer (dead once the PV product is complete) and written
-//          by TMA bulk stores; then S^T (fp32, TMEM) -> bf16 copy for the next
-//          readout and S^T <- gamma S^T before the next state MMA
+//   10..13 outputs: o = O^T / den for the chunk, staged in the chunk's Pt
+//          buffer (dead once the PV product is complete) and written by TMA
+//          bulk stores
+//   15..18 state pass: S^T (fp32, TMEM) -> bf16 copy for the next readout and
+//          S^T <- gamma S^T before the next state MMA.  The outputs of a chunk
+//          and its state pass run at the same time on separate warps, so the
+//          next readout waits only for the state pass.
 //   4      decay vectors, one chunk ahead of the compute group (prefix sums
 //          of log a, e^cum, e^(cum_last - cum), the below-diagonal column
 //          factors, gamma), two tokens per lane; then the weighted key-feature
 //          sums and z of the chunk before, eight features per lane
+// The output and state-pass roles each take four consecutive warps, so that
+// every TMEM lane quarter is read by one warp of each.
 // Per chunk the MMA issuer runs: scores of the next chunk, then the readout
 // O^T = S^T (e^cum phiQ)^T, O^T += V^T Pt^T (hi and lo), and the state
 // update S^T += (w V)^T phiK.
-constexpr int kCThreads = 480;
+constexpr int kCThreads = 608;
 
 __global__ void __launch_bounds__(kCThreads, 1)
 scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -626,9 +631,9 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         mbar_init(&X->p_consumed, 3);   // the three score-quadrant warps have loaded P
         mbar_init(&X->epib_done, 1);
         mbar_init(&X->o_full, 1);
-        mbar_init(&X->o_empty, 4);      // one arrival per output / state-pass warp
+        mbar_init(&X->o_empty, 4);      // one arrival per output warp
         mbar_init(&X->s_full, 1);
-        mbar_init(&X->sbf_ready, 4);
+        mbar_init(&X->sbf_ready, 4);     // one arrival per state-pass warp
         for (int s = 0; s < 2; ++s) {
             mbar_init(&X->den_ready[s], 1);
             mbar_init(&X->den_free[s], 4);
@@ -1074,81 +1079,15 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (lane == 0) mbar_arrive(&X->zfull[s1]);
           }
         }
-    } else {
-        // ------------------------------------------------------------ state pass
+    } else if (warp < 14) {
+        // ------------------------------------------------------------ outputs
         const int td = threadIdx.x - 320;
         const int q = warp & 3;
         const int ch = 32 * q + lane;
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
-        // prologue: start state -> bf16 copy (for the first readout) and fp32 x gamma_0
-        float dt_next = token_dt(a, b, h, (int64_t)c_begin * kC, td);
-        {
-            const float gam0 = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 2));
-            if (nch > 1) dt_next = token_dt(a, b, h, (int64_t)(c_begin + 1) * kC, td);
-            if (seg > 0) {
-                // segment start state [F][dv] (fp32, in L2): rounds of 32 feature rows
-                // x the CTA's 128 channels (16 KB) land by TMA in three rotating
-                // buffers (the Pt and w V tiles, unused until the first chunk)
-                const int row0 = (int)((bh * g.G + seg) * kF);
-                uint8_t *const pbuf = gP(0);
-                if (td == 0)
-                    for (int r = 0; r < 3; ++r) {
-                        mbar_arrive_expect_tx(&X->pro_full[r], 32 * kN * 4);
-                        tma_load_2d(pbuf + r * 32 * kN * 4, &tms, &X->pro_full[r], dv0, row0 + 32 * r);
-                    }
-#pragma unroll 1
-                for (int r = 0; r < kF / 32; ++r) {
-                    mbar_wait(&X->pro_full[r % 3], (r / 3) & 1, abort_flag, err, KID_SCAN_TC_OUT, 22);
-                    const float *buf = reinterpret_cast<const float *>(pbuf + (r % 3) * 32 * kN * 4) + ch;
-                    uint32_t v[32], pk[16];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(buf[j * kN]);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-                    tmem_st16(tmem + kColSB + 16 * r + lanebase, pk);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
-                    tmem_st32(tmem + kColS + 32 * r + lanebase, v);
-                    named_sync(2, 128);   // every thread has read this buffer
-                    if (td == 0 && r + 3 < kF / 32) {
-                        mbar_arrive_expect_tx(&X->pro_full[r % 3], 32 * kN * 4);
-                        tma_load_2d(pbuf + (r % 3) * 32 * kN * 4, &tms, &X->pro_full[r % 3], dv0, row0 + 32 * (r + 3));
-                    }
-                }
-            } else {
-                const float *src = a.S0 ? a.S0 + bh * (int64_t)kF * g.dv : nullptr;
-                for (int c0 = 0; c0 < kF; c0 += 32) {
-                    uint32_t v[32], pk[16];
-                    if (src) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(src[(int64_t)(c0 + j) * g.dv + dv0 + ch]);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0u;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-                    tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
-                    tmem_st32(tmem + kColS + c0 + lanebase, v);
-                }
-            }
-            tmem_wait_st();
-            if (td == 0) X->szero = gam0 == 0.f ? 1 : 0;
-            tc_fence_before();
-            named_sync(2, 128);   // szero is written before any warp's arrival
-            if (lane == 0) mbar_arrive(&X->sbf_ready);
-        }
         bool ok = true;
         for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
-            const bool more = it + 1 < nch;
-            float gn = 0.f;
-            if (more) {
-                gn = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 2));
-                if (it + 2 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + it + 2) * kC, td);
-            }
             // outputs of the chunk: o = O^T / den (lane = value channel, column = token)
             bool okc = ok && mbar_wait(&X->o_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 9) &&
                        mbar_wait(&X->den_ready[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 10);
@@ -1209,11 +1148,82 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (a.o_f32 && th == 0) named_sync(2, 128);   // round 0 has been read out
             }
             if (td == 0) mbar_arrive(&X->stg_free[s]);   // the Pt buffer may be rewritten
-            if (!more) {
-                ok = ok && okc;
-                break;
+            ok = ok && okc;
+            if (!ok) break;
+        }
+        // the output stores must have completed before the CTA's shared memory goes away
+        if (td == 0) bulk_wait_all();
+    } else {
+        // ------------------------------------------------------------ state pass
+        const int td = threadIdx.x - 480;
+        const int q = warp & 3;
+        const int ch = 32 * q + lane;
+        const uint32_t lanebase = (uint32_t)(32 * q) << 16;
+        // prologue: start state -> bf16 copy (for the first readout) and fp32 x gamma_0
+        float dt_next = token_dt(a, b, h, (int64_t)c_begin * kC, td);
+        {
+            const float gam0 = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 5));
+            if (nch > 1) dt_next = token_dt(a, b, h, (int64_t)(c_begin + 1) * kC, td);
+            if (seg > 0) {
+                // segment start state [F][dv] (fp32, in L2): rounds of 32 feature rows
+                // x the CTA's 128 channels (16 KB) land by TMA in three rotating
+                // buffers (the Pt and w V tiles, unused until the first chunk)
+                const int row0 = (int)((bh * g.G + seg) * kF);
+                uint8_t *const pbuf = gP(0);
+                if (td == 0)
+                    for (int r = 0; r < 3; ++r) {
+                        mbar_arrive_expect_tx(&X->pro_full[r], 32 * kN * 4);
+                        tma_load_2d(pbuf + r * 32 * kN * 4, &tms, &X->pro_full[r], dv0, row0 + 32 * r);
+                    }
+#pragma unroll 1
+                for (int r = 0; r < kF / 32; ++r) {
+                    mbar_wait(&X->pro_full[r % 3], (r / 3) & 1, abort_flag, err, KID_SCAN_TC_OUT, 22);
+                    const float *buf = reinterpret_cast<const float *>(pbuf + (r % 3) * 32 * kN * 4) + ch;
+                    uint32_t v[32], pk[16];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(buf[j * kN]);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                    tmem_st16(tmem + kColSB + 16 * r + lanebase, pk);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
+                    tmem_st32(tmem + kColS + 32 * r + lanebase, v);
+                    named_sync(5, 128);   // every thread has read this buffer
+                    if (td == 0 && r + 3 < kF / 32) {
+                        mbar_arrive_expect_tx(&X->pro_full[r % 3], 32 * kN * 4);
+                        tma_load_2d(pbuf + (r % 3) * 32 * kN * 4, &tms, &X->pro_full[r % 3], dv0, row0 + 32 * (r + 3));
+                    }
+                }
+            } else {
+                const float *src = a.S0 ? a.S0 + bh * (int64_t)kF * g.dv : nullptr;
+                for (int c0 = 0; c0 < kF; c0 += 32) {
+                    uint32_t v[32], pk[16];
+                    if (src) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(src[(int64_t)(c0 + j) * g.dv + dv0 + ch]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = 0u;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                    tmem_st16(tmem + kColSB + c0 / 2 + lanebase, pk);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * gam0);
+                    tmem_st32(tmem + kColS + c0 + lanebase, v);
+                }
             }
-            ok = named_sync_and(2, 128, okc && mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11));
+            tmem_wait_st();
+            if (td == 0) X->szero = gam0 == 0.f ? 1 : 0;
+            tc_fence_before();
+            named_sync(5, 128);   // szero is written before any warp's arrival
+            if (lane == 0) mbar_arrive(&X->sbf_ready);
+        }
+        bool ok = true;
+        for (int it = 0; it + 1 < nch; ++it) {
+            const float gn = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 5));
+            if (it + 2 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + it + 2) * kC, td);
+            ok = named_sync_and(5, 128, mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11));
             if (!ok) break;
             tc_fence_after();
             // 32-column blocks: S^T -> its bf16 copy for the next readout, and
@@ -1244,13 +1254,11 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             tmem_wait_st();
             if (td == 0) X->szero = gz ? 1 : 0;
             tc_fence_before();
-            named_sync(2, 128);   // szero is written before any warp's arrival
+            named_sync(5, 128);   // szero is written before any warp's arrival
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
-        // the MMAs of the last chunk must be complete before TMEM is released,
-        // and the output stores before the CTA's shared memory goes away
+        // the MMAs of the last chunk must be complete before TMEM is released
         if (ok && nch > 0) mbar_wait(&X->s_full, (nch - 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 12);
-        if (td == 0) bulk_wait_all();
     }
 
     tc_fence_before();

@@ -339,9 +339,8 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// 32 lanes x 32 bit, 16 consecutive columns: thread i of the warp gets lane
-// (quarter*32 + i), columns [col, col+16).
-// 32 lanes x 32 bit, 8 consecutive columns (see tmem_ld16).
+// 32 lanes x 32 bit, n consecutive columns (n = 8, 16, 32): thread i of the
+// warp gets lane (quarter*32 + i), columns [col, col+n).
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t *r) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
