@@ -18,6 +18,8 @@ Page citations (see ``hm_oracle.c`` for the full list):
         associativity, sec. 3 recurrent form, sec. 4.3 RetNet decay.
   [SSM] SSM article (quant67 56-ssm): sec. 3.2 softplus dt, sec. 4.2 affine
         composition, sec. 4.3 states recomputed in the backward pass.
+  [HM] sec. 5.1 also gives the block around the mixer: GPT-NeoX's parallel
+        residual block, x + mixer(norm1 x) + mlp(norm2 x) (``block_fwd``).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (forward) and ``tests/test_oracle_backward_pins.py`` (backward) against closed
@@ -483,6 +485,71 @@ def mixer_fwd(x, W_q, W_k, W_v, W_g, W_dt, conv_w, W_hq, W_hk, A_log, W_o,
     y = o.reshape(B * L, E) * silu(g)
     out = y @ _f64(W_o).T
     return out.reshape(B, L, D)
+
+
+# --------------------------------------------------------------------------
+# the block around the mixer ([HM] sec. 5.1)
+# --------------------------------------------------------------------------
+
+def layer_norm(x, w=None, b=None, eps=1e-5):
+    """Layer normalisation over the last axis, as the GPT-NeoX / Pythia block
+    applies it to its input before the mixer and before the MLP ([HM] sec. 5.1):
+    (x - mean) / sqrt(var + eps) * w + b, with var the population variance
+    (mean of squared deviations).  w, b: [D] or None (1 and 0)."""
+    x = _f64(x)
+    mean = x.mean(axis=-1, keepdims=True)
+    dev = x - mean
+    var = (dev * dev).mean(axis=-1, keepdims=True)
+    y = dev / np.sqrt(var + eps)
+    if w is not None:
+        y = y * _f64(w)
+    if b is not None:
+        y = y + _f64(b)
+    return y
+
+
+def _erf(x):
+    from scipy.special import erf
+    return erf(x)
+
+
+def gelu(x):
+    """GELU in its exact form, x * Phi(x) with Phi the standard normal CDF
+    written through erf: 0.5 x (1 + erf(x / sqrt 2)) (the activation of the
+    GPT-NeoX / Pythia MLP)."""
+    x = _f64(x)
+    return 0.5 * x * (1.0 + _erf(x / np.sqrt(2.0)))
+
+
+def mlp(h, W_fc1, b_fc1, W_fc2, b_fc2):
+    """The block's MLP: GELU(h W1^T + b1) W2^T + b2.  h: [..., D];
+    W_fc1: [F, D]; b_fc1: [F] or None; W_fc2: [D, F]; b_fc2: [D] or None."""
+    h = _f64(h)
+    u = h @ _f64(W_fc1).T
+    if b_fc1 is not None:
+        u = u + _f64(b_fc1)
+    y = gelu(u) @ _f64(W_fc2).T
+    if b_fc2 is not None:
+        y = y + _f64(b_fc2)
+    return y
+
+
+def block_fwd(x, ln1_w, ln1_b, ln2_w, ln2_b, W_fc1, b_fc1, W_fc2, b_fc2, mixer, eps=1e-5,
+              n_heads=8, batches=None):
+    """Parallel (GPT-NeoX / Pythia) block with the attention replaced by the
+    HedgeMamba mixer ([HM] sec. 5.1, Lst. 1): both branches read the same
+    input through their own normalisation and add into the residual,
+
+      out = x + mixer(LN1(x)) + MLP(LN2(x)).
+
+    x: [B, L, D]; ln*_w, ln*_b: [D]; MLP weights as in ``mlp``; ``mixer``: the
+    keyword arguments of ``mixer_fwd`` other than x, n_heads and batches."""
+    x = _f64(x)
+    if batches is not None:
+        x = x[list(batches)]
+    h1 = layer_norm(x, ln1_w, ln1_b, eps)
+    h2 = layer_norm(x, ln2_w, ln2_b, eps)
+    return x + mixer_fwd(h1, n_heads=n_heads, **mixer) + mlp(h2, W_fc1, b_fc1, W_fc2, b_fc2)
 
 
 def omp_threads_in_use() -> int:
