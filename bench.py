@@ -642,9 +642,11 @@ def bench_decode(cfg, args, rank, world, torch):
 
 # ---------------------------------------------------------------- mixer workload
 
-def bench_mixer(cfg, args, rank, world, torch):
+def bench_mixer(cfg, args, rank, world, torch, block=False):
     """Full mixer forward (B8 L4096 D2048 H8), one hm_mixer_fwd per step,
-    replayed from a CUDA graph."""
+    replayed from a CUDA graph; with ``block`` the parallel GPT-NeoX block
+    around it (layer norms, mixer, MLP d_model -> 4 d_model -> d_model,
+    residual), one hm_block_fwd per step."""
     import selective_ssm_sequence_b200 as hm
     peaks, peak_kind = load_peaks()
     if args.batch:
@@ -653,19 +655,28 @@ def bench_mixer(cfg, args, rank, world, torch):
     t = {k: to_dev(v, "f32" if k in ("conv_w", "A_log") else "bf16", torch) for k, v in w.items()}
     x = to_dev(wl.mixer_x(cfg), "bf16", torch)
     out = torch.empty_like(x)
-    a = hm.mixer_args(x, out, t["W_q"], t["W_k"], t["W_v"], t["W_g"], t["W_dt"], t["conv_w"],
-                      t["W_hq"], t["W_hk"], t["A_log"], t["W_o"], n_heads=cfg.H)
-    ws = hm.alloc_workspace(hm.hm_mixer_workspace_size(a))
+    d_ff = 4 * cfg.d_model
+    if block:
+        bw = {k: to_dev(v, "bf16" if k.startswith("W_") else "f32", torch)
+              for k, v in wl.block_weights(cfg, d_ff).items()}
+        a = hm.block_args(x, out, t, n_heads=cfg.H, **bw)
+        ws = hm.alloc_workspace(hm.hm_block_workspace_size(a))
+        call = lambda: hm.hm_block_fwd(a, ws)
+    else:
+        a = hm.mixer_args(x, out, t["W_q"], t["W_k"], t["W_v"], t["W_g"], t["W_dt"], t["conv_w"],
+                          t["W_hq"], t["W_hk"], t["A_log"], t["W_o"], n_heads=cfg.H)
+        ws = hm.alloc_workspace(hm.hm_mixer_workspace_size(a))
+        call = lambda: hm.hm_mixer_fwd(a, ws)
     stream = torch.cuda.current_stream()
     cap = torch.cuda.Stream()
     cap.wait_stream(stream)
     with torch.cuda.stream(cap):
-        hm.hm_mixer_fwd(a, ws)
+        call()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     n0 = hm.hm_launch_count()
     with torch.cuda.graph(g, stream=cap):
-        hm.hm_mixer_fwd(a, ws)
+        call()
     per_step = hm.hm_launch_count() - n0
     for _ in range(max(3, args.warmup)):
         g.replay()
@@ -689,15 +700,21 @@ def bench_mixer(cfg, args, rank, world, torch):
     D, E, L, B = cfg.d_model, cfg.d_model, cfg.L, cfg.B
     flops_tok = 2 * D * 4 * E + 2 * D * cfg.H + 2 * E * D + 2 * 2 * cfg.d_head * cfg.p * cfg.H \
         + 4 * 2 * cfg.p * (cfg.d_head + 1) * cfg.H + 3 * 2 * cfg.conv * E
+    if block:
+        flops_tok += 2 * 2 * D * d_ff   # the MLP's two GEMMs
     tf = flops_tok * B * L / (ms * 1e-3) / 1e12
+    name = cfg.name.replace("mixer", "block") if block else cfg.name
     return {
-        "metric": "mixer forward tokens/sec", "value": B * L * world / (ms * 1e-3), "unit": "tokens/s",
+        "metric": ("parallel block" if block else "mixer") + " forward tokens/sec",
+        "value": B * L * world / (ms * 1e-3), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": {"workload": cfg.name, "B": B, "L": L, "d_model": D, "H": cfg.H},
+        "data": "synthetic", "config": dict({"workload": name, "B": B, "L": L, "d_model": D, "H": cfg.H},
+                                            **({"d_ff": d_ff} if block else {})),
         "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tf / peaks["bf16_tflops"], "flops_per_token": flops_tok,
-                     "peak_source": peak_kind, "kernel": "whole mixer forward"},
+                     "peak_source": peak_kind,
+                     "kernel": "whole block forward" if block else "whole mixer forward"},
         "gpu_launches": per_step * args.steps,
         "clocks": sampler.summary(),
     }
@@ -832,10 +849,12 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "long", "decode", "mixer", "backward"], default="long",
+    ap.add_argument("--workload", choices=["prefill", "long", "decode", "mixer", "block", "backward"],
+                    default="long",
                     help="long: B1 H8 L32768 prefill (default, the largest single-GPU scan "
                          "workload); prefill: B4 H8 L2048; decode: 256 x 8 heads, 512 steps; "
-                         "mixer: B8 L4096 D2048; backward: hm_scan_bwd on B4 H8 L2048")
+                         "mixer: B8 L4096 D2048; block: the parallel block around that mixer "
+                         "(MLP width 8192); backward: hm_scan_bwd on B4 H8 L2048")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (decode: sequences, mixer: B) for small "
                          "profiling captures; the reported config says so")
@@ -859,8 +878,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     if args.workload == "decode":
         res = bench_decode(wl.DECODE, args, rank, world, torch)
-    elif args.workload == "mixer":
-        res = bench_mixer(wl.MIXER, args, rank, world, torch)
+    elif args.workload in ("mixer", "block"):
+        res = bench_mixer(wl.MIXER, args, rank, world, torch, block=args.workload == "block")
     elif args.workload == "backward":
         res = bench_backward(wl.PREFILL_PYTHIA, args, rank, world, torch)
     else:

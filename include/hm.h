@@ -329,6 +329,46 @@ HM_API hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t wo
                        hm_stream_t stream);
 
 /*
+ * hm_block_fwd -- the parallel GPT-NeoX / Pythia block with the HedgeMamba
+ * mixer in place of attention (HedgeMamba explainer sec. 5.1, Lst. 1: both
+ * branches read the block's input through their own norm and add into the
+ * residual):
+ *
+ *   h1  = LN(x; ln1_w, ln1_b),  h2 = LN(x; ln2_w, ln2_b)
+ *         LN(x; w, b) = (x - mean) / sqrt(var + eps) * w + b per row of D,
+ *         var the population variance
+ *   out = x + mixer(h1) + GELU(h2 W_fc1^T + b_fc1) W_fc2^T + b_fc2
+ *         GELU(u) = u * Phi(u), the exact (erf) form
+ *
+ * mixer: the hm_mixer_fwd arguments; its x is the block's input [B, L, D] and
+ * its out the block's output [B, L, D] (bf16).  ln*_w, ln*_b: [D] fp32 or NULL
+ * (1 and 0).  W_fc1 [d_ff, D], W_fc2 [D, d_ff] bf16; b_fc1 [d_ff], b_fc2 [D]
+ * fp32 or NULL.  d_ff and D multiples of 64, d_ff >= 64.
+ * The caller owns every buffer; workspace (hm_block_workspace_size bytes,
+ * 256-byte aligned) holds h1, h2, the fp32 sum x + mixer(h1), the MLP's hidden
+ * activations and the mixer's workspace.  Errors: HM_ERR_INVALID_ARG for a
+ * null or misaligned pointer, a bad size or a small workspace (nothing is
+ * launched); HM_ERR_UNSUPPORTED for sizes the tensor-core GEMM does not take;
+ * HM_ERR_CUDA for a launch failure.
+ */
+typedef struct {
+    hm_mixer_args mixer;
+    const float *ln1_w, *ln1_b;   /* [D] fp32 or NULL */
+    const float *ln2_w, *ln2_b;   /* [D] fp32 or NULL */
+    float eps;                    /* > 0 (1e-5 in Pythia) */
+    int d_ff;                     /* MLP width (4 D in Pythia) */
+    const void *W_fc1;            /* [d_ff, D] bf16 */
+    const float *b_fc1;           /* [d_ff] fp32 or NULL */
+    const void *W_fc2;            /* [D, d_ff] bf16 */
+    const float *b_fc2;           /* [D] fp32 or NULL */
+} hm_block_args;
+
+HM_API size_t hm_block_workspace_size(const hm_block_args *a);
+
+HM_API hm_status hm_block_fwd(const hm_block_args *a, void *workspace, size_t workspace_bytes,
+                       hm_stream_t stream);
+
+/*
  * hm_step_decode_noalloc -- hm_step_decode for callers that cannot allocate
  * device memory (for example a plugin whose host application owns all device
  * memory and offers no allocator, or a serving loop that must not allocate

@@ -74,6 +74,13 @@ class MixerArgs(ctypes.Structure):
                 ("W_hq", _P), ("W_hk", _P), ("A_log", _P), ("W_o", _P), ("out", _P)]
 
 
+class BlockArgs(ctypes.Structure):
+    """Mirror of hm_block_args."""
+    _fields_ = [("mixer", MixerArgs), ("ln1_w", _P), ("ln1_b", _P), ("ln2_w", _P), ("ln2_b", _P),
+                ("eps", ctypes.c_float), ("d_ff", _I), ("W_fc1", _P), ("b_fc1", _P), ("W_fc2", _P),
+                ("b_fc2", _P)]
+
+
 lib.hm_status_string.restype = ctypes.c_char_p
 lib.hm_status_string.argtypes = [_I]
 lib.hm_last_error_detail.restype = ctypes.c_char_p
@@ -95,6 +102,10 @@ lib.hm_mixer_workspace_size.restype = _SZ
 lib.hm_mixer_workspace_size.argtypes = [ctypes.POINTER(MixerArgs)]
 lib.hm_mixer_fwd.restype = _I
 lib.hm_mixer_fwd.argtypes = [ctypes.POINTER(MixerArgs), _P, _SZ, _P]
+lib.hm_block_workspace_size.restype = _SZ
+lib.hm_block_workspace_size.argtypes = [ctypes.POINTER(BlockArgs)]
+lib.hm_block_fwd.restype = _I
+lib.hm_block_fwd.argtypes = [ctypes.POINTER(BlockArgs), _P, _SZ, _P]
 lib.hm_scan_bwd_workspace_size.restype = _SZ
 lib.hm_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanBwdArgs)]
 lib.hm_scan_bwd.restype = _I
@@ -112,7 +123,7 @@ EXPORTED = ("hm_status_string", "hm_last_error_detail", "hm_version", "hm_featma
             "hm_scan_workspace_size", "hm_scan_chunked_fwd", "hm_decode_workspace_size",
             "hm_step_decode", "hm_mixer_workspace_size", "hm_mixer_fwd", "hm_get_device_error",
             "hm_launch_count", "hm_step_decode_noalloc", "hm_selftest_wait_timeout", "hm_scan_combine",
-            "hm_scan_bwd_workspace_size", "hm_scan_bwd")
+            "hm_scan_bwd_workspace_size", "hm_scan_bwd", "hm_block_workspace_size", "hm_block_fwd")
 
 
 class HMError(RuntimeError):
@@ -338,6 +349,30 @@ def hm_mixer_fwd(args: MixerArgs, workspace, stream=None) -> None:
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.hm_mixer_fwd(ctypes.byref(args), _ptr(workspace), nbytes, _stream(stream)),
            "hm_mixer_fwd")
+
+
+def block_args(x, out, mixer: dict, ln1_w, ln1_b, ln2_w, ln2_b, W_fc1, b_fc1, W_fc2, b_fc2, n_heads: int,
+               eps: float = 1e-5) -> BlockArgs:
+    """Fill an hm_block_args: ``mixer`` holds the mixer_args keywords other
+    than x, out and n_heads; x, out: [B, L, D]; W_fc1: [d_ff, D]; W_fc2: [D, d_ff]."""
+    a = BlockArgs()
+    m = mixer_args(x, out, n_heads=n_heads, **mixer)
+    a.mixer = m
+    a.ln1_w, a.ln1_b, a.ln2_w, a.ln2_b = map(_ptr, (ln1_w, ln1_b, ln2_w, ln2_b))
+    a.eps = float(eps)
+    a.d_ff = W_fc1.shape[0]
+    a.W_fc1, a.b_fc1, a.W_fc2, a.b_fc2 = map(_ptr, (W_fc1, b_fc1, W_fc2, b_fc2))
+    a._refs = (m._refs, ln1_w, ln1_b, ln2_w, ln2_b, W_fc1, b_fc1, W_fc2, b_fc2)
+    return a
+
+
+def hm_block_workspace_size(args: BlockArgs) -> int:
+    return int(lib.hm_block_workspace_size(ctypes.byref(args)))
+
+
+def hm_block_fwd(args: BlockArgs, workspace, stream=None) -> None:
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.hm_block_fwd(ctypes.byref(args), _ptr(workspace), nbytes, _stream(stream)), "hm_block_fwd")
 
 
 def hm_launch_count() -> int:

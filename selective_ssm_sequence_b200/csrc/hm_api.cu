@@ -9,7 +9,9 @@
 #include <atomic>
 #include <mutex>
 
-#include "hm_internal.h"
+#include <algorithm>
+
+#include "tc_common.cuh"
 
 namespace hm {
 
@@ -309,7 +311,7 @@ namespace {
 // ------------------------------------------------------------------ mixer
 
 struct MixerPlan {
-    size_t off_g, off_qkv_raw, off_dt, off_q, off_k, off_v, off_o, off_scan;   // byte offsets
+    size_t off_g, off_dt, off_q, off_k, off_v, off_o, off_scan;   // byte offsets
     size_t scan_bytes;
     size_t total;
     hm_scan_args scan;
@@ -337,12 +339,12 @@ hm_status check_mixer(const hm_mixer_args *a, MixerPlan *plan) {
     const size_t E = (size_t)a->E;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 256); return o; };
-    // fp32: projection output (q, k, v in turn), gate pre-activation, scan output
-    pl.off_qkv_raw = take((size_t)M * E * 4);
+    // fp32: the activated gate SiLU(x W_g^T + b_g) (a bf16 gate would add a
+    // rounding on top of y's) and dt; bf16: the gated scan output y and the
+    // conv outputs (the scan's q, k, v)
     pl.off_g = take((size_t)M * E * 4);
-    pl.off_o = take((size_t)M * E * 4);
+    pl.off_o = take((size_t)M * E * 2);
     pl.off_dt = take((size_t)M * a->H * 4);
-    // bf16: conv outputs (the scan's q, k, v); q's buffer is reused for the gated y
     pl.off_q = take((size_t)M * E * 2);
     pl.off_k = take((size_t)M * E * 2);
     pl.off_v = take((size_t)M * E * 2);
@@ -367,7 +369,60 @@ hm_status check_mixer(const hm_mixer_args *a, MixerPlan *plan) {
     return HM_OK;
 }
 
-// dt[r, h] = x[r, :] . W_dt[h, :] + b_dt[h]  (small N: one warp per row)
+// dt[r, h] = x[r, :] . W_dt[h, :] + b_dt[h]: N = H is too small for a GEMM
+// tile, so a warp takes a row and all H dot products at once (x read once, its
+// 16-byte pieces reused for every head), with W_dt staged in shared memory when
+// it fits (NH heads at compile time; the generic kernel below reads it through
+// L1).
+template <int NH>
+__global__ void dt_proj_heads_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ W,
+                                     const float *__restrict__ b, int64_t rows, int D, float *__restrict__ dt) {
+    extern __shared__ uint4 wsm[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nv = D / 8;   // 16-byte pieces per row
+    for (int i = threadIdx.x; i < NH * nv; i += blockDim.x) wsm[i] = reinterpret_cast<const uint4 *>(W)[i];
+    __syncthreads();
+    const int64_t wpb = blockDim.x >> 5;
+    for (int64_t r = blockIdx.x * wpb + warp; r < rows; r += (int64_t)gridDim.x * wpb) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + r * D);
+        float acc[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) acc[h] = 0.f;
+        for (int c = lane; c < nv; c += 32) {
+            const uint4 xv = xr[c];
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            float xf[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw[e]));
+                xf[2 * e] = t.x;
+                xf[2 * e + 1] = t.y;
+            }
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                const uint4 wv = wsm[h * nv + c];
+                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ww[e]));
+                    acc[h] = fmaf(xf[2 * e], t.x, acc[h]);
+                    acc[h] = fmaf(xf[2 * e + 1], t.y, acc[h]);
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < NH; ++h) acc[h] = warp_sum(acc[h]);
+        if (lane < NH) {
+            float v = acc[0];
+#pragma unroll
+            for (int h = 1; h < NH; ++h)
+                if (lane == h) v = acc[h];
+            dt[r * NH + lane] = v + (b ? b[lane] : 0.f);
+        }
+    }
+}
+
+// generic H: one warp per row, a dot product per head
 __global__ void dt_proj_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ W,
                                const float *__restrict__ b, int64_t rows, int D, int H,
                                float *__restrict__ dt) {
@@ -392,6 +447,38 @@ __global__ void dt_proj_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_b
         acc = warp_sum(acc);
         if (lane == 0) dt[r * H + h] = acc + (b ? b[h] : 0.f);
     }
+}
+
+template <int NH>
+cudaError_t launch_dt_heads(const void *x, const void *W, const float *b, int64_t rows, int D, float *dt,
+                            cudaStream_t s) {
+    const size_t smem = (size_t)NH * D * 2;
+    cudaError_t e = tc::ensure_smem_limit(dt_proj_heads_kernel<NH>, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (rows + 7) / 8;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)sms * 4);
+    dt_proj_heads_kernel<NH><<<grid, 256, smem, s>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)W, b, rows, D,
+                                                     dt);
+    return cudaGetLastError();
+}
+
+// dt = x W_dt^T (+ b_dt), [rows, H] fp32
+cudaError_t launch_dt_proj(const void *x, const void *W, const float *b, int64_t rows, int D, int H, float *dt,
+                           cudaStream_t s) {
+    cudaError_t e;
+    const bool staged = (size_t)H * D * 2 <= 96 * 1024;
+    if (staged && H == 8) e = launch_dt_heads<8>(x, W, b, rows, D, dt, s);
+    else if (staged && H == 4) e = launch_dt_heads<4>(x, W, b, rows, D, dt, s);
+    else if (staged && H == 16) e = launch_dt_heads<16>(x, W, b, rows, D, dt, s);
+    else {
+        const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+        dt_proj_kernel<<<blocks, 256, 0, s>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)W, b, rows, D, H, dt);
+        e = cudaGetLastError();
+    }
+    count_launches(1);
+    return e;
 }
 
 }  // namespace
@@ -444,7 +531,7 @@ namespace hm {
 namespace {
 
 // The prefill; with o_f32 (tensor-core path only) o is written as fp32.
-hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
+hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream, const void *gate = nullptr) {
     ScanPlan pl;
     hm_status st = check_scan(a, &pl);
     if (st != HM_OK) return st;
@@ -506,6 +593,7 @@ hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
     c.o_f32 = o_f32 && pl.tc;
     c.dt_scaled = (a->flags & HM_FLAG_DT_SCALED_INPUT) != 0;
     c.per_feature = (a->flags & HM_FLAG_PER_FEATURE_DECAY) != 0;
+    c.gate = pl.tc ? gate : nullptr;
     if (pl.tc)
         e = launch_scan_tc(c, ws + 2 * pl.phi_bytes + pl.lo_bytes, pl.tc_bytes,
                            DevErr{device_error_word()}, s);
@@ -517,6 +605,68 @@ hm_status scan_impl(const hm_scan_args *a, bool o_f32, hm_stream_t stream) {
 bool scan_uses_tc(const hm_scan_args *a) {
     ScanPlan pl;
     return check_scan(a, &pl) == HM_OK && pl.tc;
+}
+
+// The mixer on input x (the block passes its normalised input) into `out`,
+// with `out_ep` the epilogue of the output projection (a plain bf16 store, or
+// the block's residual addition).  Each step follows its producer without a
+// trip through HBM of its own where an epilogue can take it:
+//   q, k, v = causal conv of x W^T         (projection GEMMs, conv in the epilogue)
+//   gate    = SiLU(x W_g^T + b_g)          (GEMM, SiLU in the epilogue; kept in fp32)
+//   dt      = x W_dt^T + b_dt              (CUDA cores: 8 columns)
+//   y       = scan(q, k, v) * gate         (the gate applied as the scan stores o)
+//   out     = y W_o^T                      (GEMM, out_ep)
+hm_status mixer_run(const hm_mixer_args *a, const void *x, const MixerPlan &pl, char *ws, GemmEpiArgs out_ep,
+                    void *out, cudaStream_t s) {
+    const int64_t M = a->B * a->L;
+    if (M == 0) return HM_OK;
+    const int E = a->E, D = a->d_model, H = a->H;
+    DevErr err{device_error_word()};
+    void *gate = ws + pl.off_g, *y = ws + pl.off_o;
+    void *qc = ws + pl.off_q, *kc = ws + pl.off_k, *vc = ws + pl.off_v;
+    float *dt = (float *)(ws + pl.off_dt);
+    cudaError_t e;
+    const void *Wp[3] = {a->W_q, a->W_k, a->W_v};
+    void *dst[3] = {qc, kc, vc};
+    for (int i = 0; i < 3; ++i) {
+        GemmEpiArgs ep;
+        ep.mode = EPI_CONV_BF16;
+        ep.conv_w = a->conv_w + (size_t)i * E * a->conv_k;
+        ep.conv_k = a->conv_k;
+        ep.bias = a->conv_b ? a->conv_b + (size_t)i * E : nullptr;
+        ep.seq_len = a->L;
+        e = launch_gemm_tc_ex(x, Wp[i], M, E, D, dst[i], E, ep, err, s);
+        if (e != cudaSuccess) return cuda_fail(e, "mixer: projection GEMM with conv");
+    }
+    {
+        GemmEpiArgs ep;
+        ep.mode = EPI_SILU_F32;
+        ep.bias = a->b_g;
+        e = launch_gemm_tc_ex(x, a->W_g, M, E, D, gate, E, ep, err, s);
+        if (e != cudaSuccess) return cuda_fail(e, "mixer: gate GEMM");
+    }
+    e = launch_dt_proj(x, a->W_dt, a->b_dt, M, D, H, dt, s);
+    if (e != cudaSuccess) return cuda_fail(e, "mixer: dt projection");
+    hm_scan_args sa = pl.scan;
+    sa.q = qc; sa.k = kc; sa.v = vc;
+    sa.W_q = a->W_hq; sa.W_k = a->W_hk; sa.w_head_stride = 0;
+    sa.b_q = nullptr; sa.b_k = nullptr;
+    sa.dt = dt; sa.A_log = a->A_log;
+    sa.S0 = nullptr; sa.z0 = nullptr; sa.S_out = nullptr; sa.z_out = nullptr;
+    sa.o = y;
+    sa.workspace = ws + pl.off_scan;
+    sa.workspace_bytes = pl.scan_bytes;
+    const bool fused_gate = scan_uses_tc(&sa);
+    hm_status st = scan_impl(&sa, false, s, fused_gate ? gate : nullptr);
+    if (st != HM_OK) return st;
+    if (!fused_gate) {
+        // the CUDA-core scan stores o as it is: y = o * gate in place
+        e = launch_gate_mul(y, false, gate, M, E, y, s);
+        if (e != cudaSuccess) return cuda_fail(e, "mixer: gate");
+    }
+    e = launch_gemm_tc_ex(y, a->W_o, M, D, E, out, D, out_ep, err, s);
+    if (e != cudaSuccess) return cuda_fail(e, "mixer: out projection");
+    return HM_OK;
 }
 
 }  // namespace
@@ -588,56 +738,91 @@ hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t ws_bytes,
         return fail(HM_ERR_INVALID_ARG, "mixer: workspace must be 256-byte aligned");
     const int64_t M = a->B * a->L;
     if (M == 0) return HM_OK;
+    return mixer_run(a, a->x, pl, (char *)workspace, GemmEpiArgs{}, a->out, (cudaStream_t)stream);
+}
+
+namespace {
+
+struct BlockPlan {
+    MixerPlan mixer;
+    size_t off_h1, off_h2, off_sum, off_u, off_mixer, total;
+};
+
+hm_status check_block(const hm_block_args *a, BlockPlan *plan) {
+    if (!a) return fail(HM_ERR_INVALID_ARG, "block: null args");
+    hm_mixer_args m = a->mixer;
+    hm_status st = check_mixer(&m, &plan->mixer);
+    if (st != HM_OK) return st;
+    const int64_t M = m.B * m.L;
+    const int D = m.d_model;
+    if (a->d_ff < 64 || a->d_ff % 64 != 0 || D % 64 != 0)
+        return fail(HM_ERR_UNSUPPORTED, "block: d_ff and d_model must be multiples of 64");
+    if (!(a->eps > 0.f)) return fail(HM_ERR_INVALID_ARG, "block: eps must be > 0");
+    if (M > 0 && (!a->W_fc1 || !a->W_fc2)) return fail(HM_ERR_INVALID_ARG, "block: null MLP weight");
+    const void *ptrs[] = {a->ln1_w, a->ln1_b, a->ln2_w, a->ln2_b, a->W_fc1, a->b_fc1, a->W_fc2, a->b_fc2};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return fail(HM_ERR_INVALID_ARG, "block: pointers must be 16-byte aligned");
+    if (M > 0 && (!gemm_tc_supported(M, a->d_ff, D) || !gemm_tc_supported(M, D, a->d_ff)))
+        return fail(HM_ERR_UNSUPPORTED, "block: no tensor-core GEMM for these sizes");
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = round_up(off + bytes, 256); return o; };
+    plan->off_h1 = take((size_t)M * D * 2);
+    plan->off_h2 = take((size_t)M * D * 2);
+    plan->off_sum = take((size_t)M * D * 4);
+    plan->off_u = take((size_t)M * a->d_ff * 2);
+    plan->off_mixer = take(plan->mixer.total);
+    plan->total = off;
+    return HM_OK;
+}
+
+}  // namespace
+
+size_t hm_block_workspace_size(const hm_block_args *a) {
+    BlockPlan pl;
+    if (check_block(a, &pl) != HM_OK) return 0;
+    return pl.total;
+}
+
+hm_status hm_block_fwd(const hm_block_args *a, void *workspace, size_t ws_bytes, hm_stream_t stream) {
+    g_detail[0] = 0;
+    BlockPlan pl;
+    hm_status st = check_block(a, &pl);
+    if (st != HM_OK) return st;
+    if (!workspace || ws_bytes < pl.total)
+        return fail(HM_ERR_INVALID_ARG, "block: workspace too small (%zu < %zu bytes)", ws_bytes, pl.total);
+    if (((uintptr_t)workspace & 255u) != 0)
+        return fail(HM_ERR_INVALID_ARG, "block: workspace must be 256-byte aligned");
+    const hm_mixer_args &m = a->mixer;
+    const int64_t M = m.B * m.L;
+    if (M == 0) return HM_OK;
+    const int D = m.d_model;
     cudaStream_t s = (cudaStream_t)stream;
     char *ws = (char *)workspace;
-    const int E = a->E, D = a->d_model, H = a->H;
+    void *h1 = ws + pl.off_h1, *h2 = ws + pl.off_h2, *u = ws + pl.off_u;
+    float *sum = (float *)(ws + pl.off_sum);
     DevErr err{device_error_word()};
-    // Intermediates stay in fp32 where the next step can take fp32 (projection
-    // outputs into the conv, the gate pre-activation, the scan output into the
-    // gate): each bf16 rounding of an intermediate adds ~2^-9 relative error.
-    float *raw = (float *)(ws + pl.off_qkv_raw), *g = (float *)(ws + pl.off_g);
-    void *o = ws + pl.off_o;
-    void *qc = ws + pl.off_q, *kc = ws + pl.off_k, *vc = ws + pl.off_v;
-    float *dt = (float *)(ws + pl.off_dt);
-    cudaError_t e;
-    // q, k, v: projection (fp32) into `raw`, then the causal conv into bf16 buffers
-    const void *Wp[3] = {a->W_q, a->W_k, a->W_v};
-    void *dst[3] = {qc, kc, vc};
-    for (int i = 0; i < 3; ++i) {
-        e = launch_gemm_tc(a->x, Wp[i], M, E, D, raw, E, EPI_STORE_F32, nullptr, err, s);
-        if (e != cudaSuccess) return cuda_fail(e, "mixer: projection GEMM");
-        e = launch_causal_conv(raw, true, E, a->B, a->L, E, a->conv_k, a->conv_w + (size_t)i * E * a->conv_k,
-                               a->conv_b ? a->conv_b + (size_t)i * E : nullptr, dst[i], E, s);
-        if (e != cudaSuccess) return cuda_fail(e, "mixer: causal conv");
-    }
-    e = launch_gemm_tc(a->x, a->W_g, M, E, D, g, E, EPI_STORE_F32, a->b_g, err, s);
-    if (e != cudaSuccess) return cuda_fail(e, "mixer: gate GEMM");
-    {
-        const unsigned blocks = (unsigned)((M * 32 + 255) / 256);
-        dt_proj_kernel<<<blocks, 256, 0, s>>>((const __nv_bfloat16 *)a->x,
-                                              (const __nv_bfloat16 *)a->W_dt, a->b_dt, M, D, H, dt);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "mixer: dt projection");
-        count_launches(1);
-    }
-    hm_scan_args sa = pl.scan;
-    sa.q = qc; sa.k = kc; sa.v = vc;
-    sa.W_q = a->W_hq; sa.W_k = a->W_hk; sa.w_head_stride = 0;
-    sa.b_q = nullptr; sa.b_k = nullptr;
-    sa.dt = dt; sa.A_log = a->A_log;
-    sa.S0 = nullptr; sa.z0 = nullptr; sa.S_out = nullptr; sa.z_out = nullptr;
-    sa.o = o;
-    sa.workspace = ws + pl.off_scan;
-    sa.workspace_bytes = pl.scan_bytes;
-    const bool o_f32 = scan_uses_tc(&sa);
-    st = scan_impl(&sa, o_f32, stream);
+    cudaError_t e = launch_layernorm2(m.x, M, D, a->eps, a->ln1_w, a->ln1_b, a->ln2_w, a->ln2_b, h1, h2, s);
+    if (e != cudaSuccess) return cuda_fail(e, "block: layer norms");
+    // mixer branch: sum = x + mixer(h1), the residual added in the output projection's epilogue
+    GemmEpiArgs ep;
+    ep.mode = EPI_ADD_F32;
+    ep.res = m.x;
+    ep.ldr = D;
+    st = mixer_run(&m, h1, pl.mixer, ws + pl.off_mixer, ep, sum, s);
     if (st != HM_OK) return st;
-    // y = o * SiLU(g) (gate bias already added by the GEMM epilogue), bf16 into
-    // q's buffer; out = y W_o^T
-    e = launch_gate(o, o_f32, g, true, E, nullptr, M, E, qc, s);
-    if (e != cudaSuccess) return cuda_fail(e, "mixer: gate");
-    e = launch_gemm_tc(qc, a->W_o, M, D, E, a->out, D, EPI_STORE_BF16, nullptr, err, s);
-    if (e != cudaSuccess) return cuda_fail(e, "mixer: out projection");
+    // MLP branch: u = GELU(h2 W_fc1^T + b_fc1); out = u W_fc2^T + b_fc2 + sum
+    GemmEpiArgs e1;
+    e1.mode = EPI_GELU_BF16;
+    e1.bias = a->b_fc1;
+    e = launch_gemm_tc_ex(h2, a->W_fc1, M, a->d_ff, D, u, a->d_ff, e1, err, s);
+    if (e != cudaSuccess) return cuda_fail(e, "block: MLP up projection");
+    GemmEpiArgs e2;
+    e2.mode = EPI_ADD_BF16;
+    e2.bias = a->b_fc2;
+    e2.res = sum;
+    e2.ldr = D;
+    e = launch_gemm_tc_ex(u, a->W_fc2, M, D, a->d_ff, m.out, D, e2, err, s);
+    if (e != cudaSuccess) return cuda_fail(e, "block: MLP down projection");
     return HM_OK;
 }
 

@@ -111,6 +111,9 @@ struct ScanCore {
     float *S_out, *z_out;
     bool dt_scaled;       // HM_FLAG_DT_SCALED_INPUT: input term times softplus(dt)
     bool per_feature;     // HM_FLAG_PER_FEATURE_DECAY: A_log is [H, F]
+    // tensor-core path only: o is multiplied by this activated gate ([B, L, H,
+    // dv] fp32, the layout of o) before it is stored (the mixer's o * SiLU(g))
+    const void *gate = nullptr;
 };
 cudaError_t launch_scan_simt(const ScanCore &c, cudaStream_t s);
 
@@ -184,21 +187,38 @@ hm_status decode_enqueue(const hm_decode_args *a, const DecodePlan &plan, void *
 
 // bf16 GEMM C[M,N] = A[M,K] B[N,K]^T on tcgen05 with a fused epilogue.
 enum GemmEpi : int {
-    EPI_STORE_BF16 = 0,  // C bf16
-    EPI_STORE_F32 = 1,   // C fp32 (+ optional fp32 bias per column)
+    EPI_STORE_BF16 = 0,  // C bf16 = acc (+ bias)
+    EPI_STORE_F32 = 1,   // C fp32 = acc (+ bias)
+    EPI_CONV_BF16 = 2,   // C bf16 = depthwise causal conv of acc along each sequence (+ bias)
+    EPI_SILU_F32 = 3,    // C fp32 = SiLU(acc + bias)
+    EPI_GELU_BF16 = 4,   // C bf16 = GELU(acc + bias), exact (erf) form
+    EPI_ADD_F32 = 5,     // C fp32 = acc + bias + R, R bf16 [M, ldr]
+    EPI_ADD_BF16 = 6,    // C bf16 = acc + bias + R, R fp32 [M, ldr]
+};
+// What the GEMM's epilogue does with the fp32 accumulator tile.
+struct GemmEpiArgs {
+    GemmEpi mode = EPI_STORE_BF16;
+    const float *bias = nullptr;      // [N] per column, or null
+    const float *conv_w = nullptr;    // EPI_CONV_BF16: [N, conv_k]; bias is the conv bias
+    int conv_k = 1;                   // 1..8
+    int64_t seq_len = 0;              // EPI_CONV_BF16: row r is token r % seq_len of its sequence
+    const void *res = nullptr;        // EPI_ADD_*: residual
+    int64_t ldr = 0;
 };
 bool gemm_tc_supported(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_gemm_tc(const void *A, const void *Bm, int64_t M, int64_t N, int64_t K,
                            void *C, int64_t ldc, GemmEpi epi, const float *bias, DevErr err,
                            cudaStream_t s);
+cudaError_t launch_gemm_tc_ex(const void *A, const void *Bm, int64_t M, int64_t N, int64_t K, void *C,
+                              int64_t ldc, const GemmEpiArgs &ep, DevErr err, cudaStream_t s);
 
-// Depthwise causal conv over [B, L, C] (fp32 or bf16 in) with fp32 weights [C, K]; bf16 out.
-cudaError_t launch_causal_conv(const void *x, bool x_f32, int64_t x_ld, int64_t B, int64_t L, int C,
-                               int K, const float *w, const float *bias, void *y, int64_t y_ld,
-                               cudaStream_t s);
-
-// y[r, c] = o[r, c] * SiLU(g[r, c] + b_g[c]) (o, g fp32 or bf16; y bf16).
-cudaError_t launch_gate(const void *o, bool o_f32, const void *g, bool g_f32, int64_t g_ld,
-                        const float *b_g, int64_t rows, int E, void *y, cudaStream_t s);
+// h1, h2 = layer norms of the rows of x [rows, D] bf16 with (w1, b1) and
+// (w2, b2) (fp32 [D] each, NULL = 1 / 0), bf16 out
+cudaError_t launch_layernorm2(const void *x, int64_t rows, int D, float eps, const float *w1, const float *b1,
+                              const float *w2, const float *b2, void *h1, void *h2, cudaStream_t s);
+// y = o * gate (o fp32 or bf16; the gate fp32, already activated: SiLU(g + b_g)
+// from the gate GEMM's epilogue; y bf16, may alias o)
+cudaError_t launch_gate_mul(const void *o, bool o_f32, const void *gate, int64_t rows, int E, void *y,
+                            cudaStream_t s);
 
 }  // namespace hm

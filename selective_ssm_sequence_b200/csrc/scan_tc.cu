@@ -537,6 +537,7 @@ struct OutArgs {
     int dt_scaled;                   // step-scaled input: key j weighted by softplus(dt_j)
     const float *S0, *z0;            // segment 0 start state (caller layout) or null
     const float *S_start, *z_start;  // segments >= 1: [BH][G][F*dv], [BH][G][F]
+    const float *gate;               // o is multiplied by this (fp32, layout of o) before it is stored, or null
 };
 
 // dt of token t0 + tg for the first 64 threads of a group; -inf (log a = 0)
@@ -584,6 +585,11 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
 // update S^T += (w V)^T phiK.
 constexpr int kCThreads = 608;
 
+// GATE: o is multiplied by the mixer's activated gate before it is stored (a
+// separate instantiation, so that the plain scan carries none of its code: the
+// kernel's roles together already run more code per chunk than the
+// instruction cache holds).
+template <bool GATE>
 __global__ void __launch_bounds__(kCThreads, 1)
 scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
@@ -1088,7 +1094,28 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         bool ok = true;
         for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
-            // outputs of the chunk: o = O^T / den (lane = value channel, column = token)
+            // outputs of the chunk: o = O^T / den (lane = value channel, column = token),
+            // times the gate when there is one (in quarters of 16 tokens)
+            const int t0c = (c_begin + it) * kC;
+            float gq[16];   // the gate's values for the next quarter's tokens of this channel
+            auto load_gate = [&](int qt) {
+                const int64_t tb = t0c + 16 * qt;
+                const float *gp = a.gate + ((b * g.L + tb) * g.H + h) * (int64_t)g.dv + dv0 + ch;
+                const int tstride = g.H * g.dv;
+                const int nt = g.L - tb < 16 ? (int)(g.L - tb) : 16;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) gq[i] = i < nt ? gp[i * tstride] : 0.f;
+            };
+            if constexpr (GATE) {
+                load_gate(0);   // the loads run while this warp waits for O
+                // the next chunk's gate lines into L2: lane l fetches the line of
+                // this warp's 32 channels for tokens l and l + 32
+                const int64_t tn = t0c + kC + lane;
+                const float *gn = a.gate + ((b * g.L + tn) * g.H + h) * (int64_t)g.dv + dv0 + 32 * q;
+                if (tn < g.L) asm volatile("prefetch.global.L2 [%0];" ::"l"(gn));
+                if (tn + 32 < g.L)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(gn + 32 * (int64_t)g.H * g.dv));
+            }
             bool okc = ok && mbar_wait(&X->o_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 9) &&
                        mbar_wait(&X->den_ready[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 10);
             okc = __all_sync(0xffffffffu, okc);
@@ -1100,10 +1127,9 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             uint8_t *const stg = gP(s);
             const int cb = ch >> 6, cl = ch & 63;
             const float *rd = X->rden[s];
-            const int t0c = (c_begin + it) * kC;
 #pragma unroll 1
             for (int th = 0; th < 2; ++th) {
-                if (okc) {
+                if (okc && !GATE) {
                     tc_fence_after();
                     uint32_t r[32];
                     tmem_ld32(tmem + kColO + 32 * th + lanebase, r);
@@ -1124,6 +1150,30 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         __nv_bfloat16 *box = reinterpret_cast<__nv_bfloat16 *>(stg + th * 8192 + cb * 4096) + cl;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) box[i * 64] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                    }
+                } else if (GATE && okc) {
+                    // with the gate: quarters of 16 tokens, the next quarter's gate
+                    // values loading while this one is staged (bf16 out)
+                    tc_fence_after();
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int qt = 2 * th + hh;   // token quarter of the chunk
+                        uint32_t r[16];
+                        tmem_ld16(tmem + kColO + 16 * qt + lanebase, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i4 = 0; i4 < 4; ++i4) {
+                            const float4 d4 = *reinterpret_cast<const float4 *>(rd + 16 * qt + 4 * i4);
+                            r[4 * i4 + 0] = __float_as_uint(__uint_as_float(r[4 * i4 + 0]) * d4.x * gq[4 * i4 + 0]);
+                            r[4 * i4 + 1] = __float_as_uint(__uint_as_float(r[4 * i4 + 1]) * d4.y * gq[4 * i4 + 1]);
+                            r[4 * i4 + 2] = __float_as_uint(__uint_as_float(r[4 * i4 + 2]) * d4.z * gq[4 * i4 + 2]);
+                            r[4 * i4 + 3] = __float_as_uint(__uint_as_float(r[4 * i4 + 3]) * d4.w * gq[4 * i4 + 3]);
+                        }
+                        if (qt < 3) load_gate(qt + 1);   // under this quarter's staging
+                        __nv_bfloat16 *box =
+                            reinterpret_cast<__nv_bfloat16 *>(stg + th * 8192 + cb * 4096) + cl + 16 * hh * 64;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) box[i * 64] = __float2bfloat16_rn(__uint_as_float(r[i]));
                     }
                 }
                 if (th == 1) {
@@ -1424,6 +1474,7 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
     oa.z0 = c.z0;
     oa.S_start = S_start;
     oa.z_start = z_start;
+    oa.gate = (const float *)c.gate;
     // output tiles: boxes of 64 channels x 32 tokens, stored from unswizzled staging rows
     CUtensorMap to;
     {
@@ -1445,9 +1496,11 @@ cudaError_t launch_scan_tc_impl(const ScanCore &c, const void *phk_lo, void *ws,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
-    e = ensure_smem_limit(scan_out_kernel, kCSmem);
+    if (c.gate && c.o_f32) return cudaErrorInvalidValue;   // the gated output is bf16
+    auto out_kernel = c.gate ? scan_out_kernel<true> : scan_out_kernel<false>;
+    e = ensure_smem_limit(out_kernel, kCSmem);
     if (e != cudaSuccess) return e;
-    scan_out_kernel<<<(unsigned)(2 * g.G * BH), kCThreads, kCSmem, s>>>(tq, tk, tv, to, tss, oa, err);
+    out_kernel<<<(unsigned)(2 * g.G * BH), kCThreads, kCSmem, s>>>(tq, tk, tv, to, tss, oa, err);
     count_launches(1);
     return cudaGetLastError();
 }

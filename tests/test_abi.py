@@ -66,7 +66,8 @@ def _c_layout(struct, fields):
                                           ("hm_decode_args", "DecodeArgs"),
                                           ("hm_mixer_args", "MixerArgs"),
                                           ("hm_scan_bwd_args", "ScanBwdArgs"),
-                                          ("hm_combine_args", "CombineArgs")])
+                                          ("hm_combine_args", "CombineArgs"),
+                                          ("hm_block_args", "BlockArgs")])
 def test_struct_layouts_match_the_header(hm, cname, pyname):
     cls = getattr(hm, pyname)
     fields = [f[0] for f in cls._fields_]
@@ -123,6 +124,35 @@ def test_validation_rejects_bad_calls_before_launch(hm):
     m.B, m.L, m.d_model, m.H, m.E, m.p, m.conv_k = 1, 16, 2048, 8, 2050, 128, 4
     assert hm.lib.hm_mixer_fwd(ctypes.byref(m), None, 0, None) in (hm.HM_ERR_INVALID_ARG,
                                                                    hm.HM_ERR_UNSUPPORTED)
+
+
+def _block(hm, **kw):
+    fake = 1 << 20
+    b = hm.BlockArgs()
+    m = b.mixer
+    m.B, m.L, m.d_model, m.H, m.E, m.p, m.conv_k = 2, 300, 512, 2, 512, 128, 4
+    m.x = m.out = m.W_q = m.W_k = m.W_v = m.W_g = m.W_dt = m.conv_w = fake
+    m.W_hq = m.W_hk = m.A_log = m.W_o = fake
+    b.eps, b.d_ff, b.W_fc1, b.W_fc2 = 1e-5, 2048, fake, fake
+    for k, v in kw.items():
+        setattr(b, k, v)
+    return b
+
+
+def test_block_sizes_and_validation(hm):
+    def call(b, ws=None, n=0):
+        return hm.lib.hm_block_fwd(ctypes.byref(b), ws, n, None)
+    size = hm.hm_block_workspace_size(_block(hm))
+    M, D, dff = 600, 512, 2048
+    # h1, h2 (bf16), the fp32 residual sum and the MLP's hidden activations, plus the mixer's own
+    assert size >= M * D * (2 + 2 + 4) + M * dff * 2 + hm.hm_mixer_workspace_size(_block(hm).mixer)
+    assert call(_block(hm)) == hm.HM_ERR_INVALID_ARG                    # no workspace
+    assert b"workspace" in hm.lib.hm_last_error_detail()
+    assert call(_block(hm, eps=0.0)) == hm.HM_ERR_INVALID_ARG
+    assert call(_block(hm, d_ff=100)) == hm.HM_ERR_UNSUPPORTED
+    assert call(_block(hm, W_fc2=None)) == hm.HM_ERR_INVALID_ARG
+    assert call(_block(hm, ln1_w=(1 << 20) + 4)) == hm.HM_ERR_INVALID_ARG   # misaligned
+    assert hm.hm_block_workspace_size(_block(hm, d_ff=100)) == 0
 
 
 def test_variant_flags_are_validated_before_launch(hm):

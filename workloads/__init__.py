@@ -367,6 +367,26 @@ def mixer_weights(cfg: MixerConfig) -> Dict[str, np.ndarray]:
     }
 
 
+def block_weights(cfg: MixerConfig, d_ff: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Weights of the parallel block around the mixer: layer-norm scales
+    1 + N(0, 0.1^2) and shifts N(0, 0.1^2) (fp32 [D]); MLP d_model -> d_ff (4 d_model
+    by default) -> d_model with weights N(0, 1/fan_in) bf16 and biases
+    N(0, 0.1^2) fp32."""
+    s = cfg.seed
+    D = cfg.d_model
+    F = 4 * D if d_ff is None else d_ff
+    return {
+        "ln1_w": store(1.0 + normal(s, "ln1_w", (D,), 0.1), "f32"),
+        "ln1_b": store(normal(s, "ln1_b", (D,), 0.1), "f32"),
+        "ln2_w": store(1.0 + normal(s, "ln2_w", (D,), 0.1), "f32"),
+        "ln2_b": store(normal(s, "ln2_b", (D,), 0.1), "f32"),
+        "W_fc1": store(normal(s, "W_fc1", (F, D), math.sqrt(1.0 / D)), "bf16"),
+        "b_fc1": store(normal(s, "b_fc1", (F,), 0.1), "f32"),
+        "W_fc2": store(normal(s, "W_fc2", (D, F), math.sqrt(1.0 / F)), "bf16"),
+        "b_fc2": store(normal(s, "b_fc2", (D,), 0.1), "f32"),
+    }
+
+
 def mixer_x(cfg: MixerConfig, B: Optional[int] = None, L: Optional[int] = None) -> np.ndarray:
     B = cfg.B if B is None else B
     L = cfg.L if L is None else L
