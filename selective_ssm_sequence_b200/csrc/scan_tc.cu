@@ -570,14 +570,15 @@ __device__ __forceinline__ float chunk_total(float l, int tg, float *red, int ba
 //   10..13 outputs: o = O^T / den for the chunk, staged in the chunk's Pt
 //          buffer (dead once the PV product is complete) and written by TMA
 //          bulk stores
-//   15..18 state pass: S^T (fp32, TMEM) -> bf16 copy for the next readout and
-//          S^T <- gamma S^T before the next state MMA.  The outputs of a chunk
-//          and its state pass run at the same time on separate warps, so the
-//          next readout waits only for the state pass.
+//   15..18 z and state pass: the chunk's weighted key-feature sums and z (two
+//          features per thread, as soon as the chunk's phiK has landed), then
+//          S^T (fp32, TMEM) -> bf16 copy for the next readout and S^T <- gamma
+//          S^T before the next state MMA.  The outputs of a chunk and its
+//          state pass run at the same time on separate warps, so the next
+//          readout waits only for the state pass.
 //   4      decay vectors, one chunk ahead of the compute group (prefix sums
 //          of log a, e^cum, e^(cum_last - cum), the below-diagonal column
-//          factors, gamma), two tokens per lane; then the weighted key-feature
-//          sums and z of the chunk before, eight features per lane
+//          factors, gamma), two tokens per lane
 // The output and state-pass roles each take four consecutive warps, so that
 // every TMEM lane quarter is read by one warp of each.
 // Per chunk the MMA issuer runs: scores of the next chunk, then the readout
@@ -630,8 +631,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_init(&X->fullkv[s], 1);
             mbar_init(&X->emptyq[s], 1);
             mbar_init(&X->stg_free[s], 1);
-            // phiK + V: the chunk's MMAs and the compute group's key-feature sums
-            mbar_init(&X->emptykv[s], 2);
+            // phiK + V: the chunk's MMAs and the four state-pass warps' key-feature sums
+            mbar_init(&X->emptykv[s], 5);
         }
         mbar_init(&X->p_full, 1);
         mbar_init(&X->p_consumed, 3);   // the three score-quadrant warps have loaded P
@@ -647,8 +648,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         for (int r = 0; r < 3; ++r) mbar_init(&X->pro_full[r], 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&X->dec_full[s], 1);
-            mbar_init(&X->dec_free[s], 1);
-            mbar_init(&X->zfull[s], 1);
+            mbar_init(&X->dec_free[s], 5);   // the compute group and the four state-pass warps
+            mbar_init(&X->zfull[s], 4);      // one arrival per state-pass warp
             mbar_init(&X->zfree[s], 1);
         }
         X->abort = 0;
@@ -763,7 +764,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     } else if ((warp >= 2 && warp < 10 && warp != 4) || warp == 14) {
         // ------------------------------------------------------------ compute group
         // warps 2, 3, 14, 5, 6, 7, 8, 9 (warp 14 stands in for warp 4, which
-        // runs the decay vectors and z on the less busy SM sub-partition 0)
+        // runs the decay vectors on the less busy SM sub-partition 0)
         const int gt = (warp == 14 ? 2 : warp - 2) * 32 + lane;   // 0..255
         const int q = warp & 3;            // TMEM lane quarter of this warp
         // every exit from this loop is taken by the whole group (after a
@@ -922,7 +923,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             // (3) every thread: the query row scaled by e^cum_i, in place, and
             // phiq_i . z_prev over one quarter of the features (on the unscaled
             // bf16 values; the scale is applied to the sum).  z_prev = z after
-            // chunk it - 1 (the start z for it = 0), from the z warp: buffer
+            // chunk it - 1 (the start z for it = 0), from the state-pass warps: buffer
             // (it - 1) & 1, whose (it >> 1)-th write it is.
             okw = __all_sync(0xffffffffu, okw && mbar_wait(&X->zfull[(it - 1) & 1], (it >> 1) & 1, abort_flag,
                                                                err, KID_SCAN_TC_OUT, 24));
@@ -981,31 +982,18 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
         }
     } else if (warp == 4) {
-        // ------------------------------------------------------------ decay vectors and z
-        // Iteration c: the decay vectors of chunk c (one chunk ahead of the
-        // compute group), then z after chunk c - 1:
-        //   z_{c-1} = gamma_{c-1} z_{c-2} + sum_j w_j phik_j  (over chunk c - 1)
-        // into zb[(c - 1) & 1] for the compute group's denominators of chunk c.
-        // Lane: tokens 2 lane and 2 lane + 1 for the decay vectors (dt two
-        // chunks ahead); features 8 lane .. 8 lane + 7 for z.
-        {
-            // the start z, as the first write of buffer 1
-            const float *zi = nullptr;
-            if (seg == 0) zi = a.z0 ? a.z0 + bh * kF : nullptr;
-            else zi = a.z_start + (bh * g.G + seg) * kF;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) X->zb[1][8 * lane + e] = zi ? zi[8 * lane + e] : 0.f;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&X->zfull[1]);
-        }
+        // ------------------------------------------------------------ decay vectors
+        // Iteration c: the decay vectors of chunk c, one chunk ahead of the
+        // compute group.  Lane: tokens 2 lane and 2 lane + 1 (dt two chunks
+        // ahead).
         float da[2], db[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             da[i] = i < nch ? token_dt(a, b, h, (int64_t)(c_begin + i) * kC, 2 * lane) : -INFINITY;
             db[i] = i < nch ? token_dt(a, b, h, (int64_t)(c_begin + i) * kC, 2 * lane + 1) : -INFINITY;
         }
-        for (int c = 0; c <= nch; ++c) {
-          if (c < nch) {
+        for (int c = 0; c < nch; ++c) {
+          {
             const int sc = c & 1;
             const float l0 = hm_log_decay(da[0], alog) * kLog2e, l1 = hm_log_decay(db[0], alog) * kLog2e;
             // step-scaled input: log2 of softplus(dt) of the two tokens, added
@@ -1041,48 +1029,6 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (lane == 0) X->gam[sc] = ex2_approx(total);
             __syncwarp();
             if (lane == 0) mbar_arrive(&X->dec_full[sc]);
-          }
-          if (c >= 1) {
-            // z after chunk c - 1 (stage s1 holds its phiK; its weights and
-            // gamma are this warp's own decay vectors of parity s1)
-            const int s1 = (c - 1) & 1;
-            bool okz = mbar_wait(&X->fullkv[s1], ((c - 1) >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 25);
-            if (!__all_sync(0xffffffffu, okz)) break;
-            const uint8_t *__restrict__ base = gK(s1) + (lane >> 3) * kQKBlk;
-            const float *__restrict__ wv = X->w[s1];
-            float2 za[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) za[e] = make_float2(0.f, 0.f);
-#pragma unroll 1
-            for (int j0 = 0; j0 < kC; j0 += 8) {
-                uint4 kv[8];
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj)
-                    kv[jj] = *reinterpret_cast<const uint4 *>(base + sw128_off(j0 + jj, lane & 7));
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const float wj = wv[j0 + jj];
-                    const float2 w2 = make_float2(wj, wj);
-                    const uint32_t *pv = reinterpret_cast<const uint32_t *>(&kv[jj]);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) za[e] = fma2(unpack_bf16x2(pv[e]), w2, za[e]);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&X->emptykv[s1]);   // this warp's reads of the stage are done
-            // the buffer of z_{c-1} was last read by the compute group in chunk c - 2
-            okz = c < 2 || mbar_wait(&X->zfree[s1], ((c - 2) >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 26);
-            if (!__all_sync(0xffffffffu, okz)) break;
-            const float gm = X->gam[s1];
-            const float *__restrict__ zp = X->zb[(c - 2) & 1] + 8 * lane;
-            float *__restrict__ zn = X->zb[s1] + 8 * lane;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                zn[2 * e] = fmaf(gm, zp[2 * e], za[e].x);
-                zn[2 * e + 1] = fmaf(gm, zp[2 * e + 1], za[e].y);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&X->zfull[s1]);
           }
         }
     } else if (warp < 14) {
@@ -1209,6 +1155,15 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         const int q = warp & 3;
         const int ch = 32 * q + lane;
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
+        // the start z (z before the segment) as the first write of buffer 1;
+        // this thread's features: f0, f0 + 1 (the warp's 64-feature block)
+        const int f0 = 64 * q + 2 * lane;
+        {
+            const float *zi = seg == 0 ? (a.z0 ? a.z0 + bh * kF : nullptr) : a.z_start + (bh * g.G + seg) * kF;
+            *reinterpret_cast<float2 *>(&X->zb[1][f0]) = zi ? make_float2(zi[f0], zi[f0 + 1]) : make_float2(0.f, 0.f);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&X->zfull[1]);
+        }
         // prologue: start state -> bf16 copy (for the first readout) and fp32 x gamma_0
         float dt_next = token_dt(a, b, h, (int64_t)c_begin * kC, td);
         {
@@ -1270,7 +1225,40 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (lane == 0) mbar_arrive(&X->sbf_ready);
         }
         bool ok = true;
-        for (int it = 0; it + 1 < nch; ++it) {
+        for (int it = 0; it < nch; ++it) {
+            // z after chunk it, z_it = gamma_it z_(it-1) + sum_j w_j phik_j, into
+            // zb[it & 1] for the compute group's denominators of chunk it + 1,
+            // once the compute group has read the buffer's previous z (z_(it-2),
+            // or the start z for it = 1) in chunk it - 1: zfree, whose
+            // ((it - 1) >> 1)-th completion that is; then these warps release
+            // the chunk's stage and decay vectors
+            const int s1 = it & 1;
+            bool okz = mbar_wait(&X->dec_full[s1], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 23) &&
+                       mbar_wait(&X->fullkv[s1], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 25) &&
+                       (it < 1 || mbar_wait(&X->zfree[s1], ((it - 1) >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 26));
+            ok = named_sync_and(5, 128, okz);
+            if (!ok) break;
+            {
+                const uint8_t *__restrict__ kb = gK(s1) + q * kQKBlk + (lane & 3) * 4;
+                const float *__restrict__ wv = X->w[s1];
+                float2 za = make_float2(0.f, 0.f);
+#pragma unroll 8
+                for (int j = 0; j < kC; ++j) {
+                    const uint32_t kv = *reinterpret_cast<const uint32_t *>(kb + sw128_off(j, lane >> 2));
+                    const float wj = wv[j];
+                    za = fma2(unpack_bf16x2(kv), make_float2(wj, wj), za);
+                }
+                const float gm = X->gam[s1];
+                const float2 zp = *reinterpret_cast<const float2 *>(&X->zb[(it - 1) & 1][f0]);
+                *reinterpret_cast<float2 *>(&X->zb[s1][f0]) = make_float2(fmaf(gm, zp.x, za.x), fmaf(gm, zp.y, za.y));
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&X->emptykv[s1]);
+                    mbar_arrive(&X->dec_free[s1]);
+                    mbar_arrive(&X->zfull[s1]);
+                }
+            }
+            if (it + 1 >= nch) break;   // no state pass after the last chunk
             const float gn = fexp(chunk_total(hm_log_decay(dt_next, alog), td, X->redd, 5));
             if (it + 2 < nch) dt_next = token_dt(a, b, h, (int64_t)(c_begin + it + 2) * kC, td);
             ok = named_sync_and(5, 128, mbar_wait(&X->s_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 11));
