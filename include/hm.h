@@ -343,7 +343,7 @@ HM_API hm_status hm_mixer_fwd(const hm_mixer_args *a, void *workspace, size_t wo
  * mixer: the hm_mixer_fwd arguments; its x is the block's input [B, L, D] and
  * its out the block's output [B, L, D] (bf16).  ln*_w, ln*_b: [D] fp32 or NULL
  * (1 and 0).  W_fc1 [d_ff, D], W_fc2 [D, d_ff] bf16; b_fc1 [d_ff], b_fc2 [D]
- * fp32 or NULL.  d_ff and D multiples of 64, d_ff >= 64.
+ * fp32 or NULL.  d_ff a multiple of 64; D a multiple of 256, at most 4096.
  * The caller owns every buffer; workspace (hm_block_workspace_size bytes,
  * 256-byte aligned) holds h1, h2, the fp32 sum x + mixer(h1), the MLP's hidden
  * activations and the mixer's workspace.  Errors: HM_ERR_INVALID_ARG for a

@@ -755,8 +755,10 @@ hm_status check_block(const hm_block_args *a, BlockPlan *plan) {
     if (st != HM_OK) return st;
     const int64_t M = m.B * m.L;
     const int D = m.d_model;
-    if (a->d_ff < 64 || a->d_ff % 64 != 0 || D % 64 != 0)
-        return fail(HM_ERR_UNSUPPORTED, "block: d_ff and d_model must be multiples of 64");
+    if (a->d_ff < 64 || a->d_ff % 64 != 0)
+        return fail(HM_ERR_UNSUPPORTED, "block: d_ff must be a multiple of 64");
+    if (D % 256 != 0 || D > 4096)
+        return fail(HM_ERR_UNSUPPORTED, "block: d_model must be a multiple of 256, at most 4096");
     if (!(a->eps > 0.f)) return fail(HM_ERR_INVALID_ARG, "block: eps must be > 0");
     if (M > 0 && (!a->W_fc1 || !a->W_fc2)) return fail(HM_ERR_INVALID_ARG, "block: null MLP weight");
     const void *ptrs[] = {a->ln1_w, a->ln1_b, a->ln2_w, a->ln2_b, a->W_fc1, a->b_fc1, a->W_fc2, a->b_fc2};
