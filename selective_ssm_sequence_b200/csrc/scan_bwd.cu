@@ -20,9 +20,13 @@
 // Passes, each one CTA per (batch, head, 32 value columns) with the state in
 // registers as in the CUDA-core forward scan (warp w holds feature rows w,
 // w + 8, ..., lane = value column):
-//   P0 forward: d_t (slice 0) and the slice's share of sum_c do_t[c] n_t[c]
-//   PA forward: the slice's share of dphiq_t (+ z_t dd_t on slice 0)
-//   PB backward: the slice's share of dphik_t (+ g_t on slice 0), dv_t, dS0, dz0
+//   PA forward: the slice's shares of sum_c do_t[c] n_t[c] and of S_t dn_t
+//   PB backward: the slice's share of G_t v_t, dv_t, dS0
+// and three passes over the denominator's state alone, one CTA per (batch,
+// head) with a thread per feature: d_t (before PA), then z_t dd_t (once PA has
+// given do_t . n_t), then g_t and dz0, written as one more share.  Keeping z
+// out of the value-slice passes halves their registers, so two of their CTAs
+// fit on an SM, and PA needs only d_t, not dd_t.
 // then a reduction of the slices' shares (and the suffix sums of dlog a),
 // the feature-map backward (softmax Jacobian, dx = du W, dW = sum du x^T) and
 // the decay's (d dt = dlog a (-sigmoid(dt) e^A_log), dA_log = sum dlog a * log a).
@@ -46,7 +50,7 @@ struct BwdArgs {
     const float *S0, *z0;
     float *den;              // [B, L, H]
     float *e_part;           // [ns][B, L, H]: slices' shares of do . n
-    float *dq_part, *dk_part;   // [ns][B, L, H, F]
+    float *dq_part, *dk_part;   // [ns + 1][B, L, H, F]: the slices' shares, then the denominator's
     float *dv_out;           // [B, L, H, dv] fp32
     float *dS0, *dz0;        // nullable
 };
@@ -71,9 +75,9 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane)
 }
 
 template <int MODE, typename TIO>
-__global__ void __launch_bounds__(32 * kW)
+__global__ void __launch_bounds__(32 * kW, 2)
 bwd_pass_kernel(BwdArgs a) {
-    // MODE 0: P0, MODE 1: PA, MODE 2: PB (tokens in reverse order)
+    // MODE 1: PA, MODE 2: PB (tokens in reverse order)
     extern __shared__ float smem[];
     const int F = a.F, dv = a.dv;
     float *sq = smem;                      // [kTB][F]
@@ -83,10 +87,8 @@ bwd_pass_kernel(BwdArgs a) {
     float *sa = sg + kTB * 32;             // [kTB]       a_t
     float *sa1 = sa + kTB;                 // [kTB]       a_{t+1} (PB)
     float *sden = sa1 + kTB;               // [kTB]
-    float *sdd = sden + kTB;               // [kTB]       dd_t
-    float *red = sdd + kTB;                // [kTB][kW][32]
-    float *rden = red + kTB * kW * 32;     // [kTB][kW]
-    float *sout = rden + kTB * kW;         // [kTB][F]: the slice's shares of dphiq / dphik
+    float *red = sden + kTB;               // [kTB][kW][32]
+    float *sout = red + kTB * kW * 32;     // [kTB][F]: the slice's shares of dphiq / dphik
 
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int64_t bh = blockIdx.y;
@@ -101,16 +103,12 @@ bwd_pass_kernel(BwdArgs a) {
     const int64_t L = a.L;
     auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
 
-    float S[kMaxRows], z[kMaxRows];
+    float S[kMaxRows];
 #pragma unroll
     for (int m = 0; m < kMaxRows; ++m) {
         const int f = w + kW * m;
         S[m] = 0.f;
-        z[m] = 0.f;
-        if (MODE < 2 && f < F) {
-            if (a.S0 && col_ok) S[m] = a.S0[(bh * F + f) * dv + col];
-            if (a.z0) z[m] = a.z0[bh * F + f];
-        }
+        if (MODE < 2 && f < F && a.S0 && col_ok) S[m] = a.S0[(bh * F + f) * dv + col];
     }
     const int64_t nblk = (L + kTB - 1) / kTB;
     for (int64_t bi = 0; bi < nblk; ++bi) {
@@ -134,79 +132,55 @@ bwd_pass_kernel(BwdArgs a) {
             sa[t] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
             // a_{t+1}: the decay that carries G_{t+1} back to token t (none after the last token)
             sa1[t] = (t0 + t + 1 < L && a.dt) ? expf(hm_log_decay(a.dt[rowi(t0 + t + 1)], alog)) : 1.f;
-            if (MODE >= 1) {
-                const float dn_den = a.den[r];
-                float e = 0.f;
-                for (int s = 0; s < a.ns; ++s) e += a.e_part[(int64_t)s * a.B * L * a.H + r];
-                sden[t] = dn_den;
-                sdd[t] = -e / (dn_den * dn_den);   // dd = -(do . o) / d = -(do . n) / d^2
-            }
+            if (MODE >= 1) sden[t] = a.den[r];
         }
         __syncthreads();
         if (MODE < 2) {
             for (int t = 0; t < nt; ++t) {
                 const float at = sa[t];
                 const float vv = sv[t * 32 + lane];
-                float num = 0.f, den = 0.f;
+                float num = 0.f;
 #pragma unroll
                 for (int m = 0; m < kMaxRows; ++m) {
                     const int f = w + kW * m;
                     if (f < F) {
                         const float kf = sk[t * F + f], qf = sq[t * F + f];
                         S[m] = fmaf(at, S[m], kf * vv);
-                        z[m] = fmaf(at, z[m], kf);
                         num = fmaf(qf, S[m], num);
-                        den = fmaf(qf, z[m], den);
                     }
                 }
-                if (MODE == 0) {
-                    red[(t * kW + w) * 32 + lane] = num;
-                    if (lane == 0) rden[t * kW + w] = den;
-                } else {
-                    // the slice's share of dphiq_t[f] = sum_c S_t[f, c] dn_t[c] (+ z_t[f] dd_t),
-                    // row f = w + 8 m summed over the warp's lanes (columns)
+                red[(t * kW + w) * 32 + lane] = num;
+                if (MODE == 1) {
+                    // the slice's share of sum_c S_t[f, c] dn_t[c], row f = w + 8 m
+                    // summed over the warp's lanes (columns)
                     const float dn = sg[t * 32 + lane] / sden[t];
                     float x[kMaxRows];
 #pragma unroll
                     for (int m = 0; m < kMaxRows; ++m) x[m] = S[m] * dn;
                     const float tot = warp_reduce_scatter32(x, lane);
-                    // lane l now holds row w + 8 l; z of that row lives in lane l's z[l]
-                    float zl = 0.f;
-#pragma unroll
-                    for (int m = 0; m < kMaxRows; ++m) zl = lane == m ? z[m] : zl;
+                    // lane l now holds row w + 8 l
                     const int f = w + kW * lane;
-                    if (f < F) sout[t * F + f] = tot + (slice == 0 ? zl * sdd[t] : 0.f);
+                    if (f < F) sout[t * F + f] = tot;
                 }
             }
+            __syncthreads();
             if (MODE == 1) {
-                __syncthreads();
                 float *dq = a.dq_part + (int64_t)slice * a.B * L * a.H * F;
                 for (int i = threadIdx.x; i < nt * F; i += blockDim.x)
                     dq[rowi(t0 + i / F) * F + (i % F)] = sout[i];
             }
-            if (MODE == 0) {
-                __syncthreads();
-                // per token: d_t (slice 0) and the slice's share of do_t . n_t
-                for (int t = w; t < nt; t += kW) {
-                    float n = 0.f, d = 0.f;
-                    for (int ww = 0; ww < kW; ++ww) {
-                        n += red[(t * kW + ww) * 32 + lane];
-                        d += rden[t * kW + ww];
-                    }
-                    const float e = warp_sum(n * sg[t * 32 + lane]);
-                    const int64_t r = rowi(t0 + t);
-                    if (lane == 0) {
-                        a.e_part[(int64_t)slice * a.B * L * a.H + r] = e;
-                        if (slice == 0) a.den[r] = d;
-                    }
-                }
+            // per token: the slice's share of do_t . n_t
+            for (int t = w; t < nt; t += kW) {
+                float n = 0.f;
+                for (int ww = 0; ww < kW; ++ww) n += red[(t * kW + ww) * 32 + lane];
+                const float e = warp_sum(n * sg[t * 32 + lane]);
+                if (lane == 0) a.e_part[(int64_t)slice * a.B * L * a.H + rowi(t0 + t)] = e;
             }
         } else {
-            // PB: G_t = phiq_t dn_t^T + a_{t+1} G_{t+1} (S holds G, z holds g)
+            // PB: G_t = phiq_t dn_t^T + a_{t+1} G_{t+1} (S holds G)
             for (int t = nt - 1; t >= 0; --t) {
                 const float a1 = sa1[t];
                 const float dn = sg[t * 32 + lane] / sden[t];
-                const float dd = sdd[t];
                 const float vv = sv[t * 32 + lane];
                 float dvp = 0.f;
                 float x[kMaxRows];
@@ -217,18 +191,14 @@ bwd_pass_kernel(BwdArgs a) {
                     if (f < F) {
                         const float qf = sq[t * F + f], kf = sk[t * F + f];
                         S[m] = fmaf(a1, S[m], qf * dn);
-                        z[m] = fmaf(a1, z[m], qf * dd);
                         dvp = fmaf(S[m], kf, dvp);
                         x[m] = S[m] * vv;
                     }
                 }
-                // the slice's share of dphik_t[f] = sum_c G_t[f, c] v_t[c] (+ g_t[f])
+                // the slice's share of sum_c G_t[f, c] v_t[c]
                 const float tot = warp_reduce_scatter32(x, lane);
-                float zl = 0.f;
-#pragma unroll
-                for (int m = 0; m < kMaxRows; ++m) zl = lane == m ? z[m] : zl;
                 const int fl = w + kW * lane;
-                if (fl < F) sout[t * F + fl] = tot + (slice == 0 ? zl : 0.f);
+                if (fl < F) sout[t * F + fl] = tot;
                 red[(t * kW + w) * 32 + lane] = dvp;
             }
             __syncthreads();
@@ -244,20 +214,91 @@ bwd_pass_kernel(BwdArgs a) {
                 for (int i = threadIdx.x; i < nt * F; i += blockDim.x)
                     dk[rowi(t0 + i / F) * F + (i % F)] = sout[i];
             }
-            if (t0 == 0) {
-                // dS0 = a_1 G_1, dz0 = a_1 g_1 (a_1 = the first token's decay)
+            if (t0 == 0 && a.dS0 && col_ok) {
+                // dS0 = a_1 G_1 (a_1 = the first token's decay)
                 const float a0 = sa[0];
 #pragma unroll
                 for (int m = 0; m < kMaxRows; ++m) {
                     const int f = w + kW * m;
-                    if (f < F) {
-                        if (a.dS0 && col_ok) a.dS0[(bh * F + f) * dv + col] = a0 * S[m];
-                        if (a.dz0 && slice == 0 && lane == 0) a.dz0[bh * F + f] = a0 * z[m];
-                    }
+                    if (f < F) a.dS0[(bh * F + f) * dv + col] = a0 * S[m];
                 }
             }
         }
         __syncthreads();
+    }
+}
+
+// The denominator's state z alone, one CTA per (batch, head), thread f =
+// feature f (the same three passes as above):
+//   MODE 0 forward:  z_t = a_t z_(t-1) + phik_t, d_t = phiq_t . z_t
+//   MODE 1 forward:  z_t again; its share of dphiq_t is z_t dd_t
+//   MODE 2 backward: g_t = a_(t+1) g_(t+1) + phiq_t dd_t, its share of dphik_t;
+//                    dz0 = a_1 g_1
+// The shares go to plane ns of dq_part / dk_part, after the value slices'.
+template <int MODE>
+__global__ void __launch_bounds__(256)
+bwd_z_kernel(BwdArgs a) {
+    __shared__ float sa[kTB], sa1[kTB], sdd[kTB];
+    __shared__ float red[kTB][kW];
+    const int f = threadIdx.x, lane = f & 31, w = f >> 5;
+    const int64_t bh = blockIdx.x;
+    const int64_t b = bh / a.H;
+    const int h = (int)(bh % a.H);
+    const int F = a.F;
+    const bool fok = f < F;
+    const float alog = a.dt ? a.A_log[h] : 0.f;
+    const int64_t L = a.L;
+    const int64_t rows = a.B * L * a.H;
+    auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
+    float zs = (MODE < 2 && a.z0 && fok) ? a.z0[bh * F + f] : 0.f;
+    const int64_t nblk = (L + kTB - 1) / kTB;
+    for (int64_t bi = 0; bi < nblk; ++bi) {
+        const int64_t t0 = (MODE == 2 ? nblk - 1 - bi : bi) * kTB;
+        const int nt = (int)((L - t0) < kTB ? (L - t0) : kTB);
+        __syncthreads();
+        if (threadIdx.x < nt) {
+            const int t = threadIdx.x;
+            const int64_t r = rowi(t0 + t);
+            sa[t] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
+            sa1[t] = (t0 + t + 1 < L && a.dt) ? expf(hm_log_decay(a.dt[rowi(t0 + t + 1)], alog)) : 1.f;
+            if (MODE >= 1) {
+                const float d = a.den[r];
+                float e = 0.f;
+                for (int s = 0; s < a.ns; ++s) e += a.e_part[(int64_t)s * rows + r];
+                sdd[t] = -e / (d * d);   // dd = -(do . o) / d = -(do . n) / d^2
+            }
+        }
+        __syncthreads();
+        if (MODE < 2) {
+            for (int t = 0; t < nt; ++t) {
+                const int64_t r = rowi(t0 + t);
+                const float kf = fok ? a.phk[r * F + f] : 0.f;
+                zs = fmaf(sa[t], zs, kf);
+                if (MODE == 0) {
+                    const float p = warp_sum(fok ? a.phq[r * F + f] * zs : 0.f);
+                    if (lane == 0) red[t][w] = p;
+                } else if (fok) {
+                    a.dq_part[(int64_t)a.ns * rows * F + r * F + f] = zs * sdd[t];
+                }
+            }
+            if (MODE == 0) {
+                __syncthreads();
+                if (threadIdx.x < nt) {
+                    float d = 0.f;
+#pragma unroll
+                    for (int ww = 0; ww < kW; ++ww) d += red[threadIdx.x][ww];
+                    a.den[rowi(t0 + threadIdx.x)] = d;
+                }
+            }
+        } else {
+            for (int t = nt - 1; t >= 0; --t) {
+                const int64_t r = rowi(t0 + t);
+                const float qf = fok ? a.phq[r * F + f] : 0.f;
+                zs = fmaf(sa1[t], zs, qf * sdd[t]);
+                if (fok) a.dk_part[(int64_t)a.ns * rows * F + r * F + f] = zs;
+            }
+            if (t0 == 0 && a.dz0 && fok) a.dz0[bh * F + f] = sa[0] * zs;
+        }
     }
 }
 
@@ -273,7 +314,7 @@ bwd_reduce_kernel(BwdArgs a, float *__restrict__ dphq, float *__restrict__ dphk,
     float acc = 0.f;
     for (int f = lane; f < a.F; f += 32) {
         float sq = 0.f, sk = 0.f;
-        for (int s = 0; s < a.ns; ++s) {
+        for (int s = 0; s <= a.ns; ++s) {
             sq += a.dq_part[s * plane + r * a.F + f];
             sk += a.dk_part[s * plane + r * a.F + f];
         }
@@ -416,19 +457,21 @@ decay_bwd_kernel(const float *__restrict__ dt, const float *__restrict__ A_log, 
 template <typename TIO>
 cudaError_t run_passes(const BwdArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)a.ns, (unsigned)(a.B * a.H));
-    const size_t smem = sizeof(float) * (size_t)(3 * kTB * a.F + 2 * kTB * 32 + 4 * kTB + kTB * kW * 32 + kTB * kW);
+    const size_t smem = sizeof(float) * (size_t)(3 * kTB * a.F + 2 * kTB * 32 + 3 * kTB + kTB * kW * 32);
     cudaError_t e;
-    auto k0 = bwd_pass_kernel<0, TIO>;
     auto k1 = bwd_pass_kernel<1, TIO>;
     auto k2 = bwd_pass_kernel<2, TIO>;
-    for (auto k : {k0, k1, k2}) {
+    for (auto k : {k1, k2}) {
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k0<<<grid, 32 * kW, smem, s>>>(a);
+    const unsigned zgrid = (unsigned)(a.B * a.H);
+    bwd_z_kernel<0><<<zgrid, 256, 0, s>>>(a);
     k1<<<grid, 32 * kW, smem, s>>>(a);
+    bwd_z_kernel<1><<<zgrid, 256, 0, s>>>(a);
     k2<<<grid, 32 * kW, smem, s>>>(a);
-    count_launches(3);
+    bwd_z_kernel<2><<<zgrid, 256, 0, s>>>(a);
+    count_launches(5);
     return cudaGetLastError();
 }
 
@@ -442,7 +485,7 @@ size_t scan_bwd_workspace(const ScanBwdCore &c) {
     n += 2 * r256(rows * c.F * 4);             // phq, phk (fp32)
     n += r256(rows * 4);                       // den
     n += r256((size_t)ns * rows * 4);          // e_part
-    n += 2 * r256((size_t)ns * rows * c.F * 4);  // dq_part, dk_part
+    n += 2 * r256((size_t)(ns + 1) * rows * c.F * 4);  // dq_part, dk_part
     n += 2 * r256(rows * c.F * 4);             // dphq, dphk
     n += 2 * r256(rows * 4);                   // kd, dlog a
     if (c.W_q) n += r256(rows * c.p * 4);      // du
@@ -463,8 +506,8 @@ cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
     a.S0 = c.S0; a.z0 = c.z0;
     a.den = (float *)take(rows * 4);
     a.e_part = (float *)take((size_t)ns * rows * 4);
-    a.dq_part = (float *)take((size_t)ns * rows * c.F * 4);
-    a.dk_part = (float *)take((size_t)ns * rows * c.F * 4);
+    a.dq_part = (float *)take((size_t)(ns + 1) * rows * c.F * 4);
+    a.dk_part = (float *)take((size_t)(ns + 1) * rows * c.F * 4);
     float *dphq = (float *)take(rows * c.F * 4), *dphk = (float *)take(rows * c.F * 4);
     float *kd = (float *)take(rows * 4);
     float *dla = (float *)take(rows * 4);
