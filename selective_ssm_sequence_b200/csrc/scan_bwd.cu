@@ -17,11 +17,12 @@
 // key's phik_j . dphik_j.  It needs neither forward nor backward state, so no
 // pass has to hold S and G at once.
 //
-// Passes, each one CTA per (batch, head, 32 value columns) with the state in
-// registers as in the CUDA-core forward scan (warp w holds feature rows w,
-// w + 8, ..., lane = value column):
-//   PA forward: the slice's shares of sum_c do_t[c] n_t[c] and of S_t dn_t
-//   PB backward: the slice's share of G_t v_t, dv_t, dS0
+// Passes, each one CTA per (batch, head, 32 value columns) with the state's
+// 256 x 32 slice in registers:
+//   PA forward (a thread per feature row): the slice's shares of
+//      sum_c do_t[c] n_t[c] and of S_t dn_t
+//   PB backward (warp w holds feature rows w, w + 8, ..., lane = column, as
+//      in the CUDA-core forward scan): the slice's share of G_t v_t, dv_t, dS0
 // and three passes over the denominator's state alone, one CTA per (batch,
 // head) with a thread per feature: d_t (before PA), then z_t dd_t (once PA has
 // given do_t . n_t), then g_t and dz0, written as one more share.  Keeping z
@@ -74,10 +75,11 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane)
     return v[0];
 }
 
-template <int MODE, typename TIO>
+// PB, tokens from the last to the first (the state layout of the forward
+// CUDA-core scan: warp w holds feature rows w, w + 8, ..., lane = column).
+template <typename TIO>
 __global__ void __launch_bounds__(32 * kW, 2)
-bwd_pass_kernel(BwdArgs a) {
-    // MODE 1: PA, MODE 2: PB (tokens in reverse order)
+bwd_pb_kernel(BwdArgs a) {
     extern __shared__ float smem[];
     const int F = a.F, dv = a.dv;
     float *sq = smem;                      // [kTB][F]
@@ -103,17 +105,13 @@ bwd_pass_kernel(BwdArgs a) {
     const int64_t L = a.L;
     auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
 
-    float S[kMaxRows];
+    float S[kMaxRows];   // G, the adjoint of S, from zero after the last token
 #pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) {
-        const int f = w + kW * m;
-        S[m] = 0.f;
-        if (MODE < 2 && f < F && a.S0 && col_ok) S[m] = a.S0[(bh * F + f) * dv + col];
-    }
+    for (int m = 0; m < kMaxRows; ++m) S[m] = 0.f;
     const int64_t nblk = (L + kTB - 1) / kTB;
     for (int64_t bi = 0; bi < nblk; ++bi) {
         // PB walks the token blocks from the last to the first
-        const int64_t t0 = (MODE == 2 ? nblk - 1 - bi : bi) * kTB;
+        const int64_t t0 = (nblk - 1 - bi) * kTB;
         const int nt = (int)((L - t0) < kTB ? (L - t0) : kTB);
         for (int i = threadIdx.x; i < nt * F; i += blockDim.x) {
             const int t = i / F, f = i % F;
@@ -132,51 +130,10 @@ bwd_pass_kernel(BwdArgs a) {
             sa[t] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
             // a_{t+1}: the decay that carries G_{t+1} back to token t (none after the last token)
             sa1[t] = (t0 + t + 1 < L && a.dt) ? expf(hm_log_decay(a.dt[rowi(t0 + t + 1)], alog)) : 1.f;
-            if (MODE >= 1) sden[t] = a.den[r];
+            sden[t] = a.den[r];
         }
         __syncthreads();
-        if (MODE < 2) {
-            for (int t = 0; t < nt; ++t) {
-                const float at = sa[t];
-                const float vv = sv[t * 32 + lane];
-                float num = 0.f;
-#pragma unroll
-                for (int m = 0; m < kMaxRows; ++m) {
-                    const int f = w + kW * m;
-                    if (f < F) {
-                        const float kf = sk[t * F + f], qf = sq[t * F + f];
-                        S[m] = fmaf(at, S[m], kf * vv);
-                        num = fmaf(qf, S[m], num);
-                    }
-                }
-                red[(t * kW + w) * 32 + lane] = num;
-                if (MODE == 1) {
-                    // the slice's share of sum_c S_t[f, c] dn_t[c], row f = w + 8 m
-                    // summed over the warp's lanes (columns)
-                    const float dn = sg[t * 32 + lane] / sden[t];
-                    float x[kMaxRows];
-#pragma unroll
-                    for (int m = 0; m < kMaxRows; ++m) x[m] = S[m] * dn;
-                    const float tot = warp_reduce_scatter32(x, lane);
-                    // lane l now holds row w + 8 l
-                    const int f = w + kW * lane;
-                    if (f < F) sout[t * F + f] = tot;
-                }
-            }
-            __syncthreads();
-            if (MODE == 1) {
-                float *dq = a.dq_part + (int64_t)slice * a.B * L * a.H * F;
-                for (int i = threadIdx.x; i < nt * F; i += blockDim.x)
-                    dq[rowi(t0 + i / F) * F + (i % F)] = sout[i];
-            }
-            // per token: the slice's share of do_t . n_t
-            for (int t = w; t < nt; t += kW) {
-                float n = 0.f;
-                for (int ww = 0; ww < kW; ++ww) n += red[(t * kW + ww) * 32 + lane];
-                const float e = warp_sum(n * sg[t * 32 + lane]);
-                if (lane == 0) a.e_part[(int64_t)slice * a.B * L * a.H + rowi(t0 + t)] = e;
-            }
-        } else {
+        {
             // PB: G_t = phiq_t dn_t^T + a_{t+1} G_{t+1} (S holds G)
             for (int t = nt - 1; t >= 0; --t) {
                 const float a1 = sa1[t];
@@ -223,6 +180,99 @@ bwd_pass_kernel(BwdArgs a) {
                     if (f < F) a.dS0[(bh * F + f) * dv + col] = a0 * S[m];
                 }
             }
+        }
+        __syncthreads();
+    }
+}
+
+// PA with a thread per feature row (the 32 columns of the slice in its
+// registers): S_t[f, :] = a_t S_(t-1)[f, :] + phik_t[f] v_t and
+// u_f = sum_c S_t[f, c] do_t[c] stay within the thread; the slice's share of
+// dphiq_t[f] is u_f / d_t and its share of do_t . n_t = sum_f phiq_t[f] u_f
+// is one block reduction per token.
+template <typename TIO>
+__global__ void __launch_bounds__(256, 2)
+bwd_pa_kernel(BwdArgs a) {
+    extern __shared__ float smem[];
+    const int F = a.F, dv = a.dv;
+    float *sq = smem;                      // [kTB][F]
+    float *sk = sq + kTB * F;              // [kTB][F]
+    float *sv = sk + kTB * F;              // [kTB][32]   v
+    float *sg = sv + kTB * 32;             // [kTB][32]   do
+    float *sa = sg + kTB * 32;             // [kTB]       a_t
+    float *sden = sa + kTB;                // [kTB]
+    float *red = sden + kTB;               // [kTB][kW]
+    float *sout = red + kTB * kW;          // [kTB][F]
+
+    const int f = threadIdx.x, lane = f & 31, w = f >> 5;
+    const bool fok = f < F;
+    const int64_t bh = blockIdx.y;
+    const int64_t b = bh / a.H;
+    const int h = (int)(bh % a.H);
+    const int slice = blockIdx.x;
+    const int c0 = slice * 32;
+    const int ncol = dv - c0 < 32 ? dv - c0 : 32;
+    const float alog = a.dt ? a.A_log[h] : 0.f;
+    const TIO *v = (const TIO *)a.v;
+    const TIO *dout = (const TIO *)a.dout;
+    const int64_t L = a.L;
+    const int64_t rows = a.B * L * a.H;
+    auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
+
+    float S[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) S[c] = (a.S0 && fok && c < ncol) ? a.S0[(bh * F + f) * dv + c0 + c] : 0.f;
+    const int64_t nblk = (L + kTB - 1) / kTB;
+    for (int64_t bi = 0; bi < nblk; ++bi) {
+        const int64_t t0 = bi * kTB;
+        const int nt = (int)((L - t0) < kTB ? (L - t0) : kTB);
+        for (int i = threadIdx.x; i < nt * F; i += blockDim.x) {
+            const int t = i / F, ff = i % F;
+            sq[i] = a.phq[rowi(t0 + t) * F + ff];
+            sk[i] = a.phk[rowi(t0 + t) * F + ff];
+        }
+        for (int i = threadIdx.x; i < nt * 32; i += blockDim.x) {
+            const int t = i / 32, c = i % 32;
+            const bool ok = c < ncol;
+            sv[i] = ok ? hm_ld(v, rowi(t0 + t) * dv + c0 + c) : 0.f;
+            sg[i] = ok ? hm_ld(dout, rowi(t0 + t) * dv + c0 + c) : 0.f;
+        }
+        if (threadIdx.x < nt) {
+            const int64_t r = rowi(t0 + threadIdx.x);
+            sa[threadIdx.x] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
+            sden[threadIdx.x] = a.den[r];
+        }
+        __syncthreads();
+        for (int t = 0; t < nt; ++t) {
+            const float at = sa[t];
+            const float kf = fok ? sk[t * F + f] : 0.f;
+            float u = 0.f;
+            const float4 *v4 = reinterpret_cast<const float4 *>(sv + t * 32);
+            const float4 *g4 = reinterpret_cast<const float4 *>(sg + t * 32);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+                const float4 vv = v4[c4], gg = g4[c4];
+                S[4 * c4 + 0] = fmaf(at, S[4 * c4 + 0], kf * vv.x);
+                S[4 * c4 + 1] = fmaf(at, S[4 * c4 + 1], kf * vv.y);
+                S[4 * c4 + 2] = fmaf(at, S[4 * c4 + 2], kf * vv.z);
+                S[4 * c4 + 3] = fmaf(at, S[4 * c4 + 3], kf * vv.w);
+                u = fmaf(S[4 * c4 + 0], gg.x, u);
+                u = fmaf(S[4 * c4 + 1], gg.y, u);
+                u = fmaf(S[4 * c4 + 2], gg.z, u);
+                u = fmaf(S[4 * c4 + 3], gg.w, u);
+            }
+            if (fok) sout[t * F + f] = u / sden[t];
+            const float ep = warp_sum(fok ? sq[t * F + f] * u : 0.f);
+            if (lane == 0) red[t * kW + w] = ep;
+        }
+        __syncthreads();
+        float *dq = a.dq_part + (int64_t)slice * rows * F;
+        for (int i = threadIdx.x; i < nt * F; i += blockDim.x) dq[rowi(t0 + i / F) * F + (i % F)] = sout[i];
+        if (threadIdx.x < nt) {
+            float e = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < kW; ++ww) e += red[threadIdx.x * kW + ww];
+            a.e_part[(int64_t)slice * rows + rowi(t0 + threadIdx.x)] = e;
         }
         __syncthreads();
     }
@@ -459,15 +509,16 @@ cudaError_t run_passes(const BwdArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)a.ns, (unsigned)(a.B * a.H));
     const size_t smem = sizeof(float) * (size_t)(3 * kTB * a.F + 2 * kTB * 32 + 3 * kTB + kTB * kW * 32);
     cudaError_t e;
-    auto k1 = bwd_pass_kernel<1, TIO>;
-    auto k2 = bwd_pass_kernel<2, TIO>;
-    for (auto k : {k1, k2}) {
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
+    auto k1 = bwd_pa_kernel<TIO>;
+    auto k2 = bwd_pb_kernel<TIO>;
+    const size_t smem1 = sizeof(float) * (size_t)(3 * kTB * a.F + 2 * kTB * 32 + 2 * kTB + kTB * kW);
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     const unsigned zgrid = (unsigned)(a.B * a.H);
     bwd_z_kernel<0><<<zgrid, 256, 0, s>>>(a);
-    k1<<<grid, 32 * kW, smem, s>>>(a);
+    k1<<<grid, 256, smem1, s>>>(a);
     bwd_z_kernel<1><<<zgrid, 256, 0, s>>>(a);
     k2<<<grid, 32 * kW, smem, s>>>(a);
     bwd_z_kernel<2><<<zgrid, 256, 0, s>>>(a);
