@@ -935,12 +935,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 const float *__restrict__ zq = X->zb[(it - 1) & 1] + qf * 64;
                 float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll 1
-                for (int k0 = 0; k0 < 8; k0 += 4) {
-                    uint4 v[4];
+                for (int k0 = 0; k0 < 8; k0 += 2) {
+                    uint4 v[2];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) v[k] = *reinterpret_cast<const uint4 *>(qb + sw128_off(i, k0 + k));
+                    for (int k = 0; k < 2; ++k) v[k] = *reinterpret_cast<const uint4 *>(qb + sw128_off(i, k0 + k));
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
+                    for (int k = 0; k < 2; ++k) {
                         uint32_t *pv = reinterpret_cast<uint32_t *>(&v[k]);
                         const float4 za = *reinterpret_cast<const float4 *>(zq + (k0 + k) * 8);
                         const float4 zb = *reinterpret_cast<const float4 *>(zq + (k0 + k) * 8 + 4);
@@ -953,7 +953,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         }
                     }
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4 *>(qb + sw128_off(i, k0 + k)) = v[k];
+                    for (int k = 0; k < 2; ++k) *reinterpret_cast<uint4 *>(qb + sw128_off(i, k0 + k)) = v[k];
                 }
                 X->dotq[qf][i] = d2.x + d2.y;
             }
