@@ -6,7 +6,8 @@
 // kernel, one CTA per SM: 128 x 256 output tiles, 64-wide K blocks streamed by
 // TMA through a 4-stage ring, tcgen05.mma (bf16 -> fp32 in TMEM) issued by one
 // thread, and two TMEM accumulators so that the epilogue of one tile overlaps
-// the MMAs of the next.  Warp roles: 0 = TMA, 1 = MMA, 2..5 = epilogue.
+// the MMAs of the next.  Warp roles: 0 = TMA, 1 = MMA, 2..9 = epilogue (two
+// warps per TMEM lane quarter, one per half of the tile's 256 columns).
 //
 // The epilogue applies what follows the GEMM in the mixer and the block around
 // it (HedgeMamba explainer sec. 2.3, 5.1, 5.2), so that those steps cost no
@@ -36,6 +37,9 @@ constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 
 constexpr int kMaxConv = 8;   // conv width
+constexpr int kEpiWarps = 8;
+constexpr int kGThreads = 64 + 32 * kEpiWarps;
+constexpr int kHalfN = kBN / 2;   // columns per epilogue warp
 
 struct GAux {
     uint64_t full[kStages], empty[kStages];
@@ -59,7 +63,7 @@ __device__ __forceinline__ float gelu_f(float v) { return 0.5f * v * (1.f + erff
 template <int KC>
 __device__ __forceinline__ void conv_epilogue(GAux *X, uint32_t ta, int b, int64_t m, int64_t n0, int64_t M,
                                               int64_t N, int halo, const GemmEpiArgs &ep, __nv_bfloat16 *C,
-                                              int64_t ldc) {
+                                              int64_t ldc, int cbeg) {
     float wr[KC];   // wr[j]: the weight of token t - j
 #pragma unroll
     for (int j = 0; j < KC; ++j)
@@ -68,17 +72,26 @@ __device__ __forceinline__ void conv_epilogue(GAux *X, uint32_t ta, int b, int64
     float hist[KC - 1 > 0 ? KC - 1 : 1];   // the KC - 1 tokens before the block, oldest first
 #pragma unroll
     for (int j = 0; j < KC - 1; ++j) hist[j] = 0.f;
+    if (cbeg > 0 && KC > 1) {
+        // the second half's window starts with the last columns of the first
+        uint32_t h8[8];
+        tmem_ld8(ta + cbeg - 8, h8);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < KC - 1; ++j) hist[j] = __uint_as_float(h8[8 - (KC - 1) + j]);
+    }
     const int L = (int)ep.seq_len;
     // position in its sequence of the block's first token (negative: the
     // zero-filled tokens before the first)
-    int tpos = n0 >= 0 ? (int)(n0 % ep.seq_len) : (int)n0;
+    const int64_t nb = n0 + cbeg;
+    int tpos = nb >= 0 ? (int)(nb % ep.seq_len) : (int)nb;
     const bool live = m < M;
 #pragma unroll 1
-    for (int c0 = 0; c0 < kBN; c0 += 32) {
+    for (int c0 = cbeg; c0 < cbeg + kHalfN; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(ta + c0, r);
         tmem_wait_ld();
-        if (c0 + 32 >= kBN) {
+        if (c0 + 32 >= cbeg + kHalfN) {
             tc_fence_before();
             mbar_arrive(&X->acce[b]);
         }
@@ -119,7 +132,7 @@ __device__ __forceinline__ void conv_epilogue(GAux *X, uint32_t ta, int b, int64
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                int64_t M, int64_t N, int64_t K, void *__restrict__ C, int64_t ldc, GemmEpiArgs ep,
                DevErr err) {
@@ -144,7 +157,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ 
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&X->accf[b], 1);
-            mbar_init(&X->acce[b], 128);
+            mbar_init(&X->acce[b], 32 * kEpiWarps);
         }
         X->abort = 0;
         mbar_fence_init();
@@ -211,6 +224,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ 
     } else {
         const int q = warp & 3;
         const int row = 32 * q + lane;
+        const int cbeg = ((warp - 2) >> 2) * kHalfN;   // this warp's half of the columns
         int tl = 0;
         for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
             const int b = tl & 1;
@@ -221,18 +235,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ 
             const uint32_t ta = tmem + b * kBN + ((uint32_t)(32 * q) << 16);
             if constexpr (EPI == EPI_CONV_BF16) {
                 if (ep.conv_k == 4)
-                    conv_epilogue<4>(X, ta, b, m, n0, M, N, halo, ep, (__nv_bfloat16 *)C, ldc);
+                    conv_epilogue<4>(X, ta, b, m, n0, M, N, halo, ep, (__nv_bfloat16 *)C, ldc, cbeg);
                 else
-                    conv_epilogue<kMaxConv>(X, ta, b, m, n0, M, N, halo, ep, (__nv_bfloat16 *)C, ldc);
+                    conv_epilogue<kMaxConv>(X, ta, b, m, n0, M, N, halo, ep, (__nv_bfloat16 *)C, ldc, cbeg);
                 continue;
             }
             const bool out_row = m < M;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
+            for (int c0 = cbeg; c0 < cbeg + kHalfN; c0 += 32) {
                 uint32_t r[32];
                 tmem_ld32(ta + c0, r);
                 tmem_wait_ld();
-                if (c0 + 32 >= kBN) {
+                if (c0 + 32 >= cbeg + kHalfN) {
                     tc_fence_before();
                     mbar_arrive(&X->acce[b]);
                 }
@@ -330,7 +344,7 @@ cudaError_t launch_epi(const CUtensorMap &tma, const CUtensorMap &tmb, unsigned 
                        int64_t K, void *C, int64_t ldc, const GemmEpiArgs &ep, DevErr err, cudaStream_t s) {
     cudaError_t e = ensure_smem_limit(gemm_tc_kernel<EPI>, kGSmem);
     if (e != cudaSuccess) return e;
-    gemm_tc_kernel<EPI><<<grid, 192, kGSmem, s>>>(tma, tmb, M, N, K, C, ldc, ep, err);
+    gemm_tc_kernel<EPI><<<grid, kGThreads, kGSmem, s>>>(tma, tmb, M, N, K, C, ldc, ep, err);
     count_launches(1);
     return cudaGetLastError();
 }
