@@ -319,16 +319,24 @@ bwd_z_kernel(BwdArgs a) {
             }
         }
         __syncthreads();
+        // the block's features of this thread, all loads in flight at once
+        float xk[kTB], xq[kTB];
+#pragma unroll
+        for (int t = 0; t < kTB; ++t) {
+            const bool ok = fok && t < nt;
+            xk[t] = (MODE < 2 && ok) ? a.phk[rowi(t0 + t) * F + f] : 0.f;
+            xq[t] = (MODE != 1 && ok) ? a.phq[rowi(t0 + t) * F + f] : 0.f;
+        }
         if (MODE < 2) {
-            for (int t = 0; t < nt; ++t) {
-                const int64_t r = rowi(t0 + t);
-                const float kf = fok ? a.phk[r * F + f] : 0.f;
-                zs = fmaf(sa[t], zs, kf);
+#pragma unroll
+            for (int t = 0; t < kTB; ++t) {
+                if (t >= nt) break;
+                zs = fmaf(sa[t], zs, xk[t]);
                 if (MODE == 0) {
-                    const float p = warp_sum(fok ? a.phq[r * F + f] * zs : 0.f);
+                    const float p = warp_sum(xq[t] * zs);
                     if (lane == 0) red[t][w] = p;
                 } else if (fok) {
-                    a.dq_part[(int64_t)a.ns * rows * F + r * F + f] = zs * sdd[t];
+                    a.dq_part[(int64_t)a.ns * rows * F + rowi(t0 + t) * F + f] = zs * sdd[t];
                 }
             }
             if (MODE == 0) {
@@ -341,11 +349,11 @@ bwd_z_kernel(BwdArgs a) {
                 }
             }
         } else {
-            for (int t = nt - 1; t >= 0; --t) {
-                const int64_t r = rowi(t0 + t);
-                const float qf = fok ? a.phq[r * F + f] : 0.f;
-                zs = fmaf(sa1[t], zs, qf * sdd[t]);
-                if (fok) a.dk_part[(int64_t)a.ns * rows * F + r * F + f] = zs;
+#pragma unroll
+            for (int t = kTB - 1; t >= 0; --t) {
+                if (t >= nt) continue;
+                zs = fmaf(sa1[t], zs, xq[t] * sdd[t]);
+                if (fok) a.dk_part[(int64_t)a.ns * rows * F + rowi(t0 + t) * F + f] = zs;
             }
             if (t0 == 0 && a.dz0 && fok) a.dz0[bh * F + f] = sa[0] * zs;
         }
