@@ -59,11 +59,15 @@ def load_peaks():
 # DRAM bytes per launch of the dominant call from an ncu capture of the
 # current kernel versions (dram__bytes_read.sum + dram__bytes_write.sum,
 # summed over the call's kernels; ncu runs each kernel with cold caches), or
-# None when a kernel changed since the counters were taken.  Prefill
-# B4 H8 L2048: scan_state 33,730,816 + 2,048 + scan_carry 16,865,280 +
-# scan_out 109,435,392 + 10,352,896
-# (profiles/scan_call_traffic_prefill_B4_H8_L2048.md).
-NCU_TRAFFIC_BYTES = {("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 170386432}
+# None when a kernel changed since the counters were taken
+# (profiles/scan_call_traffic.md).  Prefill B4 H8 L2048: scan_state
+# 33,733,888 + 35,072, scan_carry 16,852,992, scan_out 109,465,600 +
+# 7,543,040.  Long context B1 H8 L32768: scan_state 240,059,648 + 3,171,584,
+# scan_carry 16,860,672, scan_out 420,714,240 + 109,503,232.
+NCU_TRAFFIC_BYTES = {
+    ("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 167630592,
+    ("scan_chunked (features precomputed)", "prefill_B1_H8_L32768_d256_F256_bf16"): 790309376,
+}
 
 # ---------------------------------------------------------------- clocks
 
