@@ -233,7 +233,10 @@ HM_API hm_status hm_scan_combine(const hm_combine_args *a, hm_stream_t stream);
  * writes the gradients with respect to q, k, v, W_q, W_k, dt, A_log and,
  * when asked, the initial state.  All gradients are fp32.  With W_q == NULL
  * (q, k are the features, F = d), grad_q and grad_k are the gradients of the
- * features and grad_W_q, grad_W_k are not written.
+ * features and grad_W_q, grad_W_k are not written.  With no tokens
+ * (B * L * H == 0) every given gradient of W_q, W_k, A_log and of the initial
+ * state is zero (grad_A_log is zeroed when A_log is given, even with dt NULL,
+ * since an empty dt tensor may come as NULL).
  * Computed on CUDA cores in fp32 from fp32 features recomputed from q, k.
  */
 typedef struct {

@@ -430,68 +430,191 @@ featmap_bwd_du_kernel(const float *__restrict__ phi, const float *__restrict__ d
         du[r * p + j] = ph[j] * (dp[j] - s) - ph[p + j] * (dp[p + j] - s);
 }
 
-// dx[r, i] = sum_j du[r, j] W[j, i]: one CTA per 32 rows, W read from L2.
-template <typename TW>
-__global__ void __launch_bounds__(256)
-featmap_bwd_dx_kernel(const float *__restrict__ du, const TW *__restrict__ W, int64_t rows, int p, int d,
-                      float *__restrict__ dx) {
-    __shared__ float sdu[32][256];
-    const int64_t r0 = (int64_t)blockIdx.x * 32;
-    for (int i = threadIdx.x; i < 32 * p; i += blockDim.x) {
-        const int rr = i / p, j = i % p;
-        sdu[rr][j] = r0 + rr < rows ? du[(r0 + rr) * p + j] : 0.f;
+// Four consecutive elements of a row as fp32; `valid` of them in bounds (the
+// rest read as 0).  vec: rows start 16-byte (fp32) / 8-byte (bf16) aligned.
+__device__ __forceinline__ float4 ld4(const float *p, int64_t i, int valid, bool vec) {
+    if (vec && valid >= 4) return *reinterpret_cast<const float4 *>(p + i);
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid > 0) r.x = p[i];
+    if (valid > 1) r.y = p[i + 1];
+    if (valid > 2) r.z = p[i + 2];
+    if (valid > 3) r.w = p[i + 3];
+    return r;
+}
+
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p, int64_t i, int valid, bool vec) {
+    if (vec && valid >= 4) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p + i);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < d; i += blockDim.x) {
-        float acc[32];
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid > 0) r.x = __bfloat162float(p[i]);
+    if (valid > 1) r.y = __bfloat162float(p[i + 1]);
+    if (valid > 2) r.z = __bfloat162float(p[i + 2]);
+    if (valid > 3) r.w = __bfloat162float(p[i + 3]);
+    return r;
+}
+
+// The feature map's two gradient products, dx = du W and dW = du^T x, as one
+// register-tiled fp32 contraction C (+)= A B on the CUDA cores: a CTA owns a
+// 128 x 128 tile of C and each thread an 8 x 8 block of it (rows ty*4.. and
+// 64 + ty*4.., columns tx*4.. and 64 + tx*4..), fed from 16-deep slices of A
+// and B in double-buffered shared memory; the next slice's global loads are in
+// flight while the current one's 16 x 64 FMAs run, and each FMA step reads two
+// float4 of A and two of B (four shared loads for 64 FMAs).
+// A is [k][m] (m contiguous; dW, where A = du^T) or, with A_MK, [m][k]
+// (dx, A = du), transposed on its way into shared memory; B is [k][n] with n
+// contiguous; C is [m][n].  Grid: (m tiles, n tiles, k splits); with SPLIT each
+// CTA covers kchunk of k and adds its tile to C (zeroed first) atomically.
+// vec: every leading dimension is a multiple of 4, so groups of 4 that are
+// fully in bounds use vector loads, stores and atomics.
+constexpr int kGM = 128, kGN = 128, kGK = 16, kGS = 132;   // kGS: padded smem row
+
+template <bool A_MK, typename TB, bool SPLIT>
+__global__ void __launch_bounds__(256, 2)
+featmap_bwd_gemm_kernel(const float *__restrict__ A, int64_t lda, const TB *__restrict__ Bm, int64_t ldb,
+                        float *__restrict__ C, int64_t ldc, int64_t M, int64_t N, int64_t K, int64_t kchunk,
+                        bool vec) {
+    __shared__ __align__(16) float As[2][kGK][kGS];
+    __shared__ __align__(16) float Bs[2][kGK][kGS];
+    const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+    const int64_t m0 = (int64_t)blockIdx.x * kGM, n0 = (int64_t)blockIdx.y * kGN;
+    const int64_t kb = SPLIT ? (int64_t)blockIdx.z * kchunk : 0;
+    const int64_t ke = SPLIT ? (kb + kchunk < K ? kb + kchunk : K) : K;
+    auto nvalid = [](int64_t lim, int64_t col) { return (int)(lim - col >= 4 ? 4 : (lim > col ? lim - col : 0)); };
+    // this thread's two groups of 4 in each slice: A (and, with A_MK, its row
+    // bound) and B at slice start k = 0; a slice at k0 adds k0 (A_MK) or
+    // k0 * ld to the pointer
+    const float *pa[2];
+    const TB *pb[2];
+    int64_t acol[2];
+    bool arow_ok[2];
 #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) acc[rr] = 0.f;
-        for (int j = 0; j < p; ++j) {
-            const float wv = hm_ld(W, (int64_t)j * d + i);
-#pragma unroll
-            for (int rr = 0; rr < 32; ++rr) acc[rr] = fmaf(sdu[rr][j], wv, acc[rr]);
+    for (int u = 0; u < 2; ++u) {
+        const int g = t + 256 * u;
+        if (A_MK) {   // four lanes per row of A: 64 contiguous bytes
+            const int64_t row = m0 + (g >> 2);
+            acol[u] = 4 * (g & 3);
+            arow_ok[u] = row < M;
+            pa[u] = A + row * lda + acol[u];
+        } else {
+            acol[u] = m0 + 4 * (g & 31);
+            arow_ok[u] = true;
+            pa[u] = A + (int64_t)(g >> 5) * lda + acol[u];
         }
+        pb[u] = Bm + (int64_t)(g >> 5) * ldb + n0 + 4 * (g & 31);
+    }
+    const int bval = nvalid(N, n0 + 4 * (t & 31));
+    float4 ra[2], rb[2];
+    auto load = [&](int64_t k0) {
 #pragma unroll
-        for (int rr = 0; rr < 32; ++rr)
-            if (r0 + rr < rows) dx[(r0 + rr) * d + i] = acc[rr];
+        for (int u = 0; u < 2; ++u) {
+            const int64_t krow = k0 + (t >> 5) + 8 * u;   // the B row (and A row without A_MK)
+            if (A_MK)
+                ra[u] = ld4(pa[u] + k0, 0, arow_ok[u] ? nvalid(ke, k0 + acol[u]) : 0, vec);
+            else
+                ra[u] = ld4(pa[u] + k0 * lda, 0, krow < ke ? nvalid(M, acol[u]) : 0, vec);
+            rb[u] = ld4(pb[u] + k0 * ldb, 0, krow < ke ? bval : 0, vec);
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int g = t + 256 * u;
+            if (A_MK) {
+                const int m = g >> 2, k = 4 * (g & 3);
+                As[buf][k][m] = ra[u].x;
+                As[buf][k + 1][m] = ra[u].y;
+                As[buf][k + 2][m] = ra[u].z;
+                As[buf][k + 3][m] = ra[u].w;
+            } else {
+                *reinterpret_cast<float4 *>(&As[buf][g >> 5][4 * (g & 31)]) = ra[u];
+            }
+            *reinterpret_cast<float4 *>(&Bs[buf][g >> 5][4 * (g & 31)]) = rb[u];
+        }
+    };
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    const int nst = ke > kb ? (int)((ke - kb + kGK - 1) / kGK) : 0;
+    if (nst == 0) return;   // (a split past the end; the launcher makes none)
+    load(kb);
+    store(0);
+    __syncthreads();
+    for (int s = 0; s < nst; ++s) {
+        const int cur = s & 1;
+        if (s + 1 < nst) load(kb + (int64_t)(s + 1) * kGK);
+#pragma unroll
+        for (int k = 0; k < kGK; ++k) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(&As[cur][k][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&As[cur][k][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[cur][k][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[cur][k][64 + tx * 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        if (s + 1 < nst) store(cur ^ 1);
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t row = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+        if (row >= M) continue;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t col = n0 + h * 64 + tx * 4;
+            const int valid = nvalid(N, col);
+            float *dst = C + row * ldc + col;
+            const float4 v = make_float4(acc[i][4 * h], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
+            if (vec && valid == 4) {
+                if (SPLIT)
+                    atomicAdd(reinterpret_cast<float4 *>(dst), v);
+                else
+                    *reinterpret_cast<float4 *>(dst) = v;
+            } else {
+                const float ve[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (e < valid) {
+                        if (SPLIT)
+                            atomicAdd(dst + e, ve[e]);
+                        else
+                            dst[e] = ve[e];
+                    }
+            }
+        }
     }
 }
 
-// dW[j, i] += sum over the CTA's rows of du[r, j] x[r, i]: CTA = (1024 rows,
-// 32 x 64 tile of dW); partial sums added to dW (zeroed first) atomically.
-template <typename TX>
-__global__ void __launch_bounds__(256)
-featmap_bwd_dw_kernel(const float *__restrict__ du, const TX *__restrict__ x, int64_t rows, int p, int d,
-                      float *__restrict__ dW) {
-    __shared__ float su[32][32];
-    __shared__ float sx[32][64];
-    const int j0 = blockIdx.y * 32, i0 = blockIdx.z * 64;
-    const int64_t r0 = (int64_t)blockIdx.x * 1024;
-    const int tj = threadIdx.x >> 3, ti = (threadIdx.x & 7) * 8;   // thread: dW[j0 + tj][i0 + ti .. +8]
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    for (int64_t rb = r0; rb < r0 + 1024 && rb < rows; rb += 32) {
-        for (int k = threadIdx.x; k < 32 * 32; k += 256) {
-            const int rr = k / 32, jj = k % 32;
-            su[rr][jj] = (rb + rr < rows && j0 + jj < p) ? du[(rb + rr) * p + j0 + jj] : 0.f;
-        }
-        for (int k = threadIdx.x; k < 32 * 64; k += 256) {
-            const int rr = k / 64, ii = k % 64;
-            sx[rr][ii] = (rb + rr < rows && i0 + ii < d) ? hm_ld(x, (rb + rr) * d + i0 + ii) : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int rr = 0; rr < 32; ++rr) {
-            const float uj = su[rr][tj];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(uj, sx[rr][ti + e], acc[e]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-        if (j0 + tj < p && i0 + ti + e < d) atomicAdd(&dW[(int64_t)(j0 + tj) * d + i0 + ti + e], acc[e]);
+// dx = du W ([rows, p] x [p, d]) and dW = du^T x ([p, rows] x [rows, d], k
+// split so that about two CTAs per SM run; dW is zeroed first).
+template <typename T>
+cudaError_t run_featmap_bwd_products(const float *du, const T *W, const T *x, int64_t rows, int p, int d,
+                                     float *dx, float *dW, cudaStream_t s) {
+    const bool vec = p % 4 == 0 && d % 4 == 0;
+    const unsigned nt = (unsigned)((d + kGN - 1) / kGN);
+    dim3 gx((unsigned)((rows + kGM - 1) / kGM), nt, 1);
+    featmap_bwd_gemm_kernel<true, T, false><<<gx, 256, 0, s>>>(du, p, W, d, dx, d, rows, d, p, p, vec);
+    cudaError_t e = cudaMemsetAsync(dW, 0, sizeof(float) * (size_t)p * d, s);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t mt = (p + kGM - 1) / kGM;
+    const int64_t want = (2 * (int64_t)sms + mt * nt - 1) / (mt * nt);
+    int64_t kchunk = (rows + want - 1) / want;
+    kchunk = (kchunk + kGK - 1) / kGK * kGK;
+    dim3 gw((unsigned)mt, nt, (unsigned)((rows + kchunk - 1) / kchunk));
+    featmap_bwd_gemm_kernel<false, T, true><<<gw, 256, 0, s>>>(du, p, x, d, dW, d, p, d, rows, kchunk, vec);
+    count_launches(2);
+    return cudaGetLastError();
 }
 
 // d dt = dlog a * (-sigmoid(dt) e^A_log);  dA_log[h] += sum dlog a * log a.
@@ -554,7 +677,20 @@ size_t scan_bwd_workspace(const ScanBwdCore &c) {
 cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
     const int ns = (c.dv + 31) / 32;
     const int64_t rows = c.B * c.L * c.H;
-    if (rows == 0) return cudaSuccess;
+    if (rows == 0) {
+        // no token reaches an output: the gradients of the weights, of A_log
+        // and of the initial state are zero
+        const size_t BH = (size_t)c.B * c.H;
+        cudaError_t e = cudaSuccess;
+        if (c.W_q && c.dW_q) e = cudaMemsetAsync(c.dW_q, 0, sizeof(float) * (size_t)c.p * c.d, s);
+        if (e == cudaSuccess && c.W_q && c.dW_k) e = cudaMemsetAsync(c.dW_k, 0, sizeof(float) * (size_t)c.p * c.d, s);
+        if (e == cudaSuccess && c.A_log && c.dA_log) e = cudaMemsetAsync(c.dA_log, 0, sizeof(float) * (size_t)c.H, s);
+        if (e == cudaSuccess && c.dS0 && BH > 0) {
+            e = cudaMemsetAsync(c.dS0, 0, sizeof(float) * BH * c.F * c.dv, s);
+            if (e == cudaSuccess) e = cudaMemsetAsync(c.dz0, 0, sizeof(float) * BH * c.F, s);
+        }
+        return e;
+    }
     auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
     char *w = (char *)ws;
     auto take = [&](size_t bytes) { char *p = w; w += r256(bytes); return p; };
@@ -601,8 +737,6 @@ cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
     count_launches(2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (c.W_q) {
-        const unsigned xb = (unsigned)((rows + 31) / 32);
-        dim3 gw((unsigned)((rows + 1023) / 1024), (unsigned)((c.p + 31) / 32), (unsigned)((c.d + 63) / 64));
         const float *dphis[2] = {dphq, dphk};
         const float *phis[2] = {phq, phk};
         const void *xs[2] = {c.q, c.k};
@@ -611,20 +745,13 @@ cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
         float *dWs[2] = {c.dW_q, c.dW_k};
         for (int m = 0; m < 2; ++m) {
             featmap_bwd_du_kernel<<<wb, 256, 0, s>>>(phis[m], dphis[m], rows, c.p, du);
-            if (c.io_dtype == HM_BF16)
-                featmap_bwd_dx_kernel<__nv_bfloat16><<<xb, 256, 0, s>>>(du, (const __nv_bfloat16 *)Ws[m], rows, c.p,
-                                                                         c.d, dxs[m]);
-            else
-                featmap_bwd_dx_kernel<float><<<xb, 256, 0, s>>>(du, (const float *)Ws[m], rows, c.p, c.d, dxs[m]);
-            e = cudaMemsetAsync(dWs[m], 0, sizeof(float) * (size_t)c.p * c.d, s);
+            count_launches(1);
+            e = c.io_dtype == HM_BF16
+                    ? run_featmap_bwd_products(du, (const __nv_bfloat16 *)Ws[m], (const __nv_bfloat16 *)xs[m], rows,
+                                               c.p, c.d, dxs[m], dWs[m], s)
+                    : run_featmap_bwd_products(du, (const float *)Ws[m], (const float *)xs[m], rows, c.p, c.d,
+                                               dxs[m], dWs[m], s);
             if (e != cudaSuccess) return e;
-            if (c.io_dtype == HM_BF16)
-                featmap_bwd_dw_kernel<__nv_bfloat16><<<gw, 256, 0, s>>>(du, (const __nv_bfloat16 *)xs[m], rows, c.p,
-                                                                         c.d, dWs[m]);
-            else
-                featmap_bwd_dw_kernel<float><<<gw, 256, 0, s>>>(du, (const float *)xs[m], rows, c.p, c.d, dWs[m]);
-            count_launches(3);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     } else {
         // caller features: their gradients are dphiq and dphik

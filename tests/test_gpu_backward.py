@@ -105,3 +105,43 @@ def test_backward_initial_state_and_caller_features(hm):
     ddt, dA = oracle.log_decay_bwd(inp["dt"], inp["A_log"], dla)
     _check(got, {"grad_q": dphq, "grad_k": dphk, "grad_v": dvv, "grad_dt": ddt, "grad_A_log": dA,
                  "grad_S0": dS0, "grad_z0": dz0}, TOL_F32)
+
+
+@pytest.mark.parametrize("d,p", [(10, 5), (260, 64)])
+def test_backward_feature_map_products_ragged(hm, d, p):
+    """The feature map's gradient products (dx = du W, dW = du^T x, the latter
+    split over tokens) at sizes off the 128 x 128 tiles: d = 10, p = 5 (no
+    vector loads; 582 rows over five row tiles, dW over 37 token splits) and
+    d = 260 (a column tile with 4 columns)."""
+    cfg = wl.ScanConfig("ragged_featmap", 2, 97, 3, d, p, 8, "f32", True, 131, math.sqrt(1.0 / d))
+    inp = wl.scan_inputs(cfg)
+    dout = wl.round_f32(wl.normal(131, "dout", inp["v"].shape))
+    got = _bwd_gpu(hm, inp, dout, "f32")
+    r = oracle.scan_bwd(inp["q"], inp["k"], inp["v"], inp["W_q"], inp["W_k"], dout, dt=inp["dt"],
+                        A_log=inp["A_log"])
+    _check(got, {"grad_q": r["dq"], "grad_k": r["dk"], "grad_v": r["dv"], "grad_W_q": r["dW_q"],
+                 "grad_W_k": r["dW_k"], "grad_dt": r["ddt"]}, TOL_F32)
+    # grad_A_log[h] = sum over tokens of dlog a_t * log a_t, whose terms cancel
+    # (sum |terms| / |sum| reaches 36 here): an fp32 sum is accurate relative
+    # to the sum of the terms' magnitudes, so that is the scale of the bar
+    la = oracle.log_decay(inp["dt"], inp["A_log"])
+    phq, phk = oracle.featmap(inp["q"], inp["W_q"]), oracle.featmap(inp["k"], inp["W_k"])
+    dla = oracle.scan_recurrent_bwd(phq, phk, inp["v"], dout, la)[3]
+    scale = np.abs(dla * la).sum(axis=(0, 1))
+    assert np.allclose(r["dA_log"], (dla * la).sum(axis=(0, 1)), rtol=1e-12)
+    assert (np.abs(got["grad_A_log"] - r["dA_log"]) <= TOL_F32 * scale).all()
+
+
+def test_backward_empty_sequence_zeroes_parameter_gradients(hm):
+    """L = 0: no token reaches an output, so the gradients of W_q, W_k, A_log
+    and of the initial state are exactly zero (the buffers start as NaN)."""
+    cfg = wl.TINY_F32
+    inp = wl.scan_inputs(cfg, B=2, L=0, seed=132)
+    inp["dt"] = np.zeros((2, 0, cfg.H))
+    inp["A_log"] = wl.round_f32(np.array([0.3, 1.1]))
+    F = 2 * cfg.p
+    S0 = np.full((2, cfg.H, F, cfg.dv), 0.5)
+    z0 = np.full((2, cfg.H, F), 0.25)
+    got = _bwd_gpu(hm, inp, np.zeros(inp["v"].shape), "f32", S0=S0, z0=z0)
+    for name in ("grad_W_q", "grad_W_k", "grad_A_log", "grad_S0", "grad_z0"):
+        assert got[name].size > 0 and (got[name] == 0).all(), name
