@@ -17,18 +17,19 @@
 // key's phik_j . dphik_j.  It needs neither forward nor backward state, so no
 // pass has to hold S and G at once.
 //
-// Passes, each one CTA per (batch, head, 32 value columns) with the state's
-// 256 x 32 slice in registers:
-//   PA forward (a thread per feature row): the slice's shares of
-//      sum_c do_t[c] n_t[c] and of S_t dn_t
-//   PB backward (warp w holds feature rows w, w + 8, ..., lane = column, as
-//      in the CUDA-core forward scan): the slice's share of G_t v_t, dv_t, dS0
-// and three passes over the denominator's state alone, one CTA per (batch,
-// head) with a thread per feature: d_t (before PA), then z_t dd_t (once PA has
-// given do_t . n_t), then g_t and dz0, written as one more share.  Keeping z
-// out of the value-slice passes halves their registers, so two of their CTAs
-// fit on an SM, and PA needs only d_t, not dd_t.
-// then a reduction of the slices' shares (and the suffix sums of dlog a),
+// Passes, each one CTA per (batch, head, 32 value columns), token blocks of
+// 16 copied by cp.async one block ahead:
+//   PA forward (a thread per feature row, the slice's 32 columns of S in its
+//      registers): the slice's shares of sum_c do_t[c] n_t[c] and of S_t dn_t;
+//      the denominator's state z rides along (a thread per feature), so PA
+//      also gives d_t
+//   PB backward (each thread an 8 x 4 block of the slice's G): the slice's
+//      share of G_t v_t, dv_t and dS0
+// and two passes over the denominator's state alone, one CTA per (batch,
+// head), run as extra CTAs of PB's launch: z_t dd_t (once PA has given
+// do_t . n_t and d_t), and g_t and dz0, each written as one more share.
+// Keeping z out of PB halves its registers, so two of its CTAs fit on an SM.
+// Then a reduction of the slices' shares (and the suffix sums of dlog a),
 // the feature-map backward (softmax Jacobian, dx = du W, dW = sum du x^T) and
 // the decay's (d dt = dlog a (-sigmoid(dt) e^A_log), dA_log = sum dlog a * log a).
 #include "hm_internal.h"
@@ -39,7 +40,6 @@ namespace {
 
 constexpr int kW = 8;        // warps
 constexpr int kTB = 16;      // tokens staged per round
-constexpr int kMaxRows = 32; // F <= 256
 
 struct BwdArgs {
     int64_t B, L;
@@ -56,155 +56,128 @@ struct BwdArgs {
     float *dS0, *dz0;        // nullable
 };
 
-// v[m] is this lane's contribution to row m (m = 0..31); afterwards v[0] of
-// lane l is the sum over the warp of row l.  Recursive halving: at step `off`
-// each lane keeps the half of its rows selected by its lane bit `off` and
-// adds the partner's copy of that half (31 shuffles instead of 32 reductions
-// of 5).
-__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int j = 0; j < off; ++j) {
-            const float send = upper ? v[j] : v[j + off];
-            const float keep = upper ? v[j + off] : v[j];
-            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-    }
-    return v[0];
+// ------------------------------------------------------------ token blocks
+
+constexpr int kFP = 256;   // feature stride of a staged row (F <= 256; zero past F)
+
+// cp.async: 16 or 4 bytes global -> shared; the bytes past src_bytes are
+// zero-filled (src_bytes = 0 reads nothing).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
 }
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
-// PB, tokens from the last to the first (the state layout of the forward
-// CUDA-core scan: warp w holds feature rows w, w + 8, ..., lane = column).
+template <typename T>
+__device__ __forceinline__ T zero_of() { return T(0.f); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 zero_of<__nv_bfloat16>() { return __float2bfloat16(0.f); }
+
+// One token block as copied from global memory: the phiq and phik rows
+// (zero past F), the slice's 32 columns of v and do in the io dtype, dt of
+// the block's tokens and of the token after it, and d_t.
 template <typename TIO>
-__global__ void __launch_bounds__(32 * kW, 2)
-bwd_pb_kernel(BwdArgs a) {
-    extern __shared__ float smem[];
-    const int F = a.F, dv = a.dv;
-    float *sq = smem;                      // [kTB][F]
-    float *sk = sq + kTB * F;              // [kTB][F]
-    float *sv = sk + kTB * F;              // [kTB][32]   v
-    float *sg = sv + kTB * 32;             // [kTB][32]   do
-    float *sa = sg + kTB * 32;             // [kTB]       a_t
-    float *sa1 = sa + kTB;                 // [kTB]       a_{t+1} (PB)
-    float *sden = sa1 + kTB;               // [kTB]
-    float *red = sden + kTB;               // [kTB][kW][32]
-    float *sout = red + kTB * kW * 32;     // [kTB][F]: the slice's shares of dphiq / dphik
+struct alignas(16) BwdBlk {
+    float q[kTB][kFP];
+    float k[kTB][kFP];
+    TIO v[kTB][32];
+    TIO g[kTB][32];
+    float dt[kTB + 1];
+    float den[kTB];
+};
 
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int64_t bh = blockIdx.y;
-    const int64_t b = bh / a.H;
-    const int h = (int)(bh % a.H);
-    const int slice = blockIdx.x;
-    const int col = slice * 32 + lane;
-    const bool col_ok = col < dv;
-    const float alog = a.dt ? a.A_log[h] : 0.f;
+// Copies tokens t0 .. t0 + nt - 1 of (b, h) (and dt of token t0 + nt) into
+// bk.  fast: every row starts 16-byte aligned (F % 4 == 0, the slice's rows of
+// v and do a multiple of 16 bytes) and the copies are cp.async, completed by
+// the caller's wait; otherwise plain loads into the same layout.
+template <typename TIO>
+__device__ __forceinline__ void issue_block(BwdBlk<TIO> *bk, const BwdArgs &a, int64_t b, int h, int64_t t0, int nt,
+                                            int c0, bool fast, bool with_den) {
+    const int F = a.F, dv = a.dv, H = a.H;
+    const int64_t L = a.L;
     const TIO *v = (const TIO *)a.v;
     const TIO *dout = (const TIO *)a.dout;
-    const int64_t L = a.L;
-    auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
-
-    float S[kMaxRows];   // G, the adjoint of S, from zero after the last token
-#pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) S[m] = 0.f;
-    const int64_t nblk = (L + kTB - 1) / kTB;
-    for (int64_t bi = 0; bi < nblk; ++bi) {
-        // PB walks the token blocks from the last to the first
-        const int64_t t0 = (nblk - 1 - bi) * kTB;
-        const int nt = (int)((L - t0) < kTB ? (L - t0) : kTB);
-        for (int i = threadIdx.x; i < nt * F; i += blockDim.x) {
-            const int t = i / F, f = i % F;
-            sq[i] = a.phq[rowi(t0 + t) * F + f];
-            sk[i] = a.phk[rowi(t0 + t) * F + f];
+    auto rowi = [&](int64_t t) { return (b * L + t) * H + h; };
+    const int tid = threadIdx.x;
+    if (fast) {
+        for (int c = tid; c < kTB * (kFP / 4); c += blockDim.x) {
+            const int t = c / (kFP / 4), f = (c % (kFP / 4)) * 4;
+            const bool ok = t < nt && f < F;
+            const int64_t off = ok ? rowi(t0 + t) * F + f : 0;
+            cp_async16(&bk->q[t][f], a.phq + off, ok ? 16 : 0);
+            cp_async16(&bk->k[t][f], a.phk + off, ok ? 16 : 0);
         }
-        for (int i = threadIdx.x; i < nt * 32; i += blockDim.x) {
-            const int t = i / 32, c = slice * 32 + (i % 32);
-            const bool ok = c < dv;
-            sv[i] = ok ? hm_ld(v, rowi(t0 + t) * dv + c) : 0.f;
-            sg[i] = ok ? hm_ld(dout, rowi(t0 + t) * dv + c) : 0.f;
+        constexpr int kPer = 16 / (int)sizeof(TIO);   // elements per 16 bytes
+        constexpr int kRow = 32 / kPer;               // 16-byte groups per token
+        for (int c = tid; c < kTB * kRow; c += blockDim.x) {
+            const int t = c / kRow, e = (c % kRow) * kPer;
+            const bool ok = t < nt && c0 + e < dv;
+            const int64_t off = ok ? rowi(t0 + t) * dv + c0 + e : 0;
+            cp_async16(&bk->v[t][e], v + off, ok ? 16 : 0);
+            cp_async16(&bk->g[t][e], dout + off, ok ? 16 : 0);
         }
-        if (threadIdx.x < nt) {
-            const int t = threadIdx.x;
-            const int64_t r = rowi(t0 + t);
-            sa[t] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
-            // a_{t+1}: the decay that carries G_{t+1} back to token t (none after the last token)
-            sa1[t] = (t0 + t + 1 < L && a.dt) ? expf(hm_log_decay(a.dt[rowi(t0 + t + 1)], alog)) : 1.f;
-            sden[t] = a.den[r];
+        if (tid <= kTB && a.dt) {
+            const bool ok = tid <= nt && t0 + tid < L;
+            cp_async4(&bk->dt[tid], a.dt + (ok ? rowi(t0 + tid) : 0), ok ? 4 : 0);
         }
-        __syncthreads();
-        {
-            // PB: G_t = phiq_t dn_t^T + a_{t+1} G_{t+1} (S holds G)
-            for (int t = nt - 1; t >= 0; --t) {
-                const float a1 = sa1[t];
-                const float dn = sg[t * 32 + lane] / sden[t];
-                const float vv = sv[t * 32 + lane];
-                float dvp = 0.f;
-                float x[kMaxRows];
-#pragma unroll
-                for (int m = 0; m < kMaxRows; ++m) {
-                    const int f = w + kW * m;
-                    x[m] = 0.f;
-                    if (f < F) {
-                        const float qf = sq[t * F + f], kf = sk[t * F + f];
-                        S[m] = fmaf(a1, S[m], qf * dn);
-                        dvp = fmaf(S[m], kf, dvp);
-                        x[m] = S[m] * vv;
-                    }
-                }
-                // the slice's share of sum_c G_t[f, c] v_t[c]
-                const float tot = warp_reduce_scatter32(x, lane);
-                const int fl = w + kW * lane;
-                if (fl < F) sout[t * F + fl] = tot;
-                red[(t * kW + w) * 32 + lane] = dvp;
-            }
-            __syncthreads();
-            for (int i = threadIdx.x; i < nt * 32; i += blockDim.x) {
-                const int t = i / 32, c = i % 32;
-                float acc = 0.f;
-                for (int ww = 0; ww < kW; ++ww) acc += red[(t * kW + ww) * 32 + c];
-                const int cc = slice * 32 + c;
-                if (cc < dv) a.dv_out[rowi(t0 + t) * dv + cc] = acc;
-            }
-            {
-                float *dk = a.dk_part + (int64_t)slice * a.B * L * a.H * F;
-                for (int i = threadIdx.x; i < nt * F; i += blockDim.x)
-                    dk[rowi(t0 + i / F) * F + (i % F)] = sout[i];
-            }
-            if (t0 == 0 && a.dS0 && col_ok) {
-                // dS0 = a_1 G_1 (a_1 = the first token's decay)
-                const float a0 = sa[0];
-#pragma unroll
-                for (int m = 0; m < kMaxRows; ++m) {
-                    const int f = w + kW * m;
-                    if (f < F) a.dS0[(bh * F + f) * dv + col] = a0 * S[m];
-                }
-            }
+        if (with_den && tid < kTB) {
+            const bool ok = tid < nt;
+            cp_async4(&bk->den[tid], a.den + (ok ? rowi(t0 + tid) : 0), ok ? 4 : 0);
         }
-        __syncthreads();
+    } else {
+        for (int c = tid; c < kTB * kFP; c += blockDim.x) {
+            const int t = c / kFP, f = c % kFP;
+            const bool ok = t < nt && f < F;
+            bk->q[t][f] = ok ? a.phq[rowi(t0 + t) * F + f] : 0.f;
+            bk->k[t][f] = ok ? a.phk[rowi(t0 + t) * F + f] : 0.f;
+        }
+        for (int c = tid; c < kTB * 32; c += blockDim.x) {
+            const int t = c / 32, e = c % 32;
+            const bool ok = t < nt && c0 + e < dv;
+            bk->v[t][e] = ok ? v[rowi(t0 + t) * dv + c0 + e] : zero_of<TIO>();
+            bk->g[t][e] = ok ? dout[rowi(t0 + t) * dv + c0 + e] : zero_of<TIO>();
+        }
+        if (tid <= kTB && a.dt) bk->dt[tid] = (tid <= nt && t0 + tid < L) ? a.dt[rowi(t0 + tid)] : 0.f;
+        if (with_den && tid < kTB) bk->den[tid] = tid < nt ? a.den[rowi(t0 + tid)] : 0.f;
     }
 }
 
-// PA with a thread per feature row (the 32 columns of the slice in its
-// registers): S_t[f, :] = a_t S_(t-1)[f, :] + phik_t[f] v_t and
-// u_f = sum_c S_t[f, c] do_t[c] stay within the thread; the slice's share of
-// dphiq_t[f] is u_f / d_t and its share of do_t . n_t = sum_f phiq_t[f] u_f
-// is one block reduction per token.
+template <typename TIO>
+__device__ __forceinline__ bool blocks_fast(const BwdArgs &a) {
+    return a.F % 4 == 0 && (a.dv * (int)sizeof(TIO)) % 16 == 0;
+}
+
+// ------------------------------------------------------------ PA
+
+// PA (forward in time), a thread per feature row f with the slice's 32
+// columns of S in registers: S_t[f, :] = a_t S_(t-1)[f, :] + phik_t[f] v_t and
+// u_f = sum_c S_t[f, c] do_t[c] (four partial sums).  The denominator's state
+// z_t[f] = a_t z_(t-1)[f] + phik_t[f] rides along, so d_t = sum_f phiq_t[f]
+// z_t[f] needs no pass of its own.  Per token the thread leaves u_f and
+// phiq_f u_f in place of the block's phiq and phik entries (read by this
+// thread alone) and phiq_f z_f beside them; at the block's end the sums over f
+// give d_t (slice 0 stores it) and the slice's share of do_t . n_t, and the
+// slice's share of dphiq_t[f] is u_f / d_t.  Blocks are copied one ahead.
 template <typename TIO>
 __global__ void __launch_bounds__(256, 2)
 bwd_pa_kernel(BwdArgs a) {
-    extern __shared__ float smem[];
-    const int F = a.F, dv = a.dv;
-    float *sq = smem;                      // [kTB][F]
-    float *sk = sq + kTB * F;              // [kTB][F]
-    float *sv = sk + kTB * F;              // [kTB][32]   v
-    float *sg = sv + kTB * 32;             // [kTB][32]   do
-    float *sa = sg + kTB * 32;             // [kTB]       a_t
-    float *sden = sa + kTB;                // [kTB]
-    float *red = sden + kTB;               // [kTB][kW]
-    float *sout = red + kTB * kW;          // [kTB][F]
+    extern __shared__ __align__(16) uint8_t smem_pa[];
+    BwdBlk<TIO> *blk = reinterpret_cast<BwdBlk<TIO> *>(smem_pa);   // two buffers
+    float *sqz = reinterpret_cast<float *>(blk + 2);               // [kTB][kFP] phiq z
+    float *sv = sqz + kTB * kFP;                                   // [kTB][32]
+    float *sg = sv + kTB * 32;                                     // [kTB][32]
+    float *sa = sg + kTB * 32;                                     // [kTB] a_t
+    float *sden = sa + kTB;                                        // [kTB] d_t
 
     const int f = threadIdx.x, lane = f & 31, w = f >> 5;
+    const int F = a.F, dv = a.dv;
     const bool fok = f < F;
     const int64_t bh = blockIdx.y;
     const int64_t b = bh / a.H;
@@ -213,40 +186,39 @@ bwd_pa_kernel(BwdArgs a) {
     const int c0 = slice * 32;
     const int ncol = dv - c0 < 32 ? dv - c0 : 32;
     const float alog = a.dt ? a.A_log[h] : 0.f;
-    const TIO *v = (const TIO *)a.v;
-    const TIO *dout = (const TIO *)a.dout;
     const int64_t L = a.L;
     const int64_t rows = a.B * L * a.H;
     auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
+    const bool fast = blocks_fast<TIO>(a);
 
     float S[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) S[c] = (a.S0 && fok && c < ncol) ? a.S0[(bh * F + f) * dv + c0 + c] : 0.f;
+    float z = (a.z0 && fok) ? a.z0[bh * F + f] : 0.f;
+    float *dq = a.dq_part + (int64_t)slice * rows * F;
     const int64_t nblk = (L + kTB - 1) / kTB;
+    auto ntok = [&](int64_t t0) { return (int)(L - t0 < kTB ? L - t0 : kTB); };
+    issue_block(&blk[0], a, b, h, 0, ntok(0), c0, fast, false);
+    cp_async_commit();
     for (int64_t bi = 0; bi < nblk; ++bi) {
         const int64_t t0 = bi * kTB;
-        const int nt = (int)((L - t0) < kTB ? (L - t0) : kTB);
-        for (int i = threadIdx.x; i < nt * F; i += blockDim.x) {
-            const int t = i / F, ff = i % F;
-            sq[i] = a.phq[rowi(t0 + t) * F + ff];
-            sk[i] = a.phk[rowi(t0 + t) * F + ff];
-        }
-        for (int i = threadIdx.x; i < nt * 32; i += blockDim.x) {
-            const int t = i / 32, c = i % 32;
-            const bool ok = c < ncol;
-            sv[i] = ok ? hm_ld(v, rowi(t0 + t) * dv + c0 + c) : 0.f;
-            sg[i] = ok ? hm_ld(dout, rowi(t0 + t) * dv + c0 + c) : 0.f;
-        }
-        if (threadIdx.x < nt) {
-            const int64_t r = rowi(t0 + threadIdx.x);
-            sa[threadIdx.x] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
-            sden[threadIdx.x] = a.den[r];
+        const int nt = ntok(t0);
+        BwdBlk<TIO> *bk = &blk[bi & 1];
+        if (bi + 1 < nblk) issue_block(&blk[(bi + 1) & 1], a, b, h, t0 + kTB, ntok(t0 + kTB), c0, fast, false);
+        cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        if (f < nt) sa[f] = a.dt ? expf(hm_log_decay(bk->dt[f], alog)) : 1.f;
+        for (int i = f; i < kTB * 32; i += blockDim.x) {
+            sv[i] = hm_ld(&bk->v[0][0], i);
+            sg[i] = hm_ld(&bk->g[0][0], i);
         }
         __syncthreads();
         for (int t = 0; t < nt; ++t) {
             const float at = sa[t];
-            const float kf = fok ? sk[t * F + f] : 0.f;
-            float u = 0.f;
+            const float qf = bk->q[t][f], kf = bk->k[t][f];
+            z = fmaf(at, z, kf);
+            float u0 = 0.f, u1 = 0.f, u2 = 0.f, u3 = 0.f;
             const float4 *v4 = reinterpret_cast<const float4 *>(sv + t * 32);
             const float4 *g4 = reinterpret_cast<const float4 *>(sg + t * 32);
 #pragma unroll
@@ -256,42 +228,55 @@ bwd_pa_kernel(BwdArgs a) {
                 S[4 * c4 + 1] = fmaf(at, S[4 * c4 + 1], kf * vv.y);
                 S[4 * c4 + 2] = fmaf(at, S[4 * c4 + 2], kf * vv.z);
                 S[4 * c4 + 3] = fmaf(at, S[4 * c4 + 3], kf * vv.w);
-                u = fmaf(S[4 * c4 + 0], gg.x, u);
-                u = fmaf(S[4 * c4 + 1], gg.y, u);
-                u = fmaf(S[4 * c4 + 2], gg.z, u);
-                u = fmaf(S[4 * c4 + 3], gg.w, u);
+                u0 = fmaf(S[4 * c4 + 0], gg.x, u0);
+                u1 = fmaf(S[4 * c4 + 1], gg.y, u1);
+                u2 = fmaf(S[4 * c4 + 2], gg.z, u2);
+                u3 = fmaf(S[4 * c4 + 3], gg.w, u3);
             }
-            if (fok) sout[t * F + f] = u / sden[t];
-            const float ep = warp_sum(fok ? sq[t * F + f] * u : 0.f);
-            if (lane == 0) red[t * kW + w] = ep;
+            const float u = (u0 + u1) + (u2 + u3);
+            bk->q[t][f] = u;
+            bk->k[t][f] = qf * u;
+            sqz[t * kFP + f] = qf * z;
         }
         __syncthreads();
-        float *dq = a.dq_part + (int64_t)slice * rows * F;
-        for (int i = threadIdx.x; i < nt * F; i += blockDim.x) dq[rowi(t0 + i / F) * F + (i % F)] = sout[i];
-        if (threadIdx.x < nt) {
-            float e = 0.f;
+        // per token (warp w: tokens w, w + 8): d_t = sum_f phiq z and the
+        // slice's share of do . n = sum_f phiq u
+        for (int tt = w; tt < nt; tt += kW) {
+            float d = 0.f, e = 0.f;
 #pragma unroll
-            for (int ww = 0; ww < kW; ++ww) e += red[threadIdx.x * kW + ww];
-            a.e_part[(int64_t)slice * rows + rowi(t0 + threadIdx.x)] = e;
+            for (int j = 0; j < kFP / 32; ++j) {
+                d += sqz[tt * kFP + lane + 32 * j];
+                e += bk->k[tt][lane + 32 * j];
+            }
+            d = warp_sum(d);
+            e = warp_sum(e);
+            if (lane == 0) {
+                sden[tt] = d;
+                const int64_t r = rowi(t0 + tt);
+                a.e_part[(int64_t)slice * rows + r] = e;
+                if (slice == 0) a.den[r] = d;
+            }
         }
+        __syncthreads();
+        if (fok)
+            for (int t = 0; t < nt; ++t) dq[rowi(t0 + t) * F + f] = bk->q[t][f] / sden[t];
+        // the buffer is copied into again two blocks on
         __syncthreads();
     }
 }
 
-// The denominator's state z alone, one CTA per (batch, head), thread f =
-// feature f (the same three passes as above):
-//   MODE 0 forward:  z_t = a_t z_(t-1) + phik_t, d_t = phiq_t . z_t
+// ------------------------------------------------------------ z passes
+
+// The denominator's state alone for one (batch, head), thread f = feature f:
 //   MODE 1 forward:  z_t again; its share of dphiq_t is z_t dd_t
 //   MODE 2 backward: g_t = a_(t+1) g_(t+1) + phiq_t dd_t, its share of dphik_t;
 //                    dz0 = a_1 g_1
-// The shares go to plane ns of dq_part / dk_part, after the value slices'.
+// (dd_t = -(do_t . o_t) / d_t = -(do_t . n_t) / d_t^2).  The shares go to
+// plane ns of dq_part / dk_part, after the value slices'.
 template <int MODE>
-__global__ void __launch_bounds__(256)
-bwd_z_kernel(BwdArgs a) {
+__device__ __forceinline__ void bwd_z_pass(const BwdArgs &a, int64_t bh) {
     __shared__ float sa[kTB], sa1[kTB], sdd[kTB];
-    __shared__ float red[kTB][kW];
-    const int f = threadIdx.x, lane = f & 31, w = f >> 5;
-    const int64_t bh = blockIdx.x;
+    const int f = threadIdx.x;
     const int64_t b = bh / a.H;
     const int h = (int)(bh % a.H);
     const int F = a.F;
@@ -300,7 +285,7 @@ bwd_z_kernel(BwdArgs a) {
     const int64_t L = a.L;
     const int64_t rows = a.B * L * a.H;
     auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
-    float zs = (MODE < 2 && a.z0 && fok) ? a.z0[bh * F + f] : 0.f;
+    float zs = (MODE == 1 && a.z0 && fok) ? a.z0[bh * F + f] : 0.f;
     const int64_t nblk = (L + kTB - 1) / kTB;
     for (int64_t bi = 0; bi < nblk; ++bi) {
         const int64_t t0 = (MODE == 2 ? nblk - 1 - bi : bi) * kTB;
@@ -311,52 +296,185 @@ bwd_z_kernel(BwdArgs a) {
             const int64_t r = rowi(t0 + t);
             sa[t] = a.dt ? expf(hm_log_decay(a.dt[r], alog)) : 1.f;
             sa1[t] = (t0 + t + 1 < L && a.dt) ? expf(hm_log_decay(a.dt[rowi(t0 + t + 1)], alog)) : 1.f;
-            if (MODE >= 1) {
-                const float d = a.den[r];
-                float e = 0.f;
-                for (int s = 0; s < a.ns; ++s) e += a.e_part[(int64_t)s * rows + r];
-                sdd[t] = -e / (d * d);   // dd = -(do . o) / d = -(do . n) / d^2
-            }
+            const float d = a.den[r];
+            float e = 0.f;
+            for (int s = 0; s < a.ns; ++s) e += a.e_part[(int64_t)s * rows + r];
+            sdd[t] = -e / (d * d);
         }
         __syncthreads();
         // the block's features of this thread, all loads in flight at once
-        float xk[kTB], xq[kTB];
+        float x[kTB];
 #pragma unroll
         for (int t = 0; t < kTB; ++t) {
             const bool ok = fok && t < nt;
-            xk[t] = (MODE < 2 && ok) ? a.phk[rowi(t0 + t) * F + f] : 0.f;
-            xq[t] = (MODE != 1 && ok) ? a.phq[rowi(t0 + t) * F + f] : 0.f;
+            x[t] = ok ? (MODE == 1 ? a.phk : a.phq)[rowi(t0 + t) * F + f] : 0.f;
         }
-        if (MODE < 2) {
+        if (MODE == 1) {
 #pragma unroll
             for (int t = 0; t < kTB; ++t) {
                 if (t >= nt) break;
-                zs = fmaf(sa[t], zs, xk[t]);
-                if (MODE == 0) {
-                    const float p = warp_sum(xq[t] * zs);
-                    if (lane == 0) red[t][w] = p;
-                } else if (fok) {
-                    a.dq_part[(int64_t)a.ns * rows * F + rowi(t0 + t) * F + f] = zs * sdd[t];
-                }
-            }
-            if (MODE == 0) {
-                __syncthreads();
-                if (threadIdx.x < nt) {
-                    float d = 0.f;
-#pragma unroll
-                    for (int ww = 0; ww < kW; ++ww) d += red[threadIdx.x][ww];
-                    a.den[rowi(t0 + threadIdx.x)] = d;
-                }
+                zs = fmaf(sa[t], zs, x[t]);
+                if (fok) a.dq_part[(int64_t)a.ns * rows * F + rowi(t0 + t) * F + f] = zs * sdd[t];
             }
         } else {
 #pragma unroll
             for (int t = kTB - 1; t >= 0; --t) {
                 if (t >= nt) continue;
-                zs = fmaf(sa1[t], zs, xq[t] * sdd[t]);
+                zs = fmaf(sa1[t], zs, x[t] * sdd[t]);
                 if (fok) a.dk_part[(int64_t)a.ns * rows * F + rowi(t0 + t) * F + f] = zs;
             }
             if (t0 == 0 && a.dz0 && fok) a.dz0[bh * F + f] = sa[0] * zs;
         }
+    }
+}
+
+// ------------------------------------------------------------ PB
+
+// PB (backward in time) over a 32-column slice: G_t = phiq_t dn_t^T +
+// a_(t+1) G_(t+1), the slice's share of G_t v_t (a row sum), dv_t = G_t^T
+// phik_t (a column sum) and dS0 = a_1 G_1.  Each thread holds an 8 x 4 block
+// of G (rows 32 w + 8 (lane >> 3) .., columns 4 (lane & 7) ..), so a row sum
+// is a reduce-scatter over 8 lanes and a column sum one over 4 lanes (then
+// over the warps at the block's end); the warp's sums go in place of its own
+// rows of the block's phiq and phik (read by this warp alone).  Blocks are
+// copied one ahead, from the last to the first.
+// The grid's first 2 B H CTAs run the z passes (modes 1 and 2), which need
+// what PA wrote and nothing of PB, on the SMs the slices leave free.
+template <typename TIO>
+__global__ void __launch_bounds__(256, 2)
+bwd_pb_kernel(BwdArgs a) {
+    const int64_t BH = a.B * a.H;
+    if ((int64_t)blockIdx.x < 2 * BH) {
+        if ((int64_t)blockIdx.x < BH)
+            bwd_z_pass<1>(a, blockIdx.x);
+        else
+            bwd_z_pass<2>(a, blockIdx.x - BH);
+        return;
+    }
+    extern __shared__ __align__(16) uint8_t smem_pb[];
+    BwdBlk<TIO> *blk = reinterpret_cast<BwdBlk<TIO> *>(smem_pb);   // two buffers
+    float *sdn = reinterpret_cast<float *>(blk + 2);               // [kTB][32] do / d
+    float *sv = sdn + kTB * 32;                                    // [kTB][32]
+    float *sa1 = sv + kTB * 32;                                    // [kTB] a_(t+1)
+    float *sa0 = sa1 + kTB;                                        // a of the first token
+
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int rgl = lane >> 3, cg = lane & 7;
+    const int r0 = 32 * w + 8 * rgl, cc = 4 * cg;
+    const int64_t idx = (int64_t)blockIdx.x - 2 * BH;
+    const int slice = (int)(idx % a.ns);
+    const int64_t bh = idx / a.ns;
+    const int64_t b = bh / a.H;
+    const int h = (int)(bh % a.H);
+    const int F = a.F, dv = a.dv;
+    const int c0 = slice * 32;
+    const float alog = a.dt ? a.A_log[h] : 0.f;
+    const int64_t L = a.L;
+    const int64_t rows = a.B * L * a.H;
+    auto rowi = [&](int64_t t) { return (b * L + t) * a.H + h; };
+    const bool fast = blocks_fast<TIO>(a);
+    float *dk = a.dk_part + (int64_t)slice * rows * F;
+
+    float G[8][4];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) G[r][c] = 0.f;
+    const int64_t nblk = (L + kTB - 1) / kTB;
+    auto first = [&](int64_t bi) { return (nblk - 1 - bi) * kTB; };
+    auto ntok = [&](int64_t t0) { return (int)(L - t0 < kTB ? L - t0 : kTB); };
+    issue_block(&blk[0], a, b, h, first(0), ntok(first(0)), c0, fast, true);
+    cp_async_commit();
+    for (int64_t bi = 0; bi < nblk; ++bi) {
+        const int64_t t0 = first(bi);
+        const int nt = ntok(t0);
+        BwdBlk<TIO> *bk = &blk[bi & 1];
+        if (bi + 1 < nblk) issue_block(&blk[(bi + 1) & 1], a, b, h, first(bi + 1), kTB, c0, fast, true);
+        cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        if (tid < nt)
+            sa1[tid] = (a.dt && t0 + tid + 1 < L) ? expf(hm_log_decay(bk->dt[tid + 1], alog)) : 1.f;
+        if (tid == 0 && t0 == 0) sa0[0] = a.dt ? expf(hm_log_decay(bk->dt[0], alog)) : 1.f;
+        for (int i = tid; i < kTB * 32; i += blockDim.x) {
+            const int t = i / 32;
+            sv[i] = hm_ld(&bk->v[0][0], i);
+            sdn[i] = t < nt ? hm_ld(&bk->g[0][0], i) / bk->den[t] : 0.f;
+        }
+        __syncthreads();
+        for (int t = nt - 1; t >= 0; --t) {
+            const float a1 = sa1[t];
+            const float4 qa = *reinterpret_cast<const float4 *>(&bk->q[t][r0]);
+            const float4 qb = *reinterpret_cast<const float4 *>(&bk->q[t][r0 + 4]);
+            const float4 ka = *reinterpret_cast<const float4 *>(&bk->k[t][r0]);
+            const float4 kb = *reinterpret_cast<const float4 *>(&bk->k[t][r0 + 4]);
+            const float4 d4v = *reinterpret_cast<const float4 *>(sdn + t * 32 + cc);
+            const float4 v4v = *reinterpret_cast<const float4 *>(sv + t * 32 + cc);
+            const float q8[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+            const float k8[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+            const float dn[4] = {d4v.x, d4v.y, d4v.z, d4v.w};
+            const float vv[4] = {v4v.x, v4v.y, v4v.z, v4v.w};
+            float x[8], y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                x[r] = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    G[r][c] = fmaf(q8[r], dn[c], a1 * G[r][c]);
+                    x[r] = fmaf(G[r][c], vv[c], x[r]);
+                    y[c] = fmaf(G[r][c], k8[r], y[c]);
+                }
+            }
+            // row sums over the 8 lanes of a row group (lane bits 0..2): lane
+            // ends with row r0 + cg = 32 w + lane
+#pragma unroll
+            for (int off = 4; off >= 1; off >>= 1) {
+                const bool upper = (lane & off) != 0;
+#pragma unroll
+                for (int j = 0; j < off; ++j) {
+                    const float send = upper ? x[j] : x[j + off];
+                    const float keep = upper ? x[j + off] : x[j];
+                    x[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+            }
+            // column sums over the warp's 4 row groups (lane bits 4, 3): lane
+            // ends with column cc + rgl
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const int off = 16 >> s, half = 2 >> s;
+                const bool upper = (lane & off) != 0;
+#pragma unroll
+                for (int j = 0; j < half; ++j) {
+                    const float send = upper ? y[j] : y[j + half];
+                    const float keep = upper ? y[j + half] : y[j];
+                    y[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                }
+            }
+            bk->q[t][32 * w + lane] = x[0];
+            bk->k[t][32 * w + cc + rgl] = y[0];
+        }
+        __syncthreads();
+        // dv_t = the warps' column sums; the slice's share of dphik_t
+        for (int i = tid; i < nt * 32; i += blockDim.x) {
+            const int t = i / 32, c = i % 32;
+            float acc = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < kW; ++ww) acc += bk->k[t][32 * ww + c];
+            if (c0 + c < dv) a.dv_out[rowi(t0 + t) * dv + c0 + c] = acc;
+        }
+        if (tid < F)
+            for (int t = 0; t < nt; ++t) dk[rowi(t0 + t) * F + tid] = bk->q[t][tid];
+        if (t0 == 0 && a.dS0) {
+            // dS0 = a_1 G_1 (a_1 = the first token's decay)
+            const float a0 = sa0[0];
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (r0 + r < F && c0 + cc + c < dv) a.dS0[(bh * F + r0 + r) * dv + c0 + cc + c] = a0 * G[r][c];
+        }
+        // the buffer is copied into again two blocks on
+        __syncthreads();
     }
 }
 
@@ -637,23 +755,18 @@ decay_bwd_kernel(const float *__restrict__ dt, const float *__restrict__ A_log, 
 
 template <typename TIO>
 cudaError_t run_passes(const BwdArgs &a, cudaStream_t s) {
-    dim3 grid((unsigned)a.ns, (unsigned)(a.B * a.H));
-    const size_t smem = sizeof(float) * (size_t)(3 * kTB * a.F + 2 * kTB * 32 + 3 * kTB + kTB * kW * 32);
-    cudaError_t e;
+    const int64_t BH = a.B * a.H;
     auto k1 = bwd_pa_kernel<TIO>;
     auto k2 = bwd_pb_kernel<TIO>;
-    const size_t smem1 = sizeof(float) * (size_t)(3 * kTB * a.F + 2 * kTB * 32 + 2 * kTB + kTB * kW);
-    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    const size_t smem1 = 2 * sizeof(BwdBlk<TIO>) + sizeof(float) * (size_t)(kTB * kFP + 2 * kTB * 32 + 2 * kTB);
+    const size_t smem2 = 2 * sizeof(BwdBlk<TIO>) + sizeof(float) * (size_t)(2 * kTB * 32 + kTB + 4);
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
     if (e != cudaSuccess) return e;
-    const unsigned zgrid = (unsigned)(a.B * a.H);
-    bwd_z_kernel<0><<<zgrid, 256, 0, s>>>(a);
-    k1<<<grid, 256, smem1, s>>>(a);
-    bwd_z_kernel<1><<<zgrid, 256, 0, s>>>(a);
-    k2<<<grid, 32 * kW, smem, s>>>(a);
-    bwd_z_kernel<2><<<zgrid, 256, 0, s>>>(a);
-    count_launches(5);
+    k1<<<dim3((unsigned)a.ns, (unsigned)BH), 256, smem1, s>>>(a);
+    k2<<<(unsigned)(2 * BH + (int64_t)a.ns * BH), 256, smem2, s>>>(a);
+    count_launches(2);
     return cudaGetLastError();
 }
 
