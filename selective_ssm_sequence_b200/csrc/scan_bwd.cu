@@ -174,7 +174,7 @@ bwd_pa_kernel(BwdArgs a) {
     float *sv = sqz + kTB * kFP;                                   // [kTB][32]
     float *sg = sv + kTB * 32;                                     // [kTB][32]
     float *sa = sg + kTB * 32;                                     // [kTB] a_t
-    float *sden = sa + kTB;                                        // [kTB] d_t
+    float *sden = sa + kTB;                                        // [kTB] 1 / d_t
 
     const int f = threadIdx.x, lane = f & 31, w = f >> 5;
     const int F = a.F, dv = a.dv;
@@ -251,7 +251,7 @@ bwd_pa_kernel(BwdArgs a) {
             d = warp_sum(d);
             e = warp_sum(e);
             if (lane == 0) {
-                sden[tt] = d;
+                sden[tt] = 1.f / d;
                 const int64_t r = rowi(t0 + tt);
                 a.e_part[(int64_t)slice * rows + r] = e;
                 if (slice == 0) a.den[r] = d;
@@ -259,7 +259,7 @@ bwd_pa_kernel(BwdArgs a) {
         }
         __syncthreads();
         if (fok)
-            for (int t = 0; t < nt; ++t) dq[rowi(t0 + t) * F + f] = bk->q[t][f] / sden[t];
+            for (int t = 0; t < nt; ++t) dq[rowi(t0 + t) * F + f] = bk->q[t][f] * sden[t];
         // the buffer is copied into again two blocks on
         __syncthreads();
     }
@@ -478,25 +478,59 @@ bwd_pb_kernel(BwdArgs a) {
     }
 }
 
-// dphiq, dphik = sums of the slices' shares, and kd_r = phik_r . dphik_r;
-// one warp per row (lanes over the features).
+// dphiq, dphik = sums of the slices' shares (and the denominator's, plane
+// ns), and kd_r = phik_r . dphik_r; one warp per row, lanes over groups of 4
+// features, the planes' loads of a group issued together (up to 9 at a
+// time) and added in plane order.
 __global__ void __launch_bounds__(256)
 bwd_reduce_kernel(BwdArgs a, float *__restrict__ dphq, float *__restrict__ dphk, float *__restrict__ kd) {
+    constexpr int kPl = 9;
     const int lane = threadIdx.x & 31;
     const int64_t rows = a.B * a.L * a.H;
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (r >= rows) return;
-    const int64_t plane = rows * (int64_t)a.F;
+    const int F = a.F, ns = a.ns;
+    const int64_t plane = rows * (int64_t)F;
+    const float *__restrict__ pq = a.dq_part + r * F;
+    const float *__restrict__ pk = a.dk_part + r * F;
     float acc = 0.f;
-    for (int f = lane; f < a.F; f += 32) {
-        float sq = 0.f, sk = 0.f;
-        for (int s = 0; s <= a.ns; ++s) {
-            sq += a.dq_part[s * plane + r * a.F + f];
-            sk += a.dk_part[s * plane + r * a.F + f];
+    if (F % 4 == 0) {
+        for (int f = 4 * lane; f < F; f += 128) {
+            float4 sq = make_float4(0.f, 0.f, 0.f, 0.f), sk = sq;
+            for (int s0 = 0; s0 <= ns; s0 += kPl) {
+                float4 vq[kPl], vk[kPl];
+#pragma unroll
+                for (int j = 0; j < kPl; ++j) {
+                    const bool ok = s0 + j <= ns;
+                    vq[j] = ok ? __ldcs(reinterpret_cast<const float4 *>(pq + (s0 + j) * plane + f)) : sq;
+                    vk[j] = ok ? __ldcs(reinterpret_cast<const float4 *>(pk + (s0 + j) * plane + f)) : sk;
+                }
+#pragma unroll
+                for (int j = 0; j < kPl; ++j) {
+                    if (s0 + j > ns) break;
+                    sq.x += vq[j].x; sq.y += vq[j].y; sq.z += vq[j].z; sq.w += vq[j].w;
+                    sk.x += vk[j].x; sk.y += vk[j].y; sk.z += vk[j].z; sk.w += vk[j].w;
+                }
+            }
+            *reinterpret_cast<float4 *>(dphq + r * F + f) = sq;
+            *reinterpret_cast<float4 *>(dphk + r * F + f) = sk;
+            const float4 k4 = *reinterpret_cast<const float4 *>(a.phk + r * F + f);
+            acc = fmaf(k4.x, sk.x, acc);
+            acc = fmaf(k4.y, sk.y, acc);
+            acc = fmaf(k4.z, sk.z, acc);
+            acc = fmaf(k4.w, sk.w, acc);
         }
-        dphq[r * a.F + f] = sq;
-        dphk[r * a.F + f] = sk;
-        acc = fmaf(a.phk[r * a.F + f], sk, acc);
+    } else {
+        for (int f = lane; f < F; f += 32) {
+            float sq = 0.f, sk = 0.f;
+            for (int s = 0; s <= ns; ++s) {
+                sq += pq[s * plane + f];
+                sk += pk[s * plane + f];
+            }
+            dphq[r * F + f] = sq;
+            dphk[r * F + f] = sk;
+            acc = fmaf(a.phk[r * F + f], sk, acc);
+        }
     }
     acc = warp_sum(acc);
     if (lane == 0) kd[r] = acc;
