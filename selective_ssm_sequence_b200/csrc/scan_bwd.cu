@@ -567,10 +567,13 @@ __global__ void to_f32_kernel(const T *__restrict__ x, int64_t n, float *__restr
 }
 
 // Feature-map backward, per row: phi = softmax([u, -u]), so
-// de = phi (.) (dphi - sum(phi (.) dphi)), du = de[:p] - de[p:].  One warp per row.
+// de = phi (.) (dphi - sum(phi (.) dphi)), du = de[:p] - de[p:].  One warp per
+// row.  With dus, du is also written as bf16 segments [hi | lo (| hi)] of
+// a row of nseg * p (hi = du rounded to bf16, lo = the rounded remainder):
+// the A operand of dx = du W on the tensor cores.
 __global__ void __launch_bounds__(256)
 featmap_bwd_du_kernel(const float *__restrict__ phi, const float *__restrict__ dphi, int64_t rows, int p,
-                      float *__restrict__ du) {
+                      float *__restrict__ du, __nv_bfloat16 *__restrict__ dus, int nseg) {
     const int lane = threadIdx.x & 31;
     const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (r >= rows) return;
@@ -578,8 +581,36 @@ featmap_bwd_du_kernel(const float *__restrict__ phi, const float *__restrict__ d
     float s = 0.f;
     for (int f = lane; f < 2 * p; f += 32) s = fmaf(ph[f], dp[f], s);
     s = warp_sum(s);
-    for (int j = lane; j < p; j += 32)
-        du[r * p + j] = ph[j] * (dp[j] - s) - ph[p + j] * (dp[p + j] - s);
+    for (int j = lane; j < p; j += 32) {
+        const float x = ph[j] * (dp[j] - s) - ph[p + j] * (dp[p + j] - s);
+        du[r * p + j] = x;
+        if (dus) {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+            __nv_bfloat16 *row = dus + r * nseg * p;
+            row[j] = hi;
+            row[p + j] = lo;
+            if (nseg == 3) row[2 * p + j] = hi;
+        }
+    }
+}
+
+// B operand of dx = du W on the tensor cores: Wt[i][s p + j] for the segments
+// s of the A operand's [hi | lo (| hi)]: W[j][i] rounded to bf16 twice, then
+// (fp32 W) its rounded remainder, so that the GEMM sums hi W_hi + lo W_hi
+// (+ hi W_lo).  A bf16 W is exact in one bf16 (two segments).
+template <typename TW>
+__global__ void __launch_bounds__(256)
+featmap_bwd_wsplit_kernel(const TW *__restrict__ W, int p, int d, int nseg, __nv_bfloat16 *__restrict__ Wt) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)p * d) return;
+    const int j = (int)(i / d), col = (int)(i % d);
+    const float w = hm_ld(W, i);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    __nv_bfloat16 *row = Wt + (int64_t)col * nseg * p;
+    row[j] = hi;
+    row[p + j] = hi;
+    if (nseg == 3) row[2 * p + j] = __float2bfloat16_rn(w - __bfloat162float(hi));
 }
 
 // Four consecutive elements of a row as fp32; `valid` of them in bounds (the
@@ -747,14 +778,32 @@ featmap_bwd_gemm_kernel(const float *__restrict__ A, int64_t lda, const TB *__re
 }
 
 // dx = du W ([rows, p] x [p, d]) and dW = du^T x ([p, rows] x [rows, d], k
-// split so that about two CTAs per SM run; dW is zeroed first).
+// split so that about two CTAs per SM run; dW is zeroed first).  With dus
+// (the du kernel's bf16 segments) and Wt, dx is one tensor-core GEMM over K =
+// nseg p: the products of the segments carry du to about 2^-17 of itself
+// (the hi and lo parts) and W exactly (bf16) or to 2^-17 (fp32); otherwise
+// the CUDA-core contraction.
 template <typename T>
-cudaError_t run_featmap_bwd_products(const float *du, const T *W, const T *x, int64_t rows, int p, int d,
-                                     float *dx, float *dW, cudaStream_t s) {
+cudaError_t run_featmap_bwd_products(const float *du, const __nv_bfloat16 *dus, __nv_bfloat16 *Wt, int nseg,
+                                     const T *W, const T *x, int64_t rows, int p, int d, float *dx, float *dW,
+                                     cudaStream_t s) {
     const bool vec = p % 4 == 0 && d % 4 == 0;
     const unsigned nt = (unsigned)((d + kGN - 1) / kGN);
-    dim3 gx((unsigned)((rows + kGM - 1) / kGM), nt, 1);
-    featmap_bwd_gemm_kernel<true, T, false><<<gx, 256, 0, s>>>(du, p, W, d, dx, d, rows, d, p, p, vec);
+    if (dus) {
+        const int64_t n = (int64_t)p * d;
+        featmap_bwd_wsplit_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(W, p, d, nseg, Wt);
+        count_launches(1);
+        GemmEpiArgs ep;
+        ep.mode = EPI_STORE_F32;
+        cudaError_t e = launch_gemm_tc_ex(dus, Wt, rows, d, (int64_t)nseg * p, dx, d, ep,
+                                          DevErr{device_error_word()}, s);
+        if (e != cudaSuccess) return e;
+        count_launches(1);
+    } else {
+        dim3 gx((unsigned)((rows + kGM - 1) / kGM), nt, 1);
+        featmap_bwd_gemm_kernel<true, T, false><<<gx, 256, 0, s>>>(du, p, W, d, dx, d, rows, d, p, p, vec);
+        count_launches(1);
+    }
     cudaError_t e = cudaMemsetAsync(dW, 0, sizeof(float) * (size_t)p * d, s);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -765,7 +814,7 @@ cudaError_t run_featmap_bwd_products(const float *du, const T *W, const T *x, in
     kchunk = (kchunk + kGK - 1) / kGK * kGK;
     dim3 gw((unsigned)mt, nt, (unsigned)((rows + kchunk - 1) / kchunk));
     featmap_bwd_gemm_kernel<false, T, true><<<gw, 256, 0, s>>>(du, p, x, d, dW, d, p, d, rows, kchunk, vec);
-    count_launches(2);
+    count_launches(1);
     return cudaGetLastError();
 }
 
@@ -804,6 +853,14 @@ cudaError_t run_passes(const BwdArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Segments of the bf16 split that carries dx = du W to the tensor cores (2
+// for a bf16 W, 3 for fp32), or 0 where the GEMM does not take the shape.
+int dx_segments(const ScanBwdCore &c) {
+    if (!c.W_q) return 0;
+    const int nseg = c.io_dtype == HM_BF16 ? 2 : 3;
+    return gemm_tc_supported(c.B * c.L * c.H, c.d, (int64_t)nseg * c.p) ? nseg : 0;
+}
+
 }  // namespace
 
 size_t scan_bwd_workspace(const ScanBwdCore &c) {
@@ -818,6 +875,8 @@ size_t scan_bwd_workspace(const ScanBwdCore &c) {
     n += 2 * r256(rows * c.F * 4);             // dphq, dphk
     n += 2 * r256(rows * 4);                   // kd, dlog a
     if (c.W_q) n += r256(rows * c.p * 4);      // du
+    if (const int nseg = dx_segments(c))      // du and W^T as bf16 segments
+        n += r256(rows * nseg * c.p * 2) + r256((size_t)c.d * nseg * c.p * 2);
     return n;
 }
 
@@ -854,6 +913,9 @@ cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
     float *kd = (float *)take(rows * 4);
     float *dla = (float *)take(rows * 4);
     float *du = c.W_q ? (float *)take(rows * c.p * 4) : nullptr;
+    const int nseg = dx_segments(c);
+    __nv_bfloat16 *dus = nseg ? (__nv_bfloat16 *)take((size_t)rows * nseg * c.p * 2) : nullptr;
+    __nv_bfloat16 *Wt = nseg ? (__nv_bfloat16 *)take((size_t)c.d * nseg * c.p * 2) : nullptr;
     a.dv_out = c.dv_out;
     a.dS0 = c.dS0;
     a.dz0 = c.dz0;
@@ -891,13 +953,13 @@ cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
         float *dxs[2] = {c.dq, c.dk};
         float *dWs[2] = {c.dW_q, c.dW_k};
         for (int m = 0; m < 2; ++m) {
-            featmap_bwd_du_kernel<<<wb, 256, 0, s>>>(phis[m], dphis[m], rows, c.p, du);
+            featmap_bwd_du_kernel<<<wb, 256, 0, s>>>(phis[m], dphis[m], rows, c.p, du, dus, nseg);
             count_launches(1);
             e = c.io_dtype == HM_BF16
-                    ? run_featmap_bwd_products(du, (const __nv_bfloat16 *)Ws[m], (const __nv_bfloat16 *)xs[m], rows,
-                                               c.p, c.d, dxs[m], dWs[m], s)
-                    : run_featmap_bwd_products(du, (const float *)Ws[m], (const float *)xs[m], rows, c.p, c.d,
-                                               dxs[m], dWs[m], s);
+                    ? run_featmap_bwd_products(du, dus, Wt, nseg, (const __nv_bfloat16 *)Ws[m],
+                                               (const __nv_bfloat16 *)xs[m], rows, c.p, c.d, dxs[m], dWs[m], s)
+                    : run_featmap_bwd_products(du, dus, Wt, nseg, (const float *)Ws[m], (const float *)xs[m], rows,
+                                               c.p, c.d, dxs[m], dWs[m], s);
             if (e != cudaSuccess) return e;
         }
     } else {

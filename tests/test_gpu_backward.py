@@ -107,12 +107,14 @@ def test_backward_initial_state_and_caller_features(hm):
                  "grad_S0": dS0, "grad_z0": dz0}, TOL_F32)
 
 
-@pytest.mark.parametrize("d,p", [(10, 5), (260, 64)])
-def test_backward_feature_map_products_ragged(hm, d, p):
+@pytest.mark.parametrize("d,p", [(10, 5), (260, 64), (64, 64)])
+def test_backward_feature_map_products_shapes(hm, d, p):
     """The feature map's gradient products (dx = du W, dW = du^T x, the latter
     split over tokens) at sizes off the 128 x 128 tiles: d = 10, p = 5 (no
-    vector loads; 582 rows over five row tiles, dW over 37 token splits) and
-    d = 260 (a column tile with 4 columns)."""
+    vector loads; 582 rows over five row tiles, dW over 37 token splits),
+    d = 260 (a column tile with 4 columns) and d = p = 64, where dx runs on
+    the tensor cores as three bf16 segments of fp32 du and W (K = 192, 582
+    rows: a ragged last row tile)."""
     cfg = wl.ScanConfig("ragged_featmap", 2, 97, 3, d, p, 8, "f32", True, 131, math.sqrt(1.0 / d))
     inp = wl.scan_inputs(cfg)
     dout = wl.round_f32(wl.normal(131, "dout", inp["v"].shape))
