@@ -237,7 +237,10 @@ HM_API hm_status hm_scan_combine(const hm_combine_args *a, hm_stream_t stream);
  * (B * L * H == 0) every given gradient of W_q, W_k, A_log and of the initial
  * state is zero (grad_A_log is zeroed when A_log is given, even with dt NULL,
  * since an empty dt tensor may come as NULL).
- * Computed on CUDA cores in fp32 from fp32 features recomputed from q, k.
+ * The recurrences run on CUDA cores in fp32, on fp32 features recomputed
+ * from q, k; the feature map's input gradient dx = du W runs on the tensor
+ * cores as one bf16 GEMM over du split into hi and lo parts (and W's own
+ * remainder for fp32 weights), which carries du to about 2^-17 of itself.
  */
 typedef struct {
     int64_t B, L;
