@@ -28,6 +28,7 @@ enum KernelId : unsigned int {
     KID_GEMM_TC = 8,
     KID_CONV = 9,
     KID_SELFTEST = 10,
+    KID_BWD_DW_TC = 11,
 };
 
 unsigned int *device_error_word();  // address of this device's error word (host)

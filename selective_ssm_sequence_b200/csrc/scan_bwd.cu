@@ -33,6 +33,7 @@
 // the feature-map backward (softmax Jacobian, dx = du W, dW = sum du x^T) and
 // the decay's (d dt = dlog a (-sigmoid(dt) e^A_log), dA_log = sum dlog a * log a).
 #include "hm_internal.h"
+#include "tc_common.cuh"
 
 namespace hm {
 
@@ -570,7 +571,8 @@ __global__ void to_f32_kernel(const T *__restrict__ x, int64_t n, float *__restr
 // de = phi (.) (dphi - sum(phi (.) dphi)), du = de[:p] - de[p:].  One warp per
 // row.  With dus, du is also written as bf16 segments [hi | lo (| hi)] of
 // a row of nseg * p (hi = du rounded to bf16, lo = the rounded remainder):
-// the A operand of dx = du W on the tensor cores.
+// the operand of dx = du W (and of dW = du^T x) on the tensor cores; du
+// itself (fp32) may then be null.
 __global__ void __launch_bounds__(256)
 featmap_bwd_du_kernel(const float *__restrict__ phi, const float *__restrict__ dphi, int64_t rows, int p,
                       float *__restrict__ du, __nv_bfloat16 *__restrict__ dus, int nseg) {
@@ -583,7 +585,7 @@ featmap_bwd_du_kernel(const float *__restrict__ phi, const float *__restrict__ d
     s = warp_sum(s);
     for (int j = lane; j < p; j += 32) {
         const float x = ph[j] * (dp[j] - s) - ph[p + j] * (dp[p + j] - s);
-        du[r * p + j] = x;
+        if (du) du[r * p + j] = x;
         if (dus) {
             const __nv_bfloat16 hi = __float2bfloat16_rn(x);
             const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
@@ -777,6 +779,169 @@ featmap_bwd_gemm_kernel(const float *__restrict__ A, int64_t lda, const TB *__re
     }
 }
 
+// ------------------------------------------------------------ dW on the tensor cores
+
+// dW = du^T x for p = 128 and bf16 x with d a multiple of 64 up to 256: each
+// CTA takes a run of 64-token blocks and accumulates du_hi^T x + du_lo^T x
+// over them in one 128 x d fp32 TMEM tile, then adds the tile to dW (zeroed
+// first) with float4 atomics.  Both operands are MN-major (tokens are the
+// contraction): 64-token x 64-feature boxes of the du kernel's bf16 [hi | lo]
+// rows and of x, loaded by TMA through a 3-stage ring.  Warp 0 loads, warp 1
+// issues the MMAs, warps 2..5 (one per TMEM lane quarter) add the tile.
+constexpr int kDwStages = 3;
+constexpr int kDwBox = 64 * 64 * 2;              // one 64-token x 64-feature bf16 box
+constexpr int kDwA = 2 * kDwBox;                 // du hi (or lo): 128 features
+constexpr int kDwStage = 2 * kDwA + 4 * kDwBox;  // hi, lo and up to 256 features of x
+constexpr int kDwSmem = kDwStages * kDwStage + 1024 + 256;
+
+struct DwAux {
+    uint64_t full[kDwStages], empty[kDwStages], dfull;
+    uint32_t tmem;
+    int abort;
+};
+
+__global__ void __launch_bounds__(192, 1)
+featmap_dw_tc_kernel(const __grid_constant__ CUtensorMap tmu, const __grid_constant__ CUtensorMap tmx,
+                     int64_t nblk, int64_t per, int p, int d, float *__restrict__ dW, DevErr err) {
+    using namespace tc;
+    extern __shared__ uint8_t smem_dw[];
+    uint8_t *smem = align_smem_1024(smem_dw);
+    DwAux *X = reinterpret_cast<DwAux *>(smem + kDwStages * kDwStage);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t blk0 = (int64_t)blockIdx.x * per;
+    const int64_t blk1 = blk0 + per < nblk ? blk0 + per : nblk;
+    const int nb = blk1 > blk0 ? (int)(blk1 - blk0) : 0;
+    const int nfb = d / 64;
+    volatile int *abort_flag = &X->abort;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDwStages; ++s) {
+            mbar_init(&X->full[s], 1);
+            mbar_init(&X->empty[s], 1);
+        }
+        mbar_init(&X->dfull, 1);
+        X->abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(&X->tmem, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = X->tmem;
+    if (warp == 0) {
+        if (elect_one()) {
+            tma_prefetch_desc(&tmu);
+            tma_prefetch_desc(&tmx);
+            int it = 0;
+            for (; it < nb; ++it) {
+                const int s = it % kDwStages;
+                if (!mbar_wait(&X->empty[s], ((it / kDwStages) & 1) ^ 1, abort_flag, err, KID_BWD_DW_TC, 1)) break;
+                uint8_t *st = smem + s * kDwStage;
+                const int r0 = (int)((blk0 + it) * 64);
+                mbar_arrive_expect_tx(&X->full[s], (uint32_t)((4 + nfb) * kDwBox));
+                for (int h = 0; h < 2; ++h)          // hi, then lo
+                    for (int fb = 0; fb < 2; ++fb)
+                        tma_load_2d(st + h * kDwA + fb * kDwBox, &tmu, &X->full[s], h * p + fb * 64, r0);
+                for (int fb = 0; fb < nfb; ++fb)
+                    tma_load_2d(st + 2 * kDwA + fb * kDwBox, &tmx, &X->full[s], fb * 64, r0);
+            }
+            // no copy may still be landing when the CTA exits
+            for (int j = it > kDwStages ? it - kDwStages : 0; j < it; ++j)
+                for (uint32_t i = 0; i < kWaitPolls; ++i)
+                    if (mbar_try_wait(&X->full[j % kDwStages], (j / kDwStages) & 1)) break;
+        }
+    } else if (warp == 1) {
+        if (elect_one()) {
+            const uint32_t idesc = idesc_bf16(128, d, true, true);
+            bool ok = true;
+            for (int it = 0; it < nb; ++it) {
+                const int s = it % kDwStages;
+                if (!mbar_wait(&X->full[s], (it / kDwStages) & 1, abort_flag, err, KID_BWD_DW_TC, 2)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = smem_u32(smem + s * kDwStage);
+                const uint32_t bx = a + 2 * kDwA;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {   // 16 tokens per MMA
+                    const uint64_t db = desc_mn_sw128(bx + k * 2048, kDwBox, 1024);
+                    mma_ss(tmem, desc_mn_sw128(a + k * 2048, kDwBox, 1024), db, idesc, (it > 0 || k > 0) ? 1u : 0u);
+                    mma_ss(tmem, desc_mn_sw128(a + kDwA + k * 2048, kDwBox, 1024), db, idesc, 1u);
+                }
+                mma_commit(&X->empty[s]);
+            }
+            if (nb > 0) {
+                mma_commit(&X->dfull);
+                // the MMAs are complete before TMEM is released, whatever the epilogue did
+                if (ok) mbar_wait(&X->dfull, 0, abort_flag, err, KID_BWD_DW_TC, 4);
+            }
+        }
+    } else {
+        // warps 2..5: TMEM lane quarter warp % 4 holds rows 32 (warp % 4) .. + 31 of dW
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        if (nb > 0 && mbar_wait(&X->dfull, 0, abort_flag, err, KID_BWD_DW_TC, 3)) {
+            tc_fence_after();
+            const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16);
+            float *dst = dW + (int64_t)row * d;
+#pragma unroll 1
+            for (int c0 = 0; c0 < d; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(ta + c0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    atomicAdd(reinterpret_cast<float4 *>(dst + c0 + 4 * u),
+                              make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                          __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3])));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// The shapes featmap_dw_tc_kernel takes (bf16 inputs: two segments).
+__host__ __device__ constexpr bool dw_tc_shape(bool have_dus, int nseg, int p, int d) {
+    return have_dus && nseg == 2 && p == 128 && d % 64 == 0 && d <= 256;
+}
+
+// dW on the tensor cores (the shapes featmap_dw_tc_kernel takes): dus is the
+// du kernel's [rows][2p] bf16 [hi | lo], x [rows][d] bf16; dW zeroed here.
+cudaError_t run_featmap_dw_tc(const __nv_bfloat16 *dus, const __nv_bfloat16 *x, int64_t rows, int p, int d,
+                              float *dW, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(dW, 0, sizeof(float) * (size_t)p * d, s);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tmu, tmx;
+    {
+        const uint64_t dims[2] = {(uint64_t)2 * p, (uint64_t)rows};
+        const uint64_t strides[1] = {(uint64_t)2 * p * 2};
+        const uint32_t box[2] = {64, 64};
+        if (!tc::make_tmap_bf16(&tmu, dus, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)d, (uint64_t)rows};
+        const uint64_t strides[1] = {(uint64_t)d * 2};
+        const uint32_t box[2] = {64, 64};
+        if (!tc::make_tmap_bf16(&tmx, x, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t nblk = (rows + 63) / 64;
+    const int64_t per = (nblk + sms - 1) / sms;
+    const unsigned grid = (unsigned)((nblk + per - 1) / per);
+    e = tc::ensure_smem_limit(featmap_dw_tc_kernel, kDwSmem);
+    if (e != cudaSuccess) return e;
+    featmap_dw_tc_kernel<<<grid, 192, kDwSmem, s>>>(tmu, tmx, nblk, per, p, d, dW, DevErr{device_error_word()});
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 // dx = du W ([rows, p] x [p, d]) and dW = du^T x ([p, rows] x [rows, d], k
 // split so that about two CTAs per SM run; dW is zeroed first).  With dus
 // (the du kernel's bf16 segments) and Wt, dx is one tensor-core GEMM over K =
@@ -803,6 +968,9 @@ cudaError_t run_featmap_bwd_products(const float *du, const __nv_bfloat16 *dus, 
         dim3 gx((unsigned)((rows + kGM - 1) / kGM), nt, 1);
         featmap_bwd_gemm_kernel<true, T, false><<<gx, 256, 0, s>>>(du, p, W, d, dx, d, rows, d, p, p, vec);
         count_launches(1);
+    }
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (dw_tc_shape(dus != nullptr, nseg, p, d)) return run_featmap_dw_tc(dus, x, rows, p, d, dW, s);
     }
     cudaError_t e = cudaMemsetAsync(dW, 0, sizeof(float) * (size_t)p * d, s);
     if (e != cudaSuccess) return e;
@@ -953,7 +1121,9 @@ cudaError_t launch_scan_bwd(const ScanBwdCore &c, void *ws, cudaStream_t s) {
         float *dxs[2] = {c.dq, c.dk};
         float *dWs[2] = {c.dW_q, c.dW_k};
         for (int m = 0; m < 2; ++m) {
-            featmap_bwd_du_kernel<<<wb, 256, 0, s>>>(phis[m], dphis[m], rows, c.p, du, dus, nseg);
+            // fp32 du only where a CUDA-core product reads it
+            float *du_f32 = dw_tc_shape(dus != nullptr, nseg, c.p, c.d) ? nullptr : du;
+            featmap_bwd_du_kernel<<<wb, 256, 0, s>>>(phis[m], dphis[m], rows, c.p, du_f32, dus, nseg);
             count_launches(1);
             e = c.io_dtype == HM_BF16
                     ? run_featmap_bwd_products(du, dus, Wt, nseg, (const __nv_bfloat16 *)Ws[m],
