@@ -238,8 +238,9 @@ HM_API hm_status hm_scan_combine(const hm_combine_args *a, hm_stream_t stream);
  * state is zero (grad_A_log is zeroed when A_log is given, even with dt NULL,
  * since an empty dt tensor may come as NULL).
  * The recurrences run on CUDA cores in fp32, on fp32 features recomputed
- * from q, k; the feature map's input gradient dx = du W runs on the tensor
- * cores as one bf16 GEMM over du split into hi and lo parts (and W's own
+ * from q, k; the feature map's gradient products dx = du W and (bf16
+ * inputs, p = 128, d a multiple of 64 up to 256) dW = du^T x run on the
+ * tensor cores over du split into bf16 hi and lo parts (and W's own
  * remainder for fp32 weights), which carries du to about 2^-17 of itself.
  */
 typedef struct {
