@@ -44,6 +44,8 @@ import workloads as wl  # noqa: E402
 # ---------------------------------------------------------------- peaks
 
 _FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the B200's spec sheet: HBM3e bandwidth and dense bf16 tensor throughput
+_SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
 def load_peaks():
@@ -413,6 +415,8 @@ def bench_prefill(cfg, args, rank, world, torch):
     else:
         roof = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": bw, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["frac_of_spec"] = roof["achieved"] / (_SPEC_PEAKS["hbm_gbs"] if roof["bound"] == "hbm"
+                                               else _SPEC_PEAKS["bf16_tflops"])
     roof["traffic"] = NCU_TRAFFIC_BYTES.get((name, cfg.name))
     roof["kernel"] = name
     roof["peak_source"] = peak_kind
@@ -446,6 +450,7 @@ def bench_prefill(cfg, args, rank, world, torch):
         "step_roofline": {"bound": "tensor", "flops_per_token_head": fl_fm + fl_sc,
                           "achieved": step_flops / (ms_step * 1e-3) / 1e12, "peak": tf,
                           "unit": "TFLOP/s", "frac": step_flops / (ms_step * 1e-3) / 1e12 / tf,
+                          "frac_of_spec": step_flops / (ms_step * 1e-3) / 1e12 / _SPEC_PEAKS["bf16_tflops"],
                           "peak_source": peak_kind},
         "breakdown_ms": {"featmap_q_and_k": 2 * ms_fmap, "scan": ms_scan,
                          "note": "scan = the call on precomputed features, timed separately; "
@@ -636,7 +641,7 @@ def bench_decode(cfg, args, rank, world, torch):
         "config": {"workload": cfg.name, "B": B, "H": H, "F": F, "dv": dv,
                    "l2": "state 1.08 GB per step, larger than L2"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "frac_of_8TBs": gbs / 8000.0,
+                     "frac": gbs / peaks["hbm_gbs"], "frac_of_spec": gbs / _SPEC_PEAKS["hbm_gbs"],
                      "bytes_per_step": state_bytes + io_bytes, "peak_source": peak_kind,
                      "kernel": "whole step (the q and k feature maps in one launch + the decode launch)"},
         "gpu_launches": per_step * steps,
@@ -716,8 +721,8 @@ def bench_mixer(cfg, args, rank, world, torch, block=False):
         "data": "synthetic", "config": dict({"workload": name, "B": B, "L": L, "d_model": D, "H": cfg.H},
                                             **({"d_ff": d_ff} if block else {})),
         "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": tf / peaks["bf16_tflops"], "flops_per_token": flops_tok,
-                     "peak_source": peak_kind,
+                     "frac": tf / peaks["bf16_tflops"], "frac_of_spec": tf / _SPEC_PEAKS["bf16_tflops"],
+                     "flops_per_token": flops_tok, "peak_source": peak_kind,
                      "kernel": "whole block forward" if block else "whole mixer forward"},
         "gpu_launches": per_step * args.steps,
         "clocks": sampler.summary(),

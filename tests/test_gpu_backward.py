@@ -147,3 +147,17 @@ def test_backward_empty_sequence_zeroes_parameter_gradients(hm):
     got = _bwd_gpu(hm, inp, np.zeros(inp["v"].shape), "f32", S0=S0, z0=z0)
     for name in ("grad_W_q", "grad_W_k", "grad_A_log", "grad_S0", "grad_z0"):
         assert got[name].size > 0 and (got[name] == 0).all(), name
+
+
+def test_backward_bf16_rows_off_16_bytes(hm):
+    """bf16 inputs whose value rows are not a multiple of 16 bytes (dv = 12):
+    the passes stage their token blocks with plain loads instead of cp.async;
+    d = 24, p = 12 (F = 24), two heads, a ragged last block of tokens."""
+    cfg = wl.ScanConfig("bf16_dv12", 2, 45, 2, 24, 12, 12, "bf16", True, 133, math.sqrt(1.0 / 24))
+    inp = wl.scan_inputs(cfg)
+    dout = wl.round_bf16(wl.normal(133, "dout", inp["v"].shape))
+    got = _bwd_gpu(hm, inp, dout, "bf16")
+    r = oracle.scan_bwd(inp["q"], inp["k"], inp["v"], inp["W_q"], inp["W_k"], dout, dt=inp["dt"],
+                        A_log=inp["A_log"])
+    _check(got, {"grad_q": r["dq"], "grad_k": r["dk"], "grad_v": r["dv"], "grad_W_q": r["dW_q"],
+                 "grad_W_k": r["dW_k"], "grad_dt": r["ddt"], "grad_A_log": r["dA_log"]}, TOL_BF16)
