@@ -495,8 +495,8 @@ struct CAux {
     float qs[2][kC];
     float w[2][kC];
     float rden[2][kC];   // 1 / den
-    float dint[2][kC];   // row sums of Pt: [0] columns 0..31, [1] columns 32..63
-    float dotq[4][kC];   // phiq_i . z_prev over each quarter of the features
+    float dint[2][2][kC];   // per chunk parity: row sums of Pt, [0] columns 0..31, [1] columns 32..63
+    float dotq[2][4][kC];   // per chunk parity: phiq_i . z_prev over each quarter of the features
     alignas(16) float zb[2][kF];   // z after chunk c in zb[c & 1]; the start z in zb[1]
     float gam[2];
     float redd[4];
@@ -504,7 +504,7 @@ struct CAux {
     // released separately
     uint64_t fullq[2], fullkv[2], emptyq[2], emptykv[2];
     uint64_t stg_free[2];   // the stage's Pt buffer, used to stage outputs, has been read out
-    uint64_t p_full, p_consumed, epib_done, o_full, o_empty, s_full, sbf_ready;
+    uint64_t p_full[2], p_consumed, epib_done, o_full, o_empty, s_full, sbf_ready;
     uint64_t den_ready[2], den_free[2];   // 1 / den of a stage written / read
     uint64_t pro_full[3];                 // start-state rounds landed (prologue staging)
     uint64_t dec_full[2], dec_free[2];    // decay vectors of a parity written / read
@@ -634,7 +634,8 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             // phiK + V: the chunk's MMAs and the four state-pass warps' key-feature sums
             mbar_init(&X->emptykv[s], 5);
         }
-        mbar_init(&X->p_full, 1);
+        mbar_init(&X->p_full[0], 1);   // the scores of a chunk of each parity
+        mbar_init(&X->p_full[1], 1);
         mbar_init(&X->p_consumed, 3);   // the three score-quadrant warps have loaded P
         mbar_init(&X->epib_done, 1);
         mbar_init(&X->o_full, 1);
@@ -718,7 +719,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     mma_ss(tmem + kColP, desc_k_sw128(sK(sc) + off), desc_k_sw128(sK(sc) + off), idP,
                            k > 0 ? 1u : 0u);
                 }
-                mma_commit(&X->p_full);
+                mma_commit(&X->p_full[c & 1]);
                 return true;
             };
             bool ok = nch > 0 && issue_scores(0);
@@ -770,23 +771,20 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         // every exit from this loop is taken by the whole group (after a
         // barrier-AND), so no thread is left waiting at a named barrier
         bool ok = named_sync_and(1, 256, true);
+        bool dok = true;   // the denominator warps' step (4) of the previous chunk went through
         for (int it = 0; it < nch; ++it) {
             const int s = it & 1;
             // (1) the chunk's decay vectors (from the decay warp; chunk 0: the
             // state prologue, which stages in the Pt and w V buffers, must also
-            // be complete before they are written)
-            const bool okd = mbar_wait(&X->dec_full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 22) &&
-                             (it > 0 || mbar_wait(&X->sbf_ready, 0, abort_flag, err, KID_SCAN_TC_OUT, 21));
-            ok = named_sync_and(1, 256, ok && okd);
-            if (!ok) break;
-            // every thread is past chunk it - 1, the last reader of the other
-            // parity's decay vectors
-            if (gt == 0 && it > 0) mbar_arrive(&X->dec_free[(it - 1) & 1]);
+            // be complete before they are written).  There is no group barrier
+            // before the chunk's work: the denominator warps may still be on
+            // step (4) of chunk it - 1, and the group meets at the end of step
+            // (3), where a failed wait of any thread ends the loop for all.
             // (2) the chunk's stage is loaded and its score MMA has completed:
             // every thread waits for both -- the score MMA reads phiQ of the
-            // stage, which step (3) scales in place -- and then meets the others
-            // at barrier 4, so that all waiters of this p_full phase are past it
-            // before p_consumed lets the next phase begin.  Score-quadrant warps
+            // stage, which step (3) scales in place.  The scores of the two
+            // chunk parities complete on barriers of their own, so a waiter
+            // never meets the next chunk's phase.  Score-quadrant warps
             // (P rows 0..31 in TMEM lanes 64..95, rows 32..63 in lanes 96..127):
             // warp 2: rows 0..31 x columns 0..31 (and the zeros of columns
             // 32..63); warp 3: rows 32..63 x columns 0..31 (all below the
@@ -795,11 +793,12 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             // arrives on p_consumed (count 3), after which the next chunk's
             // scores may overwrite it.
             const bool pwarp = warp == 2 || warp == 3 || warp == 7;
-            bool okw = mbar_wait(&X->fullkv[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8) &&
+            bool okw = dok && mbar_wait(&X->dec_full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 22) &&
+                       (it > 0 || mbar_wait(&X->sbf_ready, 0, abort_flag, err, KID_SCAN_TC_OUT, 21)) &&
+                       mbar_wait(&X->fullkv[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 8) &&
                        mbar_wait(&X->fullq[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 17) &&
-                       mbar_wait(&X->p_full, it & 1, abort_flag, err, KID_SCAN_TC_OUT, 7);
+                       mbar_wait(&X->p_full[s], (it >> 1) & 1, abort_flag, err, KID_SCAN_TC_OUT, 7);
             okw = __all_sync(0xffffffffu, okw);
-            named_sync(4, 256);
             tc_fence_after();
             const int i = 32 * (q - 2) + lane;
             const int jc = warp == 7 ? 32 : 0;
@@ -848,7 +847,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         *reinterpret_cast<uint4 *>(prow + sw128_off(i, c4)) = hi;
                         *reinterpret_cast<uint4 *>(prow + kC * 128 + sw128_off(i, c4)) = lo;
                     }
-                    X->dint[0][i] = rs2.x + rs2.y;
+                    X->dint[s][0][i] = rs2.x + rs2.y;
                 } else if (okw) {
                     const float ci = X->cum[s][i];
                     const float2 ci2 = make_float2(ci, ci);
@@ -890,7 +889,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                                 make_uint4(0u, 0u, 0u, 0u);
                         }
                     }
-                    X->dint[jc ? 1 : 0][i] = rs2.x + rs2.y;
+                    X->dint[s][jc ? 1 : 0][i] = rs2.x + rs2.y;
                 }
                 // P has been read: the next chunk's scores may overwrite it
                 tc_fence_before();
@@ -955,7 +954,7 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
                     for (int k = 0; k < 2; ++k) *reinterpret_cast<uint4 *>(qb + sw128_off(i, k0 + k)) = v[k];
                 }
-                X->dotq[qf][i] = d2.x + d2.y;
+                X->dotq[s][qf][i] = d2.x + d2.y;
             }
             fence_proxy_async_smem();
             ok = named_sync_and(1, 256, okw);
@@ -964,21 +963,26 @@ scan_out_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 mbar_arrive(&X->epib_done);
                 mbar_arrive(&X->zfree[(it - 1) & 1]);   // z_prev has been read
             }
-            // (4) denominators (once the outputs of chunk it - 2 have read this
-            // stage's 1 / den) and z; the chunk's MMAs run meanwhile
-            if (gt < kC) {
-                const int i = gt;
-                const bool okd =
-                    mbar_wait(&X->den_free[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 14);
-                const float dq = (X->dotq[0][i] + X->dotq[1][i]) + (X->dotq[2][i] + X->dotq[3][i]);
+            // (4) denominators, on warps 8 and 9 (helpers, on the SM
+            // sub-partitions the quadrant warps do not use), once the outputs of
+            // chunk it - 2 have read this stage's 1 / den; the chunk's MMAs and
+            // the other warps' chunk it + 1 run meanwhile (the row sums and dot
+            // products are kept per chunk parity).  Then the chunk's decay
+            // vectors have had their last reader.
+            if (gt >= 256 - kC) {
+                const int i = gt - (256 - kC);
+                dok = mbar_wait(&X->den_free[s], ((it >> 1) & 1) ^ 1, abort_flag, err, KID_SCAN_TC_OUT, 14);
+                const float dq = (X->dotq[s][0][i] + X->dotq[s][1][i]) + (X->dotq[s][2][i] + X->dotq[s][3][i]);
                 // the inter-chunk term with the query scale as the readout used it
                 // (rounded to bf16), so that numerator and denominator agree
                 const float qsr = __bfloat162float(__float2bfloat16_rn(X->qs[s][i]));
-                const float den = X->dint[0][i] + (i >= 32 ? X->dint[1][i] : 0.f) + qsr * dq;
+                const float den = X->dint[s][0][i] + (i >= 32 ? X->dint[s][1][i] : 0.f) + qsr * dq;
                 X->rden[s][i] = 1.f / den;
                 named_sync(3, 64);
-                if (gt == 0) mbar_arrive(&X->den_ready[s]);
-                if (!okd) ok = false;
+                if (i == 0) {
+                    mbar_arrive(&X->den_ready[s]);
+                    mbar_arrive(&X->dec_free[s]);
+                }
             }
         }
     } else if (warp == 4) {
