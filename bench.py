@@ -67,8 +67,8 @@ def load_peaks():
 # 7,543,040.  Long context B1 H8 L32768: scan_state 240,059,648 + 3,171,584,
 # scan_carry 16,860,672, scan_out 420,714,240 + 109,503,232.
 NCU_TRAFFIC_BYTES = {
-    ("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 167630592,
-    ("scan_chunked (features precomputed)", "prefill_B1_H8_L32768_d256_F256_bf16"): 790309376,
+    ("scan_chunked (features precomputed)", "prefill_B4_H8_L2048_d256_F256_bf16"): 167572736,
+    ("scan_chunked (features precomputed)", "prefill_B1_H8_L32768_d256_F256_bf16"): 790018304,
 }
 
 # ---------------------------------------------------------------- clocks
