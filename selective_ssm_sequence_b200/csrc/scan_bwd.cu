@@ -1,5 +1,7 @@
 // scan_bwd.cu -- gradients of the decayed normalised scan and of the Hedgehog
-// feature map on CUDA cores, fp32.
+// feature map: the recurrences on CUDA cores in fp32, the feature map's two
+// gradient products (dx = du W, dW = du^T x) on the tensor cores over du split
+// into bf16 hi and lo parts where the shapes allow.
 //
 // The mixer is trained (HedgeMamba explainer sec. 3: two-stage distillation),
 // and Mamba-style scans recompute their states in the backward pass instead
