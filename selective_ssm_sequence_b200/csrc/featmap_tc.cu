@@ -13,10 +13,10 @@
 //               accumulator row per thread, read from TMEM in two passes (a
 //               running max / normaliser, then the normalised features), the
 //               negate / concatenate / softmax in registers in the log2
-//               domain (one FMA-free exp2 per feature).  bf16 features leave
-//               through a per-warpgroup staging buffer and TMA stores of 128
-//               rows x 64 bytes: a thread owns a row, so direct stores would
-//               touch 32 rows (4 KB apart) per instruction.
+//               domain (one FMA-free exp2 per feature).  The features (bf16
+//               or fp32) leave through a per-warpgroup staging buffer and TMA
+//               stores of 128 rows x 64 bytes: a thread owns a row, so direct
+//               stores would touch 32 rows (1-2 KB apart) per instruction.
 // Four TMEM accumulators let the MMAs run ahead of the epilogue warpgroups.
 #include "tc_common.cuh"
 
@@ -39,7 +39,7 @@ struct FmLayout {
     static constexpr int kXBytes = kChunks * kXChunkBytes;  // one x tile
     static constexpr int kOffW = 0;
     static constexpr int kOffX = kWBytes;
-    static constexpr int kStgBytes = kBM * 64;               // output staging: 128 rows x 32 bf16
+    static constexpr int kStgBytes = kBM * 64;               // output staging: 128 rows x 64 bytes
     static constexpr int kOffStg = kOffX + kStages * kXBytes;
     static constexpr int kOffBar = kOffStg + kEpiWG * kStgBytes;
     static constexpr int kSmem = kOffBar + 256 + 1024;      // + barriers, + alignment slack
@@ -73,9 +73,8 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constan
     const bool second = blockIdx.z != 0;
     const CUtensorMap &tmx = second ? tmx1 : tmx0;
     const CUtensorMap &tmw = second ? tmw1 : tmw0;
-    const CUtensorMap &tmo = second ? tmo1 : tmo0;   // phi as (F, H, rows), 64-byte swizzle (bf16 phi)
+    const CUtensorMap &tmo = second ? tmo1 : tmo0;   // phi as (F, H, rows), 64-byte swizzle
     const float *__restrict__ bias = second ? bias1 : bias0;
-    TP *__restrict__ phi = second ? phi1 : phi0;
     __nv_bfloat16 *__restrict__ phi_lo = second ? phi_lo1 : phi_lo0;
     using Lay = FmLayout<D, P>;
     constexpr int NA = Lay::kAcc;
@@ -189,7 +188,6 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constan
             const uint32_t tbase = tmem + b * P + ((uint32_t)(q * 32) << 16);
             const int64_t t = tile * kBM + row_in_tile;
             const bool valid = t < Tv;
-            TP *out = phi + (t * Hv + h) * (int64_t)F;
             __nv_bfloat16 *lo = (phi_lo && valid) ? phi_lo + (t * Hv + h) * (int64_t)F : nullptr;
             // Everything in the log2 domain: y = u log2(e).  Pass 1: running max
             // m of |y| and normaliser Z = sum 2^(y - m) + 2^(-y - m), rescaled
@@ -282,37 +280,47 @@ featmap_tc_kernel(const __grid_constant__ CUtensorMap tmx0, const __grid_constan
                     stage_half(r, c, 1);
                 }
             } else {
-                // fp32 phi: direct 16-byte stores of each row
-                auto pass2 = [&](const uint32_t *r, int c) {
+                // fp32 phi: as the bf16 path, through the warpgroup's staging
+                // buffer, 16 features (64 bytes) of each row per TMA store of
+                // 128 rows (a thread owns a row, so direct stores would touch 32
+                // rows 1 KB apart per instruction)
+                auto stage16 = [&](const uint32_t *r, int c, int neg, int q16) {
+                    float ev[16];
 #pragma unroll
-                    for (int j0 = 0; j0 < 32; j0 += 4) {
-                        float e1[4], e2[4];
+                    for (int j = 0; j < 16; ++j) {
+                        const float y = yv(r, c, 16 * q16 + j);
+                        ev[j] = ex2_approx((neg ? -y : y) - sh);
+                    }
+                    if (wt == 0) bulk_wait_read_all();   // the previous store has read the buffer
+                    named_sync(1 + e, 128);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float y = yv(r, c, j0 + j);
-                            e1[j] = ex2_approx(y - sh);
-                            e2[j] = ex2_approx(-y - sh);
-                        }
-                        *reinterpret_cast<float4 *>(out + c + j0) = make_float4(e1[0], e1[1], e1[2], e1[3]);
-                        *reinterpret_cast<float4 *>(out + P + c + j0) = make_float4(e2[0], e2[1], e2[2], e2[3]);
+                    for (int j = 0; j < 4; ++j) {
+                        const int pc = j ^ ((row_in_tile >> 1) & 3);
+                        *reinterpret_cast<float4 *>(stg + row_in_tile * 64 + pc * 16) =
+                            make_float4(ev[4 * j], ev[4 * j + 1], ev[4 * j + 2], ev[4 * j + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    named_sync(1 + e, 128);
+                    if (wt == 0) {
+                        tma_store_3d(&tmo, stg, neg * P + c + 16 * q16, h, (int)(tile * kBM));
+                        bulk_commit();
                     }
                 };
-                uint32_t ra[32], rb[32];
-                tmem_ld32(tbase, ra);
-                tmem_wait_ld();
 #pragma unroll 1
-                for (int c = 0; c < P; c += 64) {
-                    tmem_ld32(tbase + c + 32, rb);
-                    if (valid) pass2(ra, c);
+                for (int c = 0; c < P; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c, r);
                     tmem_wait_ld();
-                    if (c + 64 < P) tmem_ld32(tbase + c + 64, ra);
-                    if (c + 64 >= P) {
+                    if (c + 32 >= P) {
+                        // the last read of this accumulator has landed
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bars->acce[b]);
                     }
-                    if (valid) pass2(rb, c + 32);
-                    tmem_wait_ld();
+                    stage16(r, c, 0, 0);
+                    stage16(r, c, 0, 1);
+                    stage16(r, c, 1, 0);
+                    stage16(r, c, 1, 1);
                 }
             }
         }
@@ -365,8 +373,15 @@ cudaError_t go(const void *x0, const void *W0, const float *bias0, void *phi0, v
         }
     }
     if constexpr (sizeof(TP) != 2) {
-        tmo[0] = tmx[0];   // unused: fp32 phi is stored directly
-        tmo[1] = tmx[nz - 1];
+        // phi [rows, F] fp32 viewed as (F, Hv, Tv); boxes of 16 features x 128 rows
+        for (int z = 0; z < nz; ++z) {
+            uint64_t dims[3] = {(uint64_t)(2 * P), (uint64_t)Hv, (uint64_t)Tv};
+            uint64_t strides[2] = {(uint64_t)(2 * P) * 4, (uint64_t)Hv * (2 * P) * 4};
+            uint32_t box[3] = {16, 1, kBM};
+            if (!tc::make_tmap(&tmo[z], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, z ? phi1 : phi0, 3, dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
+        }
     }
     if (nz == 1) {
         tmx[1] = tmx[0];
