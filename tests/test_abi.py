@@ -178,3 +178,41 @@ def test_variant_flags_are_validated_before_launch(hm):
     d.rope_base = 0.0
     d.flags = hm.HM_FLAG_DT_SCALED_INPUT                                    # needs dt
     assert hm.lib.hm_step_decode(ctypes.byref(d), None) == hm.HM_ERR_INVALID_ARG
+
+
+def _bwd(hm, **kw):
+    a = hm.ScanBwdArgs()
+    a.B, a.L, a.H, a.d, a.p, a.dv = 4, 2048, 8, 256, 128, 256
+    a.io_dtype = hm.HM_BF16
+    fake = 1 << 20  # an aligned address; validation never dereferences it
+    for n in ("q", "k", "v", "dout", "W_q", "W_k", "dt", "A_log", "grad_q", "grad_k", "grad_v", "grad_W_q",
+              "grad_W_k", "grad_dt", "grad_A_log"):
+        setattr(a, n, fake)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_backward_sizes_and_validation(hm):
+    size = lambda a: hm.hm_scan_bwd_workspace_size(a)
+    rows, F, p, d, ns = 4 * 2048 * 8, 256, 128, 256, 8
+    s_bf16 = size(_bwd(hm))
+    # the fp32 features, the value slices' shares (plus the denominator's) of
+    # dphiq and dphik, and du as bf16 hi | lo segments for the tensor cores
+    assert s_bf16 >= 2 * rows * F * 4 + 2 * (ns + 1) * rows * F * 4 + rows * 2 * p * 2
+    # fp32 inputs carry W's rounding remainder too: one more segment of du and of W^T
+    assert size(_bwd(hm, io_dtype=hm.HM_F32)) - s_bf16 == rows * p * 2 + d * p * 2
+    # a width the tensor-core GEMMs do not take (d = 250) has no segments
+    assert size(_bwd(hm, d=250)) < s_bf16
+    sizes = [size(_bwd(hm, L=L)) for L in (512, 1024, 2048)]
+    assert sizes[2] - sizes[1] <= 2 * (sizes[1] - sizes[0]) + 4096
+    call = lambda a: hm.lib.hm_scan_bwd(ctypes.byref(a), None)
+    assert call(_bwd(hm, W_k=None)) == hm.HM_ERR_INVALID_ARG
+    assert call(_bwd(hm, grad_q=None)) == hm.HM_ERR_INVALID_ARG
+    assert call(_bwd(hm, grad_dt=None)) == hm.HM_ERR_INVALID_ARG
+    assert call(_bwd(hm, S0=1 << 20)) == hm.HM_ERR_INVALID_ARG          # S0 without z0
+    assert call(_bwd(hm, q=(1 << 20) + 2)) == hm.HM_ERR_INVALID_ARG     # misaligned
+    assert call(_bwd(hm, p=300)) == hm.HM_ERR_UNSUPPORTED
+    assert size(_bwd(hm, p=300)) == 0
+    assert call(_bwd(hm)) == hm.HM_ERR_INVALID_ARG                      # no workspace
+    assert b"workspace" in hm.lib.hm_last_error_detail()
